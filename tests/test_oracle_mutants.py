@@ -1,0 +1,63 @@
+"""Planted mistakes in the oracle must be caught by its pins (no GPU).
+
+Each case copies moe_oracle.c to a temporary directory, replaces one expression
+with a plausible mistake (a dropped term, a wrong sign, index or operand, an
+off-by-one), builds it with gcc and runs every pin against that build. At least
+one pin must fail. The committed oracle is never modified.
+"""
+import os
+import shutil
+import subprocess
+
+import pytest
+
+import oracle
+import oracle_pins
+
+MUTANTS = {
+    "lse_drops_max": ("lse[t] = m + log(z);", "lse[t] = log(z);"),
+    "topk_ties_to_higher_index": ("kt[i] > kt[best]", "kt[i] >= kt[best]"),
+    "gates_wrong_index": ("s += P[(int64_t)t * E + idx[(int64_t)t * k + r]];",
+                          "s += P[(int64_t)t * E + r];"),
+    "capacity_floor": ("(int64_t)ceil(capacity_factor", "(int64_t)floor(capacity_factor"),
+    "dispatch_off_by_one": ("(rank < C) ? rank : -1", "(rank <= C) ? rank : -1"),
+    "ffn_w1_transposed": ("orc_load(ex->w1, (int64_t)f * d + j, w_dtype)",
+                          "orc_load(ex->w1, (int64_t)j * F + f, w_dtype)"),
+    "ffn_drops_b2": ("s += (double)ex->b2[n];", "s += 0.0;"),
+    "ffn_drops_b1": ("z += (double)ex->b1[f];", "z += 0.0;"),
+    "gelu_sign": ("(1.0 + erf(z / sqrt(2.0)))", "(1.0 - erf(z / sqrt(2.0)))"),
+    "swish_sign": ("z / (1.0 + exp(-z))", "z / (1.0 + exp(z))"),
+    "relu_identity": ("z > 0.0 ? z : 0.0", "z"),
+    "shared_experts_skipped": ("for (int s = 0; s < S; ++s) {", "for (int s = 0; s < 0; ++s) {"),
+    "credit_drops_gate": ("c = g[a] * sqrt(ss);", "c = sqrt(ss);"),
+    "combine_ignores_gate": ("yj[n] += g[a] * o[n];", "yj[n] += o[n];"),
+    "f_wrong_normaliser": ("((double)k * (double)T)", "((double)T)"),
+    "aux_drops_E": ("*l_aux = alpha * (double)E * aux;", "*l_aux = alpha * aux;"),
+    "zloss_not_squared": ("z += lse[t] * lse[t];", "z += lse[t];"),
+    "expert_loss_no_mean": ("expert_loss[i] /= (double)T;", "expert_loss[i] /= 1.0;"),
+    "router_drops_bias": ("s += (double)b_gate[i];", "s += 0.0;"),
+    "noise_ignored": ("v = h32[a] + noise[a];", "v = h32[a];"),
+    "selection_bias_sign": ("v = h32[a] + sel_bias[i];", "v = h32[a] - sel_bias[i];"),
+    "softmax_wrong_exponent": ("P[(int64_t)t * E + i] = exp(ht[i] - m) / z;",
+                               "P[(int64_t)t * E + i] = exp(ht[i]) / z;"),
+}
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_mutant_is_caught(name, tmp_path):
+    old, new = MUTANTS[name]
+    src = open(os.path.join(os.path.dirname(oracle.__file__), "moe_oracle.c")).read()
+    assert src.count(old) == 1, f"mutation site for {name} not found exactly once"
+    shutil.copy(os.path.join(os.path.dirname(oracle.__file__), "moe_oracle.h"), tmp_path)
+    (tmp_path / "moe_oracle.c").write_text(src.replace(old, new))
+    so = str(tmp_path / "libmutant.so")
+    subprocess.run(["gcc", "-std=c99", "-O2", "-ffp-contract=off", "-fPIC", "-shared", "-o", so,
+                    str(tmp_path / "moe_oracle.c"), "-lm"], check=True)
+    failed = []
+    with oracle.using_library(so):
+        for check in oracle_pins.ALL_CHECKS:
+            try:
+                check()
+            except AssertionError:
+                failed.append(check.__name__)
+    assert failed, f"no pin caught the planted mistake {name}"
