@@ -1,0 +1,428 @@
+#!/usr/bin/env python
+"""Benchmark of the sparse top-k MoE layer forward on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload e256] [--impl ours|reference]
+
+A step is one layer forward plus its statistics (moe_forward + moe_aux_stats
+through the C ABI) over one batch of synthetic tokens already resident in HBM.
+The default workload is the largest configuration, "e256" (T=32768, d=7168,
+d_ff=2048, E=256, k=8, one shared expert, Swish, C_f=1.25, credit statistics).
+Its inputs are larger than L2 (x 470 MB, expert weights 15 GB), so no L2 flush
+is needed between steps.
+
+With N > 1 (one process per GPU under torchrun) every rank runs its own replica
+on its own batch (weak scaling, no collective on the data path); the timed
+region is bracketed by barriers and the max over ranks is reported.
+
+Rank 0 prints one JSON line: whole-job tokens/s, the expert-GEMM roofline
+fraction measured with CUDA events inside the timed region, the end-to-end
+number with host buffers, the CPU-oracle baseline and the SM clocks.
+`--impl reference` times the CPU oracle (the reference arm) instead.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "MoE-layer fwd tokens/s; expert GEMM TFLOP/s and % of B200 roofline"
+UNIT = "tokens/s"
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=30)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="e256")
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    return ap.parse_args()
+
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        p = json.load(open(path))
+        return dict(hbm_gbs=p["hbm_gbs"], bf16=p["bf16_tflops"], bf16_sustained=p["bf16_tflops_sustained"],
+                    source="measured")
+    return dict(hbm_gbs=6650.0, bf16=1590.0, bf16_sustained=1400.0, source="fallback")
+
+
+# ---------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """nvidia-smi sampling of SM clocks and throttle reasons during the timed region."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id: str):
+        self.gpu_id = gpu_id
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", self.gpu_id, f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100", "-f", self.path], stdout=subprocess.DEVNULL, stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        rows = []
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                rows.append(parts)
+            except ValueError:
+                pass
+        os.unlink(self.path)
+        if not rows:
+            return None
+        sm = [float(r[0]) for r in rows if r[0].replace(".", "").isdigit()]
+        mx = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[4 + i].lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+def gpu_id_for(dev) -> str:
+    import torch
+    try:
+        p = torch.cuda.get_device_properties(dev)
+        return "%08x:%02x:%02x.0" % (p.pci_domain_id, p.pci_bus_id, p.pci_device_id)
+    except Exception:
+        vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+        if vis:
+            return vis.split(",")[dev]
+        return str(dev)
+
+
+# ---------------------------------------------------------------- CPU oracle sample
+
+def oracle_sample(w, x_rows, w_gate, b_gate, sel_bias, noise_rows, token_loss_rows, expert_source):
+    """Times the CPU oracle over a T_s-token batch of workload `w` (its own
+    capacity at T_s). `expert_source(experts)` returns host copies of the touched
+    experts' w1/b1/w2/b2. Returns (seconds, tokens)."""
+    import oracle
+    T_s = x_rows.shape[0]
+    ws = w.with_(T=T_s)
+    inp = dict(x=x_rows, w_gate=w_gate, b_gate=b_gate, sel_bias=sel_bias, noise=noise_rows,
+               token_loss=token_loss_rows)
+    # Untimed pre-pass: which experts does this sample touch?
+    h = oracle.router_logits(x_rows, w_gate, b_gate)
+    key = oracle.selection_keys(h.astype("float32"), noise_rows if w.top_k_method == "noisy" else None,
+                                sel_bias if w.use_selection_bias else None)
+    idx = oracle.topk(key, w.k)
+    inp.update(expert_source(sorted(set(idx.ravel().tolist()) | set(range(w.E, w.E + w.S)))))
+    t0 = time.perf_counter()
+    oracle.forward(ws, inp)
+    return time.perf_counter() - t0, T_s
+
+
+def cpu_sample_from_device(w, inp, T_s):
+    import torch
+    sl = slice(0, T_s)
+    cpu = lambda t: None if t is None else t[sl].cpu() if t.dim() and t.shape[0] == w.T else t.cpu()
+
+    def experts(es):
+        return {k: {e: inp[k][e].cpu() for e in es} for k in ("w1", "b1", "w2", "b2")}
+
+    return oracle_sample(w, inp["x"][sl].cpu(), inp["w_gate"].cpu(),
+                         None if inp.get("b_gate") is None else inp["b_gate"].cpu(),
+                         None if inp.get("sel_bias") is None else inp["sel_bias"].cpu(),
+                         None if inp.get("noise") is None else inp["noise"][sl].cpu(),
+                         None if inp.get("token_loss") is None else inp["token_loss"][sl].cpu(), experts)
+
+
+def oracle_threads():
+    import oracle
+    return oracle.max_threads()
+
+
+# ---------------------------------------------------------------- our arm
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+    from sparse_mixture_experts_gate_b200 import binding
+    from sparse_mixture_experts_gate_b200.binding import MoELayer
+    from sparse_mixture_experts_gate_b200.workloads import WORKLOADS, make_inputs, make_tokens
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+
+    w = WORKLOADS[args.workload]
+    inp = make_inputs(w, "cuda")
+    if rank > 0:  # each replica routes its own batch of tokens
+        inp.update(make_tokens(w, "cuda", seed=w.seed + 7919 * rank))
+    layer = MoELayer(w, inp)
+    T = w.T
+    x, noise, tl = inp["x"], inp.get("noise"), inp.get("token_loss")
+    out = layer.alloc_outputs(T)
+    layer.workspace(T)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        layer.forward(x, noise=noise, out=out)
+        layer.aux_stats(out, token_loss=tl)
+
+    for _ in range(max(args.warmup, 3)):
+        step()
+    torch.cuda.synchronize()
+    if layer.device_status() != 0:
+        raise RuntimeError("device status reports a timeout")
+    kept = int(out["count_kept"].sum().item())
+    rows = kept + w.S * T
+    flops_g1 = 2.0 * rows * w.F * w.d
+    flops_g2 = 2.0 * rows * w.F * w.O
+    launches_per_step = layer.launch_count()
+
+    K = args.steps
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(binding.MOE_TIMING_EVENTS)] for _ in range(K)]
+    for row in evs:  # materialise the event handles
+        for e in row:
+            e.record(stream)
+    torch.cuda.synchronize()
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clocks = ClockSampler(gpu_id_for(local))
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    time.sleep(0.3)
+    start.record(stream)
+    for i in range(K):
+        binding.moe_set_timing_events(layer.handle, [e.cuda_event for e in evs[i]])
+        step()
+    end.record(stream)
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    binding.moe_set_timing_events(layer.handle, None)
+    if world > 1:
+        dist.barrier()
+    ms = start.elapsed_time(end)
+    stage = {n: [] for n in binding.STAGES}
+    for row in evs:
+        for j, n in enumerate(binding.STAGES):
+            stage[n].append(row[j].elapsed_time(row[j + 1]))
+    ms_t = torch.tensor([ms], device=dev)
+    if world > 1:
+        dist.all_reduce(ms_t, op=dist.ReduceOp.MAX)
+    ms_max = float(ms_t.item())
+    ms_step = ms_max / K
+    value = world * T * K / (ms_max / 1e3)
+
+    # End to end through the public API with host buffers.
+    e2e = None
+    if not args.no_e2e:
+        x_h = x.cpu().pin_memory()
+        noise_h = noise.cpu().pin_memory() if noise is not None else None
+        tl_h = tl.cpu().pin_memory() if tl is not None else None
+        y_h = torch.empty_like(out["y"], device="cpu").pin_memory()
+        stat_keys = ("l_aux", "l_z", "n_dropped", "f", "p_mean", "expert_loss")
+        st_h = {k: torch.empty_like(out[k], device="cpu").pin_memory() for k in stat_keys}
+        x_d, noise_d, tl_d = torch.empty_like(x), (torch.empty_like(noise) if noise is not None else None), \
+            (torch.empty_like(tl) if tl is not None else None)
+
+        def step_e2e():
+            x_d.copy_(x_h, non_blocking=True)
+            if noise_d is not None:
+                noise_d.copy_(noise_h, non_blocking=True)
+            if tl_d is not None:
+                tl_d.copy_(tl_h, non_blocking=True)
+            layer.forward(x_d, noise=noise_d, out=out)
+            layer.aux_stats(out, token_loss=tl_d)
+            y_h.copy_(out["y"], non_blocking=True)
+            for k in stat_keys:
+                st_h[k].copy_(out[k], non_blocking=True)
+
+        for _ in range(2):
+            step_e2e()
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        s2, e2 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        Ke = max(3, min(K, 10))
+        s2.record(stream)
+        for _ in range(Ke):
+            step_e2e()
+        e2.record(stream)
+        torch.cuda.synchronize()
+        t2 = torch.tensor([s2.elapsed_time(e2)], device=dev)
+        if world > 1:
+            dist.all_reduce(t2, op=dist.ReduceOp.MAX)
+        h2d = x_h.numel() * x_h.element_size() + (noise_h.numel() * 4 if noise_h is not None else 0) + \
+            (tl_h.numel() * 4 if tl_h is not None else 0)
+        d2h = y_h.numel() * y_h.element_size() + sum(v.numel() * v.element_size() for v in st_h.values())
+        e2e = {"value": world * T * Ke / (float(t2.item()) / 1e3), "unit": UNIT, "h2d_bytes_per_step": int(h2d),
+               "d2h_bytes_per_step": int(d2h), "steps": Ke}
+
+    if rank != 0:
+        if world > 1:
+            dist.destroy_process_group()
+        return
+
+    peaks = measured_peaks()
+    g1 = statistics.mean(stage["gemm1"])
+    g2 = statistics.mean(stage["gemm2"])
+    achieved = (flops_g1 + flops_g2) / ((g1 + g2) / 1e3) / 1e12  # TFLOP/s per launch pair
+    traffic = committed_traffic(w)
+    layer_flops = flops_g1 + flops_g2
+    step_tflops = layer_flops / (ms_step / 1e3) / 1e12
+    # Algorithmic layer bytes: x once, W_g, weights of experts with a kept row, y once, routing metadata.
+    es = 2 if w.dtype == "bf16" else 4
+    touched = int((out["count_kept"] > 0).sum().item()) + w.S
+    bytes_min = T * w.d * es + w.E * w.d * 4 + touched * (w.F * w.d + w.O * w.F) * es + T * w.O * es + T * w.k * 12
+    layer_frac = max(layer_flops / (peaks["bf16"] * 1e12), bytes_min / (peaks["hbm_gbs"] * 1e9)) / (ms_step / 1e3)
+
+    cpu = None
+    if not args.no_cpu_baseline and world == 1:
+        T_s = min(64, max(8, 2 * oracle_threads()))
+        secs, n = cpu_sample_from_device(w, inp, T_s)
+        cpu = {"value": n / secs, "unit": UNIT, "cores": oracle_threads(), "kind": "oracle",
+               "sample": f"{n} tokens of {w.name} through the whole fp64 oracle forward (capacity at T={n}), "
+                         f"{secs:.1f} s"}
+
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K, "warmup": args.warmup,
+        "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": w.dtype, "data": "synthetic (seeded; x ~ N(0,1), weights ~ N(0,1/fan_in))",
+        "config": {"workload": w.name, "T": T, "d": w.d, "d_ff": w.F, "out": w.O, "E": w.E, "k": w.k, "S": w.S,
+                   "activation": w.activation, "capacity_factor": w.capacity_factor,
+                   "tokens_per_rank": T, "parallelism": f"replicas x{world}",
+                   "l2": "inputs larger than L2 (x 470 MB, expert weights 15 GB); no flush"},
+        "expert_gemm_tflops": step_tflops,
+        "layer_roofline_frac": layer_frac,
+        "roofline": {"kernel": "grouped_gemm_tc (expert GEMM 1 + 2)", "bound": "tensor", "achieved": achieved,
+                     "peak": peaks["bf16_sustained"], "unit": "TFLOP/s", "frac": achieved / peaks["bf16_sustained"],
+                     "peak_kind": f"bf16 sustained ({peaks['source']})", "traffic": traffic},
+        "stage_ms": {n: statistics.mean(v) for n, v in stage.items()},
+        "kept_rows": kept, "n_dropped": int(out["n_dropped"].item()),
+        "gpu_launches": launches_per_step * K,
+        "e2e": e2e, "cpu_baseline": cpu, "clocks": clk,
+    }
+    print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+
+
+def committed_traffic(w):
+    """DRAM bytes per expert-GEMM launch pair from the committed ncu summary, if
+    the kernel source has not changed since it was captured."""
+    import hashlib
+    path = os.path.join(ROOT, "profiles", f"grouped_gemm_tc_{w.name}_traffic.txt")
+    src = os.path.join(ROOT, "sparse_mixture_experts_gate_b200", "csrc", "gemm_tc.cu")
+    if not os.path.exists(path):
+        return None
+    sha = hashlib.sha256(open(src, "rb").read()).hexdigest()
+    vals = {}
+    for line in open(path):
+        if ":" in line:
+            k, v = line.split(":", 1)
+            vals[k.strip()] = v.strip()
+    if vals.get("kernel_source_sha256") != sha:
+        return None
+    try:
+        return float(vals["dram_bytes_per_launch_pair"])
+    except (KeyError, ValueError):
+        return None
+
+
+# ---------------------------------------------------------------- reference arm
+
+def run_reference(args):
+    import numpy as np
+    import torch
+    from sparse_mixture_experts_gate_b200.workloads import WORKLOADS, make_expert_weights, make_tokens, \
+        make_router
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    if rank != 0:
+        return
+    w = WORKLOADS[args.workload]
+    threads = oracle_threads()
+    # Calibrate: a step is a T_s-token sample sized to about 2 s of oracle work.
+    router = make_router(w, "cpu")
+    toks = make_tokens(w.with_(T=max(1, min(w.T, 256))), "cpu")
+    cache = {}
+
+    def experts(es):
+        need = [e for e in es if e not in cache]
+        if need:
+            got = make_expert_weights(w, need, "cpu")
+            for e in need:
+                cache[e] = {k: got[k][e] for k in got}
+        return {k: {e: cache[e][k] for e in es} for k in ("w1", "b1", "w2", "b2")}
+
+    def sample(n):
+        sl = slice(0, n)
+        return oracle_sample(w, toks["x"][sl], router["w_gate"], router.get("b_gate"), router.get("sel_bias"),
+                             None if toks.get("noise") is None else toks["noise"][sl],
+                             None if toks.get("token_loss") is None else toks["token_loss"][sl], experts)
+
+    t1, _ = sample(1)
+    budget_s = max(0.5, 150.0 / max(1, args.steps + args.warmup))
+    T_s = int(max(1, min(toks["x"].shape[0], budget_s / max(t1, 1e-3) * min(threads, 8))))
+    for _ in range(args.warmup):
+        sample(T_s)
+    tot, n_tok = 0.0, 0
+    for _ in range(args.steps):
+        s, n = sample(T_s)
+        tot += s
+        n_tok += n
+    value = n_tok / tot
+    desc = f"{T_s} tokens of {w.name} per step through the whole fp64 oracle forward (capacity at T={T_s})"
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * tot / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic (seeded, CPU generator)",
+            "config": {"workload": w.name, "T": w.T, "d": w.d, "d_ff": w.F, "out": w.O, "E": w.E, "k": w.k,
+                       "S": w.S, "parallelism": "host cores"},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle", "sample": desc},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

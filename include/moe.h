@@ -1,0 +1,231 @@
+/*
+ * moe.h - C ABI of the B200 (sm_100a) sparse top-k Mixture-of-Experts layer forward.
+ *
+ * One layer forward, as defined by the pages it is built from:
+ *   router logits h = W_g x (+ router bias)       "Appendix C - Acronyms & Symbols",
+ *   P = softmax(h), top-k set T_k(x), gates g_i      table "Core MoE symbols";
+ *   capacity C = ceil(C_f k T / E), dispatch into    same page, "Capacity &
+ *   per-expert buffers, overflow dropped             communication"; "Code Walkthrough -
+ *                                                    SER", "Load balancing";
+ *   expert MLP w1/b1 -> ReLU|GELU|Swish -> w2/b2,    "Code Walkthrough - SER", "The
+ *   gate-weighted combine, shared experts            gating / routing path";
+ *                                                    Appendix C "Parameter accounting";
+ *   f_i, P_i, L_aux = alpha E sum f_i P_i,           Appendix C, "Balancing";
+ *   z-loss beta mean (log sum e^h)^2
+ *   credit c = g ||o_i(x)||_2 and the expert-        "Sparse MoE Expert-Credit Loss
+ *   attributed loss l_i                              Reweighting Diagram", panel (b).
+ *
+ * Conventions for every entry point:
+ *   - Array arguments are DEVICE pointers (CUDA global memory) owned by the caller,
+ *     row-major, densely packed, and at least 16-byte aligned.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = the legacy default
+ *     stream). All device work is enqueued asynchronously on it; no entry point
+ *     synchronises the device.
+ *   - Every call that can fail returns an int status (MOE_OK = 0, negative on
+ *     error). Argument errors are detected on the host BEFORE anything is
+ *     enqueued; moe_last_error() then returns a message naming the bad argument.
+ *   - The library never allocates device memory: scratch comes from the
+ *     caller's workspace.
+ *   - NaN or Inf inputs are not supported: outputs are then unspecified, but no
+ *     kernel faults or waits forever.
+ */
+#ifndef MOE_H
+#define MOE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define MOE_API __attribute__((visibility("default")))
+#else
+#define MOE_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Status codes. */
+enum {
+    MOE_OK = 0,
+    MOE_ERR_INVALID_ARG = -1,  /* a NULL or inconsistent argument             */
+    MOE_ERR_UNSUPPORTED = -2,  /* a valid configuration this build cannot run */
+    MOE_ERR_CUDA = -3,         /* a CUDA runtime or driver call failed         */
+    MOE_ERR_WORKSPACE = -4,    /* workspace NULL, misaligned or too small      */
+    MOE_ERR_TIMEOUT = -5,      /* a bounded device-side wait gave up           */
+    MOE_ERR_STATE = -6         /* call out of order (stats before a forward)   */
+};
+
+/* Activations ("Code Walkthrough - SER", gating / routing path: ReLU, GELU, Swish).
+ * GELU is the exact form 0.5 z (1 + erf(z / sqrt 2)); Swish is z * sigmoid(z). */
+enum { MOE_ACT_RELU = 0, MOE_ACT_GELU = 1, MOE_ACT_SWISH = 2 };
+
+/* Top-k methods (same page, "Configuration"): GREEDY selects the highest logits;
+ * NOISY adds caller-supplied noise to the logits before selection. */
+enum { MOE_TOPK_GREEDY = 0, MOE_TOPK_NOISY = 1 };
+
+/* Storage type of x, w1, w2 and y. Router weights and biases are always fp32.
+ * BF16 runs the expert FFNs on the tcgen05 tensor cores (fp32 accumulation);
+ * FP32 runs them on fp32 CUDA cores. */
+enum { MOE_DTYPE_BF16 = 0, MOE_DTYPE_FP32 = 1 };
+
+/* Layer configuration. Field names follow the SER walkthrough's configuration
+ * (num_experts, num_active, input_dim, expert_dim, output_dim, top_k_method,
+ * load_balance_coef); the remaining fields carry Appendix C's symbols. */
+typedef struct {
+    int32_t num_experts;      /* E, routed experts, 1..256                          */
+    int32_t num_active;       /* k, experts per token, 1..min(E, 16)                */
+    int32_t input_dim;        /* d; multiple of 64 for BF16                         */
+    int32_t expert_dim;       /* F = d_ff; multiple of 64 for BF16                  */
+    int32_t output_dim;       /* O; multiple of 16 for BF16                         */
+    int32_t num_shared;       /* S always-on shared experts (weight 1), 0..4        */
+    float capacity_factor;    /* C_f; C = ceil(C_f k T / E). <= 0: no limit (C = T) */
+    int32_t activation;       /* MOE_ACT_*                                          */
+    int32_t top_k_method;     /* MOE_TOPK_*                                         */
+    int32_t use_selection_bias; /* 1: add weights->sel_bias b_i to the selection key */
+    int32_t dtype;            /* MOE_DTYPE_*                                        */
+    int32_t max_tokens;       /* largest T a forward may pass; 0 = no limit        */
+    float load_balance_coef;  /* alpha of L_aux                                     */
+    float z_loss_coef;        /* beta of the z-loss                                 */
+    float temperature;        /* router softmax temperature; only 1 is supported   */
+} moe_config_t;
+
+/* Defaults of the SER walkthrough's configuration: E=8, k=2, 512/1024/512,
+ * GREEDY, alpha=0.01; plus no shared experts, C_f=1.25, GELU, beta=1e-3, BF16,
+ * temperature 1. */
+MOE_API moe_config_t moe_config_default(void);
+
+/* Layer weights, BORROWED: the layer keeps the pointers (and TMA descriptors
+ * built over them), so they must stay valid and at the same address until
+ * moe_destroy. Their contents may change between forwards (e.g. an optimizer
+ * step); each forward reads the current values. Shared experts are the last S
+ * entries of the expert stacks (G = E + S groups).
+ *   w_gate   [E][d]    fp32, router matrix W_g                     (required)
+ *   b_gate   [E]       fp32, router bias                           (NULL = none)
+ *   sel_bias [E]       fp32, selection bias b_i                    (required iff use_selection_bias)
+ *   w1       [G][F][d] dtype, first expert layer (row f, column j) (required)
+ *   b1       [G][F]    fp32                                        (NULL = zero)
+ *   w2       [G][O][F] dtype, second expert layer                  (required)
+ *   b2       [G][O]    fp32                                        (NULL = zero) */
+typedef struct {
+    const float *w_gate;
+    const float *b_gate;
+    const float *sel_bias;
+    const void *w1;
+    const void *w2;
+    const float *b1;
+    const float *b2;
+} moe_weights_t;
+
+/* Optional routing outputs of a forward (any pointer may be NULL; the struct
+ * itself may be NULL). Written by moe_forward and read again by the
+ * moe_aux_stats that follows, so they must not change in between.
+ *   logits     [T][E] fp32  router logits h (clean: no noise, no selection bias)
+ *   gates      [T][k] fp32  renormalised gates g, in top-k order
+ *   topk_idx   [T][k] int32 selected experts, by descending selection key;
+ *                           equal keys go to the lower expert index
+ *   slot       [T][k] int32 rank in the expert's buffer (ascending token order),
+ *                           or -1 if the assignment was dropped by the capacity cap
+ *   count_pre  [E]    int32 selections per expert before the cap
+ *   count_kept [E]    int32 assignments kept per expert (min(count_pre, C)) */
+typedef struct {
+    float *logits;
+    float *gates;
+    int32_t *topk_idx;
+    int32_t *slot;
+    int32_t *count_pre;
+    int32_t *count_kept;
+} moe_routing_t;
+
+/* Statistics written by moe_aux_stats (device pointers; any may be NULL).
+ *   f           [E] fp32  f_i = count_pre_i / (k T)  (selections before the cap)
+ *   p_mean      [E] fp32  P_i = mean over tokens of softmax(h)_i
+ *   l_aux       [1] fp32  alpha E sum_i f_i P_i
+ *   l_z         [1] fp32  beta mean_t (log sum_i e^{h_ti})^2
+ *   n_dropped   [1] int32 assignments dropped by the capacity cap
+ *   credit      [T][k] fp32 c = g ||o_e(x_t)||_2 for kept assignments, 0 if dropped
+ *               (o_e = the expert's output before gate weighting)
+ *   expert_loss [E] fp32  l_i = (1/T) sum_t credit_{t,i} token_loss_t over kept
+ *               assignments; needs token_loss. */
+typedef struct {
+    float *f;
+    float *p_mean;
+    float *l_aux;
+    float *l_z;
+    int32_t *n_dropped;
+    float *credit;
+    float *expert_loss;
+} moe_stats_t;
+
+typedef struct moe_layer moe_layer_t; /* opaque; host state only */
+
+/* Validate `cfg`, borrow `w` and build the layer's host state (tile plans and TMA
+ * descriptors over the weights). No device memory is allocated and nothing is
+ * enqueued. On success *out owns a layer to release with moe_destroy; on error
+ * *out is set to NULL. Errors: INVALID_ARG (NULL pointer, dims out of range,
+ * k > E, missing sel_bias), UNSUPPORTED (temperature != 1, a dim not a multiple
+ * the BF16 path needs, E > 256), CUDA (no device or no sm_100 device). */
+MOE_API int moe_layer_create(const moe_config_t *cfg, const moe_weights_t *w, moe_layer_t **out);
+
+/* Bytes of device workspace a forward over T tokens needs (0 if T < 0 or the
+ * layer is NULL). The workspace holds the permuted activations, the hidden
+ * activations, the per-assignment expert outputs and the routing scratch. */
+MOE_API size_t moe_workspace_bytes(const moe_layer_t *layer, int32_t T);
+
+/* Capacity C = ceil(C_f k T / E) (T when C_f <= 0) that a forward over T tokens uses. */
+MOE_API int64_t moe_capacity(const moe_layer_t *layer, int32_t T);
+
+/* One layer forward over T >= 0 tokens.
+ *   x           [T][d] dtype   input tokens                           (required if T > 0)
+ *   logit_noise [T][E] fp32    noise added to the logits before selection;
+ *                              required for NOISY, ignored for GREEDY
+ *   workspace   >= moe_workspace_bytes(layer, T) bytes, 256-byte aligned, caller-owned;
+ *               it must stay untouched until the moe_aux_stats that follows
+ *   y           [T][O] dtype   output: sum of shared experts plus gate-weighted
+ *                              kept routed experts                    (required if T > 0)
+ *   routing     optional routing outputs (see moe_routing_t)
+ * T = 0 is valid and enqueues nothing. Errors: INVALID_ARG, WORKSPACE, CUDA
+ * (launch failure), INVALID_ARG if T > max_tokens. */
+MOE_API int moe_forward(moe_layer_t *layer, const void *x, int32_t T, const float *logit_noise,
+                void *workspace, size_t ws_bytes, void *y, const moe_routing_t *routing,
+                void *stream);
+
+/* Balancing and credit statistics of the most recent moe_forward on this layer,
+ * computed from what that forward left in its workspace (and routing buffers).
+ *   token_loss [T] fp32 per-token losses l_t (NULL: expert_loss is not written)
+ * Errors: STATE if no forward has run, INVALID_ARG if out is NULL. */
+MOE_API int moe_aux_stats(moe_layer_t *layer, const float *token_loss, const moe_stats_t *out,
+                  void *stream);
+
+/* Device status word of the most recent forward: synchronises `stream`, then
+ * returns MOE_OK, or MOE_ERR_TIMEOUT if a bounded device-side wait gave up. */
+MOE_API int moe_device_status(moe_layer_t *layer, void *stream);
+
+/* Optional stage timing with caller-owned CUDA events (cudaEvent_t passed as
+ * void*, created with timing enabled). After this call every moe_forward records
+ *   events[0] before the router,        events[1] after the router,
+ *   events[2] after the dispatch,       events[3] after the row gather,
+ *   events[4] after expert GEMM 1,      events[5] after expert GEMM 2,
+ *   events[6] after the combine,
+ * and every moe_aux_stats records events[7] after its kernels, all on the
+ * call's stream. The array is copied; events == NULL turns timing off. Nothing
+ * is allocated and nothing synchronises. */
+#define MOE_TIMING_EVENTS 8
+MOE_API int moe_set_timing_events(moe_layer_t *layer, void *const *events);
+
+/* Number of kernels the most recent moe_forward plus moe_aux_stats enqueued. */
+MOE_API int32_t moe_launch_count(const moe_layer_t *layer);
+
+/* Release the layer's host state (NULL is a no-op). Borrowed weights are untouched. */
+MOE_API void moe_destroy(moe_layer_t *layer);
+
+/* Static name of a status code ("MOE_OK", "MOE_ERR_INVALID_ARG", ...). */
+MOE_API const char *moe_status_string(int status);
+
+/* Message of the last error on the calling thread ("" if none). */
+MOE_API const char *moe_last_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* MOE_H */

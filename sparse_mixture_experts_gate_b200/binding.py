@@ -1,0 +1,272 @@
+"""ctypes binding of libmoe.so (the C ABI of include/moe.h).
+
+Argument marshalling only: every step of the layer forward runs in the CUDA
+kernels behind the C ABI. PyTorch supplies device memory and streams. If the
+library has not been built, loading it raises; there is no fallback path.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Dict, Optional
+
+PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(PKG, "libmoe.so")
+
+MOE_OK, MOE_ERR_INVALID_ARG, MOE_ERR_UNSUPPORTED, MOE_ERR_CUDA = 0, -1, -2, -3
+MOE_ERR_WORKSPACE, MOE_ERR_TIMEOUT, MOE_ERR_STATE = -4, -5, -6
+MOE_ACT = {"relu": 0, "gelu": 1, "swish": 2}
+MOE_TOPK = {"greedy": 0, "noisy": 1}
+MOE_DTYPE = {"bf16": 0, "fp32": 1}
+
+# Every symbol include/moe.h declares.
+EXPORTS = ("moe_config_default", "moe_layer_create", "moe_workspace_bytes", "moe_capacity", "moe_forward",
+           "moe_aux_stats", "moe_device_status", "moe_set_timing_events", "moe_launch_count", "moe_destroy", "moe_status_string",
+           "moe_last_error")
+
+
+class MoeConfig(ctypes.Structure):
+    _fields_ = [("num_experts", ctypes.c_int32), ("num_active", ctypes.c_int32), ("input_dim", ctypes.c_int32),
+                ("expert_dim", ctypes.c_int32), ("output_dim", ctypes.c_int32), ("num_shared", ctypes.c_int32),
+                ("capacity_factor", ctypes.c_float), ("activation", ctypes.c_int32),
+                ("top_k_method", ctypes.c_int32), ("use_selection_bias", ctypes.c_int32),
+                ("dtype", ctypes.c_int32), ("max_tokens", ctypes.c_int32), ("load_balance_coef", ctypes.c_float),
+                ("z_loss_coef", ctypes.c_float), ("temperature", ctypes.c_float)]
+
+
+class MoeWeights(ctypes.Structure):
+    _fields_ = [("w_gate", ctypes.c_void_p), ("b_gate", ctypes.c_void_p), ("sel_bias", ctypes.c_void_p),
+                ("w1", ctypes.c_void_p), ("w2", ctypes.c_void_p), ("b1", ctypes.c_void_p),
+                ("b2", ctypes.c_void_p)]
+
+
+class MoeRouting(ctypes.Structure):
+    _fields_ = [("logits", ctypes.c_void_p), ("gates", ctypes.c_void_p), ("topk_idx", ctypes.c_void_p),
+                ("slot", ctypes.c_void_p), ("count_pre", ctypes.c_void_p), ("count_kept", ctypes.c_void_p)]
+
+
+class MoeStats(ctypes.Structure):
+    _fields_ = [("f", ctypes.c_void_p), ("p_mean", ctypes.c_void_p), ("l_aux", ctypes.c_void_p),
+                ("l_z", ctypes.c_void_p), ("n_dropped", ctypes.c_void_p), ("credit", ctypes.c_void_p),
+                ("expert_loss", ctypes.c_void_p)]
+
+
+class MoEError(RuntimeError):
+    def __init__(self, code: int, where: str, message: str):
+        super().__init__(f"{where}: {moe_status_string(code)} ({code}): {message}")
+        self.code = code
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: build it with "
+                               "`python -m sparse_mixture_experts_gate_b200.build` (nvcc, sm_100a)")
+        L = ctypes.CDLL(LIB_PATH)
+        vp, i32, i64, sz = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_size_t
+        L.moe_config_default.restype = MoeConfig
+        L.moe_config_default.argtypes = []
+        L.moe_layer_create.restype = ctypes.c_int
+        L.moe_layer_create.argtypes = [ctypes.POINTER(MoeConfig), ctypes.POINTER(MoeWeights), ctypes.POINTER(vp)]
+        L.moe_workspace_bytes.restype = sz
+        L.moe_workspace_bytes.argtypes = [vp, i32]
+        L.moe_capacity.restype = i64
+        L.moe_capacity.argtypes = [vp, i32]
+        L.moe_forward.restype = ctypes.c_int
+        L.moe_forward.argtypes = [vp, vp, i32, vp, vp, sz, vp, ctypes.POINTER(MoeRouting), vp]
+        L.moe_aux_stats.restype = ctypes.c_int
+        L.moe_aux_stats.argtypes = [vp, vp, ctypes.POINTER(MoeStats), vp]
+        L.moe_device_status.restype = ctypes.c_int
+        L.moe_device_status.argtypes = [vp, vp]
+        L.moe_set_timing_events.restype = ctypes.c_int
+        L.moe_set_timing_events.argtypes = [vp, ctypes.POINTER(vp)]
+        L.moe_launch_count.restype = i32
+        L.moe_launch_count.argtypes = [vp]
+        L.moe_destroy.restype = None
+        L.moe_destroy.argtypes = [vp]
+        L.moe_status_string.restype = ctypes.c_char_p
+        L.moe_status_string.argtypes = [ctypes.c_int]
+        L.moe_last_error.restype = ctypes.c_char_p
+        L.moe_last_error.argtypes = []
+        _lib = L
+    return _lib
+
+
+def moe_status_string(code: int) -> str:
+    return lib().moe_status_string(code).decode()
+
+
+def moe_last_error() -> str:
+    return lib().moe_last_error().decode()
+
+
+def _check(rc: int, where: str) -> int:
+    if rc != MOE_OK:
+        raise MoEError(rc, where, moe_last_error())
+    return rc
+
+
+def moe_config_default() -> MoeConfig:
+    return lib().moe_config_default()
+
+
+def moe_layer_create(cfg: MoeConfig, weights: MoeWeights) -> int:
+    h = ctypes.c_void_p()
+    _check(lib().moe_layer_create(ctypes.byref(cfg), ctypes.byref(weights), ctypes.byref(h)), "moe_layer_create")
+    return h.value
+
+
+def moe_workspace_bytes(layer: int, T: int) -> int:
+    return int(lib().moe_workspace_bytes(layer, T))
+
+
+def moe_capacity(layer: int, T: int) -> int:
+    return int(lib().moe_capacity(layer, T))
+
+
+def moe_forward(layer: int, x: int, T: int, logit_noise: Optional[int], workspace: int, ws_bytes: int, y: int,
+                routing: Optional[MoeRouting], stream: int) -> int:
+    r = ctypes.byref(routing) if routing is not None else None
+    return _check(lib().moe_forward(layer, x, T, logit_noise, workspace, ws_bytes, y, r, stream), "moe_forward")
+
+
+def moe_aux_stats(layer: int, token_loss: Optional[int], stats: MoeStats, stream: int) -> int:
+    return _check(lib().moe_aux_stats(layer, token_loss, ctypes.byref(stats), stream), "moe_aux_stats")
+
+
+def moe_device_status(layer: int, stream: int) -> int:
+    return int(lib().moe_device_status(layer, stream))
+
+
+MOE_TIMING_EVENTS = 8
+STAGES = ("router", "dispatch", "gather", "gemm1", "gemm2", "combine", "stats")
+
+
+def moe_set_timing_events(layer: int, events) -> int:
+    """events: sequence of MOE_TIMING_EVENTS raw cudaEvent_t handles, or None."""
+    if events is None:
+        return _check(lib().moe_set_timing_events(layer, None), "moe_set_timing_events")
+    arr = (ctypes.c_void_p * MOE_TIMING_EVENTS)(*events)
+    return _check(lib().moe_set_timing_events(layer, arr), "moe_set_timing_events")
+
+
+def moe_launch_count(layer: int) -> int:
+    return int(lib().moe_launch_count(layer))
+
+
+def moe_destroy(layer: int) -> None:
+    lib().moe_destroy(layer)
+
+
+# ------------------------------------------------------------------ torch helper
+
+def _ptr(t) -> Optional[int]:
+    return None if t is None else t.data_ptr()
+
+
+class MoELayer:
+    """Owns the device tensors around one C-ABI layer: borrowed weights, the
+    workspace and the routing/statistics output buffers. Pointer marshalling
+    only; the forward itself is moe_forward + moe_aux_stats."""
+
+    def __init__(self, workload, weights: Dict[str, object], max_tokens: Optional[int] = None, device="cuda"):
+        import torch
+        w = workload
+        self.w = w
+        self.device = torch.device(device)
+        cfg = moe_config_default()
+        cfg.num_experts, cfg.num_active = w.E, w.k
+        cfg.input_dim, cfg.expert_dim, cfg.output_dim = w.d, w.F, w.O
+        cfg.num_shared = w.S
+        cfg.capacity_factor = w.capacity_factor
+        cfg.activation = MOE_ACT[w.activation]
+        cfg.top_k_method = MOE_TOPK[w.top_k_method]
+        cfg.use_selection_bias = int(w.use_selection_bias)
+        cfg.dtype = MOE_DTYPE[w.dtype]
+        cfg.max_tokens = max_tokens or 0
+        cfg.load_balance_coef, cfg.z_loss_coef, cfg.temperature = w.alpha, w.beta, 1.0
+        self.cfg = cfg
+        self.weights = {k: (v.to(self.device).contiguous() if v is not None else None)
+                        for k, v in weights.items()
+                        if k in ("w_gate", "b_gate", "sel_bias", "w1", "b1", "w2", "b2")}
+        ww = self.weights
+        self._cw = MoeWeights(_ptr(ww["w_gate"]), _ptr(ww.get("b_gate")), _ptr(ww.get("sel_bias")),
+                              _ptr(ww["w1"]), _ptr(ww["w2"]), _ptr(ww.get("b1")), _ptr(ww.get("b2")))
+        self.handle = moe_layer_create(cfg, self._cw)
+        self._ws = None
+        self._ws_T = -1
+        self._dt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
+
+    def close(self):
+        if getattr(self, "handle", None):
+            moe_destroy(self.handle)
+            self.handle = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    def workspace(self, T: int):
+        import torch
+        need = moe_workspace_bytes(self.handle, T)
+        if self._ws is None or self._ws.numel() < need:
+            self._ws = torch.empty(max(need, 256), dtype=torch.uint8, device=self.device)
+        return self._ws, need
+
+    def alloc_outputs(self, T: int):
+        import torch
+        w, dev = self.w, self.device
+        out = dict(
+            y=torch.empty(T, w.O, dtype=self._dt, device=dev),
+            logits=torch.empty(T, w.E, dtype=torch.float32, device=dev),
+            gates=torch.empty(T, w.k, dtype=torch.float32, device=dev),
+            topk_idx=torch.empty(T, w.k, dtype=torch.int32, device=dev),
+            slot=torch.empty(T, w.k, dtype=torch.int32, device=dev),
+            count_pre=torch.empty(w.E, dtype=torch.int32, device=dev),
+            count_kept=torch.empty(w.E, dtype=torch.int32, device=dev),
+            f=torch.empty(w.E, dtype=torch.float32, device=dev),
+            p_mean=torch.empty(w.E, dtype=torch.float32, device=dev),
+            l_aux=torch.empty(1, dtype=torch.float32, device=dev),
+            l_z=torch.empty(1, dtype=torch.float32, device=dev),
+            n_dropped=torch.empty(1, dtype=torch.int32, device=dev),
+            credit=torch.empty(T, w.k, dtype=torch.float32, device=dev),
+            expert_loss=torch.empty(w.E, dtype=torch.float32, device=dev),
+        )
+        return out
+
+    def forward(self, x, noise=None, out=None, stream=None, with_routing=True):
+        import torch
+        T = int(x.shape[0])
+        if out is None:
+            out = self.alloc_outputs(T)
+        ws, need = self.workspace(T)
+        s = stream if stream is not None else torch.cuda.current_stream(self.device).cuda_stream
+        routing = None
+        if with_routing:
+            routing = MoeRouting(_ptr(out["logits"]), _ptr(out["gates"]), _ptr(out["topk_idx"]), _ptr(out["slot"]),
+                                 _ptr(out["count_pre"]), _ptr(out["count_kept"]))
+        moe_forward(self.handle, _ptr(x), T, _ptr(noise), ws.data_ptr(), ws.numel(), _ptr(out["y"]), routing, s)
+        return out
+
+    def aux_stats(self, out, token_loss=None, stream=None):
+        import torch
+        s = stream if stream is not None else torch.cuda.current_stream(self.device).cuda_stream
+        st = MoeStats(_ptr(out["f"]), _ptr(out["p_mean"]), _ptr(out["l_aux"]), _ptr(out["l_z"]),
+                      _ptr(out["n_dropped"]), _ptr(out["credit"]),
+                      _ptr(out["expert_loss"]) if token_loss is not None else None)
+        moe_aux_stats(self.handle, _ptr(token_loss), st, s)
+        return out
+
+    def device_status(self, stream=None) -> int:
+        import torch
+        s = stream if stream is not None else torch.cuda.current_stream(self.device).cuda_stream
+        return moe_device_status(self.handle, s)
+
+    def launch_count(self) -> int:
+        return moe_launch_count(self.handle)

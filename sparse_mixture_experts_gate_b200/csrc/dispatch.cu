@@ -1,0 +1,179 @@
+// dispatch.cu - capacity-capped dispatch of token assignments to expert buffers.
+//
+// "Appendix C - Acronyms & Symbols", table "Capacity & communication": each
+// expert has a fixed buffer of C = ceil(C_f k T / E) tokens and the dispatch
+// tensor D scatters tokens into those buffers; "Code Walkthrough - SER", "Load
+// balancing": a hard per-expert cap drops overflow tokens. Priority inside an
+// expert's buffer is ascending token index (a stable ranking).
+//
+// Instead of a dense one-hot D, the dispatch is a permutation into a compact row
+// space: expert e owns rows [group_start[e], group_start[e] + kept_e), padded to
+// a multiple of the GEMM M tile, followed by one T-row segment per shared
+// expert. Three launches:
+//   count  - per 256-token chunk, a histogram of selections (shared-memory
+//            integer atomics: order-free, so deterministic);
+//   scan   - per expert, exclusive prefix over chunks; kept = min(count, C);
+//            exclusive scan of the padded kept counts -> segment starts, the
+//            M-tile -> group table and the row count;
+//   assign - per chunk, the stable rank of each assignment: chunk base +
+//            assignments to the same expert in earlier warps + earlier lanes of
+//            the same warp (a per-warp lane bitmask per expert, popcounted).
+// Also the gather of the routed token rows into the permuted layout.
+#include "moe_common.cuh"
+#include "moe_kernels.cuh"
+
+namespace moe {
+namespace {
+
+constexpr int kChunk = 256;  // tokens per chunk = threads per block
+constexpr int kMaxE = 256;
+
+__global__ void __launch_bounds__(kChunk) dispatch_count_kernel(DispatchArgs a) {
+    __shared__ int cnt[kMaxE];
+    for (int e = threadIdx.x; e < a.E; e += kChunk) cnt[e] = 0;
+    __syncthreads();
+    const int t = blockIdx.x * kChunk + threadIdx.x;
+    if (t < a.T)
+        for (int r = 0; r < a.k; ++r) atomicAdd(&cnt[a.idx[(int64_t)t * a.k + r]], 1);
+    __syncthreads();
+    for (int e = threadIdx.x; e < a.E; e += kChunk) a.chunk_count[(int64_t)blockIdx.x * a.E + e] = cnt[e];
+}
+
+// Single CTA of kMaxE threads; thread e owns expert e.
+__global__ void __launch_bounds__(kMaxE) dispatch_scan_kernel(DispatchArgs a) {
+    __shared__ int sc[kMaxE];
+    __shared__ int dropped_w[kMaxE / 32];
+    const int e = threadIdx.x, lane = e & 31, warp = e >> 5;
+    int pre = 0, kept = 0, padded = 0;
+    if (e < a.E) {
+        for (int c = 0; c < a.n_chunks; ++c) {
+            a.chunk_base[(int64_t)c * a.E + e] = pre;
+            pre += a.chunk_count[(int64_t)c * a.E + e];
+        }
+        kept = (int64_t)pre < a.C ? pre : (int)a.C;
+        padded = (kept + kBM - 1) / kBM * kBM;
+    }
+    // Inclusive scan of padded over the block (Hillis-Steele in shared memory).
+    sc[e] = padded;
+    __syncthreads();
+    for (int off = 1; off < kMaxE; off <<= 1) {
+        const int v = e >= off ? sc[e - off] : 0;
+        __syncthreads();
+        sc[e] += v;
+        __syncthreads();
+    }
+    const int start = sc[e] - padded;
+    const int routed_rows = sc[kMaxE - 1];
+    int drop = pre - kept;
+    for (int off = 16; off > 0; off >>= 1) drop += __shfl_xor_sync(0xffffffffu, drop, off);
+    if (lane == 0) dropped_w[warp] = drop;
+    if (e < a.E) {
+        a.count_pre[e] = pre;
+        a.count_kept[e] = kept;
+        if (a.user_count_pre) a.user_count_pre[e] = pre;
+        if (a.user_count_kept) a.user_count_kept[e] = kept;
+        a.group_start[e] = start;
+        a.group_rows[e] = kept;
+        for (int m = start / kBM; m < (start + padded) / kBM; ++m) a.tile_group[m] = e;
+        for (int r = start + kept; r < start + padded; ++r) a.row_assign[r] = -1;
+    }
+    // Shared experts: one T_pad-row segment each, after the routed rows.
+    const int shared_tiles = a.T_pad / kBM;
+    for (int i = e; i < a.S * shared_tiles; i += kMaxE) a.tile_group[routed_rows / kBM + i] = a.E + i / shared_tiles;
+    if (e < a.S) {
+        a.group_start[a.E + e] = routed_rows + e * a.T_pad;
+        a.group_rows[a.E + e] = a.T;
+    }
+    __syncthreads();
+    if (e == 0) {
+        int d = 0;
+        for (int w = 0; w < kMaxE / 32; ++w) d += dropped_w[w];
+        const int total = routed_rows + a.S * a.T_pad;
+        a.group_start[a.E + a.S] = total;
+        a.ctrl[kCtrlNumMTiles] = total / kBM;
+        a.ctrl[kCtrlRoutedRows] = routed_rows;
+        a.ctrl[kCtrlDropped] = d;
+    }
+}
+
+__global__ void __launch_bounds__(kChunk) dispatch_assign_kernel(DispatchArgs a) {
+    constexpr int W = kChunk / 32;
+    __shared__ uint32_t mask[W][kMaxE];
+    __shared__ int wbase[W][kMaxE];
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    for (int i = tid; i < W * kMaxE; i += kChunk) (&mask[0][0])[i] = 0u;
+    __syncthreads();
+    const int t = blockIdx.x * kChunk + tid;
+    if (t < a.T)
+        for (int r = 0; r < a.k; ++r) atomicOr(&mask[warp][a.idx[(int64_t)t * a.k + r]], 1u << lane);
+    __syncthreads();
+    for (int e = tid; e < a.E; e += kChunk) {
+        int run = a.chunk_base[(int64_t)blockIdx.x * a.E + e];
+        for (int w = 0; w < W; ++w) {
+            wbase[w][e] = run;
+            run += __popc(mask[w][e]);
+        }
+    }
+    __syncthreads();
+    if (t >= a.T) return;
+    const uint32_t lt = (1u << lane) - 1u;
+    for (int r = 0; r < a.k; ++r) {
+        const int64_t ai = (int64_t)t * a.k + r;
+        const int e = a.idx[ai];
+        const int rank = wbase[warp][e] + __popc(mask[warp][e] & lt);
+        const bool kept = (int64_t)rank < a.C;
+        a.slot[ai] = kept ? rank : -1;
+        int row = -1;
+        if (kept) {
+            row = a.group_start[e] + rank;
+            a.row_assign[row] = (int)ai;
+        }
+        a.row_of[ai] = row;
+    }
+}
+
+// One warp per row of the routed region; 16-byte vectors.
+__global__ void __launch_bounds__(256) gather_rows_kernel(GatherArgs a) {
+    const int rows = min(a.ctrl[kCtrlRoutedRows], a.max_rows);
+    const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
+    const int nwarps = (gridDim.x * blockDim.x) >> 5;
+    const int nvec = a.row_bytes / 16;
+    for (int row = warp; row < rows; row += nwarps) {
+        const int ai = a.row_assign[row];
+        uint4 *dst = reinterpret_cast<uint4 *>(static_cast<char *>(a.xp) + (int64_t)row * a.row_bytes);
+        if (ai < 0) {
+            for (int v = lane; v < nvec; v += 32) dst[v] = make_uint4(0u, 0u, 0u, 0u);
+        } else {
+            const int t = ai / a.k;
+            const uint4 *src =
+                reinterpret_cast<const uint4 *>(static_cast<const char *>(a.x) + (int64_t)t * a.row_bytes);
+            for (int v = lane; v < nvec; v += 32) dst[v] = __ldg(src + v);
+        }
+    }
+}
+
+}  // namespace
+
+cudaError_t launch_dispatch(const DispatchArgs &a, cudaStream_t s, int *launches) {
+    if (a.T <= 0) return cudaSuccess;
+    dispatch_count_kernel<<<a.n_chunks, kChunk, 0, s>>>(a);
+    dispatch_scan_kernel<<<1, kMaxE, 0, s>>>(a);
+    dispatch_assign_kernel<<<a.n_chunks, kChunk, 0, s>>>(a);
+    *launches += 3;
+    return cudaGetLastError();
+}
+
+cudaError_t launch_gather(const GatherArgs &a, cudaStream_t s, int *launches) {
+    int dev = 0, sms = 148;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const int warps_needed = a.max_rows;
+    int blocks = (warps_needed + 7) / 8;
+    if (blocks > sms * 8) blocks = sms * 8;
+    if (blocks < 1) blocks = 1;
+    gather_rows_kernel<<<blocks, 256, 0, s>>>(a);
+    ++*launches;
+    return cudaGetLastError();
+}
+
+}  // namespace moe

@@ -1,0 +1,545 @@
+// moe_api.cu - the C ABI declared in include/moe.h: argument validation, the
+// workspace plan, TMA descriptors, and the launch sequence of one MoE layer
+// forward (router -> dispatch -> gather -> expert GEMM 1 -> expert GEMM 2 ->
+// combine) and of its statistics.
+#include <algorithm>
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <string>
+
+#include "moe.h"
+#include "moe_common.cuh"
+#include "moe_kernels.cuh"
+
+using namespace moe;
+
+namespace {
+
+thread_local std::string g_last_error;
+
+int fail(int code, const char *fmt, ...) {
+    char buf[512];
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(buf, sizeof buf, fmt, ap);
+    va_end(ap);
+    g_last_error = buf;
+    return code;
+}
+
+size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+int64_t round_up(int64_t v, int64_t a) { return (v + a - 1) / a * a; }
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                  const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    if (!fn) {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    }
+    return fn;
+}
+
+// Row-major bf16 matrix [rows][inner] read in boxes of 64 x box_rows with 128B
+// swizzle (the layout the UMMA shared-memory descriptors expect).
+bool encode_bf16_2d(CUtensorMap *m, const void *base, uint64_t inner, uint64_t rows, uint32_t box_rows) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn || rows == 0) return false;
+    cuuint64_t dims[2] = {inner, rows};
+    cuuint64_t strides[1] = {inner * 2};
+    cuuint32_t box[2] = {static_cast<cuuint32_t>(kBK), box_rows};
+    cuuint32_t es[2] = {1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box, es,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+struct Plan {
+    int T = 0;
+    int64_t C = 0;
+    int T_pad = 0, n_rt = 0, n_chunks = 0, R_routed_max = 0, R_max = 0, max_mtiles = 0;
+    size_t o_ctrl, o_logits, o_idx, o_gates, o_slot, o_rowof, o_lse, o_psum, o_ccount, o_cbase, o_cpre, o_ckept,
+        o_gstart, o_grows, o_tgroup, o_rowassign, o_xp, o_h, o_o, o_norm, o_credit, o_pm, o_f;
+    size_t total = 0;
+};
+
+}  // namespace
+
+struct moe_layer {
+    moe_config_t cfg;
+    moe_weights_t w;
+    int G = 0;
+    bool tc = false;
+    int bn1 = 0, bn2 = 0, ntiles1 = 0, ntiles2 = 0;
+    int num_sms = 148;
+    CUtensorMap map_w1, map_w2;
+    // State of the most recent forward, read by moe_aux_stats.
+    bool has_forward = false;
+    Plan plan;
+    char *ws = nullptr;
+    int32_t *idx = nullptr, *count_pre = nullptr;
+    float *gates = nullptr;
+    int fwd_launches = 0, stats_launches = 0;
+    bool timing = false;
+    cudaEvent_t ev[MOE_TIMING_EVENTS];
+};
+
+namespace {
+
+int64_t capacity_of(const moe_config_t &c, int T) {
+    if (c.capacity_factor <= 0.f) return T;
+    return (int64_t)std::ceil((double)c.capacity_factor * (double)c.num_active * (double)T / (double)c.num_experts);
+}
+
+Plan make_plan(const moe_layer &L, int T) {
+    const moe_config_t &c = L.cfg;
+    Plan p;
+    p.T = T;
+    p.C = capacity_of(c, T);
+    const int E = c.num_experts, k = c.num_active, S = c.num_shared;
+    const int64_t kept_max = std::min<int64_t>((int64_t)k * T, (int64_t)E * p.C);
+    const int64_t routed = std::min<int64_t>(round_up(kept_max + (int64_t)E * (kBM - 1), kBM),
+                                             (int64_t)E * round_up(p.C, kBM));
+    p.R_routed_max = (int)routed;
+    p.T_pad = (int)round_up(T, kBM);
+    p.R_max = p.R_routed_max + S * p.T_pad;
+    p.max_mtiles = p.R_max / kBM;
+    const int rt = router_tile_tokens(E, T);
+    p.n_rt = (T + rt - 1) / rt;
+    p.n_chunks = (T + 255) / 256;
+    const size_t es = c.dtype == MOE_DTYPE_BF16 ? 2 : 4;
+    size_t off = 0;
+    auto take = [&](size_t bytes) {
+        const size_t o = off;
+        off = align_up(off + bytes, 256);
+        return o;
+    };
+    p.o_ctrl = take(kCtrlWords * 4);
+    p.o_logits = take((size_t)T * E * 4);
+    p.o_idx = take((size_t)T * k * 4);
+    p.o_gates = take((size_t)T * k * 4);
+    p.o_slot = take((size_t)T * k * 4);
+    p.o_rowof = take((size_t)T * k * 4);
+    p.o_lse = take((size_t)T * 4);
+    p.o_psum = take((size_t)p.n_rt * E * 4);
+    p.o_ccount = take((size_t)p.n_chunks * E * 4);
+    p.o_cbase = take((size_t)p.n_chunks * E * 4);
+    p.o_cpre = take((size_t)E * 4);
+    p.o_ckept = take((size_t)E * 4);
+    p.o_gstart = take((size_t)(E + S + 1) * 4);
+    p.o_grows = take((size_t)(E + S) * 4);
+    p.o_tgroup = take((size_t)p.max_mtiles * 4);
+    p.o_rowassign = take((size_t)p.R_max * 4);
+    p.o_pm = take((size_t)E * 4);
+    p.o_f = take((size_t)E * 4);
+    p.o_credit = take((size_t)T * k * 4);
+    p.o_norm = take((size_t)p.R_max * L.ntiles2 * 4);
+    p.o_xp = take((size_t)p.R_routed_max * c.input_dim * es);
+    p.o_h = take((size_t)p.R_max * c.expert_dim * es);
+    p.o_o = take((size_t)p.R_max * c.output_dim * es);
+    p.total = off;
+    return p;
+}
+
+int validate_config(const moe_config_t *c, const moe_weights_t *w) {
+    if (!c) return fail(MOE_ERR_INVALID_ARG, "cfg is NULL");
+    if (!w) return fail(MOE_ERR_INVALID_ARG, "weights is NULL");
+    if (c->num_experts < 1) return fail(MOE_ERR_INVALID_ARG, "num_experts must be >= 1 (got %d)", c->num_experts);
+    if (c->num_experts > 256)
+        return fail(MOE_ERR_UNSUPPORTED, "num_experts > 256 is not supported (got %d)", c->num_experts);
+    if (c->num_active < 1 || c->num_active > c->num_experts)
+        return fail(MOE_ERR_INVALID_ARG, "num_active must be in 1..num_experts (got %d, E=%d)", c->num_active,
+                    c->num_experts);
+    if (c->num_active > 16) return fail(MOE_ERR_UNSUPPORTED, "num_active > 16 is not supported");
+    if (c->input_dim < 1 || c->expert_dim < 1 || c->output_dim < 1)
+        return fail(MOE_ERR_INVALID_ARG, "input_dim, expert_dim and output_dim must be >= 1");
+    if (c->num_shared < 0) return fail(MOE_ERR_INVALID_ARG, "num_shared must be >= 0");
+    if (c->num_shared > 4) return fail(MOE_ERR_UNSUPPORTED, "num_shared > 4 is not supported");
+    if (c->activation < MOE_ACT_RELU || c->activation > MOE_ACT_SWISH)
+        return fail(MOE_ERR_INVALID_ARG, "unknown activation %d", c->activation);
+    if (c->top_k_method != MOE_TOPK_GREEDY && c->top_k_method != MOE_TOPK_NOISY)
+        return fail(MOE_ERR_INVALID_ARG, "unknown top_k_method %d", c->top_k_method);
+    if (c->dtype != MOE_DTYPE_BF16 && c->dtype != MOE_DTYPE_FP32)
+        return fail(MOE_ERR_INVALID_ARG, "unknown dtype %d", c->dtype);
+    if (c->max_tokens < 0) return fail(MOE_ERR_INVALID_ARG, "max_tokens must be >= 0");
+    if (!(c->temperature == 1.0f))
+        return fail(MOE_ERR_UNSUPPORTED, "router temperature other than 1 is not supported");
+    if (c->capacity_factor != c->capacity_factor) return fail(MOE_ERR_INVALID_ARG, "capacity_factor is NaN");
+    if (!w->w_gate) return fail(MOE_ERR_INVALID_ARG, "weights->w_gate is NULL");
+    if (!w->w1) return fail(MOE_ERR_INVALID_ARG, "weights->w1 is NULL");
+    if (!w->w2) return fail(MOE_ERR_INVALID_ARG, "weights->w2 is NULL");
+    if (c->use_selection_bias && !w->sel_bias)
+        return fail(MOE_ERR_INVALID_ARG, "use_selection_bias is set but weights->sel_bias is NULL");
+    if (c->dtype == MOE_DTYPE_BF16) {
+        if (c->input_dim % kBK || c->expert_dim % kBK)
+            return fail(MOE_ERR_UNSUPPORTED, "bf16 layers need input_dim and expert_dim multiples of %d", kBK);
+        if (gemm_pick_bn(c->expert_dim) == 0 || gemm_pick_bn(c->output_dim) == 0 || c->output_dim % 16)
+            return fail(MOE_ERR_UNSUPPORTED, "bf16 layers need expert_dim and output_dim multiples of 16");
+    } else {
+        if (c->input_dim % 4 || c->expert_dim % 4 || c->output_dim % 4)
+            return fail(MOE_ERR_UNSUPPORTED, "fp32 layers need input_dim, expert_dim, output_dim multiples of 4");
+    }
+    return MOE_OK;
+}
+
+cudaStream_t as_stream(void *s) { return reinterpret_cast<cudaStream_t>(s); }
+
+#define MOE_MARK(L, i, s)                                                                       \
+    do {                                                                                        \
+        if ((L)->timing) MOE_LAUNCH(cudaEventRecord((L)->ev[i], s));                            \
+    } while (0)
+
+#define MOE_LAUNCH(expr)                                                                              \
+    do {                                                                                              \
+        cudaError_t e_ = (expr);                                                                      \
+        if (e_ != cudaSuccess) return fail(MOE_ERR_CUDA, "%s failed: %s", #expr, cudaGetErrorString(e_)); \
+    } while (0)
+
+}  // namespace
+
+extern "C" {
+
+moe_config_t moe_config_default(void) {
+    moe_config_t c;
+    std::memset(&c, 0, sizeof c);
+    c.num_experts = 8;
+    c.num_active = 2;
+    c.input_dim = 512;
+    c.expert_dim = 1024;
+    c.output_dim = 512;
+    c.num_shared = 0;
+    c.capacity_factor = 1.25f;
+    c.activation = MOE_ACT_GELU;
+    c.top_k_method = MOE_TOPK_GREEDY;
+    c.use_selection_bias = 0;
+    c.dtype = MOE_DTYPE_BF16;
+    c.max_tokens = 0;
+    c.load_balance_coef = 0.01f;
+    c.z_loss_coef = 1e-3f;
+    c.temperature = 1.0f;
+    return c;
+}
+
+int moe_layer_create(const moe_config_t *cfg, const moe_weights_t *w, moe_layer_t **out) {
+    g_last_error.clear();
+    if (!out) return fail(MOE_ERR_INVALID_ARG, "out is NULL");
+    *out = nullptr;
+    int rc = validate_config(cfg, w);
+    if (rc != MOE_OK) return rc;
+    int dev = -1;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return fail(MOE_ERR_CUDA, "no CUDA device: %s", cudaGetErrorString(e));
+    int major = 0, minor = 0, sms = 0;
+    cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+    cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (major != 10 || minor != 0)
+        return fail(MOE_ERR_CUDA, "device %d is sm_%d%d; this library is built for sm_100a", dev, major, minor);
+    moe_layer *L = new moe_layer();
+    L->cfg = *cfg;
+    L->w = *w;
+    L->G = cfg->num_experts + cfg->num_shared;
+    L->num_sms = sms > 0 ? sms : 148;
+    L->tc = cfg->dtype == MOE_DTYPE_BF16;
+    if (L->tc) {
+        L->bn1 = gemm_pick_bn(cfg->expert_dim);
+        L->bn2 = gemm_pick_bn(cfg->output_dim);
+        L->ntiles1 = cfg->expert_dim / L->bn1;
+        L->ntiles2 = cfg->output_dim / L->bn2;
+        if (!encode_bf16_2d(&L->map_w1, w->w1, cfg->input_dim, (uint64_t)L->G * cfg->expert_dim, L->bn1) ||
+            !encode_bf16_2d(&L->map_w2, w->w2, cfg->expert_dim, (uint64_t)L->G * cfg->output_dim, L->bn2)) {
+            delete L;
+            return fail(MOE_ERR_CUDA, "cuTensorMapEncodeTiled failed for the expert weights (16-byte alignment?)");
+        }
+    } else {
+        L->ntiles1 = (cfg->expert_dim + kSimtBN - 1) / kSimtBN;
+        L->ntiles2 = (cfg->output_dim + kSimtBN - 1) / kSimtBN;
+    }
+    *out = L;
+    return MOE_OK;
+}
+
+size_t moe_workspace_bytes(const moe_layer_t *layer, int32_t T) {
+    if (!layer || T < 0) return 0;
+    return make_plan(*layer, T).total;
+}
+
+int64_t moe_capacity(const moe_layer_t *layer, int32_t T) {
+    if (!layer || T < 0) return -1;
+    return capacity_of(layer->cfg, T);
+}
+
+int moe_forward(moe_layer_t *L, const void *x, int32_t T, const float *logit_noise, void *workspace, size_t ws_bytes,
+                void *y, const moe_routing_t *routing, void *stream_v) {
+    g_last_error.clear();
+    if (!L) return fail(MOE_ERR_INVALID_ARG, "layer is NULL");
+    const moe_config_t &c = L->cfg;
+    if (T < 0) return fail(MOE_ERR_INVALID_ARG, "T must be >= 0 (got %d)", T);
+    if (c.max_tokens > 0 && T > c.max_tokens)
+        return fail(MOE_ERR_INVALID_ARG, "T=%d exceeds max_tokens=%d", T, c.max_tokens);
+    if (T > 0 && (!x || !y)) return fail(MOE_ERR_INVALID_ARG, "x and y are required when T > 0");
+    if (T > 0 && c.top_k_method == MOE_TOPK_NOISY && !logit_noise)
+        return fail(MOE_ERR_INVALID_ARG, "NOISY top-k needs logit_noise [T][E]");
+    const Plan p = make_plan(*L, T);
+    if (!workspace) return fail(MOE_ERR_WORKSPACE, "workspace is NULL");
+    if (reinterpret_cast<uintptr_t>(workspace) % 256)
+        return fail(MOE_ERR_WORKSPACE, "workspace must be 256-byte aligned");
+    if (ws_bytes < p.total)
+        return fail(MOE_ERR_WORKSPACE, "workspace too small: %zu bytes given, %zu needed for T=%d", ws_bytes, p.total, T);
+    if ((reinterpret_cast<uintptr_t>(x) | reinterpret_cast<uintptr_t>(y)) % 16)
+        return fail(MOE_ERR_INVALID_ARG, "x and y must be 16-byte aligned");
+
+    cudaStream_t s = as_stream(stream_v);
+    char *ws = static_cast<char *>(workspace);
+    L->has_forward = true;
+    L->plan = p;
+    L->ws = ws;
+    L->fwd_launches = 0;
+    L->stats_launches = 0;
+    int32_t *ctrl = reinterpret_cast<int32_t *>(ws + p.o_ctrl);
+    MOE_LAUNCH(cudaMemsetAsync(ctrl, 0, kCtrlWords * 4, s));
+    if (T == 0) return MOE_OK;
+    MOE_MARK(L, 0, s);
+
+    const int E = c.num_experts, k = c.num_active, S = c.num_shared;
+    const moe_routing_t *rt = routing;
+    float *logits = rt && rt->logits ? rt->logits : reinterpret_cast<float *>(ws + p.o_logits);
+    int32_t *idx = rt && rt->topk_idx ? rt->topk_idx : reinterpret_cast<int32_t *>(ws + p.o_idx);
+    float *gates = rt && rt->gates ? rt->gates : reinterpret_cast<float *>(ws + p.o_gates);
+    int32_t *slot = rt && rt->slot ? rt->slot : reinterpret_cast<int32_t *>(ws + p.o_slot);
+    L->idx = idx;
+    L->gates = gates;
+    L->count_pre = reinterpret_cast<int32_t *>(ws + p.o_cpre);
+    int *nl = &L->fwd_launches;
+
+    RouterArgs ra;
+    ra.x = x;
+    ra.x_bf16 = c.dtype == MOE_DTYPE_BF16;
+    ra.w_gate = L->w.w_gate;
+    ra.b_gate = L->w.b_gate;
+    ra.noise = c.top_k_method == MOE_TOPK_NOISY ? logit_noise : nullptr;
+    ra.sel_bias = c.use_selection_bias ? L->w.sel_bias : nullptr;
+    ra.T = T;
+    ra.d = c.input_dim;
+    ra.E = E;
+    ra.k = k;
+    ra.logits = logits;
+    ra.idx = idx;
+    ra.gates = gates;
+    ra.lse = reinterpret_cast<float *>(ws + p.o_lse);
+    ra.psum_part = reinterpret_cast<float *>(ws + p.o_psum);
+    MOE_LAUNCH(launch_router(ra, s, nl));
+    MOE_MARK(L, 1, s);
+
+    DispatchArgs da;
+    da.idx = idx;
+    da.T = T;
+    da.E = E;
+    da.k = k;
+    da.S = S;
+    da.C = p.C;
+    da.T_pad = p.T_pad;
+    da.n_chunks = p.n_chunks;
+    da.chunk_count = reinterpret_cast<int32_t *>(ws + p.o_ccount);
+    da.chunk_base = reinterpret_cast<int32_t *>(ws + p.o_cbase);
+    da.count_pre = reinterpret_cast<int32_t *>(ws + p.o_cpre);
+    da.count_kept = reinterpret_cast<int32_t *>(ws + p.o_ckept);
+    da.user_count_pre = rt ? rt->count_pre : nullptr;
+    da.user_count_kept = rt ? rt->count_kept : nullptr;
+    da.group_start = reinterpret_cast<int32_t *>(ws + p.o_gstart);
+    da.group_rows = reinterpret_cast<int32_t *>(ws + p.o_grows);
+    da.tile_group = reinterpret_cast<int32_t *>(ws + p.o_tgroup);
+    da.ctrl = ctrl;
+    da.slot = slot;
+    da.row_of = reinterpret_cast<int32_t *>(ws + p.o_rowof);
+    da.row_assign = reinterpret_cast<int32_t *>(ws + p.o_rowassign);
+    MOE_LAUNCH(launch_dispatch(da, s, nl));
+    MOE_MARK(L, 2, s);
+
+    const size_t es = c.dtype == MOE_DTYPE_BF16 ? 2 : 4;
+    GatherArgs ga;
+    ga.x = x;
+    ga.xp = ws + p.o_xp;
+    ga.row_assign = da.row_assign;
+    ga.ctrl = ctrl;
+    ga.k = k;
+    ga.row_bytes = (int)(c.input_dim * es);
+    ga.max_rows = p.R_routed_max;
+    MOE_LAUNCH(launch_gather(ga, s, nl));
+    MOE_MARK(L, 3, s);
+
+    GemmArgs g1;
+    g1.tile_group = da.tile_group;
+    g1.group_start = da.group_start;
+    g1.group_rows = da.group_rows;
+    g1.ctrl = ctrl;
+    g1.max_mtiles = p.max_mtiles;
+    g1.N = c.expert_dim;
+    g1.K = c.input_dim;
+    g1.n_tiles = L->ntiles1;
+    g1.E = E;
+    g1.use_a1 = 1;
+    g1.bias = L->w.b1;
+    g1.out = ws + p.o_h;
+    g1.norm_part = nullptr;
+    g1.act = c.activation;
+    g1.status = reinterpret_cast<uint32_t *>(ctrl + kCtrlStatus);
+    g1.num_sms = L->num_sms;
+    GemmArgs g2 = g1;
+    g2.N = c.output_dim;
+    g2.K = c.expert_dim;
+    g2.n_tiles = L->ntiles2;
+    g2.use_a1 = 0;
+    g2.bias = L->w.b2;
+    g2.out = ws + p.o_o;
+    g2.norm_part = reinterpret_cast<float *>(ws + p.o_norm);
+    g2.act = -1;
+
+    if (L->tc) {
+        CUtensorMap m_xp, m_x, m_h;
+        if (!encode_bf16_2d(&m_xp, ws + p.o_xp, c.input_dim, p.R_routed_max, kBM) ||
+            !encode_bf16_2d(&m_x, x, c.input_dim, T, kBM) ||
+            !encode_bf16_2d(&m_h, ws + p.o_h, c.expert_dim, p.R_max, kBM))
+            return fail(MOE_ERR_CUDA, "cuTensorMapEncodeTiled failed for the activations");
+        MOE_LAUNCH(launch_gemm_tc(m_xp, m_x, L->map_w1, g1, L->bn1, s, nl));
+        MOE_MARK(L, 4, s);
+        MOE_LAUNCH(launch_gemm_tc(m_h, m_h, L->map_w2, g2, L->bn2, s, nl));
+        MOE_MARK(L, 5, s);
+    } else {
+        GemmSimtArgs s1;
+        s1.g = g1;
+        s1.a0 = reinterpret_cast<const float *>(ws + p.o_xp);
+        s1.a1 = static_cast<const float *>(x);
+        s1.w = static_cast<const float *>(L->w.w1);
+        s1.max_rows = p.R_max;
+        MOE_LAUNCH(launch_gemm_simt(s1, s, nl));
+        MOE_MARK(L, 4, s);
+        GemmSimtArgs s2;
+        s2.g = g2;
+        s2.a0 = reinterpret_cast<const float *>(ws + p.o_h);
+        s2.a1 = nullptr;
+        s2.w = static_cast<const float *>(L->w.w2);
+        s2.max_rows = p.R_max;
+        MOE_LAUNCH(launch_gemm_simt(s2, s, nl));
+        MOE_MARK(L, 5, s);
+    }
+
+    CombineArgs ca;
+    ca.o = ws + p.o_o;
+    ca.norm_part = g2.norm_part;
+    ca.n_tiles = L->ntiles2;
+    ca.row_of = da.row_of;
+    ca.gates = gates;
+    ca.group_start = da.group_start;
+    ca.T = T;
+    ca.O = c.output_dim;
+    ca.E = E;
+    ca.S = S;
+    ca.k = k;
+    ca.bf16 = c.dtype == MOE_DTYPE_BF16;
+    ca.y = y;
+    ca.credit = reinterpret_cast<float *>(ws + p.o_credit);
+    MOE_LAUNCH(launch_combine(ca, s, nl));
+    MOE_MARK(L, 6, s);
+    return MOE_OK;
+}
+
+int moe_aux_stats(moe_layer_t *L, const float *token_loss, const moe_stats_t *out, void *stream_v) {
+    g_last_error.clear();
+    if (!L) return fail(MOE_ERR_INVALID_ARG, "layer is NULL");
+    if (!out) return fail(MOE_ERR_INVALID_ARG, "out is NULL");
+    if (!L->has_forward) return fail(MOE_ERR_STATE, "moe_aux_stats called before any moe_forward");
+    const Plan &p = L->plan;
+    const moe_config_t &c = L->cfg;
+    cudaStream_t s = as_stream(stream_v);
+    L->stats_launches = 0;
+    if (p.T == 0) return MOE_OK;
+    char *ws = L->ws;
+    StatsArgs sa;
+    sa.psum_part = reinterpret_cast<const float *>(ws + p.o_psum);
+    sa.n_router_tiles = p.n_rt;
+    sa.lse = reinterpret_cast<const float *>(ws + p.o_lse);
+    sa.count_pre = reinterpret_cast<const int32_t *>(ws + p.o_cpre);
+    sa.group_start = reinterpret_cast<const int32_t *>(ws + p.o_gstart);
+    sa.group_rows = reinterpret_cast<const int32_t *>(ws + p.o_grows);
+    sa.row_assign = reinterpret_cast<const int32_t *>(ws + p.o_rowassign);
+    sa.credit = reinterpret_cast<const float *>(ws + p.o_credit);
+    sa.token_loss = token_loss;
+    sa.ctrl = reinterpret_cast<const int32_t *>(ws + p.o_ctrl);
+    sa.T = p.T;
+    sa.E = c.num_experts;
+    sa.k = c.num_active;
+    sa.alpha = c.load_balance_coef;
+    sa.beta = c.z_loss_coef;
+    sa.p_mean_ws = reinterpret_cast<float *>(ws + p.o_pm);
+    sa.f_ws = reinterpret_cast<float *>(ws + p.o_f);
+    sa.f = out->f;
+    sa.p_mean = out->p_mean;
+    sa.l_aux = out->l_aux;
+    sa.l_z = out->l_z;
+    sa.expert_loss = out->expert_loss;
+    sa.n_dropped = out->n_dropped;
+    MOE_LAUNCH(launch_stats(sa, s, &L->stats_launches));
+    if (out->credit)
+        MOE_LAUNCH(cudaMemcpyAsync(out->credit, ws + p.o_credit, (size_t)p.T * c.num_active * 4,
+                                   cudaMemcpyDeviceToDevice, s));
+    MOE_MARK(L, 7, s);
+    return MOE_OK;
+}
+
+int moe_device_status(moe_layer_t *L, void *stream_v) {
+    g_last_error.clear();
+    if (!L) return fail(MOE_ERR_INVALID_ARG, "layer is NULL");
+    if (!L->has_forward) return fail(MOE_ERR_STATE, "no forward has run on this layer");
+    cudaStream_t s = as_stream(stream_v);
+    MOE_LAUNCH(cudaStreamSynchronize(s));
+    uint32_t st = 0;
+    MOE_LAUNCH(cudaMemcpy(&st, L->ws + L->plan.o_ctrl + kCtrlStatus * 4, 4, cudaMemcpyDeviceToHost));
+    if (st & kDevTimeout) return fail(MOE_ERR_TIMEOUT, "a bounded device-side wait gave up (status 0x%x)", st);
+    return MOE_OK;
+}
+
+int moe_set_timing_events(moe_layer_t *L, void *const *events) {
+    g_last_error.clear();
+    if (!L) return fail(MOE_ERR_INVALID_ARG, "layer is NULL");
+    if (!events) {
+        L->timing = false;
+        return MOE_OK;
+    }
+    for (int i = 0; i < MOE_TIMING_EVENTS; ++i) {
+        if (!events[i]) return fail(MOE_ERR_INVALID_ARG, "events[%d] is NULL", i);
+        L->ev[i] = reinterpret_cast<cudaEvent_t>(events[i]);
+    }
+    L->timing = true;
+    return MOE_OK;
+}
+
+int32_t moe_launch_count(const moe_layer_t *L) { return L ? L->fwd_launches + L->stats_launches : 0; }
+
+void moe_destroy(moe_layer_t *L) { delete L; }
+
+const char *moe_status_string(int status) {
+    switch (status) {
+        case MOE_OK: return "MOE_OK";
+        case MOE_ERR_INVALID_ARG: return "MOE_ERR_INVALID_ARG";
+        case MOE_ERR_UNSUPPORTED: return "MOE_ERR_UNSUPPORTED";
+        case MOE_ERR_CUDA: return "MOE_ERR_CUDA";
+        case MOE_ERR_WORKSPACE: return "MOE_ERR_WORKSPACE";
+        case MOE_ERR_TIMEOUT: return "MOE_ERR_TIMEOUT";
+        case MOE_ERR_STATE: return "MOE_ERR_STATE";
+        default: return "MOE_ERR_UNKNOWN";
+    }
+}
+
+const char *moe_last_error(void) { return g_last_error.c_str(); }
+
+}  // extern "C"

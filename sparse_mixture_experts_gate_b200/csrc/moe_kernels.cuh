@@ -1,0 +1,137 @@
+// moe_kernels.cuh - argument blocks and host launchers of the MoE layer kernels.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace moe {
+
+// Router: logits h = W_g x + b, P = softmax(h), log-partition, selection key,
+// top-k, renormalised gates, and per-CTA partial sums of P over its tokens.
+struct RouterArgs {
+    const void *x;          // [T][d] bf16 or fp32
+    int x_bf16;
+    const float *w_gate;    // [E][d]
+    const float *b_gate;    // [E] or null
+    const float *noise;     // [T][E] or null (added to the selection key only)
+    const float *sel_bias;  // [E] or null (added to the selection key only)
+    int T, d, E, k;
+    float *logits;          // [T][E]
+    int32_t *idx;           // [T][k]
+    float *gates;           // [T][k]
+    float *lse;             // [T]
+    float *psum_part;       // [n_router_tiles][E]
+};
+int router_tile_tokens(int E, int T);
+cudaError_t launch_router(const RouterArgs &a, cudaStream_t s, int *launches);
+
+// Dispatch: histogram, scan, stable capacity-capped ranks, row map.
+struct DispatchArgs {
+    const int32_t *idx;     // [T][k]
+    int T, E, k, S;
+    int64_t C;              // capacity
+    int T_pad;              // T rounded up to kBM (shared-expert segment length)
+    int n_chunks;           // ceil(T / 256)
+    int32_t *chunk_count;   // [n_chunks][E]
+    int32_t *chunk_base;    // [n_chunks][E]
+    int32_t *count_pre;     // [E]
+    int32_t *count_kept;    // [E]
+    int32_t *user_count_pre;   // [E] or null
+    int32_t *user_count_kept;  // [E] or null
+    int32_t *group_start;   // [E+S+1]
+    int32_t *group_rows;    // [E+S]
+    int32_t *tile_group;    // [max_mtiles]
+    int32_t *ctrl;          // control block (see kCtrl*)
+    int32_t *slot;          // [T][k]
+    int32_t *row_of;        // [T][k]
+    int32_t *row_assign;    // [R_max]  t*k + r, or -1 on padding rows
+};
+cudaError_t launch_dispatch(const DispatchArgs &a, cudaStream_t s, int *launches);
+
+// Control block words.
+enum { kCtrlStatus = 0, kCtrlNumMTiles = 1, kCtrlRoutedRows = 2, kCtrlDropped = 3, kCtrlWords = 8 };
+
+// Gather of routed token rows into the permuted row space.
+struct GatherArgs {
+    const void *x;          // [T][d]
+    void *xp;               // [R_routed_max][d]
+    const int32_t *row_assign;
+    const int32_t *ctrl;
+    int k;
+    int row_bytes;          // d * element size (multiple of 16)
+    int max_rows;           // R_routed_max
+};
+cudaError_t launch_gather(const GatherArgs &a, cudaStream_t s, int *launches);
+
+// Grouped expert GEMM: out[row] = act(A[row] . W[g]^T + b[g]) for the rows of
+// every group g (routed experts, then shared experts).
+struct GemmArgs {
+    const int32_t *tile_group;   // [max_mtiles]
+    const int32_t *group_start;  // [G+1]
+    const int32_t *group_rows;   // [G]
+    const int32_t *ctrl;         // kCtrlNumMTiles
+    int max_mtiles;              // host bound on the M tiles (clamps the device count)
+    int N, K;                    // output row length, reduction length
+    int n_tiles;                 // N / BN
+    int E;                       // groups >= E read A through the second map (if use_a1)
+    int use_a1;
+    const float *bias;           // [G][N] or null
+    void *out;                   // [rows][N]
+    float *norm_part;            // [rows][n_tiles] or null: per-tile sum of out^2 (fp32, pre-rounding)
+    int act;                     // activation code, -1 none
+    uint32_t *status;            // device status word
+    int num_sms;
+};
+// bf16 tcgen05 path; BN chosen by the host (multiple of 16, <= 256, divides N).
+int gemm_pick_bn(int N);
+cudaError_t launch_gemm_tc(const CUtensorMap &map_a0, const CUtensorMap &map_a1, const CUtensorMap &map_b,
+                           const GemmArgs &a, int BN, cudaStream_t s, int *launches);
+// fp32 CUDA-core path (A operands as plain pointers).
+struct GemmSimtArgs {
+    GemmArgs g;
+    const float *a0;   // [rows][K] (routed rows, or all rows when !use_a1)
+    const float *a1;   // [T][K] (shared-expert rows when use_a1)
+    const float *w;    // [G][N][K]
+    int max_rows;      // rows the launch covers
+};
+constexpr int kSimtBN = 32;
+cudaError_t launch_gemm_simt(const GemmSimtArgs &a, cudaStream_t s, int *launches);
+
+// Gate-weighted combine with shared experts, plus credit.
+struct CombineArgs {
+    const void *o;          // [rows][O] expert outputs
+    const float *norm_part; // [rows][n_tiles]
+    int n_tiles;
+    const int32_t *row_of;  // [T][k]
+    const float *gates;     // [T][k]
+    const int32_t *group_start;
+    int T, O, E, S, k;
+    int bf16;
+    void *y;                // [T][O]
+    float *credit;          // [T][k]
+};
+cudaError_t launch_combine(const CombineArgs &a, cudaStream_t s, int *launches);
+
+// Balancing and credit statistics.
+struct StatsArgs {
+    const float *psum_part;   // [n_router_tiles][E]
+    int n_router_tiles;
+    const float *lse;         // [T]
+    const int32_t *count_pre; // [E]
+    const int32_t *group_start;
+    const int32_t *group_rows;
+    const int32_t *row_assign;
+    const float *credit;      // [T][k]
+    const float *token_loss;  // [T] or null
+    const int32_t *ctrl;
+    int T, E, k;
+    float alpha, beta;
+    float *p_mean_ws;         // [E] scratch
+    float *f_ws;              // [E] scratch
+    float *f, *p_mean, *l_aux, *l_z, *expert_loss;  // outputs (nullable)
+    int32_t *n_dropped;
+};
+cudaError_t launch_stats(const StatsArgs &a, cudaStream_t s, int *launches);
+
+}  // namespace moe

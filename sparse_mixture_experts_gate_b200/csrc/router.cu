@@ -1,0 +1,217 @@
+// router.cu - the gating step of the MoE layer forward.
+//
+// "Appendix C - Acronyms & Symbols", table "Core MoE symbols": router logits
+// h = W_g x (one score per expert), P = softmax(h), the top-k set T_k(x) and the
+// gates g_i (renormalised probabilities of the selected experts). "Code
+// Walkthrough - SER", gating / routing path: a linear router with a bias; noisy
+// top-k adds noise to the logits before selection. Appendix C, "Balancing": the
+// per-expert selection bias b_i and the log-partition that the z-loss squares.
+//
+// One CTA computes the logits of kTM tokens for all E <= 256 experts on fp32
+// CUDA cores, K-tiled through shared memory. Warp w owns tokens w*RT .. w*RT+RT-1
+// outright and lane l holds experts l, l+32, ..., so softmax, selection and
+// gates are warp-shuffle reductions in registers with no transpose. Selection
+// keys are formed with one fp32 round-to-nearest add; ties in the key go to the
+// lower expert index. Each CTA also writes the sum over its tokens of P (fixed
+// order), which the statistics kernel reduces across CTAs.
+#include "moe_common.cuh"
+#include "moe_kernels.cuh"
+
+namespace moe {
+namespace {
+
+constexpr int kThreads = 256;
+constexpr int kWarps = kThreads / 32;
+constexpr int kKC = 32;  // K chunk staged in shared memory
+
+template <typename XT, int RE, int RT>
+__global__ void __launch_bounds__(kThreads) router_simt_kernel(RouterArgs a) {
+    constexpr int TM = kWarps * RT;   // tokens per CTA
+    constexpr int EP = 32 * RE;       // padded expert count
+    __shared__ float xs[kKC][TM + 1];
+    __shared__ float ws[kKC][EP + 1];
+    __shared__ float psum_w[kWarps][EP];
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int t_base = blockIdx.x * TM;
+    const XT *x = static_cast<const XT *>(a.x);
+
+    float acc[RT][RE];
+#pragma unroll
+    for (int i = 0; i < RT; ++i)
+#pragma unroll
+        for (int q = 0; q < RE; ++q) acc[i][q] = 0.f;
+
+    for (int k0 = 0; k0 < a.d; k0 += kKC) {
+        // Stage x[t_base .. +TM][k0 .. +KC] transposed into xs[kk][t].
+        for (int i = tid; i < TM * kKC; i += kThreads) {
+            const int t = i / kKC, kk = i % kKC;
+            const int gt = t_base + t, gk = k0 + kk;
+            xs[kk][t] = (gt < a.T && gk < a.d) ? to_f32(x[(int64_t)gt * a.d + gk]) : 0.f;
+        }
+        // Stage W_g[0 .. EP][k0 .. +KC] transposed into ws[kk][e].
+        for (int i = tid; i < EP * kKC; i += kThreads) {
+            const int e = i / kKC, kk = i % kKC;
+            const int gk = k0 + kk;
+            ws[kk][e] = (e < a.E && gk < a.d) ? a.w_gate[(int64_t)e * a.d + gk] : 0.f;
+        }
+        __syncthreads();
+#pragma unroll 8
+        for (int kk = 0; kk < kKC; ++kk) {
+            float xv[RT], wv[RE];
+#pragma unroll
+            for (int i = 0; i < RT; ++i) xv[i] = xs[kk][warp * RT + i];
+#pragma unroll
+            for (int q = 0; q < RE; ++q) wv[q] = ws[kk][lane + 32 * q];
+#pragma unroll
+            for (int i = 0; i < RT; ++i)
+#pragma unroll
+                for (int q = 0; q < RE; ++q) acc[i][q] = fmaf(xv[i], wv[q], acc[i][q]);
+        }
+        __syncthreads();
+    }
+
+    float pacc[RE];
+#pragma unroll
+    for (int q = 0; q < RE; ++q) pacc[q] = 0.f;
+
+#pragma unroll
+    for (int i = 0; i < RT; ++i) {
+        const int t = t_base + warp * RT + i;
+        if (t >= a.T) break;  // warp-uniform
+        float h[RE], key[RE];
+        float m = -INFINITY;
+#pragma unroll
+        for (int q = 0; q < RE; ++q) {
+            const int e = lane + 32 * q;
+            if (e < a.E) {
+                h[q] = acc[i][q] + (a.b_gate ? a.b_gate[e] : 0.f);
+                a.logits[(int64_t)t * a.E + e] = h[q];
+                float kv = h[q];
+                if (a.noise)
+                    kv = __fadd_rn(h[q], a.noise[(int64_t)t * a.E + e]);
+                else if (a.sel_bias)
+                    kv = __fadd_rn(h[q], a.sel_bias[e]);
+                key[q] = kv;
+                m = fmaxf(m, h[q]);
+            } else {
+                h[q] = -INFINITY;
+                key[q] = -INFINITY;
+            }
+        }
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
+        float ex[RE], z = 0.f;
+#pragma unroll
+        for (int q = 0; q < RE; ++q) {
+            ex[q] = (lane + 32 * q < a.E) ? expf(h[q] - m) : 0.f;
+            z += ex[q];
+        }
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) z += __shfl_xor_sync(0xffffffffu, z, off);
+        const float inv_z = 1.f / z;
+#pragma unroll
+        for (int q = 0; q < RE; ++q) pacc[q] += ex[q] * inv_z;
+        if (lane == 0) a.lse[t] = m + logf(z);
+
+        // Top-k by (key desc, expert index asc); the winner's clean exp(h - m)
+        // feeds the gate.
+        uint32_t taken = 0u;
+        float gsel_sum = 0.f, my_gate_num = 0.f;
+        int my_idx = -1;
+        for (int r = 0; r < a.k; ++r) {
+            float bk = -INFINITY;
+            int be = 0x7fffffff;
+#pragma unroll
+            for (int q = 0; q < RE; ++q) {
+                const int e = lane + 32 * q;
+                if (e < a.E && !(taken & (1u << q))) {
+                    if (key[q] > bk || (key[q] == bk && e < be)) {
+                        bk = key[q];
+                        be = e;
+                    }
+                }
+            }
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1) {
+                const float ok = __shfl_xor_sync(0xffffffffu, bk, off);
+                const int oe = __shfl_xor_sync(0xffffffffu, be, off);
+                if (ok > bk || (ok == bk && oe < be)) {
+                    bk = ok;
+                    be = oe;
+                }
+            }
+            // Owner lane of expert `be` marks it taken and broadcasts exp(h - m).
+            const int owner = be & 31, oq = be >> 5;
+            float num = 0.f;
+            if (lane == owner) {
+#pragma unroll
+                for (int q = 0; q < RE; ++q)
+                    if (q == oq) {
+                        taken |= (1u << q);
+                        num = ex[q];
+                    }
+            }
+            num = __shfl_sync(0xffffffffu, num, owner);
+            gsel_sum += num;
+            if (lane == r) {
+                my_gate_num = num;
+                my_idx = be;
+            }
+        }
+        if (lane < a.k) {
+            a.idx[(int64_t)t * a.k + lane] = my_idx;
+            a.gates[(int64_t)t * a.k + lane] = my_gate_num / gsel_sum;
+        }
+    }
+
+    // Per-CTA column sums of P over this CTA's tokens, warps in fixed order.
+#pragma unroll
+    for (int q = 0; q < RE; ++q) psum_w[warp][lane + 32 * q] = pacc[q];
+    __syncthreads();
+    for (int e = tid; e < a.E; e += kThreads) {
+        float s = 0.f;
+#pragma unroll
+        for (int w = 0; w < kWarps; ++w) s += psum_w[w][e];
+        a.psum_part[(int64_t)blockIdx.x * a.E + e] = s;
+    }
+}
+
+template <typename XT, int RE>
+cudaError_t launch_re(const RouterArgs &a, cudaStream_t s, int rt) {
+    if (rt == 4) {
+        constexpr int TM = kWarps * 4;
+        router_simt_kernel<XT, RE, 4><<<(a.T + TM - 1) / TM, kThreads, 0, s>>>(a);
+    } else {
+        constexpr int TM = kWarps * 1;
+        router_simt_kernel<XT, RE, 1><<<(a.T + TM - 1) / TM, kThreads, 0, s>>>(a);
+    }
+    return cudaGetLastError();
+}
+
+template <typename XT>
+cudaError_t launch_x(const RouterArgs &a, cudaStream_t s, int rt) {
+    if (a.E <= 32) return launch_re<XT, 1>(a, s, rt);
+    if (a.E <= 64) return launch_re<XT, 2>(a, s, rt);
+    if (a.E <= 128) return launch_re<XT, 4>(a, s, rt);
+    return launch_re<XT, 8>(a, s, rt);
+}
+
+int router_rt(int T) { return T >= 4096 ? 4 : 1; }
+
+}  // namespace
+
+// Tokens per router CTA (the granularity of the P partial sums).
+int router_tile_tokens(int E, int T) {
+    (void)E;
+    return kWarps * router_rt(T);
+}
+
+cudaError_t launch_router(const RouterArgs &a, cudaStream_t s, int *launches) {
+    if (a.T <= 0) return cudaSuccess;
+    ++*launches;
+    const int rt = router_rt(a.T);
+    return a.x_bf16 ? launch_x<__nv_bfloat16>(a, s, rt) : launch_x<float>(a, s, rt);
+}
+
+}  // namespace moe

@@ -89,25 +89,53 @@ _TAGS = {"x": 1, "w_gate": 2, "b_gate": 3, "sel_bias": 4, "w1": 5, "b1": 6, "w2"
          "b2": 8, "noise": 9, "token_loss": 10}
 
 
-def _gen(device: str, seed: int, tag: str) -> torch.Generator:
+def _gen(device: str, seed: int, tag: str, sub: int = 0) -> torch.Generator:
     g = torch.Generator(device=device)
-    g.manual_seed(seed * 1000 + _TAGS[tag])
+    g.manual_seed(seed * 1000 + _TAGS[tag] + 100003 * sub)
     return g
 
 
-def _normal(shape, std: float, device: str, seed: int, tag: str, out_dtype: torch.dtype,
-            chunk_dim0: bool = False) -> torch.Tensor:
+def _normal(shape, std: float, device: str, seed: int, tag: str, out_dtype: torch.dtype) -> torch.Tensor:
     g = _gen(device, seed, tag)
-    if not chunk_dim0:
-        t = torch.randn(shape, generator=g, device=device, dtype=torch.float32)
-        t.mul_(std)
-        return t.to(out_dtype)
-    # Large per-expert stacks: draw one expert at a time to bound fp32 scratch.
-    out = torch.empty(shape, device=device, dtype=out_dtype)
-    for e in range(shape[0]):
-        t = torch.randn(shape[1:], generator=g, device=device, dtype=torch.float32)
-        t.mul_(std)
-        out[e].copy_(t)
+    t = torch.randn(shape, generator=g, device=device, dtype=torch.float32)
+    t.mul_(std)
+    return t.to(out_dtype)
+
+
+def _expert_normal(e: int, shape, std: float, device: str, seed: int, tag: str,
+                   out_dtype: torch.dtype) -> torch.Tensor:
+    """One expert's slice of an expert stack, from its own generator, so any
+    subset of experts can be drawn without drawing the others."""
+    g = _gen(device, seed, tag, sub=e + 1)
+    t = torch.randn(shape, generator=g, device=device, dtype=torch.float32)
+    t.mul_(std)
+    return t.to(out_dtype)
+
+
+def _expert_stack(G: int, shape, std: float, device: str, seed: int, tag: str,
+                  out_dtype: torch.dtype) -> torch.Tensor:
+    out = torch.empty((G,) + tuple(shape), device=device, dtype=out_dtype)
+    for e in range(G):
+        out[e].copy_(_expert_normal(e, shape, std, device, seed, tag, out_dtype))
+    return out
+
+
+def make_expert_weights(w: "Workload", experts, device: str = "cpu", seed: Optional[int] = None,
+                        random_biases: bool = False) -> Dict[str, Dict[int, torch.Tensor]]:
+    """The w1, b1, w2, b2 slices of the listed experts only (dicts keyed by
+    expert index), identical to the same slices of make_inputs on that device."""
+    seed = w.seed if seed is None else seed
+    sdt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
+    out: Dict[str, Dict[int, torch.Tensor]] = {"w1": {}, "b1": {}, "w2": {}, "b2": {}}
+    for e in sorted(set(int(v) for v in experts)):
+        out["w1"][e] = _expert_normal(e, (w.F, w.d), (1.0 / w.d) ** 0.5, device, seed, "w1", sdt)
+        out["w2"][e] = _expert_normal(e, (w.O, w.F), (1.0 / w.F) ** 0.5, device, seed, "w2", sdt)
+        if random_biases:
+            out["b1"][e] = _expert_normal(e, (w.F,), (1.0 / w.d) ** 0.5, device, seed, "b1", torch.float32)
+            out["b2"][e] = _expert_normal(e, (w.O,), (1.0 / w.F) ** 0.5, device, seed, "b2", torch.float32)
+        else:
+            out["b1"][e] = torch.zeros(w.F, device=device)
+            out["b2"][e] = torch.zeros(w.O, device=device)
     return out
 
 
@@ -127,6 +155,45 @@ def load_zipf_row_scales(E: int) -> Optional[torch.Tensor]:
     return torch.tensor(vals, dtype=torch.float32)
 
 
+def make_tokens(w: Workload, device: str = "cpu", seed: Optional[int] = None) -> Dict[str, Optional[torch.Tensor]]:
+    """Per-batch inputs: x [T][d], noise [T][E] (noisy workloads), token_loss [T]."""
+    seed = w.seed if seed is None else seed
+    sdt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
+    out: Dict[str, Optional[torch.Tensor]] = {"x": _normal((w.T, w.d), 1.0, device, seed, "x", sdt)}
+    out["noise"] = _normal((w.T, w.E), 1.0 / w.E, device, seed, "noise", torch.float32) if w.noise else None
+    if w.token_loss:
+        g = _gen(device, seed, "token_loss")
+        u = torch.rand((2, w.T), generator=g, device=device, dtype=torch.float64)
+        # Gamma(2, 1) is the sum of two independent Exp(1) variates; 1 - u lies in (0, 1].
+        out["token_loss"] = (-torch.log1p(-u[0]) - torch.log1p(-u[1])).float()
+    else:
+        out["token_loss"] = None
+    return out
+
+
+def make_router(w: Workload, device: str = "cpu", seed: Optional[int] = None, random_biases: bool = False,
+                apply_zipf: bool = True) -> Dict[str, Optional[torch.Tensor]]:
+    """Router parameters: w_gate [E][d], b_gate [E] or None, sel_bias [E] or None."""
+    seed = w.seed if seed is None else seed
+    wg = _normal((w.E, w.d), (1.0 / w.d) ** 0.5, device, seed, "w_gate", torch.float32)
+    if w.zipf and apply_zipf:
+        s = load_zipf_row_scales(w.E)
+        if s is not None:
+            wg.mul_(s.to(device)[:, None])
+    out: Dict[str, Optional[torch.Tensor]] = {"w_gate": wg}
+    if w.router_bias:
+        out["b_gate"] = (_normal((w.E,), (1.0 / w.d) ** 0.5, device, seed, "b_gate", torch.float32)
+                         if random_biases else torch.zeros(w.E, device=device))
+    else:
+        out["b_gate"] = None
+    if w.use_selection_bias:
+        g = _gen(device, seed, "sel_bias")
+        out["sel_bias"] = (torch.rand(w.E, generator=g, device=device) * 0.2 - 0.1).float()
+    else:
+        out["sel_bias"] = None
+    return out
+
+
 def make_inputs(w: Workload, device: str = "cpu", seed: Optional[int] = None,
                 random_biases: bool = False, apply_zipf: bool = True) -> Dict[str, Optional[torch.Tensor]]:
     """Draw every input of one layer forward for workload `w` on `device`.
@@ -141,42 +208,15 @@ def make_inputs(w: Workload, device: str = "cpu", seed: Optional[int] = None,
     seed = w.seed if seed is None else seed
     sdt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
     G = w.n_groups
-    big = G * w.F * max(w.d, w.O) > (1 << 26)
     inp: Dict[str, Optional[torch.Tensor]] = {}
-    inp["x"] = _normal((w.T, w.d), 1.0, device, seed, "x", sdt)
-    wg = _normal((w.E, w.d), (1.0 / w.d) ** 0.5, device, seed, "w_gate", torch.float32)
-    if w.zipf and apply_zipf:
-        s = load_zipf_row_scales(w.E)
-        if s is not None:
-            wg.mul_(s.to(device)[:, None])
-    inp["w_gate"] = wg
-    if w.router_bias:
-        inp["b_gate"] = (_normal((w.E,), (1.0 / w.d) ** 0.5, device, seed, "b_gate", torch.float32)
-                         if random_biases else torch.zeros(w.E, device=device))
-    else:
-        inp["b_gate"] = None
-    if w.use_selection_bias:
-        g = _gen(device, seed, "sel_bias")
-        inp["sel_bias"] = (torch.rand(w.E, generator=g, device=device) * 0.2 - 0.1).float()
-    else:
-        inp["sel_bias"] = None
-    inp["w1"] = _normal((G, w.F, w.d), (1.0 / w.d) ** 0.5, device, seed, "w1", sdt, chunk_dim0=big)
-    inp["w2"] = _normal((G, w.O, w.F), (1.0 / w.F) ** 0.5, device, seed, "w2", sdt, chunk_dim0=big)
+    inp.update(make_tokens(w, device, seed))
+    inp.update(make_router(w, device, seed, random_biases, apply_zipf))
+    inp["w1"] = _expert_stack(G, (w.F, w.d), (1.0 / w.d) ** 0.5, device, seed, "w1", sdt)
+    inp["w2"] = _expert_stack(G, (w.O, w.F), (1.0 / w.F) ** 0.5, device, seed, "w2", sdt)
     if random_biases:
-        inp["b1"] = _normal((G, w.F), (1.0 / w.d) ** 0.5, device, seed, "b1", torch.float32)
-        inp["b2"] = _normal((G, w.O), (1.0 / w.F) ** 0.5, device, seed, "b2", torch.float32)
+        inp["b1"] = _expert_stack(G, (w.F,), (1.0 / w.d) ** 0.5, device, seed, "b1", torch.float32)
+        inp["b2"] = _expert_stack(G, (w.O,), (1.0 / w.F) ** 0.5, device, seed, "b2", torch.float32)
     else:
         inp["b1"] = torch.zeros(G, w.F, device=device)
         inp["b2"] = torch.zeros(G, w.O, device=device)
-    if w.noise:
-        inp["noise"] = _normal((w.T, w.E), 1.0 / w.E, device, seed, "noise", torch.float32)
-    else:
-        inp["noise"] = None
-    if w.token_loss:
-        g = _gen(device, seed, "token_loss")
-        u = torch.rand((2, w.T), generator=g, device=device, dtype=torch.float64)
-        # Gamma(2, 1) is the sum of two independent Exp(1) variates; 1 - u lies in (0, 1].
-        inp["token_loss"] = (-torch.log1p(-u[0]) - torch.log1p(-u[1])).float()
-    else:
-        inp["token_loss"] = None
     return inp

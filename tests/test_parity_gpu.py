@@ -1,0 +1,181 @@
+"""CUDA path vs the CPU oracle, element by element, through the C ABI (GPU)."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from gpu_harness import (check_end_to_end, check_expert_loss, check_same_logits_routing, expert_table,
+                         run_gpu)
+from sparse_mixture_experts_gate_b200.binding import MoEError, MoELayer
+from sparse_mixture_experts_gate_b200.workloads import WORKLOADS, make_inputs
+
+pytestmark = pytest.mark.gpu
+
+
+def full_check(w, inp):
+    g, layer = run_gpu(w, inp)
+    check_same_logits_routing(w, inp, g)
+    info = check_end_to_end(w, inp, g)
+    if inp.get("token_loss") is not None:
+        check_expert_loss(w, inp, g)
+    return g, info
+
+
+# ---------------------------------------------------------------- small cases
+
+def test_tiny_fp32_minimal_example():
+    """The walkthrough's minimal example: 4 experts, 2 active, 8/16/8, T=4, fp32."""
+    w = WORKLOADS["tiny"]
+    full_check(w, make_inputs(w, "cpu"))
+
+
+def test_tiny_fp32_random_biases():
+    w = WORKLOADS["tiny"].with_(T=37)
+    full_check(w, make_inputs(w, "cpu", seed=5, random_biases=True))
+
+
+@pytest.mark.parametrize("act", ["relu", "gelu", "swish"])
+def test_default_shape_ragged(act):
+    """Default SER shape, ragged T spanning several tiles, every activation,
+    random biases to exercise the fused epilogues."""
+    w = WORKLOADS["default"].with_(T=1000, activation=act)
+    full_check(w, make_inputs(w, "cpu", seed=11, random_biases=True))
+
+
+def test_default_full():
+    w = WORKLOADS["default"]
+    inp = make_inputs(w, "cpu")
+    g, info = full_check(w, inp)
+    assert g["n_dropped"][0] >= 0
+
+
+def test_e64_shape_small():
+    """Fine-grained experts (F=1408 -> N tile 176), a shared expert, selection bias."""
+    w = WORKLOADS["e64"].with_(T=700)
+    g, _ = full_check(w, make_inputs(w, "cpu", seed=3))
+    assert g["n_dropped"][0] > 0  # C_f = 1.25 at T=700 binds for some experts
+
+
+def test_decode_shape_noisy():
+    w = WORKLOADS["decode"]
+    full_check(w, make_inputs(w, "cpu"))
+
+
+def test_e256_shape_small():
+    w = WORKLOADS["e256"].with_(T=300)
+    full_check(w, make_inputs(w, "cpu", seed=9))
+
+
+# ---------------------------------------------------------------- edge cases
+
+def test_single_token():
+    w = WORKLOADS["e64"].with_(T=1)
+    full_check(w, make_inputs(w, "cpu"))
+
+
+def test_dense_reduction_E1_k1():
+    w = WORKLOADS["default"].with_(T=300, E=1, k=1, S=0, capacity_factor=0.0)
+    g, _ = full_check(w, make_inputs(w, "cpu", random_biases=True))
+    assert (g["topk_idx"] == 0).all() and np.allclose(g["gates"], 1.0)
+
+
+def test_k_equals_E_two_shared():
+    w = WORKLOADS["default"].with_(T=260, E=4, k=4, S=2, capacity_factor=0.0, activation="swish")
+    full_check(w, make_inputs(w, "cpu", seed=2, random_biases=True))
+
+
+def test_all_tokens_one_expert_heavy_drops():
+    """A large router bias on expert 0: every token selects it, and the cap
+    C = ceil(C_f k T / E) keeps only the earliest C tokens."""
+    w = WORKLOADS["default"].with_(T=900, capacity_factor=1.0, router_bias=True)
+    inp = make_inputs(w, "cpu", seed=4)
+    inp["b_gate"][0] = 50.0
+    g, _ = full_check(w, inp)
+    C = oracle.capacity(1.0, w.k, w.T, w.E)
+    assert g["count_pre"][0] == w.T and g["count_kept"][0] == C
+    assert g["n_dropped"][0] >= w.T - C
+    assert (g["slot"][:C, 0] == np.arange(C)).all() and (g["slot"][C:, 0] == -1).all()
+
+
+def test_tiny_capacity():
+    w = WORKLOADS["e64"].with_(T=200, capacity_factor=0.05)
+    g, _ = full_check(w, make_inputs(w, "cpu", seed=6))
+    assert (g["count_kept"] <= 1).all()
+
+
+def test_zero_tokens_is_a_noop():
+    w = WORKLOADS["default"]
+    inp = make_inputs(w.with_(T=4), "cpu")
+    layer = MoELayer(w, inp)
+    x = torch.empty(0, w.d, dtype=torch.bfloat16, device="cuda")
+    out = layer.forward(x)
+    layer.aux_stats(out)
+    torch.cuda.synchronize()
+    assert layer.device_status() == 0
+
+
+def test_determinism_bit_identical():
+    w = WORKLOADS["e64"].with_(T=1500)
+    inp = make_inputs(w, "cpu", seed=8)
+    g1, layer = run_gpu(w, inp)
+    g2, _ = run_gpu(w, inp, layer=layer)
+    for k in ("y", "logits", "gates", "topk_idx", "slot", "count_pre", "f", "p_mean", "l_aux", "l_z", "credit"):
+        assert np.array_equal(g1[k], g2[k], equal_nan=True), k
+
+
+def test_forward_argument_errors_on_host():
+    w = WORKLOADS["default"]
+    inp = make_inputs(w.with_(T=8), "cpu")
+    layer = MoELayer(w, inp, max_tokens=8)
+    x = inp["x"].cuda()
+    with pytest.raises(MoEError):  # T > max_tokens
+        layer.forward(torch.empty(9, w.d, dtype=torch.bfloat16, device="cuda"))
+    ws, need = layer.workspace(8)
+    from sparse_mixture_experts_gate_b200 import binding
+    y = torch.empty(8, w.O, dtype=torch.bfloat16, device="cuda")
+    s = torch.cuda.current_stream().cuda_stream
+    with pytest.raises(MoEError) as ei:
+        binding.moe_forward(layer.handle, x.data_ptr(), 8, None, ws.data_ptr(), need - 1, y.data_ptr(), None, s)
+    assert ei.value.code == binding.MOE_ERR_WORKSPACE
+    with pytest.raises(MoEError) as ei:
+        binding.moe_forward(layer.handle, x.data_ptr(), 8, None, ws.data_ptr() + 16, need, y.data_ptr(), None, s)
+    assert ei.value.code == binding.MOE_ERR_WORKSPACE
+    noisy = MoELayer(w.with_(top_k_method="noisy"), inp)
+    with pytest.raises(MoEError) as ei:
+        noisy.forward(x)  # NOISY without noise
+    assert ei.value.code == binding.MOE_ERR_INVALID_ARG
+    fresh = MoELayer(w, inp)
+    with pytest.raises(MoEError) as ei:
+        fresh.aux_stats(fresh.alloc_outputs(8))
+    assert ei.value.code == binding.MOE_ERR_STATE
+
+
+# ---------------------------------------------------------------- full sizes
+
+def _sampled_full(name, n_sample, seed=1234):
+    w = WORKLOADS[name]
+    inp = make_inputs(w, "cuda")
+    g, _ = run_gpu(w, inp, poison=False)
+    check_same_logits_routing(w, {k: (v.cpu() if v is not None else None) for k, v in inp.items()
+                                  if k in ("noise", "sel_bias")}, g)
+    rng = np.random.default_rng(seed)
+    toks = np.sort(rng.choice(w.T, size=n_sample, replace=False))
+    toks[-1] = w.T - 1  # always include the last token (ragged tail)
+    experts = g["topk_idx"][toks].ravel()
+    table = expert_table(w, inp, experts)
+    info = check_end_to_end(w, inp, g, tokens=toks, table=table)
+    if inp.get("token_loss") is not None:
+        check_expert_loss(w, {"token_loss": inp["token_loss"]}, g)
+    # Properties that hold at any size.
+    assert int(g["count_kept"].sum()) == w.k * w.T - int(g["n_dropped"][0])
+    assert int(g["count_pre"].sum()) == w.k * w.T
+    assert np.allclose(g["gates"].sum(1), 1.0, atol=1e-5)
+    return g, info
+
+
+def test_e64_full_size_sampled():
+    _sampled_full("e64", 48)
+
+
+def test_e256_full_size_sampled():
+    _sampled_full("e256", 24)
