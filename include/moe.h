@@ -190,6 +190,29 @@ MOE_API int moe_forward(moe_layer_t *layer, const void *x, int32_t T, const floa
                 void *workspace, size_t ws_bytes, void *y, const moe_routing_t *routing,
                 void *stream);
 
+/* Forward without a caller workspace. The source pages have no counterpart to
+ * this call; it exists for callers that cannot allocate device memory
+ * themselves, such as a plugin whose host application owns all device memory
+ * through its own pool, or a latency-critical loop that must not call
+ * cudaMalloc/cudaFree (they can synchronise the device).
+ * Same arguments, outputs and errors as moe_forward, minus the workspace: the
+ * scratch is a built-in device array of MOE_NOALLOC_SCRATCH_BYTES (64 MiB) that
+ * every GPU loading this library holds until process exit. Nothing is allocated.
+ *   - A T whose moe_workspace_bytes exceeds that size is rejected on the host
+ *     with MOE_ERR_WORKSPACE and nothing is enqueued (at the default SER shape,
+ *     512/1024/512 with 8 experts and 2 active, T = 4096 fits).
+ *   - The first call on a device looks up the array's device address (with that
+ *     device current); make that first call before any stream capture.
+ *   - All calls, on every layer and stream, share the one array and it keeps
+ *     the previous call's contents. The forward re-initialises everything it
+ *     reads (its control words are cleared at the start), but two calls whose
+ *     work overlaps on the GPU race on the array: serialise them (one stream,
+ *     or events). moe_aux_stats after this call reads the array too, so it must
+ *     run before the next moe_forward_noalloc. */
+#define MOE_NOALLOC_SCRATCH_BYTES (64u * 1024u * 1024u)
+MOE_API int moe_forward_noalloc(moe_layer_t *layer, const void *x, int32_t T, const float *logit_noise, void *y,
+                                const moe_routing_t *routing, void *stream);
+
 /* Balancing and credit statistics of the most recent moe_forward on this layer,
  * computed from what that forward left in its workspace (and routing buffers).
  *   token_loss [T] fp32 per-token losses l_t (NULL: expert_loss is not written)

@@ -21,7 +21,7 @@ MOE_DTYPE = {"bf16": 0, "fp32": 1}
 
 # Every symbol include/moe.h declares.
 EXPORTS = ("moe_config_default", "moe_layer_create", "moe_workspace_bytes", "moe_capacity", "moe_forward",
-           "moe_aux_stats", "moe_device_status", "moe_set_timing_events", "moe_launch_count", "moe_destroy", "moe_status_string",
+           "moe_forward_noalloc", "moe_aux_stats", "moe_device_status", "moe_set_timing_events", "moe_launch_count", "moe_destroy", "moe_status_string",
            "moe_last_error")
 
 
@@ -78,6 +78,8 @@ def lib() -> ctypes.CDLL:
         L.moe_capacity.argtypes = [vp, i32]
         L.moe_forward.restype = ctypes.c_int
         L.moe_forward.argtypes = [vp, vp, i32, vp, vp, sz, vp, ctypes.POINTER(MoeRouting), vp]
+        L.moe_forward_noalloc.restype = ctypes.c_int
+        L.moe_forward_noalloc.argtypes = [vp, vp, i32, vp, vp, ctypes.POINTER(MoeRouting), vp]
         L.moe_aux_stats.restype = ctypes.c_int
         L.moe_aux_stats.argtypes = [vp, vp, ctypes.POINTER(MoeStats), vp]
         L.moe_device_status.restype = ctypes.c_int
@@ -132,6 +134,17 @@ def moe_forward(layer: int, x: int, T: int, logit_noise: Optional[int], workspac
                 routing: Optional[MoeRouting], stream: int) -> int:
     r = ctypes.byref(routing) if routing is not None else None
     return _check(lib().moe_forward(layer, x, T, logit_noise, workspace, ws_bytes, y, r, stream), "moe_forward")
+
+
+MOE_NOALLOC_SCRATCH_BYTES = 64 * 1024 * 1024
+
+
+def moe_forward_noalloc(layer: int, x: int, T: int, logit_noise: Optional[int], y: int,
+                        routing: Optional[MoeRouting], stream: int) -> int:
+    """moe_forward with the library's built-in device scratch instead of a
+    caller workspace (for callers that cannot allocate device memory)."""
+    r = ctypes.byref(routing) if routing is not None else None
+    return _check(lib().moe_forward_noalloc(layer, x, T, logit_noise, y, r, stream), "moe_forward_noalloc")
 
 
 def moe_aux_stats(layer: int, token_loss: Optional[int], stats: MoeStats, stream: int) -> int:

@@ -74,6 +74,12 @@ struct Plan {
 
 }  // namespace
 
+namespace moe {
+// Records `msg` as the calling thread's last error (for moe_last_error) and
+// returns `code`; used by entry points defined in other files.
+int report_error(int code, const char *msg) { return fail(code, "%s", msg); }
+}  // namespace moe
+
 struct moe_layer {
     moe_config_t cfg;
     moe_weights_t w;

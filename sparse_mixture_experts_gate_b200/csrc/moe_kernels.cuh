@@ -134,4 +134,7 @@ struct StatsArgs {
 };
 cudaError_t launch_stats(const StatsArgs &a, cudaStream_t s, int *launches);
 
+// Sets the calling thread's last-error message; returns `code`.
+int report_error(int code, const char *msg);
+
 }  // namespace moe
