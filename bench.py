@@ -46,6 +46,9 @@ def parse():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    # Smaller variants of a workload, for profiler captures of the same kernels.
+    ap.add_argument("--tokens", type=int, default=None, help="override T (profiling)")
+    ap.add_argument("--experts", type=int, default=None, help="override E (profiling)")
     return ap.parse_args()
 
 
@@ -184,6 +187,10 @@ def run_ours(args):
     torch.cuda.set_device(dev)
 
     w = WORKLOADS[args.workload]
+    if args.tokens:
+        w = w.with_(T=args.tokens)
+    if args.experts:
+        w = w.with_(E=args.experts)
     inp = make_inputs(w, "cuda")
     if rank > 0:  # each replica routes its own batch of tokens
         inp.update(make_tokens(w, "cuda", seed=w.seed + 7919 * rank))
@@ -322,7 +329,7 @@ def run_ours(args):
         "config": {"workload": w.name, "T": T, "d": w.d, "d_ff": w.F, "out": w.O, "E": w.E, "k": w.k, "S": w.S,
                    "activation": w.activation, "capacity_factor": w.capacity_factor,
                    "tokens_per_rank": T, "parallelism": f"replicas x{world}",
-                   "l2": "inputs larger than L2 (x 470 MB, expert weights 15 GB); no flush"},
+                   "l2": l2_note(w)},
         "expert_gemm_tflops": step_tflops,
         "layer_roofline_frac": layer_frac,
         "roofline": {"kernel": "grouped_gemm_tc (expert GEMM 1 + 2)", "bound": "tensor", "achieved": achieved,
@@ -336,6 +343,14 @@ def run_ours(args):
     print(json.dumps(line), flush=True)
     if world > 1:
         dist.destroy_process_group()
+
+
+def l2_note(w):
+    es = 2 if w.dtype == "bf16" else 4
+    xb = w.T * w.d * es
+    wb = (w.E + w.S) * w.F * (w.d + w.O) * es
+    return (f"x {xb / 1e6:.0f} MB, expert weights {wb / 1e9:.1f} GB: "
+            + ("inputs larger than L2 (126 MB); no flush" if wb > 126e6 else "weights fit in L2"))
 
 
 def committed_traffic(w):
@@ -373,6 +388,10 @@ def run_reference(args):
     if rank != 0:
         return
     w = WORKLOADS[args.workload]
+    if args.tokens:
+        w = w.with_(T=args.tokens)
+    if args.experts:
+        w = w.with_(E=args.experts)
     threads = oracle_threads()
     # Calibrate: a step is a T_s-token sample sized to about 2 s of oracle work.
     router = make_router(w, "cpu")

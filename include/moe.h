@@ -77,7 +77,7 @@ typedef struct {
     int32_t num_active;       /* k, experts per token, 1..min(E, 16)                */
     int32_t input_dim;        /* d; multiple of 64 for BF16                         */
     int32_t expert_dim;       /* F = d_ff; multiple of 64 for BF16                  */
-    int32_t output_dim;       /* O; multiple of 16 for BF16                         */
+    int32_t output_dim;       /* O; multiple of 64 for BF16                         */
     int32_t num_shared;       /* S always-on shared experts (weight 1), 0..4        */
     float capacity_factor;    /* C_f; C = ceil(C_f k T / E). <= 0: no limit (C = T) */
     int32_t activation;       /* MOE_ACT_*                                          */
@@ -227,13 +227,13 @@ MOE_API int moe_device_status(moe_layer_t *layer, void *stream);
 /* Optional stage timing with caller-owned CUDA events (cudaEvent_t passed as
  * void*, created with timing enabled). After this call every moe_forward records
  *   events[0] before the router,        events[1] after the router,
- *   events[2] after the dispatch,       events[3] after the row gather,
- *   events[4] after expert GEMM 1,      events[5] after expert GEMM 2,
- *   events[6] after the combine,
- * and every moe_aux_stats records events[7] after its kernels, all on the
+ *   events[2] after the dispatch,       events[3] after expert GEMM 1 (and
+ *                                       the row gather that feeds it),
+ *   events[4] after expert GEMM 2,      events[5] after the combine,
+ * and every moe_aux_stats records events[6] after its kernels, all on the
  * call's stream. The array is copied; events == NULL turns timing off. Nothing
  * is allocated and nothing synchronises. */
-#define MOE_TIMING_EVENTS 8
+#define MOE_TIMING_EVENTS 7
 MOE_API int moe_set_timing_events(moe_layer_t *layer, void *const *events);
 
 /* Number of kernels the most recent moe_forward plus moe_aux_stats enqueued. */

@@ -18,7 +18,8 @@
 //   assign - per chunk, the stable rank of each assignment: chunk base +
 //            assignments to the same expert in earlier warps + earlier lanes of
 //            the same warp (a per-warp lane bitmask per expert, popcounted).
-// Also the gather of the routed token rows into the permuted layout.
+// Also the gather of the routed token rows into the permuted row space, which
+// the tensor-core expert GEMM then reads as plain 128-row TMA tiles.
 #include "moe_common.cuh"
 #include "moe_kernels.cuh"
 

@@ -23,7 +23,6 @@ __global__ void __launch_bounds__(256) grouped_gemm_simt_kernel(GemmSimtArgs p) 
     const int rows_total = min(a.ctrl[kCtrlNumMTiles], a.max_mtiles) * kBM;
     if (r0 >= rows_total) return;
     const int g = a.tile_group[r0 / kBM];
-    const bool use1 = a.use_a1 && g >= a.E;
     const int rows_valid_end = a.group_start[g] + a.group_rows[g];
     const float *w = p.w + (int64_t)g * a.N * a.K;
 
@@ -33,10 +32,11 @@ __global__ void __launch_bounds__(256) grouped_gemm_simt_kernel(GemmSimtArgs p) 
             const int row = r0 + i, kk = k0 + tx;
             float v = 0.f;
             if (row < rows_valid_end && kk < a.K) {
-                if (use1)
-                    v = p.a1[(int64_t)(row - a.group_start[g]) * a.K + kk];
-                else
-                    v = p.a0[(int64_t)row * a.K + kk];
+                int64_t arow = row;  // row space itself
+                if (p.gather) {      // token row of x: routed via the dispatch map, shared in order
+                    arow = g < a.E ? a.row_assign[row] / a.k : row - a.group_start[g];
+                }
+                v = p.a[arow * a.K + kk];
             }
             As[i][tx] = v;
             const int n = n0 + i;

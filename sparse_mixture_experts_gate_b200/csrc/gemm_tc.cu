@@ -5,247 +5,189 @@
 // dense contractions over the rows dispatched to it, so they run as one grouped
 // GEMM per layer over the permuted row space:
 //   out[row][n] = act( sum_k A[row][k] * W[g][n][k] + b[g][n] ),  g = group of row.
-// Layer 1: A = gathered x rows (routed) or x itself (shared experts), W = w1.
-// Layer 2: A = the hidden activations, W = w2; the epilogue also writes, per row
-// and N tile, the sum of squares of the fp32 outputs (for the credit norm).
-//
-// Design (one CTA per SM, persistent over 128 x BN output tiles, n fastest so
-// concurrently running CTAs share A and B tiles through L2):
-//   warp 0      TMA producer: A tile 128x64 and B tile BNx64 per stage, 128B
-//               swizzle, NS-stage ring guarded by full/empty mbarriers;
-//   warp 1      owns TMEM (512 columns = two fp32 accumulators of up to 256
-//               columns); one lane issues tcgen05.mma M=128 N=BN K=16 and
-//               tcgen05.commit to release stages and to publish accumulators;
-//   warps 2..5  epilogue: tcgen05.ld 32 lanes x 16 columns, bias, activation,
-//               bf16 store; accumulator ring of two so the epilogue of one tile
-//               overlaps the mainloop of the next.
-// Every wait is bounded (mbar_wait): on timeout the kernel flags the status
-// word, drains its own copies and MMAs, frees TMEM and returns.
+// Layer 1: A = the routed token rows gathered into row order (dispatch.cu), and
+//   x itself for the shared experts, which read every token in order.
+// Layer 2: A = the hidden activations H (already in row order);
+//   the epilogue also writes, per row and N tile, the fp32 sum of squares of
+//   the outputs (the credit's norm).
+// The pipeline (tc_pipeline.cuh): persistent CTAs over 128 x BN tiles, n fastest
+// so concurrently running CTAs share A and B tiles through L2; TMA producer
+// warp, single-lane MMA issuer, four epilogue warps, TMEM double buffering.
+// Epilogue: each warp turns its 32 accumulator rows into bf16 64 columns at a
+// time, writes them to a 128B-swizzled shared staging buffer (two per warp,
+// alternating) and one lane stores the 32 x 64 box with a TMA tensor store, so
+// global writes are whole, coalesced lines and never stall the warp. Rows past
+// an expert's kept count are padding rows of the row space (never read), so
+// tiles are stored whole.
 #include "moe_common.cuh"
 #include "moe_kernels.cuh"
+#include "tc_pipeline.cuh"
 
 namespace moe {
 namespace {
 
-constexpr int kThreads = 192;
-constexpr int kAccCols = 256;  // TMEM columns reserved per accumulator buffer
+constexpr int kStoreCols = 64;                        // columns per staged store box (128 bytes)
+constexpr int kStageBoxBytes = 32 * kStoreCols * 2;    // 32 rows x 128 bytes
+constexpr int kStagingBytes = 4 * 2 * kStageBoxBytes;  // 4 epilogue warps x 2 buffers
 
 template <int BN>
-struct TcCfg {
-    static constexpr int A_BYTES = kBM * kBK * 2;
-    static constexpr int B_BYTES = BN * kBK * 2;
-    static constexpr int STAGE = A_BYTES + B_BYTES;
-    static constexpr int NS = (200 * 1024) / STAGE < 8 ? (200 * 1024) / STAGE : 8;
-    static constexpr int SMEM = 1024 + NS * STAGE + 256;
-    static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "UMMA M=128 needs N % 16 == 0, 16..256");
-    static_assert(B_BYTES % 1024 == 0, "B tile must keep 1024-byte swizzle alignment");
-    static_assert(NS >= 2, "need at least two stages");
-};
+constexpr int gemm_smem_bytes() {
+    return (1024 + TcLayout<BN>::NS * TcLayout<BN>::STAGE + 256 + 1023) / 1024 * 1024 + kStagingBytes;
+}
 
-template <int BN>
-__global__ void __launch_bounds__(kThreads, 1)
+template <int BN, int ACT, bool NORM>
+__global__ void __launch_bounds__(kTcThreads, 1)
     grouped_gemm_tc_kernel(const __grid_constant__ CUtensorMap map_a0, const __grid_constant__ CUtensorMap map_a1,
-                           const __grid_constant__ CUtensorMap map_b, const GemmArgs a) {
-    using C = TcCfg<BN>;
-    constexpr int NS = C::NS;
+                           const __grid_constant__ CUtensorMap map_b, const __grid_constant__ CUtensorMap map_out,
+                           const GemmArgs a) {
+    static_assert(BN % kStoreCols == 0, "the N tile is stored in 64-column boxes");
     extern __shared__ uint8_t smem_raw[];
-    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint8_t *sA = smem;
-    uint8_t *sB = smem + NS * C::A_BYTES;
-    uint64_t *full = reinterpret_cast<uint64_t *>(smem + NS * C::STAGE);
-    uint64_t *empty = full + NS;
-    uint64_t *tfull = empty + NS;
-    uint64_t *tempty = tfull + 2;
-    uint64_t *mma_done = tempty + 2;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(mma_done + 1);
-
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const TcShared<BN> s = tc_carve<BN>(smem_raw);
+    uint8_t *staging = reinterpret_cast<uint8_t *>(
+        (reinterpret_cast<uintptr_t>(s.tmem_slot) + 64 + 1023) & ~uintptr_t(1023));
     if (threadIdx.x == 0) {
-        for (int s = 0; s < NS; ++s) {
-            mbar_init(&full[s], 1);
-            mbar_init(&empty[s], 1);
-        }
-        for (int i = 0; i < 2; ++i) {
-            mbar_init(&tfull[i], 1);
-            mbar_init(&tempty[i], 128);
-        }
-        mbar_init(mma_done, 1);
-        fence_barrier_init();
         tma_prefetch_desc(&map_a0);
         tma_prefetch_desc(&map_a1);
         tma_prefetch_desc(&map_b);
+        tma_prefetch_desc(&map_out);
     }
-    if (warp == 1) {
-        tmem_alloc(tmem_slot, 2 * kAccCols);
-        tmem_relinquish();
-    }
-    tc_fence_before_sync();
-    __syncthreads();
-    tc_fence_after_sync();
-    const uint32_t tmem_base = *tmem_slot;
-
+    const uint32_t tmem_base = tc_setup<BN>(s);
     const int num_m = min(a.ctrl[kCtrlNumMTiles], a.max_mtiles);
     const int total = num_m * a.n_tiles;
     const int kblocks = a.K / kBK;
-    uint32_t *status = a.status;
+    const int warp = threadIdx.x >> 5;
 
     if (warp == 0) {
-        if (lane == 0) {
-            uint32_t it = 0;
-            bool ok = true;
-            for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
-                const int m = tile / a.n_tiles, n = tile - m * a.n_tiles;
-                const int g = a.tile_group[m];
-                const CUtensorMap *ma = &map_a0;
-                int arow = m * kBM;
-                if (a.use_a1 && g >= a.E) {
-                    ma = &map_a1;
-                    arow = m * kBM - a.group_start[g];
-                }
-                const int brow = g * a.N + n * BN;
-                for (int kb = 0; kb < kblocks; ++kb, ++it) {
-                    const int s = it % NS;
-                    const uint32_t ph = (it / NS) & 1u;
-                    if (!mbar_wait(&empty[s], ph ^ 1u, status)) {
-                        ok = false;
-                        break;
-                    }
-                    mbar_arrive_expect_tx(&full[s], C::STAGE);
-                    tma_load_2d(ma, &full[s], sA + s * C::A_BYTES, kb * kBK, arow);
-                    tma_load_2d(&map_b, &full[s], sB + s * C::B_BYTES, kb * kBK, brow);
-                }
-            }
-            // Drain: every issued copy must land before the CTA may exit. On the
-            // normal path the consumer already waited for all of them.
-            if (!ok) {
-                for (uint32_t j = (it > (uint32_t)NS ? it - NS : 0u); j < it; ++j)
-                    mbar_wait_drain(&full[j % NS], (j / NS) & 1u);
-            }
-        }
-    } else if (warp == 1) {
-        if (lane == 0) {
-            constexpr uint32_t idesc = idesc_bf16_f32(kBM, BN);
-            uint32_t it = 0, tcount = 0;
-            bool ok = true;
-            for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x, ++tcount) {
-                const uint32_t acc = tcount & 1u, use = tcount >> 1;
-                if (!mbar_wait(&tempty[acc], (use & 1u) ^ 1u, status)) break;
-                tc_fence_after_sync();
-                const uint32_t d_tmem = tmem_base + acc * kAccCols;
-                for (int kb = 0; kb < kblocks; ++kb, ++it) {
-                    const int s = it % NS;
-                    const uint32_t ph = (it / NS) & 1u;
-                    if (!mbar_wait(&full[s], ph, status)) {
-                        ok = false;
-                        break;
-                    }
-                    tc_fence_after_sync();
-                    const uint64_t ad = sw128_kmajor_desc(smem_u32(sA + s * C::A_BYTES));
-                    const uint64_t bd = sw128_kmajor_desc(smem_u32(sB + s * C::B_BYTES));
-#pragma unroll
-                    for (int kk = 0; kk < kBK / 16; ++kk)
-                        tc_mma_bf16(d_tmem, ad + 2u * kk, bd + 2u * kk, idesc, (kb | kk) != 0 ? 1u : 0u);
-                    tc_commit(&empty[s]);
-                }
-                if (ok) tc_commit(&tfull[acc]);
-            }
-            // All MMAs this thread issued are complete once mma_done flips.
-            tc_commit(mma_done);
-            mbar_wait_drain(mma_done, 0u);
-        }
-    } else {
-        const int q = warp & 3;  // TMEM lane quarter this warp may access
-        const int lrow = q * 32 + lane;
-        uint32_t tcount = 0;
-        for (int tile = blockIdx.x; tile < total; tile += gridDim.x, ++tcount) {
+        const CUtensorMap *ma = &map_a0;
+        int arow = 0, brow = 0;
+        auto tile_begin = [&](int tile, int) {
             const int m = tile / a.n_tiles, n = tile - m * a.n_tiles;
-            const uint32_t acc = tcount & 1u, use = tcount >> 1;
-            // tcgen05.ld below is warp-collective: make the outcome warp-uniform.
-            const bool got = mbar_wait(&tfull[acc], use & 1u, status);
-            if (!__all_sync(0xffffffffu, got)) break;
-            tc_fence_after_sync();
             const int g = a.tile_group[m];
-            const int grow = m * kBM + lrow;
-            const bool valid = grow < a.group_start[g] + a.group_rows[g];
-            const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * kAccCols;
+            brow = g * a.N + n * BN;
+            ma = &map_a0;
+            arow = m * kBM;
+            if (a.use_a1 && g >= a.E) {  // shared expert: rows of x in token order
+                ma = &map_a1;
+                arow = m * kBM - a.group_start[g];
+            }
+        };
+        auto load = [&](int, int kb, uint8_t *sA, uint8_t *sB, uint64_t *bar, int lane) {
+            if (lane == 0) {
+                tma_load_2d(ma, bar, sA, kb * kBK, arow);
+                tma_load_2d(&map_b, bar, sB, kb * kBK, brow);
+            }
+        };
+        tc_producer<BN>(s, total, kblocks, a.status, tile_begin, load);
+    } else if (warp == 1) {
+        if ((threadIdx.x & 31) == 0) tc_mma<BN>(s, tmem_base, total, kblocks, a.status);
+    } else {
+        uint8_t *my_stage = staging + (warp - 2) * 2 * kStageBoxBytes;
+        uint32_t sub = 0;  // store boxes this warp has issued
+        auto epi = [&](int tile, uint32_t taddr, int q, int lane) {
+            const int m = tile / a.n_tiles, n = tile - m * a.n_tiles;
+            const int g = a.tile_group[m];
+            const int grow = m * kBM + q * 32 + lane;
             const float *bias = a.bias ? a.bias + (int64_t)g * a.N + n * BN : nullptr;
-            __nv_bfloat16 *orow = static_cast<__nv_bfloat16 *>(a.out) + (int64_t)grow * a.N + n * BN;
             float ss = 0.f;
 #pragma unroll 1
-            for (int c = 0; c < BN; c += 16) {
-                uint32_t r[16];
-                tmem_ld_32x32b_x16(taddr + c, r);
-                tmem_ld_wait();
-                float v[16];
+            for (int c = 0; c < BN; c += kStoreCols) {
+                uint8_t *buf = my_stage + (sub & 1u) * kStageBoxBytes;
+                if (lane == 0) bulk_wait_group_read<1>();  // the store that last used `buf` has read it
+                __syncwarp();
+                uint8_t *row = buf + lane * 128;
+#pragma unroll 1
+                for (int h = 0; h < kStoreCols; h += 32) {
+                    float4 b4[8];
 #pragma unroll
-                for (int j = 0; j < 16; ++j) {
-                    float z = __uint_as_float(r[j]);
-                    if (bias) z += __ldg(bias + c + j);
-                    z = activate(a.act, z);
-                    v[j] = z;
-                    ss = fmaf(z, z, ss);
-                }
-                if (valid) {
-                    uint4 pk[2];
-                    uint32_t *pw = reinterpret_cast<uint32_t *>(pk);
+                    for (int j = 0; j < 8; ++j)
+                        b4[j] = bias ? __ldg(reinterpret_cast<const float4 *>(bias + c + h) + j)
+                                     : make_float4(0.f, 0.f, 0.f, 0.f);
+                    uint32_t r[32];
+                    tmem_ld_32x32b_x32(taddr + c + h, r);
+                    tmem_ld_wait();
+                    uint32_t packed[16];
 #pragma unroll
                     for (int j = 0; j < 8; ++j) {
-                        __nv_bfloat162 b2 = __floats2bfloat162_rn(v[2 * j], v[2 * j + 1]);
-                        pw[j] = *reinterpret_cast<uint32_t *>(&b2);
+                        const float z0 = activate_t<ACT>(__uint_as_float(r[4 * j]) + b4[j].x);
+                        const float z1 = activate_t<ACT>(__uint_as_float(r[4 * j + 1]) + b4[j].y);
+                        const float z2 = activate_t<ACT>(__uint_as_float(r[4 * j + 2]) + b4[j].z);
+                        const float z3 = activate_t<ACT>(__uint_as_float(r[4 * j + 3]) + b4[j].w);
+                        if (NORM) {
+                            ss = fmaf(z0, z0, ss);
+                            ss = fmaf(z1, z1, ss);
+                            ss = fmaf(z2, z2, ss);
+                            ss = fmaf(z3, z3, ss);
+                        }
+                        __nv_bfloat162 p0 = __floats2bfloat162_rn(z0, z1), p1 = __floats2bfloat162_rn(z2, z3);
+                        packed[2 * j] = *reinterpret_cast<uint32_t *>(&p0);
+                        packed[2 * j + 1] = *reinterpret_cast<uint32_t *>(&p1);
                     }
-                    uint4 *dst = reinterpret_cast<uint4 *>(orow + c);
-                    dst[0] = pk[0];
-                    dst[1] = pk[1];
+                    // Row `lane`, 16-byte chunk j at chunk j ^ (row % 8): the 128B swizzle.
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        const int chunk = (h / 8) + j;
+                        *reinterpret_cast<uint4 *>(row + ((chunk ^ (lane & 7)) << 4)) =
+                            make_uint4(packed[4 * j], packed[4 * j + 1], packed[4 * j + 2], packed[4 * j + 3]);
+                    }
                 }
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) {
+                    tma_store_2d(&map_out, buf, n * BN + c, m * kBM + q * 32);
+                    bulk_commit_group();
+                }
+                ++sub;
             }
-            if (a.norm_part && valid) a.norm_part[(int64_t)grow * a.n_tiles + n] = ss;
-            tc_fence_before_sync();
-            mbar_arrive(&tempty[acc]);
-        }
+            if (NORM && grow < a.group_start[g] + a.group_rows[g])
+                a.norm_part[(int64_t)grow * a.n_tiles + n] = ss;
+        };
+        tc_epilogue<BN>(s, tmem_base, total, a.status, epi);
+        if ((threadIdx.x & 31) == 0) bulk_wait_group<0>();  // all stores complete before exit
     }
-
-    tc_fence_before_sync();
-    __syncthreads();
-    tc_fence_after_sync();
-    if (warp == 1) {
-        __syncwarp();
-        tmem_dealloc(tmem_base, 2 * kAccCols);
-    }
+    tc_teardown<BN>(s, tmem_base);
 }
 
-template <int BN>
-cudaError_t launch_bn(const CUtensorMap &m0, const CUtensorMap &m1, const CUtensorMap &mb, const GemmArgs &a,
-                      cudaStream_t s) {
-    using C = TcCfg<BN>;
-    static bool attr_set = false;
-    if (!attr_set) {
-        cudaError_t e = cudaFuncSetAttribute(grouped_gemm_tc_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             C::SMEM);
-        if (e != cudaSuccess) return e;
-        attr_set = true;
-    }
-    grouped_gemm_tc_kernel<BN><<<a.num_sms, kThreads, C::SMEM, s>>>(m0, m1, mb, a);
+template <int BN, int ACT, bool NORM>
+cudaError_t launch_inst(const CUtensorMap &m0, const CUtensorMap &m1, const CUtensorMap &mb, const CUtensorMap &mo,
+                        const GemmArgs &a, cudaStream_t s) {
+    constexpr int smem = gemm_smem_bytes<BN>();
+    static_assert(smem <= 232448, "exceeds the 227 KB of shared memory a CTA may use");
+    cudaError_t e = cudaFuncSetAttribute(grouped_gemm_tc_kernel<BN, ACT, NORM>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    grouped_gemm_tc_kernel<BN, ACT, NORM><<<a.num_sms, kTcThreads, smem, s>>>(m0, m1, mb, mo, a);
     return cudaGetLastError();
+}
+
+// Layer 1 runs with the layer's activation and no norm; layer 2 with neither.
+template <int BN>
+cudaError_t launch_bn(const CUtensorMap &m0, const CUtensorMap &m1, const CUtensorMap &mb, const CUtensorMap &mo,
+                      const GemmArgs &a, cudaStream_t s) {
+    if (a.norm_part) return launch_inst<BN, -1, true>(m0, m1, mb, mo, a, s);
+    switch (a.act) {
+        case 0: return launch_inst<BN, 0, false>(m0, m1, mb, mo, a, s);
+        case 1: return launch_inst<BN, 1, false>(m0, m1, mb, mo, a, s);
+        case 2: return launch_inst<BN, 2, false>(m0, m1, mb, mo, a, s);
+        default: return launch_inst<BN, -1, false>(m0, m1, mb, mo, a, s);
+    }
 }
 
 }  // namespace
 
 int gemm_pick_bn(int N) {
-    for (int bn = 256; bn >= 16; bn -= 16)
-        if (N % bn == 0 && (bn == 256 || bn == 176 || bn == 128 || bn == 64 || bn == 32 || bn == 16)) return bn;
+    static const int options[] = {256, 128, 64};
+    for (int bn : options)
+        if (N % bn == 0) return bn;
     return 0;
 }
 
-cudaError_t launch_gemm_tc(const CUtensorMap &m0, const CUtensorMap &m1, const CUtensorMap &mb, const GemmArgs &a,
-                           int BN, cudaStream_t s, int *launches) {
+cudaError_t launch_gemm_tc(const CUtensorMap &m0, const CUtensorMap &m1, const CUtensorMap &mb, const CUtensorMap &mo,
+                           const GemmArgs &a, int BN, cudaStream_t s, int *launches) {
     ++*launches;
     switch (BN) {
-        case 256: return launch_bn<256>(m0, m1, mb, a, s);
-        case 176: return launch_bn<176>(m0, m1, mb, a, s);
-        case 128: return launch_bn<128>(m0, m1, mb, a, s);
-        case 64: return launch_bn<64>(m0, m1, mb, a, s);
-        case 32: return launch_bn<32>(m0, m1, mb, a, s);
-        case 16: return launch_bn<16>(m0, m1, mb, a, s);
+        case 256: return launch_bn<256>(m0, m1, mb, mo, a, s);
+        case 128: return launch_bn<128>(m0, m1, mb, mo, a, s);
+        case 64: return launch_bn<64>(m0, m1, mb, mo, a, s);
         default: return cudaErrorInvalidValue;
     }
 }

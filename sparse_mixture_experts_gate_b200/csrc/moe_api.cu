@@ -66,9 +66,9 @@ bool encode_bf16_2d(CUtensorMap *m, const void *base, uint64_t inner, uint64_t r
 struct Plan {
     int T = 0;
     int64_t C = 0;
-    int T_pad = 0, n_rt = 0, n_chunks = 0, R_routed_max = 0, R_max = 0, max_mtiles = 0;
+    int T_pad = 0, n_stat_chunks = 0, n_chunks = 0, R_routed_max = 0, R_max = 0, max_mtiles = 0;
     size_t o_ctrl, o_logits, o_idx, o_gates, o_slot, o_rowof, o_lse, o_psum, o_ccount, o_cbase, o_cpre, o_ckept,
-        o_gstart, o_grows, o_tgroup, o_rowassign, o_xp, o_h, o_o, o_norm, o_credit, o_pm, o_f;
+        o_gstart, o_grows, o_tgroup, o_rowassign, o_wsplit, o_xp, o_h, o_o, o_norm, o_credit, o_pm, o_f;
     size_t total = 0;
 };
 
@@ -92,8 +92,7 @@ struct moe_layer {
     bool has_forward = false;
     Plan plan;
     char *ws = nullptr;
-    int32_t *idx = nullptr, *count_pre = nullptr;
-    float *gates = nullptr;
+    float *logits = nullptr;
     int fwd_launches = 0, stats_launches = 0;
     bool timing = false;
     cudaEvent_t ev[MOE_TIMING_EVENTS];
@@ -119,8 +118,7 @@ Plan make_plan(const moe_layer &L, int T) {
     p.T_pad = (int)round_up(T, kBM);
     p.R_max = p.R_routed_max + S * p.T_pad;
     p.max_mtiles = p.R_max / kBM;
-    const int rt = router_tile_tokens(E, T);
-    p.n_rt = (T + rt - 1) / rt;
+    p.n_stat_chunks = (T + kStatsChunk - 1) / kStatsChunk;
     p.n_chunks = (T + 255) / 256;
     const size_t es = c.dtype == MOE_DTYPE_BF16 ? 2 : 4;
     size_t off = 0;
@@ -136,7 +134,7 @@ Plan make_plan(const moe_layer &L, int T) {
     p.o_slot = take((size_t)T * k * 4);
     p.o_rowof = take((size_t)T * k * 4);
     p.o_lse = take((size_t)T * 4);
-    p.o_psum = take((size_t)p.n_rt * E * 4);
+    p.o_psum = take((size_t)p.n_stat_chunks * E * 4);
     p.o_ccount = take((size_t)p.n_chunks * E * 4);
     p.o_cbase = take((size_t)p.n_chunks * E * 4);
     p.o_cpre = take((size_t)E * 4);
@@ -149,7 +147,8 @@ Plan make_plan(const moe_layer &L, int T) {
     p.o_f = take((size_t)E * 4);
     p.o_credit = take((size_t)T * k * 4);
     p.o_norm = take((size_t)p.R_max * L.ntiles2 * 4);
-    p.o_xp = take((size_t)p.R_routed_max * c.input_dim * es);
+    p.o_wsplit = take(c.dtype == MOE_DTYPE_BF16 ? (size_t)router_tc_epad(E) * 3 * c.input_dim * 2 : 0);
+    p.o_xp = take(c.dtype == MOE_DTYPE_BF16 ? (size_t)p.R_routed_max * c.input_dim * es : 0);
     p.o_h = take((size_t)p.R_max * c.expert_dim * es);
     p.o_o = take((size_t)p.R_max * c.output_dim * es);
     p.total = off;
@@ -186,10 +185,8 @@ int validate_config(const moe_config_t *c, const moe_weights_t *w) {
     if (c->use_selection_bias && !w->sel_bias)
         return fail(MOE_ERR_INVALID_ARG, "use_selection_bias is set but weights->sel_bias is NULL");
     if (c->dtype == MOE_DTYPE_BF16) {
-        if (c->input_dim % kBK || c->expert_dim % kBK)
-            return fail(MOE_ERR_UNSUPPORTED, "bf16 layers need input_dim and expert_dim multiples of %d", kBK);
-        if (gemm_pick_bn(c->expert_dim) == 0 || gemm_pick_bn(c->output_dim) == 0 || c->output_dim % 16)
-            return fail(MOE_ERR_UNSUPPORTED, "bf16 layers need expert_dim and output_dim multiples of 16");
+        if (c->input_dim % 64 || c->expert_dim % 64 || c->output_dim % 64)
+            return fail(MOE_ERR_UNSUPPORTED, "bf16 layers need input_dim, expert_dim and output_dim multiples of 64");
     } else {
         if (c->input_dim % 4 || c->expert_dim % 4 || c->output_dim % 4)
             return fail(MOE_ERR_UNSUPPORTED, "fp32 layers need input_dim, expert_dim, output_dim multiples of 4");
@@ -322,14 +319,13 @@ int moe_forward(moe_layer_t *L, const void *x, int32_t T, const float *logit_noi
     int32_t *idx = rt && rt->topk_idx ? rt->topk_idx : reinterpret_cast<int32_t *>(ws + p.o_idx);
     float *gates = rt && rt->gates ? rt->gates : reinterpret_cast<float *>(ws + p.o_gates);
     int32_t *slot = rt && rt->slot ? rt->slot : reinterpret_cast<int32_t *>(ws + p.o_slot);
-    L->idx = idx;
-    L->gates = gates;
-    L->count_pre = reinterpret_cast<int32_t *>(ws + p.o_cpre);
+    L->logits = logits;
     int *nl = &L->fwd_launches;
+    uint32_t *status = reinterpret_cast<uint32_t *>(ctrl + kCtrlStatus);
 
     RouterArgs ra;
     ra.x = x;
-    ra.x_bf16 = c.dtype == MOE_DTYPE_BF16;
+    ra.x_bf16 = 0;
     ra.w_gate = L->w.w_gate;
     ra.b_gate = L->w.b_gate;
     ra.noise = c.top_k_method == MOE_TOPK_NOISY ? logit_noise : nullptr;
@@ -342,8 +338,27 @@ int moe_forward(moe_layer_t *L, const void *x, int32_t T, const float *logit_noi
     ra.idx = idx;
     ra.gates = gates;
     ra.lse = reinterpret_cast<float *>(ws + p.o_lse);
-    ra.psum_part = reinterpret_cast<float *>(ws + p.o_psum);
-    MOE_LAUNCH(launch_router(ra, s, nl));
+    if (L->tc) {
+        RouterTcArgs rt_args;
+        rt_args.w_gate = L->w.w_gate;
+        rt_args.b_gate = L->w.b_gate;
+        rt_args.T = T;
+        rt_args.d = c.input_dim;
+        rt_args.E = E;
+        rt_args.E_pad = router_tc_epad(E);
+        rt_args.logits = logits;
+        rt_args.status = status;
+        rt_args.num_sms = L->num_sms;
+        __nv_bfloat16 *w_split = reinterpret_cast<__nv_bfloat16 *>(ws + p.o_wsplit);
+        CUtensorMap m_xr, m_ws;
+        if (!encode_bf16_2d(&m_xr, x, c.input_dim, T, kBM) ||
+            !encode_bf16_2d(&m_ws, w_split, 3ull * c.input_dim, rt_args.E_pad, router_tc_bn(E)))
+            return fail(MOE_ERR_CUDA, "cuTensorMapEncodeTiled failed for the router operands");
+        MOE_LAUNCH(launch_router_logits_tc(m_xr, m_ws, rt_args, w_split, s, nl));
+        MOE_LAUNCH(launch_route_from_logits(ra, L->num_sms, s, nl));
+    } else {
+        MOE_LAUNCH(launch_router(ra, s, nl));
+    }
     MOE_MARK(L, 1, s);
 
     DispatchArgs da;
@@ -371,17 +386,17 @@ int moe_forward(moe_layer_t *L, const void *x, int32_t T, const float *logit_noi
     MOE_LAUNCH(launch_dispatch(da, s, nl));
     MOE_MARK(L, 2, s);
 
-    const size_t es = c.dtype == MOE_DTYPE_BF16 ? 2 : 4;
-    GatherArgs ga;
-    ga.x = x;
-    ga.xp = ws + p.o_xp;
-    ga.row_assign = da.row_assign;
-    ga.ctrl = ctrl;
-    ga.k = k;
-    ga.row_bytes = (int)(c.input_dim * es);
-    ga.max_rows = p.R_routed_max;
-    MOE_LAUNCH(launch_gather(ga, s, nl));
-    MOE_MARK(L, 3, s);
+    if (L->tc) {
+        GatherArgs ga;
+        ga.x = x;
+        ga.xp = ws + p.o_xp;
+        ga.row_assign = da.row_assign;
+        ga.ctrl = ctrl;
+        ga.k = k;
+        ga.row_bytes = c.input_dim * 2;
+        ga.max_rows = p.R_routed_max;
+        MOE_LAUNCH(launch_gather(ga, s, nl));
+    }
 
     GemmArgs g1;
     g1.tile_group = da.tile_group;
@@ -394,49 +409,54 @@ int moe_forward(moe_layer_t *L, const void *x, int32_t T, const float *logit_noi
     g1.n_tiles = L->ntiles1;
     g1.E = E;
     g1.use_a1 = 1;
+    g1.row_assign = da.row_assign;
+    g1.k = k;
+    g1.T = T;
     g1.bias = L->w.b1;
     g1.out = ws + p.o_h;
     g1.norm_part = nullptr;
     g1.act = c.activation;
-    g1.status = reinterpret_cast<uint32_t *>(ctrl + kCtrlStatus);
+    g1.status = status;
     g1.num_sms = L->num_sms;
     GemmArgs g2 = g1;
+    g2.use_a1 = 0;
     g2.N = c.output_dim;
     g2.K = c.expert_dim;
     g2.n_tiles = L->ntiles2;
-    g2.use_a1 = 0;
     g2.bias = L->w.b2;
     g2.out = ws + p.o_o;
     g2.norm_part = reinterpret_cast<float *>(ws + p.o_norm);
     g2.act = -1;
 
     if (L->tc) {
-        CUtensorMap m_xp, m_x, m_h;
+        CUtensorMap m_xp, m_x, m_h, m_hs, m_os;
         if (!encode_bf16_2d(&m_xp, ws + p.o_xp, c.input_dim, p.R_routed_max, kBM) ||
             !encode_bf16_2d(&m_x, x, c.input_dim, T, kBM) ||
-            !encode_bf16_2d(&m_h, ws + p.o_h, c.expert_dim, p.R_max, kBM))
+            !encode_bf16_2d(&m_h, ws + p.o_h, c.expert_dim, p.R_max, kBM) ||
+            !encode_bf16_2d(&m_hs, ws + p.o_h, c.expert_dim, p.R_max, 32) ||
+            !encode_bf16_2d(&m_os, ws + p.o_o, c.output_dim, p.R_max, 32))
             return fail(MOE_ERR_CUDA, "cuTensorMapEncodeTiled failed for the activations");
-        MOE_LAUNCH(launch_gemm_tc(m_xp, m_x, L->map_w1, g1, L->bn1, s, nl));
+        MOE_LAUNCH(launch_gemm_tc(m_xp, m_x, L->map_w1, m_hs, g1, L->bn1, s, nl));
+        MOE_MARK(L, 3, s);
+        MOE_LAUNCH(launch_gemm_tc(m_h, m_h, L->map_w2, m_os, g2, L->bn2, s, nl));
         MOE_MARK(L, 4, s);
-        MOE_LAUNCH(launch_gemm_tc(m_h, m_h, L->map_w2, g2, L->bn2, s, nl));
-        MOE_MARK(L, 5, s);
     } else {
         GemmSimtArgs s1;
         s1.g = g1;
-        s1.a0 = reinterpret_cast<const float *>(ws + p.o_xp);
-        s1.a1 = static_cast<const float *>(x);
+        s1.a = static_cast<const float *>(x);
+        s1.gather = 1;
         s1.w = static_cast<const float *>(L->w.w1);
         s1.max_rows = p.R_max;
         MOE_LAUNCH(launch_gemm_simt(s1, s, nl));
-        MOE_MARK(L, 4, s);
+        MOE_MARK(L, 3, s);
         GemmSimtArgs s2;
         s2.g = g2;
-        s2.a0 = reinterpret_cast<const float *>(ws + p.o_h);
-        s2.a1 = nullptr;
+        s2.a = reinterpret_cast<const float *>(ws + p.o_h);
+        s2.gather = 0;
         s2.w = static_cast<const float *>(L->w.w2);
         s2.max_rows = p.R_max;
         MOE_LAUNCH(launch_gemm_simt(s2, s, nl));
-        MOE_MARK(L, 5, s);
+        MOE_MARK(L, 4, s);
     }
 
     CombineArgs ca;
@@ -455,7 +475,7 @@ int moe_forward(moe_layer_t *L, const void *x, int32_t T, const float *logit_noi
     ca.y = y;
     ca.credit = reinterpret_cast<float *>(ws + p.o_credit);
     MOE_LAUNCH(launch_combine(ca, s, nl));
-    MOE_MARK(L, 6, s);
+    MOE_MARK(L, 5, s);
     return MOE_OK;
 }
 
@@ -471,8 +491,9 @@ int moe_aux_stats(moe_layer_t *L, const float *token_loss, const moe_stats_t *ou
     if (p.T == 0) return MOE_OK;
     char *ws = L->ws;
     StatsArgs sa;
-    sa.psum_part = reinterpret_cast<const float *>(ws + p.o_psum);
-    sa.n_router_tiles = p.n_rt;
+    sa.logits = L->logits;
+    sa.psum_part = reinterpret_cast<float *>(ws + p.o_psum);
+    sa.n_chunks = p.n_stat_chunks;
     sa.lse = reinterpret_cast<const float *>(ws + p.o_lse);
     sa.count_pre = reinterpret_cast<const int32_t *>(ws + p.o_cpre);
     sa.group_start = reinterpret_cast<const int32_t *>(ws + p.o_gstart);
@@ -498,7 +519,7 @@ int moe_aux_stats(moe_layer_t *L, const float *token_loss, const moe_stats_t *ou
     if (out->credit)
         MOE_LAUNCH(cudaMemcpyAsync(out->credit, ws + p.o_credit, (size_t)p.T * c.num_active * 4,
                                    cudaMemcpyDeviceToDevice, s));
-    MOE_MARK(L, 7, s);
+    MOE_MARK(L, 6, s);
     return MOE_OK;
 }
 

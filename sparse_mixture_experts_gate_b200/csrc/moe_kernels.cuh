@@ -7,8 +7,8 @@
 
 namespace moe {
 
-// Router: logits h = W_g x + b, P = softmax(h), log-partition, selection key,
-// top-k, renormalised gates, and per-CTA partial sums of P over its tokens.
+// Router (fp32 CUDA cores, fp32 layers): logits h = W_g x + b, max,
+// log-partition, selection key, top-k, renormalised gates.
 struct RouterArgs {
     const void *x;          // [T][d] bf16 or fp32
     int x_bf16;
@@ -21,10 +21,25 @@ struct RouterArgs {
     int32_t *idx;           // [T][k]
     float *gates;           // [T][k]
     float *lse;             // [T]
-    float *psum_part;       // [n_router_tiles][E]
 };
-int router_tile_tokens(int E, int T);
 cudaError_t launch_router(const RouterArgs &a, cudaStream_t s, int *launches);
+// Max, log-partition, keys, top-k and gates from logits already in a.logits.
+cudaError_t launch_route_from_logits(const RouterArgs &a, int num_sms, cudaStream_t s, int *launches);
+
+// Router logits on the tensor cores (bf16 layers): logits [T][E], bias included.
+struct RouterTcArgs {
+    const float *w_gate;    // [E][d] fp32, split into bf16 planes every forward
+    const float *b_gate;    // [E] or null
+    int T, d, E, E_pad;
+    float *logits;          // [T][E]
+    uint32_t *status;
+    int num_sms;
+};
+int router_tc_epad(int E);  // padded expert count (rows of the split planes)
+int router_tc_bn(int E);    // N tile of the logits GEMM (<= 128)
+// map_x: x [T][d] bf16, box 64 x 128; map_w: w_split [E_pad][3d] bf16, box 64 x router_tc_bn(E).
+cudaError_t launch_router_logits_tc(const CUtensorMap &map_x, const CUtensorMap &map_w, const RouterTcArgs &a,
+                                    __nv_bfloat16 *w_split, cudaStream_t s, int *launches);
 
 // Dispatch: histogram, scan, stable capacity-capped ranks, row map.
 struct DispatchArgs {
@@ -74,8 +89,10 @@ struct GemmArgs {
     int max_mtiles;              // host bound on the M tiles (clamps the device count)
     int N, K;                    // output row length, reduction length
     int n_tiles;                 // N / BN
-    int E;                       // groups >= E read A through the second map (if use_a1)
+    int E;                       // groups >= E are shared experts (A through the second map)
     int use_a1;
+    const int32_t *row_assign;   // [rows] t*k + r of each routed row (-1 padding)
+    int k, T;
     const float *bias;           // [G][N] or null
     void *out;                   // [rows][N]
     float *norm_part;            // [rows][n_tiles] or null: per-tile sum of out^2 (fp32, pre-rounding)
@@ -83,15 +100,18 @@ struct GemmArgs {
     uint32_t *status;            // device status word
     int num_sms;
 };
-// bf16 tcgen05 path; BN chosen by the host (multiple of 16, <= 256, divides N).
+// bf16 tcgen05 path; BN (256, 128 or 64) is the largest that divides N.
+// A rows come from map_a0 (row space: the gathered rows or H, box 64 x 128); with
+// use_a1, shared-expert groups read x itself through map_a1 (box 64 x 128).
+// map_out: the output [rows][N] bf16, box 64 x 32, 128B swizzle.
 int gemm_pick_bn(int N);
 cudaError_t launch_gemm_tc(const CUtensorMap &map_a0, const CUtensorMap &map_a1, const CUtensorMap &map_b,
-                           const GemmArgs &a, int BN, cudaStream_t s, int *launches);
-// fp32 CUDA-core path (A operands as plain pointers).
+                           const CUtensorMap &map_out, const GemmArgs &a, int BN, cudaStream_t s, int *launches);
+// fp32 CUDA-core path (A operand as a plain pointer).
 struct GemmSimtArgs {
     GemmArgs g;
-    const float *a0;   // [rows][K] (routed rows, or all rows when !use_a1)
-    const float *a1;   // [T][K] (shared-expert rows when use_a1)
+    const float *a;    // gather: x [T][K]; otherwise [rows][K]
+    int gather;
     const float *w;    // [G][N][K]
     int max_rows;      // rows the launch covers
 };
@@ -115,8 +135,9 @@ cudaError_t launch_combine(const CombineArgs &a, cudaStream_t s, int *launches);
 
 // Balancing and credit statistics.
 struct StatsArgs {
-    const float *psum_part;   // [n_router_tiles][E]
-    int n_router_tiles;
+    const float *logits;      // [T][E]
+    float *psum_part;         // [n_chunks][E] scratch: per-chunk sums of P
+    int n_chunks;             // ceil(T / kStatsChunk)
     const float *lse;         // [T]
     const int32_t *count_pre; // [E]
     const int32_t *group_start;
@@ -132,6 +153,7 @@ struct StatsArgs {
     float *f, *p_mean, *l_aux, *l_z, *expert_loss;  // outputs (nullable)
     int32_t *n_dropped;
 };
+constexpr int kStatsChunk = 128;
 cudaError_t launch_stats(const StatsArgs &a, cudaStream_t s, int *launches);
 
 // Sets the calling thread's last-error message; returns `code`.

@@ -7,13 +7,14 @@
 // top-k adds noise to the logits before selection. Appendix C, "Balancing": the
 // per-expert selection bias b_i and the log-partition that the z-loss squares.
 //
-// One CTA computes the logits of kTM tokens for all E <= 256 experts on fp32
-// CUDA cores, K-tiled through shared memory. Warp w owns tokens w*RT .. w*RT+RT-1
-// outright and lane l holds experts l, l+32, ..., so softmax, selection and
-// gates are warp-shuffle reductions in registers with no transpose. Selection
-// keys are formed with one fp32 round-to-nearest add; ties in the key go to the
-// lower expert index. Each CTA also writes the sum over its tokens of P (fixed
-// order), which the statistics kernel reduces across CTAs.
+// route_warp() is the per-token step shared by both kernels below: one warp owns
+// one token, lane l holds experts l, l+32, ..., and max, log-partition, top-k
+// and gates are warp-shuffle reductions. Selection keys are formed with one
+// fp32 round-to-nearest add; equal keys go to the lower expert index.
+//   router_simt_kernel      - fp32 layers: logits on fp32 CUDA cores (K tiled
+//                             through shared memory), then route_warp;
+//   route_from_logits_kernel - bf16 layers: route_warp over the logits the
+//                             tensor-core kernel (router_tc.cu) wrote.
 #include "moe_common.cuh"
 #include "moe_kernels.cuh"
 
@@ -24,13 +25,95 @@ constexpr int kThreads = 256;
 constexpr int kWarps = kThreads / 32;
 constexpr int kKC = 32;  // K chunk staged in shared memory
 
+// h[q] = clean logit of expert lane + 32 q (-inf for e >= E). Writes lse[t],
+// idx[t][0..k), gates[t][0..k).
+template <int RE>
+__device__ __forceinline__ void route_warp(const float (&h)[RE], int t, int lane, const RouterArgs &a) {
+    float key[RE];
+    float m = -INFINITY;
+#pragma unroll
+    for (int q = 0; q < RE; ++q) {
+        const int e = lane + 32 * q;
+        key[q] = -INFINITY;
+        if (e < a.E) {
+            float kv = h[q];
+            if (a.noise)
+                kv = __fadd_rn(h[q], a.noise[(int64_t)t * a.E + e]);
+            else if (a.sel_bias)
+                kv = __fadd_rn(h[q], a.sel_bias[e]);
+            key[q] = kv;
+            m = fmaxf(m, h[q]);
+        }
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
+    float ex[RE], z = 0.f;
+#pragma unroll
+    for (int q = 0; q < RE; ++q) {
+        ex[q] = (lane + 32 * q < a.E) ? expf(h[q] - m) : 0.f;
+        z += ex[q];
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) z += __shfl_xor_sync(0xffffffffu, z, off);
+    if (lane == 0) a.lse[t] = m + logf(z);
+
+    // Top-k by (key desc, expert index asc); the winner's clean exp(h - m)
+    // feeds its gate.
+    uint32_t taken = 0u;
+    float gsel_sum = 0.f, my_gate_num = 0.f;
+    int my_idx = -1;
+    for (int r = 0; r < a.k; ++r) {
+        float bk = -INFINITY;
+        int be = 0x7fffffff;
+#pragma unroll
+        for (int q = 0; q < RE; ++q) {
+            const int e = lane + 32 * q;
+            if (e < a.E && !(taken & (1u << q))) {
+                if (key[q] > bk || (key[q] == bk && e < be)) {
+                    bk = key[q];
+                    be = e;
+                }
+            }
+        }
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) {
+            const float ok = __shfl_xor_sync(0xffffffffu, bk, off);
+            const int oe = __shfl_xor_sync(0xffffffffu, be, off);
+            if (ok > bk || (ok == bk && oe < be)) {
+                bk = ok;
+                be = oe;
+            }
+        }
+        // The owner lane of expert `be` marks it taken and broadcasts exp(h - m).
+        const int owner = be & 31, oq = be >> 5;
+        float num = 0.f;
+        if (lane == owner) {
+#pragma unroll
+            for (int q = 0; q < RE; ++q)
+                if (q == oq) {
+                    taken |= (1u << q);
+                    num = ex[q];
+                }
+        }
+        num = __shfl_sync(0xffffffffu, num, owner);
+        gsel_sum += num;
+        if (lane == r) {
+            my_gate_num = num;
+            my_idx = be;
+        }
+    }
+    if (lane < a.k) {
+        a.idx[(int64_t)t * a.k + lane] = my_idx;
+        a.gates[(int64_t)t * a.k + lane] = my_gate_num / gsel_sum;
+    }
+}
+
 template <typename XT, int RE, int RT>
 __global__ void __launch_bounds__(kThreads) router_simt_kernel(RouterArgs a) {
     constexpr int TM = kWarps * RT;   // tokens per CTA
     constexpr int EP = 32 * RE;       // padded expert count
     __shared__ float xs[kKC][TM + 1];
     __shared__ float ws[kKC][EP + 1];
-    __shared__ float psum_w[kWarps][EP];
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int t_base = blockIdx.x * TM;
@@ -71,109 +154,38 @@ __global__ void __launch_bounds__(kThreads) router_simt_kernel(RouterArgs a) {
         __syncthreads();
     }
 
-    float pacc[RE];
-#pragma unroll
-    for (int q = 0; q < RE; ++q) pacc[q] = 0.f;
-
 #pragma unroll
     for (int i = 0; i < RT; ++i) {
         const int t = t_base + warp * RT + i;
         if (t >= a.T) break;  // warp-uniform
-        float h[RE], key[RE];
-        float m = -INFINITY;
+        float h[RE];
 #pragma unroll
         for (int q = 0; q < RE; ++q) {
             const int e = lane + 32 * q;
+            h[q] = -INFINITY;
             if (e < a.E) {
                 h[q] = acc[i][q] + (a.b_gate ? a.b_gate[e] : 0.f);
                 a.logits[(int64_t)t * a.E + e] = h[q];
-                float kv = h[q];
-                if (a.noise)
-                    kv = __fadd_rn(h[q], a.noise[(int64_t)t * a.E + e]);
-                else if (a.sel_bias)
-                    kv = __fadd_rn(h[q], a.sel_bias[e]);
-                key[q] = kv;
-                m = fmaxf(m, h[q]);
-            } else {
-                h[q] = -INFINITY;
-                key[q] = -INFINITY;
             }
         }
-#pragma unroll
-        for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
-        float ex[RE], z = 0.f;
+        route_warp<RE>(h, t, lane, a);
+    }
+}
+
+// One warp per token over logits already in memory (bias included).
+template <int RE>
+__global__ void __launch_bounds__(kThreads) route_from_logits_kernel(RouterArgs a) {
+    const int lane = threadIdx.x & 31;
+    const int warp = (blockIdx.x * kThreads + threadIdx.x) >> 5;
+    const int nwarps = (gridDim.x * kThreads) >> 5;
+    for (int t = warp; t < a.T; t += nwarps) {
+        float h[RE];
 #pragma unroll
         for (int q = 0; q < RE; ++q) {
-            ex[q] = (lane + 32 * q < a.E) ? expf(h[q] - m) : 0.f;
-            z += ex[q];
+            const int e = lane + 32 * q;
+            h[q] = e < a.E ? a.logits[(int64_t)t * a.E + e] : -INFINITY;
         }
-#pragma unroll
-        for (int off = 16; off > 0; off >>= 1) z += __shfl_xor_sync(0xffffffffu, z, off);
-        const float inv_z = 1.f / z;
-#pragma unroll
-        for (int q = 0; q < RE; ++q) pacc[q] += ex[q] * inv_z;
-        if (lane == 0) a.lse[t] = m + logf(z);
-
-        // Top-k by (key desc, expert index asc); the winner's clean exp(h - m)
-        // feeds the gate.
-        uint32_t taken = 0u;
-        float gsel_sum = 0.f, my_gate_num = 0.f;
-        int my_idx = -1;
-        for (int r = 0; r < a.k; ++r) {
-            float bk = -INFINITY;
-            int be = 0x7fffffff;
-#pragma unroll
-            for (int q = 0; q < RE; ++q) {
-                const int e = lane + 32 * q;
-                if (e < a.E && !(taken & (1u << q))) {
-                    if (key[q] > bk || (key[q] == bk && e < be)) {
-                        bk = key[q];
-                        be = e;
-                    }
-                }
-            }
-#pragma unroll
-            for (int off = 16; off > 0; off >>= 1) {
-                const float ok = __shfl_xor_sync(0xffffffffu, bk, off);
-                const int oe = __shfl_xor_sync(0xffffffffu, be, off);
-                if (ok > bk || (ok == bk && oe < be)) {
-                    bk = ok;
-                    be = oe;
-                }
-            }
-            // Owner lane of expert `be` marks it taken and broadcasts exp(h - m).
-            const int owner = be & 31, oq = be >> 5;
-            float num = 0.f;
-            if (lane == owner) {
-#pragma unroll
-                for (int q = 0; q < RE; ++q)
-                    if (q == oq) {
-                        taken |= (1u << q);
-                        num = ex[q];
-                    }
-            }
-            num = __shfl_sync(0xffffffffu, num, owner);
-            gsel_sum += num;
-            if (lane == r) {
-                my_gate_num = num;
-                my_idx = be;
-            }
-        }
-        if (lane < a.k) {
-            a.idx[(int64_t)t * a.k + lane] = my_idx;
-            a.gates[(int64_t)t * a.k + lane] = my_gate_num / gsel_sum;
-        }
-    }
-
-    // Per-CTA column sums of P over this CTA's tokens, warps in fixed order.
-#pragma unroll
-    for (int q = 0; q < RE; ++q) psum_w[warp][lane + 32 * q] = pacc[q];
-    __syncthreads();
-    for (int e = tid; e < a.E; e += kThreads) {
-        float s = 0.f;
-#pragma unroll
-        for (int w = 0; w < kWarps; ++w) s += psum_w[w][e];
-        a.psum_part[(int64_t)blockIdx.x * a.E + e] = s;
+        route_warp<RE>(h, t, lane, a);
     }
 }
 
@@ -197,21 +209,32 @@ cudaError_t launch_x(const RouterArgs &a, cudaStream_t s, int rt) {
     return launch_re<XT, 8>(a, s, rt);
 }
 
+template <int RE>
+cudaError_t launch_route(const RouterArgs &a, cudaStream_t s, int num_sms) {
+    int blocks = (a.T + kWarps - 1) / kWarps;
+    if (blocks > num_sms * 8) blocks = num_sms * 8;
+    route_from_logits_kernel<RE><<<blocks, kThreads, 0, s>>>(a);
+    return cudaGetLastError();
+}
+
 int router_rt(int T) { return T >= 4096 ? 4 : 1; }
 
 }  // namespace
-
-// Tokens per router CTA (the granularity of the P partial sums).
-int router_tile_tokens(int E, int T) {
-    (void)E;
-    return kWarps * router_rt(T);
-}
 
 cudaError_t launch_router(const RouterArgs &a, cudaStream_t s, int *launches) {
     if (a.T <= 0) return cudaSuccess;
     ++*launches;
     const int rt = router_rt(a.T);
     return a.x_bf16 ? launch_x<__nv_bfloat16>(a, s, rt) : launch_x<float>(a, s, rt);
+}
+
+cudaError_t launch_route_from_logits(const RouterArgs &a, int num_sms, cudaStream_t s, int *launches) {
+    if (a.T <= 0) return cudaSuccess;
+    ++*launches;
+    if (a.E <= 32) return launch_route<1>(a, s, num_sms);
+    if (a.E <= 64) return launch_route<2>(a, s, num_sms);
+    if (a.E <= 128) return launch_route<4>(a, s, num_sms);
+    return launch_route<8>(a, s, num_sms);
 }
 
 }  // namespace moe

@@ -1,0 +1,226 @@
+// router_tc.cu - router logits on the sm_100a tensor cores, at fp32 accuracy.
+//
+// "Appendix C - Acronyms & Symbols", table "Core MoE symbols": router logits
+// h = W_g x, one score per expert; "Code Walkthrough - SER", gating / routing
+// path: the linear router carries a bias. The routing decisions that follow
+// (softmax, selection key, top-k, gates) are integer decisions taken on these
+// fp32 logits, so the logits must be as accurate as an fp32 dot product.
+//
+// Two things make a bf16 tensor-core GEMM fp32-accurate here:
+//  * operands: every forward splits the fp32 router matrix into three bf16
+//    planes, W = hi + mid + lo (each the bf16 rounding of what the earlier
+//    planes leave; the sum matches W to ~2^-27 relative), and x is exactly
+//    bf16, so h = sum_p x . W_p is one GEMM with K = 3d whose products are
+//    exact: A is x read three times (the K coordinate wraps), B = [hi|mid|lo];
+//  * accumulation: the tensor core's fp32 accumulator does not round to
+//    nearest, and its error grows with the number of MMA steps and with the
+//    accumulator's magnitude. So the MMA starts a fresh partial every kDrain K
+//    blocks (kDrain * 4 MMA steps) and the epilogue warps add each partial into
+//    a running fp32 sum kept in TMEM, with ordinary round-to-nearest adds.
+// TMEM: two partial buffers (128 columns each, double-buffered so the MMA runs
+// ahead) and the running sum (128 columns); the N tile is <= 128 experts.
+// Output: logits [T][E] (bias included). Softmax, keys, top-k and gates are
+// taken from them by the routing kernel in router.cu.
+#include "moe_common.cuh"
+#include "moe_kernels.cuh"
+#include "tc_pipeline.cuh"
+
+namespace moe {
+namespace {
+
+constexpr int kDrain = 2;        // K blocks per partial accumulator
+constexpr int kSumCol = 256;     // TMEM column of the running sum
+
+// W_g [E][d] fp32 -> [E_pad][3d] bf16 planes (rows >= E are zero).
+__global__ void __launch_bounds__(256) router_split_kernel(const float *__restrict__ w, int E, int E_pad, int d,
+                                                           __nv_bfloat16 *__restrict__ out) {
+    const int64_t n = (int64_t)E_pad * d;
+    for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x) {
+        const int e = (int)(i / d), j = (int)(i - (int64_t)e * d);
+        const float v = e < E ? w[i] : 0.f;
+        const __nv_bfloat16 hi = __float2bfloat16_rn(v);
+        const float r1 = v - __bfloat162float(hi);  // exact: hi is v rounded to 8 mantissa bits
+        const __nv_bfloat16 mid = __float2bfloat16_rn(r1);
+        const float r2 = r1 - __bfloat162float(mid);  // exact for the same reason
+        const __nv_bfloat16 lo = __float2bfloat16_rn(r2);
+        __nv_bfloat16 *row = out + (int64_t)e * 3 * d;
+        row[j] = hi;
+        row[d + j] = mid;
+        row[2 * d + j] = lo;
+    }
+}
+
+template <int BN>
+__global__ void __launch_bounds__(kTcThreads, 1)
+    router_logits_tc_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ CUtensorMap map_w,
+                            const RouterTcArgs a) {
+    static_assert(BN <= 128, "two partial buffers and the running sum must fit in 512 TMEM columns");
+    using L = TcLayout<BN>;
+    extern __shared__ uint8_t smem_raw[];
+    const TcShared<BN> s = tc_carve<BN>(smem_raw);
+    if (threadIdx.x == 0) {
+        tma_prefetch_desc(&map_x);
+        tma_prefetch_desc(&map_w);
+    }
+    const uint32_t tmem_base = tc_setup<BN>(s);
+    const int n_tiles = a.E_pad / BN;
+    const int total = ((a.T + kBM - 1) / kBM) * n_tiles;
+    const int dblocks = a.d / kBK;
+    const int kblocks = 3 * dblocks;
+    const int groups = (kblocks + kDrain - 1) / kDrain;
+    const int warp = threadIdx.x >> 5;
+
+    if (warp == 0) {
+        int arow = 0, brow = 0;
+        auto tile_begin = [&](int tile, int) {
+            const int m = tile / n_tiles, n = tile - m * n_tiles;
+            arow = m * kBM;
+            brow = n * BN;
+        };
+        auto load = [&](int, int kb, uint8_t *sA, uint8_t *sB, uint64_t *bar, int lane) {
+            if (lane == 0) {
+                tma_load_2d(&map_x, bar, sA, (kb % dblocks) * kBK, arow);
+                tma_load_2d(&map_w, bar, sB, kb * kBK, brow);
+            }
+        };
+        tc_producer<BN>(s, total, kblocks, a.status, tile_begin, load);
+    } else if (warp == 1) {
+        if ((threadIdx.x & 31) == 0) {
+            constexpr uint32_t idesc = idesc_bf16_f32(kBM, BN);
+            uint32_t it = 0, gcount = 0;
+            bool ok = true;
+            for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
+                for (int g = 0; g < groups && ok; ++g, ++gcount) {
+                    const uint32_t buf = gcount & 1u, use = gcount >> 1;
+                    if (!mbar_wait(&s.tempty[buf], (use & 1u) ^ 1u, a.status)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after_sync();
+                    const uint32_t d_tmem = tmem_base + buf * kTcAccCols / 2;
+                    const int kb0 = g * kDrain, kb1 = min(kb0 + kDrain, kblocks);
+                    for (int kb = kb0; kb < kb1; ++kb, ++it) {
+                        const int st = it % L::NS;
+                        const uint32_t ph = (it / L::NS) & 1u;
+                        if (!mbar_wait(&s.full[st], ph, a.status)) {
+                            ok = false;
+                            break;
+                        }
+                        tc_fence_after_sync();
+                        const uint64_t ad = sw128_kmajor_desc(smem_u32(s.sA + st * L::A_BYTES));
+                        const uint64_t bd = sw128_kmajor_desc(smem_u32(s.sB + st * L::B_BYTES));
+#pragma unroll
+                        for (int kk = 0; kk < kBK / 16; ++kk)
+                            tc_mma_bf16(d_tmem, ad + 2u * kk, bd + 2u * kk, idesc, (kb != kb0 || kk != 0) ? 1u : 0u);
+                        tc_commit(&s.empty[st]);
+                    }
+                    if (ok) tc_commit(&s.tfull[buf]);
+                }
+            }
+            tc_commit(s.mma_done);
+            mbar_wait_drain(s.mma_done, 0u);
+        }
+    } else {
+        const int q = warp & 3, lane = threadIdx.x & 31;
+        uint32_t gcount = 0;
+        bool ok = true;
+        for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
+            const int m = tile / n_tiles, n = tile - m * n_tiles;
+            const int t = m * kBM + q * 32 + lane;
+            const bool valid = t < a.T;
+            const uint32_t lane_off = static_cast<uint32_t>(q * 32) << 16;
+            const uint32_t sum_addr = tmem_base + lane_off + kSumCol;
+            for (int g = 0; g < groups; ++g, ++gcount) {
+                const uint32_t buf = gcount & 1u, use = gcount >> 1;
+                const bool got = mbar_wait(&s.tfull[buf], use & 1u, a.status);
+                if (!__all_sync(0xffffffffu, got)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after_sync();
+                const uint32_t acc_addr = tmem_base + lane_off + buf * kTcAccCols / 2;
+                const bool last = g == groups - 1;
+#pragma unroll 1
+                for (int c = 0; c < BN; c += 16) {
+                    uint32_t r[16], sm[16];
+                    tmem_ld_32x32b_x16(acc_addr + c, r);
+                    if (g > 0) tmem_ld_32x32b_x16(sum_addr + c, sm);
+                    tmem_ld_wait();
+                    if (g > 0) {
+#pragma unroll
+                        for (int j = 0; j < 16; ++j)
+                            r[j] = __float_as_uint(__fadd_rn(__uint_as_float(sm[j]), __uint_as_float(r[j])));
+                    }
+                    if (!last) {
+                        tmem_st_32x32b_x16(sum_addr + c, r);
+                    } else if (valid) {
+                        const int e0 = n * BN + c;
+                        float *lrow = a.logits + (int64_t)t * a.E;
+                        if ((a.E & 3) == 0 && e0 + 16 <= a.E) {
+#pragma unroll
+                            for (int j = 0; j < 16; j += 4) {
+                                float4 v;
+                                v.x = __uint_as_float(r[j]) + (a.b_gate ? __ldg(a.b_gate + e0 + j) : 0.f);
+                                v.y = __uint_as_float(r[j + 1]) + (a.b_gate ? __ldg(a.b_gate + e0 + j + 1) : 0.f);
+                                v.z = __uint_as_float(r[j + 2]) + (a.b_gate ? __ldg(a.b_gate + e0 + j + 2) : 0.f);
+                                v.w = __uint_as_float(r[j + 3]) + (a.b_gate ? __ldg(a.b_gate + e0 + j + 3) : 0.f);
+                                *reinterpret_cast<float4 *>(lrow + e0 + j) = v;
+                            }
+                        } else {
+#pragma unroll
+                            for (int j = 0; j < 16; ++j)
+                                if (e0 + j < a.E)
+                                    lrow[e0 + j] = __uint_as_float(r[j]) + (a.b_gate ? __ldg(a.b_gate + e0 + j) : 0.f);
+                        }
+                    }
+                }
+                if (!last) tmem_st_wait();
+                tc_fence_before_sync();
+                mbar_arrive(&s.tempty[buf]);
+            }
+        }
+    }
+    tc_teardown<BN>(s, tmem_base);
+}
+
+template <int BN>
+cudaError_t launch_bn(const CUtensorMap &mx, const CUtensorMap &mw, const RouterTcArgs &a, cudaStream_t s) {
+    constexpr int smem = TcLayout<BN>::SMEM;
+    cudaError_t e =
+        cudaFuncSetAttribute(router_logits_tc_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    const int tiles = ((a.T + kBM - 1) / kBM) * (a.E_pad / BN);
+    router_logits_tc_kernel<BN><<<tiles < a.num_sms ? tiles : a.num_sms, kTcThreads, smem, s>>>(mx, mw, a);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+int router_tc_epad(int E) {
+    int p = 16;
+    while (p < E && p < 128) p <<= 1;
+    return p < E ? (E + 127) / 128 * 128 : p;
+}
+
+int router_tc_bn(int E) { return router_tc_epad(E) < 128 ? router_tc_epad(E) : 128; }
+
+cudaError_t launch_router_logits_tc(const CUtensorMap &map_x, const CUtensorMap &map_w, const RouterTcArgs &a,
+                                    __nv_bfloat16 *w_split, cudaStream_t s, int *launches) {
+    if (a.T <= 0) return cudaSuccess;
+    const int64_t n = (int64_t)a.E_pad * a.d;
+    int blocks = (int)((n + 255) / 256);
+    if (blocks > a.num_sms * 16) blocks = a.num_sms * 16;
+    router_split_kernel<<<blocks, 256, 0, s>>>(a.w_gate, a.E, a.E_pad, a.d, w_split);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    *launches += 2;
+    switch (router_tc_bn(a.E)) {
+        case 16: return launch_bn<16>(map_x, map_w, a, s);
+        case 32: return launch_bn<32>(map_x, map_w, a, s);
+        case 64: return launch_bn<64>(map_x, map_w, a, s);
+        case 128: return launch_bn<128>(map_x, map_w, a, s);
+        default: return cudaErrorInvalidValue;
+    }
+}
+
+}  // namespace moe

@@ -61,6 +61,7 @@ def _weights():
     ("input_dim", 0, binding.MOE_ERR_INVALID_ARG),
     ("input_dim", 500, binding.MOE_ERR_UNSUPPORTED),      # bf16 needs multiples of 64
     ("expert_dim", 1000, binding.MOE_ERR_UNSUPPORTED),
+    ("output_dim", 520, binding.MOE_ERR_UNSUPPORTED),     # bf16 stores 64-column boxes
     ("num_shared", -1, binding.MOE_ERR_INVALID_ARG),
     ("activation", 7, binding.MOE_ERR_INVALID_ARG),
     ("top_k_method", 5, binding.MOE_ERR_INVALID_ARG),
