@@ -82,7 +82,7 @@ __global__ void __launch_bounds__(kThreads) combine_kernel(CombineArgs a) {
         float c = 0.f;
         if (row >= 0) {
             float ss = 0.f;
-            for (int j = 0; j < a.n_tiles; ++j) ss += a.norm_part[(int64_t)row * a.n_tiles + j];
+            for (int j = 0; j < a.n_parts; ++j) ss += a.norm_part[(int64_t)row * a.n_parts + j];
             c = g * sqrtf(ss);
         }
         a.credit[ai] = c;

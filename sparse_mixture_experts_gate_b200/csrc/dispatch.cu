@@ -47,9 +47,18 @@ __global__ void __launch_bounds__(kMaxE) dispatch_scan_kernel(DispatchArgs a) {
     const int e = threadIdx.x, lane = e & 31, warp = e >> 5;
     int pre = 0, kept = 0, padded = 0;
     if (e < a.E) {
-        for (int c = 0; c < a.n_chunks; ++c) {
-            a.chunk_base[(int64_t)c * a.E + e] = pre;
-            pre += a.chunk_count[(int64_t)c * a.E + e];
+        // Exclusive prefix over chunks, loads batched so they are in flight together.
+        const int32_t *__restrict__ cnt = a.chunk_count;
+        int32_t *__restrict__ base = a.chunk_base;
+        for (int c0 = 0; c0 < a.n_chunks; c0 += 32) {
+            int v[32];
+#pragma unroll
+            for (int j = 0; j < 32; ++j) v[j] = c0 + j < a.n_chunks ? cnt[(int64_t)(c0 + j) * a.E + e] : 0;
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+                if (c0 + j < a.n_chunks) base[(int64_t)(c0 + j) * a.E + e] = pre;
+                pre += v[j];
+            }
         }
         kept = (int64_t)pre < a.C ? pre : (int)a.C;
         padded = (kept + kBM - 1) / kBM * kBM;

@@ -86,6 +86,7 @@ struct moe_layer {
     int G = 0;
     bool tc = false;
     int bn1 = 0, bn2 = 0, ntiles1 = 0, ntiles2 = 0;
+    int norm_parts = 0;  // fp32 partial sums of ||o||^2 per row (expert GEMM 2 writes them)
     int num_sms = 148;
     CUtensorMap map_w1, map_w2;
     // State of the most recent forward, read by moe_aux_stats.
@@ -146,7 +147,7 @@ Plan make_plan(const moe_layer &L, int T) {
     p.o_pm = take((size_t)E * 4);
     p.o_f = take((size_t)E * 4);
     p.o_credit = take((size_t)T * k * 4);
-    p.o_norm = take((size_t)p.R_max * L.ntiles2 * 4);
+    p.o_norm = take((size_t)p.R_max * L.norm_parts * 4);
     p.o_wsplit = take(c.dtype == MOE_DTYPE_BF16 ? (size_t)router_tc_epad(E) * 3 * c.input_dim * 2 : 0);
     p.o_xp = take(c.dtype == MOE_DTYPE_BF16 ? (size_t)p.R_routed_max * c.input_dim * es : 0);
     p.o_h = take((size_t)p.R_max * c.expert_dim * es);
@@ -258,6 +259,7 @@ int moe_layer_create(const moe_config_t *cfg, const moe_weights_t *w, moe_layer_
         L->bn2 = gemm_pick_bn(cfg->output_dim);
         L->ntiles1 = cfg->expert_dim / L->bn1;
         L->ntiles2 = cfg->output_dim / L->bn2;
+        L->norm_parts = L->ntiles2;
         if (!encode_bf16_2d(&L->map_w1, w->w1, cfg->input_dim, (uint64_t)L->G * cfg->expert_dim, L->bn1) ||
             !encode_bf16_2d(&L->map_w2, w->w2, cfg->expert_dim, (uint64_t)L->G * cfg->output_dim, L->bn2)) {
             delete L;
@@ -266,6 +268,7 @@ int moe_layer_create(const moe_config_t *cfg, const moe_weights_t *w, moe_layer_
     } else {
         L->ntiles1 = (cfg->expert_dim + kSimtBN - 1) / kSimtBN;
         L->ntiles2 = (cfg->output_dim + kSimtBN - 1) / kSimtBN;
+        L->norm_parts = L->ntiles2;
     }
     *out = L;
     return MOE_OK;
@@ -462,7 +465,7 @@ int moe_forward(moe_layer_t *L, const void *x, int32_t T, const float *logit_noi
     CombineArgs ca;
     ca.o = ws + p.o_o;
     ca.norm_part = g2.norm_part;
-    ca.n_tiles = L->ntiles2;
+    ca.n_parts = L->norm_parts;
     ca.row_of = da.row_of;
     ca.gates = gates;
     ca.group_start = da.group_start;

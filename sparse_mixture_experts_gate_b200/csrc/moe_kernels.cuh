@@ -95,7 +95,7 @@ struct GemmArgs {
     int k, T;
     const float *bias;           // [G][N] or null
     void *out;                   // [rows][N]
-    float *norm_part;            // [rows][n_tiles] or null: per-tile sum of out^2 (fp32, pre-rounding)
+    float *norm_part;            // [rows][n_tiles] or null: per-tile sum of out^2 (fp32, before rounding)
     int act;                     // activation code, -1 none
     uint32_t *status;            // device status word
     int num_sms;
@@ -121,8 +121,8 @@ cudaError_t launch_gemm_simt(const GemmSimtArgs &a, cudaStream_t s, int *launche
 // Gate-weighted combine with shared experts, plus credit.
 struct CombineArgs {
     const void *o;          // [rows][O] expert outputs
-    const float *norm_part; // [rows][n_tiles]
-    int n_tiles;
+    const float *norm_part; // [rows][n_parts]
+    int n_parts;
     const int32_t *row_of;  // [T][k]
     const float *gates;     // [T][k]
     const int32_t *group_start;

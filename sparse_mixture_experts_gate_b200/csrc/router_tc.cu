@@ -15,10 +15,10 @@
 //  * accumulation: the tensor core's fp32 accumulator does not round to
 //    nearest, and its error grows with the number of MMA steps and with the
 //    accumulator's magnitude. So the MMA starts a fresh partial every kDrain K
-//    blocks (kDrain * 4 MMA steps) and the epilogue warps add each partial into
-//    a running fp32 sum kept in TMEM, with ordinary round-to-nearest adds.
-// TMEM: two partial buffers (128 columns each, double-buffered so the MMA runs
-// ahead) and the running sum (128 columns); the N tile is <= 128 experts.
+//    blocks (kDrain * 4 MMA steps) and the epilogue adds each partial into a
+//    running fp32 sum held in registers, with ordinary round-to-nearest adds.
+// Eight epilogue warps, two per TMEM lane quarter, each own 64 of the N <= 128
+// columns of 32 tokens; TMEM holds two partial buffers so the MMA runs ahead.
 // Output: logits [T][E] (bias included). Softmax, keys, top-k and gates are
 // taken from them by the routing kernel in router.cu.
 #include "moe_common.cuh"
@@ -28,8 +28,8 @@
 namespace moe {
 namespace {
 
-constexpr int kDrain = 2;        // K blocks per partial accumulator
-constexpr int kSumCol = 256;     // TMEM column of the running sum
+constexpr int kDrain = 2;          // K blocks per partial accumulator
+constexpr int kRouterThreads = 320;  // producer, MMA, 8 epilogue warps
 
 // W_g [E][d] fp32 -> [E_pad][3d] bf16 planes (rows >= E are zero).
 __global__ void __launch_bounds__(256) router_split_kernel(const float *__restrict__ w, int E, int E_pad, int d,
@@ -51,10 +51,11 @@ __global__ void __launch_bounds__(256) router_split_kernel(const float *__restri
 }
 
 template <int BN>
-__global__ void __launch_bounds__(kTcThreads, 1)
+__global__ void __launch_bounds__(kRouterThreads, 1)
     router_logits_tc_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ CUtensorMap map_w,
                             const RouterTcArgs a) {
-    static_assert(BN <= 128, "two partial buffers and the running sum must fit in 512 TMEM columns");
+    static_assert(BN <= 128, "each epilogue thread holds BN / 2 <= 64 running sums");
+    constexpr int HALF = BN / 2;  // columns per epilogue thread
     using L = TcLayout<BN>;
     extern __shared__ uint8_t smem_raw[];
     const TcShared<BN> s = tc_carve<BN>(smem_raw);
@@ -62,7 +63,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         tma_prefetch_desc(&map_x);
         tma_prefetch_desc(&map_w);
     }
-    const uint32_t tmem_base = tc_setup<BN>(s);
+    const uint32_t tmem_base = tc_setup<BN>(s, 256);
     const int n_tiles = a.E_pad / BN;
     const int total = ((a.T + kBM - 1) / kBM) * n_tiles;
     const int dblocks = a.d / kBK;
@@ -122,14 +123,13 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         }
     } else {
         const int q = warp & 3, lane = threadIdx.x & 31;
+        const int col0 = ((warp - 2) >> 2) * HALF;  // this warp's half of the N tile
         uint32_t gcount = 0;
         bool ok = true;
         for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
             const int m = tile / n_tiles, n = tile - m * n_tiles;
             const int t = m * kBM + q * 32 + lane;
-            const bool valid = t < a.T;
-            const uint32_t lane_off = static_cast<uint32_t>(q * 32) << 16;
-            const uint32_t sum_addr = tmem_base + lane_off + kSumCol;
+            float sum[HALF];
             for (int g = 0; g < groups; ++g, ++gcount) {
                 const uint32_t buf = gcount & 1u, use = gcount >> 1;
                 const bool got = mbar_wait(&s.tfull[buf], use & 1u, a.status);
@@ -138,45 +138,45 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                     break;
                 }
                 tc_fence_after_sync();
-                const uint32_t acc_addr = tmem_base + lane_off + buf * kTcAccCols / 2;
-                const bool last = g == groups - 1;
-#pragma unroll 1
-                for (int c = 0; c < BN; c += 16) {
-                    uint32_t r[16], sm[16];
-                    tmem_ld_32x32b_x16(acc_addr + c, r);
-                    if (g > 0) tmem_ld_32x32b_x16(sum_addr + c, sm);
+                const uint32_t acc_addr =
+                    tmem_base + (static_cast<uint32_t>(q * 32) << 16) + buf * kTcAccCols / 2 + col0;
+#pragma unroll
+                for (int c = 0; c < HALF; c += 32) {
+                    uint32_t r[32];
+                    if (HALF - c >= 32) {
+                        tmem_ld_32x32b_x32(acc_addr + c, r);
+                    } else {
+                        tmem_ld_32x32b_x16(acc_addr + c, *reinterpret_cast<uint32_t(*)[16]>(&r[0]));
+                    }
                     tmem_ld_wait();
-                    if (g > 0) {
 #pragma unroll
-                        for (int j = 0; j < 16; ++j)
-                            r[j] = __float_as_uint(__fadd_rn(__uint_as_float(sm[j]), __uint_as_float(r[j])));
-                    }
-                    if (!last) {
-                        tmem_st_32x32b_x16(sum_addr + c, r);
-                    } else if (valid) {
-                        const int e0 = n * BN + c;
-                        float *lrow = a.logits + (int64_t)t * a.E;
-                        if ((a.E & 3) == 0 && e0 + 16 <= a.E) {
-#pragma unroll
-                            for (int j = 0; j < 16; j += 4) {
-                                float4 v;
-                                v.x = __uint_as_float(r[j]) + (a.b_gate ? __ldg(a.b_gate + e0 + j) : 0.f);
-                                v.y = __uint_as_float(r[j + 1]) + (a.b_gate ? __ldg(a.b_gate + e0 + j + 1) : 0.f);
-                                v.z = __uint_as_float(r[j + 2]) + (a.b_gate ? __ldg(a.b_gate + e0 + j + 2) : 0.f);
-                                v.w = __uint_as_float(r[j + 3]) + (a.b_gate ? __ldg(a.b_gate + e0 + j + 3) : 0.f);
-                                *reinterpret_cast<float4 *>(lrow + e0 + j) = v;
-                            }
-                        } else {
-#pragma unroll
-                            for (int j = 0; j < 16; ++j)
-                                if (e0 + j < a.E)
-                                    lrow[e0 + j] = __uint_as_float(r[j]) + (a.b_gate ? __ldg(a.b_gate + e0 + j) : 0.f);
-                        }
-                    }
+                    for (int j = 0; j < 32; ++j)
+                        if (c + j < HALF)
+                            sum[c + j] = g == 0 ? __uint_as_float(r[j]) : __fadd_rn(sum[c + j], __uint_as_float(r[j]));
                 }
-                if (!last) tmem_st_wait();
                 tc_fence_before_sync();
                 mbar_arrive(&s.tempty[buf]);
+            }
+            if (!ok || t >= a.T) continue;
+            const int e0 = n * BN + col0;
+            float *lrow = a.logits + (int64_t)t * a.E + e0;
+            if ((a.E & 3) == 0 && e0 + HALF <= a.E) {
+#pragma unroll
+                for (int j = 0; j < HALF; j += 4) {
+                    float4 v = make_float4(sum[j], sum[j + 1], sum[j + 2], sum[j + 3]);
+                    if (a.b_gate) {
+                        const float4 b = __ldg(reinterpret_cast<const float4 *>(a.b_gate + e0 + j));
+                        v.x += b.x;
+                        v.y += b.y;
+                        v.z += b.z;
+                        v.w += b.w;
+                    }
+                    *reinterpret_cast<float4 *>(lrow + j) = v;
+                }
+            } else {
+#pragma unroll
+                for (int j = 0; j < HALF; ++j)
+                    if (e0 + j < a.E) lrow[j] = sum[j] + (a.b_gate ? __ldg(a.b_gate + e0 + j) : 0.f);
             }
         }
     }
@@ -190,7 +190,7 @@ cudaError_t launch_bn(const CUtensorMap &mx, const CUtensorMap &mw, const Router
         cudaFuncSetAttribute(router_logits_tc_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
     const int tiles = ((a.T + kBM - 1) / kBM) * (a.E_pad / BN);
-    router_logits_tc_kernel<BN><<<tiles < a.num_sms ? tiles : a.num_sms, kTcThreads, smem, s>>>(mx, mw, a);
+    router_logits_tc_kernel<BN><<<tiles < a.num_sms ? tiles : a.num_sms, kRouterThreads, smem, s>>>(mx, mw, a);
     return cudaGetLastError();
 }
 

@@ -57,8 +57,9 @@ __device__ __forceinline__ TcShared<BN> tc_carve(uint8_t *smem_raw) {
 }
 
 // Barrier init (thread 0) and TMEM allocation (warp 1); returns the TMEM base.
+// tempty_count: epilogue threads that release an accumulator (128 = 4 warps).
 template <int BN>
-__device__ __forceinline__ uint32_t tc_setup(const TcShared<BN> &s) {
+__device__ __forceinline__ uint32_t tc_setup(const TcShared<BN> &s, uint32_t tempty_count = 128) {
     using L = TcLayout<BN>;
     const int warp = threadIdx.x >> 5;
     if (threadIdx.x == 0) {
@@ -68,7 +69,7 @@ __device__ __forceinline__ uint32_t tc_setup(const TcShared<BN> &s) {
         }
         for (int i = 0; i < 2; ++i) {
             mbar_init(&s.tfull[i], 1);
-            mbar_init(&s.tempty[i], 128);
+            mbar_init(&s.tempty[i], tempty_count);
         }
         mbar_init(s.mma_done, 1);
         fence_barrier_init();
