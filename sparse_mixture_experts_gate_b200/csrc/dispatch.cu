@@ -18,7 +18,7 @@
 //   assign - per chunk, the stable rank of each assignment: chunk base +
 //            assignments to the same expert in earlier warps + earlier lanes of
 //            the same warp (a per-warp lane bitmask per expert, popcounted).
-// Also the gather of the routed token rows into the permuted row space, which
+// Also the scatter of the routed token rows into the permuted row space, which
 // the tensor-core expert GEMM then reads as plain 128-row TMA tiles.
 #include "moe_common.cuh"
 #include "moe_kernels.cuh"
@@ -142,22 +142,27 @@ __global__ void __launch_bounds__(kChunk) dispatch_assign_kernel(DispatchArgs a)
     }
 }
 
-// One warp per row of the routed region; 16-byte vectors.
-__global__ void __launch_bounds__(256) gather_rows_kernel(GatherArgs a) {
-    const int rows = min(a.ctrl[kCtrlRoutedRows], a.max_rows);
-    const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
+// One warp per token: the token's row of x is read once and written to the
+// rows of every expert that kept it (16-byte vectors). Padding rows of the row
+// space are left as they are: the rows computed from them are never read.
+__global__ void __launch_bounds__(256) scatter_rows_kernel(ScatterArgs a) {
+    const int lane = threadIdx.x & 31;
+    const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
     const int nwarps = (gridDim.x * blockDim.x) >> 5;
     const int nvec = a.row_bytes / 16;
-    for (int row = warp; row < rows; row += nwarps) {
-        const int ai = a.row_assign[row];
-        uint4 *dst = reinterpret_cast<uint4 *>(static_cast<char *>(a.xp) + (int64_t)row * a.row_bytes);
-        if (ai < 0) {
-            for (int v = lane; v < nvec; v += 32) dst[v] = make_uint4(0u, 0u, 0u, 0u);
-        } else {
-            const int t = ai / a.k;
-            const uint4 *src =
-                reinterpret_cast<const uint4 *>(static_cast<const char *>(a.x) + (int64_t)t * a.row_bytes);
-            for (int v = lane; v < nvec; v += 32) dst[v] = __ldg(src + v);
+    for (int t = warp; t < a.T; t += nwarps) {
+        int rows[16];
+        int nk = 0;
+        for (int r = 0; r < a.k; ++r) {
+            const int row = a.row_of[(int64_t)t * a.k + r];
+            if (row >= 0) rows[nk++] = row;
+        }
+        if (nk == 0) continue;
+        const uint4 *src = reinterpret_cast<const uint4 *>(static_cast<const char *>(a.x) + (int64_t)t * a.row_bytes);
+        for (int v = lane; v < nvec; v += 32) {
+            const uint4 val = __ldg(src + v);
+            for (int i = 0; i < nk; ++i)
+                reinterpret_cast<uint4 *>(static_cast<char *>(a.xp) + (int64_t)rows[i] * a.row_bytes)[v] = val;
         }
     }
 }
@@ -173,15 +178,11 @@ cudaError_t launch_dispatch(const DispatchArgs &a, cudaStream_t s, int *launches
     return cudaGetLastError();
 }
 
-cudaError_t launch_gather(const GatherArgs &a, cudaStream_t s, int *launches) {
-    int dev = 0, sms = 148;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    const int warps_needed = a.max_rows;
-    int blocks = (warps_needed + 7) / 8;
-    if (blocks > sms * 8) blocks = sms * 8;
-    if (blocks < 1) blocks = 1;
-    gather_rows_kernel<<<blocks, 256, 0, s>>>(a);
+cudaError_t launch_scatter(const ScatterArgs &a, int num_sms, cudaStream_t s, int *launches) {
+    if (a.T <= 0) return cudaSuccess;
+    int blocks = (a.T + 7) / 8;
+    if (blocks > num_sms * 8) blocks = num_sms * 8;
+    scatter_rows_kernel<<<blocks, 256, 0, s>>>(a);
     ++*launches;
     return cudaGetLastError();
 }

@@ -5,7 +5,7 @@
 // dense contractions over the rows dispatched to it, so they run as one grouped
 // GEMM per layer over the permuted row space:
 //   out[row][n] = act( sum_k A[row][k] * W[g][n][k] + b[g][n] ),  g = group of row.
-// Layer 1: A = the routed token rows gathered into row order (dispatch.cu), and
+// Layer 1: A = the routed token rows scattered into row order (dispatch.cu), and
 //   x itself for the shared experts, which read every token in order.
 // Layer 2: A = the hidden activations H (already in row order);
 //   the epilogue also writes, per row and N tile, the fp32 sum of squares of

@@ -1,6 +1,6 @@
 // moe_api.cu - the C ABI declared in include/moe.h: argument validation, the
 // workspace plan, TMA descriptors, and the launch sequence of one MoE layer
-// forward (router -> dispatch -> gather -> expert GEMM 1 -> expert GEMM 2 ->
+// forward (router -> dispatch -> row scatter -> expert GEMM 1 -> expert GEMM 2 ->
 // combine) and of its statistics.
 #include <algorithm>
 #include <cmath>
@@ -390,15 +390,14 @@ int moe_forward(moe_layer_t *L, const void *x, int32_t T, const float *logit_noi
     MOE_MARK(L, 2, s);
 
     if (L->tc) {
-        GatherArgs ga;
-        ga.x = x;
-        ga.xp = ws + p.o_xp;
-        ga.row_assign = da.row_assign;
-        ga.ctrl = ctrl;
-        ga.k = k;
-        ga.row_bytes = c.input_dim * 2;
-        ga.max_rows = p.R_routed_max;
-        MOE_LAUNCH(launch_gather(ga, s, nl));
+        ScatterArgs sa;
+        sa.x = x;
+        sa.xp = ws + p.o_xp;
+        sa.row_of = da.row_of;
+        sa.T = T;
+        sa.k = k;
+        sa.row_bytes = c.input_dim * 2;
+        MOE_LAUNCH(launch_scatter(sa, L->num_sms, s, nl));
     }
 
     GemmArgs g1;

@@ -67,17 +67,15 @@ cudaError_t launch_dispatch(const DispatchArgs &a, cudaStream_t s, int *launches
 // Control block words.
 enum { kCtrlStatus = 0, kCtrlNumMTiles = 1, kCtrlRoutedRows = 2, kCtrlDropped = 3, kCtrlWords = 8 };
 
-// Gather of routed token rows into the permuted row space.
-struct GatherArgs {
+// Scatter of token rows into the permuted row space (rows of kept assignments).
+struct ScatterArgs {
     const void *x;          // [T][d]
     void *xp;               // [R_routed_max][d]
-    const int32_t *row_assign;
-    const int32_t *ctrl;
-    int k;
+    const int32_t *row_of;  // [T][k] row of each assignment, -1 if dropped
+    int T, k;
     int row_bytes;          // d * element size (multiple of 16)
-    int max_rows;           // R_routed_max
 };
-cudaError_t launch_gather(const GatherArgs &a, cudaStream_t s, int *launches);
+cudaError_t launch_scatter(const ScatterArgs &a, int num_sms, cudaStream_t s, int *launches);
 
 // Grouped expert GEMM: out[row] = act(A[row] . W[g]^T + b[g]) for the rows of
 // every group g (routed experts, then shared experts).
@@ -101,7 +99,7 @@ struct GemmArgs {
     int num_sms;
 };
 // bf16 tcgen05 path; BN (256, 128 or 64) is the largest that divides N.
-// A rows come from map_a0 (row space: the gathered rows or H, box 64 x 128); with
+// A rows come from map_a0 (row space: the scattered rows or H, box 64 x 128); with
 // use_a1, shared-expert groups read x itself through map_a1 (box 64 x 128).
 // map_out: the output [rows][N] bf16, box 64 x 32, 128B swizzle.
 int gemm_pick_bn(int N);
