@@ -67,6 +67,8 @@ struct Plan {
     int T = 0;
     int64_t C = 0;
     int T_pad = 0, n_stat_chunks = 0, n_chunks = 0, R_routed_max = 0, R_max = 0, max_mtiles = 0;
+    int ksplit = 1;
+    size_t o_lpart = 0;
     size_t o_ctrl, o_logits, o_idx, o_gates, o_slot, o_rowof, o_lse, o_psum, o_ccount, o_cbase, o_cpre, o_ckept,
         o_gstart, o_grows, o_tgroup, o_rowassign, o_wsplit, o_xp, o_h, o_o, o_norm, o_credit, o_pm, o_f;
     size_t total = 0;
@@ -93,7 +95,6 @@ struct moe_layer {
     bool has_forward = false;
     Plan plan;
     char *ws = nullptr;
-    float *logits = nullptr;
     int fwd_launches = 0, stats_launches = 0;
     bool timing = false;
     cudaEvent_t ev[MOE_TIMING_EVENTS];
@@ -119,7 +120,7 @@ Plan make_plan(const moe_layer &L, int T) {
     p.T_pad = (int)round_up(T, kBM);
     p.R_max = p.R_routed_max + S * p.T_pad;
     p.max_mtiles = p.R_max / kBM;
-    p.n_stat_chunks = (T + kStatsChunk - 1) / kStatsChunk;
+    p.n_stat_chunks = router_psum_blocks(T, L.num_sms, c.dtype == MOE_DTYPE_BF16);
     p.n_chunks = (T + 255) / 256;
     const size_t es = c.dtype == MOE_DTYPE_BF16 ? 2 : 4;
     size_t off = 0;
@@ -149,6 +150,8 @@ Plan make_plan(const moe_layer &L, int T) {
     p.o_credit = take((size_t)T * k * 4);
     p.o_norm = take((size_t)p.R_max * L.norm_parts * 4);
     p.o_wsplit = take(c.dtype == MOE_DTYPE_BF16 ? (size_t)router_tc_epad(E) * 3 * c.input_dim * 2 : 0);
+    p.ksplit = c.dtype == MOE_DTYPE_BF16 ? router_tc_ksplit(T, E, c.input_dim, L.num_sms) : 1;
+    p.o_lpart = take(p.ksplit > 1 ? (size_t)p.ksplit * T * E * 4 : 0);
     p.o_xp = take(c.dtype == MOE_DTYPE_BF16 ? (size_t)p.R_routed_max * c.input_dim * es : 0);
     p.o_h = take((size_t)p.R_max * c.expert_dim * es);
     p.o_o = take((size_t)p.R_max * c.output_dim * es);
@@ -322,7 +325,6 @@ int moe_forward(moe_layer_t *L, const void *x, int32_t T, const float *logit_noi
     int32_t *idx = rt && rt->topk_idx ? rt->topk_idx : reinterpret_cast<int32_t *>(ws + p.o_idx);
     float *gates = rt && rt->gates ? rt->gates : reinterpret_cast<float *>(ws + p.o_gates);
     int32_t *slot = rt && rt->slot ? rt->slot : reinterpret_cast<int32_t *>(ws + p.o_slot);
-    L->logits = logits;
     int *nl = &L->fwd_launches;
     uint32_t *status = reinterpret_cast<uint32_t *>(ctrl + kCtrlStatus);
 
@@ -341,6 +343,9 @@ int moe_forward(moe_layer_t *L, const void *x, int32_t T, const float *logit_noi
     ra.idx = idx;
     ra.gates = gates;
     ra.lse = reinterpret_cast<float *>(ws + p.o_lse);
+    ra.psum_part = reinterpret_cast<float *>(ws + p.o_psum);
+    ra.logit_part = nullptr;
+    ra.ksplit = 1;
     if (L->tc) {
         RouterTcArgs rt_args;
         rt_args.w_gate = L->w.w_gate;
@@ -350,6 +355,8 @@ int moe_forward(moe_layer_t *L, const void *x, int32_t T, const float *logit_noi
         rt_args.E = E;
         rt_args.E_pad = router_tc_epad(E);
         rt_args.logits = logits;
+        rt_args.ksplit = p.ksplit;
+        rt_args.partial = reinterpret_cast<float *>(ws + p.o_lpart);
         rt_args.status = status;
         rt_args.num_sms = L->num_sms;
         __nv_bfloat16 *w_split = reinterpret_cast<__nv_bfloat16 *>(ws + p.o_wsplit);
@@ -358,6 +365,10 @@ int moe_forward(moe_layer_t *L, const void *x, int32_t T, const float *logit_noi
             !encode_bf16_2d(&m_ws, w_split, 3ull * c.input_dim, rt_args.E_pad, router_tc_bn(E)))
             return fail(MOE_ERR_CUDA, "cuTensorMapEncodeTiled failed for the router operands");
         MOE_LAUNCH(launch_router_logits_tc(m_xr, m_ws, rt_args, w_split, s, nl));
+        if (p.ksplit > 1) {
+            ra.logit_part = rt_args.partial;
+            ra.ksplit = p.ksplit;
+        }
         MOE_LAUNCH(launch_route_from_logits(ra, L->num_sms, s, nl));
     } else {
         MOE_LAUNCH(launch_router(ra, s, nl));
@@ -493,8 +504,7 @@ int moe_aux_stats(moe_layer_t *L, const float *token_loss, const moe_stats_t *ou
     if (p.T == 0) return MOE_OK;
     char *ws = L->ws;
     StatsArgs sa;
-    sa.logits = L->logits;
-    sa.psum_part = reinterpret_cast<float *>(ws + p.o_psum);
+    sa.psum_part = reinterpret_cast<const float *>(ws + p.o_psum);
     sa.n_chunks = p.n_stat_chunks;
     sa.lse = reinterpret_cast<const float *>(ws + p.o_lse);
     sa.count_pre = reinterpret_cast<const int32_t *>(ws + p.o_cpre);

@@ -21,7 +21,11 @@ struct RouterArgs {
     int32_t *idx;           // [T][k]
     float *gates;           // [T][k]
     float *lse;             // [T]
+    float *psum_part;       // [router_psum_blocks][E]: per-block sums of P over its tokens
+    const float *logit_part;  // routing from split-K partials: [ksplit][T][E], or null
+    int ksplit;
 };
+int router_psum_blocks(int T, int num_sms, bool from_logits);
 cudaError_t launch_router(const RouterArgs &a, cudaStream_t s, int *launches);
 // Max, log-partition, keys, top-k and gates from logits already in a.logits.
 cudaError_t launch_route_from_logits(const RouterArgs &a, int num_sms, cudaStream_t s, int *launches);
@@ -31,12 +35,15 @@ struct RouterTcArgs {
     const float *w_gate;    // [E][d] fp32, split into bf16 planes every forward
     const float *b_gate;    // [E] or null
     int T, d, E, E_pad;
-    float *logits;          // [T][E]
+    float *logits;          // [T][E]   (ksplit == 1)
+    int ksplit;             // K splits (router_tc_ksplit)
+    float *partial;         // [ksplit][T][E] raw partial sums (ksplit > 1)
     uint32_t *status;
     int num_sms;
 };
 int router_tc_epad(int E);  // padded expert count (rows of the split planes)
 int router_tc_bn(int E);    // N tile of the logits GEMM (<= 128)
+int router_tc_ksplit(int T, int E, int d, int num_sms);
 // map_x: x [T][d] bf16, box 64 x 128; map_w: w_split [E_pad][3d] bf16, box 64 x router_tc_bn(E).
 cudaError_t launch_router_logits_tc(const CUtensorMap &map_x, const CUtensorMap &map_w, const RouterTcArgs &a,
                                     __nv_bfloat16 *w_split, cudaStream_t s, int *launches);
@@ -133,9 +140,8 @@ cudaError_t launch_combine(const CombineArgs &a, cudaStream_t s, int *launches);
 
 // Balancing and credit statistics.
 struct StatsArgs {
-    const float *logits;      // [T][E]
-    float *psum_part;         // [n_chunks][E] scratch: per-chunk sums of P
-    int n_chunks;             // ceil(T / kStatsChunk)
+    const float *psum_part;   // [n_chunks][E]: the router's per-block sums of P
+    int n_chunks;
     const float *lse;         // [T]
     const int32_t *count_pre; // [E]
     const int32_t *group_start;
@@ -151,7 +157,6 @@ struct StatsArgs {
     float *f, *p_mean, *l_aux, *l_z, *expert_loss;  // outputs (nullable)
     int32_t *n_dropped;
 };
-constexpr int kStatsChunk = 128;
 cudaError_t launch_stats(const StatsArgs &a, cudaStream_t s, int *launches);
 
 // Sets the calling thread's last-error message; returns `code`.

@@ -26,9 +26,11 @@ constexpr int kWarps = kThreads / 32;
 constexpr int kKC = 32;  // K chunk staged in shared memory
 
 // h[q] = clean logit of expert lane + 32 q (-inf for e >= E). Writes lse[t],
-// idx[t][0..k), gates[t][0..k).
+// idx[t][0..k), gates[t][0..k) and adds the token's probabilities P[t][e] to
+// pacc[q] (the caller's per-lane running sums over its tokens).
 template <int RE>
-__device__ __forceinline__ void route_warp(const float (&h)[RE], int t, int lane, const RouterArgs &a) {
+__device__ __forceinline__ void route_warp(const float (&h)[RE], int t, int lane, const RouterArgs &a,
+                                           float (&pacc)[RE]) {
     float key[RE];
     float m = -INFINITY;
 #pragma unroll
@@ -56,6 +58,9 @@ __device__ __forceinline__ void route_warp(const float (&h)[RE], int t, int lane
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) z += __shfl_xor_sync(0xffffffffu, z, off);
     if (lane == 0) a.lse[t] = m + logf(z);
+    const float inv_z = 1.f / z;
+#pragma unroll
+    for (int q = 0; q < RE; ++q) pacc[q] += ex[q] * inv_z;
 
     // Top-k by (key desc, expert index asc); the winner's clean exp(h - m)
     // feeds its gate.
@@ -108,6 +113,23 @@ __device__ __forceinline__ void route_warp(const float (&h)[RE], int t, int lane
     }
 }
 
+// Sums the warps' per-lane P sums in warp order and writes this block's row of
+// psum_part [blocks][E] (a fixed order, so the statistics are reproducible).
+template <int RE>
+__device__ __forceinline__ void write_block_psum(const float (&pacc)[RE], const RouterArgs &a) {
+    __shared__ float red[kWarps][32 * RE];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+#pragma unroll
+    for (int q = 0; q < RE; ++q) red[warp][lane + 32 * q] = pacc[q];
+    __syncthreads();
+    for (int e = threadIdx.x; e < a.E; e += kThreads) {
+        float s = 0.f;
+#pragma unroll
+        for (int w = 0; w < kWarps; ++w) s += red[w][e];
+        a.psum_part[(int64_t)blockIdx.x * a.E + e] = s;
+    }
+}
+
 template <typename XT, int RE, int RT>
 __global__ void __launch_bounds__(kThreads) router_simt_kernel(RouterArgs a) {
     constexpr int TM = kWarps * RT;   // tokens per CTA
@@ -154,6 +176,9 @@ __global__ void __launch_bounds__(kThreads) router_simt_kernel(RouterArgs a) {
         __syncthreads();
     }
 
+    float pacc[RE];
+#pragma unroll
+    for (int q = 0; q < RE; ++q) pacc[q] = 0.f;
 #pragma unroll
     for (int i = 0; i < RT; ++i) {
         const int t = t_base + warp * RT + i;
@@ -168,8 +193,9 @@ __global__ void __launch_bounds__(kThreads) router_simt_kernel(RouterArgs a) {
                 a.logits[(int64_t)t * a.E + e] = h[q];
             }
         }
-        route_warp<RE>(h, t, lane, a);
+        route_warp<RE>(h, t, lane, a, pacc);
     }
+    write_block_psum<RE>(pacc, a);
 }
 
 // One warp per token over logits already in memory (bias included).
@@ -178,15 +204,31 @@ __global__ void __launch_bounds__(kThreads) route_from_logits_kernel(RouterArgs 
     const int lane = threadIdx.x & 31;
     const int warp = (blockIdx.x * kThreads + threadIdx.x) >> 5;
     const int nwarps = (gridDim.x * kThreads) >> 5;
+    float pacc[RE];
+#pragma unroll
+    for (int q = 0; q < RE; ++q) pacc[q] = 0.f;
     for (int t = warp; t < a.T; t += nwarps) {
         float h[RE];
 #pragma unroll
         for (int q = 0; q < RE; ++q) {
             const int e = lane + 32 * q;
-            h[q] = e < a.E ? a.logits[(int64_t)t * a.E + e] : -INFINITY;
+            h[q] = -INFINITY;
+            if (e < a.E) {
+                if (a.logit_part) {  // split-K partials in split order, then the bias
+                    float v = a.logit_part[(int64_t)t * a.E + e];
+                    for (int sp = 1; sp < a.ksplit; ++sp)
+                        v = __fadd_rn(v, a.logit_part[((int64_t)sp * a.T + t) * a.E + e]);
+                    if (a.b_gate) v += a.b_gate[e];
+                    a.logits[(int64_t)t * a.E + e] = v;
+                    h[q] = v;
+                } else {
+                    h[q] = a.logits[(int64_t)t * a.E + e];
+                }
+            }
         }
-        route_warp<RE>(h, t, lane, a);
+        route_warp<RE>(h, t, lane, a, pacc);
     }
+    write_block_psum<RE>(pacc, a);
 }
 
 template <typename XT, int RE>
@@ -211,15 +253,24 @@ cudaError_t launch_x(const RouterArgs &a, cudaStream_t s, int rt) {
 
 template <int RE>
 cudaError_t launch_route(const RouterArgs &a, cudaStream_t s, int num_sms) {
-    int blocks = (a.T + kWarps - 1) / kWarps;
-    if (blocks > num_sms * 8) blocks = num_sms * 8;
-    route_from_logits_kernel<RE><<<blocks, kThreads, 0, s>>>(a);
+    route_from_logits_kernel<RE><<<router_psum_blocks(a.T, num_sms, true), kThreads, 0, s>>>(a);
     return cudaGetLastError();
 }
 
 int router_rt(int T) { return T >= 4096 ? 4 : 1; }
 
 }  // namespace
+
+// Blocks of the routing kernel = rows of psum_part it writes.
+int router_psum_blocks(int T, int num_sms, bool from_logits) {
+    if (T <= 0) return 0;
+    if (!from_logits) {
+        const int tm = kWarps * router_rt(T);
+        return (T + tm - 1) / tm;
+    }
+    int blocks = (T + kWarps - 1) / kWarps;
+    return blocks < num_sms * 8 ? blocks : num_sms * 8;
+}
 
 cudaError_t launch_router(const RouterArgs &a, cudaStream_t s, int *launches) {
     if (a.T <= 0) return cudaSuccess;

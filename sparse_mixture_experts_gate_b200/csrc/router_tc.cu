@@ -20,7 +20,9 @@
 // Eight epilogue warps, two per TMEM lane quarter, each own 64 of the N <= 128
 // columns of 32 tokens; TMEM holds two partial buffers so the MMA runs ahead.
 // Output: logits [T][E] (bias included). Softmax, keys, top-k and gates are
-// taken from them by the routing kernel in router.cu.
+// taken from them by the routing kernel in router.cu. With few tiles (small T)
+// the drain groups of a tile are split over ksplit CTAs (split-K); each writes
+// its fp32 partial sums and the routing kernel adds them in split order.
 #include "moe_common.cuh"
 #include "moe_kernels.cuh"
 #include "tc_pipeline.cuh"
@@ -65,16 +67,24 @@ __global__ void __launch_bounds__(kRouterThreads, 1)
     }
     const uint32_t tmem_base = tc_setup<BN>(s, 256);
     const int n_tiles = a.E_pad / BN;
-    const int total = ((a.T + kBM - 1) / kBM) * n_tiles;
+    const int ks = a.ksplit;
+    const int total = ((a.T + kBM - 1) / kBM) * n_tiles * ks;  // tile = (m * n_tiles + n) * ks + split
     const int dblocks = a.d / kBK;
     const int kblocks = 3 * dblocks;
     const int groups = (kblocks + kDrain - 1) / kDrain;
+    const int gps = (groups + ks - 1) / ks;  // drain groups per split
+    auto grange = [&](int tile) {
+        const int sp = tile % ks;
+        const int g0 = min(sp * gps, groups), g1 = min(g0 + gps, groups);
+        return make_int2(g0, g1);
+    };
     const int warp = threadIdx.x >> 5;
 
     if (warp == 0) {
         int arow = 0, brow = 0;
         auto tile_begin = [&](int tile, int) {
-            const int m = tile / n_tiles, n = tile - m * n_tiles;
+            const int mn = tile / ks;
+            const int m = mn / n_tiles, n = mn - m * n_tiles;
             arow = m * kBM;
             brow = n * BN;
         };
@@ -84,14 +94,18 @@ __global__ void __launch_bounds__(kRouterThreads, 1)
                 tma_load_2d(&map_w, bar, sB, kb * kBK, brow);
             }
         };
-        tc_producer<BN>(s, total, kblocks, a.status, tile_begin, load);
+        tc_producer_range<BN>(s, total, a.status, tile_begin, load, [&](int tile) {
+            const int2 gr = grange(tile);
+            return make_int2(gr.x * kDrain, min(gr.y * kDrain, kblocks));
+        });
     } else if (warp == 1) {
         if ((threadIdx.x & 31) == 0) {
             constexpr uint32_t idesc = idesc_bf16_f32(kBM, BN);
             uint32_t it = 0, gcount = 0;
             bool ok = true;
             for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
-                for (int g = 0; g < groups && ok; ++g, ++gcount) {
+                const int2 gr = grange(tile);
+                for (int g = gr.x; g < gr.y && ok; ++g, ++gcount) {
                     const uint32_t buf = gcount & 1u, use = gcount >> 1;
                     if (!mbar_wait(&s.tempty[buf], (use & 1u) ^ 1u, a.status)) {
                         ok = false;
@@ -127,10 +141,14 @@ __global__ void __launch_bounds__(kRouterThreads, 1)
         uint32_t gcount = 0;
         bool ok = true;
         for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
-            const int m = tile / n_tiles, n = tile - m * n_tiles;
+            const int mn = tile / ks, sp = tile % ks;
+            const int m = mn / n_tiles, n = mn - m * n_tiles;
             const int t = m * kBM + q * 32 + lane;
+            const int2 gr = grange(tile);
             float sum[HALF];
-            for (int g = 0; g < groups; ++g, ++gcount) {
+#pragma unroll
+            for (int j = 0; j < HALF; ++j) sum[j] = 0.f;
+            for (int g = gr.x; g < gr.y; ++g, ++gcount) {
                 const uint32_t buf = gcount & 1u, use = gcount >> 1;
                 const bool got = mbar_wait(&s.tfull[buf], use & 1u, a.status);
                 if (!__all_sync(0xffffffffu, got)) {
@@ -152,20 +170,22 @@ __global__ void __launch_bounds__(kRouterThreads, 1)
 #pragma unroll
                     for (int j = 0; j < 32; ++j)
                         if (c + j < HALF)
-                            sum[c + j] = g == 0 ? __uint_as_float(r[j]) : __fadd_rn(sum[c + j], __uint_as_float(r[j]));
+                            sum[c + j] = g == gr.x ? __uint_as_float(r[j]) : __fadd_rn(sum[c + j], __uint_as_float(r[j]));
                 }
                 tc_fence_before_sync();
                 mbar_arrive(&s.tempty[buf]);
             }
             if (!ok || t >= a.T) continue;
             const int e0 = n * BN + col0;
-            float *lrow = a.logits + (int64_t)t * a.E + e0;
+            // ksplit > 1: raw partial sums (the routing kernel adds splits and bias).
+            const float *bias = ks > 1 ? nullptr : a.b_gate;
+            float *lrow = (ks > 1 ? a.partial + (int64_t)sp * a.T * a.E : a.logits) + (int64_t)t * a.E + e0;
             if ((a.E & 3) == 0 && e0 + HALF <= a.E) {
 #pragma unroll
                 for (int j = 0; j < HALF; j += 4) {
                     float4 v = make_float4(sum[j], sum[j + 1], sum[j + 2], sum[j + 3]);
-                    if (a.b_gate) {
-                        const float4 b = __ldg(reinterpret_cast<const float4 *>(a.b_gate + e0 + j));
+                    if (bias) {
+                        const float4 b = __ldg(reinterpret_cast<const float4 *>(bias + e0 + j));
                         v.x += b.x;
                         v.y += b.y;
                         v.z += b.z;
@@ -176,7 +196,7 @@ __global__ void __launch_bounds__(kRouterThreads, 1)
             } else {
 #pragma unroll
                 for (int j = 0; j < HALF; ++j)
-                    if (e0 + j < a.E) lrow[j] = sum[j] + (a.b_gate ? __ldg(a.b_gate + e0 + j) : 0.f);
+                    if (e0 + j < a.E) lrow[j] = sum[j] + (bias ? __ldg(bias + e0 + j) : 0.f);
             }
         }
     }
@@ -189,7 +209,7 @@ cudaError_t launch_bn(const CUtensorMap &mx, const CUtensorMap &mw, const Router
     cudaError_t e =
         cudaFuncSetAttribute(router_logits_tc_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
-    const int tiles = ((a.T + kBM - 1) / kBM) * (a.E_pad / BN);
+    const int tiles = ((a.T + kBM - 1) / kBM) * (a.E_pad / BN) * a.ksplit;
     router_logits_tc_kernel<BN><<<tiles < a.num_sms ? tiles : a.num_sms, kRouterThreads, smem, s>>>(mx, mw, a);
     return cudaGetLastError();
 }
@@ -203,6 +223,15 @@ int router_tc_epad(int E) {
 }
 
 int router_tc_bn(int E) { return router_tc_epad(E) < 128 ? router_tc_epad(E) : 128; }
+
+int router_tc_ksplit(int T, int E, int d, int num_sms) {
+    const int tiles = ((T + kBM - 1) / kBM) * (router_tc_epad(E) / router_tc_bn(E));
+    const int groups = (3 * (d / kBK) + kDrain - 1) / kDrain;
+    if (tiles <= 0 || 2 * tiles > num_sms) return 1;
+    int ks = num_sms / tiles;
+    if (ks > groups / 8) ks = groups / 8;  // keep at least 8 drain groups per split
+    return ks < 1 ? 1 : ks;
+}
 
 cudaError_t launch_router_logits_tc(const CUtensorMap &map_x, const CUtensorMap &map_w, const RouterTcArgs &a,
                                     __nv_bfloat16 *w_split, cudaStream_t s, int *launches) {

@@ -21,18 +21,6 @@ __device__ __forceinline__ float warp_sum(float v) {
     return v;
 }
 
-// Per chunk of kStatsChunk tokens, thread e sums P[t][e] = exp(h[t][e] - lse[t])
-// over the chunk's tokens in ascending order.
-__global__ void __launch_bounds__(256) stats_psum_kernel(StatsArgs a) {
-    const int t0 = blockIdx.x * kStatsChunk;
-    const int t1 = min(t0 + kStatsChunk, a.T);
-    for (int e = threadIdx.x; e < a.E; e += blockDim.x) {
-        float s = 0.f;
-        for (int t = t0; t < t1; ++t) s += expf(a.logits[(int64_t)t * a.E + e] - a.lse[t]);
-        a.psum_part[(int64_t)blockIdx.x * a.E + e] = s;
-    }
-}
-
 // One warp per expert: P_i from the per-chunk partial sums, f_i, and the
 // attributed loss over the expert's kept rows (ascending row = ascending token).
 __global__ void __launch_bounds__(256) stats_expert_kernel(StatsArgs a) {
@@ -92,10 +80,9 @@ __global__ void __launch_bounds__(256) stats_scalar_kernel(StatsArgs a) {
 
 cudaError_t launch_stats(const StatsArgs &a, cudaStream_t s, int *launches) {
     if (a.T <= 0) return cudaSuccess;
-    stats_psum_kernel<<<a.n_chunks, 256, 0, s>>>(a);
     stats_expert_kernel<<<(a.E * 32 + 255) / 256, 256, 0, s>>>(a);
     stats_scalar_kernel<<<1, 256, 0, s>>>(a);
-    *launches += 3;
+    *launches += 2;
     return cudaGetLastError();
 }
 

@@ -100,16 +100,18 @@ __device__ __forceinline__ void tc_teardown(const TcShared<BN> &s, uint32_t tmem
 // `tile_begin(tile, lane)` runs once per tile before its first K block. Lane 0
 // owns the barrier protocol; the wait outcome is broadcast so the warp stays
 // convergent.
-template <int BN, class TileBegin, class LoadFn>
-__device__ __forceinline__ void tc_producer(const TcShared<BN> &s, int total, int kblocks, uint32_t *status,
-                                            TileBegin tile_begin, LoadFn load) {
+// As tc_producer, with a per-tile K-block range [x, y) from krange(tile).
+template <int BN, class TileBegin, class LoadFn, class KRange>
+__device__ __forceinline__ void tc_producer_range(const TcShared<BN> &s, int total, uint32_t *status,
+                                                  TileBegin tile_begin, LoadFn load, KRange krange) {
     using L = TcLayout<BN>;
     const int lane = threadIdx.x & 31;
     uint32_t it = 0;
     bool ok = true;
     for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
         tile_begin(tile, lane);
-        for (int kb = 0; kb < kblocks; ++kb) {
+        const int2 kr = krange(tile);
+        for (int kb = kr.x; kb < kr.y; ++kb) {
             const int st = it % L::NS;
             const uint32_t ph = (it / L::NS) & 1u;
             int got = 1;
@@ -131,6 +133,12 @@ __device__ __forceinline__ void tc_producer(const TcShared<BN> &s, int total, in
         for (uint32_t j = (it > (uint32_t)L::NS ? it - L::NS : 0u); j < it; ++j)
             mbar_wait_drain(&s.full[j % L::NS], (j / L::NS) & 1u);
     }
+}
+
+template <int BN, class TileBegin, class LoadFn>
+__device__ __forceinline__ void tc_producer(const TcShared<BN> &s, int total, int kblocks, uint32_t *status,
+                                            TileBegin tile_begin, LoadFn load) {
+    tc_producer_range<BN>(s, total, status, tile_begin, load, [&](int) { return make_int2(0, kblocks); });
 }
 
 // MMA role, one lane of warp 1.
