@@ -220,6 +220,27 @@ MOE_API int moe_forward_noalloc(moe_layer_t *layer, const void *x, int32_t T, co
 MOE_API int moe_aux_stats(moe_layer_t *layer, const float *token_loss, const moe_stats_t *out,
                   void *stream);
 
+/* Data-parallel statistics. The statistics are functions of sums that add over
+ * token shards ("Appendix C", "Balancing": f_i and P_i are batch fractions and
+ * means; the z-loss is a batch mean), so ranks that each run moe_forward on
+ * their own tokens get the statistics of the whole batch from:
+ *   1. moe_stat_partials: this rank's sums into `partials` (device, fp32,
+ *      MOE_STAT_PARTIALS(E) floats):
+ *        [0, E)  sum_t P[t][e]       [E, 2E)  selections per expert before the cap
+ *        [2E]    sum_t lse_t^2       [2E+1]   T        [2E+2] dropped assignments
+ *        [2E+3, 3E+3) sum over kept assignments of credit * token_loss
+ *      (the last block is zero when token_loss is NULL);
+ *   2. a sum all-reduce of `partials` across the ranks (NCCL, by the caller);
+ *   3. moe_stats_from_partials: f, p_mean, l_aux, l_z, n_dropped and (when
+ *      has_token_loss) expert_loss of the summed batch into `out`; out->credit
+ *      is per token and not written here (moe_aux_stats writes the local one).
+ * moe_aux_stats is steps 1 and 3 on this rank alone. Errors: STATE before any
+ * forward, INVALID_ARG for NULL pointers. */
+#define MOE_STAT_PARTIALS(E) (3 * (E) + 3)
+MOE_API int moe_stat_partials(moe_layer_t *layer, const float *token_loss, float *partials, void *stream);
+MOE_API int moe_stats_from_partials(moe_layer_t *layer, const float *partials, int32_t has_token_loss,
+                                    const moe_stats_t *out, void *stream);
+
 /* Device status word of the most recent forward: synchronises `stream`, then
  * returns MOE_OK, or MOE_ERR_TIMEOUT if a bounded device-side wait gave up. */
 MOE_API int moe_device_status(moe_layer_t *layer, void *stream);

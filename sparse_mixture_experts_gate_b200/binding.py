@@ -21,7 +21,7 @@ MOE_DTYPE = {"bf16": 0, "fp32": 1}
 
 # Every symbol include/moe.h declares.
 EXPORTS = ("moe_config_default", "moe_layer_create", "moe_workspace_bytes", "moe_capacity", "moe_forward",
-           "moe_forward_noalloc", "moe_aux_stats", "moe_device_status", "moe_set_timing_events", "moe_launch_count", "moe_destroy", "moe_status_string",
+           "moe_forward_noalloc", "moe_aux_stats", "moe_stat_partials", "moe_stats_from_partials", "moe_device_status", "moe_set_timing_events", "moe_launch_count", "moe_destroy", "moe_status_string",
            "moe_last_error")
 
 
@@ -82,6 +82,10 @@ def lib() -> ctypes.CDLL:
         L.moe_forward_noalloc.argtypes = [vp, vp, i32, vp, vp, ctypes.POINTER(MoeRouting), vp]
         L.moe_aux_stats.restype = ctypes.c_int
         L.moe_aux_stats.argtypes = [vp, vp, ctypes.POINTER(MoeStats), vp]
+        L.moe_stat_partials.restype = ctypes.c_int
+        L.moe_stat_partials.argtypes = [vp, vp, vp, vp]
+        L.moe_stats_from_partials.restype = ctypes.c_int
+        L.moe_stats_from_partials.argtypes = [vp, vp, i32, ctypes.POINTER(MoeStats), vp]
         L.moe_device_status.restype = ctypes.c_int
         L.moe_device_status.argtypes = [vp, vp]
         L.moe_set_timing_events.restype = ctypes.c_int
@@ -149,6 +153,29 @@ def moe_forward_noalloc(layer: int, x: int, T: int, logit_noise: Optional[int], 
 
 def moe_aux_stats(layer: int, token_loss: Optional[int], stats: MoeStats, stream: int) -> int:
     return _check(lib().moe_aux_stats(layer, token_loss, ctypes.byref(stats), stream), "moe_aux_stats")
+
+
+def moe_stat_partials(layer: int, token_loss: Optional[int], partials: int, stream: int) -> int:
+    return _check(lib().moe_stat_partials(layer, token_loss, partials, stream), "moe_stat_partials")
+
+
+def moe_stats_from_partials(layer: int, partials: int, has_token_loss: bool, stats: MoeStats, stream: int) -> int:
+    return _check(lib().moe_stats_from_partials(layer, partials, int(has_token_loss), ctypes.byref(stats), stream),
+                  "moe_stats_from_partials")
+
+
+def stat_partials_size(E: int) -> int:
+    return 3 * E + 3
+
+
+def allreduce_partials(partials, group=None):
+    """Sums the statistics' partial sums over the ranks of `group` in place
+    (a no-op without an initialised process group). Every rank must call it
+    at the same step, like any collective."""
+    import torch.distributed as dist
+    if dist.is_available() and dist.is_initialized() and dist.get_world_size(group) > 1:
+        dist.all_reduce(partials, op=dist.ReduceOp.SUM, group=group)
+    return partials
 
 
 def moe_device_status(layer: int, stream: int) -> int:
@@ -275,6 +302,21 @@ class MoELayer:
                       _ptr(out["expert_loss"]) if token_loss is not None else None)
         moe_aux_stats(self.handle, _ptr(token_loss), st, s)
         return out
+
+    def dp_aux_stats(self, out, token_loss=None, group=None, stream=None):
+        """Statistics of the whole data-parallel batch: this rank's partial sums,
+        a sum all-reduce over `group` (torch.distributed), then the statistics
+        from the summed partials. out["credit"] stays this rank's."""
+        import torch
+        s = stream if stream is not None else torch.cuda.current_stream(self.device).cuda_stream
+        self.aux_stats(out, token_loss=token_loss, stream=stream)
+        partials = torch.empty(stat_partials_size(self.w.E), dtype=torch.float32, device=self.device)
+        moe_stat_partials(self.handle, _ptr(token_loss), partials.data_ptr(), s)
+        allreduce_partials(partials, group)
+        st = MoeStats(_ptr(out["f"]), _ptr(out["p_mean"]), _ptr(out["l_aux"]), _ptr(out["l_z"]),
+                      _ptr(out["n_dropped"]), None, _ptr(out["expert_loss"]) if token_loss is not None else None)
+        moe_stats_from_partials(self.handle, partials.data_ptr(), token_loss is not None, st, s)
+        return out, partials
 
     def device_status(self, stream=None) -> int:
         import torch

@@ -79,7 +79,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         };
         tc_producer<BN>(s, total, kblocks, a.status, tile_begin, load);
     } else if (warp == 1) {
-        if ((threadIdx.x & 31) == 0) tc_mma<BN>(s, tmem_base, total, kblocks, a.status);
+        if ((threadIdx.x & 31) == 0)
+            tc_mma<BN>(s, tmem_base, total, kblocks, a.status,
+                       [&](int tile) { return tile % a.n_tiles == a.n_tiles - 1 ? a.n_last : BN; });
     } else {
         uint8_t *my_stage = staging + (warp - 2) * 2 * kStageBoxBytes;
         uint32_t sub = 0;  // store boxes this warp has issued
@@ -88,9 +90,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             const int g = a.tile_group[m];
             const int grow = m * kBM + q * 32 + lane;
             const float *bias = a.bias ? a.bias + (int64_t)g * a.N + n * BN : nullptr;
+            const int ncols = n == a.n_tiles - 1 ? a.n_last : BN;
             float ss = 0.f;
 #pragma unroll 1
-            for (int c = 0; c < BN; c += kStoreCols) {
+            for (int c = 0; c < ncols; c += kStoreCols) {
                 uint8_t *buf = my_stage + (sub & 1u) * kStageBoxBytes;
                 if (lane == 0) bulk_wait_group_read<1>();  // the store that last used `buf` has read it
                 __syncwarp();
@@ -175,10 +178,9 @@ cudaError_t launch_bn(const CUtensorMap &m0, const CUtensorMap &m1, const CUtens
 }  // namespace
 
 int gemm_pick_bn(int N) {
-    static const int options[] = {256, 128, 64};
-    for (int bn : options)
-        if (N % bn == 0) return bn;
-    return 0;
+    if (N % 64 != 0 || N <= 0) return 0;
+    if (N % 256 == 0 || N > 256) return 256;  // a ragged last tile is cheaper than a narrow BN
+    return N % 128 == 0 ? 128 : 64;
 }
 
 cudaError_t launch_gemm_tc(const CUtensorMap &m0, const CUtensorMap &m1, const CUtensorMap &mb, const CUtensorMap &mo,

@@ -70,7 +70,7 @@ struct Plan {
     int ksplit = 1;
     size_t o_lpart = 0;
     size_t o_ctrl, o_logits, o_idx, o_gates, o_slot, o_rowof, o_lse, o_psum, o_ccount, o_cbase, o_cpre, o_ckept,
-        o_gstart, o_grows, o_tgroup, o_rowassign, o_wsplit, o_xp, o_h, o_o, o_norm, o_credit, o_pm, o_f;
+        o_gstart, o_grows, o_tgroup, o_rowassign, o_wsplit, o_xp, o_h, o_o, o_norm, o_credit, o_partials;
     size_t total = 0;
 };
 
@@ -145,8 +145,7 @@ Plan make_plan(const moe_layer &L, int T) {
     p.o_grows = take((size_t)(E + S) * 4);
     p.o_tgroup = take((size_t)p.max_mtiles * 4);
     p.o_rowassign = take((size_t)p.R_max * 4);
-    p.o_pm = take((size_t)E * 4);
-    p.o_f = take((size_t)E * 4);
+    p.o_partials = take((size_t)(3 * E + 3) * 4);
     p.o_credit = take((size_t)T * k * 4);
     p.o_norm = take((size_t)p.R_max * L.norm_parts * 4);
     p.o_wsplit = take(c.dtype == MOE_DTYPE_BF16 ? (size_t)router_tc_epad(E) * 3 * c.input_dim * 2 : 0);
@@ -260,8 +259,8 @@ int moe_layer_create(const moe_config_t *cfg, const moe_weights_t *w, moe_layer_
     if (L->tc) {
         L->bn1 = gemm_pick_bn(cfg->expert_dim);
         L->bn2 = gemm_pick_bn(cfg->output_dim);
-        L->ntiles1 = cfg->expert_dim / L->bn1;
-        L->ntiles2 = cfg->output_dim / L->bn2;
+        L->ntiles1 = (cfg->expert_dim + L->bn1 - 1) / L->bn1;
+        L->ntiles2 = (cfg->output_dim + L->bn2 - 1) / L->bn2;
         L->norm_parts = L->ntiles2;
         if (!encode_bf16_2d(&L->map_w1, w->w1, cfg->input_dim, (uint64_t)L->G * cfg->expert_dim, L->bn1) ||
             !encode_bf16_2d(&L->map_w2, w->w2, cfg->expert_dim, (uint64_t)L->G * cfg->output_dim, L->bn2)) {
@@ -420,6 +419,7 @@ int moe_forward(moe_layer_t *L, const void *x, int32_t T, const float *logit_noi
     g1.N = c.expert_dim;
     g1.K = c.input_dim;
     g1.n_tiles = L->ntiles1;
+    g1.n_last = c.expert_dim - (L->ntiles1 - 1) * (L->tc ? L->bn1 : kSimtBN);
     g1.E = E;
     g1.use_a1 = 1;
     g1.row_assign = da.row_assign;
@@ -436,6 +436,7 @@ int moe_forward(moe_layer_t *L, const void *x, int32_t T, const float *logit_noi
     g2.N = c.output_dim;
     g2.K = c.expert_dim;
     g2.n_tiles = L->ntiles2;
+    g2.n_last = c.output_dim - (L->ntiles2 - 1) * (L->tc ? L->bn2 : kSimtBN);
     g2.bias = L->w.b2;
     g2.out = ws + p.o_o;
     g2.norm_part = reinterpret_cast<float *>(ws + p.o_norm);
@@ -492,16 +493,14 @@ int moe_forward(moe_layer_t *L, const void *x, int32_t T, const float *logit_noi
     return MOE_OK;
 }
 
-int moe_aux_stats(moe_layer_t *L, const float *token_loss, const moe_stats_t *out, void *stream_v) {
-    g_last_error.clear();
-    if (!L) return fail(MOE_ERR_INVALID_ARG, "layer is NULL");
-    if (!out) return fail(MOE_ERR_INVALID_ARG, "out is NULL");
-    if (!L->has_forward) return fail(MOE_ERR_STATE, "moe_aux_stats called before any moe_forward");
+}  // extern "C"
+
+namespace {
+
+// Enqueues the partial sums of the most recent forward into `partials`.
+int enqueue_partials(moe_layer_t *L, const float *token_loss, float *partials, cudaStream_t s, int *launches) {
     const Plan &p = L->plan;
     const moe_config_t &c = L->cfg;
-    cudaStream_t s = as_stream(stream_v);
-    L->stats_launches = 0;
-    if (p.T == 0) return MOE_OK;
     char *ws = L->ws;
     StatsArgs sa;
     sa.psum_part = reinterpret_cast<const float *>(ws + p.o_psum);
@@ -517,22 +516,78 @@ int moe_aux_stats(moe_layer_t *L, const float *token_loss, const moe_stats_t *ou
     sa.T = p.T;
     sa.E = c.num_experts;
     sa.k = c.num_active;
-    sa.alpha = c.load_balance_coef;
-    sa.beta = c.z_loss_coef;
-    sa.p_mean_ws = reinterpret_cast<float *>(ws + p.o_pm);
-    sa.f_ws = reinterpret_cast<float *>(ws + p.o_f);
-    sa.f = out->f;
-    sa.p_mean = out->p_mean;
-    sa.l_aux = out->l_aux;
-    sa.l_z = out->l_z;
-    sa.expert_loss = out->expert_loss;
-    sa.n_dropped = out->n_dropped;
-    MOE_LAUNCH(launch_stats(sa, s, &L->stats_launches));
+    sa.partials = partials;
+    MOE_LAUNCH(launch_stat_partials(sa, s, launches));
+    return MOE_OK;
+}
+
+int enqueue_finalize(moe_layer_t *L, const float *partials, bool has_loss, const moe_stats_t *out, cudaStream_t s,
+                     int *launches) {
+    const moe_config_t &c = L->cfg;
+    FinalizeArgs fa;
+    fa.partials = partials;
+    fa.E = c.num_experts;
+    fa.k = c.num_active;
+    fa.alpha = c.load_balance_coef;
+    fa.beta = c.z_loss_coef;
+    fa.f = out->f;
+    fa.p_mean = out->p_mean;
+    fa.l_aux = out->l_aux;
+    fa.l_z = out->l_z;
+    fa.expert_loss = has_loss ? out->expert_loss : nullptr;
+    fa.n_dropped = out->n_dropped;
+    MOE_LAUNCH(launch_stats_finalize(fa, s, launches));
+    return MOE_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int moe_aux_stats(moe_layer_t *L, const float *token_loss, const moe_stats_t *out, void *stream_v) {
+    g_last_error.clear();
+    if (!L) return fail(MOE_ERR_INVALID_ARG, "layer is NULL");
+    if (!out) return fail(MOE_ERR_INVALID_ARG, "out is NULL");
+    if (!L->has_forward) return fail(MOE_ERR_STATE, "moe_aux_stats called before any moe_forward");
+    const Plan &p = L->plan;
+    const moe_config_t &c = L->cfg;
+    cudaStream_t s = as_stream(stream_v);
+    L->stats_launches = 0;
+    if (p.T == 0) return MOE_OK;
+    float *partials = reinterpret_cast<float *>(L->ws + p.o_partials);
+    int rc = enqueue_partials(L, token_loss, partials, s, &L->stats_launches);
+    if (rc != MOE_OK) return rc;
+    rc = enqueue_finalize(L, partials, token_loss != nullptr, out, s, &L->stats_launches);
+    if (rc != MOE_OK) return rc;
     if (out->credit)
-        MOE_LAUNCH(cudaMemcpyAsync(out->credit, ws + p.o_credit, (size_t)p.T * c.num_active * 4,
+        MOE_LAUNCH(cudaMemcpyAsync(out->credit, L->ws + p.o_credit, (size_t)p.T * c.num_active * 4,
                                    cudaMemcpyDeviceToDevice, s));
     MOE_MARK(L, 6, s);
     return MOE_OK;
+}
+
+int moe_stat_partials(moe_layer_t *L, const float *token_loss, float *partials, void *stream_v) {
+    g_last_error.clear();
+    if (!L) return fail(MOE_ERR_INVALID_ARG, "layer is NULL");
+    if (!partials) return fail(MOE_ERR_INVALID_ARG, "partials is NULL");
+    if (!L->has_forward) return fail(MOE_ERR_STATE, "moe_stat_partials called before any moe_forward");
+    cudaStream_t s = as_stream(stream_v);
+    if (L->plan.T == 0) {
+        MOE_LAUNCH(cudaMemsetAsync(partials, 0, (size_t)(3 * L->cfg.num_experts + 3) * 4, s));
+        return MOE_OK;
+    }
+    int launches = 0;
+    return enqueue_partials(L, token_loss, partials, s, &launches);
+}
+
+int moe_stats_from_partials(moe_layer_t *L, const float *partials, int32_t has_token_loss, const moe_stats_t *out,
+                            void *stream_v) {
+    g_last_error.clear();
+    if (!L) return fail(MOE_ERR_INVALID_ARG, "layer is NULL");
+    if (!partials) return fail(MOE_ERR_INVALID_ARG, "partials is NULL");
+    if (!out) return fail(MOE_ERR_INVALID_ARG, "out is NULL");
+    int launches = 0;
+    return enqueue_finalize(L, partials, has_token_loss != 0, out, as_stream(stream_v), &launches);
 }
 
 int moe_device_status(moe_layer_t *L, void *stream_v) {

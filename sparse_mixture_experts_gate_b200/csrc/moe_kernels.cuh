@@ -93,7 +93,8 @@ struct GemmArgs {
     const int32_t *ctrl;         // kCtrlNumMTiles
     int max_mtiles;              // host bound on the M tiles (clamps the device count)
     int N, K;                    // output row length, reduction length
-    int n_tiles;                 // N / BN
+    int n_tiles;                 // ceil(N / BN)
+    int n_last;                  // columns of the last N tile (N - (n_tiles - 1) BN)
     int E;                       // groups >= E are shared experts (A through the second map)
     int use_a1;
     const int32_t *row_assign;   // [rows] t*k + r of each routed row (-1 padding)
@@ -105,7 +106,8 @@ struct GemmArgs {
     uint32_t *status;            // device status word
     int num_sms;
 };
-// bf16 tcgen05 path; BN (256, 128 or 64) is the largest that divides N.
+// bf16 tcgen05 path; BN is 256 when N > 256 (the last N tile may be narrower),
+// else the largest of 128 and 64 dividing N. N must be a multiple of 64.
 // A rows come from map_a0 (row space: the scattered rows or H, box 64 x 128); with
 // use_a1, shared-expert groups read x itself through map_a1 (box 64 x 128).
 // map_out: the output [rows][N] bf16, box 64 x 32, 128B swizzle.
@@ -138,7 +140,7 @@ struct CombineArgs {
 };
 cudaError_t launch_combine(const CombineArgs &a, cudaStream_t s, int *launches);
 
-// Balancing and credit statistics.
+// Balancing and credit statistics: partial sums, then finalize.
 struct StatsArgs {
     const float *psum_part;   // [n_chunks][E]: the router's per-block sums of P
     int n_chunks;
@@ -151,13 +153,18 @@ struct StatsArgs {
     const float *token_loss;  // [T] or null
     const int32_t *ctrl;
     int T, E, k;
+    float *partials;          // [3E + 3] output
+};
+cudaError_t launch_stat_partials(const StatsArgs &a, cudaStream_t s, int *launches);
+
+struct FinalizeArgs {
+    const float *partials;    // [3E + 3]
+    int E, k;
     float alpha, beta;
-    float *p_mean_ws;         // [E] scratch
-    float *f_ws;              // [E] scratch
     float *f, *p_mean, *l_aux, *l_z, *expert_loss;  // outputs (nullable)
     int32_t *n_dropped;
 };
-cudaError_t launch_stats(const StatsArgs &a, cudaStream_t s, int *launches);
+cudaError_t launch_stats_finalize(const FinalizeArgs &a, cudaStream_t s, int *launches);
 
 // Sets the calling thread's last-error message; returns `code`.
 int report_error(int code, const char *msg);

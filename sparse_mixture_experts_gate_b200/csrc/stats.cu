@@ -7,8 +7,9 @@
 // Loss Reweighting Diagram", panel (b): the expert-attributed loss
 // l_i = (1/N) sum_j c_i(x_j) l_j 1[i in T_j], N = T, over kept assignments.
 //
-// Every reduction has a fixed order (per-lane strided sums, then a fixed
-// shuffle tree), so repeated runs give bit-identical statistics.
+// The statistics are a function of sums that add over token shards, so they are
+// computed in two steps: partial sums over this forward's tokens, then the
+// statistics from (local, or all-reduced across data-parallel ranks) sums.
 #include "moe_common.cuh"
 #include "moe_kernels.cuh"
 
@@ -21,9 +22,14 @@ __device__ __forceinline__ float warp_sum(float v) {
     return v;
 }
 
-// One warp per expert: P_i from the per-chunk partial sums, f_i, and the
-// attributed loss over the expert's kept rows (ascending row = ascending token).
-__global__ void __launch_bounds__(256) stats_expert_kernel(StatsArgs a) {
+// Partial sums (additive over token shards), layout of moe_stat_partials:
+//   [0, E)       sum_t P[t][e]          [E, 2E)      selections before the cap
+//   [2E]         sum_t lse_t^2          [2E+1]       T
+//   [2E+2]       dropped assignments    [2E+3, 3E+3) sum over kept assignments
+//                                                    of credit * token_loss
+// One warp per expert; every sum has a fixed order (lane-strided, then a fixed
+// shuffle tree), so repeated runs give bit-identical results.
+__global__ void __launch_bounds__(256) stat_partials_expert_kernel(StatsArgs a) {
     const int e = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
     if (e >= a.E) return;
     float ps = 0.f;
@@ -39,18 +45,13 @@ __global__ void __launch_bounds__(256) stats_expert_kernel(StatsArgs a) {
         el = warp_sum(el);
     }
     if (lane == 0) {
-        const float pm = ps / (float)a.T;
-        const float f = (float)((double)a.count_pre[e] / ((double)a.k * (double)a.T));
-        a.p_mean_ws[e] = pm;
-        a.f_ws[e] = f;
-        if (a.p_mean) a.p_mean[e] = pm;
-        if (a.f) a.f[e] = f;
-        if (a.expert_loss && a.token_loss) a.expert_loss[e] = el / (float)a.T;
+        a.partials[e] = ps;
+        a.partials[a.E + e] = (float)a.count_pre[e];
+        a.partials[2 * a.E + 3 + e] = el;
     }
 }
 
-// Single CTA: z-loss over tokens, L_aux over experts, dropped count.
-__global__ void __launch_bounds__(256) stats_scalar_kernel(StatsArgs a) {
+__global__ void __launch_bounds__(256) stat_partials_scalar_kernel(StatsArgs a) {
     __shared__ float red[8];
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     float z = 0.f;
@@ -58,12 +59,33 @@ __global__ void __launch_bounds__(256) stats_scalar_kernel(StatsArgs a) {
     z = warp_sum(z);
     if (lane == 0) red[warp] = z;
     __syncthreads();
-    float zt = 0.f;
-    if (tid == 0)
+    if (tid == 0) {
+        float zt = 0.f;
         for (int w = 0; w < 8; ++w) zt += red[w];
-    __syncthreads();
+        a.partials[2 * a.E] = zt;
+        a.partials[2 * a.E + 1] = (float)a.T;
+        a.partials[2 * a.E + 2] = (float)a.ctrl[kCtrlDropped];
+    }
+}
+
+// Statistics from (possibly all-reduced) partial sums: f_i = count_i / (k T),
+// P_i = sum_t P / T, L_aux = alpha E sum_i f_i P_i, L_z = beta sum lse^2 / T,
+// l_i = sum credit * loss / T. One CTA; the L_aux sum is a fixed tree.
+__global__ void __launch_bounds__(256) stats_finalize_kernel(FinalizeArgs a) {
+    __shared__ float red[8];
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const float T = a.partials[2 * a.E + 1];
+    const float inv_t = T > 0.f ? 1.f / T : 0.f;
+    const float inv_kt = T > 0.f ? 1.f / ((float)a.k * T) : 0.f;
     float fp = 0.f;
-    for (int e = tid; e < a.E; e += 256) fp = fmaf(a.f_ws[e], a.p_mean_ws[e], fp);
+    for (int e = tid; e < a.E; e += 256) {
+        const float pm = a.partials[e] * inv_t;
+        const float f = a.partials[a.E + e] * inv_kt;
+        if (a.p_mean) a.p_mean[e] = pm;
+        if (a.f) a.f[e] = f;
+        if (a.expert_loss) a.expert_loss[e] = a.partials[2 * a.E + 3 + e] * inv_t;
+        fp = fmaf(f, pm, fp);
+    }
     fp = warp_sum(fp);
     if (lane == 0) red[warp] = fp;
     __syncthreads();
@@ -71,18 +93,23 @@ __global__ void __launch_bounds__(256) stats_scalar_kernel(StatsArgs a) {
         float ft = 0.f;
         for (int w = 0; w < 8; ++w) ft += red[w];
         if (a.l_aux) *a.l_aux = a.alpha * (float)a.E * ft;
-        if (a.l_z) *a.l_z = a.beta * zt / (float)a.T;
-        if (a.n_dropped) *a.n_dropped = a.ctrl[kCtrlDropped];
+        if (a.l_z) *a.l_z = a.beta * a.partials[2 * a.E] * inv_t;
+        if (a.n_dropped) *a.n_dropped = (int32_t)a.partials[2 * a.E + 2];
     }
 }
 
 }  // namespace
 
-cudaError_t launch_stats(const StatsArgs &a, cudaStream_t s, int *launches) {
-    if (a.T <= 0) return cudaSuccess;
-    stats_expert_kernel<<<(a.E * 32 + 255) / 256, 256, 0, s>>>(a);
-    stats_scalar_kernel<<<1, 256, 0, s>>>(a);
+cudaError_t launch_stat_partials(const StatsArgs &a, cudaStream_t s, int *launches) {
+    stat_partials_expert_kernel<<<(a.E * 32 + 255) / 256, 256, 0, s>>>(a);
+    stat_partials_scalar_kernel<<<1, 256, 0, s>>>(a);
     *launches += 2;
+    return cudaGetLastError();
+}
+
+cudaError_t launch_stats_finalize(const FinalizeArgs &a, cudaStream_t s, int *launches) {
+    stats_finalize_kernel<<<1, 256, 0, s>>>(a);
+    *launches += 1;
     return cudaGetLastError();
 }
 

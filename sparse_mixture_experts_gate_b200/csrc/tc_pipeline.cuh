@@ -141,15 +141,17 @@ __device__ __forceinline__ void tc_producer(const TcShared<BN> &s, int total, in
     tc_producer_range<BN>(s, total, status, tile_begin, load, [&](int) { return make_int2(0, kblocks); });
 }
 
-// MMA role, one lane of warp 1.
-template <int BN>
+// MMA role, one lane of warp 1. `ncols(tile)` is the tile's N (a multiple of
+// 16, at most BN): a narrower last tile multiplies only the first rows of the
+// staged B box.
+template <int BN, class NCols>
 __device__ __forceinline__ void tc_mma(const TcShared<BN> &s, uint32_t tmem_base, int total, int kblocks,
-                                       uint32_t *status) {
+                                       uint32_t *status, NCols ncols) {
     using L = TcLayout<BN>;
-    constexpr uint32_t idesc = idesc_bf16_f32(kBM, BN);
     uint32_t it = 0, tcount = 0;
     bool ok = true;
     for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x, ++tcount) {
+        const uint32_t idesc = idesc_bf16_f32(kBM, ncols(tile));
         const uint32_t acc = tcount & 1u, use = tcount >> 1;
         if (!mbar_wait(&s.tempty[acc], (use & 1u) ^ 1u, status)) break;
         tc_fence_after_sync();

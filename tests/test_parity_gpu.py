@@ -50,7 +50,8 @@ def test_default_full():
 
 
 def test_e64_shape_small():
-    """Fine-grained experts (F=1408 -> N tile 176), a shared expert, selection bias."""
+    """Fine-grained experts (F=1408: five 256-column N tiles and a 128-column one),
+    a shared expert, selection bias."""
     w = WORKLOADS["e64"].with_(T=700)
     g, _ = full_check(w, make_inputs(w, "cpu", seed=3))
     assert g["n_dropped"][0] > 0  # C_f = 1.25 at T=700 binds for some experts
@@ -179,3 +180,70 @@ def test_e64_full_size_sampled():
 
 def test_e256_full_size_sampled():
     _sampled_full("e256", 24)
+
+
+# ------------------------------------------------- data-parallel statistics
+
+def test_dp_stats_two_shards_through_kernels():
+    """Two shards of one batch run in turn through the same layer; their
+    partial sums (moe_stat_partials), added, give through
+    moe_stats_from_partials the statistics of the whole batch: f, P, L_aux and
+    L_z of the concatenated routing, drops and attributed loss of each shard's
+    own dispatch divided by the whole batch size."""
+    from sparse_mixture_experts_gate_b200.binding import (MoeStats, moe_stat_partials, moe_stats_from_partials,
+                                                          stat_partials_size)
+    w = WORKLOADS["e64"].with_(T=1100, token_loss=True)
+    inp = make_inputs(w, "cpu", seed=21)
+    cuts = [0, 389, w.T]
+    layer = MoELayer(w, {k: inp[k] for k in ("w_gate", "b_gate", "sel_bias", "w1", "b1", "w2", "b2")})
+    total = torch.zeros(stat_partials_size(w.E), dtype=torch.float32, device="cuda")
+    shards = []
+    s = torch.cuda.current_stream().cuda_stream
+    for lo, hi in zip(cuts[:-1], cuts[1:]):
+        sub = {k: (v[lo:hi] if (v is not None and k in ("x", "noise", "token_loss")) else v) for k, v in inp.items()}
+        g, _ = run_gpu(w.with_(T=hi - lo), sub, layer=layer)
+        part = torch.full((stat_partials_size(w.E),), float("nan"), device="cuda")
+        tl = sub["token_loss"].cuda().contiguous()
+        moe_stat_partials(layer.handle, tl.data_ptr(), part.data_ptr(), s)
+        total += part
+        shards.append(g)
+    out = layer.alloc_outputs(1)
+    for v in out.values():
+        v.fill_(-7)
+    st = MoeStats(out["f"].data_ptr(), out["p_mean"].data_ptr(), out["l_aux"].data_ptr(), out["l_z"].data_ptr(),
+                  out["n_dropped"].data_ptr(), None, out["expert_loss"].data_ptr())
+    moe_stats_from_partials(layer.handle, total.data_ptr(), True, st, s)
+    torch.cuda.synchronize()
+    dp = {k: out[k].cpu().numpy().astype(np.float64) for k in ("f", "p_mean", "l_aux", "l_z", "n_dropped",
+                                                               "expert_loss")}
+
+    # Same-logits oracle routing of the whole batch from the GPU's logits.
+    logits = np.concatenate([g["logits"] for g in shards]).astype(np.float32)
+    r = oracle.routing_from_logits(logits, w, noise=None, sel_bias=inp["sel_bias"])
+    f, pm, la, lz = oracle.balance_stats(r["P"], r["lse"], r["count_pre"], w.k, w.alpha, w.beta)
+    assert np.abs(dp["f"] - f).max() <= 1e-4
+    assert np.abs(dp["p_mean"] - pm).max() <= 1e-4
+    assert abs(dp["l_aux"][0] - la) <= 1e-4
+    assert abs(dp["l_z"][0] - lz) <= 1e-4
+    assert int(dp["n_dropped"][0]) == sum(int(g["n_dropped"][0]) for g in shards)
+    el = oracle.expert_loss(np.concatenate([g["topk_idx"] for g in shards]),
+                            np.concatenate([g["slot"] for g in shards]),
+                            np.concatenate([g["credit"] for g in shards]), inp["token_loss"], w.E)
+    assert (np.abs(dp["expert_loss"] - el) / (1 + np.abs(el))).max() <= 1e-4
+    # The one-rank helper equals moe_aux_stats on the last shard alone.
+    g_last = shards[-1]
+    out1 = layer.alloc_outputs(cuts[2] - cuts[1])
+    layer.forward(inp["x"][cuts[1]:].cuda().contiguous(), out=out1)
+    layer.dp_aux_stats(out1, token_loss=inp["token_loss"][cuts[1]:].cuda().contiguous())
+    torch.cuda.synchronize()
+    assert np.array_equal(out1["f"].cpu().numpy(), g_last["f"].astype(np.float32))
+    assert np.array_equal(out1["l_aux"].cpu().numpy(), g_last["l_aux"].astype(np.float32))
+    assert np.array_equal(out1["expert_loss"].cpu().numpy(), g_last["expert_loss"].astype(np.float32))
+
+
+def test_ragged_n_tiles_both_layers():
+    """Expert widths that are not multiples of the 256-column N tile: layer 1
+    ends with a 64-column tile (F = 1088), layer 2 with a 64-column tile that
+    also carries the credit's norm partials (O = 320)."""
+    w = WORKLOADS["default"].with_(T=777, F=1088, O=320, S=1, activation="swish")
+    full_check(w, make_inputs(w, "cpu", seed=13, random_biases=True))
