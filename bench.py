@@ -312,7 +312,12 @@ def run_ours(args):
     es = 2 if w.dtype == "bf16" else 4
     touched = int((out["count_kept"] > 0).sum().item()) + w.S
     bytes_min = T * w.d * es + w.E * w.d * 4 + touched * (w.F * w.d + w.O * w.F) * es + T * w.O * es + T * w.k * 12
-    layer_frac = max(layer_flops / (peaks["bf16"] * 1e12), bytes_min / (peaks["hbm_gbs"] * 1e9)) / (ms_step / 1e3)
+    # Ideal layer time: the slower of the expert-GEMM FLOPs at the bf16 tensor peak and the algorithmic
+    # bytes at the HBM peak. Steps run back to back hold the GPU at its power cap, so the sustained
+    # tensor peak is the denominator; the burst-peak figure is reported beside it.
+    t_bytes = bytes_min / (peaks["hbm_gbs"] * 1e9)
+    layer_frac = max(layer_flops / (peaks["bf16_sustained"] * 1e12), t_bytes) / (ms_step / 1e3)
+    layer_frac_burst = max(layer_flops / (peaks["bf16"] * 1e12), t_bytes) / (ms_step / 1e3)
 
     cpu = None
     if not args.no_cpu_baseline and world == 1:
@@ -332,7 +337,8 @@ def run_ours(args):
                    "l2": l2_note(w)},
         "expert_gemm_tflops": step_tflops,
         "layer_roofline_frac": layer_frac,
-        "roofline": {"kernel": "grouped_gemm_tc (expert GEMM 1 + 2)", "bound": "tensor", "achieved": achieved,
+        "layer_roofline_frac_burst_peak": layer_frac_burst,
+        "roofline": {"kernel": "grouped_gemm_pair (expert GEMM 1 + 2)", "bound": "tensor", "achieved": achieved,
                      "peak": peaks["bf16_sustained"], "unit": "TFLOP/s", "frac": achieved / peaks["bf16_sustained"],
                      "peak_kind": f"bf16 sustained ({peaks['source']})", "traffic": traffic},
         "stage_ms": {n: statistics.mean(v) for n, v in stage.items()},
@@ -357,8 +363,8 @@ def committed_traffic(w):
     """DRAM bytes per expert-GEMM launch pair from the committed ncu summary, if
     the kernel source has not changed since it was captured."""
     import hashlib
-    path = os.path.join(ROOT, "profiles", f"grouped_gemm_tc_{w.name}_traffic.txt")
-    src = os.path.join(ROOT, "sparse_mixture_experts_gate_b200", "csrc", "gemm_tc.cu")
+    path = os.path.join(ROOT, "profiles", f"grouped_gemm_pair_{w.name}_traffic.txt")
+    src = os.path.join(ROOT, "sparse_mixture_experts_gate_b200", "csrc", "gemm_pair.cu")
     if not os.path.exists(path):
         return None
     sha = hashlib.sha256(open(src, "rb").read()).hexdigest()

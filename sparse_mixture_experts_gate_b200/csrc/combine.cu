@@ -5,30 +5,33 @@
 // combine tensor is the gate-weighted un-scatter ("Capacity & communication"),
 // and shared experts are always on ("Parameter accounting"; weight 1 here).
 // "Sparse MoE Expert-Credit Loss Reweighting Diagram", panel (b): the credit
-// c = p ||h||_2, here the applied gate times the norm of the expert's output.
+// c = p ||h||_2, here the applied gate times the norm of the expert's output
+// row as the layer stores it (the same values the combine reads).
 //
 //   y[t] = sum_{s < S} O[shared row of t] + sum_{r < k, kept} g[t][r] O[row(t, r)]
 //
 // in fp32, in exactly that order (shared experts first, then r ascending), so
-// the result does not depend on scheduling. One CTA per token; 16-byte vector
-// loads of the expert-output rows; dropped assignments contribute nothing.
+// the result does not depend on scheduling. One warp per token; 16-byte vector
+// loads of the expert-output rows; dropped assignments contribute nothing. The
+// squared norms are summed from the same loads (per lane in column order, then
+// a fixed shuffle tree).
 #include "moe_common.cuh"
 #include "moe_kernels.cuh"
 
 namespace moe {
 namespace {
 
-constexpr int kThreads = 128;
-constexpr int kMaxK = 16;
+constexpr int kWarps = 8;  // tokens per block, one warp each
 constexpr int kMaxS = 4;
+constexpr int kBatch = 8;  // routed-term loads issued together
 
+// 16-byte vectors of expert-output elements: raw load, then unpack to fp32.
 template <typename T>
 struct Vec;
 template <>
 struct Vec<__nv_bfloat16> {
     static constexpr int N = 8;  // 8 bf16 per 16 bytes
-    __device__ static void load(const __nv_bfloat16 *p, float (&v)[8]) {
-        const uint4 u = __ldg(reinterpret_cast<const uint4 *>(p));
+    __device__ static void unpack(const uint4 &u, float (&v)[8]) {
         const __nv_bfloat162 *h = reinterpret_cast<const __nv_bfloat162 *>(&u);
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
@@ -48,12 +51,11 @@ struct Vec<__nv_bfloat16> {
 template <>
 struct Vec<float> {
     static constexpr int N = 4;
-    __device__ static void load(const float *p, float (&v)[4]) {
-        const float4 u = __ldg(reinterpret_cast<const float4 *>(p));
-        v[0] = u.x;
-        v[1] = u.y;
-        v[2] = u.z;
-        v[3] = u.w;
+    __device__ static void unpack(const uint4 &u, float (&v)[4]) {
+        v[0] = __uint_as_float(u.x);
+        v[1] = __uint_as_float(u.y);
+        v[2] = __uint_as_float(u.z);
+        v[3] = __uint_as_float(u.w);
     }
     __device__ static void store(float *p, const float (&v)[4]) {
         *reinterpret_cast<float4 *>(p) = make_float4(v[0], v[1], v[2], v[3]);
@@ -61,66 +63,115 @@ struct Vec<float> {
 };
 
 template <typename T>
-__global__ void __launch_bounds__(kThreads) combine_kernel(CombineArgs a) {
+__device__ __forceinline__ uint4 load_raw(const T *p) {
+    return __ldg(reinterpret_cast<const uint4 *>(p));
+}
+
+// NB: batches of eight routed terms the kernel is built for (k <= 8 NB).
+template <typename T, int NB>
+__global__ void __launch_bounds__(kWarps * 32, 2) combine_kernel(CombineArgs a) {
     constexpr int V = Vec<T>::N;
-    __shared__ int s_row[kMaxK + kMaxS];
-    __shared__ float s_g[kMaxK + kMaxS];
-    const int t = blockIdx.x;
-    const int nsh = a.S;
-    const int tid = threadIdx.x;
-    if (tid < nsh) {
-        s_row[tid] = a.group_start[a.E + tid] + t;
-        s_g[tid] = 1.f;
-    } else if (tid < nsh + a.k) {
-        const int r = tid - nsh;
-        const int64_t ai = (int64_t)t * a.k + r;
-        const int row = a.row_of[ai];
-        const float g = a.gates[ai];
-        s_row[tid] = row;
-        s_g[tid] = g;
-        // Credit of this assignment: gate times the norm of the expert output.
-        float c = 0.f;
-        if (row >= 0) {
-            float ss = 0.f;
-            for (int j = 0; j < a.n_parts; ++j) ss += a.norm_part[(int64_t)row * a.n_parts + j];
-            c = g * sqrtf(ss);
-        }
-        a.credit[ai] = c;
+    constexpr int kMaxK = NB * kBatch;
+    const int lane = threadIdx.x & 31;
+    const int t = blockIdx.x * kWarps + (threadIdx.x >> 5);
+    if (t >= a.T) return;
+    const int nsh = a.S, k = a.k;
+    int my_row = -1;
+    float my_g = 0.f;
+    if (lane < k) {
+        my_row = a.row_of[(int64_t)t * k + lane];
+        my_g = a.gates[(int64_t)t * k + lane];
     }
-    __syncthreads();
+    int srow[kMaxS], rrow[kMaxK];
+    float rg[kMaxK];
+#pragma unroll
+    for (int i = 0; i < kMaxS; ++i) srow[i] = i < nsh ? a.group_start[a.E + i] + t : -1;
+#pragma unroll
+    for (int r = 0; r < kMaxK; ++r) {  // lanes >= k hold row -1
+        rrow[r] = __shfl_sync(0xffffffffu, my_row, r);
+        rg[r] = __shfl_sync(0xffffffffu, my_g, r);
+    }
     const T *o = static_cast<const T *>(a.o);
     T *y = static_cast<T *>(a.y) + (int64_t)t * a.O;
-    const int nterm = nsh + a.k;
-    for (int c = tid * V; c < a.O; c += kThreads * V) {
+    // Per routed term, this lane's part of ||o||^2.
+    float ss[kMaxK];
+#pragma unroll
+    for (int r = 0; r < kMaxK; ++r) ss[r] = 0.f;
+    for (int c = lane * V; c < a.O; c += 32 * V) {
+        // Every term's vector (shared terms and the first eight routed terms)
+        // is requested before any is used, so a lane has them all in flight.
+        uint4 us[kMaxS], ur[kBatch];
+#pragma unroll
+        for (int i = 0; i < kMaxS; ++i)
+            if (srow[i] >= 0) us[i] = load_raw(o + (int64_t)srow[i] * a.O + c);
+#pragma unroll
+        for (int i = 0; i < kBatch; ++i)
+            if (rrow[i] >= 0) ur[i] = load_raw(o + (int64_t)rrow[i] * a.O + c);
         float acc[V];
 #pragma unroll
         for (int j = 0; j < V; ++j) acc[j] = 0.f;
-        for (int i = 0; i < nterm; ++i) {
-            const int row = s_row[i];
-            if (row < 0) continue;
-            const float g = s_g[i];
+#pragma unroll
+        for (int i = 0; i < kMaxS; ++i) {
+            if (srow[i] < 0) continue;
             float v[V];
-            Vec<T>::load(o + (int64_t)row * a.O + c, v);
-            if (i < nsh) {
+            Vec<T>::unpack(us[i], v);
 #pragma unroll
-                for (int j = 0; j < V; ++j) acc[j] += v[j];
-            } else {
+            for (int j = 0; j < V; ++j) acc[j] += v[j];
+        }
 #pragma unroll
-                for (int j = 0; j < V; ++j) acc[j] = fmaf(g, v[j], acc[j]);
+        for (int r0 = 0; r0 < kMaxK; r0 += kBatch) {
+            if (r0 >= k) break;
+            if (r0 > 0) {  // further batches (k > 8)
+#pragma unroll
+                for (int i = 0; i < kBatch; ++i)
+                    if (rrow[r0 + i] >= 0) ur[i] = load_raw(o + (int64_t)rrow[r0 + i] * a.O + c);
+            }
+#pragma unroll
+            for (int i = 0; i < kBatch; ++i) {
+                const int r = r0 + i;
+                if (rrow[r] < 0) continue;
+                float v[V];
+                Vec<T>::unpack(ur[i], v);
+#pragma unroll
+                for (int j = 0; j < V; ++j) {
+                    acc[j] = fmaf(rg[r], v[j], acc[j]);
+                    ss[r] = fmaf(v[j], v[j], ss[r]);
+                }
             }
         }
         Vec<T>::store(y + c, acc);
     }
+    // Credit of each routed assignment: gate times the norm of the expert
+    // output row as stored (fixed shuffle tree).
+    float credit = 0.f;
+#pragma unroll
+    for (int r = 0; r < kMaxK; ++r) {
+        if (r >= k) break;
+        float v = ss[r];
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
+        if (lane == r && rrow[r] >= 0) credit = rg[r] * sqrtf(v);
+    }
+    if (lane < k) a.credit[(int64_t)t * k + lane] = credit;
 }
 
 }  // namespace
 
 cudaError_t launch_combine(const CombineArgs &a, cudaStream_t s, int *launches) {
     if (a.T <= 0) return cudaSuccess;
-    if (a.bf16)
-        combine_kernel<__nv_bfloat16><<<a.T, kThreads, 0, s>>>(a);
-    else
-        combine_kernel<float><<<a.T, kThreads, 0, s>>>(a);
+    const int blocks = (a.T + kWarps - 1) / kWarps;
+    if (a.k > 2 * kBatch) return cudaErrorInvalidValue;
+    if (a.bf16) {
+        if (a.k <= kBatch)
+            combine_kernel<__nv_bfloat16, 1><<<blocks, kWarps * 32, 0, s>>>(a);
+        else
+            combine_kernel<__nv_bfloat16, 2><<<blocks, kWarps * 32, 0, s>>>(a);
+    } else {
+        if (a.k <= kBatch)
+            combine_kernel<float, 1><<<blocks, kWarps * 32, 0, s>>>(a);
+        else
+            combine_kernel<float, 2><<<blocks, kWarps * 32, 0, s>>>(a);
+    }
     ++*launches;
     return cudaGetLastError();
 }

@@ -8,18 +8,20 @@
 //
 // Instead of a dense one-hot D, the dispatch is a permutation into a compact row
 // space: expert e owns rows [group_start[e], group_start[e] + kept_e), padded to
-// a multiple of the GEMM M tile, followed by one T-row segment per shared
-// expert. Three launches:
+// a multiple of 32 rows, followed by one T-row segment per shared expert (also
+// padded to 32). Three launches:
 //   count  - per 256-token chunk, a histogram of selections (shared-memory
 //            integer atomics: order-free, so deterministic);
 //   scan   - per expert, exclusive prefix over chunks; kept = min(count, C);
-//            exclusive scan of the padded kept counts -> segment starts, the
-//            M-tile -> group table and the row count;
+//            exclusive scans of the padded kept counts and of their token
+//            tiles -> segment starts, the 32-row block -> group table, the
+//            token-tile table of the expert GEMM ({group, first row, rows},
+//            at most 256 rows each) and the row and tile counts;
 //   assign - per chunk, the stable rank of each assignment: chunk base +
 //            assignments to the same expert in earlier warps + earlier lanes of
 //            the same warp (a per-warp lane bitmask per expert, popcounted).
 // Also the scatter of the routed token rows into the permuted row space, which
-// the tensor-core expert GEMM then reads as plain 128-row TMA tiles.
+// the tensor-core expert GEMM then reads as plain TMA tiles.
 #include "moe_common.cuh"
 #include "moe_kernels.cuh"
 
@@ -42,10 +44,11 @@ __global__ void __launch_bounds__(kChunk) dispatch_count_kernel(DispatchArgs a) 
 
 // Single CTA of kMaxE threads; thread e owns expert e.
 __global__ void __launch_bounds__(kMaxE) dispatch_scan_kernel(DispatchArgs a) {
-    __shared__ int sc[kMaxE];
+    __shared__ int sc_rows[kMaxE];
+    __shared__ int sc_tiles[kMaxE];
     __shared__ int dropped_w[kMaxE / 32];
     const int e = threadIdx.x, lane = e & 31, warp = e >> 5;
-    int pre = 0, kept = 0, padded = 0;
+    int pre = 0, kept = 0, padded = 0, tiles = 0;
     if (e < a.E) {
         // Exclusive prefix over chunks, loads batched so they are in flight together.
         const int32_t *__restrict__ cnt = a.chunk_count;
@@ -61,19 +64,24 @@ __global__ void __launch_bounds__(kMaxE) dispatch_scan_kernel(DispatchArgs a) {
             }
         }
         kept = (int64_t)pre < a.C ? pre : (int)a.C;
-        padded = (kept + kBM - 1) / kBM * kBM;
+        padded = (kept + kRowBlock - 1) / kRowBlock * kRowBlock;
+        tiles = (padded + kTokTile - 1) / kTokTile;
     }
-    // Inclusive scan of padded over the block (Hillis-Steele in shared memory).
-    sc[e] = padded;
+    // Inclusive scans of the padded rows and of the token tiles over the block
+    // (Hillis-Steele in shared memory).
+    sc_rows[e] = padded;
+    sc_tiles[e] = tiles;
     __syncthreads();
     for (int off = 1; off < kMaxE; off <<= 1) {
-        const int v = e >= off ? sc[e - off] : 0;
+        const int vr = e >= off ? sc_rows[e - off] : 0;
+        const int vt = e >= off ? sc_tiles[e - off] : 0;
         __syncthreads();
-        sc[e] += v;
+        sc_rows[e] += vr;
+        sc_tiles[e] += vt;
         __syncthreads();
     }
-    const int start = sc[e] - padded;
-    const int routed_rows = sc[kMaxE - 1];
+    const int start = sc_rows[e] - padded, tile0 = sc_tiles[e] - tiles;
+    const int routed_rows = sc_rows[kMaxE - 1], routed_tiles = sc_tiles[kMaxE - 1];
     int drop = pre - kept;
     for (int off = 16; off > 0; off >>= 1) drop += __shfl_xor_sync(0xffffffffu, drop, off);
     if (lane == 0) dropped_w[warp] = drop;
@@ -84,12 +92,21 @@ __global__ void __launch_bounds__(kMaxE) dispatch_scan_kernel(DispatchArgs a) {
         if (a.user_count_kept) a.user_count_kept[e] = kept;
         a.group_start[e] = start;
         a.group_rows[e] = kept;
-        for (int m = start / kBM; m < (start + padded) / kBM; ++m) a.tile_group[m] = e;
+        for (int b = start / kRowBlock; b < (start + padded) / kRowBlock; ++b) a.block_group[b] = e;
         for (int r = start + kept; r < start + padded; ++r) a.row_assign[r] = -1;
+        for (int i = 0; i < tiles; ++i)
+            a.tok_tiles[tile0 + i] = make_int4(e, start + i * kTokTile, min(kTokTile, padded - i * kTokTile), 0);
     }
     // Shared experts: one T_pad-row segment each, after the routed rows.
-    const int shared_tiles = a.T_pad / kBM;
-    for (int i = e; i < a.S * shared_tiles; i += kMaxE) a.tile_group[routed_rows / kBM + i] = a.E + i / shared_tiles;
+    const int shared_blocks = a.T_pad / kRowBlock;
+    const int shared_tiles = (a.T_pad + kTokTile - 1) / kTokTile;
+    for (int i = e; i < a.S * shared_blocks; i += kMaxE)
+        a.block_group[routed_rows / kRowBlock + i] = a.E + i / shared_blocks;
+    for (int i = e; i < a.S * shared_tiles; i += kMaxE) {
+        const int sh = i / shared_tiles, j = i - sh * shared_tiles;
+        a.tok_tiles[routed_tiles + i] = make_int4(a.E + sh, routed_rows + sh * a.T_pad + j * kTokTile,
+                                                  min(kTokTile, a.T_pad - j * kTokTile), 0);
+    }
     if (e < a.S) {
         a.group_start[a.E + e] = routed_rows + e * a.T_pad;
         a.group_rows[a.E + e] = a.T;
@@ -100,7 +117,8 @@ __global__ void __launch_bounds__(kMaxE) dispatch_scan_kernel(DispatchArgs a) {
         for (int w = 0; w < kMaxE / 32; ++w) d += dropped_w[w];
         const int total = routed_rows + a.S * a.T_pad;
         a.group_start[a.E + a.S] = total;
-        a.ctrl[kCtrlNumMTiles] = total / kBM;
+        a.ctrl[kCtrlNumRowBlocks] = total / kRowBlock;
+        a.ctrl[kCtrlNumTokTiles] = routed_tiles + a.S * shared_tiles;
         a.ctrl[kCtrlRoutedRows] = routed_rows;
         a.ctrl[kCtrlDropped] = d;
     }

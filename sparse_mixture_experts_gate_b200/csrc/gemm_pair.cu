@@ -1,0 +1,319 @@
+// gemm_pair.cu - grouped expert GEMM on CTA pairs (sm_100a tcgen05 cta_group::2).
+//
+// "Code Walkthrough - SER", gating / routing path: each selected expert runs its
+// two-layer MLP, w1/b1 -> activation -> w2/b2, on the rows dispatched to it;
+// shared experts ("Appendix C - Acronyms & Symbols", "Parameter accounting")
+// run the same MLP on every token. Both layers of every expert are dense
+// contractions, computed here as one grouped GEMM per layer over the permuted
+// row space:
+//   out[row][f] = act( sum_k A[row][k] W[g][f][k] + b[g][f] ),  g = group of row.
+// Layer 1: A = the routed token rows scattered into row order (dispatch.cu), or
+// x itself for the shared experts, which read every token in order.
+// Layer 2: A = the hidden activations H (already in row order).
+//
+// Operand roles. The tensor cores compute out^T: the MMA's M side is 256 output
+// features (weights W[g], 128 per CTA of the pair) and its N side is a token
+// tile of up to 256 rows of one expert. Each expert's rows are padded only to a
+// multiple of 32 (the row space's block), instead of to the M extent, and the
+// weight tile, the operand every token of the expert shares, is split across
+// the pair so that each SM stages half of it.
+//
+// Per CTA (192 threads): warp 0 loads (TMA, signalling the leader's stage
+// barrier, which expects both CTAs' bytes), warp 1 owns TMEM (2 accumulators x
+// 256 columns) and, in the leader, issues the pair MMAs and commits stages and
+// accumulators to both CTAs at once; warps 2..5 drain this CTA's 128 features:
+// each warp reads 32 features x 32 tokens from TMEM, adds the bias, applies the
+// activation, writes them transposed (token-major, bf16) to a shared staging box
+// and stores the box with a TMA tensor store. The epilogue releases an
+// accumulator by arriving on the leader's barrier (8 warps per tile).
+//
+// Every wait is bounded (mbar_wait); on a timeout the roles stop, the leader
+// drains its MMAs, copies in flight are given time to land, both CTAs meet at
+// the cluster barrier, and TMEM is freed.
+#include "moe_common.cuh"
+#include "moe_kernels.cuh"
+
+namespace moe {
+namespace {
+
+constexpr int kThreads = 192;
+constexpr int kFeatPair = 256;                     // MMA M: features per pair tile
+constexpr int kFeatCta = 128;                      // features per CTA
+constexpr int kABytes = kFeatCta * kBK * 2;        // 16 KB: 128 weight rows x 64 K
+constexpr int kBBytes = (kTokTile / 2) * kBK * 2;  // 16 KB: up to 128 token rows x 64 K
+constexpr int kStage = kABytes + kBBytes;
+constexpr int kStages = 6;
+constexpr int kAccCols = 256;
+constexpr int kBoxTok = 32, kBoxFeat = 32;          // store box: 32 tokens x 32 features
+constexpr int kBoxBytes = kBoxTok * kBoxFeat * 2;
+constexpr int kStaging = 4 * 2 * kBoxBytes;         // 4 epilogue warps x 2 boxes
+constexpr int kRowsPerLoad16 = 16;                  // rows of the narrow token box
+constexpr int kSmem = 1024 + kStages * kStage + kStaging + 256;
+static_assert(kSmem <= 232448, "exceeds the 227 KB of shared memory a CTA may use");
+static_assert(kTokTile == 256 && kTokTile % (2 * kRowsPerLoad16) == 0, "token tile layout");
+
+struct Smem {
+    uint8_t *sA, *sB, *staging;
+    uint64_t *full, *empty, *tfull, *tempty, *mma_done;
+    uint32_t *tmem_slot;
+};
+
+__device__ __forceinline__ Smem carve(uint8_t *raw) {
+    uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(raw) + 1023) & ~uintptr_t(1023));
+    Smem s;
+    s.sA = base;
+    s.sB = base + kStages * kABytes;
+    s.staging = base + kStages * kStage;
+    s.full = reinterpret_cast<uint64_t *>(s.staging + kStaging);
+    s.empty = s.full + kStages;
+    s.tfull = s.empty + kStages;
+    s.tempty = s.tfull + 2;
+    s.mma_done = s.tempty + 2;
+    s.tmem_slot = reinterpret_cast<uint32_t *>(s.mma_done + 1);
+    return s;
+}
+
+template <int ACT>
+__global__ void __launch_bounds__(kThreads, 1)
+    grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap map_w, const __grid_constant__ CUtensorMap map_t,
+                             const __grid_constant__ CUtensorMap map_t16, const __grid_constant__ CUtensorMap map_s,
+                             const __grid_constant__ CUtensorMap map_s16, const __grid_constant__ CUtensorMap map_out,
+                             const PairGemmArgs a) {
+    extern __shared__ uint8_t smem_raw[];
+    const Smem s = carve(smem_raw);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t rank = cluster_ctarank();
+    const bool leader = rank == 0;
+    const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
+
+    if (threadIdx.x == 0) {
+        tma_prefetch_desc(&map_w);
+        tma_prefetch_desc(&map_t);
+        tma_prefetch_desc(&map_t16);
+        tma_prefetch_desc(&map_s);
+        tma_prefetch_desc(&map_s16);
+        tma_prefetch_desc(&map_out);
+        for (int i = 0; i < kStages; ++i) {
+            mbar_init(&s.full[i], 1);
+            mbar_init(&s.empty[i], 1);
+        }
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&s.tfull[i], 1);
+            mbar_init(&s.tempty[i], 8);  // 4 epilogue warps in each CTA
+        }
+        mbar_init(s.mma_done, 1);
+        fence_barrier_init();
+    }
+    if (warp == 1) {
+        tmem_alloc_pair(s.tmem_slot, 2 * kAccCols);
+        tmem_relinquish_pair();
+    }
+    tc_fence_before_sync();
+    cluster_sync_all();  // barriers of both CTAs initialised, TMEM allocated in both
+    tc_fence_after_sync();
+    const uint32_t tmem_base = *s.tmem_slot;
+
+    const int n_tt = min(a.ctrl[kCtrlNumTokTiles], a.max_tok_tiles);
+    const int total = n_tt * a.n_ftiles;
+    const int kblocks = a.K / kBK;
+    bool ok = true;
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ producer
+        uint32_t it = 0;
+        for (int u = pair; u < total && ok; u += npairs) {
+            const int tt = u / a.n_ftiles, j = u - tt * a.n_ftiles;
+            const int4 tile = a.tok_tiles[tt];  // {group, first row, rows, -}
+            const int g = tile.x, ntok = tile.z;
+            const CUtensorMap *mt = &map_t, *mt16 = &map_t16;
+            int trow = tile.y + static_cast<int>(rank) * (ntok / 2);
+            if (a.use_s && g >= a.E) {  // shared expert: rows of x in token order
+                mt = &map_s;
+                mt16 = &map_s16;
+                trow -= a.group_start[g];
+            }
+            const int wrow = g * a.N + j * kFeatPair + static_cast<int>(rank) * kFeatCta;
+            const uint32_t tx_bytes = 2u * kABytes + static_cast<uint32_t>(ntok) * kBK * 2u;
+            const int n16 = ntok / (2 * kRowsPerLoad16);
+            for (int kb = 0; kb < kblocks; ++kb, ++it) {
+                const int st = it % kStages;
+                const uint32_t ph = (it / kStages) & 1u;
+                int got = 1;
+                if (lane == 0) got = mbar_wait(&s.empty[st], ph ^ 1u, a.status) ? 1 : 0;
+                got = __shfl_sync(0xffffffffu, got, 0);
+                if (!got) {
+                    ok = false;
+                    break;
+                }
+                if (lane == 0 && leader) mbar_arrive_expect_tx(&s.full[st], tx_bytes);
+                __syncwarp();
+                const uint32_t bar = mapa_shared(smem_u32(&s.full[st]), 0);
+                uint8_t *sA = s.sA + st * kABytes, *sB = s.sB + st * kBBytes;
+                if (lane == 0) tma_load_2d_pair(&map_w, bar, sA, kb * kBK, wrow);
+                if (ntok == kTokTile) {
+                    if (lane == 1) tma_load_2d_pair(mt, bar, sB, kb * kBK, trow);
+                } else if (lane < n16) {
+                    tma_load_2d_pair(mt16, bar, sB + lane * kRowsPerLoad16 * 128, kb * kBK,
+                                     trow + lane * kRowsPerLoad16);
+                }
+            }
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ MMA (leader)
+        if (leader && lane == 0) {
+            uint32_t it = 0, tcount = 0;
+            for (int u = pair; u < total && ok; u += npairs, ++tcount) {
+                const int ntok = a.tok_tiles[u / a.n_ftiles].z;
+                const uint32_t idesc = idesc_bf16_f32(kFeatPair, ntok);
+                const uint32_t acc = tcount & 1u, use = tcount >> 1;
+                if (!mbar_wait(&s.tempty[acc], (use & 1u) ^ 1u, a.status)) break;
+                tc_fence_after_sync();
+                const uint32_t d_tmem = tmem_base + acc * kAccCols;
+                for (int kb = 0; kb < kblocks; ++kb, ++it) {
+                    const int st = it % kStages;
+                    const uint32_t ph = (it / kStages) & 1u;
+                    if (!mbar_wait(&s.full[st], ph, a.status)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after_sync();
+                    const uint64_t ad = sw128_kmajor_desc(smem_u32(s.sA + st * kABytes));
+                    const uint64_t bd = sw128_kmajor_desc(smem_u32(s.sB + st * kBBytes));
+#pragma unroll
+                    for (int kk = 0; kk < kBK / 16; ++kk)
+                        tc_mma_bf16_pair(d_tmem, ad + 2u * kk, bd + 2u * kk, idesc, (kb | kk) != 0 ? 1u : 0u);
+                    tc_commit_pair_mc(&s.empty[st], 0x3);
+                }
+                if (ok) tc_commit_pair_mc(&s.tfull[acc], 0x3);
+            }
+            tc_commit_pair(s.mma_done);
+            mbar_wait_drain(s.mma_done, 0u);
+        }
+    } else {
+        // ------------------------------------------------------------ epilogue
+        const int q = warp & 3;  // TMEM lane quarter this warp may access
+        uint8_t *my_stage = s.staging + (warp - 2) * 2 * kBoxBytes;
+        uint32_t sub = 0, tcount = 0;
+        for (int u = pair; u < total; u += npairs, ++tcount) {
+            const int tt = u / a.n_ftiles, j = u - tt * a.n_ftiles;
+            const int4 tile = a.tok_tiles[tt];
+            const int g = tile.x, row0 = tile.y, ntok = tile.z;
+            const int fcol = j * kFeatPair + static_cast<int>(rank) * kFeatCta + q * 32;
+            const uint32_t acc = tcount & 1u, use = tcount >> 1;
+            int got = 1;  // one lane waits; tcgen05.ld below is warp-collective
+            if (lane == 0) got = mbar_wait_idle(&s.tfull[acc], use & 1u, a.status) ? 1 : 0;
+            if (!__shfl_sync(0xffffffffu, got, 0)) break;
+            tc_fence_after_sync();
+            if (fcol < a.N) {  // the last feature tile of a ragged N has an idle half
+                const float b = a.bias ? __ldg(a.bias + (int64_t)g * a.N + fcol + lane) : 0.f;
+                const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * kAccCols;
+#pragma unroll 1
+                for (int c = 0; c < ntok; c += kBoxTok) {
+                    uint8_t *buf = my_stage + (sub & 1u) * kBoxBytes;
+                    if (lane == 0) bulk_wait_group_read<1>();  // the store that last used `buf` has read it
+                    __syncwarp();
+                    uint32_t r[32];
+                    tmem_ld_32x32b_x32(taddr + c, r);
+                    tmem_ld_wait();
+                    // Lane = feature, register = token; the box is token-major
+                    // (64 bytes per token). Neighbouring lanes trade one value per
+                    // token pair, so the even lane holds features (f, f+1) of
+                    // token t and the odd lane those of token t+1: one bf16x2
+                    // conversion and one 32-bit store each, the two rows in
+                    // opposite bank halves.
+                    const uint32_t odd = lane & 1u;
+                    uint32_t *words = reinterpret_cast<uint32_t *>(buf) + (lane >> 1);
+#pragma unroll
+                    for (int t = 0; t < 32; t += 2) {
+                        const float z0 = activate_t<ACT>(__uint_as_float(r[t]) + b);
+                        const float z1 = activate_t<ACT>(__uint_as_float(r[t + 1]) + b);
+                        const float other = __shfl_xor_sync(0xffffffffu, odd ? z0 : z1, 1);
+                        __nv_bfloat162 p = odd ? __floats2bfloat162_rn(other, z1) : __floats2bfloat162_rn(z0, other);
+                        words[(t + odd) * (kBoxFeat / 2)] = *reinterpret_cast<uint32_t *>(&p);
+                    }
+                    fence_proxy_async_smem();
+                    __syncwarp();
+                    if (lane == 0) {
+                        tma_store_2d(&map_out, buf, fcol, row0 + c);
+                        bulk_commit_group();
+                    }
+                    ++sub;
+                }
+            }
+            tc_fence_before_sync();
+            __syncwarp();
+            if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(&s.tempty[acc]), 0));
+        }
+        if (lane == 0) bulk_wait_group<0>();  // all stores complete before exit
+    }
+
+    // A role that gave up may leave its own TMA loads in flight; they land
+    // within microseconds, so give them a millisecond before the pair meets.
+    if (!ok || *reinterpret_cast<volatile uint32_t *>(a.status) != kDevOk) spin_ns(1000000ull);
+    tc_fence_before_sync();
+    cluster_sync_all();
+    tc_fence_after_sync();
+    if (warp == 1) {
+        __syncwarp();
+        tmem_dealloc_pair(tmem_base, 2 * kAccCols);
+    }
+}
+
+template <int ACT>
+cudaError_t launch_act(const CUtensorMap &mw, const CUtensorMap &mt, const CUtensorMap &mt16, const CUtensorMap &ms,
+                       const CUtensorMap &ms16, const CUtensorMap &mo, const PairGemmArgs &a, cudaStream_t st) {
+    auto kern = grouped_gemm_pair_kernel<ACT>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
+    if (e != cudaSuccess) return e;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(2 * a.num_pairs, 1, 1);
+    cfg.blockDim = dim3(kThreads, 1, 1);
+    cfg.dynamicSmemBytes = kSmem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, mw, mt, mt16, ms, ms16, mo, a);
+}
+
+}  // namespace
+
+int gemm_pair_max_pairs(int num_sms) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(2 * (num_sms / 2), 1, 1);
+    cfg.blockDim = dim3(kThreads, 1, 1);
+    cfg.dynamicSmemBytes = kSmem;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    auto kern = grouped_gemm_pair_kernel<-1>;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem) != cudaSuccess) return 0;
+    int clusters = 0;
+    if (cudaOccupancyMaxActiveClusters(&clusters, kern, &cfg) != cudaSuccess) return 0;
+    return clusters < num_sms / 2 ? clusters : num_sms / 2;
+}
+
+int gemm_pair_ftiles(int N) { return (N + kFeatPair - 1) / kFeatPair; }
+
+cudaError_t launch_gemm_pair(const CUtensorMap &map_w, const CUtensorMap &map_t, const CUtensorMap &map_t16,
+                             const CUtensorMap &map_s, const CUtensorMap &map_s16, const CUtensorMap &map_out,
+                             const PairGemmArgs &a, cudaStream_t s, int *launches) {
+    if (a.num_pairs <= 0) return cudaErrorInvalidConfiguration;
+    ++*launches;
+    switch (a.act) {
+        case 0: return launch_act<0>(map_w, map_t, map_t16, map_s, map_s16, map_out, a, s);
+        case 1: return launch_act<1>(map_w, map_t, map_t16, map_s, map_s16, map_out, a, s);
+        case 2: return launch_act<2>(map_w, map_t, map_t16, map_s, map_s16, map_out, a, s);
+        default: return launch_act<-1>(map_w, map_t, map_t16, map_s, map_s16, map_out, a, s);
+    }
+}
+
+}  // namespace moe

@@ -51,6 +51,8 @@ EncodeTiledFn encode_fn() {
 
 // Row-major bf16 matrix [rows][inner] read in boxes of 64 x box_rows with 128B
 // swizzle (the layout the UMMA shared-memory descriptors expect).
+// Row-major bf16 [rows][inner] operand map: box of 64 elements (128 bytes) x
+// box_rows, 128B swizzle (the UMMA K-major layout).
 bool encode_bf16_2d(CUtensorMap *m, const void *base, uint64_t inner, uint64_t rows, uint32_t box_rows) {
     EncodeTiledFn fn = encode_fn();
     if (!fn || rows == 0) return false;
@@ -63,14 +65,29 @@ bool encode_bf16_2d(CUtensorMap *m, const void *base, uint64_t inner, uint64_t r
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Row-major bf16 [rows][inner] output map for the expert GEMM's stores: box of
+// 32 x 32 elements, no swizzle.
+bool encode_bf16_store(CUtensorMap *m, const void *base, uint64_t inner, uint64_t rows) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn || rows == 0) return false;
+    cuuint64_t dims[2] = {inner, rows};
+    cuuint64_t strides[1] = {inner * 2};
+    cuuint32_t box[2] = {32, 32};
+    cuuint32_t es[2] = {1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box, es,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 struct Plan {
     int T = 0;
     int64_t C = 0;
-    int T_pad = 0, n_stat_chunks = 0, n_chunks = 0, R_routed_max = 0, R_max = 0, max_mtiles = 0;
+    int T_pad = 0, n_stat_chunks = 0, n_chunks = 0, R_routed_max = 0, R_max = 0, max_row_blocks = 0;
+    int max_tok_tiles = 0;
     int ksplit = 1;
     size_t o_lpart = 0;
     size_t o_ctrl, o_logits, o_idx, o_gates, o_slot, o_rowof, o_lse, o_psum, o_ccount, o_cbase, o_cpre, o_ckept,
-        o_gstart, o_grows, o_tgroup, o_rowassign, o_wsplit, o_xp, o_h, o_o, o_norm, o_credit, o_partials;
+        o_gstart, o_grows, o_bgroup, o_toktiles, o_rowassign, o_wsplit, o_xp, o_h, o_o, o_credit, o_partials;
     size_t total = 0;
 };
 
@@ -87,9 +104,8 @@ struct moe_layer {
     moe_weights_t w;
     int G = 0;
     bool tc = false;
-    int bn1 = 0, bn2 = 0, ntiles1 = 0, ntiles2 = 0;
-    int norm_parts = 0;  // fp32 partial sums of ||o||^2 per row (expert GEMM 2 writes them)
     int num_sms = 148;
+    int num_pairs = 0;  // co-resident 2-CTA clusters of the expert GEMM
     CUtensorMap map_w1, map_w2;
     // State of the most recent forward, read by moe_aux_stats.
     bool has_forward = false;
@@ -114,12 +130,15 @@ Plan make_plan(const moe_layer &L, int T) {
     p.C = capacity_of(c, T);
     const int E = c.num_experts, k = c.num_active, S = c.num_shared;
     const int64_t kept_max = std::min<int64_t>((int64_t)k * T, (int64_t)E * p.C);
-    const int64_t routed = std::min<int64_t>(round_up(kept_max + (int64_t)E * (kBM - 1), kBM),
-                                             (int64_t)E * round_up(p.C, kBM));
+    const int64_t routed = std::min<int64_t>(round_up(kept_max + (int64_t)E * (kRowBlock - 1), kRowBlock),
+                                             (int64_t)E * round_up(p.C, kRowBlock));
     p.R_routed_max = (int)routed;
-    p.T_pad = (int)round_up(T, kBM);
+    p.T_pad = (int)round_up(T, kRowBlock);
     p.R_max = p.R_routed_max + S * p.T_pad;
-    p.max_mtiles = p.R_max / kBM;
+    p.max_row_blocks = p.R_max / kRowBlock;
+    // Each expert's segment splits into ceil(rows / 256) token tiles of >= 32 rows.
+    p.max_tok_tiles = (int)std::min<int64_t>(routed / kTokTile + E, routed / kRowBlock) +
+                      S * (int)((p.T_pad + kTokTile - 1) / kTokTile);
     p.n_stat_chunks = router_psum_blocks(T, L.num_sms, c.dtype == MOE_DTYPE_BF16);
     p.n_chunks = (T + 255) / 256;
     const size_t es = c.dtype == MOE_DTYPE_BF16 ? 2 : 4;
@@ -143,11 +162,11 @@ Plan make_plan(const moe_layer &L, int T) {
     p.o_ckept = take((size_t)E * 4);
     p.o_gstart = take((size_t)(E + S + 1) * 4);
     p.o_grows = take((size_t)(E + S) * 4);
-    p.o_tgroup = take((size_t)p.max_mtiles * 4);
+    p.o_bgroup = take((size_t)p.max_row_blocks * 4);
+    p.o_toktiles = take((size_t)std::max(p.max_tok_tiles, 1) * 16);
     p.o_rowassign = take((size_t)p.R_max * 4);
     p.o_partials = take((size_t)(3 * E + 3) * 4);
     p.o_credit = take((size_t)T * k * 4);
-    p.o_norm = take((size_t)p.R_max * L.norm_parts * 4);
     p.o_wsplit = take(c.dtype == MOE_DTYPE_BF16 ? (size_t)router_tc_epad(E) * 3 * c.input_dim * 2 : 0);
     p.ksplit = c.dtype == MOE_DTYPE_BF16 ? router_tc_ksplit(T, E, c.input_dim, L.num_sms) : 1;
     p.o_lpart = take(p.ksplit > 1 ? (size_t)p.ksplit * T * E * 4 : 0);
@@ -257,20 +276,16 @@ int moe_layer_create(const moe_config_t *cfg, const moe_weights_t *w, moe_layer_
     L->num_sms = sms > 0 ? sms : 148;
     L->tc = cfg->dtype == MOE_DTYPE_BF16;
     if (L->tc) {
-        L->bn1 = gemm_pick_bn(cfg->expert_dim);
-        L->bn2 = gemm_pick_bn(cfg->output_dim);
-        L->ntiles1 = (cfg->expert_dim + L->bn1 - 1) / L->bn1;
-        L->ntiles2 = (cfg->output_dim + L->bn2 - 1) / L->bn2;
-        L->norm_parts = L->ntiles2;
-        if (!encode_bf16_2d(&L->map_w1, w->w1, cfg->input_dim, (uint64_t)L->G * cfg->expert_dim, L->bn1) ||
-            !encode_bf16_2d(&L->map_w2, w->w2, cfg->expert_dim, (uint64_t)L->G * cfg->output_dim, L->bn2)) {
+        if (!encode_bf16_2d(&L->map_w1, w->w1, cfg->input_dim, (uint64_t)L->G * cfg->expert_dim, 128) ||
+            !encode_bf16_2d(&L->map_w2, w->w2, cfg->expert_dim, (uint64_t)L->G * cfg->output_dim, 128)) {
             delete L;
             return fail(MOE_ERR_CUDA, "cuTensorMapEncodeTiled failed for the expert weights (16-byte alignment?)");
         }
-    } else {
-        L->ntiles1 = (cfg->expert_dim + kSimtBN - 1) / kSimtBN;
-        L->ntiles2 = (cfg->output_dim + kSimtBN - 1) / kSimtBN;
-        L->norm_parts = L->ntiles2;
+        L->num_pairs = gemm_pair_max_pairs(L->num_sms);
+        if (L->num_pairs <= 0) {
+            delete L;
+            return fail(MOE_ERR_CUDA, "no 2-CTA cluster of the expert GEMM fits on device %d", dev);
+        }
     }
     *out = L;
     return MOE_OK;
@@ -391,7 +406,8 @@ int moe_forward(moe_layer_t *L, const void *x, int32_t T, const float *logit_noi
     da.user_count_kept = rt ? rt->count_kept : nullptr;
     da.group_start = reinterpret_cast<int32_t *>(ws + p.o_gstart);
     da.group_rows = reinterpret_cast<int32_t *>(ws + p.o_grows);
-    da.tile_group = reinterpret_cast<int32_t *>(ws + p.o_tgroup);
+    da.block_group = reinterpret_cast<int32_t *>(ws + p.o_bgroup);
+    da.tok_tiles = reinterpret_cast<int4 *>(ws + p.o_toktiles);
     da.ctrl = ctrl;
     da.slot = slot;
     da.row_of = reinterpret_cast<int32_t *>(ws + p.o_rowof);
@@ -410,73 +426,76 @@ int moe_forward(moe_layer_t *L, const void *x, int32_t T, const float *logit_noi
         MOE_LAUNCH(launch_scatter(sa, L->num_sms, s, nl));
     }
 
-    GemmArgs g1;
-    g1.tile_group = da.tile_group;
-    g1.group_start = da.group_start;
-    g1.group_rows = da.group_rows;
-    g1.ctrl = ctrl;
-    g1.max_mtiles = p.max_mtiles;
-    g1.N = c.expert_dim;
-    g1.K = c.input_dim;
-    g1.n_tiles = L->ntiles1;
-    g1.n_last = c.expert_dim - (L->ntiles1 - 1) * (L->tc ? L->bn1 : kSimtBN);
-    g1.E = E;
-    g1.use_a1 = 1;
-    g1.row_assign = da.row_assign;
-    g1.k = k;
-    g1.T = T;
-    g1.bias = L->w.b1;
-    g1.out = ws + p.o_h;
-    g1.norm_part = nullptr;
-    g1.act = c.activation;
-    g1.status = status;
-    g1.num_sms = L->num_sms;
-    GemmArgs g2 = g1;
-    g2.use_a1 = 0;
-    g2.N = c.output_dim;
-    g2.K = c.expert_dim;
-    g2.n_tiles = L->ntiles2;
-    g2.n_last = c.output_dim - (L->ntiles2 - 1) * (L->tc ? L->bn2 : kSimtBN);
-    g2.bias = L->w.b2;
-    g2.out = ws + p.o_o;
-    g2.norm_part = reinterpret_cast<float *>(ws + p.o_norm);
-    g2.act = -1;
-
     if (L->tc) {
-        CUtensorMap m_xp, m_x, m_h, m_hs, m_os;
-        if (!encode_bf16_2d(&m_xp, ws + p.o_xp, c.input_dim, p.R_routed_max, kBM) ||
-            !encode_bf16_2d(&m_x, x, c.input_dim, T, kBM) ||
-            !encode_bf16_2d(&m_h, ws + p.o_h, c.expert_dim, p.R_max, kBM) ||
-            !encode_bf16_2d(&m_hs, ws + p.o_h, c.expert_dim, p.R_max, 32) ||
-            !encode_bf16_2d(&m_os, ws + p.o_o, c.output_dim, p.R_max, 32))
+        PairGemmArgs g1;
+        g1.tok_tiles = da.tok_tiles;
+        g1.group_start = da.group_start;
+        g1.ctrl = ctrl;
+        g1.max_tok_tiles = p.max_tok_tiles;
+        g1.N = c.expert_dim;
+        g1.K = c.input_dim;
+        g1.n_ftiles = gemm_pair_ftiles(c.expert_dim);
+        g1.E = E;
+        g1.use_s = 1;
+        g1.bias = L->w.b1;
+        g1.act = c.activation;
+        g1.status = status;
+        g1.num_pairs = L->num_pairs;
+        PairGemmArgs g2 = g1;
+        g2.N = c.output_dim;
+        g2.K = c.expert_dim;
+        g2.n_ftiles = gemm_pair_ftiles(c.output_dim);
+        g2.use_s = 0;
+        g2.bias = L->w.b2;
+        g2.act = -1;
+        CUtensorMap m_xp, m_xp16, m_x, m_x16, m_h, m_h16, m_hs, m_os;
+        if (!encode_bf16_2d(&m_xp, ws + p.o_xp, c.input_dim, p.R_routed_max, 128) ||
+            !encode_bf16_2d(&m_xp16, ws + p.o_xp, c.input_dim, p.R_routed_max, 16) ||
+            !encode_bf16_2d(&m_x, x, c.input_dim, T, 128) || !encode_bf16_2d(&m_x16, x, c.input_dim, T, 16) ||
+            !encode_bf16_2d(&m_h, ws + p.o_h, c.expert_dim, p.R_max, 128) ||
+            !encode_bf16_2d(&m_h16, ws + p.o_h, c.expert_dim, p.R_max, 16) ||
+            !encode_bf16_store(&m_hs, ws + p.o_h, c.expert_dim, p.R_max) ||
+            !encode_bf16_store(&m_os, ws + p.o_o, c.output_dim, p.R_max))
             return fail(MOE_ERR_CUDA, "cuTensorMapEncodeTiled failed for the activations");
-        MOE_LAUNCH(launch_gemm_tc(m_xp, m_x, L->map_w1, m_hs, g1, L->bn1, s, nl));
+        MOE_LAUNCH(launch_gemm_pair(L->map_w1, m_xp, m_xp16, m_x, m_x16, m_hs, g1, s, nl));
         MOE_MARK(L, 3, s);
-        MOE_LAUNCH(launch_gemm_tc(m_h, m_h, L->map_w2, m_os, g2, L->bn2, s, nl));
+        MOE_LAUNCH(launch_gemm_pair(L->map_w2, m_h, m_h16, m_h, m_h16, m_os, g2, s, nl));
         MOE_MARK(L, 4, s);
     } else {
         GemmSimtArgs s1;
-        s1.g = g1;
+        s1.block_group = da.block_group;
+        s1.group_start = da.group_start;
+        s1.group_rows = da.group_rows;
+        s1.ctrl = ctrl;
+        s1.max_row_blocks = p.max_row_blocks;
+        s1.N = c.expert_dim;
+        s1.K = c.input_dim;
+        s1.E = E;
+        s1.k = k;
+        s1.row_assign = da.row_assign;
+        s1.bias = L->w.b1;
+        s1.out = reinterpret_cast<float *>(ws + p.o_h);
+        s1.act = c.activation;
         s1.a = static_cast<const float *>(x);
         s1.gather = 1;
         s1.w = static_cast<const float *>(L->w.w1);
-        s1.max_rows = p.R_max;
         MOE_LAUNCH(launch_gemm_simt(s1, s, nl));
         MOE_MARK(L, 3, s);
-        GemmSimtArgs s2;
-        s2.g = g2;
+        GemmSimtArgs s2 = s1;
+        s2.N = c.output_dim;
+        s2.K = c.expert_dim;
+        s2.bias = L->w.b2;
+        s2.out = reinterpret_cast<float *>(ws + p.o_o);
+        s2.act = -1;
         s2.a = reinterpret_cast<const float *>(ws + p.o_h);
         s2.gather = 0;
         s2.w = static_cast<const float *>(L->w.w2);
-        s2.max_rows = p.R_max;
         MOE_LAUNCH(launch_gemm_simt(s2, s, nl));
         MOE_MARK(L, 4, s);
     }
 
     CombineArgs ca;
     ca.o = ws + p.o_o;
-    ca.norm_part = g2.norm_part;
-    ca.n_parts = L->norm_parts;
     ca.row_of = da.row_of;
     ca.gates = gates;
     ca.group_start = da.group_start;

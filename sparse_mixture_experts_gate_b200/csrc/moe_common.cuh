@@ -16,6 +16,11 @@ namespace moe {
 constexpr int kBM = 128;
 // K extent of one pipeline stage: 64 bf16 = 128 bytes, one 128B-swizzle row.
 constexpr int kBK = 64;
+// Every expert's row segment in the permuted row space is padded to a multiple
+// of kRowBlock rows; the expert GEMM covers a segment with token tiles of at
+// most kTokTile rows (the MMA's N), each a multiple of kRowBlock.
+constexpr int kRowBlock = 32;
+constexpr int kTokTile = 256;
 
 // Device status word values (bit flags, OR-ed together).
 enum : uint32_t { kDevOk = 0u, kDevTimeout = 1u };
@@ -69,6 +74,9 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
 // false, without waiting further, once the shared status word is non-zero
 // (another role or CTA gave up) or after kWaitLimitNs; in the latter case it
 // sets kDevTimeout in the status word itself. Never traps, never spins forever.
+// The status word (a global load) is only polled once the wait has lasted
+// kStatusPollNs, so a normal short wait spins on the barrier alone.
+constexpr uint64_t kStatusPollNs = 20000ull;
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, uint32_t *status) {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = global_timer_ns();
@@ -76,8 +84,28 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, uint32
 #pragma unroll 1
         for (int i = 0; i < 32; ++i)
             if (mbar_try_wait(bar, parity)) return true;
-        if (*reinterpret_cast<volatile uint32_t *>(status) != kDevOk) return false;
-        if (global_timer_ns() - t0 > kWaitLimitNs) {
+        const uint64_t dt = global_timer_ns() - t0;
+        if (dt > kStatusPollNs && *reinterpret_cast<volatile uint32_t *>(status) != kDevOk) return false;
+        if (dt > kWaitLimitNs) {
+            atomicOr(status, kDevTimeout);
+            return false;
+        }
+    }
+}
+
+// The same for a wait that is expected to be long and whose end is not
+// latency-critical (an epilogue waiting for the next accumulator): after the
+// first microsecond it sleeps between polls, leaving issue slots and shared
+// memory bandwidth to the roles that are working.
+__device__ __forceinline__ bool mbar_wait_idle(uint64_t *bar, uint32_t parity, uint32_t *status) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = global_timer_ns();
+    for (;;) {
+        if (mbar_try_wait(bar, parity)) return true;
+        const uint64_t dt = global_timer_ns() - t0;
+        if (dt > 1000ull) __nanosleep(256);
+        if (dt > kStatusPollNs && *reinterpret_cast<volatile uint32_t *>(status) != kDevOk) return false;
+        if (dt > kWaitLimitNs) {
             atomicOr(status, kDevTimeout);
             return false;
         }
@@ -248,6 +276,96 @@ __device__ __forceinline__ uint64_t sw128_kmajor_desc(uint32_t smem_addr) {
 __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N) {
     return (1u << 4) | (1u << 7) | (1u << 10) | (static_cast<uint32_t>(N >> 3) << 17) |
            (static_cast<uint32_t>(M >> 4) << 24);
+}
+
+// ------------------------------------------------------- CTA pairs (cta_group::2)
+//
+// Two CTAs of a 2-CTA cluster run one MMA of M = 256 together: the leader
+// (cluster rank 0) issues it, each CTA holds half of A (its 128 rows) and half
+// of B (N/2 rows) in its own shared memory at the same offsets, and each CTA's
+// TMEM receives its 128 rows of the accumulator.
+
+__device__ __forceinline__ uint32_t cluster_ctarank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+
+// Shared::cluster address of the variable at shared::cta address `addr` in
+// the cluster's CTA `rank`.
+__device__ __forceinline__ uint32_t mapa_shared(uint32_t addr, uint32_t rank) {
+    uint32_t r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(addr), "r"(rank));
+    return r;
+}
+
+// Every thread of both CTAs arrives, then waits for all of them.
+__device__ __forceinline__ void cluster_sync_all() {
+    asm volatile("barrier.cluster.arrive.release;\n\tbarrier.cluster.wait.acquire;" ::: "memory");
+}
+
+// Arrive on an mbarrier given by its shared::cluster address (own or peer CTA).
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t bar_cluster_addr) {
+    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(bar_cluster_addr) : "memory");
+}
+
+// TMA load into this CTA's shared memory whose completion is signalled on an
+// mbarrier of either CTA of the pair (the leader's, for the pair's MMA).
+__device__ __forceinline__ void tma_load_2d_pair(const CUtensorMap *map, uint32_t bar_cluster_addr, void *dst,
+                                                 int32_t c0, int32_t c1) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%3, %4}], [%2];" ::"r"(smem_u32(dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(bar_cluster_addr), "r"(c0), "r"(c1)
+        : "memory");
+}
+
+__device__ __forceinline__ void tmem_alloc_pair(uint32_t *dst_smem, uint32_t ncols) {
+    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(dst_smem)),
+                 "r"(ncols)
+                 : "memory");
+}
+
+__device__ __forceinline__ void tmem_relinquish_pair() {
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols) {
+    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+
+// The pair's MMA, issued by one thread of the leader CTA.
+__device__ __forceinline__ void tc_mma_bf16_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                                 uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+// Arrives once on the mbarrier at the same shared-memory offset in every CTA
+// of `cta_mask` when the pair MMAs this thread issued so far have completed.
+__device__ __forceinline__ void tc_commit_pair_mc(uint64_t *bar, uint16_t cta_mask) {
+    asm volatile(
+        "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(
+            smem_u32(bar)),
+        "h"(cta_mask)
+        : "memory");
+}
+
+// As tc_commit, for pair MMAs, on this CTA's own barrier.
+__device__ __forceinline__ void tc_commit_pair(uint64_t *bar) {
+    asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
+                 : "memory");
+}
+
+// Spins for about `ns` nanoseconds (used only on the way out after a timeout).
+__device__ __forceinline__ void spin_ns(uint64_t ns) {
+    const uint64_t t0 = global_timer_ns();
+    while (global_timer_ns() - t0 < ns) {
+    }
 }
 
 // ------------------------------------------------------------------ misc

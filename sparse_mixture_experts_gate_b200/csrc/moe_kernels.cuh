@@ -53,7 +53,7 @@ struct DispatchArgs {
     const int32_t *idx;     // [T][k]
     int T, E, k, S;
     int64_t C;              // capacity
-    int T_pad;              // T rounded up to kBM (shared-expert segment length)
+    int T_pad;              // T rounded up to kRowBlock (shared-expert segment length)
     int n_chunks;           // ceil(T / 256)
     int32_t *chunk_count;   // [n_chunks][E]
     int32_t *chunk_base;    // [n_chunks][E]
@@ -63,7 +63,8 @@ struct DispatchArgs {
     int32_t *user_count_kept;  // [E] or null
     int32_t *group_start;   // [E+S+1]
     int32_t *group_rows;    // [E+S]
-    int32_t *tile_group;    // [max_mtiles]
+    int32_t *block_group;   // [max_row_blocks]: group of each 32-row block
+    int4 *tok_tiles;        // [max_tok_tiles]: {group, first row, rows, 0}
     int32_t *ctrl;          // control block (see kCtrl*)
     int32_t *slot;          // [T][k]
     int32_t *row_of;        // [T][k]
@@ -72,7 +73,14 @@ struct DispatchArgs {
 cudaError_t launch_dispatch(const DispatchArgs &a, cudaStream_t s, int *launches);
 
 // Control block words.
-enum { kCtrlStatus = 0, kCtrlNumMTiles = 1, kCtrlRoutedRows = 2, kCtrlDropped = 3, kCtrlWords = 8 };
+enum {
+    kCtrlStatus = 0,
+    kCtrlNumRowBlocks = 1,
+    kCtrlRoutedRows = 2,
+    kCtrlDropped = 3,
+    kCtrlNumTokTiles = 4,
+    kCtrlWords = 8
+};
 
 // Scatter of token rows into the permuted row space (rows of kept assignments).
 struct ScatterArgs {
@@ -86,50 +94,54 @@ cudaError_t launch_scatter(const ScatterArgs &a, int num_sms, cudaStream_t s, in
 
 // Grouped expert GEMM: out[row] = act(A[row] . W[g]^T + b[g]) for the rows of
 // every group g (routed experts, then shared experts).
-struct GemmArgs {
-    const int32_t *tile_group;   // [max_mtiles]
+//
+// bf16 tensor-core path on CTA pairs (gemm_pair.cu): work unit = (token tile,
+// 256-feature tile). map_w: the weight stack [G*N][K] (box 64 x 128);
+// map_t / map_t16: the token rows in row order (box 64 x 128 and 64 x 16);
+// map_s / map_s16: with use_s, the token rows of shared-expert groups (x itself,
+// in token order); map_out: [rows][N] bf16, box 32 x 32, no swizzle.
+// N and K must be multiples of 64.
+struct PairGemmArgs {
+    const int4 *tok_tiles;       // [max_tok_tiles] {group, first row, rows, 0}
     const int32_t *group_start;  // [G+1]
-    const int32_t *group_rows;   // [G]
-    const int32_t *ctrl;         // kCtrlNumMTiles
-    int max_mtiles;              // host bound on the M tiles (clamps the device count)
-    int N, K;                    // output row length, reduction length
-    int n_tiles;                 // ceil(N / BN)
-    int n_last;                  // columns of the last N tile (N - (n_tiles - 1) BN)
-    int E;                       // groups >= E are shared experts (A through the second map)
-    int use_a1;
-    const int32_t *row_assign;   // [rows] t*k + r of each routed row (-1 padding)
-    int k, T;
+    const int32_t *ctrl;         // kCtrlNumTokTiles, kCtrlStatus
+    int max_tok_tiles;           // host bound (clamps the device count)
+    int N, K;
+    int n_ftiles;                // ceil(N / 256)
+    int E;                       // groups >= E are shared experts
+    int use_s;
     const float *bias;           // [G][N] or null
-    void *out;                   // [rows][N]
-    float *norm_part;            // [rows][n_tiles] or null: per-tile sum of out^2 (fp32, before rounding)
     int act;                     // activation code, -1 none
     uint32_t *status;            // device status word
-    int num_sms;
+    int num_pairs;               // clusters of 2 CTAs to launch
 };
-// bf16 tcgen05 path; BN is 256 when N > 256 (the last N tile may be narrower),
-// else the largest of 128 and 64 dividing N. N must be a multiple of 64.
-// A rows come from map_a0 (row space: the scattered rows or H, box 64 x 128); with
-// use_a1, shared-expert groups read x itself through map_a1 (box 64 x 128).
-// map_out: the output [rows][N] bf16, box 64 x 32, 128B swizzle.
-int gemm_pick_bn(int N);
-cudaError_t launch_gemm_tc(const CUtensorMap &map_a0, const CUtensorMap &map_a1, const CUtensorMap &map_b,
-                           const CUtensorMap &map_out, const GemmArgs &a, int BN, cudaStream_t s, int *launches);
-// fp32 CUDA-core path (A operand as a plain pointer).
+int gemm_pair_max_pairs(int num_sms);
+int gemm_pair_ftiles(int N);
+cudaError_t launch_gemm_pair(const CUtensorMap &map_w, const CUtensorMap &map_t, const CUtensorMap &map_t16,
+                             const CUtensorMap &map_s, const CUtensorMap &map_s16, const CUtensorMap &map_out,
+                             const PairGemmArgs &a, cudaStream_t s, int *launches);
+
+// fp32 CUDA-core path: 32 x 32 output tiles over the 32-row blocks.
 struct GemmSimtArgs {
-    GemmArgs g;
-    const float *a;    // gather: x [T][K]; otherwise [rows][K]
+    const int32_t *block_group;  // [max_row_blocks]
+    const int32_t *group_start;  // [G+1]
+    const int32_t *group_rows;   // [G]
+    const int32_t *ctrl;         // kCtrlNumRowBlocks
+    int max_row_blocks;
+    int N, K, E, k;
+    const int32_t *row_assign;   // [rows] t*k + r of each routed row (-1 padding)
+    const float *bias;           // [G][N] or null
+    float *out;                  // [rows][N]
+    int act;
+    const float *a;              // gather: x [T][K]; otherwise [rows][K]
     int gather;
-    const float *w;    // [G][N][K]
-    int max_rows;      // rows the launch covers
+    const float *w;              // [G][N][K]
 };
-constexpr int kSimtBN = 32;
 cudaError_t launch_gemm_simt(const GemmSimtArgs &a, cudaStream_t s, int *launches);
 
 // Gate-weighted combine with shared experts, plus credit.
 struct CombineArgs {
     const void *o;          // [rows][O] expert outputs
-    const float *norm_part; // [rows][n_parts]
-    int n_parts;
     const int32_t *row_of;  // [T][k]
     const float *gates;     // [T][k]
     const int32_t *group_start;

@@ -150,8 +150,9 @@ __global__ void __launch_bounds__(kRouterThreads, 1)
             for (int j = 0; j < HALF; ++j) sum[j] = 0.f;
             for (int g = gr.x; g < gr.y; ++g, ++gcount) {
                 const uint32_t buf = gcount & 1u, use = gcount >> 1;
-                const bool got = mbar_wait(&s.tfull[buf], use & 1u, a.status);
-                if (!__all_sync(0xffffffffu, got)) {
+                int got = 1;
+                if (lane == 0) got = mbar_wait(&s.tfull[buf], use & 1u, a.status) ? 1 : 0;
+                if (!__shfl_sync(0xffffffffu, got, 0)) {
                     ok = false;
                     break;
                 }

@@ -188,9 +188,10 @@ __device__ __forceinline__ void tc_epilogue(const TcShared<BN> &s, uint32_t tmem
     uint32_t tcount = 0;
     for (int tile = blockIdx.x; tile < total; tile += gridDim.x, ++tcount) {
         const uint32_t acc = tcount & 1u, use = tcount >> 1;
-        // tcgen05.ld is warp-collective: make the wait outcome warp-uniform.
-        const bool got = mbar_wait(&s.tfull[acc], use & 1u, status);
-        if (!__all_sync(0xffffffffu, got)) break;
+        // tcgen05.ld is warp-collective: one lane waits, the outcome is broadcast.
+        int got = 1;
+        if (lane == 0) got = mbar_wait_idle(&s.tfull[acc], use & 1u, status) ? 1 : 0;
+        if (!__shfl_sync(0xffffffffu, got, 0)) break;
         tc_fence_after_sync();
         const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * kTcAccCols;
         epi(tile, taddr, q, lane);
