@@ -18,6 +18,12 @@
 // weight tile, the operand every token of the expert shares, is split across
 // the pair so that each SM stages half of it.
 //
+// Units are handed out in index order from a global counter (see post_unit),
+// so the pairs at work hold a contiguous run of units whatever their lengths:
+// with a static round-robin the pairs drift apart over the ~140 waves of the
+// E = 256 layer and the L2 reuse of the weight tiles collapses (GEMM 1 read
+// 41.6 GB from DRAM instead of ~15 GB).
+//
 // Per CTA (192 threads): warp 0 loads (TMA, signalling the leader's stage
 // barrier, which expects both CTAs' bytes), warp 1 owns TMEM (2 accumulators x
 // 256 columns) and, in the leader, issues the pair MMAs and commits stages and
@@ -48,14 +54,17 @@ constexpr int kBoxTok = 32, kBoxFeat = 32;          // store box: 32 tokens x 32
 constexpr int kBoxBytes = kBoxTok * kBoxFeat * 2;
 constexpr int kStaging = 4 * 2 * kBoxBytes;         // 4 epilogue warps x 2 boxes
 constexpr int kRowsPerLoad16 = 16;                  // rows of the narrow token box
-constexpr int kSmem = 1024 + kStages * kStage + kStaging + 256;
+constexpr int kRing = 8;            // unit-index ring between the leader's producer and the consumers
+constexpr int kRingConsumers = 10;  // leader: MMA thread + 4 epilogue warps; peer: producer + 4 epilogue warps
+constexpr int kSmem = 1024 + kStages * kStage + kStaging + 512;
 static_assert(kSmem <= 232448, "exceeds the 227 KB of shared memory a CTA may use");
 static_assert(kTokTile == 256 && kTokTile % (2 * kRowsPerLoad16) == 0, "token tile layout");
 
 struct Smem {
     uint8_t *sA, *sB, *staging;
-    uint64_t *full, *empty, *tfull, *tempty, *mma_done;
+    uint64_t *full, *empty, *tfull, *tempty, *mma_done, *ring_full, *ring_empty;
     uint32_t *tmem_slot;
+    int32_t *ring;
 };
 
 __device__ __forceinline__ Smem carve(uint8_t *raw) {
@@ -69,7 +78,10 @@ __device__ __forceinline__ Smem carve(uint8_t *raw) {
     s.tfull = s.empty + kStages;
     s.tempty = s.tfull + 2;
     s.mma_done = s.tempty + 2;
-    s.tmem_slot = reinterpret_cast<uint32_t *>(s.mma_done + 1);
+    s.ring_full = s.mma_done + 1;
+    s.ring_empty = s.ring_full + kRing;
+    s.tmem_slot = reinterpret_cast<uint32_t *>(s.ring_empty + kRing);
+    s.ring = reinterpret_cast<int32_t *>(s.tmem_slot + 4);
     return s;
 }
 
@@ -84,7 +96,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const uint32_t rank = cluster_ctarank();
     const bool leader = rank == 0;
-    const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
 
     if (threadIdx.x == 0) {
         tma_prefetch_desc(&map_w);
@@ -102,6 +113,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(&s.tempty[i], 8);  // 4 epilogue warps in each CTA
         }
         mbar_init(s.mma_done, 1);
+        for (int i = 0; i < kRing; ++i) {
+            mbar_init(&s.ring_full[i], 1);
+            mbar_init(&s.ring_empty[i], kRingConsumers);  // used in the leader only
+        }
         fence_barrier_init();
     }
     if (warp == 1) {
@@ -118,10 +133,42 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int kblocks = a.K / kBK;
     bool ok = true;
 
+    // Units (token tile, feature tile) are handed out in index order from a
+    // global counter, so the pairs working at any moment hold a contiguous run
+    // of units and share their weight and token tiles through L2, however
+    // unequal the units' lengths. The leader's producer takes each unit and
+    // posts it to a ring in both CTAs; every consumer reads entry i for its
+    // i-th unit and releases it on the leader's ring_empty. -1 ends the work.
+    auto post_unit = [&](uint32_t i) -> int {  // leader's producer, lane 0
+        const uint32_t slot = i % kRing, ph = (i / kRing) & 1u;
+        if (!mbar_wait_cluster(&s.ring_empty[slot], ph ^ 1u, a.status)) return -2;
+        int u = atomicAdd(a.work_counter, 1);
+        if (u >= total) u = -1;
+        s.ring[slot] = u;
+        st_shared_cluster_u32(mapa_shared(smem_u32(&s.ring[slot]), 1), static_cast<uint32_t>(u));
+        mbar_arrive(&s.ring_full[slot]);
+        mbar_arrive_cluster(mapa_shared(smem_u32(&s.ring_full[slot]), 1));
+        return u;
+    };
+    auto take_unit = [&](uint32_t i) -> int {  // one thread of each consumer
+        const uint32_t slot = i % kRing, ph = (i / kRing) & 1u;
+        if (!mbar_wait_cluster(&s.ring_full[slot], ph, a.status)) return -2;
+        const int u = *reinterpret_cast<volatile int32_t *>(&s.ring[slot]);
+        mbar_arrive_cluster(mapa_shared(smem_u32(&s.ring_empty[slot]), 0));
+        return u;
+    };
+
     if (warp == 0) {
         // ------------------------------------------------------------ producer
         uint32_t it = 0;
-        for (int u = pair; u < total && ok; u += npairs) {
+        for (uint32_t i = 0; ok; ++i) {
+            int u = 0;
+            if (lane == 0) u = leader ? post_unit(i) : take_unit(i);
+            u = __shfl_sync(0xffffffffu, u, 0);
+            if (u < 0) {
+                ok = u == -1;
+                break;
+            }
             const int tt = u / a.n_ftiles, j = u - tt * a.n_ftiles;
             const int4 tile = a.tok_tiles[tt];  // {group, first row, rows, -}
             const int g = tile.x, ntok = tile.z;
@@ -161,8 +208,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA (leader)
         if (leader && lane == 0) {
-            uint32_t it = 0, tcount = 0;
-            for (int u = pair; u < total && ok; u += npairs, ++tcount) {
+            uint32_t it = 0;
+            for (uint32_t tcount = 0; ok; ++tcount) {
+                const int u = take_unit(tcount);
+                if (u < 0) {
+                    ok = u == -1;
+                    break;
+                }
                 const int ntok = a.tok_tiles[u / a.n_ftiles].z;
                 const uint32_t idesc = idesc_bf16_f32(kFeatPair, ntok);
                 const uint32_t acc = tcount & 1u, use = tcount >> 1;
@@ -193,8 +245,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         // ------------------------------------------------------------ epilogue
         const int q = warp & 3;  // TMEM lane quarter this warp may access
         uint8_t *my_stage = s.staging + (warp - 2) * 2 * kBoxBytes;
-        uint32_t sub = 0, tcount = 0;
-        for (int u = pair; u < total; u += npairs, ++tcount) {
+        uint32_t sub = 0;
+        for (uint32_t tcount = 0;; ++tcount) {
+            int u = 0;
+            if (lane == 0) u = take_unit(tcount);
+            u = __shfl_sync(0xffffffffu, u, 0);
+            if (u < 0) break;
             const int tt = u / a.n_ftiles, j = u - tt * a.n_ftiles;
             const int4 tile = a.tok_tiles[tt];
             const int g = tile.x, row0 = tile.y, ntok = tile.z;

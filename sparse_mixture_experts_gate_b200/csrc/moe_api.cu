@@ -440,6 +440,7 @@ int moe_forward(moe_layer_t *L, const void *x, int32_t T, const float *logit_noi
         g1.bias = L->w.b1;
         g1.act = c.activation;
         g1.status = status;
+        g1.work_counter = ctrl + kCtrlWork1;
         g1.num_pairs = L->num_pairs;
         PairGemmArgs g2 = g1;
         g2.N = c.output_dim;
@@ -448,6 +449,7 @@ int moe_forward(moe_layer_t *L, const void *x, int32_t T, const float *logit_noi
         g2.use_s = 0;
         g2.bias = L->w.b2;
         g2.act = -1;
+        g2.work_counter = ctrl + kCtrlWork2;
         CUtensorMap m_xp, m_xp16, m_x, m_x16, m_h, m_h16, m_hs, m_os;
         if (!encode_bf16_2d(&m_xp, ws + p.o_xp, c.input_dim, p.R_routed_max, 128) ||
             !encode_bf16_2d(&m_xp16, ws + p.o_xp, c.input_dim, p.R_routed_max, 16) ||

@@ -79,6 +79,8 @@ enum {
     kCtrlRoutedRows = 2,
     kCtrlDropped = 3,
     kCtrlNumTokTiles = 4,
+    kCtrlWork1 = 5,  // unit counters of the two expert GEMM launches
+    kCtrlWork2 = 6,
     kCtrlWords = 8
 };
 
@@ -113,6 +115,7 @@ struct PairGemmArgs {
     const float *bias;           // [G][N] or null
     int act;                     // activation code, -1 none
     uint32_t *status;            // device status word
+    int32_t *work_counter;       // zero before the launch; units are handed out in order
     int num_pairs;               // clusters of 2 CTAs to launch
 };
 int gemm_pair_max_pairs(int num_sms);
