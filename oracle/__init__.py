@@ -60,6 +60,10 @@ def _configure(L):
                                       i32, vp, ctypes.POINTER(Expert), vp, vp, vp, vp, vp]
     L.orc_balance_stats.argtypes = [i32, i32, i32, vp, vp, vp, dbl, dbl, vp, vp, vp, vp]
     L.orc_expert_loss.argtypes = [i32, i32, i32, vp, vp, vp, vp, vp]
+    L.orc_importance.argtypes = [i32, i32, i32, vp, vp, vp]
+    L.orc_cv_squared.argtypes = [i32, vp]
+    L.orc_cv_squared.restype = dbl
+    L.orc_selection_bias_update.argtypes = [i32, i32, i64, vp, ctypes.c_float, vp]
     L.orc_max_threads.restype = i32
     return L
 
@@ -263,6 +267,30 @@ def expert_loss(idx, slot, credit, token_loss, E: int) -> np.ndarray:
     T, k = idx.shape
     out = np.empty(E, np.float64)
     lib().orc_expert_loss(T, E, k, _p(idx), _p(slot), _p(credit), _p(tl), _p(out))
+    return out
+
+
+def importance(idx, g, E: int) -> np.ndarray:
+    """Sum of the routed gate weights per expert ("Load balancing")."""
+    idx = np.ascontiguousarray(idx, dtype=np.int32)
+    g = np.ascontiguousarray(g, dtype=np.float64)
+    T, k = idx.shape
+    out = np.empty(E, np.float64)
+    lib().orc_importance(T, E, k, _p(idx), _p(g), _p(out))
+    return out
+
+
+def cv_squared(v) -> float:
+    """Squared coefficient of variation, population variance ("Load balancing")."""
+    v = np.ascontiguousarray(v, dtype=np.float64)
+    return float(lib().orc_cv_squared(int(v.size), _p(v)))
+
+
+def selection_bias_update(b, load, k: int, T: int, gamma: float) -> np.ndarray:
+    """b_i + gamma sign(kT/E - load_i), rounded to fp32 ("Balancing")."""
+    out = np.ascontiguousarray(np.array(b, dtype=np.float32).copy())
+    ld = np.ascontiguousarray(np.asarray(load, dtype=np.int64))
+    lib().orc_selection_bias_update(int(out.size), int(k), int(T), _p(ld), float(gamma), _p(out))
     return out
 
 

@@ -262,6 +262,42 @@ void orc_expert_loss(int T, int E, int k, const int32_t *idx, const int32_t *slo
         expert_loss[i] /= (double)T;
 }
 
+/* Load balancing: importance = sum of routed gate weights per expert. */
+void orc_importance(int T, int E, int k, const int32_t *idx, const double *g, double *imp)
+{
+    for (int i = 0; i < E; ++i)
+        imp[i] = 0.0;
+    for (int t = 0; t < T; ++t)
+        for (int r = 0; r < k; ++r)
+            imp[idx[(int64_t)t * k + r]] += g[(int64_t)t * k + r];
+}
+
+/* Load balancing: squared coefficient of variation (population variance). */
+double orc_cv_squared(int n, const double *v)
+{
+    double mean = 0.0;
+    for (int i = 0; i < n; ++i)
+        mean += v[i];
+    mean /= (double)n;
+    if (mean == 0.0)
+        return 0.0;
+    double var = 0.0;
+    for (int i = 0; i < n; ++i)
+        var += (v[i] - mean) * (v[i] - mean);
+    var /= (double)n;
+    return var / (mean * mean);
+}
+
+/* Balancing: b_i <- b_i + gamma sign(kT/E - load_i), rounded to fp32. */
+void orc_selection_bias_update(int E, int k, int64_t T, const int64_t *load, float gamma, float *b)
+{
+    for (int i = 0; i < E; ++i) {
+        const int64_t diff = (int64_t)k * T - (int64_t)E * load[i];
+        const double s = diff > 0 ? 1.0 : (diff < 0 ? -1.0 : 0.0);
+        b[i] = (float)((double)b[i] + (double)gamma * s);
+    }
+}
+
 #ifdef _OPENMP
 #include <omp.h>
 #endif

@@ -129,6 +129,24 @@ void orc_expert_loss(int T, int E, int k, const int32_t *idx, const int32_t *slo
                      const double *credit, const float *token_loss, double *expert_loss);
 
 /* Threads the oracle's parallel loops use (1 when built without OpenMP). */
+/* [W] "Load balancing": an importance loss "balances total importance per
+ * expert". Importance of expert i = the sum over the batch of the gate weights
+ * routed to it (renormalised gates g, every selection, before capacity drops).
+ * idx, g [T][k] -> imp [E]. */
+void orc_importance(int T, int E, int k, const int32_t *idx, const double *g, double *imp);
+
+/* [W] "Load balancing": a "coefficient-of-variation style balance across
+ * experts". Squared coefficient of variation of v[0..n): population variance
+ * over the squared mean (0 when the mean is 0). */
+double orc_cv_squared(int n, const double *v);
+
+/* [C] "Balancing": per-expert selection bias b_i (aux-loss-free balancing) with
+ * update rate gamma: b_i <- b_i + gamma * sign(mean load - load_i), load_i =
+ * selections of expert i before capacity, mean load = k T / E (the sign is
+ * decided exactly, on k T - E load_i). The sum is rounded once to the bias's
+ * fp32 storage. load [E]; b [E] updated in place. */
+void orc_selection_bias_update(int E, int k, int64_t T, const int64_t *load, float gamma, float *b);
+
 int orc_max_threads(void);
 
 #ifdef __cplusplus

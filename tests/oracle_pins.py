@@ -403,6 +403,54 @@ def check_credit_is_gate_times_norm():
             assert abs(out["credit"][t, r] - want) <= 1e-12 * (1 + abs(want))
 
 
+def check_cv_squared():
+    """[W] "Load balancing" (coefficient-of-variation style balance): equal loads
+    give 0; m equal non-zero loads out of n give n/m - 1; two loads a, b give
+    ((a - b) / (a + b))^2; scaling every load leaves it unchanged."""
+    assert oracle.cv_squared([7, 7, 7, 7, 7]) == 0.0
+    for n, m in ((4, 1), (4, 2), (8, 3), (256, 8)):
+        v = [5.0] * m + [0.0] * (n - m)
+        assert abs(oracle.cv_squared(v) - (n / m - 1)) <= 1e-12 * (n / m)
+    a, b = 3.0, 11.0
+    assert abs(oracle.cv_squared([a, b]) - ((a - b) / (a + b)) ** 2) < 1e-15
+    rng = np.random.default_rng(5)
+    v = rng.random(13)
+    assert abs(oracle.cv_squared(v) - oracle.cv_squared(4.0 * v)) < 1e-13
+    assert oracle.cv_squared([0.0, 0.0, 0.0]) == 0.0
+
+
+def check_importance():
+    """[W] "Load balancing" (importance per expert): with k = 1 every gate is 1,
+    so the importance is the selection count; the importances of a batch sum to
+    T (each token's gates sum to 1); a hand-worked case."""
+    rng = np.random.default_rng(6)
+    T, E = 40, 6
+    idx1 = rng.integers(0, E, size=(T, 1)).astype(np.int32)
+    imp1 = oracle.importance(idx1, np.ones((T, 1)), E)
+    assert np.array_equal(imp1, np.bincount(idx1[:, 0], minlength=E).astype(np.float64))
+    idx = np.array([rng.permutation(E)[:3] for _ in range(T)], np.int32)
+    g = rng.random((T, 3))
+    g /= g.sum(1, keepdims=True)
+    assert abs(oracle.importance(idx, g, E).sum() - T) < 1e-12
+    hand = oracle.importance(np.array([[0, 1], [1, 2]]), np.array([[0.7, 0.3], [0.6, 0.4]]), 4)
+    assert np.allclose(hand, [0.7, 0.9, 0.4, 0.0], atol=1e-15)
+
+
+def check_selection_bias_update():
+    """[C] "Balancing" (b_i, update rate gamma): experts above the mean load kT/E
+    move down by gamma, those below move up, those at the mean stay; gamma = 0
+    changes nothing; the result is the fp32 rounding of the exact sum."""
+    # E=4, k=2, T=6: mean load 3.
+    b = oracle.selection_bias_update([0.0, 0.0, 0.0, 0.0], [5, 3, 3, 1], 2, 6, 0.5)
+    assert b.tolist() == [-0.5, 0.0, 0.0, 0.5]
+    b0 = np.array([0.1, -0.2, 0.3, 0.05], np.float32)
+    assert np.array_equal(oracle.selection_bias_update(b0, [9, 0, 1, 2], 3, 4, 0.0), b0)
+    # Mean load 12 * 3 / 5 = 7.2 is not an integer: loads 7 and 8 straddle it.
+    b1 = oracle.selection_bias_update(b0.tolist() + [0.0], [7, 8, 7, 8, 6], 3, 12, 1e-3)
+    want = np.float32(np.array(b0.tolist() + [0.0], np.float64) + 1e-3 * np.array([1, -1, 1, -1, 1]))
+    assert np.array_equal(b1, want.astype(np.float32))
+
+
 def check_minimal_example_shapes():
     """[W] "Minimal example": 4 experts, 2 active, dims 8/16/8, a (4, 8) input;
     the forward yields a (4, 8) output, 2 distinct experts per token, gates

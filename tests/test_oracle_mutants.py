@@ -38,6 +38,13 @@ MUTANTS = {
     "router_drops_bias": ("s += (double)b_gate[i];", "s += 0.0;"),
     "noise_ignored": ("v = h32[a] + noise[a];", "v = h32[a];"),
     "selection_bias_sign": ("v = h32[a] + sel_bias[i];", "v = h32[a] - sel_bias[i];"),
+    "cv_sample_variance": ("var /= (double)n;", "var /= (double)(n - 1);"),
+    "cv_not_squared_mean": ("return var / (mean * mean);", "return var / mean;"),
+    "importance_counts_only": ("imp[idx[(int64_t)t * k + r]] += g[(int64_t)t * k + r];",
+                               "imp[idx[(int64_t)t * k + r]] += 1.0;"),
+    "bias_update_sign": ("const double s = diff > 0 ? 1.0 : (diff < 0 ? -1.0 : 0.0);",
+                         "const double s = diff > 0 ? -1.0 : (diff < 0 ? 1.0 : 0.0);"),
+    "bias_update_mean_off": ("(int64_t)k * T - (int64_t)E * load[i]", "(int64_t)T - (int64_t)E * load[i]"),
     "softmax_wrong_exponent": ("P[(int64_t)t * E + i] = exp(ht[i] - m) / z;",
                                "P[(int64_t)t * E + i] = exp(ht[i]) / z;"),
 }
