@@ -138,15 +138,25 @@ typedef struct {
 } moe_routing_t;
 
 /* Statistics written by moe_aux_stats (device pointers; any may be NULL).
+ * "Appendix C - Acronyms & Symbols", table "Balancing"; "Code Walkthrough -
+ * SER", "Load balancing"; "Sparse MoE Expert-Credit Loss Reweighting Diagram",
+ * panel (b).
  *   f           [E] fp32  f_i = count_pre_i / (k T)  (selections before the cap)
  *   p_mean      [E] fp32  P_i = mean over tokens of softmax(h)_i
  *   l_aux       [1] fp32  alpha E sum_i f_i P_i
  *   l_z         [1] fp32  beta mean_t (log sum_i e^{h_ti})^2
  *   n_dropped   [1] int32 assignments dropped by the capacity cap
  *   credit      [T][k] fp32 c = g ||o_e(x_t)||_2 for kept assignments, 0 if dropped
- *               (o_e = the expert's output before gate weighting)
+ *               (o_e = the expert's output before gate weighting, as stored)
  *   expert_loss [E] fp32  l_i = (1/T) sum_t credit_{t,i} token_loss_t over kept
- *               assignments; needs token_loss. */
+ *               assignments; needs token_loss
+ *   importance  [E] fp32  sum over the batch of the renormalised gates routed to
+ *               expert i (every selection, before the cap)
+ *   cv_load     [1] fp32  squared coefficient of variation of count_pre
+ *               (population variance / mean^2; 0 for a zero mean)
+ *   cv_importance [1] fp32 the same for importance
+ *   l_total     [1] fp32  l_aux + l_z (the weighted sum of the balance and
+ *               z-losses with load_balance_coef and z_loss_coef) */
 typedef struct {
     float *f;
     float *p_mean;
@@ -155,6 +165,10 @@ typedef struct {
     int32_t *n_dropped;
     float *credit;
     float *expert_loss;
+    float *importance;
+    float *cv_load;
+    float *cv_importance;
+    float *l_total;
 } moe_stats_t;
 
 typedef struct moe_layer moe_layer_t; /* opaque; host state only */
@@ -229,17 +243,33 @@ MOE_API int moe_aux_stats(moe_layer_t *layer, const float *token_loss, const moe
  *        [0, E)  sum_t P[t][e]       [E, 2E)  selections per expert before the cap
  *        [2E]    sum_t lse_t^2       [2E+1]   T        [2E+2] dropped assignments
  *        [2E+3, 3E+3) sum over kept assignments of credit * token_loss
- *      (the last block is zero when token_loss is NULL);
+ *                     (zero when token_loss is NULL)
+ *        [3E+3, 4E+3) importance: sum of the selections' gates per expert
+ *      Counts travel as fp32 and are exact up to 2^24 per expert;
  *   2. a sum all-reduce of `partials` across the ranks (NCCL, by the caller);
- *   3. moe_stats_from_partials: f, p_mean, l_aux, l_z, n_dropped and (when
- *      has_token_loss) expert_loss of the summed batch into `out`; out->credit
- *      is per token and not written here (moe_aux_stats writes the local one).
+ *   3. moe_stats_from_partials: every statistic of moe_stats_t except credit
+ *      (per token; moe_aux_stats writes the local one) for the summed batch,
+ *      expert_loss only when has_token_loss.
  * moe_aux_stats is steps 1 and 3 on this rank alone. Errors: STATE before any
  * forward, INVALID_ARG for NULL pointers. */
-#define MOE_STAT_PARTIALS(E) (3 * (E) + 3)
+#define MOE_STAT_PARTIALS(E) (4 * (E) + 3)
 MOE_API int moe_stat_partials(moe_layer_t *layer, const float *token_loss, float *partials, void *stream);
 MOE_API int moe_stats_from_partials(moe_layer_t *layer, const float *partials, int32_t has_token_loss,
                                     const moe_stats_t *out, void *stream);
+
+/* Aux-loss-free balancing ("Appendix C - Acronyms & Symbols", table
+ * "Balancing": per-expert selection bias b_i, update rate gamma). Enqueues on
+ * `stream`, for every expert e:
+ *     sel_bias[e] += gamma * sign(k T / E - load_e)
+ * where load_e is the expert's selection count before the cap: taken from
+ * `partials` (MOE_STAT_PARTIALS(E) floats, e.g. summed across data-parallel
+ * ranks, T from the same sums) or, when partials is NULL, from the most recent
+ * moe_forward of this layer. The sign is decided on integers; the one fp32 add
+ * is the only rounding. sel_bias: device [E] fp32, updated in place (pass the
+ * layer's own weights->sel_bias to make the next forward use it). Errors:
+ * INVALID_ARG (NULL sel_bias, NaN gamma), STATE (no partials and no forward). */
+MOE_API int moe_update_selection_bias(moe_layer_t *layer, const float *partials, float gamma, float *sel_bias,
+                                      void *stream);
 
 /* Device status word of the most recent forward: synchronises `stream`, then
  * returns MOE_OK, or MOE_ERR_TIMEOUT if a bounded device-side wait gave up. */

@@ -21,7 +21,8 @@ MOE_DTYPE = {"bf16": 0, "fp32": 1}
 
 # Every symbol include/moe.h declares.
 EXPORTS = ("moe_config_default", "moe_layer_create", "moe_workspace_bytes", "moe_capacity", "moe_forward",
-           "moe_forward_noalloc", "moe_aux_stats", "moe_stat_partials", "moe_stats_from_partials", "moe_device_status", "moe_set_timing_events", "moe_launch_count", "moe_destroy", "moe_status_string",
+           "moe_forward_noalloc", "moe_aux_stats", "moe_stat_partials", "moe_stats_from_partials",
+           "moe_update_selection_bias", "moe_device_status", "moe_set_timing_events", "moe_launch_count", "moe_destroy", "moe_status_string",
            "moe_last_error")
 
 
@@ -48,7 +49,8 @@ class MoeRouting(ctypes.Structure):
 class MoeStats(ctypes.Structure):
     _fields_ = [("f", ctypes.c_void_p), ("p_mean", ctypes.c_void_p), ("l_aux", ctypes.c_void_p),
                 ("l_z", ctypes.c_void_p), ("n_dropped", ctypes.c_void_p), ("credit", ctypes.c_void_p),
-                ("expert_loss", ctypes.c_void_p)]
+                ("expert_loss", ctypes.c_void_p), ("importance", ctypes.c_void_p), ("cv_load", ctypes.c_void_p),
+                ("cv_importance", ctypes.c_void_p), ("l_total", ctypes.c_void_p)]
 
 
 class MoEError(RuntimeError):
@@ -86,6 +88,8 @@ def lib() -> ctypes.CDLL:
         L.moe_stat_partials.argtypes = [vp, vp, vp, vp]
         L.moe_stats_from_partials.restype = ctypes.c_int
         L.moe_stats_from_partials.argtypes = [vp, vp, i32, ctypes.POINTER(MoeStats), vp]
+        L.moe_update_selection_bias.restype = ctypes.c_int
+        L.moe_update_selection_bias.argtypes = [vp, vp, ctypes.c_float, vp, vp]
         L.moe_device_status.restype = ctypes.c_int
         L.moe_device_status.argtypes = [vp, vp]
         L.moe_set_timing_events.restype = ctypes.c_int
@@ -165,7 +169,12 @@ def moe_stats_from_partials(layer: int, partials: int, has_token_loss: bool, sta
 
 
 def stat_partials_size(E: int) -> int:
-    return 3 * E + 3
+    return 4 * E + 3
+
+
+def moe_update_selection_bias(layer: int, partials: Optional[int], gamma: float, sel_bias: int, stream: int) -> int:
+    return _check(lib().moe_update_selection_bias(layer, partials, float(gamma), sel_bias, stream),
+                  "moe_update_selection_bias")
 
 
 def allreduce_partials(partials, group=None):
@@ -277,6 +286,10 @@ class MoELayer:
             n_dropped=torch.empty(1, dtype=torch.int32, device=dev),
             credit=torch.empty(T, w.k, dtype=torch.float32, device=dev),
             expert_loss=torch.empty(w.E, dtype=torch.float32, device=dev),
+            importance=torch.empty(w.E, dtype=torch.float32, device=dev),
+            cv_load=torch.empty(1, dtype=torch.float32, device=dev),
+            cv_importance=torch.empty(1, dtype=torch.float32, device=dev),
+            l_total=torch.empty(1, dtype=torch.float32, device=dev),
         )
         return out
 
@@ -297,11 +310,24 @@ class MoELayer:
     def aux_stats(self, out, token_loss=None, stream=None):
         import torch
         s = stream if stream is not None else torch.cuda.current_stream(self.device).cuda_stream
-        st = MoeStats(_ptr(out["f"]), _ptr(out["p_mean"]), _ptr(out["l_aux"]), _ptr(out["l_z"]),
-                      _ptr(out["n_dropped"]), _ptr(out["credit"]),
-                      _ptr(out["expert_loss"]) if token_loss is not None else None)
-        moe_aux_stats(self.handle, _ptr(token_loss), st, s)
+        moe_aux_stats(self.handle, _ptr(token_loss), self._stats_struct(out, token_loss is not None, True), s)
         return out
+
+    @staticmethod
+    def _stats_struct(out, with_loss: bool, with_credit: bool) -> "MoeStats":
+        g = lambda k: _ptr(out.get(k))
+        return MoeStats(g("f"), g("p_mean"), g("l_aux"), g("l_z"), g("n_dropped"),
+                        g("credit") if with_credit else None, g("expert_loss") if with_loss else None,
+                        g("importance"), g("cv_load"), g("cv_importance"), g("l_total"))
+
+    def update_selection_bias(self, gamma: float, partials=None, stream=None):
+        """sel_bias += gamma * sign(kT/E - load) in place on the layer's own selection
+        bias, loads from `partials` (e.g. all-reduced) or from the last forward."""
+        import torch
+        if self.weights.get("sel_bias") is None:
+            raise ValueError("the layer has no selection bias")
+        s = stream if stream is not None else torch.cuda.current_stream(self.device).cuda_stream
+        moe_update_selection_bias(self.handle, _ptr(partials), gamma, self.weights["sel_bias"].data_ptr(), s)
 
     def dp_aux_stats(self, out, token_loss=None, group=None, stream=None):
         """Statistics of the whole data-parallel batch: this rank's partial sums,
@@ -313,9 +339,8 @@ class MoELayer:
         partials = torch.empty(stat_partials_size(self.w.E), dtype=torch.float32, device=self.device)
         moe_stat_partials(self.handle, _ptr(token_loss), partials.data_ptr(), s)
         allreduce_partials(partials, group)
-        st = MoeStats(_ptr(out["f"]), _ptr(out["p_mean"]), _ptr(out["l_aux"]), _ptr(out["l_z"]),
-                      _ptr(out["n_dropped"]), None, _ptr(out["expert_loss"]) if token_loss is not None else None)
-        moe_stats_from_partials(self.handle, partials.data_ptr(), token_loss is not None, st, s)
+        moe_stats_from_partials(self.handle, partials.data_ptr(), token_loss is not None,
+                                self._stats_struct(out, token_loss is not None, False), s)
         return out, partials
 
     def device_status(self, stream=None) -> int:

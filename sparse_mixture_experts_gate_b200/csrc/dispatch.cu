@@ -13,13 +13,17 @@
 //   count  - per 256-token chunk, a histogram of selections (shared-memory
 //            integer atomics: order-free, so deterministic);
 //   scan   - per expert, exclusive prefix over chunks; kept = min(count, C);
+//            the exclusive scan of the selection counts (pre_start);
 //            exclusive scans of the padded kept counts and of their token
 //            tiles -> segment starts, the 32-row block -> group table, the
 //            token-tile table of the expert GEMM ({group, first row, rows},
 //            at most 256 rows each) and the row and tile counts;
 //   assign - per chunk, the stable rank of each assignment: chunk base +
 //            assignments to the same expert in earlier warps + earlier lanes of
-//            the same warp (a per-warp lane bitmask per expert, popcounted).
+//            the same warp (a per-warp lane bitmask per expert, popcounted);
+//            every selection's gate is also written at pre_start[e] + rank, so
+//            each expert's gates lie together in token order (the importance
+//            statistic sums them in that fixed order).
 // Also the scatter of the routed token rows into the permuted row space, which
 // the tensor-core expert GEMM then reads as plain TMA tiles.
 #include "moe_common.cuh"
@@ -46,6 +50,7 @@ __global__ void __launch_bounds__(kChunk) dispatch_count_kernel(DispatchArgs a) 
 __global__ void __launch_bounds__(kMaxE) dispatch_scan_kernel(DispatchArgs a) {
     __shared__ int sc_rows[kMaxE];
     __shared__ int sc_tiles[kMaxE];
+    __shared__ int sc_pre[kMaxE];
     __shared__ int dropped_w[kMaxE / 32];
     const int e = threadIdx.x, lane = e & 31, warp = e >> 5;
     int pre = 0, kept = 0, padded = 0, tiles = 0;
@@ -71,13 +76,16 @@ __global__ void __launch_bounds__(kMaxE) dispatch_scan_kernel(DispatchArgs a) {
     // (Hillis-Steele in shared memory).
     sc_rows[e] = padded;
     sc_tiles[e] = tiles;
+    sc_pre[e] = pre;
     __syncthreads();
     for (int off = 1; off < kMaxE; off <<= 1) {
         const int vr = e >= off ? sc_rows[e - off] : 0;
         const int vt = e >= off ? sc_tiles[e - off] : 0;
+        const int vp = e >= off ? sc_pre[e - off] : 0;
         __syncthreads();
         sc_rows[e] += vr;
         sc_tiles[e] += vt;
+        sc_pre[e] += vp;
         __syncthreads();
     }
     const int start = sc_rows[e] - padded, tile0 = sc_tiles[e] - tiles;
@@ -92,6 +100,7 @@ __global__ void __launch_bounds__(kMaxE) dispatch_scan_kernel(DispatchArgs a) {
         if (a.user_count_kept) a.user_count_kept[e] = kept;
         a.group_start[e] = start;
         a.group_rows[e] = kept;
+        a.pre_start[e] = sc_pre[e] - pre;
         for (int b = start / kRowBlock; b < (start + padded) / kRowBlock; ++b) a.block_group[b] = e;
         for (int r = start + kept; r < start + padded; ++r) a.row_assign[r] = -1;
         for (int i = 0; i < tiles; ++i)
@@ -149,6 +158,7 @@ __global__ void __launch_bounds__(kChunk) dispatch_assign_kernel(DispatchArgs a)
         const int64_t ai = (int64_t)t * a.k + r;
         const int e = a.idx[ai];
         const int rank = wbase[warp][e] + __popc(mask[warp][e] & lt);
+        a.gate_sorted[a.pre_start[e] + rank] = a.gates[ai];
         const bool kept = (int64_t)rank < a.C;
         a.slot[ai] = kept ? rank : -1;
         int row = -1;

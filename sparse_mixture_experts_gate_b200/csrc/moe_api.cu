@@ -87,7 +87,8 @@ struct Plan {
     int ksplit = 1;
     size_t o_lpart = 0;
     size_t o_ctrl, o_logits, o_idx, o_gates, o_slot, o_rowof, o_lse, o_psum, o_ccount, o_cbase, o_cpre, o_ckept,
-        o_gstart, o_grows, o_bgroup, o_toktiles, o_rowassign, o_wsplit, o_xp, o_h, o_o, o_credit, o_partials;
+        o_gstart, o_grows, o_bgroup, o_toktiles, o_rowassign, o_wsplit, o_xp, o_h, o_o, o_credit, o_partials,
+        o_prestart, o_gsorted;
     size_t total = 0;
 };
 
@@ -165,7 +166,9 @@ Plan make_plan(const moe_layer &L, int T) {
     p.o_bgroup = take((size_t)p.max_row_blocks * 4);
     p.o_toktiles = take((size_t)std::max(p.max_tok_tiles, 1) * 16);
     p.o_rowassign = take((size_t)p.R_max * 4);
-    p.o_partials = take((size_t)(3 * E + 3) * 4);
+    p.o_partials = take((size_t)(4 * E + 3) * 4);
+    p.o_prestart = take((size_t)E * 4);
+    p.o_gsorted = take((size_t)T * k * 4);
     p.o_credit = take((size_t)T * k * 4);
     p.o_wsplit = take(c.dtype == MOE_DTYPE_BF16 ? (size_t)router_tc_epad(E) * 3 * c.input_dim * 2 : 0);
     p.ksplit = c.dtype == MOE_DTYPE_BF16 ? router_tc_ksplit(T, E, c.input_dim, L.num_sms) : 1;
@@ -412,6 +415,9 @@ int moe_forward(moe_layer_t *L, const void *x, int32_t T, const float *logit_noi
     da.slot = slot;
     da.row_of = reinterpret_cast<int32_t *>(ws + p.o_rowof);
     da.row_assign = reinterpret_cast<int32_t *>(ws + p.o_rowassign);
+    da.gates = gates;
+    da.pre_start = reinterpret_cast<int32_t *>(ws + p.o_prestart);
+    da.gate_sorted = reinterpret_cast<float *>(ws + p.o_gsorted);
     MOE_LAUNCH(launch_dispatch(da, s, nl));
     MOE_MARK(L, 2, s);
 
@@ -534,6 +540,8 @@ int enqueue_partials(moe_layer_t *L, const float *token_loss, float *partials, c
     sa.credit = reinterpret_cast<const float *>(ws + p.o_credit);
     sa.token_loss = token_loss;
     sa.ctrl = reinterpret_cast<const int32_t *>(ws + p.o_ctrl);
+    sa.pre_start = reinterpret_cast<const int32_t *>(ws + p.o_prestart);
+    sa.gate_sorted = reinterpret_cast<const float *>(ws + p.o_gsorted);
     sa.T = p.T;
     sa.E = c.num_experts;
     sa.k = c.num_active;
@@ -557,6 +565,10 @@ int enqueue_finalize(moe_layer_t *L, const float *partials, bool has_loss, const
     fa.l_z = out->l_z;
     fa.expert_loss = has_loss ? out->expert_loss : nullptr;
     fa.n_dropped = out->n_dropped;
+    fa.importance = out->importance;
+    fa.cv_load = out->cv_load;
+    fa.cv_importance = out->cv_importance;
+    fa.l_total = out->l_total;
     MOE_LAUNCH(launch_stats_finalize(fa, s, launches));
     return MOE_OK;
 }
@@ -594,7 +606,7 @@ int moe_stat_partials(moe_layer_t *L, const float *token_loss, float *partials, 
     if (!L->has_forward) return fail(MOE_ERR_STATE, "moe_stat_partials called before any moe_forward");
     cudaStream_t s = as_stream(stream_v);
     if (L->plan.T == 0) {
-        MOE_LAUNCH(cudaMemsetAsync(partials, 0, (size_t)(3 * L->cfg.num_experts + 3) * 4, s));
+        MOE_LAUNCH(cudaMemsetAsync(partials, 0, (size_t)(4 * L->cfg.num_experts + 3) * 4, s));
         return MOE_OK;
     }
     int launches = 0;
@@ -609,6 +621,27 @@ int moe_stats_from_partials(moe_layer_t *L, const float *partials, int32_t has_t
     if (!out) return fail(MOE_ERR_INVALID_ARG, "out is NULL");
     int launches = 0;
     return enqueue_finalize(L, partials, has_token_loss != 0, out, as_stream(stream_v), &launches);
+}
+
+int moe_update_selection_bias(moe_layer_t *L, const float *partials, float gamma, float *sel_bias, void *stream_v) {
+    g_last_error.clear();
+    if (!L) return fail(MOE_ERR_INVALID_ARG, "layer is NULL");
+    if (!sel_bias) return fail(MOE_ERR_INVALID_ARG, "sel_bias is NULL");
+    if (gamma != gamma) return fail(MOE_ERR_INVALID_ARG, "gamma is NaN");
+    if (!partials && !L->has_forward)
+        return fail(MOE_ERR_STATE, "moe_update_selection_bias without partials needs a previous moe_forward");
+    BiasUpdateArgs ba;
+    ba.partials = partials;
+    ba.count_pre = partials ? nullptr : reinterpret_cast<const int32_t *>(L->ws + L->plan.o_cpre);
+    ba.T = partials ? 0 : L->plan.T;
+    ba.E = L->cfg.num_experts;
+    ba.k = L->cfg.num_active;
+    ba.gamma = gamma;
+    ba.sel_bias = sel_bias;
+    if (!partials && ba.T == 0) return MOE_OK;
+    int launches = 0;
+    MOE_LAUNCH(launch_bias_update(ba, as_stream(stream_v), &launches));
+    return MOE_OK;
 }
 
 int moe_device_status(moe_layer_t *L, void *stream_v) {

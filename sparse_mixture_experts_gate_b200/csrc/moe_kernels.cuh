@@ -69,6 +69,9 @@ struct DispatchArgs {
     int32_t *slot;          // [T][k]
     int32_t *row_of;        // [T][k]
     int32_t *row_assign;    // [R_max]  t*k + r, or -1 on padding rows
+    const float *gates;     // [T][k]
+    int32_t *pre_start;     // [E]: exclusive scan of count_pre
+    float *gate_sorted;     // [T*k]: every selection's gate, grouped by expert, token order
 };
 cudaError_t launch_dispatch(const DispatchArgs &a, cudaStream_t s, int *launches);
 
@@ -167,19 +170,32 @@ struct StatsArgs {
     const float *credit;      // [T][k]
     const float *token_loss;  // [T] or null
     const int32_t *ctrl;
+    const int32_t *pre_start; // [E]
+    const float *gate_sorted; // [T*k]
     int T, E, k;
-    float *partials;          // [3E + 3] output
+    float *partials;          // [4E + 3] output
 };
 cudaError_t launch_stat_partials(const StatsArgs &a, cudaStream_t s, int *launches);
 
 struct FinalizeArgs {
-    const float *partials;    // [3E + 3]
+    const float *partials;    // [4E + 3]
     int E, k;
     float alpha, beta;
     float *f, *p_mean, *l_aux, *l_z, *expert_loss;  // outputs (nullable)
     int32_t *n_dropped;
+    float *importance, *cv_load, *cv_importance, *l_total;
 };
 cudaError_t launch_stats_finalize(const FinalizeArgs &a, cudaStream_t s, int *launches);
+
+// Aux-loss-free balancing: b_e += gamma sign(k T / E - load_e).
+struct BiasUpdateArgs {
+    const float *partials;     // [4E + 3] (loads and T from the sums) or null
+    const int32_t *count_pre;  // [E], used when partials is null
+    int T, E, k;
+    float gamma;
+    float *sel_bias;           // [E] in place
+};
+cudaError_t launch_bias_update(const BiasUpdateArgs &a, cudaStream_t s, int *launches);
 
 // Sets the calling thread's last-error message; returns `code`.
 int report_error(int code, const char *msg);

@@ -27,6 +27,7 @@ __device__ __forceinline__ float warp_sum(float v) {
 //   [2E]         sum_t lse_t^2          [2E+1]       T
 //   [2E+2]       dropped assignments    [2E+3, 3E+3) sum over kept assignments
 //                                                    of credit * token_loss
+//   [3E+3, 4E+3) importance: sum of the selections' gates per expert
 // One warp per expert; every sum has a fixed order (lane-strided, then a fixed
 // shuffle tree), so repeated runs give bit-identical results.
 __global__ void __launch_bounds__(256) stat_partials_expert_kernel(StatsArgs a) {
@@ -44,10 +45,18 @@ __global__ void __launch_bounds__(256) stat_partials_expert_kernel(StatsArgs a) 
         }
         el = warp_sum(el);
     }
+    // Importance: this expert's selection gates, in token order.
+    float imp = 0.f;
+    {
+        const int g0 = a.pre_start[e], n = a.count_pre[e];
+        for (int j = lane; j < n; j += 32) imp += a.gate_sorted[g0 + j];
+        imp = warp_sum(imp);
+    }
     if (lane == 0) {
         a.partials[e] = ps;
         a.partials[a.E + e] = (float)a.count_pre[e];
         a.partials[2 * a.E + 3 + e] = el;
+        a.partials[3 * a.E + 3 + e] = imp;
     }
 }
 
@@ -68,34 +77,85 @@ __global__ void __launch_bounds__(256) stat_partials_scalar_kernel(StatsArgs a) 
     }
 }
 
+// Sum over the 256 threads of one CTA in a fixed order (shuffle tree, then the
+// eight warp sums in order); every thread gets the result.
+__device__ __forceinline__ float block_sum_256(float v, float *red) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    v = warp_sum(v);
+    __syncthreads();  // `red` may still be read from a previous call
+    if (lane == 0) red[warp] = v;
+    __syncthreads();
+    float t = 0.f;
+#pragma unroll
+    for (int w = 0; w < 8; ++w) t += red[w];
+    return t;
+}
+
+// Squared coefficient of variation of one value per thread (threads >= n hold
+// nothing): population variance over the squared mean, 0 when the mean is 0.
+__device__ __forceinline__ float block_cv_squared(float v, bool valid, int n, float *red) {
+    const float mean = block_sum_256(valid ? v : 0.f, red) / (float)n;
+    const float d = valid ? v - mean : 0.f;
+    const float var = block_sum_256(d * d, red) / (float)n;
+    return mean != 0.f ? var / (mean * mean) : 0.f;
+}
+
 // Statistics from (possibly all-reduced) partial sums: f_i = count_i / (k T),
 // P_i = sum_t P / T, L_aux = alpha E sum_i f_i P_i, L_z = beta sum lse^2 / T,
-// l_i = sum credit * loss / T. One CTA; the L_aux sum is a fixed tree.
+// l_i = sum credit * loss / T, importance_i, the squared coefficients of
+// variation of the loads and of the importances, and L_aux + L_z. One CTA of
+// 256 threads (E <= 256), thread e owns expert e; every sum is a fixed tree.
 __global__ void __launch_bounds__(256) stats_finalize_kernel(FinalizeArgs a) {
     __shared__ float red[8];
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int e = threadIdx.x;
+    const bool own = e < a.E;
     const float T = a.partials[2 * a.E + 1];
     const float inv_t = T > 0.f ? 1.f / T : 0.f;
     const float inv_kt = T > 0.f ? 1.f / ((float)a.k * T) : 0.f;
-    float fp = 0.f;
-    for (int e = tid; e < a.E; e += 256) {
-        const float pm = a.partials[e] * inv_t;
-        const float f = a.partials[a.E + e] * inv_kt;
+    float pm = 0.f, f = 0.f, load = 0.f, imp = 0.f;
+    if (own) {
+        pm = a.partials[e] * inv_t;
+        load = a.partials[a.E + e];
+        f = load * inv_kt;
+        imp = a.partials[3 * a.E + 3 + e];
         if (a.p_mean) a.p_mean[e] = pm;
         if (a.f) a.f[e] = f;
         if (a.expert_loss) a.expert_loss[e] = a.partials[2 * a.E + 3 + e] * inv_t;
-        fp = fmaf(f, pm, fp);
+        if (a.importance) a.importance[e] = imp;
     }
-    fp = warp_sum(fp);
-    if (lane == 0) red[warp] = fp;
-    __syncthreads();
-    if (tid == 0) {
-        float ft = 0.f;
-        for (int w = 0; w < 8; ++w) ft += red[w];
-        if (a.l_aux) *a.l_aux = a.alpha * (float)a.E * ft;
-        if (a.l_z) *a.l_z = a.beta * a.partials[2 * a.E] * inv_t;
+    const float fp = block_sum_256(own ? f * pm : 0.f, red);
+    const float cv_load = block_cv_squared(load, own, a.E, red);
+    const float cv_imp = block_cv_squared(imp, own, a.E, red);
+    if (e == 0) {
+        const float l_aux = a.alpha * (float)a.E * fp;
+        const float l_z = a.beta * a.partials[2 * a.E] * inv_t;
+        if (a.l_aux) *a.l_aux = l_aux;
+        if (a.l_z) *a.l_z = l_z;
+        if (a.l_total) *a.l_total = l_aux + l_z;
         if (a.n_dropped) *a.n_dropped = (int32_t)a.partials[2 * a.E + 2];
+        if (a.cv_load) *a.cv_load = cv_load;
+        if (a.cv_importance) *a.cv_importance = cv_imp;
     }
+}
+
+// Aux-loss-free balancing ("Balancing": per-expert selection bias b_i, update
+// rate gamma): b_e += gamma * sign(k T / E - load_e). The sign is decided on
+// integers (k T - E load_e); gamma * sign is exact, so the one fp32 add is the
+// only rounding. One CTA, thread e owns expert e.
+__global__ void __launch_bounds__(256) bias_update_kernel(BiasUpdateArgs a) {
+    const int e = threadIdx.x;
+    if (e >= a.E) return;
+    int64_t load, T;
+    if (a.partials) {
+        load = (int64_t)a.partials[a.E + e];
+        T = (int64_t)a.partials[2 * a.E + 1];
+    } else {
+        load = a.count_pre[e];
+        T = a.T;
+    }
+    const int64_t diff = (int64_t)a.k * T - (int64_t)a.E * load;
+    const float sgn = diff > 0 ? 1.f : (diff < 0 ? -1.f : 0.f);
+    a.sel_bias[e] = __fadd_rn(a.sel_bias[e], a.gamma * sgn);
 }
 
 }  // namespace
@@ -109,6 +169,12 @@ cudaError_t launch_stat_partials(const StatsArgs &a, cudaStream_t s, int *launch
 
 cudaError_t launch_stats_finalize(const FinalizeArgs &a, cudaStream_t s, int *launches) {
     stats_finalize_kernel<<<1, 256, 0, s>>>(a);
+    *launches += 1;
+    return cudaGetLastError();
+}
+
+cudaError_t launch_bias_update(const BiasUpdateArgs &a, cudaStream_t s, int *launches) {
+    bias_update_kernel<<<1, 256, 0, s>>>(a);
     *launches += 1;
     return cudaGetLastError();
 }

@@ -91,6 +91,15 @@ def check_same_logits_routing(w, inp, g):
     assert np.abs(g["p_mean"] - pm).max() <= STAT_TOL
     assert abs(g["l_aux"][0] - la) <= STAT_TOL
     assert abs(g["l_z"][0] - lz) <= STAT_TOL
+    # Load-balancing extras: importance from the GPU's own gates (fp32 sums of
+    # fp32 gates), the CVs of counts and importances, the weighted total.
+    imp = oracle.importance(g["topk_idx"], g["gates"], w.E)
+    assert np.abs(g["importance"] - imp).max() <= STAT_TOL * (1 + np.abs(imp).max()), "importance"
+    cvl = oracle.cv_squared(r["count_pre"])
+    assert abs(g["cv_load"][0] - cvl) <= STAT_TOL * (1 + cvl), "cv of the loads"
+    cvi = oracle.cv_squared(imp)
+    assert abs(g["cv_importance"][0] - cvi) <= STAT_TOL * (1 + cvi), "cv of the importances"
+    assert np.float32(g["l_total"][0]) == np.float32(np.float32(g["l_aux"][0]) + np.float32(g["l_z"][0]))
     return r
 
 

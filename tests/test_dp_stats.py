@@ -42,12 +42,13 @@ def shard_partials(w, inp, lo: int, hi: int) -> np.ndarray:
     shard = {k: (v[lo:hi] if (v is not None and k in ("x", "noise", "token_loss")) else v) for k, v in inp.items()}
     o = oracle.forward(w, shard)
     E = w.E
-    p = np.zeros(3 * E + 3, np.float64)
+    p = np.zeros(4 * E + 3, np.float64)
     p[:E] = o["P"].sum(axis=0)
     p[E:2 * E] = o["count_pre"]
     p[2 * E] = float((o["lse"] ** 2).sum())
     p[2 * E + 1] = hi - lo
     p[2 * E + 2] = o["n_dropped"]
+    p[3 * E + 3:] = oracle.importance(o["idx"], o["gates"], E)
     tl = shard["token_loss"].double().numpy()
     for t in range(hi - lo):
         for r in range(w.k):
@@ -60,8 +61,12 @@ def stats_from_partials(p: np.ndarray, E: int, k: int, alpha: float, beta: float
     T = p[2 * E + 1]
     pm = p[:E] / T
     f = p[E:2 * E] / (k * T)
-    return dict(f=f, p_mean=pm, l_aux=alpha * E * float((f * pm).sum()), l_z=beta * p[2 * E] / T,
-                n_dropped=int(p[2 * E + 2]), expert_loss=p[2 * E + 3:] / T)
+    import oracle
+    l_aux, l_z = alpha * E * float((f * pm).sum()), beta * p[2 * E] / T
+    imp = p[3 * E + 3:]
+    return dict(f=f, p_mean=pm, l_aux=l_aux, l_z=l_z, l_total=l_aux + l_z, n_dropped=int(p[2 * E + 2]),
+                expert_loss=p[2 * E + 3:3 * E + 3] / T, importance=imp,
+                cv_load=oracle.cv_squared(p[E:2 * E]), cv_importance=oracle.cv_squared(imp))
 
 
 def _rank_main(rank: int, port: int, result_dir: str):
@@ -104,6 +109,10 @@ def test_dp_stats_two_gloo_ranks(tmp_path):
     assert np.allclose(dp["p_mean"], whole["p_mean"], rtol=0, atol=1e-12)
     assert abs(dp["l_aux"] - whole["l_aux"]) <= 1e-12
     assert abs(dp["l_z"] - whole["l_z"]) <= 1e-12
+    imp_whole = oracle.importance(whole["idx"], whole["gates"], w.E)
+    assert np.allclose(dp["importance"], imp_whole, rtol=1e-12, atol=1e-12)
+    assert abs(dp["cv_load"] - oracle.cv_squared(whole["count_pre"])) <= 1e-12
+    assert abs(dp["cv_importance"] - oracle.cv_squared(imp_whole)) <= 1e-12
     # Capacity is per shard, so drops and the attributed loss follow each
     # shard's own dispatch, divided by the whole batch's size.
     cuts = _bounds(w.T, WORLD)

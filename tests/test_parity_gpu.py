@@ -210,12 +210,12 @@ def test_dp_stats_two_shards_through_kernels():
     out = layer.alloc_outputs(1)
     for v in out.values():
         v.fill_(-7)
-    st = MoeStats(out["f"].data_ptr(), out["p_mean"].data_ptr(), out["l_aux"].data_ptr(), out["l_z"].data_ptr(),
-                  out["n_dropped"].data_ptr(), None, out["expert_loss"].data_ptr())
+    st = MoELayer._stats_struct(out, True, False)
     moe_stats_from_partials(layer.handle, total.data_ptr(), True, st, s)
     torch.cuda.synchronize()
     dp = {k: out[k].cpu().numpy().astype(np.float64) for k in ("f", "p_mean", "l_aux", "l_z", "n_dropped",
-                                                               "expert_loss")}
+                                                               "expert_loss", "importance", "cv_load",
+                                                               "cv_importance")}
 
     # Same-logits oracle routing of the whole batch from the GPU's logits.
     logits = np.concatenate([g["logits"] for g in shards]).astype(np.float32)
@@ -226,6 +226,11 @@ def test_dp_stats_two_shards_through_kernels():
     assert abs(dp["l_aux"][0] - la) <= 1e-4
     assert abs(dp["l_z"][0] - lz) <= 1e-4
     assert int(dp["n_dropped"][0]) == sum(int(g["n_dropped"][0]) for g in shards)
+    imp = oracle.importance(np.concatenate([g["topk_idx"] for g in shards]),
+                            np.concatenate([g["gates"] for g in shards]), w.E)
+    assert np.abs(dp["importance"] - imp).max() <= 1e-4 * (1 + imp.max())
+    assert abs(dp["cv_load"][0] - oracle.cv_squared(r["count_pre"])) <= 1e-4
+    assert abs(dp["cv_importance"][0] - oracle.cv_squared(imp)) <= 1e-4
     el = oracle.expert_loss(np.concatenate([g["topk_idx"] for g in shards]),
                             np.concatenate([g["slot"] for g in shards]),
                             np.concatenate([g["credit"] for g in shards]), inp["token_loss"], w.E)
@@ -247,3 +252,39 @@ def test_ragged_n_tiles_both_layers():
     also carries the credit's norm partials (O = 320)."""
     w = WORKLOADS["default"].with_(T=777, F=1088, O=320, S=1, activation="swish")
     full_check(w, make_inputs(w, "cpu", seed=13, random_biases=True))
+
+
+def test_selection_bias_update_bit_exact():
+    """Aux-loss-free balancing ("Balancing": b_i with update rate gamma): the
+    update from this forward's loads and the one from summed partials of two
+    shards match the oracle's update on the same loads bit for bit, and the
+    next forward selects with the updated bias."""
+    from sparse_mixture_experts_gate_b200.binding import moe_stat_partials, stat_partials_size
+    w = WORKLOADS["e64"].with_(T=900)
+    inp = make_inputs(w, "cpu", seed=31)
+    g, layer = run_gpu(w, inp)
+    b0 = layer.weights["sel_bias"].cpu().numpy().copy()
+    layer.update_selection_bias(1e-3)
+    torch.cuda.synchronize()
+    want = oracle.selection_bias_update(b0, g["count_pre"], w.k, w.T, 1e-3)
+    assert np.array_equal(layer.weights["sel_bias"].cpu().numpy(), want)
+    # From the partial sums of two shards (the data-parallel path).
+    b1 = layer.weights["sel_bias"].cpu().numpy().copy()
+    total = torch.zeros(stat_partials_size(w.E), device="cuda")
+    loads = np.zeros(w.E, np.int64)
+    s = torch.cuda.current_stream().cuda_stream
+    for lo, hi in ((0, 500), (500, w.T)):
+        sub = {k: (v[lo:hi] if (v is not None and k in ("x", "noise", "token_loss")) else v) for k, v in inp.items()}
+        gs, _ = run_gpu(w.with_(T=hi - lo), sub, layer=layer)
+        part = torch.empty(stat_partials_size(w.E), device="cuda")
+        moe_stat_partials(layer.handle, None, part.data_ptr(), s)
+        total += part
+        loads += gs["count_pre"]
+    layer.update_selection_bias(-2e-3, partials=total)
+    torch.cuda.synchronize()
+    want = oracle.selection_bias_update(b1, loads, w.k, w.T, -2e-3)
+    assert np.array_equal(layer.weights["sel_bias"].cpu().numpy(), want)
+    # The next forward routes with the updated bias (same-logits check).
+    inp2 = dict(inp, sel_bias=layer.weights["sel_bias"].cpu())
+    g2, _ = run_gpu(w, inp2, layer=layer)
+    check_same_logits_routing(w, inp2, g2)
