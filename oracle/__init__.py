@@ -61,6 +61,10 @@ def _configure(L):
     L.orc_balance_stats.argtypes = [i32, i32, i32, vp, vp, vp, dbl, dbl, vp, vp, vp, vp]
     L.orc_expert_loss.argtypes = [i32, i32, i32, vp, vp, vp, vp, vp]
     L.orc_importance.argtypes = [i32, i32, i32, vp, vp, vp]
+    L.orc_experts_credit_hidden.argtypes = [i32, vp, i32, i32, i32, i32, i32, i32, i32, vp,
+                                            ctypes.POINTER(Expert), vp, vp, vp, vp]
+    L.orc_dro_update.argtypes = [i32, dbl, dbl, vp, vp, vp]
+    L.orc_dro_update.restype = dbl
     L.orc_cv_squared.argtypes = [i32, vp]
     L.orc_cv_squared.restype = dbl
     L.orc_selection_bias_update.argtypes = [i32, i32, i64, vp, ctypes.c_float, vp]
@@ -243,6 +247,30 @@ def experts_combine(tokens: Sequence[int], x, table: ExpertTable, idx, slot, g,
     lib().orc_experts_combine(n, _p(tok), T, d, F, O, E, S, k, ACT[act], xd, table.w_dtype,
                               _p(xs), table.arr, _p(idx), _p(slot), _p(g), _p(y), _p(cr))
     return y, cr
+
+
+def experts_credit_hidden(tokens: Sequence[int], x, table: ExpertTable, idx, slot, g, d: int, F: int, E: int,
+                          act: str) -> np.ndarray:
+    """Credit g * ||act(w1 x + b1)|| of each kept assignment (the hidden-activation reading)."""
+    xs, xd = as_storage(x)
+    idx = np.ascontiguousarray(idx, dtype=np.int32)
+    slot = np.ascontiguousarray(slot, dtype=np.int32)
+    g = np.ascontiguousarray(g, dtype=np.float64)
+    k = idx.shape[1]
+    tok = np.ascontiguousarray(np.asarray(tokens, dtype=np.int32))
+    cr = np.empty((tok.shape[0], k), np.float64)
+    lib().orc_experts_credit_hidden(tok.shape[0], _p(tok), d, F, E, k, ACT[act], xd, table.w_dtype, _p(xs),
+                                    table.arr, _p(idx), _p(slot), _p(g), _p(cr))
+    return cr
+
+
+def dro_update(l, lhat, mu, ema: float, eta: float):
+    """EMA of the expert losses, mu <- softmax(mu + eta lhat), and sum_i mu_i l_i."""
+    l = np.ascontiguousarray(l, dtype=np.float64)
+    lh = np.ascontiguousarray(np.array(lhat, dtype=np.float64).copy())
+    m = np.ascontiguousarray(np.array(mu, dtype=np.float64).copy())
+    obj = lib().orc_dro_update(int(l.size), float(ema), float(eta), _p(l), _p(lh), _p(m))
+    return lh, m, float(obj)
 
 
 def balance_stats(P, lse, count_pre, k: int, alpha: float, beta: float):

@@ -156,11 +156,10 @@ static double activation(int act, double z)
     }
 }
 
-/* SER walkthrough: an expert's two-layer MLP, w1/b1 -> activation -> w2/b2. */
-void orc_expert_ffn(int d, int F, int O, int act, int w_dtype, const orc_expert *ex,
-                    const double *x, double *o)
+/* SER walkthrough: the first half of an expert's MLP, a = act(w1 x + b1). */
+static void expert_hidden(int d, int F, int act, int w_dtype, const orc_expert *ex, const double *x,
+                          double *a)
 {
-    double *a = (double *)malloc(sizeof(double) * (size_t)F);
     for (int f = 0; f < F; ++f) {
         double z = 0.0;
         for (int j = 0; j < d; ++j)
@@ -169,6 +168,14 @@ void orc_expert_ffn(int d, int F, int O, int act, int w_dtype, const orc_expert 
             z += (double)ex->b1[f];
         a[f] = activation(act, z);
     }
+}
+
+/* SER walkthrough: an expert's two-layer MLP, w1/b1 -> activation -> w2/b2. */
+void orc_expert_ffn(int d, int F, int O, int act, int w_dtype, const orc_expert *ex,
+                    const double *x, double *o)
+{
+    double *a = (double *)malloc(sizeof(double) * (size_t)F);
+    expert_hidden(d, F, act, w_dtype, ex, x, a);
     for (int n = 0; n < O; ++n) {
         double s = 0.0;
         for (int f = 0; f < F; ++f)
@@ -222,6 +229,59 @@ void orc_experts_combine(int n_tokens, const int32_t *tokens, int T, int d, int 
         free(o);
         free(xt);
     }
+}
+
+/* Credit diagram, panel (b), with ||h|| read as the hidden activation's norm. */
+void orc_experts_credit_hidden(int n_tokens, const int32_t *tokens, int d, int F, int E, int k,
+                               int act, int x_dtype, int w_dtype, const void *x,
+                               const orc_expert *experts, const int32_t *idx, const int32_t *slot,
+                               const double *g, double *credit)
+{
+    (void)E;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int j = 0; j < n_tokens; ++j) {
+        int t = tokens[j];
+        double *xt = (double *)malloc(sizeof(double) * (size_t)d);
+        double *a = (double *)malloc(sizeof(double) * (size_t)F);
+        for (int c = 0; c < d; ++c)
+            xt[c] = orc_load(x, (int64_t)t * d + c, x_dtype);
+        for (int r = 0; r < k; ++r) {
+            int64_t as = (int64_t)t * k + r;
+            double c = 0.0;
+            if (slot[as] >= 0) {
+                expert_hidden(d, F, act, w_dtype, &experts[idx[as]], xt, a);
+                double ss = 0.0;
+                for (int f = 0; f < F; ++f)
+                    ss += a[f] * a[f];
+                c = g[as] * sqrt(ss);
+            }
+            credit[(int64_t)j * k + r] = c;
+        }
+        free(a);
+        free(xt);
+    }
+}
+
+/* Credit diagram, panel (c): EMA of the expert losses, mu <- softmax(mu + eta lhat),
+ * and sum_i mu_i l_i. */
+double orc_dro_update(int E, double ema, double eta, const double *l, double *lhat, double *mu)
+{
+    double m = -INFINITY;
+    for (int i = 0; i < E; ++i) {
+        lhat[i] = ema * lhat[i] + (1.0 - ema) * l[i];
+        const double z = mu[i] + eta * lhat[i];
+        if (z > m)
+            m = z;
+    }
+    double s = 0.0;
+    for (int i = 0; i < E; ++i)
+        s += exp(mu[i] + eta * lhat[i] - m);
+    double obj = 0.0;
+    for (int i = 0; i < E; ++i) {
+        mu[i] = exp(mu[i] + eta * lhat[i] - m) / s;
+        obj += mu[i] * l[i];
+    }
+    return obj;
 }
 
 /* Appendix C, "Balancing": f_i, P_i, L_aux = alpha E sum_i f_i P_i and the router

@@ -115,6 +115,22 @@ void orc_experts_combine(int n_tokens, const int32_t *tokens, int T, int d, int 
                          const void *x, const orc_expert *experts, const int32_t *idx,
                          const int32_t *slot, const double *g, double *y, double *credit);
 
+/* [D] panel (b), second reading of ||h_{l,i}||: the norm of expert i's hidden
+ * activation a = act(w1 x + b1) (length F) instead of its output. For each listed
+ * token t = tokens[j]: credit[j][r] = g[t][r] * ||a_{idx[t][r]}(x_t)||_2 if kept,
+ * else 0. Arguments as orc_experts_combine. */
+void orc_experts_credit_hidden(int n_tokens, const int32_t *tokens, int d, int F, int E, int k,
+                               int act, int x_dtype, int w_dtype, const void *x,
+                               const orc_expert *experts, const int32_t *idx, const int32_t *slot,
+                               const double *g, double *credit);
+
+/* [D] panel (c), the layer-wise bookkeeping: the EMA tracker
+ *   lhat_i <- ema * lhat_i + (1 - ema) * l_i,
+ * the expert weights mu <- softmax(mu + eta * lhat) (mu as printed, not its log),
+ * and the objective term of this layer sum_i mu_i l_i with the updated mu.
+ * l [E]; lhat, mu [E] updated in place; returns the objective term. */
+double orc_dro_update(int E, double ema, double eta, const double *l, double *lhat, double *mu);
+
 /* [C] "Balancing": f_i = fraction of the batch's selections dispatched to expert
  * i (count_pre_i / (k T)), P_i = mean_t P[t][i], L_aux = alpha E sum_i f_i P_i,
  * L_z = beta mean_t lse_t^2. */

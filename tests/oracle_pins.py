@@ -451,6 +451,47 @@ def check_selection_bias_update():
     assert np.array_equal(b1, want.astype(np.float32))
 
 
+def check_credit_hidden_dense():
+    """[D] panel (b), hidden-activation reading: with E = 1, k = 1 the credit is
+    g * ||act(w1 x + b1)||_2 of the one expert, checked against torch fp64 for
+    every activation; a dropped assignment has credit 0."""
+    for act in ("relu", "gelu", "swish"):
+        w = WORKLOADS["tiny"].with_(T=6, d=12, F=20, O=8, E=1, k=1, S=0, activation=act, dtype="fp32")
+        inp = make_inputs(w, "cpu", seed=8, random_biases=True)
+        table = oracle.ExpertTable(1, inp["w1"], inp["b1"], inp["w2"], inp["b2"])
+        idx = np.zeros((w.T, 1), np.int32)
+        slot = np.zeros((w.T, 1), np.int32)
+        slot[2, 0] = -1
+        g = np.linspace(0.5, 1.0, w.T).reshape(w.T, 1)
+        cr = oracle.experts_credit_hidden(range(w.T), inp["x"], table, idx, slot, g, w.d, w.F, w.E, act)
+        x = inp["x"].double()
+        z = x @ inp["w1"][0].double().T + inp["b1"][0].double()
+        a = {"relu": torch.relu, "gelu": lambda v: torch.nn.functional.gelu(v), "swish": torch.nn.functional.silu}[act](z)
+        want = g[:, 0] * torch.linalg.vector_norm(a, dim=1).numpy()
+        want[2] = 0.0
+        assert np.allclose(cr[:, 0], want, rtol=1e-12, atol=1e-14)
+
+
+def check_dro_update():
+    """[D] panel (c): ema = 0 tracks the loss, ema = 1 keeps the tracker; eta = 0
+    with uniform weights keeps them uniform; two experts give the logistic
+    closed form; the weights sum to 1 and the objective is sum mu_i l_i."""
+    l = np.array([0.3, 1.2, 0.7, 0.1])
+    lh0 = np.array([0.5, 0.5, 0.5, 0.5])
+    lh, _, _ = oracle.dro_update(l, lh0, np.full(4, 0.25), 0.0, 1.0)
+    assert np.allclose(lh, l, rtol=0, atol=0)
+    lh, _, _ = oracle.dro_update(l, lh0, np.full(4, 0.25), 1.0, 1.0)
+    assert np.array_equal(lh, lh0)
+    _, mu, obj = oracle.dro_update(l, lh0, np.full(4, 0.25), 0.9, 0.0)
+    assert np.allclose(mu, 0.25, rtol=0, atol=1e-15) and abs(obj - l.mean()) < 1e-15
+    l2, lh2, mu2, ema, eta = np.array([2.0, 0.5]), np.array([1.0, 3.0]), np.array([0.4, 0.6]), 0.8, 1.7
+    lh_new = ema * lh2 + (1 - ema) * l2
+    p0 = 1.0 / (1.0 + math.exp(-((mu2[0] + eta * lh_new[0]) - (mu2[1] + eta * lh_new[1]))))
+    lh_o, mu_o, obj = oracle.dro_update(l2, lh2, mu2, ema, eta)
+    assert abs(mu_o[0] - p0) < 1e-14 and abs(mu_o.sum() - 1.0) < 1e-15
+    assert abs(obj - (mu_o[0] * l2[0] + mu_o[1] * l2[1])) < 1e-15
+
+
 def check_minimal_example_shapes():
     """[W] "Minimal example": 4 experts, 2 active, dims 8/16/8, a (4, 8) input;
     the forward yields a (4, 8) output, 2 distinct experts per token, gates

@@ -45,6 +45,10 @@ MUTANTS = {
     "bias_update_sign": ("const double s = diff > 0 ? 1.0 : (diff < 0 ? -1.0 : 0.0);",
                          "const double s = diff > 0 ? -1.0 : (diff < 0 ? 1.0 : 0.0);"),
     "bias_update_mean_off": ("(int64_t)k * T - (int64_t)E * load[i]", "(int64_t)T - (int64_t)E * load[i]"),
+    "hidden_credit_drops_gate": ("c = g[as] * sqrt(ss);", "c = sqrt(ss);"),
+    "dro_ema_swapped": ("lhat[i] = ema * lhat[i] + (1.0 - ema) * l[i];", "lhat[i] = (1.0 - ema) * lhat[i] + ema * l[i];"),
+    "dro_eta_dropped": ("s += exp(mu[i] + eta * lhat[i] - m);", "s += exp(mu[i] - m);"),
+    "dro_objective_old_mu": ("obj += mu[i] * l[i];", "obj += lhat[i] * l[i];"),
     "softmax_wrong_exponent": ("P[(int64_t)t * E + i] = exp(ht[i] - m) / z;",
                                "P[(int64_t)t * E + i] = exp(ht[i]) / z;"),
 }
