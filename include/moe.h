@@ -69,6 +69,11 @@ enum { MOE_TOPK_GREEDY = 0, MOE_TOPK_NOISY = 1 };
  * FP32 runs them on fp32 CUDA cores. */
 enum { MOE_DTYPE_BF16 = 0, MOE_DTYPE_FP32 = 1 };
 
+/* Which vector's norm the expert credit c = g ||h||_2 uses ("Sparse MoE
+ * Expert-Credit Loss Reweighting Diagram", panel (b)): the expert's output
+ * (default) or its hidden activation act(w1 x + b1). */
+enum { MOE_CREDIT_OUTPUT = 0, MOE_CREDIT_HIDDEN = 1 };
+
 /* Layer configuration. Field names follow the SER walkthrough's configuration
  * (num_experts, num_active, input_dim, expert_dim, output_dim, top_k_method,
  * load_balance_coef); the remaining fields carry Appendix C's symbols. */
@@ -88,6 +93,7 @@ typedef struct {
     float load_balance_coef;  /* alpha of L_aux                                     */
     float z_loss_coef;        /* beta of the z-loss                                 */
     float temperature;        /* router softmax temperature; only 1 is supported   */
+    int32_t credit_norm;      /* MOE_CREDIT_*                                       */
 } moe_config_t;
 
 /* Defaults of the SER walkthrough's configuration: E=8, k=2, 512/1024/512,
@@ -270,6 +276,17 @@ MOE_API int moe_stats_from_partials(moe_layer_t *layer, const float *partials, i
  * INVALID_ARG (NULL sel_bias, NaN gamma), STATE (no partials and no forward). */
 MOE_API int moe_update_selection_bias(moe_layer_t *layer, const float *partials, float gamma, float *sel_bias,
                                       void *stream);
+
+/* Layer-wise reweighting bookkeeping ("Sparse MoE Expert-Credit Loss
+ * Reweighting Diagram", panel (c)), enqueued on `stream` for one layer:
+ *     lhat_e <- ema * lhat_e + (1 - ema) * expert_loss_e
+ *     mu     <- softmax(mu + eta * lhat)          (mu as printed, not its log)
+ *     *objective = sum_e mu_e * expert_loss_e     (updated mu; NULL to skip)
+ * expert_loss: device [E] fp32 (e.g. moe_stats_t.expert_loss); lhat, mu: device
+ * [E] fp32, updated in place; objective: device [1] fp32 or NULL. fp32, fixed
+ * reduction order. Errors: INVALID_ARG for NULL arrays or non-finite ema/eta. */
+MOE_API int moe_dro_update(moe_layer_t *layer, const float *expert_loss, float ema, float eta, float *lhat,
+                           float *mu, float *objective, void *stream);
 
 /* Device status word of the most recent forward: synchronises `stream`, then
  * returns MOE_OK, or MOE_ERR_TIMEOUT if a bounded device-side wait gave up. */

@@ -18,11 +18,12 @@ MOE_ERR_WORKSPACE, MOE_ERR_TIMEOUT, MOE_ERR_STATE = -4, -5, -6
 MOE_ACT = {"relu": 0, "gelu": 1, "swish": 2}
 MOE_TOPK = {"greedy": 0, "noisy": 1}
 MOE_DTYPE = {"bf16": 0, "fp32": 1}
+MOE_CREDIT = {"output": 0, "hidden": 1}
 
 # Every symbol include/moe.h declares.
 EXPORTS = ("moe_config_default", "moe_layer_create", "moe_workspace_bytes", "moe_capacity", "moe_forward",
            "moe_forward_noalloc", "moe_aux_stats", "moe_stat_partials", "moe_stats_from_partials",
-           "moe_update_selection_bias", "moe_device_status", "moe_set_timing_events", "moe_launch_count", "moe_destroy", "moe_status_string",
+           "moe_update_selection_bias", "moe_dro_update", "moe_device_status", "moe_set_timing_events", "moe_launch_count", "moe_destroy", "moe_status_string",
            "moe_last_error")
 
 
@@ -32,7 +33,7 @@ class MoeConfig(ctypes.Structure):
                 ("capacity_factor", ctypes.c_float), ("activation", ctypes.c_int32),
                 ("top_k_method", ctypes.c_int32), ("use_selection_bias", ctypes.c_int32),
                 ("dtype", ctypes.c_int32), ("max_tokens", ctypes.c_int32), ("load_balance_coef", ctypes.c_float),
-                ("z_loss_coef", ctypes.c_float), ("temperature", ctypes.c_float)]
+                ("z_loss_coef", ctypes.c_float), ("temperature", ctypes.c_float), ("credit_norm", ctypes.c_int32)]
 
 
 class MoeWeights(ctypes.Structure):
@@ -90,6 +91,8 @@ def lib() -> ctypes.CDLL:
         L.moe_stats_from_partials.argtypes = [vp, vp, i32, ctypes.POINTER(MoeStats), vp]
         L.moe_update_selection_bias.restype = ctypes.c_int
         L.moe_update_selection_bias.argtypes = [vp, vp, ctypes.c_float, vp, vp]
+        L.moe_dro_update.restype = ctypes.c_int
+        L.moe_dro_update.argtypes = [vp, vp, ctypes.c_float, ctypes.c_float, vp, vp, vp, vp]
         L.moe_device_status.restype = ctypes.c_int
         L.moe_device_status.argtypes = [vp, vp]
         L.moe_set_timing_events.restype = ctypes.c_int
@@ -187,6 +190,12 @@ def allreduce_partials(partials, group=None):
     return partials
 
 
+def moe_dro_update(layer: int, expert_loss: int, ema: float, eta: float, lhat: int, mu: int,
+                   objective: Optional[int], stream: int) -> int:
+    return _check(lib().moe_dro_update(layer, expert_loss, float(ema), float(eta), lhat, mu, objective, stream),
+                  "moe_dro_update")
+
+
 def moe_device_status(layer: int, stream: int) -> int:
     return int(lib().moe_device_status(layer, stream))
 
@@ -238,6 +247,7 @@ class MoELayer:
         cfg.dtype = MOE_DTYPE[w.dtype]
         cfg.max_tokens = max_tokens or 0
         cfg.load_balance_coef, cfg.z_loss_coef, cfg.temperature = w.alpha, w.beta, 1.0
+        cfg.credit_norm = MOE_CREDIT[w.credit_norm]
         self.cfg = cfg
         self.weights = {k: (v.to(self.device).contiguous() if v is not None else None)
                         for k, v in weights.items()

@@ -150,7 +150,7 @@ __global__ void __launch_bounds__(kWarps * 32, 2) combine_kernel(CombineArgs a) 
         float v = ss[r];
 #pragma unroll
         for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
-        if (lane == r && rrow[r] >= 0) credit = rg[r] * sqrtf(v);
+        if (lane == r && rrow[r] >= 0) credit = rg[r] * sqrtf(a.row_norm2 ? a.row_norm2[rrow[r]] : v);
     }
     if (lane < k) a.credit[(int64_t)t * k + lane] = credit;
 }

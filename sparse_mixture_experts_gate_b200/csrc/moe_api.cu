@@ -88,7 +88,7 @@ struct Plan {
     size_t o_lpart = 0;
     size_t o_ctrl, o_logits, o_idx, o_gates, o_slot, o_rowof, o_lse, o_psum, o_ccount, o_cbase, o_cpre, o_ckept,
         o_gstart, o_grows, o_bgroup, o_toktiles, o_rowassign, o_wsplit, o_xp, o_h, o_o, o_credit, o_partials,
-        o_prestart, o_gsorted;
+        o_prestart, o_gsorted, o_rownorm;
     size_t total = 0;
 };
 
@@ -169,6 +169,7 @@ Plan make_plan(const moe_layer &L, int T) {
     p.o_partials = take((size_t)(4 * E + 3) * 4);
     p.o_prestart = take((size_t)E * 4);
     p.o_gsorted = take((size_t)T * k * 4);
+    p.o_rownorm = take(c.credit_norm == MOE_CREDIT_HIDDEN ? (size_t)p.R_routed_max * 4 : 0);
     p.o_credit = take((size_t)T * k * 4);
     p.o_wsplit = take(c.dtype == MOE_DTYPE_BF16 ? (size_t)router_tc_epad(E) * 3 * c.input_dim * 2 : 0);
     p.ksplit = c.dtype == MOE_DTYPE_BF16 ? router_tc_ksplit(T, E, c.input_dim, L.num_sms) : 1;
@@ -204,6 +205,8 @@ int validate_config(const moe_config_t *c, const moe_weights_t *w) {
     if (!(c->temperature == 1.0f))
         return fail(MOE_ERR_UNSUPPORTED, "router temperature other than 1 is not supported");
     if (c->capacity_factor != c->capacity_factor) return fail(MOE_ERR_INVALID_ARG, "capacity_factor is NaN");
+    if (c->credit_norm != MOE_CREDIT_OUTPUT && c->credit_norm != MOE_CREDIT_HIDDEN)
+        return fail(MOE_ERR_INVALID_ARG, "unknown credit_norm %d", c->credit_norm);
     if (!w->w_gate) return fail(MOE_ERR_INVALID_ARG, "weights->w_gate is NULL");
     if (!w->w1) return fail(MOE_ERR_INVALID_ARG, "weights->w1 is NULL");
     if (!w->w2) return fail(MOE_ERR_INVALID_ARG, "weights->w2 is NULL");
@@ -502,8 +505,22 @@ int moe_forward(moe_layer_t *L, const void *x, int32_t T, const float *logit_noi
         MOE_MARK(L, 4, s);
     }
 
+    float *row_norm2 = nullptr;
+    if (c.credit_norm == MOE_CREDIT_HIDDEN) {
+        RowNormArgs rn;
+        rn.m = ws + p.o_h;
+        rn.n = c.expert_dim;
+        rn.bf16 = L->tc ? 1 : 0;
+        rn.row_assign = da.row_assign;
+        rn.ctrl = ctrl;
+        rn.max_rows = p.R_routed_max;
+        rn.norm2 = row_norm2 = reinterpret_cast<float *>(ws + p.o_rownorm);
+        MOE_LAUNCH(launch_row_norms(rn, L->num_sms, s, nl));
+    }
+
     CombineArgs ca;
     ca.o = ws + p.o_o;
+    ca.row_norm2 = row_norm2;
     ca.row_of = da.row_of;
     ca.gates = gates;
     ca.group_start = da.group_start;
@@ -641,6 +658,25 @@ int moe_update_selection_bias(moe_layer_t *L, const float *partials, float gamma
     if (!partials && ba.T == 0) return MOE_OK;
     int launches = 0;
     MOE_LAUNCH(launch_bias_update(ba, as_stream(stream_v), &launches));
+    return MOE_OK;
+}
+
+int moe_dro_update(moe_layer_t *L, const float *expert_loss, float ema, float eta, float *lhat, float *mu,
+                   float *objective, void *stream_v) {
+    g_last_error.clear();
+    if (!L) return fail(MOE_ERR_INVALID_ARG, "layer is NULL");
+    if (!expert_loss || !lhat || !mu) return fail(MOE_ERR_INVALID_ARG, "expert_loss, lhat and mu are required");
+    if (!std::isfinite(ema) || !std::isfinite(eta)) return fail(MOE_ERR_INVALID_ARG, "ema and eta must be finite");
+    DroArgs da;
+    da.l = expert_loss;
+    da.lhat = lhat;
+    da.mu = mu;
+    da.objective = objective;
+    da.E = L->cfg.num_experts;
+    da.ema = ema;
+    da.eta = eta;
+    int launches = 0;
+    MOE_LAUNCH(launch_dro_update(da, as_stream(stream_v), &launches));
     return MOE_OK;
 }
 

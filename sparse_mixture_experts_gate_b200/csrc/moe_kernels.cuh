@@ -148,6 +148,7 @@ cudaError_t launch_gemm_simt(const GemmSimtArgs &a, cudaStream_t s, int *launche
 // Gate-weighted combine with shared experts, plus credit.
 struct CombineArgs {
     const void *o;          // [rows][O] expert outputs
+    const float *row_norm2; // [rows] squared norms the credit uses instead of ||o||^2, or null
     const int32_t *row_of;  // [T][k]
     const float *gates;     // [T][k]
     const int32_t *group_start;
@@ -186,6 +187,28 @@ struct FinalizeArgs {
     float *importance, *cv_load, *cv_importance, *l_total;
 };
 cudaError_t launch_stats_finalize(const FinalizeArgs &a, cudaStream_t s, int *launches);
+
+// Squared norms of the routed rows of a [rows][n] matrix (H, for the credit's
+// hidden-activation reading); padding rows are skipped.
+struct RowNormArgs {
+    const void *m;
+    int n, bf16;
+    const int32_t *row_assign;  // [rows], -1 on padding rows
+    const int32_t *ctrl;        // kCtrlRoutedRows
+    int max_rows;
+    float *norm2;               // [rows]
+};
+cudaError_t launch_row_norms(const RowNormArgs &a, int num_sms, cudaStream_t s, int *launches);
+
+// Panel (c) bookkeeping: EMA of the expert losses, mu <- softmax(mu + eta lhat),
+// objective sum mu l.
+struct DroArgs {
+    const float *l;
+    float *lhat, *mu, *objective;
+    int E;
+    float ema, eta;
+};
+cudaError_t launch_dro_update(const DroArgs &a, cudaStream_t s, int *launches);
 
 // Aux-loss-free balancing: b_e += gamma sign(k T / E - load_e).
 struct BiasUpdateArgs {

@@ -158,6 +158,75 @@ __global__ void __launch_bounds__(256) bias_update_kernel(BiasUpdateArgs a) {
     a.sel_bias[e] = __fadd_rn(a.sel_bias[e], a.gamma * sgn);
 }
 
+// Squared norm of every routed row (warp per row, 16-byte loads, fp32 sums in
+// lane-strided then shuffle-tree order). The credit's hidden-activation reading
+// ("Sparse MoE Expert-Credit Loss Reweighting Diagram", panel (b)) uses the
+// rows of H as stored.
+__global__ void __launch_bounds__(256) row_norms_kernel(RowNormArgs a) {
+    const int lane = threadIdx.x & 31;
+    const int rows = min(a.ctrl[kCtrlRoutedRows], a.max_rows);
+    const int nwarps = (gridDim.x * blockDim.x) >> 5;
+    for (int row = (blockIdx.x * blockDim.x + threadIdx.x) >> 5; row < rows; row += nwarps) {
+        if (a.row_assign[row] < 0) continue;
+        float ss = 0.f;
+        if (a.bf16) {
+            const uint4 *p = reinterpret_cast<const uint4 *>(static_cast<const __nv_bfloat16 *>(a.m) + (int64_t)row * a.n);
+            for (int v = lane; v < a.n / 8; v += 32) {
+                const uint4 u = __ldg(p + v);
+                const __nv_bfloat162 *h = reinterpret_cast<const __nv_bfloat162 *>(&u);
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    const float2 f = __bfloat1622float2(h[j]);
+                    ss = fmaf(f.x, f.x, ss);
+                    ss = fmaf(f.y, f.y, ss);
+                }
+            }
+        } else {
+            const float4 *p = reinterpret_cast<const float4 *>(static_cast<const float *>(a.m) + (int64_t)row * a.n);
+            for (int v = lane; v < a.n / 4; v += 32) {
+                const float4 f = __ldg(p + v);
+                ss = fmaf(f.x, f.x, ss);
+                ss = fmaf(f.y, f.y, ss);
+                ss = fmaf(f.z, f.z, ss);
+                ss = fmaf(f.w, f.w, ss);
+            }
+        }
+        ss = warp_sum(ss);
+        if (lane == 0) a.norm2[row] = ss;
+    }
+}
+
+// Panel (c) of the reweighting diagram, one layer: lhat <- ema lhat + (1-ema) l,
+// mu <- softmax(mu + eta lhat), objective = sum mu l. One CTA, thread e owns
+// expert e; max and sums are fixed trees.
+__global__ void __launch_bounds__(256) dro_update_kernel(DroArgs a) {
+    __shared__ float red[8];
+    const int e = threadIdx.x;
+    const bool own = e < a.E;
+    float l = 0.f, z = -INFINITY;
+    if (own) {
+        l = a.l[e];
+        const float lh = fmaf(a.ema, a.lhat[e], (1.f - a.ema) * l);
+        a.lhat[e] = lh;
+        z = fmaf(a.eta, lh, a.mu[e]);
+    }
+    // block max
+    float m = z;
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
+    if ((e & 31) == 0) red[e >> 5] = m;
+    __syncthreads();
+    m = red[0];
+#pragma unroll
+    for (int w = 1; w < 8; ++w) m = fmaxf(m, red[w]);
+    const float ex = own ? expf(z - m) : 0.f;
+    const float sum = block_sum_256(ex, red);
+    const float mu = ex / sum;
+    if (own) a.mu[e] = mu;
+    const float obj = block_sum_256(own ? mu * l : 0.f, red);
+    if (e == 0 && a.objective) *a.objective = obj;
+}
+
 }  // namespace
 
 cudaError_t launch_stat_partials(const StatsArgs &a, cudaStream_t s, int *launches) {
@@ -169,6 +238,21 @@ cudaError_t launch_stat_partials(const StatsArgs &a, cudaStream_t s, int *launch
 
 cudaError_t launch_stats_finalize(const FinalizeArgs &a, cudaStream_t s, int *launches) {
     stats_finalize_kernel<<<1, 256, 0, s>>>(a);
+    *launches += 1;
+    return cudaGetLastError();
+}
+
+cudaError_t launch_row_norms(const RowNormArgs &a, int num_sms, cudaStream_t s, int *launches) {
+    int blocks = (a.max_rows + 7) / 8;
+    if (blocks > num_sms * 8) blocks = num_sms * 8;
+    if (blocks < 1) return cudaSuccess;
+    row_norms_kernel<<<blocks, 256, 0, s>>>(a);
+    *launches += 1;
+    return cudaGetLastError();
+}
+
+cudaError_t launch_dro_update(const DroArgs &a, cudaStream_t s, int *launches) {
+    dro_update_kernel<<<1, 256, 0, s>>>(a);
     *launches += 1;
     return cudaGetLastError();
 }

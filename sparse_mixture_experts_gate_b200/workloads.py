@@ -62,6 +62,7 @@ class Workload:
     noise: bool = False               # draw [T][E] logit noise (noisy top-k)
     zipf: bool = False                # scale router rows for skewed popularity
     token_loss: bool = False          # draw per-token losses for the credit stats
+    credit_norm: str = "output"       # credit ||h||: the expert's "output" or its "hidden" activation
     seed: int = 42
 
     def with_(self, **kw) -> "Workload":

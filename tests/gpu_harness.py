@@ -137,6 +137,9 @@ def check_end_to_end(w, inp, g, tokens=None, table=None):
     tol = Y_TOL[w.dtype]
     err = np.abs(g["y"][toks] - y) / (1.0 + np.abs(y))
     assert err.max() <= tol, f"y: max scaled error {err.max():.3e} > {tol}"
+    if w.credit_norm == "hidden":  # norm of act(w1 x + b1) instead of the output
+        credit = oracle.experts_credit_hidden(toks, inp["x"].cpu(), table, g["topk_idx"], g["slot"], g["gates"],
+                                              w.d, w.F, w.E, w.activation)
     cerr = np.abs(g["credit"][toks] - credit) / (1.0 + np.abs(credit))
     assert cerr.max() <= CREDIT_TOL[w.dtype], f"credit: max scaled error {cerr.max():.3e}"
     return dict(n_near_ties=int(ties.sum()), y_err=float(err.max()), credit_err=float(cerr.max()))

@@ -288,3 +288,38 @@ def test_selection_bias_update_bit_exact():
     inp2 = dict(inp, sel_bias=layer.weights["sel_bias"].cpu())
     g2, _ = run_gpu(w, inp2, layer=layer)
     check_same_logits_routing(w, inp2, g2)
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "fp32"])
+def test_credit_hidden_activation_norm(dtype):
+    """Credit with ||h|| read as the hidden activation's norm ("Sparse MoE
+    Expert-Credit Loss Reweighting Diagram", panel (b)), and the attributed
+    loss built from it."""
+    w = WORKLOADS["default"].with_(T=333, E=6, k=2, S=1, F=1088 if dtype == "bf16" else 96,
+                                   d=256 if dtype == "bf16" else 64, O=320 if dtype == "bf16" else 48,
+                                   activation="swish", dtype=dtype, credit_norm="hidden", token_loss=True,
+                                   capacity_factor=1.0)
+    full_check(w, make_inputs(w, "cpu", seed=17, random_biases=True))
+
+
+def test_dro_update_matches_oracle():
+    """Panel (c) bookkeeping: EMA of the expert losses, mu <- softmax(mu + eta lhat)
+    and the objective sum mu l, fp32 on the GPU against the fp64 oracle."""
+    from sparse_mixture_experts_gate_b200.binding import moe_dro_update
+    w = WORKLOADS["default"].with_(T=64, d=64, F=64, O=64, E=200, k=4)
+    layer = MoELayer(w, make_inputs(w, "cpu", seed=3))
+    rng = np.random.default_rng(9)
+    l = rng.gamma(2.0, 0.5, w.E)
+    lhat = rng.gamma(2.0, 0.5, w.E)
+    mu = rng.dirichlet(np.ones(w.E))
+    dl, dlh, dmu = (torch.tensor(v, dtype=torch.float32, device="cuda") for v in (l, lhat, mu))
+    obj = torch.empty(1, device="cuda")
+    for ema, eta in ((0.9, 0.5), (0.0, 3.0), (1.0, 0.0)):
+        lh0, mu0 = dlh.cpu().numpy().astype(np.float64), dmu.cpu().numpy().astype(np.float64)
+        moe_dro_update(layer.handle, dl.data_ptr(), ema, eta, dlh.data_ptr(), dmu.data_ptr(), obj.data_ptr(),
+                       torch.cuda.current_stream().cuda_stream)
+        torch.cuda.synchronize()
+        want_lh, want_mu, want_obj = oracle.dro_update(dl.cpu().numpy(), lh0, mu0, ema, eta)
+        assert np.abs(dlh.cpu().numpy() - want_lh).max() <= 1e-6 * (1 + np.abs(want_lh).max())
+        assert np.abs(dmu.cpu().numpy() - want_mu).max() <= 1e-6
+        assert abs(obj.item() - want_obj) <= 1e-6 * (1 + abs(want_obj))
