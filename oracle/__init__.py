@@ -61,6 +61,8 @@ def _configure(L):
     L.orc_balance_stats.argtypes = [i32, i32, i32, vp, vp, vp, dbl, dbl, vp, vp, vp, vp]
     L.orc_expert_loss.argtypes = [i32, i32, i32, vp, vp, vp, vp, vp]
     L.orc_importance.argtypes = [i32, i32, i32, vp, vp, vp]
+    L.orc_dispatch_rank_major.argtypes = [i32, i32, i32, i64, vp, vp, vp, vp, vp]
+    L.orc_router_mlp.argtypes = [i32, i32, i32, i32, vp, i32, vp, vp, vp, vp, vp]
     L.orc_experts_credit_hidden.argtypes = [i32, vp, i32, i32, i32, i32, i32, i32, i32, vp,
                                             ctypes.POINTER(Expert), vp, vp, vp, vp]
     L.orc_dro_update.argtypes = [i32, dbl, dbl, vp, vp, vp]
@@ -179,15 +181,33 @@ def capacity(capacity_factor: float, k: int, T: int, E: int) -> int:
     return int(lib().orc_capacity(float(capacity_factor), k, T, E))
 
 
-def dispatch(idx: np.ndarray, E: int, C: int):
+def dispatch(idx: np.ndarray, E: int, C: int, priority: str = "token"):
+    """Capacity-capped ranks; priority "token" (ascending token index) or "rank"
+    (first choices of all tokens, then second choices, ...)."""
     idx = np.ascontiguousarray(idx, dtype=np.int32)
     T, k = idx.shape
     slot = np.empty((T, k), np.int32)
     cpre = np.empty(E, np.int32)
     ckept = np.empty(E, np.int32)
     nd = np.zeros(1, np.int32)
-    lib().orc_dispatch(T, E, k, int(C), _p(idx), _p(slot), _p(cpre), _p(ckept), _p(nd))
+    fn = lib().orc_dispatch if priority == "token" else lib().orc_dispatch_rank_major
+    fn(T, E, k, int(C), _p(idx), _p(slot), _p(cpre), _p(ckept), _p(nd))
     return slot, cpre, ckept, int(nd[0])
+
+
+def router_mlp(x, w1, b1, w2, b2) -> np.ndarray:
+    """MLP gate logits h = W_2 relu(W_1 x + b_1) + b_2 in double."""
+    xs, xd = as_storage(x)
+    T, d = xs.shape
+    w1 = _f32(w1)
+    w2 = _f32(w2)
+    H, E = w1.shape[0], w2.shape[0]
+    b1 = _f32(b1) if b1 is not None else None
+    b2 = _f32(b2) if b2 is not None else None
+    h = np.empty((T, E), np.float64)
+    lib().orc_router_mlp(T, d, H, E, _p(xs), xd, _p(w1), _p(b1) if b1 is not None else None, _p(w2),
+                         _p(b2) if b2 is not None else None, _p(h))
+    return h
 
 
 class ExpertTable:
@@ -334,7 +354,7 @@ def routing_from_logits(h32, w, noise=None, sel_bias=None) -> Dict[str, object]:
     P, lse = softmax_lse(h32.astype(np.float64))
     g = gates(P, idx)
     C = capacity(w.capacity_factor, w.k, T, E)
-    slot, cpre, ckept, nd = dispatch(idx, E, C)
+    slot, cpre, ckept, nd = dispatch(idx, E, C, getattr(w, "capacity_priority", "token"))
     return dict(key=key, idx=idx, P=P, lse=lse, gates=g, C=C, slot=slot,
                 count_pre=cpre, count_kept=ckept, n_dropped=nd)
 
@@ -349,7 +369,10 @@ def forward(w, inp: Dict[str, object], tokens: Optional[Sequence[int]] = None,
     a subset of tokens; the statistics that need every token's credit are then
     skipped."""
     x = inp["x"]
-    h = router_logits(x, inp["w_gate"], inp.get("b_gate"))
+    if getattr(w, "mlp_gater", False):
+        h = router_mlp(x, inp["gater_w1"], inp.get("gater_b1"), inp["w_gate"], inp.get("b_gate"))
+    else:
+        h = router_logits(x, inp["w_gate"], inp.get("b_gate"))
     T, E = h.shape
     P, lse = softmax_lse(h)
     out: Dict[str, object] = dict(h=h, P=P, lse=lse)
@@ -358,7 +381,7 @@ def forward(w, inp: Dict[str, object], tokens: Optional[Sequence[int]] = None,
     idx = topk(key, w.k)
     g = gates(P, idx)
     C = capacity(w.capacity_factor, w.k, T, E)
-    slot, cpre, ckept, nd = dispatch(idx, E, C)
+    slot, cpre, ckept, nd = dispatch(idx, E, C, getattr(w, "capacity_priority", "token"))
     out.update(h32=h32, key=key, idx=idx, gates=g, C=C, slot=slot, count_pre=cpre,
                count_kept=ckept, n_dropped=nd)
     f, pm, la, lz = balance_stats(P, lse, cpre, w.k, w.alpha, w.beta)

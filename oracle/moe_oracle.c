@@ -144,6 +144,55 @@ void orc_dispatch(int T, int E, int k, int64_t C, const int32_t *idx, int32_t *s
     *n_dropped = dropped;
 }
 
+/* Capacity cap with rank-major priority: queues filled choice by choice. */
+void orc_dispatch_rank_major(int T, int E, int k, int64_t C, const int32_t *idx, int32_t *slot,
+                             int32_t *count_pre, int32_t *count_kept, int32_t *n_dropped)
+{
+    for (int e = 0; e < E; ++e)
+        count_pre[e] = 0;
+    for (int r = 0; r < k; ++r) {
+        for (int t = 0; t < T; ++t) {
+            int e = idx[(int64_t)t * k + r];
+            int32_t rank = count_pre[e];
+            count_pre[e] = rank + 1;
+            slot[(int64_t)t * k + r] = (rank < C) ? rank : -1;
+        }
+    }
+    int32_t dropped = 0;
+    for (int e = 0; e < E; ++e) {
+        count_kept[e] = (count_pre[e] < C) ? count_pre[e] : (int32_t)C;
+        dropped += count_pre[e] - count_kept[e];
+    }
+    *n_dropped = dropped;
+}
+
+/* SER walkthrough: the optional MLP gate, h = W_2 relu(W_1 x + b_1) + b_2. */
+void orc_router_mlp(int T, int d, int H, int E, const void *x, int x_dtype, const float *w1,
+                    const float *b1, const float *w2, const float *b2, double *h)
+{
+#pragma omp parallel for schedule(static)
+    for (int t = 0; t < T; ++t) {
+        double *z = (double *)malloc(sizeof(double) * (size_t)H);
+        for (int u = 0; u < H; ++u) {
+            double s = 0.0;
+            for (int j = 0; j < d; ++j)
+                s += (double)w1[(int64_t)u * d + j] * orc_load(x, (int64_t)t * d + j, x_dtype);
+            if (b1)
+                s += (double)b1[u];
+            z[u] = s > 0.0 ? s : 0.0;
+        }
+        for (int i = 0; i < E; ++i) {
+            double s = 0.0;
+            for (int u = 0; u < H; ++u)
+                s += (double)w2[(int64_t)i * H + u] * z[u];
+            if (b2)
+                s += (double)b2[i];
+            h[(int64_t)t * E + i] = s;
+        }
+        free(z);
+    }
+}
+
 static double activation(int act, double z)
 {
     switch (act) {

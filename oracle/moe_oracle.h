@@ -84,6 +84,21 @@ int64_t orc_capacity(double capacity_factor, int k, int T, int E);
 void orc_dispatch(int T, int E, int k, int64_t C, const int32_t *idx, int32_t *slot,
                   int32_t *count_pre, int32_t *count_kept, int32_t *n_dropped);
 
+/* The same capacity cap with GShard's rank-major priority (the reading of
+ * "Capacity & communication" taken for capacity_priority = rank): every token's
+ * first choice joins the queues in token order, then every token's second
+ * choice, and so on. Outputs as orc_dispatch. */
+void orc_dispatch_rank_major(int T, int E, int k, int64_t C, const int32_t *idx, int32_t *slot,
+                             int32_t *count_pre, int32_t *count_kept, int32_t *n_dropped);
+
+/* [W] "Configuration" (use_mlp_gater, gater_hidden_dim) and "The gating /
+ * routing path" (gate logits "via the router/router_bias linear layer, or the
+ * optional MLP gate"): h = W_2 relu(W_1 x + b_1) + b_2 with hidden width H.
+ * x [T][d] (x_dtype), w1 [H][d], b1 [H] or NULL, w2 [E][H], b2 [E] or NULL (fp32)
+ * -> h [T][E]. */
+void orc_router_mlp(int T, int d, int H, int E, const void *x, int x_dtype, const float *w1,
+                    const float *b1, const float *w2, const float *b2, double *h);
+
 /* One expert's weights ([C] "Core MoE symbols": expert i is an FFN with its own
  * weights; [W]: w1/b1 -> activation -> w2/b2). w1 [F][d], w2 [O][F] in w_dtype;
  * b1 [F], b2 [O] fp32 or NULL. */

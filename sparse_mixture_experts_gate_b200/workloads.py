@@ -63,6 +63,9 @@ class Workload:
     zipf: bool = False                # scale router rows for skewed popularity
     token_loss: bool = False          # draw per-token losses for the credit stats
     credit_norm: str = "output"       # credit ||h||: the expert's "output" or its "hidden" activation
+    capacity_priority: str = "token"  # capacity queue order: "token" index, or "rank" (choice by choice)
+    mlp_gater: bool = False           # router logits from an MLP gate (hidden width gater_hidden)
+    gater_hidden: int = 128
     seed: int = 42
 
     def with_(self, **kw) -> "Workload":
@@ -87,7 +90,7 @@ WORKLOADS: Dict[str, Workload] = {
 }
 
 _TAGS = {"x": 1, "w_gate": 2, "b_gate": 3, "sel_bias": 4, "w1": 5, "b1": 6, "w2": 7,
-         "b2": 8, "noise": 9, "token_loss": 10}
+         "b2": 8, "noise": 9, "token_loss": 10, "gater_w1": 11, "gater_b1": 12}
 
 
 def _gen(device: str, seed: int, tag: str, sub: int = 0) -> torch.Generator:
@@ -174,14 +177,22 @@ def make_tokens(w: Workload, device: str = "cpu", seed: Optional[int] = None) ->
 
 def make_router(w: Workload, device: str = "cpu", seed: Optional[int] = None, random_biases: bool = False,
                 apply_zipf: bool = True) -> Dict[str, Optional[torch.Tensor]]:
-    """Router parameters: w_gate [E][d], b_gate [E] or None, sel_bias [E] or None."""
+    """Router parameters: w_gate [E][d], b_gate [E] or None, sel_bias [E] or None.
+    With an MLP gate: gater_w1 [H][d] ~ N(0, 1/d), gater_b1 [H] (zero, or
+    N(0, 1/d) with random_biases), and w_gate [E][H] ~ N(0, 1/H) its output layer."""
     seed = w.seed if seed is None else seed
-    wg = _normal((w.E, w.d), (1.0 / w.d) ** 0.5, device, seed, "w_gate", torch.float32)
+    fan = w.gater_hidden if w.mlp_gater else w.d
+    wg = _normal((w.E, fan), (1.0 / fan) ** 0.5, device, seed, "w_gate", torch.float32)
     if w.zipf and apply_zipf:
         s = load_zipf_row_scales(w.E)
         if s is not None:
             wg.mul_(s.to(device)[:, None])
-    out: Dict[str, Optional[torch.Tensor]] = {"w_gate": wg}
+    out: Dict[str, Optional[torch.Tensor]] = {"w_gate": wg, "gater_w1": None, "gater_b1": None}
+    if w.mlp_gater:
+        H = w.gater_hidden
+        out["gater_w1"] = _normal((H, w.d), (1.0 / w.d) ** 0.5, device, seed, "gater_w1", torch.float32)
+        out["gater_b1"] = (_normal((H,), (1.0 / w.d) ** 0.5, device, seed, "gater_b1", torch.float32)
+                           if random_biases else torch.zeros(H, device=device))
     if w.router_bias:
         out["b_gate"] = (_normal((w.E,), (1.0 / w.d) ** 0.5, device, seed, "b_gate", torch.float32)
                          if random_biases else torch.zeros(w.E, device=device))

@@ -492,6 +492,60 @@ def check_dro_update():
     assert abs(obj - (mu_o[0] * l2[0] + mu_o[1] * l2[1])) < 1e-15
 
 
+def check_dispatch_rank_major():
+    """GShard-style priority (capacity_priority = rank): a hand-worked case where
+    it differs from token order; k = 1 makes the two orders equal; a queue
+    simulation over (choice, token) order; per-expert counts and the number of
+    drops do not depend on the order."""
+    # T=3, k=2, E=2, C=2. Rank-major: choice 0: t0->e0 (rank 0), t1->e1 (0),
+    # t2->e0 (1); choice 1: t0->e1 (1), t1->e0 (2: dropped), t2->e1 (2: dropped).
+    # Token order instead: e0 sees t0, t1, t2 and e1 sees t0, t1, t2, so both of
+    # t2's choices drop.
+    idx = np.array([[0, 1], [1, 0], [0, 1]], np.int32)
+    slot, cpre, ckept, nd = oracle.dispatch(idx, 2, 2, "rank")
+    assert slot.tolist() == [[0, 1], [0, -1], [1, -1]] and nd == 2
+    slot_t, _, _, nd_t = oracle.dispatch(idx, 2, 2, "token")
+    assert slot_t.tolist() == [[0, 0], [1, 1], [-1, -1]] and nd_t == 2
+    rng = np.random.default_rng(12)
+    T, E = 50, 7
+    idx1 = rng.integers(0, E, size=(T, 1)).astype(np.int32)
+    assert np.array_equal(oracle.dispatch(idx1, E, 5, "rank")[0], oracle.dispatch(idx1, E, 5, "token")[0])
+    k, C = 3, 12
+    idx3 = np.array([rng.permutation(E)[:k] for _ in range(T)], np.int32)
+    slot, cpre, ckept, nd = oracle.dispatch(idx3, E, C, "rank")
+    fill = [0] * E
+    want = np.empty((T, k), np.int32)
+    for r in range(k):
+        for t in range(T):
+            e = idx3[t, r]
+            want[t, r] = fill[e] if fill[e] < C else -1
+            fill[e] += 1
+    assert np.array_equal(slot, want)
+    _, cpre_t, ckept_t, nd_t = oracle.dispatch(idx3, E, C, "token")
+    assert np.array_equal(cpre, cpre_t) and np.array_equal(ckept, ckept_t) and nd == nd_t
+
+
+def check_router_mlp():
+    """[W] optional MLP gate: h = W_2 relu(W_1 x + b_1) + b_2 against numpy fp64;
+    a hand-worked two-unit case (one hidden unit clipped by the ReLU)."""
+    rng = np.random.default_rng(13)
+    T, d, H, E = 9, 12, 7, 5
+    x = rng.standard_normal((T, d)).astype(np.float32)
+    w1 = rng.standard_normal((H, d)).astype(np.float32)
+    b1 = rng.standard_normal(H).astype(np.float32)
+    w2 = rng.standard_normal((E, H)).astype(np.float32)
+    b2 = rng.standard_normal(E).astype(np.float32)
+    h = oracle.router_mlp(x, w1, b1, w2, b2)
+    z = np.maximum(x.astype(np.float64) @ w1.astype(np.float64).T + b1, 0.0)
+    assert np.allclose(h, z @ w2.astype(np.float64).T + b2, rtol=1e-13, atol=1e-13)
+    # x = (1, 2); unit 0 = x0 + x1 = 3, unit 1 = x0 - x1 - 1 = -2 -> 0;
+    # h0 = 2*3 + 5*0 + 0.5 = 6.5, h1 = -1*3 + 1*0 = -3.
+    hx = oracle.router_mlp(np.array([[1.0, 2.0]], np.float32), np.array([[1, 1], [1, -1]], np.float32),
+                           np.array([0, -1], np.float32), np.array([[2, 5], [-1, 1]], np.float32),
+                           np.array([0.5, 0.0], np.float32))
+    assert hx.tolist() == [[6.5, -3.0]]
+
+
 def check_minimal_example_shapes():
     """[W] "Minimal example": 4 experts, 2 active, dims 8/16/8, a (4, 8) input;
     the forward yields a (4, 8) output, 2 distinct experts per token, gates

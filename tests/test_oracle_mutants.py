@@ -20,7 +20,8 @@ MUTANTS = {
     "gates_wrong_index": ("s += P[(int64_t)t * E + idx[(int64_t)t * k + r]];",
                           "s += P[(int64_t)t * E + r];"),
     "capacity_floor": ("(int64_t)ceil(capacity_factor", "(int64_t)floor(capacity_factor"),
-    "dispatch_off_by_one": ("(rank < C) ? rank : -1", "(rank <= C) ? rank : -1"),
+    "dispatch_off_by_one": ("count_pre[e] = rank + 1;\n            slot[(int64_t)t * k + r] = (rank < C) ? rank : -1;\n        }\n    }\n    int32_t dropped = 0;\n    for (int e = 0; e < E; ++e) {\n        count_kept[e] = (count_pre[e] < C) ? count_pre[e] : (int32_t)C;\n        dropped += count_pre[e] - count_kept[e];\n    }\n    *n_dropped = dropped;\n}\n\n/* Capacity cap with rank-major",
+                            "count_pre[e] = rank + 1;\n            slot[(int64_t)t * k + r] = (rank <= C) ? rank : -1;\n        }\n    }\n    int32_t dropped = 0;\n    for (int e = 0; e < E; ++e) {\n        count_kept[e] = (count_pre[e] < C) ? count_pre[e] : (int32_t)C;\n        dropped += count_pre[e] - count_kept[e];\n    }\n    *n_dropped = dropped;\n}\n\n/* Capacity cap with rank-major"),
     "ffn_w1_transposed": ("orc_load(ex->w1, (int64_t)f * d + j, w_dtype)",
                           "orc_load(ex->w1, (int64_t)j * F + f, w_dtype)"),
     "ffn_drops_b2": ("s += (double)ex->b2[n];", "s += 0.0;"),
@@ -49,6 +50,10 @@ MUTANTS = {
     "dro_ema_swapped": ("lhat[i] = ema * lhat[i] + (1.0 - ema) * l[i];", "lhat[i] = (1.0 - ema) * lhat[i] + ema * l[i];"),
     "dro_eta_dropped": ("s += exp(mu[i] + eta * lhat[i] - m);", "s += exp(mu[i] - m);"),
     "dro_objective_old_mu": ("obj += mu[i] * l[i];", "obj += lhat[i] * l[i];"),
+    "rank_major_token_order": ("    for (int r = 0; r < k; ++r) {\n        for (int t = 0; t < T; ++t) {\n            int e = idx[(int64_t)t * k + r];",
+                               "    for (int t = 0; t < T; ++t) {\n        for (int r = 0; r < k; ++r) {\n            int e = idx[(int64_t)t * k + r];"),
+    "mlp_no_relu": ("z[u] = s > 0.0 ? s : 0.0;", "z[u] = s;"),
+    "mlp_drops_b1": ("                s += (double)b1[u];", "                s += 0.0;"),
     "softmax_wrong_exponent": ("P[(int64_t)t * E + i] = exp(ht[i] - m) / z;",
                                "P[(int64_t)t * E + i] = exp(ht[i]) / z;"),
 }
