@@ -74,6 +74,12 @@ enum { MOE_DTYPE_BF16 = 0, MOE_DTYPE_FP32 = 1 };
  * (default) or its hidden activation act(w1 x + b1). */
 enum { MOE_CREDIT_OUTPUT = 0, MOE_CREDIT_HIDDEN = 1 };
 
+/* Order in which assignments fill an expert's capacity ("Appendix C",
+ * "Capacity & communication"; the pages fix none): TOKEN = ascending token
+ * index, each token's choices together; RANK = every token's first choice (in
+ * token order), then every second choice, and so on (GShard's order). */
+enum { MOE_PRIORITY_TOKEN = 0, MOE_PRIORITY_RANK = 1 };
+
 /* Layer configuration. Field names follow the SER walkthrough's configuration
  * (num_experts, num_active, input_dim, expert_dim, output_dim, top_k_method,
  * load_balance_coef); the remaining fields carry Appendix C's symbols. */
@@ -94,6 +100,9 @@ typedef struct {
     float z_loss_coef;        /* beta of the z-loss                                 */
     float temperature;        /* router softmax temperature; only 1 is supported   */
     int32_t credit_norm;      /* MOE_CREDIT_*                                       */
+    int32_t capacity_priority; /* MOE_PRIORITY_*                                    */
+    int32_t use_mlp_gater;    /* 1: logits from the MLP gate (SER "Configuration") */
+    int32_t gater_hidden_dim; /* H of the MLP gate, 1..256 (default 128)           */
 } moe_config_t;
 
 /* Defaults of the SER walkthrough's configuration: E=8, k=2, 512/1024/512,
@@ -107,7 +116,12 @@ MOE_API moe_config_t moe_config_default(void);
  * step); each forward reads the current values. Shared experts are the last S
  * entries of the expert stacks (G = E + S groups).
  *   w_gate   [E][d]    fp32, router matrix W_g                     (required)
- *   b_gate   [E]       fp32, router bias                           (NULL = none)
+ *            [E][H]    with use_mlp_gater: the gate's output layer W_2
+ *   b_gate   [E]       fp32, router bias (the gate's b_2)          (NULL = none)
+ *   gater_w1 [H][d]    fp32, the MLP gate's hidden layer W_1        (required iff use_mlp_gater)
+ *   gater_b1 [H]       fp32, its bias b_1                          (NULL = zero)
+ * The MLP gate ("Code Walkthrough - SER": "via the router/router_bias linear
+ * layer, or the optional MLP gate") is h = W_2 relu(W_1 x + b_1) + b_2.
  *   sel_bias [E]       fp32, selection bias b_i                    (required iff use_selection_bias)
  *   w1       [G][F][d] dtype, first expert layer (row f, column j) (required)
  *   b1       [G][F]    fp32                                        (NULL = zero)
@@ -121,6 +135,8 @@ typedef struct {
     const void *w2;
     const float *b1;
     const float *b2;
+    const float *gater_w1;
+    const float *gater_b1;
 } moe_weights_t;
 
 /* Optional routing outputs of a forward (any pointer may be NULL; the struct

@@ -344,6 +344,14 @@ def selection_bias_update(b, load, k: int, T: int, gamma: float) -> np.ndarray:
 
 # ---------------------------------------------------------------- whole layer
 
+def layer_capacity_factor(w) -> float:
+    """The capacity factor as a layer holds it: the configuration stores C_f in
+    fp32, so C = ceil(C_f k T / E) is formed (in double) from fl32(C_f). For C_f
+    = 0.6, for instance, fl32(0.6) k T / E can exceed an integer that 0.6 k T / E
+    equals exactly."""
+    return float(np.float32(w.capacity_factor))
+
+
 def routing_from_logits(h32, w, noise=None, sel_bias=None) -> Dict[str, object]:
     """Selection, top-k and dispatch from given fp32 logits (the integer
     decisions), with P, lse and gates formed in double from those logits."""
@@ -353,7 +361,7 @@ def routing_from_logits(h32, w, noise=None, sel_bias=None) -> Dict[str, object]:
     idx = topk(key, w.k)
     P, lse = softmax_lse(h32.astype(np.float64))
     g = gates(P, idx)
-    C = capacity(w.capacity_factor, w.k, T, E)
+    C = capacity(layer_capacity_factor(w), w.k, T, E)
     slot, cpre, ckept, nd = dispatch(idx, E, C, getattr(w, "capacity_priority", "token"))
     return dict(key=key, idx=idx, P=P, lse=lse, gates=g, C=C, slot=slot,
                 count_pre=cpre, count_kept=ckept, n_dropped=nd)
@@ -380,7 +388,7 @@ def forward(w, inp: Dict[str, object], tokens: Optional[Sequence[int]] = None,
     key = selection_keys(h32, inp.get("noise"), inp.get("sel_bias"))
     idx = topk(key, w.k)
     g = gates(P, idx)
-    C = capacity(w.capacity_factor, w.k, T, E)
+    C = capacity(layer_capacity_factor(w), w.k, T, E)
     slot, cpre, ckept, nd = dispatch(idx, E, C, getattr(w, "capacity_priority", "token"))
     out.update(h32=h32, key=key, idx=idx, gates=g, C=C, slot=slot, count_pre=cpre,
                count_kept=ckept, n_dropped=nd)

@@ -19,6 +19,7 @@ MOE_ACT = {"relu": 0, "gelu": 1, "swish": 2}
 MOE_TOPK = {"greedy": 0, "noisy": 1}
 MOE_DTYPE = {"bf16": 0, "fp32": 1}
 MOE_CREDIT = {"output": 0, "hidden": 1}
+MOE_PRIORITY = {"token": 0, "rank": 1}
 
 # Every symbol include/moe.h declares.
 EXPORTS = ("moe_config_default", "moe_layer_create", "moe_workspace_bytes", "moe_capacity", "moe_forward",
@@ -33,13 +34,15 @@ class MoeConfig(ctypes.Structure):
                 ("capacity_factor", ctypes.c_float), ("activation", ctypes.c_int32),
                 ("top_k_method", ctypes.c_int32), ("use_selection_bias", ctypes.c_int32),
                 ("dtype", ctypes.c_int32), ("max_tokens", ctypes.c_int32), ("load_balance_coef", ctypes.c_float),
-                ("z_loss_coef", ctypes.c_float), ("temperature", ctypes.c_float), ("credit_norm", ctypes.c_int32)]
+                ("z_loss_coef", ctypes.c_float), ("temperature", ctypes.c_float), ("credit_norm", ctypes.c_int32),
+                ("capacity_priority", ctypes.c_int32), ("use_mlp_gater", ctypes.c_int32),
+                ("gater_hidden_dim", ctypes.c_int32)]
 
 
 class MoeWeights(ctypes.Structure):
     _fields_ = [("w_gate", ctypes.c_void_p), ("b_gate", ctypes.c_void_p), ("sel_bias", ctypes.c_void_p),
                 ("w1", ctypes.c_void_p), ("w2", ctypes.c_void_p), ("b1", ctypes.c_void_p),
-                ("b2", ctypes.c_void_p)]
+                ("b2", ctypes.c_void_p), ("gater_w1", ctypes.c_void_p), ("gater_b1", ctypes.c_void_p)]
 
 
 class MoeRouting(ctypes.Structure):
@@ -248,13 +251,17 @@ class MoELayer:
         cfg.max_tokens = max_tokens or 0
         cfg.load_balance_coef, cfg.z_loss_coef, cfg.temperature = w.alpha, w.beta, 1.0
         cfg.credit_norm = MOE_CREDIT[w.credit_norm]
+        cfg.capacity_priority = MOE_PRIORITY[w.capacity_priority]
+        cfg.use_mlp_gater = int(w.mlp_gater)
+        cfg.gater_hidden_dim = w.gater_hidden
         self.cfg = cfg
         self.weights = {k: (v.to(self.device).contiguous() if v is not None else None)
                         for k, v in weights.items()
-                        if k in ("w_gate", "b_gate", "sel_bias", "w1", "b1", "w2", "b2")}
+                        if k in ("w_gate", "b_gate", "sel_bias", "w1", "b1", "w2", "b2", "gater_w1", "gater_b1")}
         ww = self.weights
         self._cw = MoeWeights(_ptr(ww["w_gate"]), _ptr(ww.get("b_gate")), _ptr(ww.get("sel_bias")),
-                              _ptr(ww["w1"]), _ptr(ww["w2"]), _ptr(ww.get("b1")), _ptr(ww.get("b2")))
+                              _ptr(ww["w1"]), _ptr(ww["w2"]), _ptr(ww.get("b1")), _ptr(ww.get("b2")),
+                              _ptr(ww.get("gater_w1")), _ptr(ww.get("gater_b1")))
         self.handle = moe_layer_create(cfg, self._cw)
         self._ws = None
         self._ws_T = -1

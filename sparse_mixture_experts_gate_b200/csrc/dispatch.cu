@@ -4,7 +4,8 @@
 // expert has a fixed buffer of C = ceil(C_f k T / E) tokens and the dispatch
 // tensor D scatters tokens into those buffers; "Code Walkthrough - SER", "Load
 // balancing": a hard per-expert cap drops overflow tokens. Priority inside an
-// expert's buffer is ascending token index (a stable ranking).
+// expert's buffer is ascending token index (a stable ranking), or, with
+// rank-major priority, every token's first choice before any second choice.
 //
 // Instead of a dense one-hot D, the dispatch is a permutation into a compact row
 // space: expert e owns rows [group_start[e], group_start[e] + kept_e), padded to
@@ -35,13 +36,21 @@ namespace {
 constexpr int kChunk = 256;  // tokens per chunk = threads per block
 constexpr int kMaxE = 256;
 
+// The assignments in capacity-priority order: item i holds assignments
+// t*k + r for r < k (token order, item = token t), or the single assignment
+// (i mod T)*k + i/T (rank-major, item = r T + t).
+__device__ __forceinline__ int items_per(const DispatchArgs &a) { return a.rank_major ? 1 : a.k; }
+__device__ __forceinline__ int64_t assignment_of(const DispatchArgs &a, int i, int j) {
+    return a.rank_major ? (int64_t)(i % a.T) * a.k + i / a.T : (int64_t)i * a.k + j;
+}
+
 __global__ void __launch_bounds__(kChunk) dispatch_count_kernel(DispatchArgs a) {
     __shared__ int cnt[kMaxE];
     for (int e = threadIdx.x; e < a.E; e += kChunk) cnt[e] = 0;
     __syncthreads();
-    const int t = blockIdx.x * kChunk + threadIdx.x;
-    if (t < a.T)
-        for (int r = 0; r < a.k; ++r) atomicAdd(&cnt[a.idx[(int64_t)t * a.k + r]], 1);
+    const int i = blockIdx.x * kChunk + threadIdx.x;
+    if (i < a.n_items)
+        for (int j = 0; j < items_per(a); ++j) atomicAdd(&cnt[a.idx[assignment_of(a, i, j)]], 1);
     __syncthreads();
     for (int e = threadIdx.x; e < a.E; e += kChunk) a.chunk_count[(int64_t)blockIdx.x * a.E + e] = cnt[e];
 }
@@ -140,9 +149,9 @@ __global__ void __launch_bounds__(kChunk) dispatch_assign_kernel(DispatchArgs a)
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     for (int i = tid; i < W * kMaxE; i += kChunk) (&mask[0][0])[i] = 0u;
     __syncthreads();
-    const int t = blockIdx.x * kChunk + tid;
-    if (t < a.T)
-        for (int r = 0; r < a.k; ++r) atomicOr(&mask[warp][a.idx[(int64_t)t * a.k + r]], 1u << lane);
+    const int item = blockIdx.x * kChunk + tid;
+    if (item < a.n_items)
+        for (int j = 0; j < items_per(a); ++j) atomicOr(&mask[warp][a.idx[assignment_of(a, item, j)]], 1u << lane);
     __syncthreads();
     for (int e = tid; e < a.E; e += kChunk) {
         int run = a.chunk_base[(int64_t)blockIdx.x * a.E + e];
@@ -152,10 +161,10 @@ __global__ void __launch_bounds__(kChunk) dispatch_assign_kernel(DispatchArgs a)
         }
     }
     __syncthreads();
-    if (t >= a.T) return;
+    if (item >= a.n_items) return;
     const uint32_t lt = (1u << lane) - 1u;
-    for (int r = 0; r < a.k; ++r) {
-        const int64_t ai = (int64_t)t * a.k + r;
+    for (int j = 0; j < items_per(a); ++j) {
+        const int64_t ai = assignment_of(a, item, j);
         const int e = a.idx[ai];
         const int rank = wbase[warp][e] + __popc(mask[warp][e] & lt);
         a.gate_sorted[a.pre_start[e] + rank] = a.gates[ai];

@@ -88,7 +88,7 @@ struct Plan {
     size_t o_lpart = 0;
     size_t o_ctrl, o_logits, o_idx, o_gates, o_slot, o_rowof, o_lse, o_psum, o_ccount, o_cbase, o_cpre, o_ckept,
         o_gstart, o_grows, o_bgroup, o_toktiles, o_rowassign, o_wsplit, o_xp, o_h, o_o, o_credit, o_partials,
-        o_prestart, o_gsorted, o_rownorm;
+        o_prestart, o_gsorted, o_rownorm, o_gz;
     size_t total = 0;
 };
 
@@ -140,8 +140,11 @@ Plan make_plan(const moe_layer &L, int T) {
     // Each expert's segment splits into ceil(rows / 256) token tiles of >= 32 rows.
     p.max_tok_tiles = (int)std::min<int64_t>(routed / kTokTile + E, routed / kRowBlock) +
                       S * (int)((p.T_pad + kTokTile - 1) / kTokTile);
-    p.n_stat_chunks = router_psum_blocks(T, L.num_sms, c.dtype == MOE_DTYPE_BF16);
-    p.n_chunks = (T + 255) / 256;
+    // bf16 linear routers route from the tensor-core logits; the MLP gate and
+    // fp32 layers route inside the CUDA-core router kernel.
+    p.n_stat_chunks = router_psum_blocks(T, L.num_sms, c.dtype == MOE_DTYPE_BF16 && !c.use_mlp_gater);
+    const int64_t n_items = c.capacity_priority == MOE_PRIORITY_RANK ? (int64_t)k * T : T;
+    p.n_chunks = (int)((n_items + 255) / 256);
     const size_t es = c.dtype == MOE_DTYPE_BF16 ? 2 : 4;
     size_t off = 0;
     auto take = [&](size_t bytes) {
@@ -171,8 +174,10 @@ Plan make_plan(const moe_layer &L, int T) {
     p.o_gsorted = take((size_t)T * k * 4);
     p.o_rownorm = take(c.credit_norm == MOE_CREDIT_HIDDEN ? (size_t)p.R_routed_max * 4 : 0);
     p.o_credit = take((size_t)T * k * 4);
-    p.o_wsplit = take(c.dtype == MOE_DTYPE_BF16 ? (size_t)router_tc_epad(E) * 3 * c.input_dim * 2 : 0);
-    p.ksplit = c.dtype == MOE_DTYPE_BF16 ? router_tc_ksplit(T, E, c.input_dim, L.num_sms) : 1;
+    const int E_tc = c.use_mlp_gater ? c.gater_hidden_dim : E;  // rows of the tensor-core router matrix
+    p.o_wsplit = take(c.dtype == MOE_DTYPE_BF16 ? (size_t)router_tc_epad(E_tc) * 3 * c.input_dim * 2 : 0);
+    p.ksplit = c.dtype == MOE_DTYPE_BF16 && !c.use_mlp_gater ? router_tc_ksplit(T, E, c.input_dim, L.num_sms) : 1;
+    p.o_gz = take(c.use_mlp_gater ? (size_t)T * c.gater_hidden_dim * 4 : 0);
     p.o_lpart = take(p.ksplit > 1 ? (size_t)p.ksplit * T * E * 4 : 0);
     p.o_xp = take(c.dtype == MOE_DTYPE_BF16 ? (size_t)p.R_routed_max * c.input_dim * es : 0);
     p.o_h = take((size_t)p.R_max * c.expert_dim * es);
@@ -207,6 +212,15 @@ int validate_config(const moe_config_t *c, const moe_weights_t *w) {
     if (c->capacity_factor != c->capacity_factor) return fail(MOE_ERR_INVALID_ARG, "capacity_factor is NaN");
     if (c->credit_norm != MOE_CREDIT_OUTPUT && c->credit_norm != MOE_CREDIT_HIDDEN)
         return fail(MOE_ERR_INVALID_ARG, "unknown credit_norm %d", c->credit_norm);
+    if (c->capacity_priority != MOE_PRIORITY_TOKEN && c->capacity_priority != MOE_PRIORITY_RANK)
+        return fail(MOE_ERR_INVALID_ARG, "unknown capacity_priority %d", c->capacity_priority);
+    if (c->use_mlp_gater != 0 && c->use_mlp_gater != 1)
+        return fail(MOE_ERR_INVALID_ARG, "use_mlp_gater must be 0 or 1");
+    if (c->use_mlp_gater) {
+        if (c->gater_hidden_dim < 1 || c->gater_hidden_dim > 256)
+            return fail(MOE_ERR_UNSUPPORTED, "gater_hidden_dim must be in 1..256 (got %d)", c->gater_hidden_dim);
+        if (!w->gater_w1) return fail(MOE_ERR_INVALID_ARG, "use_mlp_gater is set but weights->gater_w1 is NULL");
+    }
     if (!w->w_gate) return fail(MOE_ERR_INVALID_ARG, "weights->w_gate is NULL");
     if (!w->w1) return fail(MOE_ERR_INVALID_ARG, "weights->w1 is NULL");
     if (!w->w2) return fail(MOE_ERR_INVALID_ARG, "weights->w2 is NULL");
@@ -257,6 +271,10 @@ moe_config_t moe_config_default(void) {
     c.load_balance_coef = 0.01f;
     c.z_loss_coef = 1e-3f;
     c.temperature = 1.0f;
+    c.credit_norm = MOE_CREDIT_OUTPUT;
+    c.capacity_priority = MOE_PRIORITY_TOKEN;
+    c.use_mlp_gater = 0;
+    c.gater_hidden_dim = 128;
     return c;
 }
 
@@ -366,7 +384,49 @@ int moe_forward(moe_layer_t *L, const void *x, int32_t T, const float *logit_noi
     ra.psum_part = reinterpret_cast<float *>(ws + p.o_psum);
     ra.logit_part = nullptr;
     ra.ksplit = 1;
-    if (L->tc) {
+    ra.x_relu = 0;
+    ra.logits_only = 0;
+    if (c.use_mlp_gater) {
+        // Hidden layer z = W_1 x + b_1 (pre-activations, [T][H] fp32), then the
+        // output layer h = W_2 relu(z) + b_2 and the routing in one kernel.
+        const int H = c.gater_hidden_dim;
+        float *z = reinterpret_cast<float *>(ws + p.o_gz);
+        if (L->tc) {
+            RouterTcArgs rt_args;
+            rt_args.w_gate = L->w.gater_w1;
+            rt_args.b_gate = L->w.gater_b1;
+            rt_args.T = T;
+            rt_args.d = c.input_dim;
+            rt_args.E = H;
+            rt_args.E_pad = router_tc_epad(H);
+            rt_args.logits = z;
+            rt_args.ksplit = 1;
+            rt_args.partial = nullptr;
+            rt_args.status = status;
+            rt_args.num_sms = L->num_sms;
+            __nv_bfloat16 *w_split = reinterpret_cast<__nv_bfloat16 *>(ws + p.o_wsplit);
+            CUtensorMap m_xr, m_ws;
+            if (!encode_bf16_2d(&m_xr, x, c.input_dim, T, kBM) ||
+                !encode_bf16_2d(&m_ws, w_split, 3ull * c.input_dim, rt_args.E_pad, router_tc_bn(H)))
+                return fail(MOE_ERR_CUDA, "cuTensorMapEncodeTiled failed for the gate operands");
+            MOE_LAUNCH(launch_router_logits_tc(m_xr, m_ws, rt_args, w_split, s, nl));
+        } else {
+            RouterArgs rh = ra;
+            rh.w_gate = L->w.gater_w1;
+            rh.b_gate = L->w.gater_b1;
+            rh.E = H;
+            rh.logits = z;
+            rh.logits_only = 1;
+            rh.noise = nullptr;
+            rh.sel_bias = nullptr;
+            MOE_LAUNCH(launch_router(rh, s, nl));
+        }
+        ra.x = z;
+        ra.x_bf16 = 0;
+        ra.x_relu = 1;
+        ra.d = H;
+        MOE_LAUNCH(launch_router(ra, s, nl));
+    } else if (L->tc) {
         RouterTcArgs rt_args;
         rt_args.w_gate = L->w.w_gate;
         rt_args.b_gate = L->w.b_gate;
@@ -398,6 +458,8 @@ int moe_forward(moe_layer_t *L, const void *x, int32_t T, const float *logit_noi
     DispatchArgs da;
     da.idx = idx;
     da.T = T;
+    da.rank_major = c.capacity_priority == MOE_PRIORITY_RANK ? 1 : 0;
+    da.n_items = da.rank_major ? k * T : T;
     da.E = E;
     da.k = k;
     da.S = S;

@@ -24,6 +24,8 @@ struct RouterArgs {
     float *psum_part;       // [router_psum_blocks][E]: per-block sums of P over its tokens
     const float *logit_part;  // routing from split-K partials: [ksplit][T][E], or null
     int ksplit;
+    int x_relu;             // fp32 router only: relu(x) is the router's input (MLP gate output layer)
+    int logits_only;        // fp32 router only: write logits (+ bias) and stop (MLP gate hidden layer)
 };
 int router_psum_blocks(int T, int num_sms, bool from_logits);
 cudaError_t launch_router(const RouterArgs &a, cudaStream_t s, int *launches);
@@ -52,9 +54,11 @@ cudaError_t launch_router_logits_tc(const CUtensorMap &map_x, const CUtensorMap 
 struct DispatchArgs {
     const int32_t *idx;     // [T][k]
     int T, E, k, S;
+    int rank_major;         // capacity priority: 0 token order, 1 choice by choice (item = r T + t)
+    int n_items;            // T (token order) or k T (rank-major)
     int64_t C;              // capacity
     int T_pad;              // T rounded up to kRowBlock (shared-expert segment length)
-    int n_chunks;           // ceil(T / 256)
+    int n_chunks;           // ceil(n_items / 256)
     int32_t *chunk_count;   // [n_chunks][E]
     int32_t *chunk_base;    // [n_chunks][E]
     int32_t *count_pre;     // [E]

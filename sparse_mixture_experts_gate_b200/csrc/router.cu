@@ -15,6 +15,11 @@
 //                             through shared memory), then route_warp;
 //   route_from_logits_kernel - bf16 layers: route_warp over the logits the
 //                             tensor-core kernel (router_tc.cu) wrote.
+// The optional MLP gate (same page, "Configuration": use_mlp_gater,
+// gater_hidden_dim) is h = W_g relu(W_1 x + b_1) + b: its hidden layer is a
+// router pass with W_1 and logits_only (or the tensor-core kernel for bf16 x),
+// its output layer router_simt_kernel over the hidden pre-activations with
+// x_relu set.
 #include "moe_common.cuh"
 #include "moe_kernels.cuh"
 
@@ -152,7 +157,9 @@ __global__ void __launch_bounds__(kThreads) router_simt_kernel(RouterArgs a) {
         for (int i = tid; i < TM * kKC; i += kThreads) {
             const int t = i / kKC, kk = i % kKC;
             const int gt = t_base + t, gk = k0 + kk;
-            xs[kk][t] = (gt < a.T && gk < a.d) ? to_f32(x[(int64_t)gt * a.d + gk]) : 0.f;
+            float v = (gt < a.T && gk < a.d) ? to_f32(x[(int64_t)gt * a.d + gk]) : 0.f;
+            if (a.x_relu) v = fmaxf(v, 0.f);
+            xs[kk][t] = v;
         }
         // Stage W_g[0 .. EP][k0 .. +KC] transposed into ws[kk][e].
         for (int i = tid; i < EP * kKC; i += kThreads) {
@@ -176,6 +183,19 @@ __global__ void __launch_bounds__(kThreads) router_simt_kernel(RouterArgs a) {
         __syncthreads();
     }
 
+    if (a.logits_only) {  // a hidden layer: pre-activations only, no routing
+#pragma unroll
+        for (int i = 0; i < RT; ++i) {
+            const int t = t_base + warp * RT + i;
+            if (t >= a.T) break;
+#pragma unroll
+            for (int q = 0; q < RE; ++q) {
+                const int e = lane + 32 * q;
+                if (e < a.E) a.logits[(int64_t)t * a.E + e] = acc[i][q] + (a.b_gate ? a.b_gate[e] : 0.f);
+            }
+        }
+        return;
+    }
     float pacc[RE];
 #pragma unroll
     for (int q = 0; q < RE; ++q) pacc[q] = 0.f;

@@ -39,7 +39,7 @@ def run_gpu(w, inp, layer: MoELayer = None, poison: bool = True):
     """One forward + aux stats through the C ABI; returns numpy copies."""
     dev = "cuda"
     if layer is None:
-        layer = MoELayer(w, {k: inp[k] for k in ("w_gate", "b_gate", "sel_bias", "w1", "b1", "w2", "b2")})
+        layer = MoELayer(w, inp)
     x = inp["x"].to(dev).contiguous()
     noise = inp["noise"].to(dev).contiguous() if inp.get("noise") is not None else None
     tl = inp["token_loss"].to(dev).contiguous() if inp.get("token_loss") is not None else None
@@ -120,7 +120,12 @@ def check_end_to_end(w, inp, g, tokens=None, table=None):
     T = inp["x"].shape[0]
     toks = np.arange(T) if tokens is None else np.asarray(tokens)
     x_rows = inp["x"][torch.as_tensor(toks)].cpu()
-    h = oracle.router_logits(x_rows, inp["w_gate"].cpu(), inp["b_gate"].cpu() if inp.get("b_gate") is not None else None)
+    bg = inp["b_gate"].cpu() if inp.get("b_gate") is not None else None
+    if w.mlp_gater:
+        g1 = inp["gater_b1"].cpu() if inp.get("gater_b1") is not None else None
+        h = oracle.router_mlp(x_rows, inp["gater_w1"].cpu(), g1, inp["w_gate"].cpu(), bg)
+    else:
+        h = oracle.router_logits(x_rows, inp["w_gate"].cpu(), bg)
     assert np.abs(g["logits"][toks] - h).max() <= LOGIT_TOL, np.abs(g["logits"][toks] - h).max()
     noise = inp["noise"].cpu()[torch.as_tensor(toks)] if (w.top_k_method == "noisy") else None
     sb = inp.get("sel_bias").cpu() if w.use_selection_bias else None

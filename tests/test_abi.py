@@ -68,6 +68,9 @@ def _weights():
     ("dtype", 9, binding.MOE_ERR_INVALID_ARG),
     ("temperature", 0.5, binding.MOE_ERR_UNSUPPORTED),
     ("max_tokens", -3, binding.MOE_ERR_INVALID_ARG),
+    ("credit_norm", 4, binding.MOE_ERR_INVALID_ARG),
+    ("capacity_priority", 2, binding.MOE_ERR_INVALID_ARG),
+    ("use_mlp_gater", 3, binding.MOE_ERR_INVALID_ARG),
 ])
 def test_create_rejects_bad_config_on_host(L, field, value, code):
     c = binding.moe_config_default()
@@ -95,6 +98,19 @@ def test_create_rejects_missing_weights(L):
     assert L.moe_layer_create(ctypes.byref(c), None, ctypes.byref(h)) == binding.MOE_ERR_INVALID_ARG
 
 
+def test_mlp_gate_config_checked_on_host(L):
+    c = binding.moe_config_default()
+    c.use_mlp_gater = 1
+    h = ctypes.c_void_p()
+    assert L.moe_layer_create(ctypes.byref(c), ctypes.byref(_weights()), ctypes.byref(h)) == binding.MOE_ERR_INVALID_ARG
+    assert "gater_w1" in binding.moe_last_error()
+    w = _weights()
+    w.gater_w1 = 0x1000
+    for H in (0, 257):
+        c.gater_hidden_dim = H
+        assert L.moe_layer_create(ctypes.byref(c), ctypes.byref(w), ctypes.byref(h)) == binding.MOE_ERR_UNSUPPORTED
+
+
 def test_null_layer_calls_fail_cleanly(L):
     assert binding.moe_workspace_bytes(None, 16) == 0
     assert binding.moe_capacity(None, 16) == -1
@@ -103,6 +119,10 @@ def test_null_layer_calls_fail_cleanly(L):
     assert L.moe_aux_stats(None, None, ctypes.byref(st), None) == binding.MOE_ERR_INVALID_ARG
     assert L.moe_device_status(None, None) == binding.MOE_ERR_INVALID_ARG
     assert binding.moe_launch_count(None) == 0
+    assert L.moe_update_selection_bias(None, None, ctypes.c_float(0.1), None, None) == binding.MOE_ERR_INVALID_ARG
+    assert L.moe_dro_update(None, None, ctypes.c_float(0.9), ctypes.c_float(1.0), None, None, None, None) == \
+        binding.MOE_ERR_INVALID_ARG
+    assert L.moe_stat_partials(None, None, None, None) == binding.MOE_ERR_INVALID_ARG
     binding.moe_destroy(None)
 
 

@@ -195,7 +195,7 @@ def test_dp_stats_two_shards_through_kernels():
     w = WORKLOADS["e64"].with_(T=1100, token_loss=True)
     inp = make_inputs(w, "cpu", seed=21)
     cuts = [0, 389, w.T]
-    layer = MoELayer(w, {k: inp[k] for k in ("w_gate", "b_gate", "sel_bias", "w1", "b1", "w2", "b2")})
+    layer = MoELayer(w, inp)
     total = torch.zeros(stat_partials_size(w.E), dtype=torch.float32, device="cuda")
     shards = []
     s = torch.cuda.current_stream().cuda_stream
@@ -323,3 +323,34 @@ def test_dro_update_matches_oracle():
         assert np.abs(dlh.cpu().numpy() - want_lh).max() <= 1e-6 * (1 + np.abs(want_lh).max())
         assert np.abs(dmu.cpu().numpy() - want_mu).max() <= 1e-6
         assert abs(obj.item() - want_obj) <= 1e-6 * (1 + abs(want_obj))
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "fp32"])
+def test_rank_major_capacity_priority(dtype):
+    """GShard-style capacity priority (every first choice before any second
+    choice): bit-exact slots and drops on the same logits, with heavy drops."""
+    w = WORKLOADS["default"].with_(T=1500, E=16, k=4, S=0, capacity_factor=0.6, capacity_priority="rank",
+                                   dtype=dtype, d=128 if dtype == "bf16" else 64,
+                                   F=256 if dtype == "bf16" else 64, O=128 if dtype == "bf16" else 64)
+    inp = make_inputs(w, "cpu", seed=23)
+    g, layer = run_gpu(w, inp)
+    # C_f = 0.6 is stored as fp32 (0.600000024): C = ceil(fl32(C_f) k T / E).
+    from sparse_mixture_experts_gate_b200.binding import moe_capacity
+    assert moe_capacity(layer.handle, w.T) == oracle.capacity(oracle.layer_capacity_factor(w), w.k, w.T, w.E)
+    check_same_logits_routing(w, inp, g)
+    check_end_to_end(w, inp, g)
+    assert g["n_dropped"][0] > 0
+    # The priority changes which assignments drop, not how many per expert.
+    r_tok = oracle.routing_from_logits(g["logits"].astype(np.float32), w.with_(capacity_priority="token"))
+    assert np.array_equal(g["count_kept"], r_tok["count_kept"])
+    assert not np.array_equal(g["slot"], r_tok["slot"])
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "fp32"])
+def test_mlp_gate_router(dtype):
+    """The optional MLP gate (use_mlp_gater, hidden 128): logits against the
+    oracle's h = W_2 relu(W_1 x + b_1) + b_2, routing and outputs as usual."""
+    w = WORKLOADS["default"].with_(T=700, E=24, k=3, S=1, mlp_gater=True, router_bias=True, dtype=dtype,
+                                   d=256 if dtype == "bf16" else 64, F=256 if dtype == "bf16" else 64,
+                                   O=128 if dtype == "bf16" else 32, use_selection_bias=True)
+    full_check(w, make_inputs(w, "cpu", seed=29, random_biases=True))
