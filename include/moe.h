@@ -53,7 +53,8 @@ enum {
     MOE_ERR_CUDA = -3,         /* a CUDA runtime or driver call failed         */
     MOE_ERR_WORKSPACE = -4,    /* workspace NULL, misaligned or too small      */
     MOE_ERR_TIMEOUT = -5,      /* a bounded device-side wait gave up           */
-    MOE_ERR_STATE = -6         /* call out of order (stats before a forward)   */
+    MOE_ERR_STATE = -6,        /* call out of order (stats before a forward)   */
+    MOE_ERR_INTERNAL = -7      /* a self-check found the library misbehaving   */
 };
 
 /* Activations ("Code Walkthrough - SER", gating / routing path: ReLU, GELU, Swish).
@@ -303,6 +304,15 @@ MOE_API int moe_update_selection_bias(moe_layer_t *layer, const float *partials,
  * reduction order. Errors: INVALID_ARG for NULL arrays or non-finite ema/eta. */
 MOE_API int moe_dro_update(moe_layer_t *layer, const float *expert_loss, float ema, float eta, float *lhat,
                            float *mu, float *objective, void *stream);
+
+/* Self-check of the bounded waits the tcgen05 kernels rely on (no counterpart
+ * on the pages): one GPU thread waits on an mbarrier that nothing arrives on;
+ * after the wait limit (2 s) it records the timeout and returns, as every role
+ * of the expert GEMM and router kernels does when a wait runs out. Synchronises
+ * `stream`. Returns MOE_OK when the timeout was detected and reported as
+ * designed (the context stays usable), MOE_ERR_INTERNAL if it was not,
+ * MOE_ERR_CUDA on a CUDA error. Takes about two seconds. */
+MOE_API int moe_selftest_bounded_wait(void *stream);
 
 /* Device status word of the most recent forward: synchronises `stream`, then
  * returns MOE_OK, or MOE_ERR_TIMEOUT if a bounded device-side wait gave up. */

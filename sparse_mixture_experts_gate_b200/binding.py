@@ -14,7 +14,7 @@ PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(PKG, "libmoe.so")
 
 MOE_OK, MOE_ERR_INVALID_ARG, MOE_ERR_UNSUPPORTED, MOE_ERR_CUDA = 0, -1, -2, -3
-MOE_ERR_WORKSPACE, MOE_ERR_TIMEOUT, MOE_ERR_STATE = -4, -5, -6
+MOE_ERR_WORKSPACE, MOE_ERR_TIMEOUT, MOE_ERR_STATE, MOE_ERR_INTERNAL = -4, -5, -6, -7
 MOE_ACT = {"relu": 0, "gelu": 1, "swish": 2}
 MOE_TOPK = {"greedy": 0, "noisy": 1}
 MOE_DTYPE = {"bf16": 0, "fp32": 1}
@@ -24,7 +24,7 @@ MOE_PRIORITY = {"token": 0, "rank": 1}
 # Every symbol include/moe.h declares.
 EXPORTS = ("moe_config_default", "moe_layer_create", "moe_workspace_bytes", "moe_capacity", "moe_forward",
            "moe_forward_noalloc", "moe_aux_stats", "moe_stat_partials", "moe_stats_from_partials",
-           "moe_update_selection_bias", "moe_dro_update", "moe_device_status", "moe_set_timing_events", "moe_launch_count", "moe_destroy", "moe_status_string",
+           "moe_update_selection_bias", "moe_dro_update", "moe_selftest_bounded_wait", "moe_device_status", "moe_set_timing_events", "moe_launch_count", "moe_destroy", "moe_status_string",
            "moe_last_error")
 
 
@@ -96,6 +96,8 @@ def lib() -> ctypes.CDLL:
         L.moe_update_selection_bias.argtypes = [vp, vp, ctypes.c_float, vp, vp]
         L.moe_dro_update.restype = ctypes.c_int
         L.moe_dro_update.argtypes = [vp, vp, ctypes.c_float, ctypes.c_float, vp, vp, vp, vp]
+        L.moe_selftest_bounded_wait.restype = ctypes.c_int
+        L.moe_selftest_bounded_wait.argtypes = [vp]
         L.moe_device_status.restype = ctypes.c_int
         L.moe_device_status.argtypes = [vp, vp]
         L.moe_set_timing_events.restype = ctypes.c_int
@@ -197,6 +199,10 @@ def moe_dro_update(layer: int, expert_loss: int, ema: float, eta: float, lhat: i
                    objective: Optional[int], stream: int) -> int:
     return _check(lib().moe_dro_update(layer, expert_loss, float(ema), float(eta), lhat, mu, objective, stream),
                   "moe_dro_update")
+
+
+def moe_selftest_bounded_wait(stream: int) -> int:
+    return _check(lib().moe_selftest_bounded_wait(stream), "moe_selftest_bounded_wait")
 
 
 def moe_device_status(layer: int, stream: int) -> int:
@@ -367,3 +373,76 @@ class MoELayer:
 
     def launch_count(self) -> int:
         return moe_launch_count(self.handle)
+
+
+class HostPipeline:
+    """Forwards whose inputs and outputs live in pinned host memory, pipelined:
+    step i's host-to-device input copy (on an upload stream), its forward and
+    statistics (compute stream) and its result copy back (download stream)
+    overlap with the neighbouring steps'. Two device slots alternate; events
+    order every reuse of a slot, so each step's result is exactly what a
+    serial copy-forward-copy would give.
+
+    submit() enqueues one step and returns at once; synchronize() waits for all
+    submitted steps. The host tensors of a step must stay untouched until
+    synchronize() (or until the step's download has completed)."""
+
+    STAT_KEYS = ("l_aux", "l_z", "n_dropped", "f", "p_mean", "expert_loss", "importance", "cv_load",
+                 "cv_importance", "l_total")
+
+    def __init__(self, layer: "MoELayer", T: int, with_noise: bool = False, with_loss: bool = False):
+        import torch
+        self.layer, self.T = layer, T
+        dev = layer.device
+        w = layer.w
+        self.up = torch.cuda.Stream(dev)
+        self.comp = torch.cuda.Stream(dev)
+        self.down = torch.cuda.Stream(dev)
+        self.slots = []
+        for _ in range(2):
+            self.slots.append(dict(
+                x=torch.empty(T, w.d, dtype=layer._dt, device=dev),
+                noise=torch.empty(T, w.E, dtype=torch.float32, device=dev) if with_noise else None,
+                loss=torch.empty(T, dtype=torch.float32, device=dev) if with_loss else None,
+                out=layer.alloc_outputs(T),
+                uploaded=torch.cuda.Event(), computed=torch.cuda.Event(), downloaded=torch.cuda.Event(),
+                used=False))
+        layer.workspace(T)
+        self.n = 0
+
+    def submit(self, x_h, y_h, noise_h=None, loss_h=None, stats_h=None):
+        """One step: x_h [T][d] (pinned host, the layer's dtype) in, y_h [T][O] out;
+        optional noise [T][E] and token losses [T] in, and a dict of pinned host
+        tensors (keys of STAT_KEYS) that receive the step's statistics."""
+        import torch
+        sl = self.slots[self.n % 2]
+        self.n += 1
+        with torch.cuda.stream(self.up):
+            if sl["used"]:
+                self.up.wait_event(sl["computed"])  # the slot's previous forward has read its inputs
+            sl["x"].copy_(x_h, non_blocking=True)
+            if noise_h is not None:
+                sl["noise"].copy_(noise_h, non_blocking=True)
+            if loss_h is not None:
+                sl["loss"].copy_(loss_h, non_blocking=True)
+            sl["uploaded"].record(self.up)
+        with torch.cuda.stream(self.comp):
+            self.comp.wait_event(sl["uploaded"])
+            if sl["used"]:
+                self.comp.wait_event(sl["downloaded"])  # the slot's previous results have left
+            s = self.comp.cuda_stream
+            self.layer.forward(sl["x"], noise=sl["noise"] if noise_h is not None else None, out=sl["out"], stream=s)
+            self.layer.aux_stats(sl["out"], token_loss=sl["loss"] if loss_h is not None else None, stream=s)
+            sl["computed"].record(self.comp)
+        with torch.cuda.stream(self.down):
+            self.down.wait_event(sl["computed"])
+            y_h.copy_(sl["out"]["y"], non_blocking=True)
+            for k, v in (stats_h or {}).items():
+                v.copy_(sl["out"][k], non_blocking=True)
+            sl["downloaded"].record(self.down)
+        sl["used"] = True
+
+    def synchronize(self):
+        self.down.synchronize()
+        self.comp.synchronize()
+        self.up.synchronize()

@@ -782,6 +782,7 @@ const char *moe_status_string(int status) {
         case MOE_ERR_WORKSPACE: return "MOE_ERR_WORKSPACE";
         case MOE_ERR_TIMEOUT: return "MOE_ERR_TIMEOUT";
         case MOE_ERR_STATE: return "MOE_ERR_STATE";
+        case MOE_ERR_INTERNAL: return "MOE_ERR_INTERNAL";
         default: return "MOE_ERR_UNKNOWN";
     }
 }

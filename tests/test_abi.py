@@ -44,7 +44,7 @@ def test_config_default_mirrors_ser_configuration(L):
 def test_status_strings(L):
     for code, name in ((0, "MOE_OK"), (-1, "MOE_ERR_INVALID_ARG"), (-2, "MOE_ERR_UNSUPPORTED"),
                        (-3, "MOE_ERR_CUDA"), (-4, "MOE_ERR_WORKSPACE"), (-5, "MOE_ERR_TIMEOUT"),
-                       (-6, "MOE_ERR_STATE")):
+                       (-6, "MOE_ERR_STATE"), (-7, "MOE_ERR_INTERNAL")):
         assert binding.moe_status_string(code) == name
 
 

@@ -354,3 +354,43 @@ def test_mlp_gate_router(dtype):
                                    d=256 if dtype == "bf16" else 64, F=256 if dtype == "bf16" else 64,
                                    O=128 if dtype == "bf16" else 32, use_selection_bias=True)
     full_check(w, make_inputs(w, "cpu", seed=29, random_biases=True))
+
+
+def test_host_pipeline_matches_serial_forward():
+    """binding.HostPipeline (pinned host inputs and outputs, copies overlapped
+    with the neighbouring steps' compute) gives bit-for-bit the results of the
+    plain device forward, for several different batches in flight."""
+    from sparse_mixture_experts_gate_b200.binding import HostPipeline
+    from sparse_mixture_experts_gate_b200.workloads import make_tokens
+    w = WORKLOADS["e64"].with_(T=640, token_loss=True)
+    inp = make_inputs(w, "cpu", seed=41)
+    layer = MoELayer(w, inp)
+    batches = [make_tokens(w, "cpu", seed=100 + i) for i in range(4)]
+    want = []
+    for b in batches:
+        out = layer.forward(b["x"].cuda(), out=None)
+        layer.aux_stats(out, token_loss=b["token_loss"].cuda())
+        torch.cuda.synchronize()
+        want.append({k: v.cpu().clone() for k, v in out.items()})
+    pipe = HostPipeline(layer, w.T, with_loss=True)
+    ys = [torch.empty(w.T, w.O, dtype=torch.bfloat16).pin_memory() for _ in batches]
+    sts = [{k: torch.empty_like(want[0][k]).pin_memory() for k in HostPipeline.STAT_KEYS} for _ in batches]
+    xs = [b["x"].pin_memory() for b in batches]
+    ls = [b["token_loss"].pin_memory() for b in batches]
+    for i in range(len(batches)):
+        pipe.submit(xs[i], ys[i], loss_h=ls[i], stats_h=sts[i])
+    pipe.synchronize()
+    for i in range(len(batches)):
+        assert torch.equal(ys[i], want[i]["y"]), f"batch {i}: y differs"
+        for k in HostPipeline.STAT_KEYS:
+            assert torch.equal(sts[i][k], want[i][k]), f"batch {i}: {k} differs"
+
+
+def test_bounded_wait_times_out_and_context_survives():
+    """Failure detection without a GPU fault: a wait on a barrier nothing
+    arrives on gives up after its limit and reports the timeout; afterwards the
+    context still runs a forward that matches the oracle."""
+    from sparse_mixture_experts_gate_b200.binding import moe_selftest_bounded_wait
+    assert moe_selftest_bounded_wait(torch.cuda.current_stream().cuda_stream) == 0
+    w = WORKLOADS["default"].with_(T=300)
+    full_check(w, make_inputs(w, "cpu", seed=2))
