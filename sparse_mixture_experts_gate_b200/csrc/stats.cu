@@ -28,55 +28,6 @@ __device__ __forceinline__ float warp_sum(float v) {
 //   [2E+2]       dropped assignments    [2E+3, 3E+3) sum over kept assignments
 //                                                    of credit * token_loss
 //   [3E+3, 4E+3) importance: sum of the selections' gates per expert
-// One warp per expert; every sum has a fixed order (lane-strided, then a fixed
-// shuffle tree), so repeated runs give bit-identical results.
-__global__ void __launch_bounds__(256) stat_partials_expert_kernel(StatsArgs a) {
-    const int e = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
-    if (e >= a.E) return;
-    float ps = 0.f;
-    for (int i = lane; i < a.n_chunks; i += 32) ps += a.psum_part[(int64_t)i * a.E + e];
-    ps = warp_sum(ps);
-    float el = 0.f;
-    if (a.token_loss) {
-        const int r0 = a.group_start[e], r1 = r0 + a.group_rows[e];
-        for (int row = r0 + lane; row < r1; row += 32) {
-            const int ai = a.row_assign[row];
-            el += a.credit[ai] * a.token_loss[ai / a.k];
-        }
-        el = warp_sum(el);
-    }
-    // Importance: this expert's selection gates, in token order.
-    float imp = 0.f;
-    {
-        const int g0 = a.pre_start[e], n = a.count_pre[e];
-        for (int j = lane; j < n; j += 32) imp += a.gate_sorted[g0 + j];
-        imp = warp_sum(imp);
-    }
-    if (lane == 0) {
-        a.partials[e] = ps;
-        a.partials[a.E + e] = (float)a.count_pre[e];
-        a.partials[2 * a.E + 3 + e] = el;
-        a.partials[3 * a.E + 3 + e] = imp;
-    }
-}
-
-__global__ void __launch_bounds__(256) stat_partials_scalar_kernel(StatsArgs a) {
-    __shared__ float red[8];
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    float z = 0.f;
-    for (int t = tid; t < a.T; t += 256) z = fmaf(a.lse[t], a.lse[t], z);
-    z = warp_sum(z);
-    if (lane == 0) red[warp] = z;
-    __syncthreads();
-    if (tid == 0) {
-        float zt = 0.f;
-        for (int w = 0; w < 8; ++w) zt += red[w];
-        a.partials[2 * a.E] = zt;
-        a.partials[2 * a.E + 1] = (float)a.T;
-        a.partials[2 * a.E + 2] = (float)a.ctrl[kCtrlDropped];
-    }
-}
-
 // Sum over the 256 threads of one CTA in a fixed order (shuffle tree, then the
 // eight warp sums in order); every thread gets the result.
 __device__ __forceinline__ float block_sum_256(float v, float *red) {
@@ -89,6 +40,51 @@ __device__ __forceinline__ float block_sum_256(float v, float *red) {
 #pragma unroll
     for (int w = 0; w < 8; ++w) t += red[w];
     return t;
+}
+
+// One CTA per expert (CTA E does the per-token scalars); every sum has a fixed
+// order (thread-strided, then a fixed shuffle tree and warp order), so repeated
+// runs give bit-identical results.
+__global__ void __launch_bounds__(256) stat_partials_kernel(StatsArgs a) {
+    __shared__ float red[8];
+    const int tid = threadIdx.x;
+    if (blockIdx.x == a.E) {  // sum_t lse_t^2, T, drops
+        float z = 0.f;
+        for (int t = tid; t < a.T; t += 256) z = fmaf(a.lse[t], a.lse[t], z);
+        z = block_sum_256(z, red);
+        if (tid == 0) {
+            a.partials[2 * a.E] = z;
+            a.partials[2 * a.E + 1] = (float)a.T;
+            a.partials[2 * a.E + 2] = (float)a.ctrl[kCtrlDropped];
+        }
+        return;
+    }
+    const int e = blockIdx.x;
+    float ps = 0.f;
+    for (int i = tid; i < a.n_chunks; i += 256) ps += a.psum_part[(int64_t)i * a.E + e];
+    ps = block_sum_256(ps, red);
+    float el = 0.f;
+    if (a.token_loss) {
+        const int r0 = a.group_start[e], r1 = r0 + a.group_rows[e];
+        for (int row = r0 + tid; row < r1; row += 256) {
+            const int ai = a.row_assign[row];
+            el += a.credit[ai] * a.token_loss[ai / a.k];
+        }
+        el = block_sum_256(el, red);
+    }
+    // Importance: this expert's selection gates, in priority order.
+    float imp = 0.f;
+    {
+        const int g0 = a.pre_start[e], n = a.count_pre[e];
+        for (int j = tid; j < n; j += 256) imp += a.gate_sorted[g0 + j];
+        imp = block_sum_256(imp, red);
+    }
+    if (tid == 0) {
+        a.partials[e] = ps;
+        a.partials[a.E + e] = (float)a.count_pre[e];
+        a.partials[2 * a.E + 3 + e] = el;
+        a.partials[3 * a.E + 3 + e] = imp;
+    }
 }
 
 // Squared coefficient of variation of one value per thread (threads >= n hold
@@ -230,9 +226,8 @@ __global__ void __launch_bounds__(256) dro_update_kernel(DroArgs a) {
 }  // namespace
 
 cudaError_t launch_stat_partials(const StatsArgs &a, cudaStream_t s, int *launches) {
-    stat_partials_expert_kernel<<<(a.E * 32 + 255) / 256, 256, 0, s>>>(a);
-    stat_partials_scalar_kernel<<<1, 256, 0, s>>>(a);
-    *launches += 2;
+    stat_partials_kernel<<<a.E + 1, 256, 0, s>>>(a);
+    *launches += 1;
     return cudaGetLastError();
 }
 
