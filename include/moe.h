@@ -104,6 +104,8 @@ typedef struct {
     int32_t capacity_priority; /* MOE_PRIORITY_*                                    */
     int32_t use_mlp_gater;    /* 1: logits from the MLP gate (SER "Configuration") */
     int32_t gater_hidden_dim; /* H of the MLP gate, 1..256 (default 128)           */
+    int32_t ep_size;          /* expert-parallel group size G (1 = all experts here) */
+    int32_t ep_rank;          /* this rank's place in it, 0..G-1                    */
 } moe_config_t;
 
 /* Defaults of the SER walkthrough's configuration: E=8, k=2, 512/1024/512,
@@ -123,6 +125,9 @@ MOE_API moe_config_t moe_config_default(void);
  *   gater_b1 [H]       fp32, its bias b_1                          (NULL = zero)
  * The MLP gate ("Code Walkthrough - SER": "via the router/router_bias linear
  * layer, or the optional MLP gate") is h = W_2 relu(W_1 x + b_1) + b_2.
+ * With ep_size = G > 1 the expert stacks hold only this rank's E/G routed
+ * experts (global ids ep_rank*E/G ..), then the S shared experts; the router
+ * (w_gate, b_gate, sel_bias) covers all E experts.
  *   sel_bias [E]       fp32, selection bias b_i                    (required iff use_selection_bias)
  *   w1       [G][F][d] dtype, first expert layer (row f, column j) (required)
  *   b1       [G][F]    fp32                                        (NULL = zero)
@@ -304,6 +309,44 @@ MOE_API int moe_update_selection_bias(moe_layer_t *layer, const float *partials,
  * reduction order. Errors: INVALID_ARG for NULL arrays or non-finite ema/eta. */
 MOE_API int moe_dro_update(moe_layer_t *layer, const float *expert_loss, float ema, float eta, float *lhat,
                            float *mu, float *objective, void *stream);
+
+/* Expert parallelism ("Appendix C - Acronyms & Symbols", "Capacity &
+ * communication": with expert-parallel degree G each device holds E/G experts
+ * and tokens reach them by an all-to-all dispatch and come back by an
+ * all-to-all combine). For layers created with ep_size = G > 1 (bf16 only);
+ * moe_forward returns MOE_ERR_STATE for them. One forward on every rank:
+ *   1. moe_ep_dispatch: router, top-k, dispatch with this rank's capacity
+ *      C = ceil(C_f k T / E) over all E experts, and the rows of the kept
+ *      assignments scattered into the row space (expert-major, each expert's
+ *      rows padded to 32). Arguments as moe_forward without y.
+ *   2. moe_ep_layout (synchronises `stream`): expert_rows (host [E]) = rows of
+ *      each expert's padded segment; rows_in / rows_out = device pointers to the
+ *      row space's input rows [sum expert_rows][d] (send buffer) and output rows
+ *      [..][O] (receive buffer of step 5), valid until the next dispatch. The
+ *      rows for rank q are the contiguous segments of experts q E/G ..
+ *      (q+1) E/G - 1.
+ *   3. the caller's all-to-all (e.g. NCCL): send each rank its segments and
+ *      its E/G expert_rows entries; receive R rows, source-major.
+ *   4. moe_ep_experts: the expert MLPs of this rank's experts on the received
+ *      rows: recv_x [R][d] bf16, recv_rows device [G][E/G] int32 (padded rows
+ *      per source and local expert, summing to R), recv_out [R][O] bf16 out;
+ *      workspace of moe_ep_experts_workspace_bytes(R) bytes, 256-byte aligned.
+ *      R must be a multiple of 32.
+ *   5. the caller's all-to-all back: recv_out rows to their sources, into
+ *      rows_out at the positions their inputs left from.
+ *   6. moe_ep_combine: the shared experts on this rank's tokens and the
+ *      gate-weighted combine into y [T][O]; moe_aux_stats may follow.
+ * x and the workspace of step 1 must stay valid and unchanged until step 6 (the
+ * shared experts read x there).
+ * Errors: STATE for layers with ep_size 1 or calls out of order, INVALID_ARG,
+ * WORKSPACE, CUDA as elsewhere. */
+MOE_API int moe_ep_dispatch(moe_layer_t *layer, const void *x, int32_t T, const float *logit_noise, void *workspace,
+                            size_t ws_bytes, const moe_routing_t *routing, void *stream);
+MOE_API int moe_ep_layout(moe_layer_t *layer, int32_t *expert_rows, void **rows_in, void **rows_out, void *stream);
+MOE_API size_t moe_ep_experts_workspace_bytes(const moe_layer_t *layer, int32_t R);
+MOE_API int moe_ep_experts(moe_layer_t *layer, const void *recv_x, const int32_t *recv_rows, int32_t R,
+                           void *recv_out, void *workspace, size_t ws_bytes, void *stream);
+MOE_API int moe_ep_combine(moe_layer_t *layer, void *y, void *stream);
 
 /* Self-check of the bounded waits the tcgen05 kernels rely on (no counterpart
  * on the pages): one GPU thread waits on an mbarrier that nothing arrives on;

@@ -24,7 +24,8 @@ MOE_PRIORITY = {"token": 0, "rank": 1}
 # Every symbol include/moe.h declares.
 EXPORTS = ("moe_config_default", "moe_layer_create", "moe_workspace_bytes", "moe_capacity", "moe_forward",
            "moe_forward_noalloc", "moe_aux_stats", "moe_stat_partials", "moe_stats_from_partials",
-           "moe_update_selection_bias", "moe_dro_update", "moe_selftest_bounded_wait", "moe_device_status", "moe_set_timing_events", "moe_launch_count", "moe_destroy", "moe_status_string",
+           "moe_update_selection_bias", "moe_dro_update", "moe_selftest_bounded_wait",
+           "moe_ep_dispatch", "moe_ep_layout", "moe_ep_experts_workspace_bytes", "moe_ep_experts", "moe_ep_combine", "moe_device_status", "moe_set_timing_events", "moe_launch_count", "moe_destroy", "moe_status_string",
            "moe_last_error")
 
 
@@ -36,7 +37,7 @@ class MoeConfig(ctypes.Structure):
                 ("dtype", ctypes.c_int32), ("max_tokens", ctypes.c_int32), ("load_balance_coef", ctypes.c_float),
                 ("z_loss_coef", ctypes.c_float), ("temperature", ctypes.c_float), ("credit_norm", ctypes.c_int32),
                 ("capacity_priority", ctypes.c_int32), ("use_mlp_gater", ctypes.c_int32),
-                ("gater_hidden_dim", ctypes.c_int32)]
+                ("gater_hidden_dim", ctypes.c_int32), ("ep_size", ctypes.c_int32), ("ep_rank", ctypes.c_int32)]
 
 
 class MoeWeights(ctypes.Structure):
@@ -96,6 +97,16 @@ def lib() -> ctypes.CDLL:
         L.moe_update_selection_bias.argtypes = [vp, vp, ctypes.c_float, vp, vp]
         L.moe_dro_update.restype = ctypes.c_int
         L.moe_dro_update.argtypes = [vp, vp, ctypes.c_float, ctypes.c_float, vp, vp, vp, vp]
+        L.moe_ep_dispatch.restype = ctypes.c_int
+        L.moe_ep_dispatch.argtypes = [vp, vp, i32, vp, vp, sz, ctypes.POINTER(MoeRouting), vp]
+        L.moe_ep_layout.restype = ctypes.c_int
+        L.moe_ep_layout.argtypes = [vp, vp, ctypes.POINTER(vp), ctypes.POINTER(vp), vp]
+        L.moe_ep_experts_workspace_bytes.restype = sz
+        L.moe_ep_experts_workspace_bytes.argtypes = [vp, i32]
+        L.moe_ep_experts.restype = ctypes.c_int
+        L.moe_ep_experts.argtypes = [vp, vp, vp, i32, vp, vp, sz, vp]
+        L.moe_ep_combine.restype = ctypes.c_int
+        L.moe_ep_combine.argtypes = [vp, vp, vp]
         L.moe_selftest_bounded_wait.restype = ctypes.c_int
         L.moe_selftest_bounded_wait.argtypes = [vp]
         L.moe_device_status.restype = ctypes.c_int
@@ -240,7 +251,8 @@ class MoELayer:
     workspace and the routing/statistics output buffers. Pointer marshalling
     only; the forward itself is moe_forward + moe_aux_stats."""
 
-    def __init__(self, workload, weights: Dict[str, object], max_tokens: Optional[int] = None, device="cuda"):
+    def __init__(self, workload, weights: Dict[str, object], max_tokens: Optional[int] = None, device="cuda",
+                 ep_size: int = 1, ep_rank: int = 0):
         import torch
         w = workload
         self.w = w
@@ -260,6 +272,7 @@ class MoELayer:
         cfg.capacity_priority = MOE_PRIORITY[w.capacity_priority]
         cfg.use_mlp_gater = int(w.mlp_gater)
         cfg.gater_hidden_dim = w.gater_hidden
+        cfg.ep_size, cfg.ep_rank = ep_size, ep_rank
         self.cfg = cfg
         self.weights = {k: (v.to(self.device).contiguous() if v is not None else None)
                         for k, v in weights.items()
@@ -366,6 +379,68 @@ class MoELayer:
                                 self._stats_struct(out, token_loss is not None, False), s)
         return out, partials
 
+    # ------------------------------------------------------ expert parallelism
+    # A layer created with ep_size = G > 1 holds experts ep_rank*E/G .. of the
+    # stacks it is given (then the shared experts). ep_forward runs the whole
+    # forward over torch.distributed; the three phases below are the pieces.
+
+    def ep_dispatch(self, x, noise=None, out=None, stream=None):
+        """Phase 1: routing and dispatch of this rank's tokens. Returns (out,
+        send rows [n][d], output rows [n][O] (the row space, views of the
+        workspace), expert_rows: padded rows per expert, a host list)."""
+        import torch
+        T = int(x.shape[0])
+        if out is None:
+            out = self.alloc_outputs(T)
+        ws, _ = self.workspace(T)
+        s = stream if stream is not None else torch.cuda.current_stream(self.device).cuda_stream
+        routing = MoeRouting(_ptr(out["logits"]), _ptr(out["gates"]), _ptr(out["topk_idx"]), _ptr(out["slot"]),
+                             _ptr(out["count_pre"]), _ptr(out["count_kept"]))
+        _check(lib().moe_ep_dispatch(self.handle, _ptr(x), T, _ptr(noise), ws.data_ptr(), ws.numel(),
+                                     ctypes.byref(routing), s), "moe_ep_dispatch")
+        rows = (ctypes.c_int32 * self.w.E)()
+        rin, rout = ctypes.c_void_p(), ctypes.c_void_p()
+        _check(lib().moe_ep_layout(self.handle, rows, ctypes.byref(rin), ctypes.byref(rout), s), "moe_ep_layout")
+        n = int(sum(rows))
+        esz = 2 if self.w.dtype == "bf16" else 4
+        oi, oo = rin.value - ws.data_ptr(), rout.value - ws.data_ptr()
+        send = ws[oi:oi + n * self.w.d * esz].view(self._dt).view(n, self.w.d)
+        back = ws[oo:oo + n * self.w.O * esz].view(self._dt).view(n, self.w.O)
+        return out, send, back, list(rows)
+
+    def ep_experts(self, recv_x, recv_rows, stream=None):
+        """Phase 3: this rank's experts on the received rows (recv_rows: device
+        int32 [G][E/G], padded rows per source and local expert). Returns [R][O]."""
+        import torch
+        R = int(recv_x.shape[0])
+        recv_out = torch.empty(R, self.w.O, dtype=self._dt, device=self.device)
+        need = lib().moe_ep_experts_workspace_bytes(self.handle, R)
+        if getattr(self, "_ws2", None) is None or self._ws2.numel() < need:
+            self._ws2 = torch.empty(max(need, 256), dtype=torch.uint8, device=self.device)
+        s = stream if stream is not None else torch.cuda.current_stream(self.device).cuda_stream
+        rr = recv_rows.to(torch.int32).contiguous()
+        _check(lib().moe_ep_experts(self.handle, _ptr(recv_x.contiguous()), rr.data_ptr(), R, recv_out.data_ptr(),
+                                    self._ws2.data_ptr(), self._ws2.numel(), s), "moe_ep_experts")
+        return recv_out
+
+    def ep_combine(self, out, stream=None):
+        """Phase 5: shared experts and the combine into out["y"]."""
+        import torch
+        s = stream if stream is not None else torch.cuda.current_stream(self.device).cuda_stream
+        _check(lib().moe_ep_combine(self.handle, _ptr(out["y"]), s), "moe_ep_combine")
+        return out
+
+    def ep_forward(self, x, noise=None, out=None, group=None):
+        """The whole expert-parallel forward: dispatch, all-to-all of the rows
+        (and of the per-expert row counts), this rank's experts, all-to-all
+        back, combine. Every rank of `group` calls it at the same step."""
+        G = self.cfg.ep_size
+        out, send, back, rows = self.ep_dispatch(x, noise=noise, out=out)
+        recv_x, recv_rows, send_splits, recv_splits = ep_exchange(send, rows, G, group)
+        recv_out = self.ep_experts(recv_x, recv_rows)
+        ep_return(recv_out, back, send_splits, recv_splits, group)
+        return self.ep_combine(out)
+
     def device_status(self, stream=None) -> int:
         import torch
         s = stream if stream is not None else torch.cuda.current_stream(self.device).cuda_stream
@@ -373,6 +448,45 @@ class MoELayer:
 
     def launch_count(self) -> int:
         return moe_launch_count(self.handle)
+
+
+def ep_send_splits(expert_rows, G: int):
+    """Rows this rank sends to each rank q: the padded segments of q's experts
+    (experts q E/G .. (q+1) E/G - 1, contiguous in the row space)."""
+    El = len(expert_rows) // G
+    return [int(sum(expert_rows[q * El:(q + 1) * El])) for q in range(G)]
+
+
+def ep_exchange(send_rows, expert_rows, G: int, group=None):
+    """All-to-all dispatch: every rank sends each rank its E/G per-expert row
+    counts and then its rows. Returns (received rows [R][d], received counts
+    [G][E/G] (source-major, on the rows' device), send splits, receive splits)."""
+    import torch
+    import torch.distributed as dist
+    El = len(expert_rows) // G
+    dev = send_rows.device
+    cnt_send = torch.tensor(expert_rows, dtype=torch.int32, device=dev)
+    cnt_recv = torch.empty_like(cnt_send)
+    dist.all_to_all_single(cnt_recv, cnt_send, group=group)
+    send_splits = ep_send_splits(expert_rows, G)
+    recv_counts = cnt_recv.view(G, El)
+    recv_splits = [int(v) for v in recv_counts.sum(1).tolist()]
+    recv = torch.empty(sum(recv_splits), send_rows.shape[1], dtype=send_rows.dtype, device=dev)
+    dist.all_to_all_single(recv, send_rows[:sum(send_splits)].contiguous(), recv_splits, send_splits, group=group)
+    return recv, recv_counts, send_splits, recv_splits
+
+
+def ep_return(recv_out, back_rows, send_splits, recv_splits, group=None):
+    """All-to-all combine: the expert outputs of the received rows go back to
+    their sources, into the row positions their inputs left from."""
+    import torch.distributed as dist
+    n = sum(send_splits)
+    if n == back_rows.shape[0] and back_rows.is_contiguous():
+        dist.all_to_all_single(back_rows, recv_out, send_splits, recv_splits, group=group)
+    else:
+        tmp = back_rows.new_empty((n, back_rows.shape[1]))
+        dist.all_to_all_single(tmp, recv_out, send_splits, recv_splits, group=group)
+        back_rows[:n].copy_(tmp)
 
 
 class HostPipeline:

@@ -137,6 +137,7 @@ __global__ void __launch_bounds__(kMaxE) dispatch_scan_kernel(DispatchArgs a) {
         a.group_start[a.E + a.S] = total;
         a.ctrl[kCtrlNumRowBlocks] = total / kRowBlock;
         a.ctrl[kCtrlNumTokTiles] = routed_tiles + a.S * shared_tiles;
+        a.ctrl[kCtrlRoutedTiles] = routed_tiles;
         a.ctrl[kCtrlRoutedRows] = routed_rows;
         a.ctrl[kCtrlDropped] = d;
     }
@@ -205,6 +206,42 @@ __global__ void __launch_bounds__(256) scatter_rows_kernel(ScatterArgs a) {
 }
 
 }  // namespace
+
+// Token tiles over rows received from G ranks: segment s = (source s / El,
+// local expert s % El) holds recv_rows[s] rows (a multiple of 32), split into
+// tiles of at most 256 rows. One CTA, thread s owns segment s (G El <= 256).
+__global__ void __launch_bounds__(kMaxE) ep_tiles_kernel(EpTilesArgs a) {
+    __shared__ int sc_rows[kMaxE];
+    __shared__ int sc_tiles[kMaxE];
+    const int s = threadIdx.x, nseg = a.G * a.El;
+    const int rows = s < nseg ? a.recv_rows[s] : 0;
+    const int tiles = (rows + kTokTile - 1) / kTokTile;
+    sc_rows[s] = rows;
+    sc_tiles[s] = tiles;
+    __syncthreads();
+    for (int off = 1; off < kMaxE; off <<= 1) {
+        const int vr = s >= off ? sc_rows[s - off] : 0;
+        const int vt = s >= off ? sc_tiles[s - off] : 0;
+        __syncthreads();
+        sc_rows[s] += vr;
+        sc_tiles[s] += vt;
+        __syncthreads();
+    }
+    const int row0 = sc_rows[s] - rows, tile0 = sc_tiles[s] - tiles;
+    const bool fits = sc_rows[kMaxE - 1] <= a.R;  // a layout larger than the buffer runs nothing
+    if (fits && s < nseg)
+        for (int i = 0; i < tiles; ++i)
+            a.tiles[tile0 + i] = make_int4(s % a.El, row0 + i * kTokTile, min(kTokTile, rows - i * kTokTile), 0);
+    if (s < kCtrlWords) a.ctrl[s] = 0;
+    __syncthreads();
+    if (s == 0) a.ctrl[kCtrlNumTokTiles] = fits ? sc_tiles[kMaxE - 1] : 0;
+}
+
+cudaError_t launch_ep_tiles(const EpTilesArgs &a, cudaStream_t s, int *launches) {
+    ep_tiles_kernel<<<1, kMaxE, 0, s>>>(a);
+    ++*launches;
+    return cudaGetLastError();
+}
 
 cudaError_t launch_dispatch(const DispatchArgs &a, cudaStream_t s, int *launches) {
     if (a.T <= 0) return cudaSuccess;

@@ -128,8 +128,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_after_sync();
     const uint32_t tmem_base = *s.tmem_slot;
 
-    const int n_tt = min(a.ctrl[kCtrlNumTokTiles], a.max_tok_tiles);
+    const int4 *tok_tiles = a.tok_tiles + (a.tile_base_word >= 0 ? a.ctrl[a.tile_base_word] : 0);
+    const int n_tt = a.fixed_tiles > 0 ? a.fixed_tiles : min(a.ctrl[kCtrlNumTokTiles], a.max_tok_tiles);
     const int total = n_tt * a.n_ftiles;
+    // Weight-stack index of group g (shared groups may sit at another base).
+    auto wgroup = [&](int g) { return g < a.E ? g : a.w_shared_base + (g - a.E); };
     const int kblocks = a.K / kBK;
     bool ok = true;
 
@@ -170,7 +173,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 break;
             }
             const int tt = u / a.n_ftiles, j = u - tt * a.n_ftiles;
-            const int4 tile = a.tok_tiles[tt];  // {group, first row, rows, -}
+            const int4 tile = tok_tiles[tt];  // {group, first row, rows, -}
             const int g = tile.x, ntok = tile.z;
             const CUtensorMap *mt = &map_t, *mt16 = &map_t16;
             int trow = tile.y + static_cast<int>(rank) * (ntok / 2);
@@ -179,7 +182,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 mt16 = &map_s16;
                 trow -= a.group_start[g];
             }
-            const int wrow = g * a.N + j * kFeatPair + static_cast<int>(rank) * kFeatCta;
+            const int wrow = wgroup(g) * a.N + j * kFeatPair + static_cast<int>(rank) * kFeatCta;
             const uint32_t tx_bytes = 2u * kABytes + static_cast<uint32_t>(ntok) * kBK * 2u;
             const int n16 = ntok / (2 * kRowsPerLoad16);
             for (int kb = 0; kb < kblocks; ++kb, ++it) {
@@ -215,7 +218,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     ok = u == -1;
                     break;
                 }
-                const int ntok = a.tok_tiles[u / a.n_ftiles].z;
+                const int ntok = tok_tiles[u / a.n_ftiles].z;
                 const uint32_t idesc = idesc_bf16_f32(kFeatPair, ntok);
                 const uint32_t acc = tcount & 1u, use = tcount >> 1;
                 if (!mbar_wait(&s.tempty[acc], (use & 1u) ^ 1u, a.status)) break;
@@ -252,7 +255,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             u = __shfl_sync(0xffffffffu, u, 0);
             if (u < 0) break;
             const int tt = u / a.n_ftiles, j = u - tt * a.n_ftiles;
-            const int4 tile = a.tok_tiles[tt];
+            const int4 tile = tok_tiles[tt];
             const int g = tile.x, row0 = tile.y, ntok = tile.z;
             const int fcol = j * kFeatPair + static_cast<int>(rank) * kFeatCta + q * 32;
             const uint32_t acc = tcount & 1u, use = tcount >> 1;
@@ -261,7 +264,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (!__shfl_sync(0xffffffffu, got, 0)) break;
             tc_fence_after_sync();
             if (fcol < a.N) {  // the last feature tile of a ragged N has an idle half
-                const float b = a.bias ? __ldg(a.bias + (int64_t)g * a.N + fcol + lane) : 0.f;
+                const float b = a.bias ? __ldg(a.bias + (int64_t)wgroup(g) * a.N + fcol + lane) : 0.f;
                 const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * kAccCols;
 #pragma unroll 1
                 for (int c = 0; c < ntok; c += kBoxTok) {

@@ -8,6 +8,7 @@
 #include <cstdio>
 #include <cstring>
 #include <string>
+#include <vector>
 
 #include "moe.h"
 #include "moe_common.cuh"
@@ -103,7 +104,8 @@ int report_error(int code, const char *msg) { return fail(code, "%s", msg); }
 struct moe_layer {
     moe_config_t cfg;
     moe_weights_t w;
-    int G = 0;
+    int G = 0;         // groups in the weight stacks: routed experts held here + shared
+    int E_weights = 0; // routed experts held in the weight stacks (E, or E / ep_size)
     bool tc = false;
     int num_sms = 148;
     int num_pairs = 0;  // co-resident 2-CTA clusters of the expert GEMM
@@ -113,6 +115,8 @@ struct moe_layer {
     Plan plan;
     char *ws = nullptr;
     int fwd_launches = 0, stats_launches = 0;
+    const void *fx = nullptr;  // the forward's tokens and gates, for the later phases
+    float *fgates = nullptr;
     bool timing = false;
     cudaEvent_t ev[MOE_TIMING_EVENTS];
 };
@@ -214,6 +218,18 @@ int validate_config(const moe_config_t *c, const moe_weights_t *w) {
         return fail(MOE_ERR_INVALID_ARG, "unknown credit_norm %d", c->credit_norm);
     if (c->capacity_priority != MOE_PRIORITY_TOKEN && c->capacity_priority != MOE_PRIORITY_RANK)
         return fail(MOE_ERR_INVALID_ARG, "unknown capacity_priority %d", c->capacity_priority);
+    if (c->ep_size < 1 || c->ep_rank < 0 || c->ep_rank >= c->ep_size)
+        return fail(MOE_ERR_INVALID_ARG, "ep_size must be >= 1 and 0 <= ep_rank < ep_size (got %d, %d)", c->ep_size,
+                    c->ep_rank);
+    if (c->ep_size > 1) {
+        if (c->num_experts % c->ep_size)
+            return fail(MOE_ERR_INVALID_ARG, "num_experts (%d) must be a multiple of ep_size (%d)", c->num_experts,
+                        c->ep_size);
+        if (c->dtype != MOE_DTYPE_BF16)
+            return fail(MOE_ERR_UNSUPPORTED, "expert parallelism runs bf16 layers (tensor-core expert GEMMs)");
+        if (c->credit_norm == MOE_CREDIT_HIDDEN)
+            return fail(MOE_ERR_UNSUPPORTED, "the hidden-activation credit needs the hidden rows on the token's rank");
+    }
     if (c->use_mlp_gater != 0 && c->use_mlp_gater != 1)
         return fail(MOE_ERR_INVALID_ARG, "use_mlp_gater must be 0 or 1");
     if (c->use_mlp_gater) {
@@ -275,6 +291,8 @@ moe_config_t moe_config_default(void) {
     c.capacity_priority = MOE_PRIORITY_TOKEN;
     c.use_mlp_gater = 0;
     c.gater_hidden_dim = 128;
+    c.ep_size = 1;
+    c.ep_rank = 0;
     return c;
 }
 
@@ -296,7 +314,8 @@ int moe_layer_create(const moe_config_t *cfg, const moe_weights_t *w, moe_layer_
     moe_layer *L = new moe_layer();
     L->cfg = *cfg;
     L->w = *w;
-    L->G = cfg->num_experts + cfg->num_shared;
+    L->E_weights = cfg->num_experts / (cfg->ep_size > 1 ? cfg->ep_size : 1);
+    L->G = L->E_weights + cfg->num_shared;
     L->num_sms = sms > 0 ? sms : 148;
     L->tc = cfg->dtype == MOE_DTYPE_BF16;
     if (L->tc) {
@@ -325,15 +344,19 @@ int64_t moe_capacity(const moe_layer_t *layer, int32_t T) {
     return capacity_of(layer->cfg, T);
 }
 
-int moe_forward(moe_layer_t *L, const void *x, int32_t T, const float *logit_noise, void *workspace, size_t ws_bytes,
-                void *y, const moe_routing_t *routing, void *stream_v) {
-    g_last_error.clear();
-    if (!L) return fail(MOE_ERR_INVALID_ARG, "layer is NULL");
+}  // extern "C"
+
+namespace {
+
+// Router, dispatch and row scatter of one forward (everything before the
+// expert GEMMs); records what the later phases need in the layer.
+int fwd_route(moe_layer_t *L, const void *x, int32_t T, const float *logit_noise, void *workspace, size_t ws_bytes,
+              const moe_routing_t *routing, cudaStream_t s) {
     const moe_config_t &c = L->cfg;
     if (T < 0) return fail(MOE_ERR_INVALID_ARG, "T must be >= 0 (got %d)", T);
     if (c.max_tokens > 0 && T > c.max_tokens)
         return fail(MOE_ERR_INVALID_ARG, "T=%d exceeds max_tokens=%d", T, c.max_tokens);
-    if (T > 0 && (!x || !y)) return fail(MOE_ERR_INVALID_ARG, "x and y are required when T > 0");
+    if (T > 0 && !x) return fail(MOE_ERR_INVALID_ARG, "x is required when T > 0");
     if (T > 0 && c.top_k_method == MOE_TOPK_NOISY && !logit_noise)
         return fail(MOE_ERR_INVALID_ARG, "NOISY top-k needs logit_noise [T][E]");
     const Plan p = make_plan(*L, T);
@@ -342,10 +365,8 @@ int moe_forward(moe_layer_t *L, const void *x, int32_t T, const float *logit_noi
         return fail(MOE_ERR_WORKSPACE, "workspace must be 256-byte aligned");
     if (ws_bytes < p.total)
         return fail(MOE_ERR_WORKSPACE, "workspace too small: %zu bytes given, %zu needed for T=%d", ws_bytes, p.total, T);
-    if ((reinterpret_cast<uintptr_t>(x) | reinterpret_cast<uintptr_t>(y)) % 16)
-        return fail(MOE_ERR_INVALID_ARG, "x and y must be 16-byte aligned");
+    if (reinterpret_cast<uintptr_t>(x) % 16) return fail(MOE_ERR_INVALID_ARG, "x must be 16-byte aligned");
 
-    cudaStream_t s = as_stream(stream_v);
     char *ws = static_cast<char *>(workspace);
     L->has_forward = true;
     L->plan = p;
@@ -363,6 +384,8 @@ int moe_forward(moe_layer_t *L, const void *x, int32_t T, const float *logit_noi
     int32_t *idx = rt && rt->topk_idx ? rt->topk_idx : reinterpret_cast<int32_t *>(ws + p.o_idx);
     float *gates = rt && rt->gates ? rt->gates : reinterpret_cast<float *>(ws + p.o_gates);
     int32_t *slot = rt && rt->slot ? rt->slot : reinterpret_cast<int32_t *>(ws + p.o_slot);
+    L->fx = x;
+    L->fgates = gates;
     int *nl = &L->fwd_launches;
     uint32_t *status = reinterpret_cast<uint32_t *>(ctrl + kCtrlStatus);
 
@@ -496,6 +519,27 @@ int moe_forward(moe_layer_t *L, const void *x, int32_t T, const float *logit_noi
         sa.row_bytes = c.input_dim * 2;
         MOE_LAUNCH(launch_scatter(sa, L->num_sms, s, nl));
     }
+    return MOE_OK;
+}
+
+// Expert GEMMs over the forward's row space: every group, or (EP) only the
+// shared experts' groups.
+int fwd_expert_gemms(moe_layer_t *L, cudaStream_t s, bool shared_only) {
+    const moe_config_t &c = L->cfg;
+    const Plan &p = L->plan;
+    char *ws = L->ws;
+    const void *x = L->fx;
+    const int T = p.T, E = c.num_experts, k = c.num_active, S = c.num_shared;
+    if (T == 0 || (shared_only && S == 0)) return MOE_OK;
+    int *nl = &L->fwd_launches;
+    int32_t *ctrl = reinterpret_cast<int32_t *>(ws + p.o_ctrl);
+    uint32_t *status = reinterpret_cast<uint32_t *>(ctrl + kCtrlStatus);
+    DispatchArgs da;
+    da.tok_tiles = reinterpret_cast<int4 *>(ws + p.o_toktiles);
+    da.group_start = reinterpret_cast<int32_t *>(ws + p.o_gstart);
+    da.group_rows = reinterpret_cast<int32_t *>(ws + p.o_grows);
+    da.block_group = reinterpret_cast<int32_t *>(ws + p.o_bgroup);
+    da.row_assign = reinterpret_cast<int32_t *>(ws + p.o_rowassign);
 
     if (L->tc) {
         PairGemmArgs g1;
@@ -507,6 +551,11 @@ int moe_forward(moe_layer_t *L, const void *x, int32_t T, const float *logit_noi
         g1.K = c.input_dim;
         g1.n_ftiles = gemm_pair_ftiles(c.expert_dim);
         g1.E = E;
+        g1.w_shared_base = L->E_weights;
+        if (shared_only) {  // the shared experts' tiles follow the routed ones
+            g1.tile_base_word = kCtrlRoutedTiles;
+            g1.fixed_tiles = S * ((p.T_pad + kTokTile - 1) / kTokTile);
+        }
         g1.use_s = 1;
         g1.bias = L->w.b1;
         g1.act = c.activation;
@@ -567,6 +616,23 @@ int moe_forward(moe_layer_t *L, const void *x, int32_t T, const float *logit_noi
         MOE_MARK(L, 4, s);
     }
 
+    return MOE_OK;
+}
+
+// Credit norms (hidden reading) and the combine of the forward's outputs.
+int fwd_combine(moe_layer_t *L, void *y, cudaStream_t s) {
+    const moe_config_t &c = L->cfg;
+    const Plan &p = L->plan;
+    char *ws = L->ws;
+    const int T = p.T, E = c.num_experts, k = c.num_active, S = c.num_shared;
+    if (T == 0) return MOE_OK;
+    int *nl = &L->fwd_launches;
+    int32_t *ctrl = reinterpret_cast<int32_t *>(ws + p.o_ctrl);
+    DispatchArgs da;
+    da.row_of = reinterpret_cast<int32_t *>(ws + p.o_rowof);
+    da.row_assign = reinterpret_cast<int32_t *>(ws + p.o_rowassign);
+    da.group_start = reinterpret_cast<int32_t *>(ws + p.o_gstart);
+    float *gates = L->fgates;
     float *row_norm2 = nullptr;
     if (c.credit_norm == MOE_CREDIT_HIDDEN) {
         RowNormArgs rn;
@@ -597,6 +663,162 @@ int moe_forward(moe_layer_t *L, const void *x, int32_t T, const float *logit_noi
     MOE_LAUNCH(launch_combine(ca, s, nl));
     MOE_MARK(L, 5, s);
     return MOE_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int moe_forward(moe_layer_t *L, const void *x, int32_t T, const float *logit_noise, void *workspace, size_t ws_bytes,
+                void *y, const moe_routing_t *routing, void *stream_v) {
+    g_last_error.clear();
+    if (!L) return fail(MOE_ERR_INVALID_ARG, "layer is NULL");
+    if (L->cfg.ep_size > 1)
+        return fail(MOE_ERR_STATE, "an expert-parallel layer runs moe_ep_dispatch / moe_ep_experts / moe_ep_combine");
+    if (T > 0 && !y) return fail(MOE_ERR_INVALID_ARG, "y is required when T > 0");
+    if (reinterpret_cast<uintptr_t>(y) % 16) return fail(MOE_ERR_INVALID_ARG, "y must be 16-byte aligned");
+    cudaStream_t s = as_stream(stream_v);
+    int rc = fwd_route(L, x, T, logit_noise, workspace, ws_bytes, routing, s);
+    if (rc != MOE_OK || T == 0) return rc;
+    rc = fwd_expert_gemms(L, s, false);
+    if (rc != MOE_OK) return rc;
+    return fwd_combine(L, y, s);
+}
+
+// ------------------------------------------------------------ expert parallelism
+
+int moe_ep_dispatch(moe_layer_t *L, const void *x, int32_t T, const float *logit_noise, void *workspace,
+                    size_t ws_bytes, const moe_routing_t *routing, void *stream_v) {
+    g_last_error.clear();
+    if (!L) return fail(MOE_ERR_INVALID_ARG, "layer is NULL");
+    if (L->cfg.ep_size < 2) return fail(MOE_ERR_STATE, "moe_ep_* calls are for layers with ep_size > 1");
+    return fwd_route(L, x, T, logit_noise, workspace, ws_bytes, routing, as_stream(stream_v));
+}
+
+int moe_ep_layout(moe_layer_t *L, int32_t *expert_rows, void **rows_in, void **rows_out, void *stream_v) {
+    g_last_error.clear();
+    if (!L) return fail(MOE_ERR_INVALID_ARG, "layer is NULL");
+    if (!expert_rows) return fail(MOE_ERR_INVALID_ARG, "expert_rows is NULL");
+    if (!L->has_forward) return fail(MOE_ERR_STATE, "moe_ep_layout before moe_ep_dispatch");
+    const int E = L->cfg.num_experts;
+    const Plan &p = L->plan;
+    if (rows_in) *rows_in = L->ws + p.o_xp;
+    if (rows_out) *rows_out = L->ws + p.o_o;
+    if (p.T == 0) {
+        std::memset(expert_rows, 0, sizeof(int32_t) * E);
+        return MOE_OK;
+    }
+    std::vector<int32_t> gs(E + 1);
+    cudaStream_t s = as_stream(stream_v);
+    MOE_LAUNCH(cudaMemcpyAsync(gs.data(), L->ws + p.o_gstart, sizeof(int32_t) * (E + 1), cudaMemcpyDeviceToHost, s));
+    MOE_LAUNCH(cudaStreamSynchronize(s));
+    for (int e = 0; e < E; ++e) expert_rows[e] = gs[e + 1] - gs[e];
+    return MOE_OK;
+}
+
+namespace {
+struct EpPlan {
+    size_t o_ctrl, o_tiles, o_h, total;
+    int max_tiles;
+};
+EpPlan ep_plan(const moe_layer &L, int R) {
+    EpPlan q;
+    const int E = L.cfg.num_experts;
+    q.max_tiles = std::max(1, std::min(R / kTokTile + E, R / kRowBlock));
+    size_t off = 0;
+    auto take = [&](size_t bytes) {
+        const size_t o = off;
+        off = align_up(off + bytes, 256);
+        return o;
+    };
+    q.o_ctrl = take(kCtrlWords * 4);
+    q.o_tiles = take((size_t)q.max_tiles * 16);
+    q.o_h = take((size_t)R * L.cfg.expert_dim * 2);
+    q.total = off;
+    return q;
+}
+}  // namespace
+
+size_t moe_ep_experts_workspace_bytes(const moe_layer_t *L, int32_t R) {
+    if (!L || R < 0) return 0;
+    return ep_plan(*L, R).total;
+}
+
+int moe_ep_experts(moe_layer_t *L, const void *recv_x, const int32_t *recv_rows, int32_t R, void *recv_out,
+                   void *workspace, size_t ws_bytes, void *stream_v) {
+    g_last_error.clear();
+    if (!L) return fail(MOE_ERR_INVALID_ARG, "layer is NULL");
+    const moe_config_t &c = L->cfg;
+    if (c.ep_size < 2) return fail(MOE_ERR_STATE, "moe_ep_* calls are for layers with ep_size > 1");
+    if (R < 0) return fail(MOE_ERR_INVALID_ARG, "R must be >= 0");
+    if (R % kRowBlock) return fail(MOE_ERR_INVALID_ARG, "R must be a multiple of %d (got %d)", kRowBlock, R);
+    if (R == 0) return MOE_OK;
+    if (!recv_x || !recv_rows || !recv_out || !workspace)
+        return fail(MOE_ERR_INVALID_ARG, "recv_x, recv_rows, recv_out and workspace are required");
+    const EpPlan q = ep_plan(*L, R);
+    if (reinterpret_cast<uintptr_t>(workspace) % 256) return fail(MOE_ERR_WORKSPACE, "workspace must be 256-byte aligned");
+    if (ws_bytes < q.total) return fail(MOE_ERR_WORKSPACE, "workspace too small: %zu given, %zu needed", ws_bytes, q.total);
+    if ((reinterpret_cast<uintptr_t>(recv_x) | reinterpret_cast<uintptr_t>(recv_out)) % 16)
+        return fail(MOE_ERR_INVALID_ARG, "recv_x and recv_out must be 16-byte aligned");
+    cudaStream_t s = as_stream(stream_v);
+    char *ws = static_cast<char *>(workspace);
+    int32_t *ctrl = reinterpret_cast<int32_t *>(ws + q.o_ctrl);
+    int4 *tiles = reinterpret_cast<int4 *>(ws + q.o_tiles);
+    int launches = 0;
+    EpTilesArgs ta;
+    ta.recv_rows = recv_rows;
+    ta.G = c.ep_size;
+    ta.El = L->E_weights;
+    ta.R = R;
+    ta.tiles = tiles;
+    ta.ctrl = ctrl;
+    MOE_LAUNCH(launch_ep_tiles(ta, s, &launches));
+
+    PairGemmArgs g1;
+    g1.tok_tiles = tiles;
+    g1.group_start = nullptr;
+    g1.ctrl = ctrl;
+    g1.max_tok_tiles = q.max_tiles;
+    g1.N = c.expert_dim;
+    g1.K = c.input_dim;
+    g1.n_ftiles = gemm_pair_ftiles(c.expert_dim);
+    g1.E = L->E_weights;  // every received group is a routed expert held here
+    g1.w_shared_base = L->E_weights;
+    g1.use_s = 0;
+    g1.bias = L->w.b1;
+    g1.act = c.activation;
+    g1.status = reinterpret_cast<uint32_t *>(ctrl + kCtrlStatus);
+    g1.work_counter = ctrl + kCtrlWork1;
+    g1.num_pairs = L->num_pairs;
+    PairGemmArgs g2 = g1;
+    g2.N = c.output_dim;
+    g2.K = c.expert_dim;
+    g2.n_ftiles = gemm_pair_ftiles(c.output_dim);
+    g2.bias = L->w.b2;
+    g2.act = -1;
+    g2.work_counter = ctrl + kCtrlWork2;
+    CUtensorMap m_x, m_x16, m_h, m_h16, m_hs, m_os;
+    if (!encode_bf16_2d(&m_x, recv_x, c.input_dim, R, 128) || !encode_bf16_2d(&m_x16, recv_x, c.input_dim, R, 16) ||
+        !encode_bf16_2d(&m_h, ws + q.o_h, c.expert_dim, R, 128) ||
+        !encode_bf16_2d(&m_h16, ws + q.o_h, c.expert_dim, R, 16) ||
+        !encode_bf16_store(&m_hs, ws + q.o_h, c.expert_dim, R) || !encode_bf16_store(&m_os, recv_out, c.output_dim, R))
+        return fail(MOE_ERR_CUDA, "cuTensorMapEncodeTiled failed for the received rows");
+    MOE_LAUNCH(launch_gemm_pair(L->map_w1, m_x, m_x16, m_x, m_x16, m_hs, g1, s, &launches));
+    MOE_LAUNCH(launch_gemm_pair(L->map_w2, m_h, m_h16, m_h, m_h16, m_os, g2, s, &launches));
+    return MOE_OK;
+}
+
+int moe_ep_combine(moe_layer_t *L, void *y, void *stream_v) {
+    g_last_error.clear();
+    if (!L) return fail(MOE_ERR_INVALID_ARG, "layer is NULL");
+    if (L->cfg.ep_size < 2) return fail(MOE_ERR_STATE, "moe_ep_* calls are for layers with ep_size > 1");
+    if (!L->has_forward) return fail(MOE_ERR_STATE, "moe_ep_combine before moe_ep_dispatch");
+    if (L->plan.T > 0 && !y) return fail(MOE_ERR_INVALID_ARG, "y is required when T > 0");
+    if (reinterpret_cast<uintptr_t>(y) % 16) return fail(MOE_ERR_INVALID_ARG, "y must be 16-byte aligned");
+    cudaStream_t s = as_stream(stream_v);
+    int rc = fwd_expert_gemms(L, s, true);
+    if (rc != MOE_OK) return rc;
+    return fwd_combine(L, y, s);
 }
 
 }  // extern "C"

@@ -88,6 +88,7 @@ enum {
     kCtrlNumTokTiles = 4,
     kCtrlWork1 = 5,  // unit counters of the two expert GEMM launches
     kCtrlWork2 = 6,
+    kCtrlRoutedTiles = 7,  // token tiles of the routed experts (the shared experts' follow)
     kCtrlWords = 8
 };
 
@@ -118,6 +119,9 @@ struct PairGemmArgs {
     int N, K;
     int n_ftiles;                // ceil(N / 256)
     int E;                       // groups >= E are shared experts
+    int w_shared_base = 0;       // weight-stack index of the first shared group (E, or the local count)
+    int tile_base_word = -1;     // ctrl word holding the index of the first tile to run, or -1 (tile 0)
+    int fixed_tiles = 0;         // > 0: run this many tiles instead of ctrl[kCtrlNumTokTiles]
     int use_s;
     const float *bias;           // [G][N] or null
     int act;                     // activation code, -1 none
@@ -191,6 +195,17 @@ struct FinalizeArgs {
     float *importance, *cv_load, *cv_importance, *l_total;
 };
 cudaError_t launch_stats_finalize(const FinalizeArgs &a, cudaStream_t s, int *launches);
+
+// Expert parallelism: the token-tile table of rows received from G source
+// ranks, laid out source-major, each source's rows grouped by local expert and
+// padded to 32 rows (the sender's row space).
+struct EpTilesArgs {
+    const int32_t *recv_rows;  // [G][E_local] padded rows
+    int G, El, R;
+    int4 *tiles;               // out: {local expert, first row, rows, 0}
+    int32_t *ctrl;             // out: kCtrlNumTokTiles (status and counters zeroed)
+};
+cudaError_t launch_ep_tiles(const EpTilesArgs &a, cudaStream_t s, int *launches);
 
 // Squared norms of the routed rows of a [rows][n] matrix (H, for the credit's
 // hidden-activation reading); padding rows are skipped.

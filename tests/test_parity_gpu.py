@@ -394,3 +394,63 @@ def test_bounded_wait_times_out_and_context_survives():
     assert moe_selftest_bounded_wait(torch.cuda.current_stream().cuda_stream) == 0
     w = WORKLOADS["default"].with_(T=300)
     full_check(w, make_inputs(w, "cpu", seed=2))
+
+
+def _emulated_all_to_all(inputs, splits):
+    """What all_to_all_single delivers to each rank q: from every rank r, in
+    rank order, the rows r sends to q (splits[r][q] rows after the earlier ones)."""
+    G = len(inputs)
+    outs = []
+    for q in range(G):
+        parts = []
+        for r in range(G):
+            off = sum(splits[r][:q])
+            parts.append(inputs[r][off:off + splits[r][q]])
+        outs.append(torch.cat(parts))
+    return outs
+
+
+def test_expert_parallel_two_ranks_emulated_on_one_gpu():
+    """Expert parallelism ("Capacity & communication": E/G experts per device,
+    all-to-all dispatch and combine) with G = 2 ranks emulated in one process:
+    each rank routes its own tokens with its own capacity, its rows go to the
+    owner of each expert, the owners run their experts, the results come back,
+    each rank adds its shared expert and combines. Each rank's y and credit
+    match the oracle on that rank's tokens with all experts."""
+    from sparse_mixture_experts_gate_b200.binding import ep_send_splits
+    from sparse_mixture_experts_gate_b200.workloads import make_tokens
+    G = 2
+    w = WORKLOADS["e64"].with_(T=500, E=16, k=4, S=1, d=256, F=384, O=320, capacity_factor=1.0)
+    inp = make_inputs(w, "cpu", seed=51, random_biases=True)
+    El = w.E // G
+    layers, batches = [], []
+    for r in range(G):
+        local = dict(inp)
+        for key in ("w1", "b1", "w2", "b2"):
+            local[key] = torch.cat([inp[key][r * El:(r + 1) * El], inp[key][w.E:]])
+        layers.append(MoELayer(w, local, ep_size=G, ep_rank=r))
+        batches.append(make_tokens(w, "cpu", seed=300 + r))
+    xs = [b["x"].cuda() for b in batches]  # x must stay valid until ep_combine (shared experts read it)
+    phase1 = [layers[r].ep_dispatch(xs[r]) for r in range(G)]
+    splits = [ep_send_splits(ph[3], G) for ph in phase1]
+    recv = _emulated_all_to_all([ph[1] for ph in phase1], splits)
+    counts = [torch.tensor([phase1[r][3][q * El:(q + 1) * El] for r in range(G)], dtype=torch.int32).cuda()
+              for q in range(G)]
+    outs = [layers[q].ep_experts(recv[q], counts[q]) for q in range(G)]
+    # Back: rank q returns to rank r the rows r sent it, in the same order.
+    back_splits = [[sum(phase1[r][3][q * El:(q + 1) * El]) for r in range(G)] for q in range(G)]
+    returned = _emulated_all_to_all(outs, back_splits)
+    for r in range(G):
+        phase1[r][2][:returned[r].shape[0]].copy_(returned[r])
+        layers[r].ep_combine(phase1[r][0])
+        layers[r].aux_stats(phase1[r][0])
+    torch.cuda.synchronize()
+    table = expert_table(w, inp)
+    for r in range(G):
+        assert layers[r].device_status() == 0
+        out = phase1[r][0]
+        g = {k: (v.float().cpu().numpy().astype(np.float64) if v.is_floating_point() else v.cpu().numpy())
+             for k, v in out.items()}
+        binp = dict(inp, x=batches[r]["x"], token_loss=None, noise=None)
+        check_same_logits_routing(w, binp, g)
+        check_end_to_end(w, binp, g, table=table)
