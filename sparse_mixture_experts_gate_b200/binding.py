@@ -504,7 +504,8 @@ class HostPipeline:
     STAT_KEYS = ("l_aux", "l_z", "n_dropped", "f", "p_mean", "expert_loss", "importance", "cv_load",
                  "cv_importance", "l_total")
 
-    def __init__(self, layer: "MoELayer", T: int, with_noise: bool = False, with_loss: bool = False):
+    def __init__(self, layer: "MoELayer", T: int, with_noise: bool = False, with_loss: bool = False,
+                 use_graphs: bool = True):
         import torch
         self.layer, self.T = layer, T
         dev = layer.device
@@ -515,13 +516,18 @@ class HostPipeline:
         self.slots = []
         for _ in range(2):
             self.slots.append(dict(
-                x=torch.empty(T, w.d, dtype=layer._dt, device=dev),
-                noise=torch.empty(T, w.E, dtype=torch.float32, device=dev) if with_noise else None,
-                loss=torch.empty(T, dtype=torch.float32, device=dev) if with_loss else None,
+                x=torch.zeros(T, w.d, dtype=layer._dt, device=dev),
+                noise=torch.zeros(T, w.E, dtype=torch.float32, device=dev) if with_noise else None,
+                loss=torch.zeros(T, dtype=torch.float32, device=dev) if with_loss else None,
                 out=layer.alloc_outputs(T),
                 uploaded=torch.cuda.Event(), computed=torch.cuda.Event(), downloaded=torch.cuda.Event(),
                 used=False))
         layer.workspace(T)
+        # Each slot's forward + statistics as one CUDA graph over its buffers.
+        self.graphs = None
+        if use_graphs:
+            self.graphs = [StepGraph(layer, sl["x"], noise=sl["noise"], token_loss=sl["loss"], out=sl["out"])
+                           for sl in self.slots]
         self.n = 0
 
     def submit(self, x_h, y_h, noise_h=None, loss_h=None, stats_h=None):
@@ -544,9 +550,12 @@ class HostPipeline:
             self.comp.wait_event(sl["uploaded"])
             if sl["used"]:
                 self.comp.wait_event(sl["downloaded"])  # the slot's previous results have left
-            s = self.comp.cuda_stream
-            self.layer.forward(sl["x"], noise=sl["noise"] if noise_h is not None else None, out=sl["out"], stream=s)
-            self.layer.aux_stats(sl["out"], token_loss=sl["loss"] if loss_h is not None else None, stream=s)
+            if self.graphs is not None:
+                self.graphs[(self.n - 1) % 2].replay()
+            else:
+                s = self.comp.cuda_stream
+                self.layer.forward(sl["x"], noise=sl["noise"], out=sl["out"], stream=s)
+                self.layer.aux_stats(sl["out"], token_loss=sl["loss"], stream=s)
             sl["computed"].record(self.comp)
         with torch.cuda.stream(self.down):
             self.down.wait_event(sl["computed"])
@@ -560,3 +569,35 @@ class HostPipeline:
         self.down.synchronize()
         self.comp.synchronize()
         self.up.synchronize()
+
+
+class StepGraph:
+    """One forward + statistics captured as a CUDA graph over fixed device
+    buffers (x, noise, token loss in; out's tensors written), so that a step
+    replays as one graph launch instead of a dozen kernel launches. Refill the
+    input tensors in place and call replay(); the layer's workspace and the
+    output tensors are the ones the graph was captured with."""
+
+    def __init__(self, layer: "MoELayer", x, noise=None, token_loss=None, out=None):
+        import torch
+        self.layer, self.x, self.noise, self.token_loss = layer, x, noise, token_loss
+        T = int(x.shape[0])
+        self.out = out if out is not None else layer.alloc_outputs(T)
+        layer.workspace(T)  # allocate before capture
+        side = torch.cuda.Stream(layer.device)
+        side.wait_stream(torch.cuda.current_stream(layer.device))
+        with torch.cuda.stream(side):  # one eager step: host-side set-up outside the capture
+            self._step()
+        torch.cuda.current_stream(layer.device).wait_stream(side)
+        torch.cuda.synchronize(layer.device)
+        self.graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(self.graph):
+            self._step()
+
+    def _step(self):
+        self.layer.forward(self.x, noise=self.noise, out=self.out)
+        self.layer.aux_stats(self.out, token_loss=self.token_loss)
+
+    def replay(self):
+        self.graph.replay()
+        return self.out

@@ -322,7 +322,7 @@ template <int ACT>
 cudaError_t launch_act(const CUtensorMap &mw, const CUtensorMap &mt, const CUtensorMap &mt16, const CUtensorMap &ms,
                        const CUtensorMap &ms16, const CUtensorMap &mo, const PairGemmArgs &a, cudaStream_t st) {
     auto kern = grouped_gemm_pair_kernel<ACT>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
+    cudaError_t e = set_smem_limit_once<grouped_gemm_pair_kernel<ACT>>(kSmem);
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(2 * a.num_pairs, 1, 1);

@@ -9,6 +9,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <atomic>
+
 namespace moe {
 
 // Rows of the expert GEMM's M tile. Every expert's row segment in the permuted
@@ -405,6 +407,22 @@ __device__ __forceinline__ void spin_ns(uint64_t ns) {
 }
 
 // ------------------------------------------------------------------ misc
+
+// Raises kernel K's dynamic shared-memory limit once per device (the first
+// launch), so that later launches, including ones captured into a CUDA graph,
+// make no attribute call.
+template <auto K>
+inline cudaError_t set_smem_limit_once(int bytes) {
+    static std::atomic<uint64_t> done{0};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    const uint64_t bit = 1ull << (dev & 63);
+    if (done.load() & bit) return cudaSuccess;
+    e = cudaFuncSetAttribute(K, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e == cudaSuccess) done.fetch_or(bit);
+    return e;
+}
 
 template <typename T>
 __device__ __forceinline__ float to_f32(T v);

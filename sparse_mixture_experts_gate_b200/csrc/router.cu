@@ -48,7 +48,9 @@ __device__ __forceinline__ void route_warp(const float (&h)[RE], int t, int lane
                 kv = __fadd_rn(h[q], a.noise[(int64_t)t * a.E + e]);
             else if (a.sel_bias)
                 kv = __fadd_rn(h[q], a.sel_bias[e]);
-            key[q] = kv;
+            // A NaN key (NaN input) selects like -inf: every pick is still a
+            // valid, distinct expert index (the lowest free one).
+            key[q] = kv != kv ? -INFINITY : kv;
             m = fmaxf(m, h[q]);
         }
     }

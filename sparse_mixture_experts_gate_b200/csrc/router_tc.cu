@@ -207,8 +207,7 @@ __global__ void __launch_bounds__(kRouterThreads, 1)
 template <int BN>
 cudaError_t launch_bn(const CUtensorMap &mx, const CUtensorMap &mw, const RouterTcArgs &a, cudaStream_t s) {
     constexpr int smem = TcLayout<BN>::SMEM;
-    cudaError_t e =
-        cudaFuncSetAttribute(router_logits_tc_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    cudaError_t e = set_smem_limit_once<router_logits_tc_kernel<BN>>(smem);
     if (e != cudaSuccess) return e;
     const int tiles = ((a.T + kBM - 1) / kBM) * (a.E_pad / BN) * a.ksplit;
     router_logits_tc_kernel<BN><<<tiles < a.num_sms ? tiles : a.num_sms, kRouterThreads, smem, s>>>(mx, mw, a);

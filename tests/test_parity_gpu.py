@@ -454,3 +454,46 @@ def test_expert_parallel_two_ranks_emulated_on_one_gpu():
         binp = dict(inp, x=batches[r]["x"], token_loss=None, noise=None)
         check_same_logits_routing(w, binp, g)
         check_end_to_end(w, binp, g, table=table)
+
+
+def test_cuda_graph_step_matches_eager():
+    """binding.StepGraph: the forward + statistics captured once and replayed
+    (inputs refilled in place) gives bit-for-bit the eager results."""
+    from sparse_mixture_experts_gate_b200.binding import StepGraph
+    from sparse_mixture_experts_gate_b200.workloads import make_tokens
+    w = WORKLOADS["e64"].with_(T=512, token_loss=True)
+    inp = make_inputs(w, "cpu", seed=61)
+    layer = MoELayer(w, inp)
+    b0, b1 = make_tokens(w, "cpu", seed=70), make_tokens(w, "cpu", seed=71)
+    x = b0["x"].cuda()
+    tl = b0["token_loss"].cuda()
+    graph = StepGraph(layer, x, token_loss=tl)
+    for b in (b1, b0, b1):
+        x.copy_(b["x"].cuda())
+        tl.copy_(b["token_loss"].cuda())
+        got = {k: v.clone() for k, v in graph.replay().items()}
+        torch.cuda.synchronize()
+        want = layer.forward(b["x"].cuda())
+        layer.aux_stats(want, token_loss=b["token_loss"].cuda())
+        torch.cuda.synchronize()
+        for k in want:
+            assert torch.equal(got[k], want[k]), f"{k} differs between graph replay and eager"
+
+
+def test_nan_tokens_route_to_valid_experts():
+    """NaN inputs are outside the contract, but they must not make the layer
+    fault or hang: a NaN token's keys select like -inf (the lowest free expert
+    indices), so routing stays valid, and tokens without NaNs keep finite outputs."""
+    w = WORKLOADS["default"].with_(T=300, E=8, k=2, capacity_factor=0.0)
+    inp = make_inputs(w, "cpu", seed=81)
+    x = inp["x"].clone()
+    bad = [3, 77, 150]
+    x[bad] = float("nan")
+    g, layer = run_gpu(w, dict(inp, x=x))
+    idx = g["topk_idx"]
+    assert ((idx >= 0) & (idx < w.E)).all()
+    assert all(len(set(r)) == w.k for r in idx.tolist())
+    for t in bad:
+        assert sorted(idx[t].tolist()) == list(range(w.k))
+    good = np.setdiff1d(np.arange(w.T), bad)
+    assert np.isfinite(g["y"][good]).all()
