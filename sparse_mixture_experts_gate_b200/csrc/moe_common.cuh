@@ -13,8 +13,8 @@
 
 namespace moe {
 
-// Rows of the expert GEMM's M tile. Every expert's row segment in the permuted
-// row space is padded to a multiple of this, so no M tile straddles two experts.
+// Rows (tokens) of the router's tensor-core M tile; also the rows of a full
+// 128-row TMA box.
 constexpr int kBM = 128;
 // K extent of one pipeline stage: 64 bf16 = 128 bytes, one 128B-swizzle row.
 constexpr int kBK = 64;

@@ -1,14 +1,12 @@
-// tc_pipeline.cuh - the persistent, warp-specialised tcgen05 pipeline shared by
-// the expert GEMM and the tensor-core router.
+// tc_pipeline.cuh - the one-CTA tcgen05 pipeline pieces of the tensor-core
+// router (router_tc.cu): shared-memory layout of the stage ring, barrier and
+// TMEM set-up and teardown, and the TMA producer role.
 //
 // One CTA per SM walks a static tile sequence (tile = blockIdx.x, += gridDim.x).
 //   warp 0      producer: per K block, waits for a free stage, posts the
 //               expected bytes and issues TMA loads (the kernel's load functor);
-//   warp 1      owns TMEM (2 x 256 fp32 columns); one lane issues
-//               tcgen05.mma (M = 128, N = BN, K = 16) per 16-wide K slice and
-//               commits stages back to the producer and accumulators to the
-//               epilogue;
-//   warps 2..5  epilogue (the kernel's functor), one TMEM lane quarter each.
+//   warp 1      owns TMEM (2 x 256 fp32 columns) and issues the MMAs;
+//   other warps the kernel's epilogue.
 // All waits are bounded (mbar_wait); on a timeout every role stops, in-flight
 // copies and MMAs are drained, TMEM is freed and the kernel returns with the
 // status word flagged.
@@ -99,8 +97,7 @@ __device__ __forceinline__ void tc_teardown(const TcShared<BN> &s, uint32_t tmem
 // bar, lane)` issues the stage's TMA loads (any lane may issue some of them);
 // `tile_begin(tile, lane)` runs once per tile before its first K block. Lane 0
 // owns the barrier protocol; the wait outcome is broadcast so the warp stays
-// convergent.
-// As tc_producer, with a per-tile K-block range [x, y) from krange(tile).
+// convergent. Tile `tile` covers K blocks [x, y) of krange(tile).
 template <int BN, class TileBegin, class LoadFn, class KRange>
 __device__ __forceinline__ void tc_producer_range(const TcShared<BN> &s, int total, uint32_t *status,
                                                   TileBegin tile_begin, LoadFn load, KRange krange) {
@@ -132,71 +129,6 @@ __device__ __forceinline__ void tc_producer_range(const TcShared<BN> &s, int tot
     if (!ok && lane == 0) {
         for (uint32_t j = (it > (uint32_t)L::NS ? it - L::NS : 0u); j < it; ++j)
             mbar_wait_drain(&s.full[j % L::NS], (j / L::NS) & 1u);
-    }
-}
-
-template <int BN, class TileBegin, class LoadFn>
-__device__ __forceinline__ void tc_producer(const TcShared<BN> &s, int total, int kblocks, uint32_t *status,
-                                            TileBegin tile_begin, LoadFn load) {
-    tc_producer_range<BN>(s, total, status, tile_begin, load, [&](int) { return make_int2(0, kblocks); });
-}
-
-// MMA role, one lane of warp 1. `ncols(tile)` is the tile's N (a multiple of
-// 16, at most BN): a narrower last tile multiplies only the first rows of the
-// staged B box.
-template <int BN, class NCols>
-__device__ __forceinline__ void tc_mma(const TcShared<BN> &s, uint32_t tmem_base, int total, int kblocks,
-                                       uint32_t *status, NCols ncols) {
-    using L = TcLayout<BN>;
-    uint32_t it = 0, tcount = 0;
-    bool ok = true;
-    for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x, ++tcount) {
-        const uint32_t idesc = idesc_bf16_f32(kBM, ncols(tile));
-        const uint32_t acc = tcount & 1u, use = tcount >> 1;
-        if (!mbar_wait(&s.tempty[acc], (use & 1u) ^ 1u, status)) break;
-        tc_fence_after_sync();
-        const uint32_t d_tmem = tmem_base + acc * kTcAccCols;
-        for (int kb = 0; kb < kblocks; ++kb, ++it) {
-            const int st = it % L::NS;
-            const uint32_t ph = (it / L::NS) & 1u;
-            if (!mbar_wait(&s.full[st], ph, status)) {
-                ok = false;
-                break;
-            }
-            tc_fence_after_sync();
-            const uint64_t ad = sw128_kmajor_desc(smem_u32(s.sA + st * L::A_BYTES));
-            const uint64_t bd = sw128_kmajor_desc(smem_u32(s.sB + st * L::B_BYTES));
-#pragma unroll
-            for (int kk = 0; kk < kBK / 16; ++kk)
-                tc_mma_bf16(d_tmem, ad + 2u * kk, bd + 2u * kk, idesc, (kb | kk) != 0 ? 1u : 0u);
-            tc_commit(&s.empty[st]);
-        }
-        if (ok) tc_commit(&s.tfull[acc]);
-    }
-    // All MMAs this thread issued are complete once mma_done flips.
-    tc_commit(s.mma_done);
-    mbar_wait_drain(s.mma_done, 0u);
-}
-
-// Epilogue role, warps 2..5. `epi(tile, taddr, q, lane)` reads the accumulator
-// at `taddr` (lane quarter q already folded in: taddr addresses lane 32q).
-template <int BN, class EpiFn>
-__device__ __forceinline__ void tc_epilogue(const TcShared<BN> &s, uint32_t tmem_base, int total, uint32_t *status,
-                                            EpiFn epi) {
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int q = warp & 3;  // TMEM lane quarter this warp may access
-    uint32_t tcount = 0;
-    for (int tile = blockIdx.x; tile < total; tile += gridDim.x, ++tcount) {
-        const uint32_t acc = tcount & 1u, use = tcount >> 1;
-        // tcgen05.ld is warp-collective: one lane waits, the outcome is broadcast.
-        int got = 1;
-        if (lane == 0) got = mbar_wait_idle(&s.tfull[acc], use & 1u, status) ? 1 : 0;
-        if (!__shfl_sync(0xffffffffu, got, 0)) break;
-        tc_fence_after_sync();
-        const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * kTcAccCols;
-        epi(tile, taddr, q, lane);
-        tc_fence_before_sync();
-        mbar_arrive(&s.tempty[acc]);
     }
 }
 
