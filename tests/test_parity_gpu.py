@@ -497,3 +497,13 @@ def test_nan_tokens_route_to_valid_experts():
         assert sorted(idx[t].tolist()) == list(range(w.k))
     good = np.setdiff1d(np.arange(w.T), bad)
     assert np.isfinite(g["y"][good]).all()
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "fp32"])
+def test_many_active_experts_k16(dtype):
+    """k = 16 of E = 40 (the largest k the layer takes): the combine's second
+    batch of routed terms, top-k over two expert lanes per warp lane group."""
+    w = WORKLOADS["default"].with_(T=200, E=40, k=16, S=1, capacity_factor=1.0, dtype=dtype,
+                                   d=128 if dtype == "bf16" else 32, F=128 if dtype == "bf16" else 32,
+                                   O=128 if dtype == "bf16" else 32, token_loss=True)
+    full_check(w, make_inputs(w, "cpu", seed=91, random_biases=True))
