@@ -224,10 +224,19 @@ int router_tc_epad(int E) {
 
 int router_tc_bn(int E) { return router_tc_epad(E) < 128 ? router_tc_epad(E) : 128; }
 
+// K splits. With fewer tiles than half the SMs, enough splits to fill them
+// (at least 8 drain groups per split). Otherwise 1 or 2, whichever needs fewer
+// waves of tiles per unit of work (ceil(tiles ks / SMs) / ks): two splits turn
+// 3.46 waves (E=256, T=32768: 512 tiles on 148 SMs) into 7 half-length ones,
+// for one extra [T][E] fp32 partial written and read.
 int router_tc_ksplit(int T, int E, int d, int num_sms) {
     const int tiles = ((T + kBM - 1) / kBM) * (router_tc_epad(E) / router_tc_bn(E));
     const int groups = (3 * (d / kBK) + kDrain - 1) / kDrain;
-    if (tiles <= 0 || 2 * tiles > num_sms) return 1;
+    if (tiles <= 0 || num_sms <= 0) return 1;
+    if (2 * tiles > num_sms) {
+        const int w1 = (tiles + num_sms - 1) / num_sms, w2 = (2 * tiles + num_sms - 1) / num_sms;
+        return (w2 < 2 * w1 && groups >= 16) ? 2 : 1;
+    }
     int ks = num_sms / tiles;
     if (ks > groups / 8) ks = groups / 8;  // keep at least 8 drain groups per split
     return ks < 1 ? 1 : ks;
