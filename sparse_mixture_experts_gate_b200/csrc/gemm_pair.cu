@@ -142,15 +142,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     // unequal the units' lengths. The leader's producer takes each unit and
     // posts it to a ring in both CTAs; every consumer reads entry i for its
     // i-th unit and releases it on the leader's ring_empty. -1 ends the work.
-    // The leader's producer takes unit i+1 from the counter when it starts
-    // unit i, so the atomic's round trip overlaps unit i's loads.
-    auto fetch_unit = [&]() -> int {
-        const int u = atomicAdd(a.work_counter, 1);
-        return u < total ? u : -1;
-    };
-    auto post_unit = [&](uint32_t i, int u) -> int {  // leader's producer, lane 0
+    auto post_unit = [&](uint32_t i) -> int {  // leader's producer, lane 0
         const uint32_t slot = i % kRing, ph = (i / kRing) & 1u;
         if (!mbar_wait_cluster(&s.ring_empty[slot], ph ^ 1u, a.status)) return -2;
+        int u = atomicAdd(a.work_counter, 1);
+        if (u >= total) u = -1;
         s.ring[slot] = u;
         st_shared_cluster_u32(mapa_shared(smem_u32(&s.ring[slot]), 1), static_cast<uint32_t>(u));
         mbar_arrive(&s.ring_full[slot]);
@@ -168,17 +164,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (warp == 0) {
         // ------------------------------------------------------------ producer
         uint32_t it = 0;
-        int u_next = (leader && lane == 0) ? fetch_unit() : 0;
         for (uint32_t i = 0; ok; ++i) {
             int u = 0;
-            if (lane == 0) {
-                if (leader) {
-                    u = post_unit(i, u_next);
-                    if (u >= 0) u_next = fetch_unit();  // consumed when unit i's loads are issued
-                } else {
-                    u = take_unit(i);
-                }
-            }
+            if (lane == 0) u = leader ? post_unit(i) : take_unit(i);
             u = __shfl_sync(0xffffffffu, u, 0);
             if (u < 0) {
                 ok = u == -1;
