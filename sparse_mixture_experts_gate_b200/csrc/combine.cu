@@ -11,17 +11,19 @@
 //   y[t] = sum_{s < S} O[shared row of t] + sum_{r < k, kept} g[t][r] O[row(t, r)]
 //
 // in fp32, in exactly that order (shared experts first, then r ascending), so
-// the result does not depend on scheduling. One warp per token; 16-byte vector
-// loads of the expert-output rows; dropped assignments contribute nothing. The
-// squared norms are summed from the same loads (per lane in column order, then
-// a fixed shuffle tree).
+// the result does not depend on scheduling. One warp per token, or for short
+// batches a block of eight warps per token, each taking every eighth 256-column
+// stretch; 16-byte vector loads of the expert-output rows; dropped assignments
+// contribute nothing. The squared norms are summed from the same loads (per
+// lane in column order, then a fixed shuffle tree, then the warps of a block in
+// order).
 #include "moe_common.cuh"
 #include "moe_kernels.cuh"
 
 namespace moe {
 namespace {
 
-constexpr int kWarps = 8;  // tokens per block, one warp each
+constexpr int kWarps = 8;  // warps per block
 constexpr int kMaxS = 4;
 constexpr int kBatch = 8;  // routed-term loads issued together
 
@@ -68,13 +70,16 @@ __device__ __forceinline__ uint4 load_raw(const T *p) {
 }
 
 // NB: batches of eight routed terms the kernel is built for (k <= 8 NB).
-template <typename T, int NB>
+// SL: warps per token, 1 or kWarps (then a block holds one token).
+template <typename T, int NB, int SL>
 __global__ void __launch_bounds__(kWarps * 32, 2) combine_kernel(CombineArgs a) {
+    static_assert(SL == 1 || SL == kWarps, "one token per warp or per block");
     constexpr int V = Vec<T>::N;
     constexpr int kMaxK = NB * kBatch;
-    const int lane = threadIdx.x & 31;
-    const int t = blockIdx.x * kWarps + (threadIdx.x >> 5);
-    if (t >= a.T) return;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int t = SL == 1 ? blockIdx.x * kWarps + warp : blockIdx.x;
+    const int slice = SL == 1 ? 0 : warp;
+    if (t >= a.T) return;  // uniform over the block when SL > 1
     const int nsh = a.S, k = a.k;
     int my_row = -1;
     float my_g = 0.f;
@@ -97,7 +102,7 @@ __global__ void __launch_bounds__(kWarps * 32, 2) combine_kernel(CombineArgs a) 
     float ss[kMaxK];
 #pragma unroll
     for (int r = 0; r < kMaxK; ++r) ss[r] = 0.f;
-    for (int c = lane * V; c < a.O; c += 32 * V) {
+    for (int c = (slice * 32 + lane) * V; c < a.O; c += SL * 32 * V) {
         // Every term's vector (shared terms and the first eight routed terms)
         // is requested before any is used, so a lane has them all in flight.
         uint4 us[kMaxS], ur[kBatch];
@@ -142,7 +147,8 @@ __global__ void __launch_bounds__(kWarps * 32, 2) combine_kernel(CombineArgs a) 
         Vec<T>::store(y + c, acc);
     }
     // Credit of each routed assignment: gate times the norm of the expert
-    // output row as stored (fixed shuffle tree).
+    // output row as stored (fixed shuffle tree, then the slices in order).
+    __shared__ float part[SL > 1 ? SL : 1][kMaxK];
     float credit = 0.f;
 #pragma unroll
     for (int r = 0; r < kMaxK; ++r) {
@@ -150,27 +156,50 @@ __global__ void __launch_bounds__(kWarps * 32, 2) combine_kernel(CombineArgs a) 
         float v = ss[r];
 #pragma unroll
         for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
-        if (lane == r && rrow[r] >= 0) credit = rg[r] * sqrtf(a.row_norm2 ? a.row_norm2[rrow[r]] : v);
+        if (SL > 1) {
+            if (lane == 0) part[slice][r] = v;
+        } else if (lane == r && rrow[r] >= 0) {
+            credit = rg[r] * sqrtf(a.row_norm2 ? a.row_norm2[rrow[r]] : v);
+        }
+    }
+    if (SL > 1) {
+        __syncthreads();
+        if (slice != 0) return;
+        if (lane < k && my_row >= 0) {
+            float v = 0.f;
+#pragma unroll
+            for (int w = 0; w < SL; ++w) v += part[w][lane];
+            credit = my_g * sqrtf(a.row_norm2 ? a.row_norm2[my_row] : v);
+        }
     }
     if (lane < k) a.credit[(int64_t)t * k + lane] = credit;
 }
 
+template <typename T, int NB>
+void launch_t(const CombineArgs &a, int num_sms, cudaStream_t s) {
+    // A block per token while one warp per token would leave fewer than eight
+    // warps per SM.
+    if (a.T < kWarps * num_sms)
+        combine_kernel<T, NB, kWarps><<<a.T, kWarps * 32, 0, s>>>(a);
+    else
+        combine_kernel<T, NB, 1><<<(a.T + kWarps - 1) / kWarps, kWarps * 32, 0, s>>>(a);
+}
+
 }  // namespace
 
-cudaError_t launch_combine(const CombineArgs &a, cudaStream_t s, int *launches) {
+cudaError_t launch_combine(const CombineArgs &a, int num_sms, cudaStream_t s, int *launches) {
     if (a.T <= 0) return cudaSuccess;
-    const int blocks = (a.T + kWarps - 1) / kWarps;
     if (a.k > 2 * kBatch) return cudaErrorInvalidValue;
     if (a.bf16) {
         if (a.k <= kBatch)
-            combine_kernel<__nv_bfloat16, 1><<<blocks, kWarps * 32, 0, s>>>(a);
+            launch_t<__nv_bfloat16, 1>(a, num_sms, s);
         else
-            combine_kernel<__nv_bfloat16, 2><<<blocks, kWarps * 32, 0, s>>>(a);
+            launch_t<__nv_bfloat16, 2>(a, num_sms, s);
     } else {
         if (a.k <= kBatch)
-            combine_kernel<float, 1><<<blocks, kWarps * 32, 0, s>>>(a);
+            launch_t<float, 1>(a, num_sms, s);
         else
-            combine_kernel<float, 2><<<blocks, kWarps * 32, 0, s>>>(a);
+            launch_t<float, 2>(a, num_sms, s);
     }
     ++*launches;
     return cudaGetLastError();

@@ -180,27 +180,40 @@ __global__ void __launch_bounds__(kChunk) dispatch_assign_kernel(DispatchArgs a)
     }
 }
 
-// One warp per token: the token's row of x is read once and written to the
-// rows of every expert that kept it (16-byte vectors). Padding rows of the row
-// space are left as they are: the rows computed from them are never read.
+// Work item = (token, chunk of kScatterVec x 32 16-byte vectors of its row);
+// one warp per item, so a short batch still spreads over every SM. The warp
+// loads the chunk of x once (all of a lane's vectors in flight together) and
+// writes it to the rows of every expert that kept the token. Padding rows of
+// the row space are left as they are: the rows computed from them are never
+// read.
+constexpr int kScatterVec = 4;
+
 __global__ void __launch_bounds__(256) scatter_rows_kernel(ScatterArgs a) {
     const int lane = threadIdx.x & 31;
     const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
     const int nwarps = (gridDim.x * blockDim.x) >> 5;
     const int nvec = a.row_bytes / 16;
-    for (int t = warp; t < a.T; t += nwarps) {
-        int rows[16];
-        int nk = 0;
-        for (int r = 0; r < a.k; ++r) {
-            const int row = a.row_of[(int64_t)t * a.k + r];
-            if (row >= 0) rows[nk++] = row;
-        }
-        if (nk == 0) continue;
+    const int nchunk = (nvec + 32 * kScatterVec - 1) / (32 * kScatterVec);
+    const int64_t items = (int64_t)a.T * nchunk;
+    for (int64_t it = warp; it < items; it += nwarps) {
+        const int t = static_cast<int>(it / nchunk), j = static_cast<int>(it - (int64_t)t * nchunk);
+        const int my_row = lane < a.k ? a.row_of[(int64_t)t * a.k + lane] : -1;  // k <= 16
+        uint32_t live = __ballot_sync(0xffffffffu, my_row >= 0);
+        if (live == 0) continue;
         const uint4 *src = reinterpret_cast<const uint4 *>(static_cast<const char *>(a.x) + (int64_t)t * a.row_bytes);
-        for (int v = lane; v < nvec; v += 32) {
-            const uint4 val = __ldg(src + v);
-            for (int i = 0; i < nk; ++i)
-                reinterpret_cast<uint4 *>(static_cast<char *>(a.xp) + (int64_t)rows[i] * a.row_bytes)[v] = val;
+        const int v0 = j * 32 * kScatterVec + lane;
+        uint4 val[kScatterVec];
+#pragma unroll
+        for (int u = 0; u < kScatterVec; ++u)
+            if (v0 + 32 * u < nvec) val[u] = __ldg(src + v0 + 32 * u);
+        while (live) {
+            const int i = __ffs(live) - 1;
+            live &= live - 1;
+            const int row = __shfl_sync(0xffffffffu, my_row, i);
+            uint4 *dst = reinterpret_cast<uint4 *>(static_cast<char *>(a.xp) + (int64_t)row * a.row_bytes);
+#pragma unroll
+            for (int u = 0; u < kScatterVec; ++u)
+                if (v0 + 32 * u < nvec) dst[v0 + 32 * u] = val[u];
         }
     }
 }
@@ -254,8 +267,9 @@ cudaError_t launch_dispatch(const DispatchArgs &a, cudaStream_t s, int *launches
 
 cudaError_t launch_scatter(const ScatterArgs &a, int num_sms, cudaStream_t s, int *launches) {
     if (a.T <= 0) return cudaSuccess;
-    int blocks = (a.T + 7) / 8;
-    if (blocks > num_sms * 8) blocks = num_sms * 8;
+    const int64_t nchunk = (a.row_bytes / 16 + 32 * kScatterVec - 1) / (32 * kScatterVec);
+    const int64_t items = (int64_t)a.T * nchunk;
+    const int blocks = (int)std::min<int64_t>((items + 7) / 8, (int64_t)num_sms * 8);
     scatter_rows_kernel<<<blocks, 256, 0, s>>>(a);
     ++*launches;
     return cudaGetLastError();

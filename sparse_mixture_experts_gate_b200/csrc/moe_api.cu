@@ -660,7 +660,7 @@ int fwd_combine(moe_layer_t *L, void *y, cudaStream_t s) {
     ca.bf16 = c.dtype == MOE_DTYPE_BF16;
     ca.y = y;
     ca.credit = reinterpret_cast<float *>(ws + p.o_credit);
-    MOE_LAUNCH(launch_combine(ca, s, nl));
+    MOE_LAUNCH(launch_combine(ca, L->num_sms, s, nl));
     MOE_MARK(L, 5, s);
     return MOE_OK;
 }

@@ -165,7 +165,7 @@ struct CombineArgs {
     void *y;                // [T][O]
     float *credit;          // [T][k]
 };
-cudaError_t launch_combine(const CombineArgs &a, cudaStream_t s, int *launches);
+cudaError_t launch_combine(const CombineArgs &a, int num_sms, cudaStream_t s, int *launches);
 
 // Balancing and credit statistics: partial sums, then finalize.
 struct StatsArgs {
