@@ -30,12 +30,27 @@ constexpr int kThreads = 256;
 constexpr int kWarps = kThreads / 32;
 constexpr int kKC = 32;  // K chunk staged in shared memory
 
+// The selection key's addend for expert lane + 32 q of token t: the logit
+// noise, else the per-expert selection bias; returns false (no addend) for
+// plain routing. Callers load it before their own stores so that the loads
+// are in flight together.
+template <int RE>
+__device__ __forceinline__ bool key_addend(int t, int lane, const RouterArgs &a, float (&kadd)[RE]) {
+    const float *src = a.noise ? a.noise + (int64_t)t * a.E : a.sel_bias;
+#pragma unroll
+    for (int q = 0; q < RE; ++q) {
+        const int e = lane + 32 * q;
+        kadd[q] = (src && e < a.E) ? src[e] : 0.f;
+    }
+    return src != nullptr;
+}
+
 // h[q] = clean logit of expert lane + 32 q (-inf for e >= E). Writes lse[t],
 // idx[t][0..k), gates[t][0..k) and adds the token's probabilities P[t][e] to
 // pacc[q] (the caller's per-lane running sums over its tokens).
 template <int RE>
-__device__ __forceinline__ void route_warp(const float (&h)[RE], int t, int lane, const RouterArgs &a,
-                                           float (&pacc)[RE]) {
+__device__ __forceinline__ void route_warp(const float (&h)[RE], bool has_add, const float (&kadd)[RE], int t,
+                                           int lane, const RouterArgs &a, float (&pacc)[RE]) {
     float key[RE];
     float m = -INFINITY;
 #pragma unroll
@@ -44,10 +59,7 @@ __device__ __forceinline__ void route_warp(const float (&h)[RE], int t, int lane
         key[q] = -INFINITY;
         if (e < a.E) {
             float kv = h[q];
-            if (a.noise)
-                kv = __fadd_rn(h[q], a.noise[(int64_t)t * a.E + e]);
-            else if (a.sel_bias)
-                kv = __fadd_rn(h[q], a.sel_bias[e]);
+            if (has_add) kv = __fadd_rn(h[q], kadd[q]);
             // A NaN key (NaN input) selects like -inf: every pick is still a
             // valid, distinct expert index (the lowest free one).
             key[q] = kv != kv ? -INFINITY : kv;
@@ -205,6 +217,8 @@ __global__ void __launch_bounds__(kThreads) router_simt_kernel(RouterArgs a) {
     for (int i = 0; i < RT; ++i) {
         const int t = t_base + warp * RT + i;
         if (t >= a.T) break;  // warp-uniform
+        float kadd[RE];
+        const bool has_add = key_addend<RE>(t, lane, a, kadd);
         float h[RE];
 #pragma unroll
         for (int q = 0; q < RE; ++q) {
@@ -215,7 +229,7 @@ __global__ void __launch_bounds__(kThreads) router_simt_kernel(RouterArgs a) {
                 a.logits[(int64_t)t * a.E + e] = h[q];
             }
         }
-        route_warp<RE>(h, t, lane, a, pacc);
+        route_warp<RE>(h, has_add, kadd, t, lane, a, pacc);
     }
     write_block_psum<RE>(pacc, a);
 }
@@ -230,25 +244,56 @@ __global__ void __launch_bounds__(kThreads) route_from_logits_kernel(RouterArgs 
 #pragma unroll
     for (int q = 0; q < RE; ++q) pacc[q] = 0.f;
     for (int t = warp; t < a.T; t += nwarps) {
+        float kadd[RE];
+        const bool has_add = key_addend<RE>(t, lane, a, kadd);
         float h[RE];
+        if (a.logit_part) {
+            // Split-K partials added in split order, then the bias; the loads
+            // of four splits are issued together.
+            const int64_t plane = (int64_t)a.T * a.E;
+            const float *part = a.logit_part + (int64_t)t * a.E;
 #pragma unroll
-        for (int q = 0; q < RE; ++q) {
-            const int e = lane + 32 * q;
-            h[q] = -INFINITY;
-            if (e < a.E) {
-                if (a.logit_part) {  // split-K partials in split order, then the bias
-                    float v = a.logit_part[(int64_t)t * a.E + e];
-                    for (int sp = 1; sp < a.ksplit; ++sp)
-                        v = __fadd_rn(v, a.logit_part[((int64_t)sp * a.T + t) * a.E + e]);
-                    if (a.b_gate) v += a.b_gate[e];
-                    a.logits[(int64_t)t * a.E + e] = v;
-                    h[q] = v;
-                } else {
-                    h[q] = a.logits[(int64_t)t * a.E + e];
+            for (int q = 0; q < RE; ++q) {
+                const int e = lane + 32 * q;
+                h[q] = e < a.E ? part[e] : -INFINITY;
+            }
+            int sp = 1;
+            for (; sp + 3 < a.ksplit; sp += 4) {
+                float p[4][RE];
+#pragma unroll
+                for (int i = 0; i < 4; ++i)
+#pragma unroll
+                    for (int q = 0; q < RE; ++q) {
+                        const int e = lane + 32 * q;
+                        p[i][q] = e < a.E ? part[(sp + i) * plane + e] : 0.f;
+                    }
+#pragma unroll
+                for (int i = 0; i < 4; ++i)
+#pragma unroll
+                    for (int q = 0; q < RE; ++q) h[q] = __fadd_rn(h[q], p[i][q]);
+            }
+            for (; sp < a.ksplit; ++sp)
+#pragma unroll
+                for (int q = 0; q < RE; ++q) {
+                    const int e = lane + 32 * q;
+                    if (e < a.E) h[q] = __fadd_rn(h[q], part[sp * plane + e]);
+                }
+#pragma unroll
+            for (int q = 0; q < RE; ++q) {
+                const int e = lane + 32 * q;
+                if (e < a.E) {
+                    if (a.b_gate) h[q] += a.b_gate[e];
+                    a.logits[(int64_t)t * a.E + e] = h[q];
                 }
             }
+        } else {
+#pragma unroll
+            for (int q = 0; q < RE; ++q) {
+                const int e = lane + 32 * q;
+                h[q] = e < a.E ? a.logits[(int64_t)t * a.E + e] : -INFINITY;
+            }
         }
-        route_warp<RE>(h, t, lane, a, pacc);
+        route_warp<RE>(h, has_add, kadd, t, lane, a, pacc);
     }
     write_block_psum<RE>(pacc, a);
 }
