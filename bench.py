@@ -337,8 +337,13 @@ def run_ours(args):
 
     cpu = None
     if not args.no_cpu_baseline and world == 1:
-        T_s = min(64, max(8, 2 * oracle_threads()))
+        # A first sample calibrates; the reported one is sized to about 12 s of
+        # oracle work (at most 512 tokens).
+        T_s = min(w.T, 64, max(8, 2 * oracle_threads()))
         secs, n = cpu_sample_from_device(w, inp, T_s)
+        if secs < 8.0 and T_s < min(w.T, 512):
+            T_s = int(min(w.T, 512, max(T_s + 1, T_s * 12.0 / max(secs, 1e-3))))
+            secs, n = cpu_sample_from_device(w, inp, T_s)
         cpu = {"value": n / secs, "unit": UNIT, "cores": oracle_threads(), "kind": "oracle",
                "sample": f"{n} tokens of {w.name} through the whole fp64 oracle forward (capacity at T={n}), "
                          f"{secs:.1f} s"}
