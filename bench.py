@@ -93,24 +93,25 @@ class ClockSampler:
             self.proc.wait(timeout=5)
         except subprocess.TimeoutExpired:
             self.proc.kill()
-        rows = []
-        for line in open(self.path):
-            parts = [p.strip() for p in line.split(",")]
-            if len(parts) < 8:
-                continue
-            try:
-                rows.append(parts)
-            except ValueError:
-                pass
+        with open(self.path) as f:
+            lines = f.readlines()
         os.unlink(self.path)
-        if not rows:
-            return None
-        sm = [float(r[0]) for r in rows if r[0].replace(".", "").isdigit()]
-        mx = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({names[i] for r in rows for i in range(4) if r[4 + i].lower() == "active"})
-        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
-                "reasons": reasons, "samples": len(rows)}
+        return summarize_clock_rows(lines)
+
+
+def summarize_clock_rows(lines):
+    """Median SM clock, max clock and the throttle reasons seen, from
+    nvidia-smi CSV rows of ClockSampler.FIELDS (no header, no units)."""
+    rows = [[p.strip() for p in line.split(",")] for line in lines]
+    rows = [r for r in rows if len(r) >= 8]
+    if not rows:
+        return None
+    sm = [float(r[0]) for r in rows if r[0].replace(".", "").isdigit()]
+    mx = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+    names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+    reasons = sorted({names[i] for r in rows for i in range(4) if r[4 + i].lower() == "active"})
+    return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+            "reasons": reasons, "samples": len(rows)}
 
 
 def gpu_id_for(dev) -> str:
