@@ -387,6 +387,9 @@ def committed_traffic(w):
     """DRAM bytes per expert-GEMM launch pair from the committed ncu summary, if
     the kernel source has not changed since it was captured."""
     import hashlib
+    from sparse_mixture_experts_gate_b200.workloads import WORKLOADS
+    if WORKLOADS.get(w.name) != w:  # a resized workload (--tokens / --experts): not the captured one
+        return None
     path = os.path.join(ROOT, "profiles", f"grouped_gemm_pair_{w.name}_traffic.txt")
     src = os.path.join(ROOT, "sparse_mixture_experts_gate_b200", "csrc", "gemm_pair.cu")
     if not os.path.exists(path):
