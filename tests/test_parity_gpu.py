@@ -499,11 +499,14 @@ def test_nan_tokens_route_to_valid_experts():
     assert np.isfinite(g["y"][good]).all()
 
 
+@pytest.mark.parametrize("T", [200, 1500])
 @pytest.mark.parametrize("dtype", ["bf16", "fp32"])
-def test_many_active_experts_k16(dtype):
+def test_many_active_experts_k16(dtype, T):
     """k = 16 of E = 40 (the largest k the layer takes): the combine's second
-    batch of routed terms, top-k over two expert lanes per warp lane group."""
-    w = WORKLOADS["default"].with_(T=200, E=40, k=16, S=1, capacity_factor=1.0, dtype=dtype,
+    batch of routed terms, top-k over two expert lanes per warp lane group.
+    T = 200 runs the combine with a block per token, T = 1500 (more than
+    eight tokens per SM) with a warp per token."""
+    w = WORKLOADS["default"].with_(T=T, E=40, k=16, S=1, capacity_factor=1.0, dtype=dtype,
                                    d=128 if dtype == "bf16" else 32, F=128 if dtype == "bf16" else 32,
                                    O=128 if dtype == "bf16" else 32, token_loss=True)
     full_check(w, make_inputs(w, "cpu", seed=91, random_biases=True))
