@@ -44,19 +44,22 @@ __device__ __forceinline__ int64_t assignment_of(const DispatchArgs &a, int i, i
     return a.rank_major ? (int64_t)(i % a.T) * a.k + i / a.T : (int64_t)i * a.k + j;
 }
 
-__global__ void __launch_bounds__(kChunk) dispatch_count_kernel(DispatchArgs a) {
+// Per-chunk expert histogram (one block of kChunk threads per chunk).
+__device__ __forceinline__ void dispatch_count(const DispatchArgs &a, int chunk) {
     __shared__ int cnt[kMaxE];
     for (int e = threadIdx.x; e < a.E; e += kChunk) cnt[e] = 0;
     __syncthreads();
-    const int i = blockIdx.x * kChunk + threadIdx.x;
+    const int i = chunk * kChunk + threadIdx.x;
     if (i < a.n_items)
         for (int j = 0; j < items_per(a); ++j) atomicAdd(&cnt[a.idx[assignment_of(a, i, j)]], 1);
     __syncthreads();
-    for (int e = threadIdx.x; e < a.E; e += kChunk) a.chunk_count[(int64_t)blockIdx.x * a.E + e] = cnt[e];
+    for (int e = threadIdx.x; e < a.E; e += kChunk) a.chunk_count[(int64_t)chunk * a.E + e] = cnt[e];
 }
 
+__global__ void __launch_bounds__(kChunk) dispatch_count_kernel(DispatchArgs a) { dispatch_count(a, blockIdx.x); }
+
 // Single CTA of kMaxE threads; thread e owns expert e.
-__global__ void __launch_bounds__(kMaxE) dispatch_scan_kernel(DispatchArgs a) {
+__device__ __forceinline__ void dispatch_scan(const DispatchArgs &a) {
     __shared__ int sc_rows[kMaxE];
     __shared__ int sc_tiles[kMaxE];
     __shared__ int sc_pre[kMaxE];
@@ -143,19 +146,23 @@ __global__ void __launch_bounds__(kMaxE) dispatch_scan_kernel(DispatchArgs a) {
     }
 }
 
-__global__ void __launch_bounds__(kChunk) dispatch_assign_kernel(DispatchArgs a) {
+__global__ void __launch_bounds__(kMaxE) dispatch_scan_kernel(DispatchArgs a) { dispatch_scan(a); }
+
+// Stable ranks within the chunk on top of the chunk's per-expert bases; slot,
+// row, row owner and the gate in expert order for every assignment.
+__device__ __forceinline__ void dispatch_assign(const DispatchArgs &a, int chunk) {
     constexpr int W = kChunk / 32;
     __shared__ uint32_t mask[W][kMaxE];
     __shared__ int wbase[W][kMaxE];
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     for (int i = tid; i < W * kMaxE; i += kChunk) (&mask[0][0])[i] = 0u;
     __syncthreads();
-    const int item = blockIdx.x * kChunk + tid;
+    const int item = chunk * kChunk + tid;
     if (item < a.n_items)
         for (int j = 0; j < items_per(a); ++j) atomicOr(&mask[warp][a.idx[assignment_of(a, item, j)]], 1u << lane);
     __syncthreads();
     for (int e = tid; e < a.E; e += kChunk) {
-        int run = a.chunk_base[(int64_t)blockIdx.x * a.E + e];
+        int run = a.chunk_base[(int64_t)chunk * a.E + e];
         for (int w = 0; w < W; ++w) {
             wbase[w][e] = run;
             run += __popc(mask[w][e]);
@@ -178,6 +185,18 @@ __global__ void __launch_bounds__(kChunk) dispatch_assign_kernel(DispatchArgs a)
         }
         a.row_of[ai] = row;
     }
+}
+
+__global__ void __launch_bounds__(kChunk) dispatch_assign_kernel(DispatchArgs a) { dispatch_assign(a, blockIdx.x); }
+
+// A batch of one chunk: the three steps in one block, ordered by block
+// barriers (which also order the block's global writes before its reads).
+__global__ void __launch_bounds__(kChunk) dispatch_one_chunk_kernel(DispatchArgs a) {
+    dispatch_count(a, 0);
+    __syncthreads();
+    dispatch_scan(a);
+    __syncthreads();
+    dispatch_assign(a, 0);
 }
 
 // Work item = (token, chunk of kScatterVec x 32 16-byte vectors of its row);
@@ -258,6 +277,12 @@ cudaError_t launch_ep_tiles(const EpTilesArgs &a, cudaStream_t s, int *launches)
 
 cudaError_t launch_dispatch(const DispatchArgs &a, cudaStream_t s, int *launches) {
     if (a.T <= 0) return cudaSuccess;
+    static_assert(kChunk == kMaxE, "the one-block path runs all three steps with the same threads");
+    if (a.n_chunks == 1) {
+        dispatch_one_chunk_kernel<<<1, kChunk, 0, s>>>(a);
+        *launches += 1;
+        return cudaGetLastError();
+    }
     dispatch_count_kernel<<<a.n_chunks, kChunk, 0, s>>>(a);
     dispatch_scan_kernel<<<1, kMaxE, 0, s>>>(a);
     dispatch_assign_kernel<<<a.n_chunks, kChunk, 0, s>>>(a);
