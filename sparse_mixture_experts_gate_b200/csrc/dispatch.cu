@@ -63,9 +63,10 @@ __device__ __forceinline__ void dispatch_scan(const DispatchArgs &a) {
     __shared__ int sc_rows[kMaxE];
     __shared__ int sc_tiles[kMaxE];
     __shared__ int sc_pre[kMaxE];
+    __shared__ int sc_nar[kMaxE];
     __shared__ int dropped_w[kMaxE / 32];
     const int e = threadIdx.x, lane = e & 31, warp = e >> 5;
-    int pre = 0, kept = 0, padded = 0, tiles = 0;
+    int pre = 0, kept = 0, padded = 0, tiles = 0, nars = 0;
     if (e < a.E) {
         // Exclusive prefix over chunks, loads batched so they are in flight together.
         const int32_t *__restrict__ cnt = a.chunk_count;
@@ -83,25 +84,29 @@ __device__ __forceinline__ void dispatch_scan(const DispatchArgs &a) {
         kept = (int64_t)pre < a.C ? pre : (int)a.C;
         padded = (kept + kRowBlock - 1) / kRowBlock * kRowBlock;
         tiles = (padded + kTokTile - 1) / kTokTile;
+        nars = (padded + kNarrowTile - 1) / kNarrowTile;
     }
     // Inclusive scans of the padded rows and of the token tiles over the block
     // (Hillis-Steele in shared memory).
     sc_rows[e] = padded;
     sc_tiles[e] = tiles;
     sc_pre[e] = pre;
+    sc_nar[e] = nars;
     __syncthreads();
     for (int off = 1; off < kMaxE; off <<= 1) {
         const int vr = e >= off ? sc_rows[e - off] : 0;
         const int vt = e >= off ? sc_tiles[e - off] : 0;
         const int vp = e >= off ? sc_pre[e - off] : 0;
+        const int vn = e >= off ? sc_nar[e - off] : 0;
         __syncthreads();
         sc_rows[e] += vr;
         sc_tiles[e] += vt;
         sc_pre[e] += vp;
+        sc_nar[e] += vn;
         __syncthreads();
     }
     const int start = sc_rows[e] - padded, tile0 = sc_tiles[e] - tiles;
-    const int routed_rows = sc_rows[kMaxE - 1], routed_tiles = sc_tiles[kMaxE - 1];
+    const int routed_rows = sc_rows[kMaxE - 1], routed_tiles = sc_tiles[kMaxE - 1], routed_nar = sc_nar[kMaxE - 1];
     int drop = pre - kept;
     for (int off = 16; off > 0; off >>= 1) drop += __shfl_xor_sync(0xffffffffu, drop, off);
     if (lane == 0) dropped_w[warp] = drop;
@@ -117,6 +122,12 @@ __device__ __forceinline__ void dispatch_scan(const DispatchArgs &a) {
         for (int r = start + kept; r < start + padded; ++r) a.row_assign[r] = -1;
         for (int i = 0; i < tiles; ++i)
             a.tok_tiles[tile0 + i] = make_int4(e, start + i * kTokTile, min(kTokTile, padded - i * kTokTile), 0);
+        if (a.narrow_tiles) {
+            const int n0 = sc_nar[e] - nars;
+            for (int i = 0; i < nars; ++i)
+                a.narrow_tiles[n0 + i] =
+                    make_int4(e, start + i * kNarrowTile, min(kNarrowTile, padded - i * kNarrowTile), 0);
+        }
     }
     // Shared experts: one T_pad-row segment each, after the routed rows.
     const int shared_blocks = a.T_pad / kRowBlock;
@@ -128,6 +139,13 @@ __device__ __forceinline__ void dispatch_scan(const DispatchArgs &a) {
         a.tok_tiles[routed_tiles + i] = make_int4(a.E + sh, routed_rows + sh * a.T_pad + j * kTokTile,
                                                   min(kTokTile, a.T_pad - j * kTokTile), 0);
     }
+    const int shared_nar = (a.T_pad + kNarrowTile - 1) / kNarrowTile;
+    if (a.narrow_tiles)
+        for (int i = e; i < a.S * shared_nar; i += kMaxE) {
+            const int sh = i / shared_nar, j = i - sh * shared_nar;
+            a.narrow_tiles[routed_nar + i] = make_int4(a.E + sh, routed_rows + sh * a.T_pad + j * kNarrowTile,
+                                                       min(kNarrowTile, a.T_pad - j * kNarrowTile), 0);
+        }
     if (e < a.S) {
         a.group_start[a.E + e] = routed_rows + e * a.T_pad;
         a.group_rows[a.E + e] = a.T;
@@ -141,6 +159,7 @@ __device__ __forceinline__ void dispatch_scan(const DispatchArgs &a) {
         a.ctrl[kCtrlNumRowBlocks] = total / kRowBlock;
         a.ctrl[kCtrlNumTokTiles] = routed_tiles + a.S * shared_tiles;
         a.ctrl[kCtrlRoutedTiles] = routed_tiles;
+        a.ctrl[kCtrlNumNarrowTiles] = a.narrow_tiles ? routed_nar + a.S * shared_nar : 0;
         a.ctrl[kCtrlRoutedRows] = routed_rows;
         a.ctrl[kCtrlDropped] = d;
     }

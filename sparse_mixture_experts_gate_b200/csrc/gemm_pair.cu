@@ -46,9 +46,6 @@ constexpr int kThreads = 192;
 constexpr int kFeatPair = 256;                     // MMA M: features per pair tile
 constexpr int kFeatCta = 128;                      // features per CTA
 constexpr int kABytes = kFeatCta * kBK * 2;        // 16 KB: 128 weight rows x 64 K
-constexpr int kBBytes = (kTokTile / 2) * kBK * 2;  // 16 KB: up to 128 token rows x 64 K
-constexpr int kStage = kABytes + kBBytes;
-constexpr int kStages = 6;
 constexpr int kAccCols = 256;
 constexpr int kBoxTok = 32, kBoxFeat = 32;          // store box: 32 tokens x 32 features
 constexpr int kBoxBytes = kBoxTok * kBoxFeat * 2;
@@ -56,9 +53,22 @@ constexpr int kStaging = 4 * 2 * kBoxBytes;         // 4 epilogue warps x 2 boxe
 constexpr int kRowsPerLoad16 = 16;                  // rows of the narrow token box
 constexpr int kRing = 8;            // unit-index ring between the leader's producer and the consumers
 constexpr int kRingConsumers = 10;  // leader: MMA thread + 4 epilogue warps; peer: producer + 4 epilogue warps
-constexpr int kSmem = 1024 + kStages * kStage + kStaging + 512;
-static_assert(kSmem <= 232448, "exceeds the 227 KB of shared memory a CTA may use");
 static_assert(kTokTile == 256 && kTokTile % (2 * kRowsPerLoad16) == 0, "token tile layout");
+static_assert(kNarrowTile % (2 * kRowsPerLoad16) == 0, "narrow token tile layout");
+
+// Stage layout for token tiles of up to TILE rows (each CTA stages TILE / 2):
+// 256-row tiles with 6 stages of 32 KB, or narrow 64-row tiles with 10 stages
+// of 20 KB, which keeps 160 KB of weight tiles in flight per SM when the
+// token tiles are short and the GEMM streams weights.
+template <int TILE>
+struct PairCfg {
+    static constexpr int kB = (TILE / 2) * kBK * 2;
+    static constexpr int kStage = kABytes + kB;
+    static constexpr int kStages = TILE == kTokTile ? 6 : 10;
+    static constexpr int kSmem = 1024 + kStages * kStage + kStaging + 512;
+    static_assert(kSmem <= 232448, "exceeds the 227 KB of shared memory a CTA may use");
+    static_assert(kB % 1024 == 0, "B stages keep the 1024-byte swizzle alignment");
+};
 
 struct Smem {
     uint8_t *sA, *sB, *staging;
@@ -67,15 +77,17 @@ struct Smem {
     int32_t *ring;
 };
 
+template <int TILE>
 __device__ __forceinline__ Smem carve(uint8_t *raw) {
+    using C = PairCfg<TILE>;
     uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(raw) + 1023) & ~uintptr_t(1023));
     Smem s;
     s.sA = base;
-    s.sB = base + kStages * kABytes;
-    s.staging = base + kStages * kStage;
+    s.sB = base + C::kStages * kABytes;
+    s.staging = base + C::kStages * C::kStage;
     s.full = reinterpret_cast<uint64_t *>(s.staging + kStaging);
-    s.empty = s.full + kStages;
-    s.tfull = s.empty + kStages;
+    s.empty = s.full + C::kStages;
+    s.tfull = s.empty + C::kStages;
     s.tempty = s.tfull + 2;
     s.mma_done = s.tempty + 2;
     s.ring_full = s.mma_done + 1;
@@ -85,14 +97,16 @@ __device__ __forceinline__ Smem carve(uint8_t *raw) {
     return s;
 }
 
-template <int ACT>
+template <int ACT, int TILE>
 __global__ void __launch_bounds__(kThreads, 1)
     grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap map_w, const __grid_constant__ CUtensorMap map_t,
                              const __grid_constant__ CUtensorMap map_t16, const __grid_constant__ CUtensorMap map_s,
                              const __grid_constant__ CUtensorMap map_s16, const __grid_constant__ CUtensorMap map_out,
                              const PairGemmArgs a) {
+    using C = PairCfg<TILE>;
+    constexpr int kStages = C::kStages;
     extern __shared__ uint8_t smem_raw[];
-    const Smem s = carve(smem_raw);
+    const Smem s = carve<TILE>(smem_raw);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const uint32_t rank = cluster_ctarank();
     const bool leader = rank == 0;
@@ -129,7 +143,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t tmem_base = *s.tmem_slot;
 
     const int4 *tok_tiles = a.tok_tiles + (a.tile_base_word >= 0 ? a.ctrl[a.tile_base_word] : 0);
-    const int n_tt = a.fixed_tiles > 0 ? a.fixed_tiles : min(a.ctrl[kCtrlNumTokTiles], a.max_tok_tiles);
+    const int n_tt = a.fixed_tiles > 0 ? a.fixed_tiles : min(a.ctrl[a.tiles_count_word], a.max_tok_tiles);
     const int total = n_tt * a.n_ftiles;
     // Weight-stack index of group g (shared groups may sit at another base).
     auto wgroup = [&](int g) { return g < a.E ? g : a.w_shared_base + (g - a.E); };
@@ -198,7 +212,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (lane == 0 && leader) mbar_arrive_expect_tx(&s.full[st], tx_bytes);
                 __syncwarp();
                 const uint32_t bar = mapa_shared(smem_u32(&s.full[st]), 0);
-                uint8_t *sA = s.sA + st * kABytes, *sB = s.sB + st * kBBytes;
+                uint8_t *sA = s.sA + st * kABytes, *sB = s.sB + st * C::kB;
                 if (lane == 0) tma_load_2d_pair(&map_w, bar, sA, kb * kBK, wrow);
                 if (ntok == kTokTile) {
                     if (lane == 1) tma_load_2d_pair(mt, bar, sB, kb * kBK, trow);
@@ -233,7 +247,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                     tc_fence_after_sync();
                     const uint64_t ad = sw128_kmajor_desc(smem_u32(s.sA + st * kABytes));
-                    const uint64_t bd = sw128_kmajor_desc(smem_u32(s.sB + st * kBBytes));
+                    const uint64_t bd = sw128_kmajor_desc(smem_u32(s.sB + st * C::kB));
 #pragma unroll
                     for (int kk = 0; kk < kBK / 16; ++kk)
                         tc_mma_bf16_pair(d_tmem, ad + 2u * kk, bd + 2u * kk, idesc, (kb | kk) != 0 ? 1u : 0u);
@@ -318,11 +332,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
 }
 
-template <int ACT>
+template <int ACT, int TILE>
 cudaError_t launch_act(const CUtensorMap &mw, const CUtensorMap &mt, const CUtensorMap &mt16, const CUtensorMap &ms,
                        const CUtensorMap &ms16, const CUtensorMap &mo, const PairGemmArgs &a, cudaStream_t st) {
-    auto kern = grouped_gemm_pair_kernel<ACT>;
-    cudaError_t e = set_smem_limit_once<grouped_gemm_pair_kernel<ACT>>(kSmem);
+    constexpr int kSmem = PairCfg<TILE>::kSmem;
+    auto kern = grouped_gemm_pair_kernel<ACT, TILE>;
+    cudaError_t e = set_smem_limit_once<grouped_gemm_pair_kernel<ACT, TILE>>(kSmem);
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(2 * a.num_pairs, 1, 1);
@@ -345,6 +360,9 @@ int gemm_pair_max_pairs(int num_sms) {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(2 * (num_sms / 2), 1, 1);
     cfg.blockDim = dim3(kThreads, 1, 1);
+    // The larger of the two stage layouts; both allow one CTA per SM.
+    constexpr int kSmem = PairCfg<kNarrowTile>::kSmem > PairCfg<kTokTile>::kSmem ? PairCfg<kNarrowTile>::kSmem
+                                                                                   : PairCfg<kTokTile>::kSmem;
     cfg.dynamicSmemBytes = kSmem;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -353,7 +371,7 @@ int gemm_pair_max_pairs(int num_sms) {
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    auto kern = grouped_gemm_pair_kernel<-1>;
+    auto kern = grouped_gemm_pair_kernel<-1, kTokTile>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem) != cudaSuccess) return 0;
     int clusters = 0;
     if (cudaOccupancyMaxActiveClusters(&clusters, kern, &cfg) != cudaSuccess) return 0;
@@ -367,11 +385,19 @@ cudaError_t launch_gemm_pair(const CUtensorMap &map_w, const CUtensorMap &map_t,
                              const PairGemmArgs &a, cudaStream_t s, int *launches) {
     if (a.num_pairs <= 0) return cudaErrorInvalidConfiguration;
     ++*launches;
+    if (a.narrow) {
+        switch (a.act) {
+            case 0: return launch_act<0, kNarrowTile>(map_w, map_t, map_t16, map_s, map_s16, map_out, a, s);
+            case 1: return launch_act<1, kNarrowTile>(map_w, map_t, map_t16, map_s, map_s16, map_out, a, s);
+            case 2: return launch_act<2, kNarrowTile>(map_w, map_t, map_t16, map_s, map_s16, map_out, a, s);
+            default: return launch_act<-1, kNarrowTile>(map_w, map_t, map_t16, map_s, map_s16, map_out, a, s);
+        }
+    }
     switch (a.act) {
-        case 0: return launch_act<0>(map_w, map_t, map_t16, map_s, map_s16, map_out, a, s);
-        case 1: return launch_act<1>(map_w, map_t, map_t16, map_s, map_s16, map_out, a, s);
-        case 2: return launch_act<2>(map_w, map_t, map_t16, map_s, map_s16, map_out, a, s);
-        default: return launch_act<-1>(map_w, map_t, map_t16, map_s, map_s16, map_out, a, s);
+        case 0: return launch_act<0, kTokTile>(map_w, map_t, map_t16, map_s, map_s16, map_out, a, s);
+        case 1: return launch_act<1, kTokTile>(map_w, map_t, map_t16, map_s, map_s16, map_out, a, s);
+        case 2: return launch_act<2, kTokTile>(map_w, map_t, map_t16, map_s, map_s16, map_out, a, s);
+        default: return launch_act<-1, kTokTile>(map_w, map_t, map_t16, map_s, map_s16, map_out, a, s);
     }
 }
 

@@ -84,11 +84,11 @@ struct Plan {
     int T = 0;
     int64_t C = 0;
     int T_pad = 0, n_stat_chunks = 0, n_chunks = 0, R_routed_max = 0, R_max = 0, max_row_blocks = 0;
-    int max_tok_tiles = 0;
+    int max_tok_tiles = 0, max_narrow_tiles = 0;
     int ksplit = 1;
     size_t o_lpart = 0;
     size_t o_ctrl, o_logits, o_idx, o_gates, o_slot, o_rowof, o_lse, o_psum, o_ccount, o_cbase, o_cpre, o_ckept,
-        o_gstart, o_grows, o_bgroup, o_toktiles, o_rowassign, o_wsplit, o_xp, o_h, o_o, o_credit, o_partials,
+        o_gstart, o_grows, o_bgroup, o_toktiles, o_narrowtiles, o_rowassign, o_wsplit, o_xp, o_h, o_o, o_credit, o_partials,
         o_prestart, o_gsorted, o_rownorm, o_gz;
     size_t total = 0;
 };
@@ -128,6 +128,15 @@ int64_t capacity_of(const moe_config_t &c, int T) {
     return (int64_t)std::ceil((double)c.capacity_factor * (double)c.num_active * (double)T / (double)c.num_experts);
 }
 
+// The expert GEMMs run narrow units (token tiles of at most kNarrowTile rows,
+// a deeper pipeline of weight tiles) when the experts' segments average at
+// most kNarrowTile rows: there the GEMMs stream the weights and the token
+// tiles are short anyway (decode-sized batches).
+bool narrow_gemm(const moe_layer *L, int T) {
+    const moe_config_t &c = L->cfg;
+    return L->tc && (int64_t)c.num_active * T <= (int64_t)kNarrowTile * c.num_experts;
+}
+
 Plan make_plan(const moe_layer &L, int T) {
     const moe_config_t &c = L.cfg;
     Plan p;
@@ -144,6 +153,8 @@ Plan make_plan(const moe_layer &L, int T) {
     // Each expert's segment splits into ceil(rows / 256) token tiles of >= 32 rows.
     p.max_tok_tiles = (int)std::min<int64_t>(routed / kTokTile + E, routed / kRowBlock) +
                       S * (int)((p.T_pad + kTokTile - 1) / kTokTile);
+    p.max_narrow_tiles = (int)std::min<int64_t>(routed / kNarrowTile + E, routed / kRowBlock) +
+                         S * (int)((p.T_pad + kNarrowTile - 1) / kNarrowTile);
     // bf16 linear routers route from the tensor-core logits; the MLP gate and
     // fp32 layers route inside the CUDA-core router kernel.
     p.n_stat_chunks = router_psum_blocks(T, L.num_sms, c.dtype == MOE_DTYPE_BF16 && !c.use_mlp_gater);
@@ -172,6 +183,7 @@ Plan make_plan(const moe_layer &L, int T) {
     p.o_grows = take((size_t)(E + S) * 4);
     p.o_bgroup = take((size_t)p.max_row_blocks * 4);
     p.o_toktiles = take((size_t)std::max(p.max_tok_tiles, 1) * 16);
+    p.o_narrowtiles = take((size_t)std::max(p.max_narrow_tiles, 1) * 16);
     p.o_rowassign = take((size_t)p.R_max * 4);
     p.o_partials = take((size_t)(4 * E + 3) * 4);
     p.o_prestart = take((size_t)E * 4);
@@ -499,6 +511,7 @@ int fwd_route(moe_layer_t *L, const void *x, int32_t T, const float *logit_noise
     da.group_rows = reinterpret_cast<int32_t *>(ws + p.o_grows);
     da.block_group = reinterpret_cast<int32_t *>(ws + p.o_bgroup);
     da.tok_tiles = reinterpret_cast<int4 *>(ws + p.o_toktiles);
+    da.narrow_tiles = narrow_gemm(L, T) ? reinterpret_cast<int4 *>(ws + p.o_narrowtiles) : nullptr;
     da.ctrl = ctrl;
     da.slot = slot;
     da.row_of = reinterpret_cast<int32_t *>(ws + p.o_rowof);
@@ -555,6 +568,12 @@ int fwd_expert_gemms(moe_layer_t *L, cudaStream_t s, bool shared_only) {
         if (shared_only) {  // the shared experts' tiles follow the routed ones
             g1.tile_base_word = kCtrlRoutedTiles;
             g1.fixed_tiles = S * ((p.T_pad + kTokTile - 1) / kTokTile);
+        }
+        if (!shared_only && narrow_gemm(L, T)) {
+            g1.tok_tiles = reinterpret_cast<const int4 *>(ws + p.o_narrowtiles);
+            g1.tiles_count_word = kCtrlNumNarrowTiles;
+            g1.max_tok_tiles = p.max_narrow_tiles;
+            g1.narrow = 1;
         }
         g1.use_s = 1;
         g1.bias = L->w.b1;

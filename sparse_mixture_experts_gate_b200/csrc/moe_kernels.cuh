@@ -69,6 +69,7 @@ struct DispatchArgs {
     int32_t *group_rows;    // [E+S]
     int32_t *block_group;   // [max_row_blocks]: group of each 32-row block
     int4 *tok_tiles;        // [max_tok_tiles]: {group, first row, rows, 0}
+    int4 *narrow_tiles = nullptr;  // [max_narrow_tiles]: the same with at most kNarrowTile rows, or null
     int32_t *ctrl;          // control block (see kCtrl*)
     int32_t *slot;          // [T][k]
     int32_t *row_of;        // [T][k]
@@ -89,8 +90,14 @@ enum {
     kCtrlWork1 = 5,  // unit counters of the two expert GEMM launches
     kCtrlWork2 = 6,
     kCtrlRoutedTiles = 7,  // token tiles of the routed experts (the shared experts' follow)
-    kCtrlWords = 8
+    kCtrlNumNarrowTiles = 8,
+    kCtrlWords = 9
 };
+
+// Rows of a narrow token tile: for short expert segments the expert GEMM
+// stages at most kNarrowTile / 2 token rows per CTA, leaving room for a
+// deeper pipeline of weight tiles.
+constexpr int kNarrowTile = 64;
 
 // Scatter of token rows into the permuted row space (rows of kept assignments).
 struct ScatterArgs {
@@ -121,7 +128,9 @@ struct PairGemmArgs {
     int E;                       // groups >= E are shared experts
     int w_shared_base = 0;       // weight-stack index of the first shared group (E, or the local count)
     int tile_base_word = -1;     // ctrl word holding the index of the first tile to run, or -1 (tile 0)
-    int fixed_tiles = 0;         // > 0: run this many tiles instead of ctrl[kCtrlNumTokTiles]
+    int fixed_tiles = 0;         // > 0: run this many tiles instead of ctrl[tiles_count_word]
+    int tiles_count_word = kCtrlNumTokTiles;  // ctrl word holding the tile count
+    int narrow = 0;              // 1: tok_tiles holds narrow tiles (at most kNarrowTile rows)
     int use_s;
     const float *bias;           // [G][N] or null
     int act;                     // activation code, -1 none
