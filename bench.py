@@ -14,9 +14,15 @@ With N > 1 (one process per GPU under torchrun) every rank runs its own replica
 on its own batch (weak scaling, no collective on the data path); the timed
 region is bracketed by barriers and the max over ranks is reported.
 
-Rank 0 prints one JSON line: whole-job tokens/s, the expert-GEMM roofline
-fraction measured with CUDA events inside the timed region, the end-to-end
-number with host buffers, the CPU-oracle baseline and the SM clocks.
+`--gpus N` without a launcher starts the N ranks itself (torch.distributed.run
+on 127.0.0.1, bounded by `timeout`).
+
+Rank 0 prints one JSON line: whole-job tokens/s, the layer and expert-GEMM
+roofline fractions measured with CUDA events inside the timed region (against
+the burst bf16 peak, the sustained one beside it), the end-to-end number with
+host buffers, the CPU-oracle baseline and the SM clocks. Under "configs" the
+same line carries the device measurement of the other named configurations
+(tiny, default, e64, decode), each timed the same way after the headline one.
 `--impl reference` times the CPU oracle (the reference arm) instead.
 """
 from __future__ import annotations
@@ -46,6 +52,7 @@ def parse():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-extras", action="store_true", help="time the headline workload only")
     # Smaller variants of a workload, for profiler captures of the same kernels.
     ap.add_argument("--tokens", type=int, default=None, help="override T (profiling)")
     ap.add_argument("--experts", type=int, default=None, help="override E (profiling)")
@@ -170,28 +177,40 @@ def oracle_threads():
 
 # ---------------------------------------------------------------- our arm
 
-def run_ours(args):
+def layer_roofline(w, kept, touched, ms_step, peaks):
+    """Roofline numbers of one layer step from the algorithmic work: expert-GEMM
+    FLOPs (kept + shared rows) and minimum bytes (x once, W_g, the weights of
+    experts with a kept row, y once, routing metadata). The layer's ideal time
+    is the slower of the FLOPs at the bf16 tensor peak and the bytes at the HBM
+    peak; the burst tensor peak is the headline denominator (a step timed over a
+    fraction of a second), the sustained one is reported beside it."""
+    rows = kept + w.S * w.T
+    flops = 2.0 * rows * w.F * (w.d + w.O)
+    es = 2 if w.dtype == "bf16" else 4
+    bytes_min = (w.T * w.d * es + w.E * w.d * 4 + touched * (w.F * w.d + w.O * w.F) * es + w.T * w.O * es
+                 + w.T * w.k * 12)
+    t = ms_step / 1e3
+    t_flop = flops / (peaks["bf16"] * 1e12)
+    t_flop_s = flops / (peaks["bf16_sustained"] * 1e12)
+    t_bytes = bytes_min / (peaks["hbm_gbs"] * 1e9)
+    return {"flops": flops, "bytes_min": bytes_min, "bound": "tensor" if t_flop >= t_bytes else "hbm",
+            "expert_gemm_tflops": flops / t / 1e12, "hbm_gbs": bytes_min / t / 1e9,
+            "layer_roofline_frac": max(t_flop, t_bytes) / t,
+            "layer_roofline_frac_sustained": max(t_flop_s, t_bytes) / t,
+            "hbm_frac": t_bytes / t}
+
+
+def measure(w, args, dev, rank, world, headline):
+    """Times one workload: an instrumented eager loop (per-stage CUDA events
+    recorded by the library), then the step replayed as a CUDA graph (the
+    timed number), then, for the headline workload, the end-to-end pipeline
+    with host buffers. Every rank runs the same collectives in the same order."""
     import torch
     import torch.distributed as dist
     from sparse_mixture_experts_gate_b200 import binding
     from sparse_mixture_experts_gate_b200.binding import MoELayer
-    from sparse_mixture_experts_gate_b200.workloads import WORKLOADS, make_inputs, make_tokens
+    from sparse_mixture_experts_gate_b200.workloads import make_inputs, make_tokens
 
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
-    if world > 1:
-        import datetime
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
-    dev = torch.device("cuda", local)
-    torch.cuda.set_device(dev)
-
-    w = WORKLOADS[args.workload]
-    if args.tokens:
-        w = w.with_(T=args.tokens)
-    if args.experts:
-        w = w.with_(E=args.experts)
     inp = make_inputs(w, "cuda")
     if rank > 0:  # each replica routes its own batch of tokens
         inp.update(make_tokens(w, "cuda", seed=w.seed + 7919 * rank))
@@ -201,22 +220,24 @@ def run_ours(args):
     out = layer.alloc_outputs(T)
     layer.workspace(T)
     stream = torch.cuda.current_stream()
+    fits_l2 = not inputs_exceed_l2(w)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev) if fits_l2 else None
 
     def step():
         layer.forward(x, noise=noise, out=out)
         layer.aux_stats(out, token_loss=tl)
 
-    for _ in range(max(args.warmup, 3)):
+    W = max(args.warmup, 3)
+    for _ in range(W):
         step()
     torch.cuda.synchronize()
     if layer.device_status() != 0:
-        raise RuntimeError("device status reports a timeout")
+        raise RuntimeError(f"{w.name}: device status reports a timeout")
     kept = int(out["count_kept"].sum().item())
-    rows = kept + w.S * T
-    flops_g1 = 2.0 * rows * w.F * w.d
-    flops_g2 = 2.0 * rows * w.F * w.O
+    touched = int((out["count_kept"] > 0).sum().item()) + w.S
     launches_per_step = layer.launch_count()
 
+    # Per-stage times from the library's stage events (eager launches).
     K = args.steps
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(binding.MOE_TIMING_EVENTS)] for _ in range(K)]
     for row in evs:  # materialise the event handles
@@ -224,51 +245,46 @@ def run_ours(args):
             e.record(stream)
     torch.cuda.synchronize()
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    clocks = ClockSampler(gpu_id_for(local))
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
-    clocks.start()
-    time.sleep(0.3)
     start.record(stream)
     for i in range(K):
+        if flush is not None:
+            flush.fill_(i & 0xFF)
         binding.moe_set_timing_events(layer.handle, [e.cuda_event for e in evs[i]])
         step()
     end.record(stream)
     torch.cuda.synchronize()
-    clk = clocks.stop()
     binding.moe_set_timing_events(layer.handle, None)
-    if world > 1:
-        dist.barrier()
-    ms = start.elapsed_time(end)
     stage = {n: [] for n in binding.STAGES}
     for row in evs:
         for j, n in enumerate(binding.STAGES):
             stage[n].append(row[j].elapsed_time(row[j + 1]))
-    # The headline timing replays the step as one CUDA graph (the same kernels on
-    # the same buffers, without per-launch host overhead); the instrumented
-    # eager loop above gives the per-stage times.
+    eager_steps = [row[0].elapsed_time(row[-1]) for row in evs]
+
+    # The timed number: the step replayed as one CUDA graph (the same kernels on
+    # the same buffers, without per-launch host overhead).
     graph = binding.StepGraph(layer, x, noise=noise, token_loss=tl, out=out)
-    for _ in range(max(args.warmup, 3)):
+    for _ in range(W):
         graph.replay()
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
-    clocks = ClockSampler(gpu_id_for(local))
+    clocks = ClockSampler(gpu_id_for(dev.index))
     clocks.start()
     time.sleep(0.3)
-    if inputs_exceed_l2(w):
+    if flush is None:
         start.record(stream)
         for _ in range(K):
             graph.replay()
         end.record(stream)
         torch.cuda.synchronize()
-        ms_graph = start.elapsed_time(end)
+        ms = start.elapsed_time(end)
     else:
         # The layer's data fits in L2: before every timed step a 256 MB write
-        # (twice L2) evicts it, outside the step's events.
-        flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+        # (twice L2) evicts it, outside the step's own events.
         ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
         for i in range(K):
             flush.fill_(i & 0xFF)
@@ -276,28 +292,27 @@ def run_ours(args):
             graph.replay()
             ev[i][1].record(stream)
         torch.cuda.synchronize()
-        ms_graph = sum(a.elapsed_time(b) for a, b in ev)
-        del flush
+        ms = sum(a.elapsed_time(b) for a, b in ev)
     clk = clocks.stop()
     if world > 1:
         dist.barrier()
-    ms_eager = ms
-    ms = ms_graph
     if layer.device_status() != 0:
-        raise RuntimeError("device status reports a timeout")
+        raise RuntimeError(f"{w.name}: device status reports a timeout")
     ms_t = torch.tensor([ms], device=dev)
     if world > 1:
         dist.all_reduce(ms_t, op=dist.ReduceOp.MAX)
     ms_max = float(ms_t.item())
-    ms_step = ms_max / K
-    value = world * T * K / (ms_max / 1e3)
+    res = dict(w=w, inp=inp, T=T, K=K, ms_max=ms_max, ms_step=ms_max / K, ms_eager=statistics.mean(eager_steps),
+               stage={n: statistics.mean(v) for n, v in stage.items()}, kept=kept, touched=touched,
+               n_dropped=int(out["n_dropped"].item()), launches_per_step=launches_per_step, clocks=clk,
+               value=world * T * K / (ms_max / 1e3))
 
     # End to end through the public API with host buffers: binding.HostPipeline
     # uploads each step's inputs from pinned host memory, runs the forward and
     # statistics, and downloads y and the statistics, overlapping the copies of
     # one step with the neighbouring steps' compute (two device slots).
-    e2e = None
-    if not args.no_e2e:
+    res["e2e"] = None
+    if headline and not args.no_e2e:
         x_h = x.cpu().pin_memory()
         noise_h = noise.cpu().pin_memory() if noise is not None else None
         tl_h = tl.cpu().pin_memory() if tl is not None else None
@@ -323,36 +338,85 @@ def run_ours(args):
         h2d = x_h.numel() * x_h.element_size() + (noise_h.numel() * 4 if noise_h is not None else 0) + \
             (tl_h.numel() * 4 if tl_h is not None else 0)
         d2h = y_h[0].numel() * y_h[0].element_size() + sum(v.numel() * v.element_size() for v in st_h[0].values())
-        e2e = {"value": world * T * Ke / (float(t2.item()) / 1e3), "unit": UNIT, "h2d_bytes_per_step": int(h2d),
-               "d2h_bytes_per_step": int(d2h), "steps": Ke,
-               "how": "binding.HostPipeline: pinned-host inputs uploaded, forward + statistics, y and statistics "
-                      "downloaded every step; copies of one step overlap the neighbouring steps' compute"}
+        res["e2e"] = {"value": world * T * Ke / (float(t2.item()) / 1e3), "unit": UNIT,
+                      "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h), "steps": Ke,
+                      "how": "binding.HostPipeline: pinned-host inputs uploaded, forward + statistics, y and "
+                             "statistics downloaded every step; copies of one step overlap the neighbouring "
+                             "steps' compute"}
+        del pipe
+    del graph, layer, out, flush
+    return res
 
-    if rank != 0:
-        if world > 1:
-            dist.destroy_process_group()
-        return
 
-    peaks = measured_peaks()
-    g1 = statistics.mean(stage["gemm1"])
-    g2 = statistics.mean(stage["gemm2"])
-    achieved = (flops_g1 + flops_g2) / ((g1 + g2) / 1e3) / 1e12  # TFLOP/s per launch pair
-    traffic = committed_traffic(w)
-    layer_flops = flops_g1 + flops_g2
-    step_tflops = layer_flops / (ms_step / 1e3) / 1e12
-    # Algorithmic layer bytes: x once, W_g, weights of experts with a kept row, y once, routing metadata.
-    es = 2 if w.dtype == "bf16" else 4
-    touched = int((out["count_kept"] > 0).sum().item()) + w.S
-    bytes_min = T * w.d * es + w.E * w.d * 4 + touched * (w.F * w.d + w.O * w.F) * es + T * w.O * es + T * w.k * 12
-    # Ideal layer time: the slower of the expert-GEMM FLOPs at the bf16 tensor peak and the algorithmic
-    # bytes at the HBM peak. Steps run back to back hold the GPU at its power cap, so the sustained
-    # tensor peak is the denominator; the burst-peak figure is reported beside it.
-    t_bytes = bytes_min / (peaks["hbm_gbs"] * 1e9)
-    layer_frac = max(layer_flops / (peaks["bf16_sustained"] * 1e12), t_bytes) / (ms_step / 1e3)
-    layer_frac_burst = max(layer_flops / (peaks["bf16"] * 1e12), t_bytes) / (ms_step / 1e3)
+def gemm_roofline(r, peaks):
+    """The expert GEMMs (both launches) between their own stage events. A
+    tensor-bound layer: the algorithmic FLOPs of the kept and shared rows over
+    their mean duration, against the bf16 tensor peak. An HBM-bound layer
+    (decode-sized batches): the weight bytes of the experts with a kept row
+    (the bytes the two GEMMs must stream) over the same duration, against the
+    HBM peak."""
+    w = r["w"]
+    rows = r["kept"] + w.S * w.T
+    ms = r["stage"]["gemm1"] + r["stage"]["gemm2"]
+    lr = layer_roofline(w, r["kept"], r["touched"], r["ms_step"], peaks)
+    if lr["bound"] == "hbm":
+        es = 2 if w.dtype == "bf16" else 4
+        wbytes = r["touched"] * (w.F * w.d + w.O * w.F) * es
+        achieved = wbytes / (ms / 1e3) / 1e9
+        return {"kernel": "grouped_gemm_pair (expert GEMM 1 + 2)", "bound": "hbm", "achieved": achieved,
+                "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"],
+                "peak_kind": f"HBM copy ({peaks['source']})", "algorithmic_bytes": wbytes}
+    achieved = 2.0 * rows * w.F * (w.d + w.O) / (ms / 1e3) / 1e12
+    return {"kernel": "grouped_gemm_pair (expert GEMM 1 + 2)", "bound": "tensor", "achieved": achieved,
+            "peak": peaks["bf16"], "unit": "TFLOP/s", "frac": achieved / peaks["bf16"],
+            "frac_sustained": achieved / peaks["bf16_sustained"],
+            "peak_kind": f"bf16 burst ({peaks['source']}); frac_sustained against the sustained peak"}
 
+
+def config_summary(r, peaks):
+    """The sub-object of one non-headline configuration."""
+    w = r["w"]
+    d = {"T": w.T, "d": w.d, "d_ff": w.F, "out": w.O, "E": w.E, "k": w.k, "S": w.S, "dtype": w.dtype,
+         "ms_per_step": r["ms_step"], "value": r["value"], "unit": UNIT, "steps": r["K"],
+         "ms_per_step_eager": r["ms_eager"], "stage_ms": r["stage"], "kept_rows": r["kept"],
+         "n_dropped": r["n_dropped"], "gpu_launches": r["launches_per_step"] * r["K"], "clocks": r["clocks"],
+         "l2": l2_note(w)}
+    if w.dtype == "bf16":
+        d.update(layer_roofline(w, r["kept"], r["touched"], r["ms_step"], peaks))
+        d["roofline"] = gemm_roofline(r, peaks)
+    else:
+        d["bound"] = "latency"
+        d["note"] = "fp32 layer on CUDA cores at T=4: launch-latency bound, no roofline"
+    return d
+
+
+EXTRA_CONFIGS = ("tiny", "default", "e64", "decode")
+
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+    from sparse_mixture_experts_gate_b200.workloads import WORKLOADS
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+
+    w = WORKLOADS[args.workload]
+    if args.tokens:
+        w = w.with_(T=args.tokens)
+    if args.experts:
+        w = w.with_(E=args.experts)
+    head = measure(w, args, dev, rank, world, headline=True)
+    inp = head.pop("inp")
     cpu = None
-    if not args.no_cpu_baseline and world == 1:
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
         # A first sample calibrates; the reported one is sized to about 12 s of
         # oracle work (at most 512 tokens).
         T_s = min(w.T, 64, max(8, 2 * oracle_threads()))
@@ -363,28 +427,48 @@ def run_ours(args):
         cpu = {"value": n / secs, "unit": UNIT, "cores": oracle_threads(), "kind": "oracle",
                "sample": f"{n} tokens of {w.name} through the whole fp64 oracle forward (capacity at T={n}), "
                          f"{secs:.1f} s"}
+    del inp
+    torch.cuda.empty_cache()
+    extras = {}
+    if args.workload == "e256" and not (args.tokens or args.experts or args.no_extras):
+        for name in EXTRA_CONFIGS:
+            r = measure(WORKLOADS[name], args, dev, rank, world, headline=False)
+            del r["inp"]
+            torch.cuda.empty_cache()
+            extras[name] = config_summary(r, measured_peaks())
+
+    if rank != 0:
+        if world > 1:
+            dist.destroy_process_group()
+        return
+
+    peaks = measured_peaks()
+    lr = layer_roofline(w, head["kept"], head["touched"], head["ms_step"], peaks)
+    roof = gemm_roofline(head, peaks)
+    roof["traffic"] = committed_traffic(w, head["kept"] + w.S * w.T)
 
     line = {
-        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K, "warmup": args.warmup,
-        "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": w.dtype, "data": "synthetic (seeded; x ~ N(0,1), weights ~ N(0,1/fan_in))",
-        "config": {"workload": w.name, "T": T, "d": w.d, "d_ff": w.F, "out": w.O, "E": w.E, "k": w.k, "S": w.S,
+        "metric": METRIC, "value": head["value"], "unit": UNIT, "n_gpus": world, "steps": head["K"],
+        "warmup": args.warmup, "ms_per_step": head["ms_step"], "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": w.dtype, "data": "synthetic (seeded; x ~ N(0,1), weights ~ N(0,1/fan_in))",
+        "config": {"workload": w.name, "T": w.T, "d": w.d, "d_ff": w.F, "out": w.O, "E": w.E, "k": w.k, "S": w.S,
                    "activation": w.activation, "capacity_factor": w.capacity_factor,
-                   "tokens_per_rank": T, "parallelism": f"replicas x{world}",
-                   "l2": l2_note(w)},
-        "expert_gemm_tflops": step_tflops,
-        "layer_roofline_frac": layer_frac,
-        "layer_roofline_frac_burst_peak": layer_frac_burst,
-        "roofline": {"kernel": "grouped_gemm_pair (expert GEMM 1 + 2)", "bound": "tensor", "achieved": achieved,
-                     "peak": peaks["bf16_sustained"], "unit": "TFLOP/s", "frac": achieved / peaks["bf16_sustained"],
-                     "peak_kind": f"bf16 sustained ({peaks['source']})", "traffic": traffic},
-        "stage_ms": {n: statistics.mean(v) for n, v in stage.items()},
+                   "tokens_per_rank": w.T, "parallelism": f"replicas x{world}", "l2": l2_note(w)},
+        "expert_gemm_tflops": lr["expert_gemm_tflops"],
+        "layer_roofline_frac": lr["layer_roofline_frac"],
+        "layer_roofline_frac_sustained": lr["layer_roofline_frac_sustained"],
+        "layer_bound": lr["bound"],
+        "roofline": roof,
+        "stage_ms": head["stage"],
         "launch": "cuda_graph (one graph per step); stage_ms from an instrumented eager loop",
-        "ms_per_step_eager": ms_eager / K,
-        "kept_rows": kept, "n_dropped": int(out["n_dropped"].item()),
-        "gpu_launches": launches_per_step * K,
-        "e2e": e2e, "cpu_baseline": cpu, "clocks": clk,
+        "ms_per_step_eager": head["ms_eager"],
+        "kept_rows": head["kept"], "n_dropped": head["n_dropped"],
+        "gpu_launches": head["launches_per_step"] * head["K"],
+        "e2e": head["e2e"], "cpu_baseline": cpu, "clocks": head["clocks"],
+        "peaks": {k: peaks[k] for k in ("bf16", "bf16_sustained", "hbm_gbs", "source")},
     }
+    if extras:
+        line["configs"] = extras
     print(json.dumps(line), flush=True)
     if world > 1:
         dist.destroy_process_group()
@@ -412,12 +496,15 @@ def l2_note(w):
                else "inputs fit in L2 (126 MB): a 256 MB write before every timed step, outside its events"))
 
 
-def committed_traffic(w):
-    """DRAM bytes per expert-GEMM launch pair from the committed ncu summary, if
-    the kernel source has not changed since it was captured."""
+def committed_traffic(w, rows):
+    """DRAM bytes per expert-GEMM launch pair for workload `w` with `rows` kept
+    plus shared rows, from the committed ncu summary of a scaled case of the same
+    per-expert shape (fewer experts and tokens, a few GB on the device), scaled
+    by the rows processed. None when the kernel source changed since the capture
+    or the workload was resized on the command line."""
     import hashlib
     from sparse_mixture_experts_gate_b200.workloads import WORKLOADS
-    if WORKLOADS.get(w.name) != w:  # a resized workload (--tokens / --experts): not the captured one
+    if WORKLOADS.get(w.name) != w:
         return None
     path = os.path.join(ROOT, "profiles", f"grouped_gemm_pair_{w.name}_traffic.txt")
     src = os.path.join(ROOT, "sparse_mixture_experts_gate_b200", "csrc", "gemm_pair.cu")
@@ -432,8 +519,8 @@ def committed_traffic(w):
     if vals.get("kernel_source_sha256") != sha:
         return None
     try:
-        return float(vals["dram_bytes_per_launch_pair"])
-    except (KeyError, ValueError):
+        return float(vals["dram_bytes_per_launch_pair"]) * rows / float(vals["capture_rows"])
+    except (KeyError, ValueError, ZeroDivisionError):
         return None
 
 
@@ -497,8 +584,26 @@ def run_reference(args):
     print(json.dumps(line), flush=True)
 
 
+def torchrun_argv(argv, n: int, port: int, limit_s: int = 1800):
+    """The command that runs this script as n ranks of one node (one process
+    per GPU, rendezvous on 127.0.0.1), bounded from outside by `timeout`."""
+    return ["timeout", "-k", "60", str(limit_s), sys.executable, "-m", "torch.distributed.run", "--nnodes=1",
+            f"--nproc-per-node={n}", "--master-addr=127.0.0.1", f"--master-port={port}",
+            os.path.join(ROOT, "bench.py")] + list(argv)
+
+
+def free_port() -> int:
+    import socket
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
 def main():
     args = parse()
+    if args.gpus > 1 and "WORLD_SIZE" not in os.environ:
+        # Not started by a launcher: start the N ranks here; rank 0 prints the line.
+        sys.exit(subprocess.call(torchrun_argv(sys.argv[1:], args.gpus, free_port())))
     if args.impl == "reference":
         run_reference(args)
     else:

@@ -24,8 +24,9 @@
  *   - Every call that can fail returns an int status (MOE_OK = 0, negative on
  *     error). Argument errors are detected on the host BEFORE anything is
  *     enqueued; moe_last_error() then returns a message naming the bad argument.
- *   - The library never allocates device memory: scratch comes from the
- *     caller's workspace.
+ *   - The library never allocates device memory at run time: scratch comes
+ *     from the caller's workspace or, for moe_forward_noalloc only, from the
+ *     fixed built-in device array documented at that declaration.
  *   - NaN or Inf inputs are not supported: outputs are then unspecified, but no
  *     kernel faults or waits forever.
  */
@@ -183,8 +184,10 @@ typedef struct {
  *   cv_load     [1] fp32  squared coefficient of variation of count_pre
  *               (population variance / mean^2; 0 for a zero mean)
  *   cv_importance [1] fp32 the same for importance
- *   l_total     [1] fp32  l_aux + l_z (the weighted sum of the balance and
- *               z-losses with load_balance_coef and z_loss_coef) */
+ *   l_total     [1] fp32  the walkthrough's weighted aux_loss: load_balance_coef
+ *               * cv_load + l_z ("Load balancing": load_balance_coef * load_balance
+ *               + z_loss_coef * z_loss, load_balance being the coefficient-of-
+ *               variation style balance loss; l_z already carries z_loss_coef) */
 typedef struct {
     float *f;
     float *p_mean;
@@ -244,7 +247,10 @@ MOE_API int moe_forward(moe_layer_t *layer, const void *x, int32_t T, const floa
  *     with MOE_ERR_WORKSPACE and nothing is enqueued (at the default SER shape,
  *     512/1024/512 with 8 experts and 2 active, T = 4096 fits).
  *   - The first call on a device looks up the array's device address (with that
- *     device current); make that first call before any stream capture.
+ *     device current); make that first call before any stream capture. The
+ *     address is cached for the life of the process: after cudaDeviceReset (or
+ *     anything else that destroys and re-creates the device's primary context)
+ *     the cache is stale and this call must not be used on that device again.
  *   - All calls, on every layer and stream, share the one array and it keeps
  *     the previous call's contents. The forward re-initialises everything it
  *     reads (its control words are cleared at the start), but two calls whose
@@ -364,13 +370,15 @@ MOE_API int moe_device_status(moe_layer_t *layer, void *stream);
 /* Optional stage timing with caller-owned CUDA events (cudaEvent_t passed as
  * void*, created with timing enabled). After this call every moe_forward records
  *   events[0] before the router,        events[1] after the router,
- *   events[2] after the dispatch,       events[3] after expert GEMM 1 (and
- *                                       the row gather that feeds it),
- *   events[4] after expert GEMM 2,      events[5] after the combine,
- * and every moe_aux_stats records events[6] after its kernels, all on the
+ *   events[2] after the dispatch,       events[3] after the row scatter that
+ *                                       feeds expert GEMM 1 (fp32 layers have
+ *                                       none: events[3] follows events[2]),
+ *   events[4] after expert GEMM 1,      events[5] after expert GEMM 2,
+ *   events[6] after the combine,
+ * and every moe_aux_stats records events[7] after its kernels, all on the
  * call's stream. The array is copied; events == NULL turns timing off. Nothing
  * is allocated and nothing synchronises. */
-#define MOE_TIMING_EVENTS 7
+#define MOE_TIMING_EVENTS 8
 MOE_API int moe_set_timing_events(moe_layer_t *layer, void *const *events);
 
 /* Number of kernels the most recent moe_forward plus moe_aux_stats enqueued. */

@@ -69,6 +69,8 @@ def _configure(L):
     L.orc_dro_update.restype = dbl
     L.orc_cv_squared.argtypes = [i32, vp]
     L.orc_cv_squared.restype = dbl
+    L.orc_aux_loss.argtypes = [i32, i32, vp, vp, dbl, dbl]
+    L.orc_aux_loss.restype = dbl
     L.orc_selection_bias_update.argtypes = [i32, i32, i64, vp, ctypes.c_float, vp]
     L.orc_max_threads.restype = i32
     return L
@@ -334,6 +336,16 @@ def cv_squared(v) -> float:
     return float(lib().orc_cv_squared(int(v.size), _p(v)))
 
 
+def aux_loss(count_pre, lse, load_balance_coef: float, z_loss_coef: float) -> float:
+    """The walkthrough's aux_loss ("Load balancing"): load_balance_coef times the
+    coefficient-of-variation style balance loss of the selection counts, plus
+    z_loss_coef times the mean squared log-partition."""
+    cpre = np.ascontiguousarray(count_pre, dtype=np.int32)
+    lse = np.ascontiguousarray(lse, dtype=np.float64)
+    return float(lib().orc_aux_loss(int(lse.size), int(cpre.size), _p(cpre), _p(lse), float(load_balance_coef),
+                                    float(z_loss_coef)))
+
+
 def selection_bias_update(b, load, k: int, T: int, gamma: float) -> np.ndarray:
     """b_i + gamma sign(kT/E - load_i), rounded to fp32 ("Balancing")."""
     out = np.ascontiguousarray(np.array(b, dtype=np.float32).copy())
@@ -393,7 +405,7 @@ def forward(w, inp: Dict[str, object], tokens: Optional[Sequence[int]] = None,
     out.update(h32=h32, key=key, idx=idx, gates=g, C=C, slot=slot, count_pre=cpre,
                count_kept=ckept, n_dropped=nd)
     f, pm, la, lz = balance_stats(P, lse, cpre, w.k, w.alpha, w.beta)
-    out.update(f=f, p_mean=pm, l_aux=la, l_z=lz)
+    out.update(f=f, p_mean=pm, l_aux=la, l_z=lz, aux_loss=aux_loss(cpre, lse, w.alpha, w.beta))
     r_idx, r_slot, r_g = idx, slot, g
     if routing is not None:
         r_idx, r_slot, r_g = routing["idx"], routing["slot"], routing["gates"]

@@ -397,6 +397,24 @@ double orc_cv_squared(int n, const double *v)
     return var / (mean * mean);
 }
 
+/* Load balancing: aux_loss = load_balance_coef * (CV^2 of the selection counts)
+ * + z_loss_coef * mean_t lse_t^2. */
+double orc_aux_loss(int T, int E, const int32_t *count_pre, const double *lse, double load_balance_coef,
+                    double z_loss_coef)
+{
+    double *load = (double *)malloc(sizeof(double) * (size_t)E);
+    for (int i = 0; i < E; ++i)
+        load[i] = (double)count_pre[i];
+    const double balance = orc_cv_squared(E, load);
+    free(load);
+    double z = 0.0;
+    for (int t = 0; t < T; ++t) {
+        const double v = lse[t];
+        z += v * v;
+    }
+    return load_balance_coef * balance + z_loss_coef * (z / (double)T);
+}
+
 /* Balancing: b_i <- b_i + gamma sign(kT/E - load_i), rounded to fp32. */
 void orc_selection_bias_update(int E, int k, int64_t T, const int64_t *load, float gamma, float *b)
 {

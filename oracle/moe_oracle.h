@@ -171,6 +171,15 @@ void orc_importance(int T, int E, int k, const int32_t *idx, const double *g, do
  * over the squared mean (0 when the mean is 0). */
 double orc_cv_squared(int n, const double *v);
 
+/* [W] "Load balancing": the weighted combination the walkthrough's aux_loss
+ * returns, load_balance_coef * load_balance + z_loss_coef * z_loss. Its
+ * load_balance term is the walkthrough's coefficient-of-variation style balance
+ * loss (the squared coefficient of variation of the per-expert selection counts
+ * before capacity, as orc_cv_squared), its z_loss term the mean over tokens of
+ * the squared log-partition. count_pre [E], lse [T]. */
+double orc_aux_loss(int T, int E, const int32_t *count_pre, const double *lse, double load_balance_coef,
+                    double z_loss_coef);
+
 /* [C] "Balancing": per-expert selection bias b_i (aux-loss-free balancing) with
  * update rate gamma: b_i <- b_i + gamma * sign(mean load - load_i), load_i =
  * selections of expert i before capacity, mean load = k T / E (the sign is

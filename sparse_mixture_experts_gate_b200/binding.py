@@ -220,8 +220,8 @@ def moe_device_status(layer: int, stream: int) -> int:
     return int(lib().moe_device_status(layer, stream))
 
 
-MOE_TIMING_EVENTS = 7
-STAGES = ("router", "dispatch", "gemm1", "gemm2", "combine", "stats")
+MOE_TIMING_EVENTS = 8
+STAGES = ("router", "dispatch", "scatter", "gemm1", "gemm2", "combine", "stats")
 
 
 def moe_set_timing_events(layer: int, events) -> int:

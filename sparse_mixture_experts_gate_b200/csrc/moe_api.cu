@@ -532,6 +532,7 @@ int fwd_route(moe_layer_t *L, const void *x, int32_t T, const float *logit_noise
         sa.row_bytes = c.input_dim * 2;
         MOE_LAUNCH(launch_scatter(sa, L->num_sms, s, nl));
     }
+    MOE_MARK(L, 3, s);
     return MOE_OK;
 }
 
@@ -599,9 +600,9 @@ int fwd_expert_gemms(moe_layer_t *L, cudaStream_t s, bool shared_only) {
             !encode_bf16_store(&m_os, ws + p.o_o, c.output_dim, p.R_max))
             return fail(MOE_ERR_CUDA, "cuTensorMapEncodeTiled failed for the activations");
         MOE_LAUNCH(launch_gemm_pair(L->map_w1, m_xp, m_xp16, m_x, m_x16, m_hs, g1, s, nl));
-        MOE_MARK(L, 3, s);
-        MOE_LAUNCH(launch_gemm_pair(L->map_w2, m_h, m_h16, m_h, m_h16, m_os, g2, s, nl));
         MOE_MARK(L, 4, s);
+        MOE_LAUNCH(launch_gemm_pair(L->map_w2, m_h, m_h16, m_h, m_h16, m_os, g2, s, nl));
+        MOE_MARK(L, 5, s);
     } else {
         GemmSimtArgs s1;
         s1.block_group = da.block_group;
@@ -621,7 +622,7 @@ int fwd_expert_gemms(moe_layer_t *L, cudaStream_t s, bool shared_only) {
         s1.gather = 1;
         s1.w = static_cast<const float *>(L->w.w1);
         MOE_LAUNCH(launch_gemm_simt(s1, s, nl));
-        MOE_MARK(L, 3, s);
+        MOE_MARK(L, 4, s);
         GemmSimtArgs s2 = s1;
         s2.N = c.output_dim;
         s2.K = c.expert_dim;
@@ -632,7 +633,7 @@ int fwd_expert_gemms(moe_layer_t *L, cudaStream_t s, bool shared_only) {
         s2.gather = 0;
         s2.w = static_cast<const float *>(L->w.w2);
         MOE_LAUNCH(launch_gemm_simt(s2, s, nl));
-        MOE_MARK(L, 4, s);
+        MOE_MARK(L, 5, s);
     }
 
     return MOE_OK;
@@ -680,7 +681,7 @@ int fwd_combine(moe_layer_t *L, void *y, cudaStream_t s) {
     ca.y = y;
     ca.credit = reinterpret_cast<float *>(ws + p.o_credit);
     MOE_LAUNCH(launch_combine(ca, L->num_sms, s, nl));
-    MOE_MARK(L, 5, s);
+    MOE_MARK(L, 6, s);
     return MOE_OK;
 }
 
@@ -915,7 +916,7 @@ int moe_aux_stats(moe_layer_t *L, const float *token_loss, const moe_stats_t *ou
     if (out->credit)
         MOE_LAUNCH(cudaMemcpyAsync(out->credit, L->ws + p.o_credit, (size_t)p.T * c.num_active * 4,
                                    cudaMemcpyDeviceToDevice, s));
-    MOE_MARK(L, 6, s);
+    MOE_MARK(L, 7, s);
     return MOE_OK;
 }
 

@@ -99,7 +99,10 @@ __device__ __forceinline__ float block_cv_squared(float v, bool valid, int n, fl
 // Statistics from (possibly all-reduced) partial sums: f_i = count_i / (k T),
 // P_i = sum_t P / T, L_aux = alpha E sum_i f_i P_i, L_z = beta sum lse^2 / T,
 // l_i = sum credit * loss / T, importance_i, the squared coefficients of
-// variation of the loads and of the importances, and L_aux + L_z. One CTA of
+// variation of the loads and of the importances, and the weighted aux loss
+// alpha CV^2(loads) + L_z ("Code Walkthrough - SER", "Load balancing": aux_loss
+// = load_balance_coef * load_balance + z_loss_coef * z_loss, load_balance
+// being the coefficient-of-variation style loss of the loads). One CTA of
 // 256 threads (E <= 256), thread e owns expert e; every sum is a fixed tree.
 __global__ void __launch_bounds__(256) stats_finalize_kernel(FinalizeArgs a) {
     __shared__ float red[8];
@@ -127,7 +130,7 @@ __global__ void __launch_bounds__(256) stats_finalize_kernel(FinalizeArgs a) {
         const float l_z = a.beta * a.partials[2 * a.E] * inv_t;
         if (a.l_aux) *a.l_aux = l_aux;
         if (a.l_z) *a.l_z = l_z;
-        if (a.l_total) *a.l_total = l_aux + l_z;
+        if (a.l_total) *a.l_total = a.alpha * cv_load + l_z;
         if (a.n_dropped) *a.n_dropped = (int32_t)a.partials[2 * a.E + 2];
         if (a.cv_load) *a.cv_load = cv_load;
         if (a.cv_importance) *a.cv_importance = cv_imp;

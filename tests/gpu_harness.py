@@ -18,7 +18,9 @@ Tolerances (bf16 operands with fp32 accumulation, fp32 routing and statistics):
     CPU recomputation with the hidden vector rounded to bf16 matches the GPU
     credit to ~1e-5 relative. 2e-3 is that unit roundoff, ten times tighter than
     the 2e-2 (1 + |y|) bound on the bf16-operand outputs themselves;
-  * expert-attributed loss, reduced from the GPU's own credit: 1e-4 (1 + |value|).
+  * expert-attributed loss: reduced from the GPU's own credit, 1e-4 (1 + |value|);
+    against the oracle's own l_i (from the oracle's credit on the same routing),
+    the credit bound carried through the sum (check_expert_loss_vs_oracle).
 """
 from __future__ import annotations
 
@@ -92,14 +94,15 @@ def check_same_logits_routing(w, inp, g):
     assert abs(g["l_aux"][0] - la) <= STAT_TOL
     assert abs(g["l_z"][0] - lz) <= STAT_TOL
     # Load-balancing extras: importance from the GPU's own gates (fp32 sums of
-    # fp32 gates), the CVs of counts and importances, the weighted total.
+    # fp32 gates), the CVs of counts and importances, the weighted aux loss.
     imp = oracle.importance(g["topk_idx"], g["gates"], w.E)
     assert np.abs(g["importance"] - imp).max() <= STAT_TOL * (1 + np.abs(imp).max()), "importance"
     cvl = oracle.cv_squared(r["count_pre"])
     assert abs(g["cv_load"][0] - cvl) <= STAT_TOL * (1 + cvl), "cv of the loads"
     cvi = oracle.cv_squared(imp)
     assert abs(g["cv_importance"][0] - cvi) <= STAT_TOL * (1 + cvi), "cv of the importances"
-    assert np.float32(g["l_total"][0]) == np.float32(np.float32(g["l_aux"][0]) + np.float32(g["l_z"][0]))
+    lt = oracle.aux_loss(r["count_pre"], r["lse"], w.alpha, w.beta)
+    assert abs(g["l_total"][0] - lt) <= STAT_TOL * (1 + abs(lt)), "weighted aux loss"
     return r
 
 
@@ -147,7 +150,27 @@ def check_end_to_end(w, inp, g, tokens=None, table=None):
                                               w.d, w.F, w.E, w.activation)
     cerr = np.abs(g["credit"][toks] - credit) / (1.0 + np.abs(credit))
     assert cerr.max() <= CREDIT_TOL[w.dtype], f"credit: max scaled error {cerr.max():.3e}"
-    return dict(n_near_ties=int(ties.sum()), y_err=float(err.max()), credit_err=float(cerr.max()))
+    info = dict(n_near_ties=int(ties.sum()), y_err=float(err.max()), credit_err=float(cerr.max()))
+    if tokens is None and inp.get("token_loss") is not None:
+        info["expert_loss_err"] = check_expert_loss_vs_oracle(w, inp, g, credit)
+    return info
+
+
+def check_expert_loss_vs_oracle(w, inp, g, credit_oracle):
+    """The GPU's expert-attributed loss against the oracle's own l_i, built from
+    the oracle's credit on the same routing. The bound follows from the credit
+    bound: l_i = (1/T) sum c l_t over i's kept assignments, so each credit's
+    error CREDIT_TOL (1 + |c|) enters weighted by its token loss; the fp32 sum
+    itself adds STAT_TOL (1 + |l_i|)."""
+    tl = inp["token_loss"].cpu().double().numpy()
+    T = tl.shape[0]
+    el = oracle.expert_loss(g["topk_idx"], g["slot"], credit_oracle, inp["token_loss"].cpu(), w.E)
+    kept = g["slot"] >= 0
+    per = np.where(kept, CREDIT_TOL[w.dtype] * (1.0 + np.abs(credit_oracle)) * tl[:, None], 0.0)
+    bound = np.bincount(g["topk_idx"][kept], weights=per[kept], minlength=w.E) / T + STAT_TOL * (1 + np.abs(el))
+    diff = np.abs(g["expert_loss"] - el)
+    assert (diff <= bound).all(), f"expert loss: max error {diff.max():.3e}, worst margin {(diff - bound).max():.3e}"
+    return float((diff / bound).max())
 
 
 def check_expert_loss(w, inp, g):
@@ -155,3 +178,61 @@ def check_expert_loss(w, inp, g):
     el = oracle.expert_loss(g["topk_idx"], g["slot"], g["credit"], inp["token_loss"].cpu(), w.E)
     err = np.abs(g["expert_loss"] - el) / (1.0 + np.abs(el))
     assert err.max() <= STAT_TOL, err.max()
+
+
+def stratified_tokens(g, w, tile_rows: int, min_tokens: int = 0, seed: int = 1234, candidates: int = 32):
+    """A sample of tokens that together reach every unit of work the expert
+    GEMMs hand out: for every routed expert, a token in each of its token tiles
+    (slots [j tile_rows, (j + 1) tile_rows) of its segment) and the token in its
+    last kept slot; for every shared expert, a token in each tile of the token
+    axis; and the batch's last token. A token covers its k experts' tiles at
+    once, so the items are covered greedily (for each uncovered item, the
+    candidate token that covers most uncovered items), then random tokens are
+    added up to `min_tokens`. Every output column of a sampled token is compared,
+    so every feature tile of both GEMMs is reached for each of those tiles."""
+    rng = np.random.default_rng(seed)
+    idx, slot = g["topk_idx"], g["slot"]
+    T, k = idx.shape
+    kept = g["count_kept"].astype(np.int64)
+    n_tiles = (kept + tile_rows - 1) // tile_rows
+    base = np.concatenate([[0], np.cumsum(n_tiles)])
+    n_routed = int(base[-1])
+    n_last = int((kept > 0).sum())
+    last_id = np.full(w.E, -1, np.int64)
+    last_id[kept > 0] = n_routed + np.arange(n_last)
+    n_shared_tiles = (T + tile_rows - 1) // tile_rows if w.S > 0 else 0
+    cover = [set() for _ in range(T)]
+    holders = {}
+    for t in range(T):
+        for r in range(k):
+            s_ = int(slot[t, r])
+            if s_ < 0:
+                continue
+            e = int(idx[t, r])
+            items = [int(base[e] + s_ // tile_rows)]
+            if s_ == kept[e] - 1:
+                items.append(int(last_id[e]))
+            for it in items:
+                cover[t].add(it)
+                holders.setdefault(it, []).append(t)
+        if n_shared_tiles:
+            it = n_routed + n_last + t // tile_rows
+            cover[t].add(it)
+            holders.setdefault(it, []).append(t)
+    uncovered = set(holders)
+    chosen = {T - 1}
+    uncovered -= cover[T - 1]
+    for it in sorted(holders):
+        if it not in uncovered:
+            continue
+        hs = holders[it]
+        cands = hs if len(hs) <= candidates else [hs[i] for i in rng.choice(len(hs), candidates, replace=False)]
+        best = max(cands, key=lambda t: len(cover[t] & uncovered))
+        chosen.add(best)
+        uncovered -= cover[best]
+    assert not uncovered
+    n_items = n_routed + n_last + n_shared_tiles
+    if len(chosen) < min_tokens:
+        rest = np.setdiff1d(np.arange(T), np.fromiter(chosen, np.int64))
+        chosen.update(rng.choice(rest, min(len(rest), min_tokens - len(chosen)), replace=False).tolist())
+    return np.array(sorted(chosen), np.int64), n_items

@@ -419,6 +419,34 @@ def check_cv_squared():
     assert oracle.cv_squared([0.0, 0.0, 0.0]) == 0.0
 
 
+def check_aux_loss():
+    """[W] "Load balancing": aux_loss = load_balance_coef * load_balance +
+    z_loss_coef * z_loss, load_balance the coefficient-of-variation style loss of
+    the selection counts. Closed forms: uniform routing (W_g = 0, k = E) leaves
+    only beta (log E)^2; with z_loss_coef = 0, m equal non-zero loads of n give
+    alpha (n/m - 1) and two loads a, b give alpha ((a - b) / (a + b))^2; a
+    hand-worked log-partition vector; the value ignores the order of the experts."""
+    w = WORKLOADS["tiny"].with_(T=12, d=8, F=8, O=8, E=4, k=4, S=0, dtype="fp32", capacity_factor=0.0)
+    inp = make_inputs(w, "cpu", seed=3)
+    inp["w_gate"] = torch.zeros_like(inp["w_gate"])
+    inp["b_gate"] = None
+    out = oracle.forward(w, inp)
+    assert abs(oracle.aux_loss(out["count_pre"], out["lse"], 0.01, 1e-3) - 1e-3 * math.log(4) ** 2) <= 1e-15
+    lse0 = np.zeros(5)
+    for n, m in ((4, 1), (8, 3), (256, 8)):
+        load = [9] * m + [0] * (n - m)
+        assert abs(oracle.aux_loss(load, lse0, 0.25, 7.0) - 0.25 * (n / m - 1)) <= 1e-12 * (n / m)
+    assert abs(oracle.aux_loss([3, 11], lse0, 0.5, 7.0) - 0.5 * (8 / 14) ** 2) <= 1e-15
+    # lse = 1, 2, 3: mean square 14/3; equal loads: no balance term.
+    assert abs(oracle.aux_loss([5, 5], [1.0, 2.0, 3.0], 0.5, 0.3) - 0.3 * 14 / 3) <= 1e-15
+    rng = np.random.default_rng(12)
+    load = rng.integers(0, 50, 16)
+    lse = rng.normal(size=30)
+    a = oracle.aux_loss(load, lse, 0.01, 1e-3)
+    assert a == oracle.aux_loss(load[::-1].copy(), lse, 0.01, 1e-3)
+    assert abs(oracle.aux_loss(load, lse, 0.01, 0.0) - 0.01 * oracle.cv_squared(load)) <= 1e-15
+
+
 def check_importance():
     """[W] "Load balancing" (importance per expert): with k = 1 every gate is 1,
     so the importance is the selection count; the importances of a batch sum to

@@ -26,6 +26,14 @@ def test_header_declares_the_binding_exports():
     assert declared_symbols() == sorted(binding.EXPORTS)
 
 
+def test_header_constants_match_the_binding():
+    src = open(os.path.join(ROOT, "include", "moe.h")).read()
+    ev = int(re.search(r"#define MOE_TIMING_EVENTS (\d+)", src).group(1))
+    assert ev == binding.MOE_TIMING_EVENTS == len(binding.STAGES) + 1
+    m = re.search(r"#define MOE_NOALLOC_SCRATCH_BYTES \((\d+)u \* (\d+)u \* (\d+)u\)", src)
+    assert int(m.group(1)) * int(m.group(2)) * int(m.group(3)) == binding.MOE_NOALLOC_SCRATCH_BYTES
+
+
 def test_library_exports_every_declared_symbol(L):
     for name in declared_symbols():
         assert hasattr(L, name), name

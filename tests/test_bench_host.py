@@ -1,6 +1,7 @@
 """bench.py's host side on CPU: the reference arm's JSON line (the CPU oracle
-timed on a small workload), its silence on ranks other than 0, and the
-parsing of the nvidia-smi clock samples that accompany every timed run."""
+timed on a small workload), its silence on ranks other than 0, the N-rank
+launch that `--gpus N` starts by itself, and the parsing of the nvidia-smi
+clock samples that accompany every timed run."""
 import json
 import os
 import subprocess
@@ -57,3 +58,26 @@ def test_clock_rows_summary():
         ["1200, 1965, 700, 0x8, Active, Not Active, Active, Not Active\n"])
     assert hot["reasons"] == ["hw_slowdown", "sw_thermal_slowdown"]
     assert bench.summarize_clock_rows([]) is None
+
+
+def test_torchrun_command_for_n_ranks():
+    argv = bench.torchrun_argv(["--gpus", "4", "--steps", "3"], 4, 29555, limit_s=600)
+    assert argv[:4] == ["timeout", "-k", "60", "600"]
+    i = argv.index("torch.distributed.run")
+    assert argv[i - 1] == "-m" and "--nnodes=1" in argv and "--nproc-per-node=4" in argv
+    assert "--master-addr=127.0.0.1" in argv and "--master-port=29555" in argv
+    assert argv[-4:] == ["--gpus", "4", "--steps", "3"] and argv[-5].endswith("bench.py")
+
+
+def test_gpus_flag_starts_that_many_ranks():
+    """`bench.py --gpus 2` without a launcher starts two ranks (here the CPU
+    reference arm, which rank 0 alone runs): one JSON line, n_gpus = 2."""
+    e = {k: v for k, v in os.environ.items() if k not in ("WORLD_SIZE", "RANK", "LOCAL_RANK")}
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--gpus", "2", "--impl", "reference",
+                        "--workload", "tiny", "--steps", "1", "--warmup", "1"], capture_output=True, text=True,
+                       timeout=600, env=e, cwd=ROOT)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [l for l in r.stdout.splitlines() if l.strip().startswith("{")]
+    assert len(lines) == 1, r.stdout
+    d = json.loads(lines[0])
+    assert d["impl"] == "reference" and d["n_gpus"] == 2

@@ -64,7 +64,8 @@ def stats_from_partials(p: np.ndarray, E: int, k: int, alpha: float, beta: float
     import oracle
     l_aux, l_z = alpha * E * float((f * pm).sum()), beta * p[2 * E] / T
     imp = p[3 * E + 3:]
-    return dict(f=f, p_mean=pm, l_aux=l_aux, l_z=l_z, l_total=l_aux + l_z, n_dropped=int(p[2 * E + 2]),
+    return dict(f=f, p_mean=pm, l_aux=l_aux, l_z=l_z, l_total=alpha * oracle.cv_squared(p[E:2 * E]) + l_z,
+                n_dropped=int(p[2 * E + 2]),
                 expert_loss=p[2 * E + 3:3 * E + 3] / T, importance=imp,
                 cv_load=oracle.cv_squared(p[E:2 * E]), cv_importance=oracle.cv_squared(imp))
 
@@ -113,6 +114,7 @@ def test_dp_stats_two_gloo_ranks(tmp_path):
     assert np.allclose(dp["importance"], imp_whole, rtol=1e-12, atol=1e-12)
     assert abs(dp["cv_load"] - oracle.cv_squared(whole["count_pre"])) <= 1e-12
     assert abs(dp["cv_importance"] - oracle.cv_squared(imp_whole)) <= 1e-12
+    assert abs(dp["l_total"] - whole["aux_loss"]) <= 1e-12
     # Capacity is per shard, so drops and the attributed loss follow each
     # shard's own dispatch, divided by the whole batch's size.
     cuts = _bounds(w.T, WORLD)
@@ -144,5 +146,6 @@ def test_stats_from_partials_matches_unsharded_oracle_on_one_shard():
     dp = stats_from_partials(p, w.E, w.k, w.alpha, w.beta)
     assert np.allclose(dp["f"], o["f"], atol=1e-12) and np.allclose(dp["p_mean"], o["p_mean"], atol=1e-12)
     assert abs(dp["l_aux"] - o["l_aux"]) <= 1e-12 and abs(dp["l_z"] - o["l_z"]) <= 1e-12
+    assert abs(dp["l_total"] - o["aux_loss"]) <= 1e-12
     assert np.allclose(dp["expert_loss"], o["expert_loss"], atol=1e-12)
     assert dp["n_dropped"] == o["n_dropped"]

@@ -54,6 +54,11 @@ MUTANTS = {
                                "    for (int t = 0; t < T; ++t) {\n        for (int r = 0; r < k; ++r) {\n            int e = idx[(int64_t)t * k + r];"),
     "mlp_no_relu": ("z[u] = s > 0.0 ? s : 0.0;", "z[u] = s;"),
     "mlp_drops_b1": ("                s += (double)b1[u];", "                s += 0.0;"),
+    "aux_loss_coefs_swapped": ("return load_balance_coef * balance + z_loss_coef * (z / (double)T);",
+                               "return z_loss_coef * balance + load_balance_coef * (z / (double)T);"),
+    "aux_loss_z_not_mean": ("return load_balance_coef * balance + z_loss_coef * (z / (double)T);",
+                            "return load_balance_coef * balance + z_loss_coef * z;"),
+    "aux_loss_lse_not_squared": ("z += v * v;", "z += v;"),
     "softmax_wrong_exponent": ("P[(int64_t)t * E + i] = exp(ht[i] - m) / z;",
                                "P[(int64_t)t * E + i] = exp(ht[i]) / z;"),
 }

@@ -5,7 +5,7 @@ import torch
 
 import oracle
 from gpu_harness import (check_end_to_end, check_expert_loss, check_same_logits_routing, expert_table,
-                         run_gpu)
+                         run_gpu, stratified_tokens)
 from sparse_mixture_experts_gate_b200.binding import MoEError, MoELayer
 from sparse_mixture_experts_gate_b200.workloads import WORKLOADS, make_inputs
 
@@ -153,15 +153,18 @@ def test_forward_argument_errors_on_host():
 
 # ---------------------------------------------------------------- full sizes
 
-def _sampled_full(name, n_sample, seed=1234):
+def _sampled_full(name, min_tokens):
+    """The full-size workload in the launch configuration the benchmark times:
+    routing, dispatch and statistics over every token (same-logits mode); y and
+    credit on a stratified sample of tokens that reaches every token tile of
+    every expert (both GEMMs, every feature tile), the last kept row of every
+    expert, every shared-expert tile and the last token."""
     w = WORKLOADS[name]
     inp = make_inputs(w, "cuda")
     g, _ = run_gpu(w, inp, poison=False)
     check_same_logits_routing(w, {k: (v.cpu() if v is not None else None) for k, v in inp.items()
                                   if k in ("noise", "sel_bias")}, g)
-    rng = np.random.default_rng(seed)
-    toks = np.sort(rng.choice(w.T, size=n_sample, replace=False))
-    toks[-1] = w.T - 1  # always include the last token (ragged tail)
+    toks, n_items = stratified_tokens(g, w, tile_rows=256, min_tokens=min_tokens)
     experts = g["topk_idx"][toks].ravel()
     table = expert_table(w, inp, experts)
     info = check_end_to_end(w, inp, g, tokens=toks, table=table)
@@ -171,15 +174,16 @@ def _sampled_full(name, n_sample, seed=1234):
     assert int(g["count_kept"].sum()) == w.k * w.T - int(g["n_dropped"][0])
     assert int(g["count_pre"].sum()) == w.k * w.T
     assert np.allclose(g["gates"].sum(1), 1.0, atol=1e-5)
+    print(f"{name}: {len(toks)} sampled tokens cover {n_items} GEMM tiles and last rows; y_err {info['y_err']:.2e}")
     return g, info
 
 
 def test_e64_full_size_sampled():
-    _sampled_full("e64", 48)
+    _sampled_full("e64", 128)
 
 
 def test_e256_full_size_sampled():
-    _sampled_full("e256", 24)
+    _sampled_full("e256", 512)
 
 
 # ------------------------------------------------- data-parallel statistics
@@ -493,8 +497,8 @@ def test_nan_tokens_route_to_valid_experts():
     idx = g["topk_idx"]
     assert ((idx >= 0) & (idx < w.E)).all()
     assert all(len(set(r)) == w.k for r in idx.tolist())
-    for t in bad:
-        assert sorted(idx[t].tolist()) == list(range(w.k))
+    for t in bad:  # every key ties at -inf: the lowest indices, in ascending order
+        assert idx[t].tolist() == list(range(w.k))
     good = np.setdiff1d(np.arange(w.T), bad)
     assert np.isfinite(g["y"][good]).all()
 
@@ -510,3 +514,45 @@ def test_many_active_experts_k16(dtype, T):
                                    d=128 if dtype == "bf16" else 32, F=128 if dtype == "bf16" else 32,
                                    O=128 if dtype == "bf16" else 32, token_loss=True)
     full_check(w, make_inputs(w, "cpu", seed=91, random_biases=True))
+
+
+@pytest.mark.parametrize("E,d,mode", [(24, 256, "greedy"), (24, 256, "selection_bias"), (24, 256, "noisy"),
+                                      (160, 2048, "greedy")])
+def test_exact_ties_go_to_the_lower_index(E, d, mode):
+    """Finite keys that tie exactly: duplicated router rows give bit-identical
+    logits (same operands, same accumulation order, on the tensor cores too, in
+    different N tiles and K splits at E = 160, d = 2048), and equal selection
+    bias or equal noise keeps the keys equal. The top-k must list the same
+    experts in the same order as the oracle's (key descending, lower index
+    first on ties), both where a tie straddles the k-th place and where several
+    tied experts are all selected."""
+    w = WORKLOADS["default"].with_(T=700, E=E, k=4, S=0, d=d, F=256, O=256, capacity_factor=1.0,
+                                   top_k_method="noisy" if mode == "noisy" else "greedy",
+                                   use_selection_bias=mode == "selection_bias")
+    inp = make_inputs(w, "cpu", seed=37)
+    groups = [[3, 10, 17], [6, 21]] if E == 24 else [[5, 70, 150], [20, 140]]
+    wg = inp["w_gate"]
+    for grp in groups:
+        wg[grp[0]] *= 2.0  # selected often, so that ties decide many tokens
+        for e in grp[1:]:
+            wg[e] = wg[grp[0]]
+            if mode == "selection_bias":
+                inp["sel_bias"][e] = inp["sel_bias"][grp[0]]
+            if mode == "noisy":
+                inp["noise"][:, e] = inp["noise"][:, grp[0]]
+    g, _ = full_check(w, inp)
+    idx = g["topk_idx"]
+    straddle = together = 0
+    for grp in groups:
+        for e in grp[1:]:
+            assert np.array_equal(g["logits"][:, e], g["logits"][:, grp[0]]), "duplicated rows, different logits"
+        for t in range(w.T):
+            sel = [e for e in idx[t].tolist() if e in grp]
+            if 0 < len(sel) < len(grp):  # the tie straddles the k-th place: the lowest indices win
+                straddle += 1
+                assert sel == grp[:len(sel)], (t, sel, grp)
+            if len(sel) >= 2:  # tied experts listed next to each other, lower index first
+                together += 1
+                pos = [idx[t].tolist().index(e) for e in sel]
+                assert pos == list(range(pos[0], pos[0] + len(sel))), (t, idx[t])
+    assert straddle > 0 and together > 0, (straddle, together)

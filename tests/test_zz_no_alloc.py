@@ -4,14 +4,15 @@ moe_forward_noalloc is for callers that cannot allocate device memory
 themselves (a plugin whose host application owns all device memory through its
 own pool, or a loop that must not call cudaMalloc/cudaFree); it runs the same
 forward with the library's built-in 64 MiB device scratch instead of a caller
-workspace. These checks compare it with the workspace entry point on two calls
-in a row, and check that an oversized batch is refused on the host.
+workspace. Both entry points launch the same kernels on the same inputs, and
+those kernels are deterministic (every output has one fixed summation order),
+so the results must be identical bit for bit on each of two calls in a row.
+An oversized batch must be refused on the host.
 """
 import numpy as np
 import pytest
 import torch
 
-from gpu_harness import STAT_TOL, Y_TOL
 from sparse_mixture_experts_gate_b200 import binding
 from sparse_mixture_experts_gate_b200.binding import MoEError, MoELayer, MoeRouting
 from sparse_mixture_experts_gate_b200.workloads import WORKLOADS, make_inputs
@@ -49,12 +50,9 @@ def test_noalloc_matches_workspace_forward_on_two_calls():
         torch.cuda.synchronize()
         assert layer.device_status() == 0
         got = _host(out)
-        err = np.abs(got["y"] - ref["y"]) / (1.0 + np.abs(ref["y"]))
-        assert err.max() <= Y_TOL[w.dtype], (call, err.max())
-        for k in ("topk_idx", "slot", "count_pre", "count_kept", "n_dropped"):
+        for k in ("y", "topk_idx", "slot", "count_pre", "count_kept", "n_dropped", "logits", "gates", "f",
+                  "p_mean", "l_aux", "l_z", "credit", "importance", "cv_load", "cv_importance", "l_total"):
             assert np.array_equal(got[k], ref[k]), (call, k)
-        for k in ("logits", "gates", "f", "p_mean", "l_aux", "l_z", "credit"):
-            assert np.abs(got[k] - ref[k]).max() <= STAT_TOL, (call, k)
 
 
 def test_noalloc_refuses_a_batch_beyond_its_scratch():
