@@ -261,6 +261,21 @@ MOE_API int moe_forward(moe_layer_t *layer, const void *x, int32_t T, const floa
 MOE_API int moe_forward_noalloc(moe_layer_t *layer, const void *x, int32_t T, const float *logit_noise, void *y,
                                 const moe_routing_t *routing, void *stream);
 
+/* Router planes kept across forwards (bf16 layers; no counterpart on the pages).
+ * The tensor-core router reads the fp32 router matrix (w_gate, or the MLP gate's
+ * gater_w1) as three bf16 planes hi + mid + lo, [E_pad][3 d] bf16, and by default
+ * every forward splits it again into its workspace, one extra launch.
+ * moe_prepare_router splits it once, enqueued on `stream`, into `planes`
+ * (device, caller-owned, >= moe_router_planes_bytes(layer) bytes, 256-byte
+ * aligned, valid until it is replaced or the layer is destroyed), and every later
+ * forward of this layer reads the planes from there and does not split. The
+ * planes hold the matrix as it was when this call ran: after changing the router
+ * weights call it again. planes = NULL returns to splitting every forward.
+ * Errors: INVALID_ARG, UNSUPPORTED (fp32 layers), WORKSPACE (too small or
+ * misaligned), CUDA. moe_router_planes_bytes is 0 for fp32 layers or NULL. */
+MOE_API size_t moe_router_planes_bytes(const moe_layer_t *layer);
+MOE_API int moe_prepare_router(moe_layer_t *layer, void *planes, size_t bytes, void *stream);
+
 /* Balancing and credit statistics of the most recent moe_forward on this layer,
  * computed from what that forward left in its workspace (and routing buffers).
  *   token_loss [T] fp32 per-token losses l_t (NULL: expert_loss is not written)
@@ -362,6 +377,20 @@ MOE_API int moe_ep_combine(moe_layer_t *layer, void *y, void *stream);
  * designed (the context stays usable), MOE_ERR_INTERNAL if it was not,
  * MOE_ERR_CUDA on a CUDA error. Takes about two seconds. */
 MOE_API int moe_selftest_bounded_wait(void *stream);
+
+/* Self-check of the bounded waits inside the real expert GEMM (no counterpart on
+ * the pages): one moe_forward of this layer over x [T][d] (GREEDY top-k, bf16,
+ * ep_size 1, d >= 192) with workspace and y as for moe_forward, in which expert
+ * GEMM 1's leader CTAs announce the bytes of their third pipeline stage but load
+ * none of them, and every wait of that launch gives up after 20 ms. The MMA
+ * role's wait runs out, the kernel's roles stop, drain their copies and MMAs and
+ * free TMEM, the rest of the forward runs on the unfinished outputs (y is
+ * unspecified), and moe_device_status then reports MOE_ERR_TIMEOUT. Synchronises
+ * `stream`. Returns MOE_OK when the timeout was detected and reported, MOE_ERR_
+ * INTERNAL if it was not, the errors of moe_forward otherwise. The layer and
+ * context stay usable: the next moe_forward runs normally. */
+MOE_API int moe_selftest_gemm_timeout(moe_layer_t *layer, const void *x, int32_t T, void *workspace, size_t ws_bytes,
+                                      void *y, void *stream);
 
 /* Device status word of the most recent forward: synchronises `stream`, then
  * returns MOE_OK, or MOE_ERR_TIMEOUT if a bounded device-side wait gave up. */

@@ -24,7 +24,7 @@ MOE_PRIORITY = {"token": 0, "rank": 1}
 # Every symbol include/moe.h declares.
 EXPORTS = ("moe_config_default", "moe_layer_create", "moe_workspace_bytes", "moe_capacity", "moe_forward",
            "moe_forward_noalloc", "moe_aux_stats", "moe_stat_partials", "moe_stats_from_partials",
-           "moe_update_selection_bias", "moe_dro_update", "moe_selftest_bounded_wait",
+           "moe_update_selection_bias", "moe_dro_update", "moe_selftest_bounded_wait", "moe_selftest_gemm_timeout", "moe_router_planes_bytes", "moe_prepare_router",
            "moe_ep_dispatch", "moe_ep_layout", "moe_ep_experts_workspace_bytes", "moe_ep_experts", "moe_ep_combine", "moe_device_status", "moe_set_timing_events", "moe_launch_count", "moe_destroy", "moe_status_string",
            "moe_last_error")
 
@@ -109,6 +109,12 @@ def lib() -> ctypes.CDLL:
         L.moe_ep_combine.argtypes = [vp, vp, vp]
         L.moe_selftest_bounded_wait.restype = ctypes.c_int
         L.moe_selftest_bounded_wait.argtypes = [vp]
+        L.moe_router_planes_bytes.restype = sz
+        L.moe_router_planes_bytes.argtypes = [vp]
+        L.moe_prepare_router.restype = ctypes.c_int
+        L.moe_prepare_router.argtypes = [vp, vp, sz, vp]
+        L.moe_selftest_gemm_timeout.restype = ctypes.c_int
+        L.moe_selftest_gemm_timeout.argtypes = [vp, vp, i32, vp, sz, vp, vp]
         L.moe_device_status.restype = ctypes.c_int
         L.moe_device_status.argtypes = [vp, vp]
         L.moe_set_timing_events.restype = ctypes.c_int
@@ -216,6 +222,19 @@ def moe_selftest_bounded_wait(stream: int) -> int:
     return _check(lib().moe_selftest_bounded_wait(stream), "moe_selftest_bounded_wait")
 
 
+def moe_router_planes_bytes(layer: int) -> int:
+    return int(lib().moe_router_planes_bytes(layer))
+
+
+def moe_prepare_router(layer: int, planes: Optional[int], nbytes: int, stream: int) -> int:
+    return _check(lib().moe_prepare_router(layer, planes, nbytes, stream), "moe_prepare_router")
+
+
+def moe_selftest_gemm_timeout(layer: int, x: int, T: int, workspace: int, ws_bytes: int, y: int, stream: int) -> int:
+    return _check(lib().moe_selftest_gemm_timeout(layer, x, T, workspace, ws_bytes, y, stream),
+                  "moe_selftest_gemm_timeout")
+
+
 def moe_device_status(layer: int, stream: int) -> int:
     return int(lib().moe_device_status(layer, stream))
 
@@ -296,6 +315,19 @@ class MoELayer:
             self.close()
         except Exception:
             pass
+
+    def prepare_router(self, stream=None):
+        """Split the router matrix into bf16 planes once (moe_prepare_router) into
+        a buffer this object keeps; later forwards skip the per-forward split.
+        Call again after changing the router weights."""
+        import torch
+        n = moe_router_planes_bytes(self.handle)
+        if n == 0:
+            return
+        if getattr(self, "_planes", None) is None or self._planes.numel() < n:
+            self._planes = torch.empty(n, dtype=torch.uint8, device=self.device)
+        s = stream if stream is not None else torch.cuda.current_stream(self.device).cuda_stream
+        moe_prepare_router(self.handle, self._planes.data_ptr(), self._planes.numel(), s)
 
     def workspace(self, T: int):
         import torch

@@ -10,9 +10,10 @@
 // Instead of a dense one-hot D, the dispatch is a permutation into a compact row
 // space: expert e owns rows [group_start[e], group_start[e] + kept_e), padded to
 // a multiple of 32 rows, followed by one T-row segment per shared expert (also
-// padded to 32). Three launches:
+// padded to 32). Two launches (one block for a batch of one chunk):
 //   count  - per 256-token chunk, a histogram of selections (shared-memory
-//            integer atomics: order-free, so deterministic);
+//            integer atomics: order-free, so deterministic); the CTA that
+//            counts the last chunk then runs the scan:
 //   scan   - per expert, exclusive prefix over chunks; kept = min(count, C);
 //            the exclusive scan of the selection counts (pre_start);
 //            exclusive scans of the padded kept counts and of their token
@@ -56,7 +57,6 @@ __device__ __forceinline__ void dispatch_count(const DispatchArgs &a, int chunk)
     for (int e = threadIdx.x; e < a.E; e += kChunk) a.chunk_count[(int64_t)chunk * a.E + e] = cnt[e];
 }
 
-__global__ void __launch_bounds__(kChunk) dispatch_count_kernel(DispatchArgs a) { dispatch_count(a, blockIdx.x); }
 
 // Single CTA of kMaxE threads; thread e owns expert e.
 __device__ __forceinline__ void dispatch_scan(const DispatchArgs &a) {
@@ -74,7 +74,7 @@ __device__ __forceinline__ void dispatch_scan(const DispatchArgs &a) {
         for (int c0 = 0; c0 < a.n_chunks; c0 += 32) {
             int v[32];
 #pragma unroll
-            for (int j = 0; j < 32; ++j) v[j] = c0 + j < a.n_chunks ? cnt[(int64_t)(c0 + j) * a.E + e] : 0;
+            for (int j = 0; j < 32; ++j) v[j] = c0 + j < a.n_chunks ? __ldcg(cnt + (int64_t)(c0 + j) * a.E + e) : 0;
 #pragma unroll
             for (int j = 0; j < 32; ++j) {
                 if (c0 + j < a.n_chunks) base[(int64_t)(c0 + j) * a.E + e] = pre;
@@ -165,7 +165,24 @@ __device__ __forceinline__ void dispatch_scan(const DispatchArgs &a) {
     }
 }
 
-__global__ void __launch_bounds__(kMaxE) dispatch_scan_kernel(DispatchArgs a) { dispatch_scan(a); }
+// Count, then scan in the CTA that counts the last chunk (the other CTAs'
+// counts are read from L2); the counter is left at zero again.
+__global__ void __launch_bounds__(kChunk) dispatch_count_scan_kernel(DispatchArgs a) {
+    __shared__ int last;
+    dispatch_count(a, blockIdx.x);
+    __threadfence();  // this thread's counts are visible before the chunk is counted
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        const int old = atomicAdd(a.ctrl + kCtrlDispatchDone, 1);
+        last = old == (int)gridDim.x - 1;
+        if (last) {
+            __threadfence();
+            a.ctrl[kCtrlDispatchDone] = 0;
+        }
+    }
+    __syncthreads();
+    if (last) dispatch_scan(a);
+}
 
 // Stable ranks within the chunk on top of the chunk's per-expert bases; slot,
 // row, row owner and the gate in expert order for every assignment.
@@ -302,10 +319,9 @@ cudaError_t launch_dispatch(const DispatchArgs &a, cudaStream_t s, int *launches
         *launches += 1;
         return cudaGetLastError();
     }
-    dispatch_count_kernel<<<a.n_chunks, kChunk, 0, s>>>(a);
-    dispatch_scan_kernel<<<1, kMaxE, 0, s>>>(a);
+    dispatch_count_scan_kernel<<<a.n_chunks, kChunk, 0, s>>>(a);
     dispatch_assign_kernel<<<a.n_chunks, kChunk, 0, s>>>(a);
-    *launches += 3;
+    *launches += 2;
     return cudaGetLastError();
 }
 

@@ -158,7 +158,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // i-th unit and releases it on the leader's ring_empty. -1 ends the work.
     auto post_unit = [&](uint32_t i) -> int {  // leader's producer, lane 0
         const uint32_t slot = i % kRing, ph = (i / kRing) & 1u;
-        if (!mbar_wait_cluster(&s.ring_empty[slot], ph ^ 1u, a.status)) return -2;
+        if (!mbar_wait_cluster(&s.ring_empty[slot], ph ^ 1u, a.status, a.wait_limit_ns)) return -2;
         int u = atomicAdd(a.work_counter, 1);
         if (u >= total) u = -1;
         s.ring[slot] = u;
@@ -169,7 +169,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     };
     auto take_unit = [&](uint32_t i) -> int {  // one thread of each consumer
         const uint32_t slot = i % kRing, ph = (i / kRing) & 1u;
-        if (!mbar_wait_cluster(&s.ring_full[slot], ph, a.status)) return -2;
+        if (!mbar_wait_cluster(&s.ring_full[slot], ph, a.status, a.wait_limit_ns)) return -2;
         const int u = *reinterpret_cast<volatile int32_t *>(&s.ring[slot]);
         mbar_arrive_cluster(mapa_shared(smem_u32(&s.ring_empty[slot]), 0));
         return u;
@@ -203,7 +203,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const int st = it % kStages;
                 const uint32_t ph = (it / kStages) & 1u;
                 int got = 1;
-                if (lane == 0) got = mbar_wait(&s.empty[st], ph ^ 1u, a.status) ? 1 : 0;
+                if (lane == 0) got = mbar_wait(&s.empty[st], ph ^ 1u, a.status, a.wait_limit_ns) ? 1 : 0;
                 got = __shfl_sync(0xffffffffu, got, 0);
                 if (!got) {
                     ok = false;
@@ -211,6 +211,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 if (lane == 0 && leader) mbar_arrive_expect_tx(&s.full[st], tx_bytes);
                 __syncwarp();
+                // Self-test of the timeout path: the leader announces this
+                // stage's bytes but loads none of its own, so the stage never
+                // completes and the MMA role's bounded wait runs out.
+                if (leader && static_cast<int>(it) == a.skip_stage) continue;
                 const uint32_t bar = mapa_shared(smem_u32(&s.full[st]), 0);
                 uint8_t *sA = s.sA + st * kABytes, *sB = s.sB + st * C::kB;
                 if (lane == 0) tma_load_2d_pair(&map_w, bar, sA, kb * kBK, wrow);
@@ -235,13 +239,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const int ntok = tok_tiles[u / a.n_ftiles].z;
                 const uint32_t idesc = idesc_bf16_f32(kFeatPair, ntok);
                 const uint32_t acc = tcount & 1u, use = tcount >> 1;
-                if (!mbar_wait(&s.tempty[acc], (use & 1u) ^ 1u, a.status)) break;
+                if (!mbar_wait(&s.tempty[acc], (use & 1u) ^ 1u, a.status, a.wait_limit_ns)) break;
                 tc_fence_after_sync();
                 const uint32_t d_tmem = tmem_base + acc * kAccCols;
                 for (int kb = 0; kb < kblocks; ++kb, ++it) {
                     const int st = it % kStages;
                     const uint32_t ph = (it / kStages) & 1u;
-                    if (!mbar_wait(&s.full[st], ph, a.status)) {
+                    if (!mbar_wait(&s.full[st], ph, a.status, a.wait_limit_ns)) {
                         ok = false;
                         break;
                     }
@@ -274,7 +278,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int fcol = j * kFeatPair + static_cast<int>(rank) * kFeatCta + q * 32;
             const uint32_t acc = tcount & 1u, use = tcount >> 1;
             int got = 1;  // one lane waits; tcgen05.ld below is warp-collective
-            if (lane == 0) got = mbar_wait_idle(&s.tfull[acc], use & 1u, a.status) ? 1 : 0;
+            if (lane == 0) got = mbar_wait_idle(&s.tfull[acc], use & 1u, a.status, a.wait_limit_ns) ? 1 : 0;
             if (!__shfl_sync(0xffffffffu, got, 0)) break;
             tc_fence_after_sync();
             if (fcol < a.N) {  // the last feature tile of a ragged N has an idle half

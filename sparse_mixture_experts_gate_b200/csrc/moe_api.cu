@@ -85,9 +85,9 @@ struct Plan {
     int64_t C = 0;
     int T_pad = 0, n_stat_chunks = 0, n_chunks = 0, R_routed_max = 0, R_max = 0, max_row_blocks = 0;
     int max_tok_tiles = 0, max_narrow_tiles = 0;
-    int ksplit = 1;
-    size_t o_lpart = 0;
-    size_t o_ctrl, o_logits, o_idx, o_gates, o_slot, o_rowof, o_lse, o_psum, o_ccount, o_cbase, o_cpre, o_ckept,
+    int ksplit = 1, n_mtiles = 0;  // the fused router's K splits and token tiles
+    size_t o_lpart = 0, ctrl_bytes = 0;
+    size_t o_ctrl, o_rcnt, o_logits, o_idx, o_gates, o_slot, o_rowof, o_lse, o_psum, o_ccount, o_cbase, o_cpre, o_ckept,
         o_gstart, o_grows, o_bgroup, o_toktiles, o_narrowtiles, o_rowassign, o_wsplit, o_xp, o_h, o_o, o_credit, o_partials,
         o_prestart, o_gsorted, o_rownorm, o_gz;
     size_t total = 0;
@@ -109,6 +109,9 @@ struct moe_layer {
     bool tc = false;
     int num_sms = 148;
     int num_pairs = 0;  // co-resident 2-CTA clusters of the expert GEMM
+    int router_pairs = 0;  // and of the fused router
+    int selftest_skip_stage = -1;  // moe_selftest_gemm_timeout only: GEMM 1's skipped stage
+    void *planes = nullptr;        // moe_prepare_router's persistent bf16 planes of the router matrix, or null
     CUtensorMap map_w1, map_w2;
     // State of the most recent forward, read by moe_aux_stats.
     bool has_forward = false;
@@ -155,9 +158,12 @@ Plan make_plan(const moe_layer &L, int T) {
                       S * (int)((p.T_pad + kTokTile - 1) / kTokTile);
     p.max_narrow_tiles = (int)std::min<int64_t>(routed / kNarrowTile + E, routed / kRowBlock) +
                          S * (int)((p.T_pad + kNarrowTile - 1) / kNarrowTile);
-    // bf16 linear routers route from the tensor-core logits; the MLP gate and
-    // fp32 layers route inside the CUDA-core router kernel.
-    p.n_stat_chunks = router_psum_blocks(T, L.num_sms, c.dtype == MOE_DTYPE_BF16 && !c.use_mlp_gater);
+    // bf16 linear routers route in the fused tensor-core kernel (a P-sum row
+    // per half tile of 128 tokens); the MLP gate and fp32 layers route in the
+    // CUDA-core router kernel.
+    const bool fused_routes = c.dtype == MOE_DTYPE_BF16 && !c.use_mlp_gater;
+    p.n_mtiles = c.dtype == MOE_DTYPE_BF16 ? router_fused_mtiles(T) : 0;
+    p.n_stat_chunks = fused_routes ? 2 * p.n_mtiles : router_psum_blocks(T);
     const int64_t n_items = c.capacity_priority == MOE_PRIORITY_RANK ? (int64_t)k * T : T;
     p.n_chunks = (int)((n_items + 255) / 256);
     const size_t es = c.dtype == MOE_DTYPE_BF16 ? 2 : 4;
@@ -168,6 +174,8 @@ Plan make_plan(const moe_layer &L, int T) {
         return o;
     };
     p.o_ctrl = take(kCtrlWords * 4);
+    p.o_rcnt = take((size_t)2 * p.n_mtiles * 4);  // the fused router's arrival counters
+    p.ctrl_bytes = off - p.o_ctrl;                // control words and counters: zeroed every forward
     p.o_logits = take((size_t)T * E * 4);
     p.o_idx = take((size_t)T * k * 4);
     p.o_gates = take((size_t)T * k * 4);
@@ -191,10 +199,12 @@ Plan make_plan(const moe_layer &L, int T) {
     p.o_rownorm = take(c.credit_norm == MOE_CREDIT_HIDDEN ? (size_t)p.R_routed_max * 4 : 0);
     p.o_credit = take((size_t)T * k * 4);
     const int E_tc = c.use_mlp_gater ? c.gater_hidden_dim : E;  // rows of the tensor-core router matrix
-    p.o_wsplit = take(c.dtype == MOE_DTYPE_BF16 ? (size_t)router_tc_epad(E_tc) * 3 * c.input_dim * 2 : 0);
-    p.ksplit = c.dtype == MOE_DTYPE_BF16 && !c.use_mlp_gater ? router_tc_ksplit(T, E, c.input_dim, L.num_sms) : 1;
+    const bool tc = c.dtype == MOE_DTYPE_BF16;
+    p.o_wsplit = take(tc ? (size_t)router_fused_epad(E_tc) * 3 * c.input_dim * 2 : 0);
+    p.ksplit = tc ? router_fused_ksplit(T, E_tc, c.input_dim, L.router_pairs) : 1;
+    const int pieces = tc ? p.ksplit * (router_fused_epad(E_tc) / router_fused_bn(E_tc)) : 1;
     p.o_gz = take(c.use_mlp_gater ? (size_t)T * c.gater_hidden_dim * 4 : 0);
-    p.o_lpart = take(p.ksplit > 1 ? (size_t)p.ksplit * T * E * 4 : 0);
+    p.o_lpart = take(pieces > 1 ? (size_t)p.n_mtiles * 256 * router_fused_epad(E_tc) * p.ksplit * 4 : 0);
     p.o_xp = take(c.dtype == MOE_DTYPE_BF16 ? (size_t)p.R_routed_max * c.input_dim * es : 0);
     p.o_h = take((size_t)p.R_max * c.expert_dim * es);
     p.o_o = take((size_t)p.R_max * c.output_dim * es);
@@ -337,9 +347,10 @@ int moe_layer_create(const moe_config_t *cfg, const moe_weights_t *w, moe_layer_
             return fail(MOE_ERR_CUDA, "cuTensorMapEncodeTiled failed for the expert weights (16-byte alignment?)");
         }
         L->num_pairs = gemm_pair_max_pairs(L->num_sms);
-        if (L->num_pairs <= 0) {
+        L->router_pairs = router_fused_max_pairs(L->num_sms);
+        if (L->num_pairs <= 0 || L->router_pairs <= 0) {
             delete L;
-            return fail(MOE_ERR_CUDA, "no 2-CTA cluster of the expert GEMM fits on device %d", dev);
+            return fail(MOE_ERR_CUDA, "no 2-CTA cluster of the expert GEMM or router fits on device %d", dev);
         }
     }
     *out = L;
@@ -386,7 +397,7 @@ int fwd_route(moe_layer_t *L, const void *x, int32_t T, const float *logit_noise
     L->fwd_launches = 0;
     L->stats_launches = 0;
     int32_t *ctrl = reinterpret_cast<int32_t *>(ws + p.o_ctrl);
-    MOE_LAUNCH(cudaMemsetAsync(ctrl, 0, kCtrlWords * 4, s));
+    MOE_LAUNCH(cudaMemsetAsync(ctrl, 0, p.ctrl_bytes, s));
     if (T == 0) return MOE_OK;
     MOE_MARK(L, 0, s);
 
@@ -417,34 +428,54 @@ int fwd_route(moe_layer_t *L, const void *x, int32_t T, const float *logit_noise
     ra.gates = gates;
     ra.lse = reinterpret_cast<float *>(ws + p.o_lse);
     ra.psum_part = reinterpret_cast<float *>(ws + p.o_psum);
-    ra.logit_part = nullptr;
-    ra.ksplit = 1;
     ra.x_relu = 0;
     ra.logits_only = 0;
+    // The tensor-core router (bf16 x): W_g, or the MLP gate's hidden matrix,
+    // split into bf16 planes, then one fused kernel.
+    auto fused = [&](const float *w, const float *b, int rows, float *out_logits, int route) -> int {
+        const int E_pad = router_fused_epad(rows), BN = router_fused_bn(rows);
+        __nv_bfloat16 *w_split = reinterpret_cast<__nv_bfloat16 *>(ws + p.o_wsplit);
+        if (L->planes)  // split once by moe_prepare_router
+            w_split = static_cast<__nv_bfloat16 *>(L->planes);
+        else
+            MOE_LAUNCH(launch_router_split(w, rows, E_pad, c.input_dim, w_split, L->num_sms, s, nl));
+        CUtensorMap m_xr, m_ws;
+        if (!encode_bf16_2d(&m_xr, x, c.input_dim, T, kBM) ||
+            !encode_bf16_2d(&m_ws, w_split, 3ull * c.input_dim, E_pad, BN / 2))
+            return fail(MOE_ERR_CUDA, "cuTensorMapEncodeTiled failed for the router operands");
+        RouterFusedArgs fa;
+        fa.b_gate = b;
+        fa.noise = route ? ra.noise : nullptr;
+        fa.sel_bias = route ? ra.sel_bias : nullptr;
+        fa.T = T;
+        fa.d = c.input_dim;
+        fa.E = rows;
+        fa.k = k;
+        fa.BN = BN;
+        fa.n_tiles = E_pad / BN;
+        fa.ksplit = p.ksplit;
+        fa.n_mtiles = p.n_mtiles;
+        fa.route = route;
+        fa.logits = out_logits;
+        fa.idx = idx;
+        fa.gates = gates;
+        fa.lse = ra.lse;
+        fa.psum_part = ra.psum_part;
+        fa.part = reinterpret_cast<float *>(ws + p.o_lpart);
+        fa.counters = reinterpret_cast<int32_t *>(ws + p.o_rcnt);
+        fa.status = status;
+        fa.num_pairs = L->router_pairs;
+        MOE_LAUNCH(launch_router_fused(m_xr, m_ws, fa, s, nl));
+        return MOE_OK;
+    };
     if (c.use_mlp_gater) {
         // Hidden layer z = W_1 x + b_1 (pre-activations, [T][H] fp32), then the
         // output layer h = W_2 relu(z) + b_2 and the routing in one kernel.
         const int H = c.gater_hidden_dim;
         float *z = reinterpret_cast<float *>(ws + p.o_gz);
         if (L->tc) {
-            RouterTcArgs rt_args;
-            rt_args.w_gate = L->w.gater_w1;
-            rt_args.b_gate = L->w.gater_b1;
-            rt_args.T = T;
-            rt_args.d = c.input_dim;
-            rt_args.E = H;
-            rt_args.E_pad = router_tc_epad(H);
-            rt_args.logits = z;
-            rt_args.ksplit = 1;
-            rt_args.partial = nullptr;
-            rt_args.status = status;
-            rt_args.num_sms = L->num_sms;
-            __nv_bfloat16 *w_split = reinterpret_cast<__nv_bfloat16 *>(ws + p.o_wsplit);
-            CUtensorMap m_xr, m_ws;
-            if (!encode_bf16_2d(&m_xr, x, c.input_dim, T, kBM) ||
-                !encode_bf16_2d(&m_ws, w_split, 3ull * c.input_dim, rt_args.E_pad, router_tc_bn(H)))
-                return fail(MOE_ERR_CUDA, "cuTensorMapEncodeTiled failed for the gate operands");
-            MOE_LAUNCH(launch_router_logits_tc(m_xr, m_ws, rt_args, w_split, s, nl));
+            const int rc = fused(L->w.gater_w1, L->w.gater_b1, H, z, 0);
+            if (rc != MOE_OK) return rc;
         } else {
             RouterArgs rh = ra;
             rh.w_gate = L->w.gater_w1;
@@ -462,29 +493,8 @@ int fwd_route(moe_layer_t *L, const void *x, int32_t T, const float *logit_noise
         ra.d = H;
         MOE_LAUNCH(launch_router(ra, s, nl));
     } else if (L->tc) {
-        RouterTcArgs rt_args;
-        rt_args.w_gate = L->w.w_gate;
-        rt_args.b_gate = L->w.b_gate;
-        rt_args.T = T;
-        rt_args.d = c.input_dim;
-        rt_args.E = E;
-        rt_args.E_pad = router_tc_epad(E);
-        rt_args.logits = logits;
-        rt_args.ksplit = p.ksplit;
-        rt_args.partial = reinterpret_cast<float *>(ws + p.o_lpart);
-        rt_args.status = status;
-        rt_args.num_sms = L->num_sms;
-        __nv_bfloat16 *w_split = reinterpret_cast<__nv_bfloat16 *>(ws + p.o_wsplit);
-        CUtensorMap m_xr, m_ws;
-        if (!encode_bf16_2d(&m_xr, x, c.input_dim, T, kBM) ||
-            !encode_bf16_2d(&m_ws, w_split, 3ull * c.input_dim, rt_args.E_pad, router_tc_bn(E)))
-            return fail(MOE_ERR_CUDA, "cuTensorMapEncodeTiled failed for the router operands");
-        MOE_LAUNCH(launch_router_logits_tc(m_xr, m_ws, rt_args, w_split, s, nl));
-        if (p.ksplit > 1) {
-            ra.logit_part = rt_args.partial;
-            ra.ksplit = p.ksplit;
-        }
-        MOE_LAUNCH(launch_route_from_logits(ra, L->num_sms, s, nl));
+        const int rc = fused(L->w.w_gate, L->w.b_gate, E, logits, 1);
+        if (rc != MOE_OK) return rc;
     } else {
         MOE_LAUNCH(launch_router(ra, s, nl));
     }
@@ -583,6 +593,10 @@ int fwd_expert_gemms(moe_layer_t *L, cudaStream_t s, bool shared_only) {
         g1.work_counter = ctrl + kCtrlWork1;
         g1.num_pairs = L->num_pairs;
         PairGemmArgs g2 = g1;
+        if (L->selftest_skip_stage >= 0) {  // the timeout self-test: GEMM 1 misses one stage's loads
+            g1.skip_stage = L->selftest_skip_stage;
+            g1.wait_limit_ns = kSelftestWaitNs;
+        }
         g2.N = c.output_dim;
         g2.K = c.expert_dim;
         g2.n_ftiles = gemm_pair_ftiles(c.output_dim);
@@ -845,8 +859,10 @@ int moe_ep_combine(moe_layer_t *L, void *y, void *stream_v) {
 
 namespace {
 
-// Enqueues the partial sums of the most recent forward into `partials`.
-int enqueue_partials(moe_layer_t *L, const float *token_loss, float *partials, cudaStream_t s, int *launches) {
+// Enqueues the partial sums of the most recent forward into `partials` (and,
+// with fin, the statistics from them in the same launch).
+int enqueue_partials(moe_layer_t *L, const float *token_loss, float *partials, cudaStream_t s, int *launches,
+                     const FinalizeArgs *fin = nullptr) {
     const Plan &p = L->plan;
     const moe_config_t &c = L->cfg;
     char *ws = L->ws;
@@ -867,12 +883,12 @@ int enqueue_partials(moe_layer_t *L, const float *token_loss, float *partials, c
     sa.E = c.num_experts;
     sa.k = c.num_active;
     sa.partials = partials;
-    MOE_LAUNCH(launch_stat_partials(sa, s, launches));
+    sa.done_counter = reinterpret_cast<int32_t *>(ws + p.o_ctrl) + kCtrlStatsDone;
+    MOE_LAUNCH(launch_stat_partials(sa, fin, s, launches));
     return MOE_OK;
 }
 
-int enqueue_finalize(moe_layer_t *L, const float *partials, bool has_loss, const moe_stats_t *out, cudaStream_t s,
-                     int *launches) {
+FinalizeArgs finalize_args(const moe_layer_t *L, const float *partials, bool has_loss, const moe_stats_t *out) {
     const moe_config_t &c = L->cfg;
     FinalizeArgs fa;
     fa.partials = partials;
@@ -890,6 +906,12 @@ int enqueue_finalize(moe_layer_t *L, const float *partials, bool has_loss, const
     fa.cv_load = out->cv_load;
     fa.cv_importance = out->cv_importance;
     fa.l_total = out->l_total;
+    return fa;
+}
+
+int enqueue_finalize(moe_layer_t *L, const float *partials, bool has_loss, const moe_stats_t *out, cudaStream_t s,
+                     int *launches) {
+    const FinalizeArgs fa = finalize_args(L, partials, has_loss, out);
     MOE_LAUNCH(launch_stats_finalize(fa, s, launches));
     return MOE_OK;
 }
@@ -909,9 +931,8 @@ int moe_aux_stats(moe_layer_t *L, const float *token_loss, const moe_stats_t *ou
     L->stats_launches = 0;
     if (p.T == 0) return MOE_OK;
     float *partials = reinterpret_cast<float *>(L->ws + p.o_partials);
-    int rc = enqueue_partials(L, token_loss, partials, s, &L->stats_launches);
-    if (rc != MOE_OK) return rc;
-    rc = enqueue_finalize(L, partials, token_loss != nullptr, out, s, &L->stats_launches);
+    const FinalizeArgs fin = finalize_args(L, partials, token_loss != nullptr, out);
+    int rc = enqueue_partials(L, token_loss, partials, s, &L->stats_launches, &fin);
     if (rc != MOE_OK) return rc;
     if (out->credit)
         MOE_LAUNCH(cudaMemcpyAsync(out->credit, L->ws + p.o_credit, (size_t)p.T * c.num_active * 4,
@@ -981,6 +1002,55 @@ int moe_dro_update(moe_layer_t *L, const float *expert_loss, float ema, float et
     da.eta = eta;
     int launches = 0;
     MOE_LAUNCH(launch_dro_update(da, as_stream(stream_v), &launches));
+    return MOE_OK;
+}
+
+size_t moe_router_planes_bytes(const moe_layer_t *L) {
+    if (!L || !L->tc) return 0;
+    const int rows = L->cfg.use_mlp_gater ? L->cfg.gater_hidden_dim : L->cfg.num_experts;
+    return (size_t)router_fused_epad(rows) * 3 * L->cfg.input_dim * 2;
+}
+
+int moe_prepare_router(moe_layer_t *L, void *planes, size_t bytes, void *stream_v) {
+    g_last_error.clear();
+    if (!L) return fail(MOE_ERR_INVALID_ARG, "layer is NULL");
+    if (!L->tc) return fail(MOE_ERR_UNSUPPORTED, "fp32 layers route on CUDA cores from the fp32 router matrix");
+    if (!planes) {
+        L->planes = nullptr;
+        return MOE_OK;
+    }
+    const size_t need = moe_router_planes_bytes(L);
+    if (bytes < need) return fail(MOE_ERR_WORKSPACE, "router planes: %zu bytes given, %zu needed", bytes, need);
+    if (reinterpret_cast<uintptr_t>(planes) % 256) return fail(MOE_ERR_WORKSPACE, "planes must be 256-byte aligned");
+    const moe_config_t &c = L->cfg;
+    const int rows = c.use_mlp_gater ? c.gater_hidden_dim : c.num_experts;
+    const float *w = c.use_mlp_gater ? L->w.gater_w1 : L->w.w_gate;
+    int launches = 0;
+    MOE_LAUNCH(launch_router_split(w, rows, router_fused_epad(rows), c.input_dim, static_cast<__nv_bfloat16 *>(planes),
+                                   L->num_sms, as_stream(stream_v), &launches));
+    L->planes = planes;
+    return MOE_OK;
+}
+
+int moe_selftest_gemm_timeout(moe_layer_t *L, const void *x, int32_t T, void *workspace, size_t ws_bytes, void *y,
+                              void *stream_v) {
+    g_last_error.clear();
+    if (!L) return fail(MOE_ERR_INVALID_ARG, "layer is NULL");
+    if (!L->tc || L->cfg.ep_size > 1)
+        return fail(MOE_ERR_UNSUPPORTED, "the self-test runs the tensor-core expert GEMM of a bf16 layer, ep_size 1");
+    if (L->cfg.top_k_method != MOE_TOPK_GREEDY) return fail(MOE_ERR_UNSUPPORTED, "the self-test needs GREEDY top-k");
+    if (T <= 0) return fail(MOE_ERR_INVALID_ARG, "the self-test needs T > 0");
+    if (L->cfg.input_dim < 3 * kBK)
+        return fail(MOE_ERR_UNSUPPORTED, "the self-test needs input_dim >= %d (three K stages)", 3 * kBK);
+    L->selftest_skip_stage = 2;
+    int rc = moe_forward(L, x, T, nullptr, workspace, ws_bytes, y, nullptr, stream_v);
+    L->selftest_skip_stage = -1;
+    if (rc != MOE_OK) return rc;
+    cudaStream_t s = as_stream(stream_v);
+    MOE_LAUNCH(cudaStreamSynchronize(s));
+    uint32_t st = 0;
+    MOE_LAUNCH(cudaMemcpy(&st, L->ws + L->plan.o_ctrl + kCtrlStatus * 4, 4, cudaMemcpyDeviceToHost));
+    if (!(st & kDevTimeout)) return fail(MOE_ERR_INTERNAL, "expert GEMM 1 missed a stage but reported no timeout");
     return MOE_OK;
 }
 

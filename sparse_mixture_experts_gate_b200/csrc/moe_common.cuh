@@ -29,6 +29,8 @@ enum : uint32_t { kDevOk = 0u, kDevTimeout = 1u };
 
 // A bounded wait gives up after this long (wall clock, %globaltimer ns).
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
+// The shorter limit of the expert GEMM launch that the timeout self-test runs.
+constexpr uint64_t kSelftestWaitNs = 20000000ull;
 
 __device__ __forceinline__ uint32_t smem_u32(const void *p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -79,7 +81,8 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
 // The status word (a global load) is only polled once the wait has lasted
 // kStatusPollNs, so a normal short wait spins on the barrier alone.
 constexpr uint64_t kStatusPollNs = 20000ull;
-__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, uint32_t *status) {
+__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, uint32_t *status,
+                                          uint64_t limit_ns = kWaitLimitNs) {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = global_timer_ns();
     for (;;) {
@@ -88,7 +91,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, uint32
             if (mbar_try_wait(bar, parity)) return true;
         const uint64_t dt = global_timer_ns() - t0;
         if (dt > kStatusPollNs && *reinterpret_cast<volatile uint32_t *>(status) != kDevOk) return false;
-        if (dt > kWaitLimitNs) {
+        if (dt > limit_ns) {
             atomicOr(status, kDevTimeout);
             return false;
         }
@@ -99,7 +102,8 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, uint32
 // latency-critical (an epilogue waiting for the next accumulator): after the
 // first microsecond it sleeps between polls, leaving issue slots and shared
 // memory bandwidth to the roles that are working.
-__device__ __forceinline__ bool mbar_wait_idle(uint64_t *bar, uint32_t parity, uint32_t *status) {
+__device__ __forceinline__ bool mbar_wait_idle(uint64_t *bar, uint32_t parity, uint32_t *status,
+                                               uint64_t limit_ns = kWaitLimitNs) {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = global_timer_ns();
     for (;;) {
@@ -107,7 +111,7 @@ __device__ __forceinline__ bool mbar_wait_idle(uint64_t *bar, uint32_t parity, u
         const uint64_t dt = global_timer_ns() - t0;
         if (dt > 1000ull) __nanosleep(256);
         if (dt > kStatusPollNs && *reinterpret_cast<volatile uint32_t *>(status) != kDevOk) return false;
-        if (dt > kWaitLimitNs) {
+        if (dt > limit_ns) {
             atomicOr(status, kDevTimeout);
             return false;
         }
@@ -321,7 +325,8 @@ __device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t *bar, uint32_t pa
 }
 
 // Bounded wait with cluster-scope acquire (same limits as mbar_wait).
-__device__ __forceinline__ bool mbar_wait_cluster(uint64_t *bar, uint32_t parity, uint32_t *status) {
+__device__ __forceinline__ bool mbar_wait_cluster(uint64_t *bar, uint32_t parity, uint32_t *status,
+                                                  uint64_t limit_ns = kWaitLimitNs) {
     if (mbar_try_wait_cluster(bar, parity)) return true;
     const uint64_t t0 = global_timer_ns();
     for (;;) {
@@ -330,7 +335,7 @@ __device__ __forceinline__ bool mbar_wait_cluster(uint64_t *bar, uint32_t parity
             if (mbar_try_wait_cluster(bar, parity)) return true;
         const uint64_t dt = global_timer_ns() - t0;
         if (dt > kStatusPollNs && *reinterpret_cast<volatile uint32_t *>(status) != kDevOk) return false;
-        if (dt > kWaitLimitNs) {
+        if (dt > limit_ns) {
             atomicOr(status, kDevTimeout);
             return false;
         }

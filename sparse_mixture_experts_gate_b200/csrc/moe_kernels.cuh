@@ -5,10 +5,12 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include "moe_common.cuh"
+
 namespace moe {
 
-// Router (fp32 CUDA cores, fp32 layers): logits h = W_g x + b, max,
-// log-partition, selection key, top-k, renormalised gates.
+// Router on fp32 CUDA cores (fp32 layers, and the MLP gate's output layer):
+// logits h = W_g x + b, max, log-partition, selection key, top-k, gates.
 struct RouterArgs {
     const void *x;          // [T][d] bf16 or fp32
     int x_bf16;
@@ -22,33 +24,44 @@ struct RouterArgs {
     float *gates;           // [T][k]
     float *lse;             // [T]
     float *psum_part;       // [router_psum_blocks][E]: per-block sums of P over its tokens
-    const float *logit_part;  // routing from split-K partials: [ksplit][T][E], or null
-    int ksplit;
     int x_relu;             // fp32 router only: relu(x) is the router's input (MLP gate output layer)
     int logits_only;        // fp32 router only: write logits (+ bias) and stop (MLP gate hidden layer)
 };
-int router_psum_blocks(int T, int num_sms, bool from_logits);
+int router_psum_blocks(int T);
 cudaError_t launch_router(const RouterArgs &a, cudaStream_t s, int *launches);
-// Max, log-partition, keys, top-k and gates from logits already in a.logits.
-cudaError_t launch_route_from_logits(const RouterArgs &a, int num_sms, cudaStream_t s, int *launches);
 
-// Router logits on the tensor cores (bf16 layers): logits [T][E], bias included.
-struct RouterTcArgs {
-    const float *w_gate;    // [E][d] fp32, split into bf16 planes every forward
+// Router of bf16 layers in one kernel (router_fused.cu): logits on the tensor
+// cores from three bf16 planes of W_g, then (route = 1) softmax, log-partition,
+// keys, top-k, gates and the per-half-tile P sums. Units: token tiles of 256,
+// expert tiles of BN, ksplit K splits.
+struct RouterFusedArgs {
     const float *b_gate;    // [E] or null
-    int T, d, E, E_pad;
-    float *logits;          // [T][E]   (ksplit == 1)
-    int ksplit;             // K splits (router_tc_ksplit)
-    float *partial;         // [ksplit][T][E] raw partial sums (ksplit > 1)
+    const float *noise;     // [T][E] or null (added to the selection key only)
+    const float *sel_bias;  // [E] or null (added to the selection key only)
+    int T, d, E, k;
+    int BN, n_tiles, ksplit, n_mtiles;
+    int route;              // 0: logits (+ bias) only, e.g. the MLP gate's hidden layer
+    float *logits;          // [T][E]
+    int32_t *idx;           // [T][k]
+    float *gates;           // [T][k]
+    float *lse;             // [T]
+    float *psum_part;       // [2 n_mtiles][E]: P summed over each half tile of 128 tokens
+    float *part;            // [n_mtiles n_tiles ksplit][256][BN] partial sums when n_tiles ksplit > 1
+    int32_t *counters;      // [2 n_mtiles], zero before the launch
     uint32_t *status;
-    int num_sms;
+    int num_pairs;          // CTA pairs to launch at most
 };
-int router_tc_epad(int E);  // padded expert count (rows of the split planes)
-int router_tc_bn(int E);    // N tile of the logits GEMM (<= 128)
-int router_tc_ksplit(int T, int E, int d, int num_sms);
-// map_x: x [T][d] bf16, box 64 x 128; map_w: w_split [E_pad][3d] bf16, box 64 x router_tc_bn(E).
-cudaError_t launch_router_logits_tc(const CUtensorMap &map_x, const CUtensorMap &map_w, const RouterTcArgs &a,
-                                    __nv_bfloat16 *w_split, cudaStream_t s, int *launches);
+int router_fused_epad(int E);    // padded expert count (rows of the split planes): 32, 64, 128 or 256
+int router_fused_bn(int E);      // expert tile: E_pad up to 128
+int router_fused_mtiles(int T);  // token tiles of 256
+int router_fused_ksplit(int T, int E, int d, int num_pairs);
+int router_fused_max_pairs(int num_sms);
+// W_g [E][d] fp32 -> w_split [E_pad][3d] bf16: planes hi | mid | lo, rows >= E zero.
+cudaError_t launch_router_split(const float *w_gate, int E, int E_pad, int d, __nv_bfloat16 *w_split, int num_sms,
+                                cudaStream_t s, int *launches);
+// map_x: x [T][d] bf16, box 64 x 128; map_w: w_split, box 64 x BN/2.
+cudaError_t launch_router_fused(const CUtensorMap &map_x, const CUtensorMap &map_w, const RouterFusedArgs &a,
+                                cudaStream_t s, int *launches);
 
 // Dispatch: histogram, scan, stable capacity-capped ranks, row map.
 struct DispatchArgs {
@@ -91,7 +104,9 @@ enum {
     kCtrlWork2 = 6,
     kCtrlRoutedTiles = 7,  // token tiles of the routed experts (the shared experts' follow)
     kCtrlNumNarrowTiles = 8,
-    kCtrlWords = 9
+    kCtrlStatsDone = 9,      // CTAs of the statistics kernel done (its last CTA resets it)
+    kCtrlDispatchDone = 10,  // chunks counted by the dispatch (its last CTA resets it)
+    kCtrlWords = 11
 };
 
 // Rows of a narrow token tile: for short expert segments the expert GEMM
@@ -137,6 +152,11 @@ struct PairGemmArgs {
     uint32_t *status;            // device status word
     int32_t *work_counter;       // zero before the launch; units are handed out in order
     int num_pairs;               // clusters of 2 CTAs to launch
+    // Self-test of the bounded waits only (moe_selftest_gemm_timeout): the
+    // leader's producer skips its loads of this pipeline stage (-1: none), and
+    // every wait of the launch gives up after wait_limit_ns.
+    int skip_stage = -1;
+    uint64_t wait_limit_ns = kWaitLimitNs;
 };
 int gemm_pair_max_pairs(int num_sms);
 int gemm_pair_ftiles(int N);
@@ -192,8 +212,8 @@ struct StatsArgs {
     const float *gate_sorted; // [T*k]
     int T, E, k;
     float *partials;          // [4E + 3] output
+    int32_t *done_counter;    // zero; counts the CTAs done when the finalize is fused
 };
-cudaError_t launch_stat_partials(const StatsArgs &a, cudaStream_t s, int *launches);
 
 struct FinalizeArgs {
     const float *partials;    // [4E + 3]
@@ -203,6 +223,8 @@ struct FinalizeArgs {
     int32_t *n_dropped;
     float *importance, *cv_load, *cv_importance, *l_total;
 };
+// fin != null: the last CTA also forms the statistics (one launch in all).
+cudaError_t launch_stat_partials(const StatsArgs &a, const FinalizeArgs *fin, cudaStream_t s, int *launches);
 cudaError_t launch_stats_finalize(const FinalizeArgs &a, cudaStream_t s, int *launches);
 
 // Expert parallelism: the token-tile table of rows received from G source

@@ -42,11 +42,16 @@ __device__ __forceinline__ float block_sum_256(float v, float *red) {
     return t;
 }
 
+__device__ __forceinline__ void finalize_body(const FinalizeArgs &a, float *red);
+
 // One CTA per expert (CTA E does the per-token scalars); every sum has a fixed
 // order (thread-strided, then a fixed shuffle tree and warp order), so repeated
-// runs give bit-identical results.
-__global__ void __launch_bounds__(256) stat_partials_kernel(StatsArgs a) {
+// runs give bit-identical results. With `fin` set, the CTA that writes the last
+// partial words (counted on done_counter) also forms the statistics from them,
+// so that moe_aux_stats is one launch; it leaves the counter at zero again.
+__global__ void __launch_bounds__(256) stat_partials_kernel(StatsArgs a, FinalizeArgs fin, int fuse) {
     __shared__ float red[8];
+    __shared__ int last;
     const int tid = threadIdx.x;
     if (blockIdx.x == a.E) {  // sum_t lse_t^2, T, drops
         float z = 0.f;
@@ -57,34 +62,46 @@ __global__ void __launch_bounds__(256) stat_partials_kernel(StatsArgs a) {
             a.partials[2 * a.E + 1] = (float)a.T;
             a.partials[2 * a.E + 2] = (float)a.ctrl[kCtrlDropped];
         }
-        return;
-    }
-    const int e = blockIdx.x;
-    float ps = 0.f;
-    for (int i = tid; i < a.n_chunks; i += 256) ps += a.psum_part[(int64_t)i * a.E + e];
-    ps = block_sum_256(ps, red);
-    float el = 0.f;
-    if (a.token_loss) {
-        const int r0 = a.group_start[e], r1 = r0 + a.group_rows[e];
-        for (int row = r0 + tid; row < r1; row += 256) {
-            const int ai = a.row_assign[row];
-            el += a.credit[ai] * a.token_loss[ai / a.k];
+    } else {
+        const int e = blockIdx.x;
+        float ps = 0.f;
+        for (int i = tid; i < a.n_chunks; i += 256) ps += a.psum_part[(int64_t)i * a.E + e];
+        ps = block_sum_256(ps, red);
+        float el = 0.f;
+        if (a.token_loss) {
+            const int r0 = a.group_start[e], r1 = r0 + a.group_rows[e];
+            for (int row = r0 + tid; row < r1; row += 256) {
+                const int ai = a.row_assign[row];
+                el += a.credit[ai] * a.token_loss[ai / a.k];
+            }
+            el = block_sum_256(el, red);
         }
-        el = block_sum_256(el, red);
+        // Importance: this expert's selection gates, in priority order.
+        float imp = 0.f;
+        {
+            const int g0 = a.pre_start[e], n = a.count_pre[e];
+            for (int j = tid; j < n; j += 256) imp += a.gate_sorted[g0 + j];
+            imp = block_sum_256(imp, red);
+        }
+        if (tid == 0) {
+            a.partials[e] = ps;
+            a.partials[a.E + e] = (float)a.count_pre[e];
+            a.partials[2 * a.E + 3 + e] = el;
+            a.partials[3 * a.E + 3 + e] = imp;
+        }
     }
-    // Importance: this expert's selection gates, in priority order.
-    float imp = 0.f;
-    {
-        const int g0 = a.pre_start[e], n = a.count_pre[e];
-        for (int j = tid; j < n; j += 256) imp += a.gate_sorted[g0 + j];
-        imp = block_sum_256(imp, red);
-    }
+    if (!fuse) return;
     if (tid == 0) {
-        a.partials[e] = ps;
-        a.partials[a.E + e] = (float)a.count_pre[e];
-        a.partials[2 * a.E + 3 + e] = el;
-        a.partials[3 * a.E + 3 + e] = imp;
+        __threadfence();  // this CTA's partial words are visible before it is counted
+        const int old = atomicAdd(a.done_counter, 1);
+        last = old == (int)gridDim.x - 1;
+        if (last) {
+            __threadfence();
+            *a.done_counter = 0;  // ready for the next call
+        }
     }
+    __syncthreads();
+    if (last) finalize_body(fin, red);
 }
 
 // Squared coefficient of variation of one value per thread (threads >= n hold
@@ -104,22 +121,23 @@ __device__ __forceinline__ float block_cv_squared(float v, bool valid, int n, fl
 // = load_balance_coef * load_balance + z_loss_coef * z_loss, load_balance
 // being the coefficient-of-variation style loss of the loads). One CTA of
 // 256 threads (E <= 256), thread e owns expert e; every sum is a fixed tree.
-__global__ void __launch_bounds__(256) stats_finalize_kernel(FinalizeArgs a) {
-    __shared__ float red[8];
+// The partial sums may have been written by other CTAs of the same launch, so
+// they are read from L2.
+__device__ __forceinline__ void finalize_body(const FinalizeArgs &a, float *red) {
     const int e = threadIdx.x;
     const bool own = e < a.E;
-    const float T = a.partials[2 * a.E + 1];
+    const float T = __ldcg(a.partials + 2 * a.E + 1);
     const float inv_t = T > 0.f ? 1.f / T : 0.f;
     const float inv_kt = T > 0.f ? 1.f / ((float)a.k * T) : 0.f;
     float pm = 0.f, f = 0.f, load = 0.f, imp = 0.f;
     if (own) {
-        pm = a.partials[e] * inv_t;
-        load = a.partials[a.E + e];
+        pm = __ldcg(a.partials + e) * inv_t;
+        load = __ldcg(a.partials + a.E + e);
         f = load * inv_kt;
-        imp = a.partials[3 * a.E + 3 + e];
+        imp = __ldcg(a.partials + 3 * a.E + 3 + e);
         if (a.p_mean) a.p_mean[e] = pm;
         if (a.f) a.f[e] = f;
-        if (a.expert_loss) a.expert_loss[e] = a.partials[2 * a.E + 3 + e] * inv_t;
+        if (a.expert_loss) a.expert_loss[e] = __ldcg(a.partials + 2 * a.E + 3 + e) * inv_t;
         if (a.importance) a.importance[e] = imp;
     }
     const float fp = block_sum_256(own ? f * pm : 0.f, red);
@@ -127,14 +145,19 @@ __global__ void __launch_bounds__(256) stats_finalize_kernel(FinalizeArgs a) {
     const float cv_imp = block_cv_squared(imp, own, a.E, red);
     if (e == 0) {
         const float l_aux = a.alpha * (float)a.E * fp;
-        const float l_z = a.beta * a.partials[2 * a.E] * inv_t;
+        const float l_z = a.beta * __ldcg(a.partials + 2 * a.E) * inv_t;
         if (a.l_aux) *a.l_aux = l_aux;
         if (a.l_z) *a.l_z = l_z;
         if (a.l_total) *a.l_total = a.alpha * cv_load + l_z;
-        if (a.n_dropped) *a.n_dropped = (int32_t)a.partials[2 * a.E + 2];
+        if (a.n_dropped) *a.n_dropped = (int32_t)__ldcg(a.partials + 2 * a.E + 2);
         if (a.cv_load) *a.cv_load = cv_load;
         if (a.cv_importance) *a.cv_importance = cv_imp;
     }
+}
+
+__global__ void __launch_bounds__(256) stats_finalize_kernel(FinalizeArgs a) {
+    __shared__ float red[8];
+    finalize_body(a, red);
 }
 
 // Aux-loss-free balancing ("Balancing": per-expert selection bias b_i, update
@@ -228,8 +251,9 @@ __global__ void __launch_bounds__(256) dro_update_kernel(DroArgs a) {
 
 }  // namespace
 
-cudaError_t launch_stat_partials(const StatsArgs &a, cudaStream_t s, int *launches) {
-    stat_partials_kernel<<<a.E + 1, 256, 0, s>>>(a);
+cudaError_t launch_stat_partials(const StatsArgs &a, const FinalizeArgs *fin, cudaStream_t s, int *launches) {
+    FinalizeArgs none = {};
+    stat_partials_kernel<<<a.E + 1, 256, 0, s>>>(a, fin ? *fin : none, fin ? 1 : 0);
     *launches += 1;
     return cudaGetLastError();
 }

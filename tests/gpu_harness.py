@@ -129,7 +129,8 @@ def check_end_to_end(w, inp, g, tokens=None, table=None):
         h = oracle.router_mlp(x_rows, inp["gater_w1"].cpu(), g1, inp["w_gate"].cpu(), bg)
     else:
         h = oracle.router_logits(x_rows, inp["w_gate"].cpu(), bg)
-    assert np.abs(g["logits"][toks] - h).max() <= LOGIT_TOL, np.abs(g["logits"][toks] - h).max()
+    logit_err = float(np.abs(g["logits"][toks] - h).max())
+    assert logit_err <= LOGIT_TOL, logit_err
     noise = inp["noise"].cpu()[torch.as_tensor(toks)] if (w.top_k_method == "noisy") else None
     sb = inp.get("sel_bias").cpu() if w.use_selection_bias else None
     key = oracle.selection_keys(h.astype(np.float32), noise, sb)
@@ -150,7 +151,7 @@ def check_end_to_end(w, inp, g, tokens=None, table=None):
                                               w.d, w.F, w.E, w.activation)
     cerr = np.abs(g["credit"][toks] - credit) / (1.0 + np.abs(credit))
     assert cerr.max() <= CREDIT_TOL[w.dtype], f"credit: max scaled error {cerr.max():.3e}"
-    info = dict(n_near_ties=int(ties.sum()), y_err=float(err.max()), credit_err=float(cerr.max()))
+    info = dict(n_near_ties=int(ties.sum()), y_err=float(err.max()), credit_err=float(cerr.max()), logit_err=logit_err)
     if tokens is None and inp.get("token_loss") is not None:
         info["expert_loss_err"] = check_expert_loss_vs_oracle(w, inp, g, credit)
     return info

@@ -174,7 +174,8 @@ def _sampled_full(name, min_tokens):
     assert int(g["count_kept"].sum()) == w.k * w.T - int(g["n_dropped"][0])
     assert int(g["count_pre"].sum()) == w.k * w.T
     assert np.allclose(g["gates"].sum(1), 1.0, atol=1e-5)
-    print(f"{name}: {len(toks)} sampled tokens cover {n_items} GEMM tiles and last rows; y_err {info['y_err']:.2e}")
+    print(f"{name}: {len(toks)} sampled tokens cover {n_items} GEMM tiles and last rows; y_err {info['y_err']:.2e}, "
+          f"logit_err {info['logit_err']:.2e}")
     return g, info
 
 
@@ -400,6 +401,28 @@ def test_bounded_wait_times_out_and_context_survives():
     full_check(w, make_inputs(w, "cpu", seed=2))
 
 
+def test_expert_gemm_timeout_drains_and_context_survives():
+    """Failure detection inside the real expert GEMM: GEMM 1's leader CTAs skip
+    one stage's loads (a test-only launch argument) and the launch's waits give
+    up after 20 ms. The MMA role's wait runs out, every role drains and the
+    kernel returns; the device status reports the timeout; the same layer and
+    context then run a forward that matches the oracle."""
+    from sparse_mixture_experts_gate_b200 import binding
+    w = WORKLOADS["default"].with_(T=600)
+    inp = make_inputs(w, "cpu", seed=2)
+    layer = MoELayer(w, inp)
+    x = inp["x"].cuda()
+    ws, need = layer.workspace(w.T)
+    y = torch.empty(w.T, w.O, dtype=torch.bfloat16, device="cuda")
+    s = torch.cuda.current_stream().cuda_stream
+    assert binding.moe_selftest_gemm_timeout(layer.handle, x.data_ptr(), w.T, ws.data_ptr(), ws.numel(),
+                                             y.data_ptr(), s) == 0
+    assert layer.device_status() == binding.MOE_ERR_TIMEOUT
+    g, _ = run_gpu(w, inp, layer=layer)  # asserts a clean status itself
+    check_same_logits_routing(w, inp, g)
+    check_end_to_end(w, inp, g)
+
+
 def _emulated_all_to_all(inputs, splits):
     """What all_to_all_single delivers to each rank q: from every rank r, in
     rank order, the rows r sends to q (splits[r][q] rows after the earlier ones)."""
@@ -527,7 +550,7 @@ def test_exact_ties_go_to_the_lower_index(E, d, mode):
     first on ties), both where a tie straddles the k-th place and where several
     tied experts are all selected."""
     w = WORKLOADS["default"].with_(T=700, E=E, k=4, S=0, d=d, F=256, O=256, capacity_factor=1.0,
-                                   top_k_method="noisy" if mode == "noisy" else "greedy",
+                                   top_k_method="noisy" if mode == "noisy" else "greedy", noise=mode == "noisy",
                                    use_selection_bias=mode == "selection_bias")
     inp = make_inputs(w, "cpu", seed=37)
     groups = [[3, 10, 17], [6, 21]] if E == 24 else [[5, 70, 150], [20, 140]]
@@ -556,3 +579,25 @@ def test_exact_ties_go_to_the_lower_index(E, d, mode):
                 pos = [idx[t].tolist().index(e) for e in sel]
                 assert pos == list(range(pos[0], pos[0] + len(sel))), (t, idx[t])
     assert straddle > 0 and together > 0, (straddle, together)
+
+
+def test_prepared_router_planes():
+    """moe_prepare_router: the router matrix split once into persistent planes
+    gives bit-for-bit the results of the per-forward split with one launch
+    fewer, and after the weights change, a new prepare makes the next forward
+    follow the new matrix."""
+    w = WORKLOADS["e64"].with_(T=900, token_loss=True)
+    inp = make_inputs(w, "cpu", seed=44)
+    g1, layer = run_gpu(w, inp)
+    layer.prepare_router()
+    g2, _ = run_gpu(w, inp, layer=layer)
+    assert g2["launches"] == g1["launches"] - 1
+    for k in ("y", "logits", "gates", "topk_idx", "slot", "count_pre", "f", "p_mean", "l_aux", "l_z", "credit",
+              "expert_loss"):
+        assert np.array_equal(g1[k], g2[k]), k
+    layer.weights["w_gate"].mul_(-0.5)
+    layer.prepare_router()
+    inp2 = dict(inp, w_gate=layer.weights["w_gate"].cpu())
+    g3, _ = run_gpu(w, inp2, layer=layer)
+    check_same_logits_routing(w, inp2, g3)
+    check_end_to_end(w, inp2, g3)
