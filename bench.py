@@ -56,6 +56,7 @@ def parse():
     # Smaller variants of a workload, for profiler captures of the same kernels.
     ap.add_argument("--tokens", type=int, default=None, help="override T (profiling)")
     ap.add_argument("--experts", type=int, default=None, help="override E (profiling)")
+    ap.add_argument("--dff", type=int, default=None, help="override d_ff (profiling the router at full E and d)")
     return ap.parse_args()
 
 
@@ -417,6 +418,8 @@ def run_ours(args):
         w = w.with_(T=args.tokens)
     if args.experts:
         w = w.with_(E=args.experts)
+    if args.dff:
+        w = w.with_(F=args.dff)
     head = measure(w, args, dev, rank, world, headline=True)
     inp = head.pop("inp")
     cpu = None
@@ -434,7 +437,7 @@ def run_ours(args):
     del inp
     torch.cuda.empty_cache()
     extras = {}
-    if args.workload == "e256" and not (args.tokens or args.experts or args.no_extras):
+    if args.workload == "e256" and not (args.tokens or args.experts or args.dff or args.no_extras):
         for name in EXTRA_CONFIGS:
             r = measure(WORKLOADS[name], args, dev, rank, world, headline=False)
             del r["inp"]

@@ -170,9 +170,9 @@ __device__ __forceinline__ void dispatch_scan(const DispatchArgs &a) {
 __global__ void __launch_bounds__(kChunk) dispatch_count_scan_kernel(DispatchArgs a) {
     __shared__ int last;
     dispatch_count(a, blockIdx.x);
-    __threadfence();  // this thread's counts are visible before the chunk is counted
-    __syncthreads();
+    __syncthreads();  // the block's counts, then one device-scope fence publishes them
     if (threadIdx.x == 0) {
+        __threadfence();
         const int old = atomicAdd(a.ctrl + kCtrlDispatchDone, 1);
         last = old == (int)gridDim.x - 1;
         if (last) {

@@ -115,63 +115,88 @@ __device__ __forceinline__ Unit unit_of(const RouterFusedArgs &a, int u) {
 // Logits of the 128 tokens of half tile (m, rank) from the finished units
 // (pieces > 1): sum over the K splits of each expert tile's partials, in split
 // order, plus the bias, written to the logits output. All epilogue threads
-// share the work, four experts of one token per item, every split's load of an
-// item in flight together.
+// share the work, four experts of one token per item; a thread keeps up to 16
+// loads in flight (several items' splits at once), so a half tile costs a few
+// L2 round trips rather than one per item.
 template <int BN>
 __device__ __forceinline__ void merge_half_tile(const RouterFusedArgs &a, int m, int rank, int et) {
     constexpr int kEpiWarps = RCfg<BN>::kEpiWarps;
-    const int E4 = (a.E + 3) / 4;  // items per token
-    const int ks = a.ksplit;
+    constexpr int kNT = kEpiWarps * 32;
+    // Loads in flight per thread: eight, or four with 128-expert tiles (whose
+    // epilogue threads hold 64 running sums).
+    constexpr int kL = BN == 128 ? 4 : 8;
+    const int ks = a.ksplit;                       // 1, 2, 4 or 8
+    const int per_batch = ks >= kL ? 1 : kL / ks;  // items per batch
+    const int E4 = (a.E + 3) / 4;                  // items per token
     const bool vec_out = (a.E & 3) == 0;
-    for (int item = et; item < kTokCta * E4; item += kEpiWarps * 32) {
-        const int i = item / E4, e = (item - i * E4) * 4;
-        const int tl = rank * kTokCta + i;
-        const int t = m * kTokTileR + tl;
-        if (t >= a.T) continue;
-        const int n = e / BN, c = e - n * BN;  // BN is a multiple of 4: the item stays in one tile
-        const float4 *p = reinterpret_cast<const float4 *>(
-            a.part + ((int64_t)((m * a.n_tiles + n) * ks) * kTokTileR + tl) * BN + c);
-        const int64_t stride = (int64_t)kTokTileR * BN / 4;
-        // Splits in batches of four loads, added in split order.
-        float4 h = make_float4(0.f, 0.f, 0.f, 0.f);
-        for (int sp0 = 0; sp0 < ks; sp0 += 4) {
-            float4 v[4];
+    const int64_t stride = (int64_t)kTokTileR * BN / 4;  // float4s between two splits of a tile
+    const int n_items = kTokCta * E4;
+    const int t0 = m * kTokTileR + rank * kTokCta;
+    for (int base = et; base < n_items; base += kNT * per_batch) {
+        // Load slot j = (item base + (j / ks) * kNT, split j % ks); with more
+        // splits than slots, the item's remaining splits are added below.
+        float4 v[kL];
 #pragma unroll
-            for (int j = 0; j < 4; ++j)
-                if (sp0 + j < ks) v[j] = __ldcg(p + (sp0 + j) * stride);
-#pragma unroll
-            for (int j = 0; j < 4; ++j)
-                if (sp0 + j < ks) {
-                    if (sp0 + j == 0) {
-                        h = v[0];
-                    } else {
-                        h.x = __fadd_rn(h.x, v[j].x);
-                        h.y = __fadd_rn(h.y, v[j].y);
-                        h.z = __fadd_rn(h.z, v[j].z);
-                        h.w = __fadd_rn(h.w, v[j].w);
-                    }
-                }
+        for (int j = 0; j < kL; ++j) {
+            const int item = base + (j / ks) * kNT;
+            const int i = item / E4, e = (item - i * E4) * 4;
+            if (item < n_items && t0 + i < a.T) {
+                const int n = e / BN, c = e - n * BN;  // BN is a multiple of 4: one tile per item
+                const float4 *src = reinterpret_cast<const float4 *>(
+                    a.part + ((int64_t)((m * a.n_tiles + n) * ks) * kTokTileR + rank * kTokCta + i) * BN + c);
+                if (j % ks < kL) v[j] = __ldcg(src + (j % ks) * stride);
+            }
         }
-        float hv[4] = {h.x, h.y, h.z, h.w};
-        float *row = a.logits + (int64_t)t * a.E + e;
-        if (a.b_gate)
+        // Sums in split order; an item's logits are written after its last split.
+        float4 h = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-            for (int j = 0; j < 4; ++j)
-                if (e + j < a.E) hv[j] = __fadd_rn(hv[j], __ldg(a.b_gate + e + j));
-        if (vec_out) {
-            *reinterpret_cast<float4 *>(row) = make_float4(hv[0], hv[1], hv[2], hv[3]);
-        } else {
+        for (int j = 0; j < kL; ++j) {
+            const int sp = j % ks;
+            if (sp == 0) {
+                h = v[j];
+            } else {
+                h.x = __fadd_rn(h.x, v[j].x);
+                h.y = __fadd_rn(h.y, v[j].y);
+                h.z = __fadd_rn(h.z, v[j].z);
+                h.w = __fadd_rn(h.w, v[j].w);
+            }
+            if (sp != ks - 1 && j != kL - 1) continue;
+            const int item = base + (j / ks) * kNT;
+            const int i = item / E4, e = (item - i * E4) * 4;
+            if (item >= n_items || t0 + i >= a.T) continue;
+            if (ks > kL) {  // the splits beyond the slots, in order
+                const int n = e / BN, c = e - n * BN;
+                const float4 *src = reinterpret_cast<const float4 *>(
+                    a.part + ((int64_t)((m * a.n_tiles + n) * ks) * kTokTileR + rank * kTokCta + i) * BN + c);
+                for (int sp2 = kL; sp2 < ks; ++sp2) {
+                    const float4 w = __ldcg(src + sp2 * stride);
+                    h.x = __fadd_rn(h.x, w.x);
+                    h.y = __fadd_rn(h.y, w.y);
+                    h.z = __fadd_rn(h.z, w.z);
+                    h.w = __fadd_rn(h.w, w.w);
+                }
+            }
+            float hv[4] = {h.x, h.y, h.z, h.w};
+            if (a.b_gate)
 #pragma unroll
-            for (int j = 0; j < 4; ++j)
-                if (e + j < a.E) row[j] = hv[j];
+                for (int q = 0; q < 4; ++q)
+                    if (e + q < a.E) hv[q] = __fadd_rn(hv[q], __ldg(a.b_gate + e + q));
+            float *row = a.logits + (int64_t)(t0 + i) * a.E + e;
+            if (vec_out) {
+                *reinterpret_cast<float4 *>(row) = make_float4(hv[0], hv[1], hv[2], hv[3]);
+            } else {
+#pragma unroll
+                for (int q = 0; q < 4; ++q)
+                    if (e + q < a.E) row[q] = hv[q];
+            }
         }
     }
 }
 
 // Routes the 128 tokens of half tile (m, rank) from their logits: a warp per
-// token (route_common.cuh), the next token's logits and key addends loaded
-// before the current token is routed; then this warp's per-expert P sums into
-// the shared reduction rows.
+// token (route_common.cuh), the next token's logits (and noise) loaded before
+// the current token is routed; a selection bias, the same for every token, is
+// loaded once. Then this warp's per-expert P sums go to the shared rows.
 template <int BN, int RE>
 __device__ __forceinline__ void route_half_tile(const RouterFusedArgs &a, const RSmem &s, int m, int rank, int ew,
                                                 int lane) {
@@ -179,35 +204,47 @@ __device__ __forceinline__ void route_half_tile(const RouterFusedArgs &a, const 
     float pacc[RE];
 #pragma unroll
     for (int q = 0; q < RE; ++q) pacc[q] = 0.f;
-    auto load = [&](int i, float (&h)[RE], float (&kadd)[RE]) -> bool {
-        const int t = m * kTokTileR + rank * kTokCta + i;
+    const int t0 = m * kTokTileR + rank * kTokCta;
+    const bool has_add = a.noise != nullptr || a.sel_bias != nullptr;
+    float kadd[RE];
+    if (!a.noise) key_addend<RE>(t0, lane, a, kadd);  // the selection bias (or nothing)
+    auto load = [&](int i, float (&h)[RE], float (&nz)[RE]) -> bool {
+        const int t = t0 + i;
         if (i >= kTokCta || t >= a.T) return false;
 #pragma unroll
         for (int q = 0; q < RE; ++q) {
             const int e = lane + 32 * q;
             h[q] = e < a.E ? __ldcg(a.logits + (int64_t)t * a.E + e) : -INFINITY;
+            if (a.noise) nz[q] = e < a.E ? __ldg(a.noise + (int64_t)t * a.E + e) : 0.f;
         }
-        key_addend<RE>(t, lane, a, kadd);
         return true;
     };
-    const bool has_add = a.noise != nullptr || a.sel_bias != nullptr;
-    float h[RE], kadd[RE];
-    if constexpr (RE <= 4) {  // the next token's loads in flight while this one is routed
-        float h2[RE], kadd2[RE];
-        bool have = load(ew, h, kadd);
+    float h[RE], nz[RE];
+    if constexpr (BN < 128) {  // the next token's loads in flight while this one is routed
+        float h2[RE], nz2[RE];
+        bool have = load(ew, h, nz);
         for (int i = ew; have; i += kEpiWarps) {
-            const bool next = load(i + kEpiWarps, h2, kadd2);
-            route_warp<RE>(h, has_add, kadd, m * kTokTileR + rank * kTokCta + i, lane, a, pacc);
+            const bool next = load(i + kEpiWarps, h2, nz2);
+            if (a.noise) {
+                route_warp<RE>(h, has_add, nz, t0 + i, lane, a, pacc);
+            } else {
+                route_warp<RE>(h, has_add, kadd, t0 + i, lane, a, pacc);
+            }
 #pragma unroll
             for (int q = 0; q < RE; ++q) {
                 h[q] = h2[q];
-                kadd[q] = kadd2[q];
+                nz[q] = nz2[q];
             }
             have = next;
         }
-    } else {  // 256 experts: registers are short; each token's loads are already eight in flight
-        for (int i = ew; load(i, h, kadd); i += kEpiWarps)
-            route_warp<RE>(h, has_add, kadd, m * kTokTileR + rank * kTokCta + i, lane, a, pacc);
+    } else {  // 128-expert tiles: the registers go to the running sums; no prefetch
+        for (int i = ew; load(i, h, nz); i += kEpiWarps) {
+            if (a.noise) {
+                route_warp<RE>(h, has_add, nz, t0 + i, lane, a, pacc);
+            } else {
+                route_warp<RE>(h, has_add, kadd, t0 + i, lane, a, pacc);
+            }
+        }
     }
 #pragma unroll
     for (int q = 0; q < RE; ++q) s.red[ew * 256 + lane + 32 * q] = pacc[q];
@@ -387,18 +424,20 @@ __global__ void __launch_bounds__(RCfg<BN>::kThreads, 1)
 #pragma unroll
                 for (int j = 0; j < COLS; j += 4) prow[j / 4] = make_float4(sum[j], sum[j + 1], sum[j + 2], sum[j + 3]);
             }
-            __threadfence();  // this thread's results are visible device-wide before the arrival is counted
-            __syncwarp();
             // Count the unit on the half tile's counter once all epilogue warps
-            // have written; the CTA that completes the half tile routes it.
+            // have written (their arrivals release the writes to the counting
+            // thread, whose device-scope fence then publishes them all); the CTA
+            // that completes the half tile routes it.
+            __syncwarp();
             if (lane == 0) mbar_arrive(s.epi_done);
             if (ew == 0) {
                 int flag = 0;
                 if (lane == 0) {
                     if (mbar_wait(s.epi_done, epi_n & 1u, a.status)) {
+                        __threadfence();
                         const int old = atomicAdd(a.counters + un.m * 2 + static_cast<int>(rank), 1);
                         flag = old == a.n_tiles * a.ksplit - 1 ? 1 : 0;
-                        __threadfence();
+                        __threadfence();  // the other CTAs' partials are read after this
                     } else {
                         flag = -1;
                     }
@@ -407,10 +446,10 @@ __global__ void __launch_bounds__(RCfg<BN>::kThreads, 1)
                 }
             }
             ++epi_n;
-            int flag = 0;
-            if (lane == 0)
-                flag = mbar_wait(s.route_go, go_n & 1u, a.status) ? *reinterpret_cast<volatile int32_t *>(s.flag) : -1;
-            flag = __shfl_sync(0xffffffffu, flag, 0);
+            // Every lane acquires route_go: the routing below reads partials
+            // that other CTAs wrote before their arrivals were counted.
+            int flag = mbar_wait_all_lanes(s.route_go, go_n & 1u, a.status) ? *reinterpret_cast<volatile int32_t *>(s.flag)
+                                                                            : -1;
             if (flag < 0) {
                 ok = false;
                 break;
@@ -418,26 +457,26 @@ __global__ void __launch_bounds__(RCfg<BN>::kThreads, 1)
             if (flag) {
                 if (a.n_tiles * a.ksplit > 1) {
                     merge_half_tile<BN>(a, un.m, static_cast<int>(rank), ew * 32 + lane);
-                    // Every warp's logits written before any warp routes from them.
-                    __threadfence();
+                    // Every warp's logits written before any lane routes from them.
+                    __threadfence_block();
                     __syncwarp();
                     if (lane == 0) mbar_arrive(s.epi_done);
-                    int got = 1;
-                    if (lane == 0) got = mbar_wait(s.epi_done, epi_n & 1u, a.status) ? 1 : 0;
+                    const bool got = mbar_wait_all_lanes(s.epi_done, epi_n & 1u, a.status);
                     ++epi_n;
-                    if (!__shfl_sync(0xffffffffu, got, 0)) {
+                    if (!got) {
                         ok = false;
                         break;
                     }
                 }
                 if (a.route) {
                     route_half_tile<BN, RE>(a, s, un.m, static_cast<int>(rank), ew, lane);
-                    // The half tile's P sums: every warp's row, added in warp order.
+                    // The half tile's P sums: every warp's row, added in warp order
+                    // (every lane acquires the rows the other warps wrote).
+                    __syncwarp();
                     if (lane == 0) mbar_arrive(s.epi_done);
-                    int got = 1;
-                    if (lane == 0) got = mbar_wait(s.epi_done, epi_n & 1u, a.status) ? 1 : 0;
+                    const bool got = mbar_wait_all_lanes(s.epi_done, epi_n & 1u, a.status);
                     ++epi_n;
-                    if (!__shfl_sync(0xffffffffu, got, 0)) {
+                    if (!got) {
                         ok = false;
                         break;
                     }
@@ -530,14 +569,15 @@ int router_fused_bn(int E) { return router_fused_epad(E) < 128 ? router_fused_ep
 int router_fused_mtiles(int T) { return (T + kTokTileR - 1) / kTokTileR; }
 
 // K splits: the fewest waves of units per unit of work, ceil(units ks / pairs) / ks,
-// over ks = 1..8 with at least one drain group per split; ties keep fewer splits.
+// over ks = 1, 2, 4, 8 with at least one drain group per split; ties keep fewer
+// splits.
 int router_fused_ksplit(int T, int E, int d, int num_pairs) {
     const int units = router_fused_mtiles(T) * (router_fused_epad(E) / router_fused_bn(E));
     const int dblocks = d / kBK;
     if (units <= 0 || num_pairs <= 0) return 1;
     int best = 1;
     double best_cost = 1e30;
-    for (int ks = 1; ks <= 8 && ks <= dblocks / kDrain; ++ks) {
+    for (int ks = 1; ks <= 8 && ks <= dblocks / kDrain; ks *= 2) {
         const double cost = (double)((units * ks + num_pairs - 1) / num_pairs) / ks;
         if (cost < best_cost - 1e-9) {
             best_cost = cost;
