@@ -159,11 +159,15 @@ Plan make_plan(const moe_layer &L, int T) {
     p.max_narrow_tiles = (int)std::min<int64_t>(routed / kNarrowTile + E, routed / kRowBlock) +
                          S * (int)((p.T_pad + kNarrowTile - 1) / kNarrowTile);
     // bf16 linear routers route in the fused tensor-core kernel (a P-sum row
-    // per half tile of 128 tokens); the MLP gate and fp32 layers route in the
+    // per CTA of its launch); the MLP gate and fp32 layers route in the
     // CUDA-core router kernel.
     const bool fused_routes = c.dtype == MOE_DTYPE_BF16 && !c.use_mlp_gater;
-    p.n_mtiles = c.dtype == MOE_DTYPE_BF16 ? router_fused_mtiles(T) : 0;
-    p.n_stat_chunks = fused_routes ? 2 * p.n_mtiles : router_psum_blocks(T);
+    const int E_tc = c.use_mlp_gater ? c.gater_hidden_dim : E;  // rows of the tensor-core router matrix
+    const bool tc = c.dtype == MOE_DTYPE_BF16;
+    p.n_mtiles = tc ? router_fused_mtiles(T) : 0;
+    p.ksplit = tc ? router_fused_ksplit(T, E_tc, c.input_dim, L.router_pairs) : 1;
+    const int pieces = tc ? p.ksplit * (router_fused_epad(E_tc) / router_fused_bn(E_tc)) : 1;
+    p.n_stat_chunks = fused_routes ? router_fused_ctas(p.n_mtiles * pieces, L.router_pairs) : router_psum_blocks(T);
     const int64_t n_items = c.capacity_priority == MOE_PRIORITY_RANK ? (int64_t)k * T : T;
     p.n_chunks = (int)((n_items + 255) / 256);
     const size_t es = c.dtype == MOE_DTYPE_BF16 ? 2 : 4;
@@ -174,7 +178,7 @@ Plan make_plan(const moe_layer &L, int T) {
         return o;
     };
     p.o_ctrl = take(kCtrlWords * 4);
-    p.o_rcnt = take((size_t)2 * p.n_mtiles * 4);  // the fused router's arrival counters
+    p.o_rcnt = take(16);                           // the fused router's grid-barrier counter
     p.ctrl_bytes = off - p.o_ctrl;                // control words and counters: zeroed every forward
     p.o_logits = take((size_t)T * E * 4);
     p.o_idx = take((size_t)T * k * 4);
@@ -198,11 +202,7 @@ Plan make_plan(const moe_layer &L, int T) {
     p.o_gsorted = take((size_t)T * k * 4);
     p.o_rownorm = take(c.credit_norm == MOE_CREDIT_HIDDEN ? (size_t)p.R_routed_max * 4 : 0);
     p.o_credit = take((size_t)T * k * 4);
-    const int E_tc = c.use_mlp_gater ? c.gater_hidden_dim : E;  // rows of the tensor-core router matrix
-    const bool tc = c.dtype == MOE_DTYPE_BF16;
     p.o_wsplit = take(tc ? (size_t)router_fused_epad(E_tc) * 3 * c.input_dim * 2 : 0);
-    p.ksplit = tc ? router_fused_ksplit(T, E_tc, c.input_dim, L.router_pairs) : 1;
-    const int pieces = tc ? p.ksplit * (router_fused_epad(E_tc) / router_fused_bn(E_tc)) : 1;
     p.o_gz = take(c.use_mlp_gater ? (size_t)T * c.gater_hidden_dim * 4 : 0);
     p.o_lpart = take(pieces > 1 ? (size_t)p.n_mtiles * 256 * router_fused_epad(E_tc) * p.ksplit * 4 : 0);
     p.o_xp = take(c.dtype == MOE_DTYPE_BF16 ? (size_t)p.R_routed_max * c.input_dim * es : 0);

@@ -30,10 +30,11 @@ struct RouterArgs {
 int router_psum_blocks(int T);
 cudaError_t launch_router(const RouterArgs &a, cudaStream_t s, int *launches);
 
-// Router of bf16 layers in one kernel (router_fused.cu): logits on the tensor
-// cores from three bf16 planes of W_g, then (route = 1) softmax, log-partition,
-// keys, top-k, gates and the per-half-tile P sums. Units: token tiles of 256,
-// expert tiles of BN, ksplit K splits.
+// Router of bf16 layers in one cooperative kernel (router_fused.cu): logits on
+// the tensor cores from three bf16 planes of W_g, then, after a grid-wide
+// barrier, (route = 1) softmax, log-partition, keys, top-k, gates and a row of
+// P sums per CTA. Units: token tiles of 256, expert tiles of BN, ksplit K
+// splits.
 struct RouterFusedArgs {
     const float *b_gate;    // [E] or null
     const float *noise;     // [T][E] or null (added to the selection key only)
@@ -45,9 +46,9 @@ struct RouterFusedArgs {
     int32_t *idx;           // [T][k]
     float *gates;           // [T][k]
     float *lse;             // [T]
-    float *psum_part;       // [2 n_mtiles][E]: P summed over each half tile of 128 tokens
+    float *psum_part;       // [router_fused_ctas][E]: P summed over each CTA's tokens
     float *part;            // [n_mtiles n_tiles ksplit][256][BN] partial sums when n_tiles ksplit > 1
-    int32_t *counters;      // [2 n_mtiles], zero before the launch
+    int32_t *counters;      // [1] grid-barrier counter, zero before the launch
     uint32_t *status;
     int num_pairs;          // CTA pairs to launch at most
 };
@@ -56,6 +57,8 @@ int router_fused_bn(int E);      // expert tile: E_pad up to 128
 int router_fused_mtiles(int T);  // token tiles of 256
 int router_fused_ksplit(int T, int E, int d, int num_pairs);
 int router_fused_max_pairs(int num_sms);
+// CTAs the launch has for `units` units (2 per pair): the rows of psum_part.
+int router_fused_ctas(int units, int num_pairs);
 // W_g [E][d] fp32 -> w_split [E_pad][3d] bf16: planes hi | mid | lo, rows >= E zero.
 cudaError_t launch_router_split(const float *w_gate, int E, int E_pad, int d, __nv_bfloat16 *w_split, int num_sms,
                                 cudaStream_t s, int *launches);

@@ -25,18 +25,22 @@
 // so x is read once for all three planes. Each CTA's TMEM holds its 128 tokens x
 // BN experts in two partial buffers so that the MMAs run ahead of the drains.
 //
-// Routing. Each CTA writes its finished unit (fp32 partial sums, or the logits
-// themselves when a token tile is one unit) and counts it on its half tile's
-// arrival counter; the CTA that completes a half tile (128 tokens) adds the
-// partials in a fixed order (expert tile, then K split), adds the bias, writes
-// the logits and routes the 128 tokens, a warp per token (route_common.cuh).
-// Nothing waits for another CTA: the last to arrive does the work.
+// Routing. Two phases in the one launch. Phase A: every unit's CTA pair
+// writes its result (the logits themselves when a token tile is one unit,
+// otherwise fp32 partial sums). A grid-wide barrier follows (the launch is
+// cooperative, so every CTA is resident; the wait is bounded). Phase B: every
+// warp of every CTA takes tokens of its CTA's contiguous share, adds each
+// token's partials in a fixed order (K split), adds the bias, writes the
+// logits and routes the token (route_common.cuh), so the routing is spread over
+// all SMs; each CTA writes one row of per-expert P sums (its warps' sums added
+// in warp order).
 //
 // Roles (320 threads per CTA): warp 0 loads (TMA), warp 1 owns TMEM and, in
 // the leader, issues the MMAs; warps 2..9 drain the accumulators (two warps per
-// TMEM lane quarter, BN/2 columns each) and route. Every wait is bounded; on a
-// timeout the roles stop, in-flight copies and MMAs are drained, both CTAs meet
-// at the cluster barrier and TMEM is freed.
+// TMEM lane quarter, BN/2 columns each). In phase B all ten warps route. Every
+// wait is bounded; on a timeout the roles stop, in-flight copies and MMAs are
+// drained, phase B is skipped, both CTAs meet at the cluster barrier and TMEM is
+// freed.
 #include "moe_common.cuh"
 #include "moe_kernels.cuh"
 #include "route_common.cuh"
@@ -59,7 +63,8 @@ struct RCfg {
     static constexpr int kStage = kA + 3 * kBHalf;
     static constexpr int kStages = (200 * 1024) / kStage < 8 ? (200 * 1024) / kStage : 8;
     static constexpr int kTmemCols = 2 * BN;              // two partial buffers
-    static constexpr int kRedBytes = kEpiWarps * 256 * 4;  // per-warp P sums of a half tile
+    static constexpr int kWarps = kThreads / 32;
+    static constexpr int kRedBytes = kWarps * 256 * 4;     // per-warp P sums of phase B
     static constexpr int kCols = BN / (kEpiWarps / 4);     // accumulator columns per epilogue thread
     static constexpr int kSmem = 1024 + kStages * kStage + kRedBytes + 512;
     static_assert(BN == 32 || BN == 64 || BN == 128, "expert tile");
@@ -70,9 +75,8 @@ struct RCfg {
 struct RSmem {
     uint8_t *stages;
     float *red;
-    uint64_t *full, *empty, *tfull, *tempty, *mma_done, *epi_done, *route_go;
+    uint64_t *full, *empty, *tfull, *tempty, *mma_done;
     uint32_t *tmem_slot;
-    int32_t *flag;
 };
 
 template <int BN>
@@ -87,10 +91,7 @@ __device__ __forceinline__ RSmem rcarve(uint8_t *raw) {
     s.tfull = s.empty + C::kStages;
     s.tempty = s.tfull + 2;
     s.mma_done = s.tempty + 2;
-    s.epi_done = s.mma_done + 1;
-    s.route_go = s.epi_done + 1;
-    s.tmem_slot = reinterpret_cast<uint32_t *>(s.route_go + 1);
-    s.flag = reinterpret_cast<int32_t *>(s.tmem_slot + 2);
+    s.tmem_slot = reinterpret_cast<uint32_t *>(s.mma_done + 1);
     return s;
 }
 
@@ -112,142 +113,112 @@ __device__ __forceinline__ Unit unit_of(const RouterFusedArgs &a, int u) {
     return r;
 }
 
-// Logits of the 128 tokens of half tile (m, rank) from the finished units
-// (pieces > 1): sum over the K splits of each expert tile's partials, in split
-// order, plus the bias, written to the logits output. All epilogue threads
-// share the work, four experts of one token per item; a thread keeps up to 16
-// loads in flight (several items' splits at once), so a half tile costs a few
-// L2 round trips rather than one per item.
-template <int BN>
-__device__ __forceinline__ void merge_half_tile(const RouterFusedArgs &a, int m, int rank, int et) {
-    constexpr int kEpiWarps = RCfg<BN>::kEpiWarps;
-    constexpr int kNT = kEpiWarps * 32;
-    // Loads in flight per thread: eight, or four with 128-expert tiles (whose
-    // epilogue threads hold 64 running sums).
-    constexpr int kL = BN == 128 ? 4 : 8;
-    const int ks = a.ksplit;                       // 1, 2, 4 or 8
-    const int per_batch = ks >= kL ? 1 : kL / ks;  // items per batch
-    const int E4 = (a.E + 3) / 4;                  // items per token
-    const bool vec_out = (a.E & 3) == 0;
-    const int64_t stride = (int64_t)kTokTileR * BN / 4;  // float4s between two splits of a tile
-    const int n_items = kTokCta * E4;
-    const int t0 = m * kTokTileR + rank * kTokCta;
-    for (int base = et; base < n_items; base += kNT * per_batch) {
-        // Load slot j = (item base + (j / ks) * kNT, split j % ks); with more
-        // splits than slots, the item's remaining splits are added below.
-        float4 v[kL];
-#pragma unroll
-        for (int j = 0; j < kL; ++j) {
-            const int item = base + (j / ks) * kNT;
-            const int i = item / E4, e = (item - i * E4) * 4;
-            if (item < n_items && t0 + i < a.T) {
-                const int n = e / BN, c = e - n * BN;  // BN is a multiple of 4: one tile per item
-                const float4 *src = reinterpret_cast<const float4 *>(
-                    a.part + ((int64_t)((m * a.n_tiles + n) * ks) * kTokTileR + rank * kTokCta + i) * BN + c);
-                if (j % ks < kL) v[j] = __ldcg(src + (j % ks) * stride);
-            }
-        }
-        // Sums in split order; an item's logits are written after its last split.
-        float4 h = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-        for (int j = 0; j < kL; ++j) {
-            const int sp = j % ks;
-            if (sp == 0) {
-                h = v[j];
-            } else {
-                h.x = __fadd_rn(h.x, v[j].x);
-                h.y = __fadd_rn(h.y, v[j].y);
-                h.z = __fadd_rn(h.z, v[j].z);
-                h.w = __fadd_rn(h.w, v[j].w);
-            }
-            if (sp != ks - 1 && j != kL - 1) continue;
-            const int item = base + (j / ks) * kNT;
-            const int i = item / E4, e = (item - i * E4) * 4;
-            if (item >= n_items || t0 + i >= a.T) continue;
-            if (ks > kL) {  // the splits beyond the slots, in order
-                const int n = e / BN, c = e - n * BN;
-                const float4 *src = reinterpret_cast<const float4 *>(
-                    a.part + ((int64_t)((m * a.n_tiles + n) * ks) * kTokTileR + rank * kTokCta + i) * BN + c);
-                for (int sp2 = kL; sp2 < ks; ++sp2) {
-                    const float4 w = __ldcg(src + sp2 * stride);
-                    h.x = __fadd_rn(h.x, w.x);
-                    h.y = __fadd_rn(h.y, w.y);
-                    h.z = __fadd_rn(h.z, w.z);
-                    h.w = __fadd_rn(h.w, w.w);
-                }
-            }
-            float hv[4] = {h.x, h.y, h.z, h.w};
-            if (a.b_gate)
-#pragma unroll
-                for (int q = 0; q < 4; ++q)
-                    if (e + q < a.E) hv[q] = __fadd_rn(hv[q], __ldg(a.b_gate + e + q));
-            float *row = a.logits + (int64_t)(t0 + i) * a.E + e;
-            if (vec_out) {
-                *reinterpret_cast<float4 *>(row) = make_float4(hv[0], hv[1], hv[2], hv[3]);
-            } else {
-#pragma unroll
-                for (int q = 0; q < 4; ++q)
-                    if (e + q < a.E) row[q] = hv[q];
-            }
-        }
-    }
-}
-
-// Routes the 128 tokens of half tile (m, rank) from their logits: a warp per
-// token (route_common.cuh), the next token's logits (and noise) loaded before
-// the current token is routed; a selection bias, the same for every token, is
-// loaded once. Then this warp's per-expert P sums go to the shared rows.
+// Phase B for tokens [t_begin, t_end): a warp per token. The token's logits
+// are read (one unit per tile) or formed from the partials of its K splits,
+// added in split order two splits' loads at a time, plus the bias, and
+// written; then route_warp. A selection bias, the same for every token, is
+// loaded once. Leaves this warp's per-expert P sums in red[warp][.].
 template <int BN, int RE>
-__device__ __forceinline__ void route_half_tile(const RouterFusedArgs &a, const RSmem &s, int m, int rank, int ew,
-                                                int lane) {
-    constexpr int kEpiWarps = RCfg<BN>::kEpiWarps;
+__device__ __forceinline__ void route_tokens(const RouterFusedArgs &a, float *red, int warp, int nwarps, int lane,
+                                             int t_begin, int t_end) {
     float pacc[RE];
 #pragma unroll
     for (int q = 0; q < RE; ++q) pacc[q] = 0.f;
-    const int t0 = m * kTokTileR + rank * kTokCta;
+    const int ks = a.ksplit;
+    const bool merged = a.n_tiles * ks == 1;
     const bool has_add = a.noise != nullptr || a.sel_bias != nullptr;
     float kadd[RE];
-    if (!a.noise) key_addend<RE>(t0, lane, a, kadd);  // the selection bias (or nothing)
-    auto load = [&](int i, float (&h)[RE], float (&nz)[RE]) -> bool {
-        const int t = t0 + i;
-        if (i >= kTokCta || t >= a.T) return false;
+    if (!a.noise) key_addend<RE>(0, lane, a, kadd);  // the selection bias (or nothing)
+    const int64_t split_stride = (int64_t)kTokTileR * BN;
+    for (int t = t_begin + warp; t < t_end; t += nwarps) {
+        float h[RE];
+        if (merged) {
 #pragma unroll
-        for (int q = 0; q < RE; ++q) {
-            const int e = lane + 32 * q;
-            h[q] = e < a.E ? __ldcg(a.logits + (int64_t)t * a.E + e) : -INFINITY;
-            if (a.noise) nz[q] = e < a.E ? __ldg(a.noise + (int64_t)t * a.E + e) : 0.f;
-        }
-        return true;
-    };
-    float h[RE], nz[RE];
-    if constexpr (BN < 128) {  // the next token's loads in flight while this one is routed
-        float h2[RE], nz2[RE];
-        bool have = load(ew, h, nz);
-        for (int i = ew; have; i += kEpiWarps) {
-            const bool next = load(i + kEpiWarps, h2, nz2);
-            if (a.noise) {
-                route_warp<RE>(h, has_add, nz, t0 + i, lane, a, pacc);
-            } else {
-                route_warp<RE>(h, has_add, kadd, t0 + i, lane, a, pacc);
+            for (int q = 0; q < RE; ++q) {
+                const int e = lane + 32 * q;
+                h[q] = e < a.E ? __ldcg(a.logits + (int64_t)t * a.E + e) : -INFINITY;
+            }
+        } else {
+            const int m = t / kTokTileR, tl = t - m * kTokTileR;
+            int64_t off[RE];
+#pragma unroll
+            for (int q = 0; q < RE; ++q) {
+                const int e = lane + 32 * q;
+                const int n = e / BN, c = e - n * BN;
+                off[q] = ((int64_t)((m * a.n_tiles + n) * ks) * kTokTileR + tl) * BN + c;
+            }
+            for (int sp = 0; sp < ks; sp += 2) {
+                float v0[RE], v1[RE];
+#pragma unroll
+                for (int q = 0; q < RE; ++q) {
+                    const bool in = lane + 32 * q < a.E;
+                    v0[q] = in ? __ldcg(a.part + off[q] + sp * split_stride) : 0.f;
+                    v1[q] = in && sp + 1 < ks ? __ldcg(a.part + off[q] + (sp + 1) * split_stride) : 0.f;
+                }
+#pragma unroll
+                for (int q = 0; q < RE; ++q) {
+                    h[q] = sp == 0 ? v0[q] : __fadd_rn(h[q], v0[q]);
+                    if (sp + 1 < ks) h[q] = __fadd_rn(h[q], v1[q]);
+                }
             }
 #pragma unroll
             for (int q = 0; q < RE; ++q) {
-                h[q] = h2[q];
-                nz[q] = nz2[q];
+                const int e = lane + 32 * q;
+                if (e < a.E) {
+                    if (a.b_gate) h[q] = __fadd_rn(h[q], __ldg(a.b_gate + e));
+                    a.logits[(int64_t)t * a.E + e] = h[q];
+                } else {
+                    h[q] = -INFINITY;
+                }
             }
-            have = next;
         }
-    } else {  // 128-expert tiles: the registers go to the running sums; no prefetch
-        for (int i = ew; load(i, h, nz); i += kEpiWarps) {
-            if (a.noise) {
-                route_warp<RE>(h, has_add, nz, t0 + i, lane, a, pacc);
-            } else {
-                route_warp<RE>(h, has_add, kadd, t0 + i, lane, a, pacc);
+        if (!a.route) continue;
+        if (a.noise) {
+            float nz[RE];
+#pragma unroll
+            for (int q = 0; q < RE; ++q) {
+                const int e = lane + 32 * q;
+                nz[q] = e < a.E ? __ldg(a.noise + (int64_t)t * a.E + e) : 0.f;
             }
+            route_warp<RE>(h, has_add, nz, t, lane, a, pacc);
+        } else {
+            route_warp<RE>(h, has_add, kadd, t, lane, a, pacc);
         }
     }
 #pragma unroll
-    for (int q = 0; q < RE; ++q) s.red[ew * 256 + lane + 32 * q] = pacc[q];
+    for (int q = 0; q < RE; ++q) red[warp * 256 + lane + 32 * q] = pacc[q];
+}
+
+// Grid-wide barrier of the cooperative launch: every CTA counts itself once
+// its phase A writes are done and waits (bounded) until all have. Returns the
+// same verdict in every thread: true if all CTAs arrived and no bounded wait
+// anywhere gave up (phase B may run), false otherwise.
+__device__ __forceinline__ bool grid_barrier(int32_t *counter, uint32_t *status) {
+    __shared__ int go_s;
+    __syncthreads();  // every role of this CTA is done with phase A
+    if (threadIdx.x == 0) {
+        __threadfence();  // publishes the CTA's results (observed through the barrier above)
+        atomicAdd(counter, 1);
+        int go = 1;
+        const uint64_t t0 = global_timer_ns();
+        while (*reinterpret_cast<volatile int32_t *>(counter) < (int)gridDim.x) {
+            if (*reinterpret_cast<volatile uint32_t *>(status) != kDevOk) {
+                go = 0;
+                break;
+            }
+            if (global_timer_ns() - t0 > kWaitLimitNs) {
+                atomicOr(status, kDevTimeout);
+                go = 0;
+                break;
+            }
+            __nanosleep(64);
+        }
+        __threadfence();  // the other CTAs' results are read after this
+        if (*reinterpret_cast<volatile uint32_t *>(status) != kDevOk) go = 0;
+        go_s = go;
+    }
+    __syncthreads();
+    return go_s != 0;
 }
 
 template <int BN, int RE>
@@ -277,8 +248,6 @@ __global__ void __launch_bounds__(RCfg<BN>::kThreads, 1)
             mbar_init(&s.tempty[i], 2 * kEpiWarps);  // the epilogue warps of both CTAs
         }
         mbar_init(s.mma_done, 1);
-        mbar_init(s.epi_done, kEpiWarps);
-        mbar_init(s.route_go, 1);
         fence_barrier_init();
     }
     if (warp == 1) {
@@ -366,14 +335,12 @@ __global__ void __launch_bounds__(RCfg<BN>::kThreads, 1)
             mbar_wait_drain(s.mma_done, 0u);
         }
     } else {
-        // ------------------------------------------------------------ epilogue + routing
+        // ------------------------------------------------------------ epilogue (phase A)
         const int ew = warp - 2;
         const int q = warp & 3;                  // TMEM lane quarter this warp may access
         const int col0 = (ew >> 2) * COLS;       // this warp's columns of the expert tile
-        // Phases completed so far of epi_done (once per unit, once more per
-        // routed half tile) and of route_go (once per unit).
-        uint32_t gcount = 0, epi_n = 0, go_n = 0;
-        for (int u = pair; u < total && ok; u += n_pairs, ++go_n) {
+        uint32_t gcount = 0;
+        for (int u = pair; u < total && ok; u += n_pairs) {
             const Unit un = unit_of(a, u);
             float sum[COLS];
 #pragma unroll
@@ -408,7 +375,8 @@ __global__ void __launch_bounds__(RCfg<BN>::kThreads, 1)
                 if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(&s.tempty[buf]), 0));
             }
             if (!ok) break;
-            // The finished unit: logits (one unit per tile) or partial sums.
+            // The finished unit: the logits (bias added) when a token tile is
+            // one unit, otherwise this split's partial sums.
             const int tl = static_cast<int>(rank) * kTokCta + q * 32 + lane;
             const int t = un.m * kTokTileR + tl;
             const int e0 = un.n * BN + col0;
@@ -424,80 +392,30 @@ __global__ void __launch_bounds__(RCfg<BN>::kThreads, 1)
 #pragma unroll
                 for (int j = 0; j < COLS; j += 4) prow[j / 4] = make_float4(sum[j], sum[j + 1], sum[j + 2], sum[j + 3]);
             }
-            // Count the unit on the half tile's counter once all epilogue warps
-            // have written (their arrivals release the writes to the counting
-            // thread, whose device-scope fence then publishes them all); the CTA
-            // that completes the half tile routes it.
-            __syncwarp();
-            if (lane == 0) mbar_arrive(s.epi_done);
-            if (ew == 0) {
-                int flag = 0;
-                if (lane == 0) {
-                    if (mbar_wait(s.epi_done, epi_n & 1u, a.status)) {
-                        __threadfence();
-                        const int old = atomicAdd(a.counters + un.m * 2 + static_cast<int>(rank), 1);
-                        flag = old == a.n_tiles * a.ksplit - 1 ? 1 : 0;
-                        __threadfence();  // the other CTAs' partials are read after this
-                    } else {
-                        flag = -1;
-                    }
-                    *s.flag = flag;
-                    mbar_arrive(s.route_go);
-                }
-            }
-            ++epi_n;
-            // Every lane acquires route_go: the routing below reads partials
-            // that other CTAs wrote before their arrivals were counted.
-            int flag = mbar_wait_all_lanes(s.route_go, go_n & 1u, a.status) ? *reinterpret_cast<volatile int32_t *>(s.flag)
-                                                                            : -1;
-            if (flag < 0) {
-                ok = false;
-                break;
-            }
-            if (flag) {
-                if (a.n_tiles * a.ksplit > 1) {
-                    merge_half_tile<BN>(a, un.m, static_cast<int>(rank), ew * 32 + lane);
-                    // Every warp's logits written before any lane routes from them.
-                    __threadfence_block();
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(s.epi_done);
-                    const bool got = mbar_wait_all_lanes(s.epi_done, epi_n & 1u, a.status);
-                    ++epi_n;
-                    if (!got) {
-                        ok = false;
-                        break;
-                    }
-                }
-                if (a.route) {
-                    route_half_tile<BN, RE>(a, s, un.m, static_cast<int>(rank), ew, lane);
-                    // The half tile's P sums: every warp's row, added in warp order
-                    // (every lane acquires the rows the other warps wrote).
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(s.epi_done);
-                    const bool got = mbar_wait_all_lanes(s.epi_done, epi_n & 1u, a.status);
-                    ++epi_n;
-                    if (!got) {
-                        ok = false;
-                        break;
-                    }
-                    float *prow = a.psum_part + (int64_t)(un.m * 2 + static_cast<int>(rank)) * a.E;
-                    for (int e = ew * 32 + lane; e < a.E; e += kEpiWarps * 32) {
-                        float v = 0.f;
-#pragma unroll
-                        for (int w = 0; w < kEpiWarps; ++w) v += s.red[w * 256 + e];
-                        prow[e] = v;
-                    }
-                    // s.red is written again only by a later routing, which
-                    // starts after a route_go phase that needs every warp's
-                    // epi_done arrival, made after this loop.
-                }
-            }
         }
     }
 
     // A role that gave up may leave its own TMA loads in flight; give them a
     // millisecond to land before the pair meets.
     if (!ok || *reinterpret_cast<volatile uint32_t *>(a.status) != kDevOk) spin_ns(1000000ull);
+
+    // ---------------------------------------------------------------- phase B
+    if (grid_barrier(a.counters, a.status)) {
+        const int nb = gridDim.x;
+        const int chunk = (a.T + nb - 1) / nb;
+        const int t_begin = min(a.T, (int)blockIdx.x * chunk), t_end = min(a.T, t_begin + chunk);
+        route_tokens<BN, RE>(a, s.red, warp, C::kWarps, lane, t_begin, t_end);
+        if (a.route) {
+            __syncthreads();
+            // This CTA's row of P sums: the warps' sums added in warp order.
+            for (int e = threadIdx.x; e < a.E; e += C::kThreads) {
+                float v = 0.f;
+#pragma unroll
+                for (int w = 0; w < C::kWarps; ++w) v += s.red[w * 256 + e];
+                a.psum_part[(int64_t)blockIdx.x * a.E + e] = v;
+            }
+        }
+    }
     tc_fence_before_sync();
     cluster_sync_all();
     tc_fence_after_sync();
@@ -513,19 +431,22 @@ cudaError_t launch_cfg(const CUtensorMap &mx, const CUtensorMap &mw, const Route
     cudaError_t e = set_smem_limit_once<router_fused_kernel<BN, RE>>(kSmem);
     if (e != cudaSuccess) return e;
     const int total = a.n_mtiles * a.n_tiles * a.ksplit;
-    const int pairs = total < a.num_pairs ? total : a.num_pairs;
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(2 * pairs, 1, 1);
+    cfg.gridDim = dim3(router_fused_ctas(total, a.num_pairs), 1, 1);
     cfg.blockDim = dim3(RCfg<BN>::kThreads, 1, 1);
     cfg.dynamicSmemBytes = kSmem;
     cfg.stream = s;
-    cudaLaunchAttribute attr[1];
+    // Cooperative: phase B starts after a grid-wide barrier, which needs every
+    // CTA resident at once (the grid is at most the co-resident pairs).
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = 2;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeCooperative;
+    attr[1].val.cooperative = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = 2;
     return cudaLaunchKernelEx(&cfg, router_fused_kernel<BN, RE>, mx, mw, a);
 }
 
@@ -586,6 +507,8 @@ int router_fused_ksplit(int T, int E, int d, int num_pairs) {
     }
     return best;
 }
+
+int router_fused_ctas(int units, int num_pairs) { return 2 * (units < num_pairs ? units : num_pairs); }
 
 int router_fused_max_pairs(int num_sms) {
     cudaLaunchConfig_t cfg = {};
