@@ -75,7 +75,7 @@ struct RCfg {
 struct RSmem {
     uint8_t *stages;
     float *red;
-    uint64_t *full, *empty, *tfull, *tempty, *mma_done;
+    uint64_t *full, *empty, *tfull, *tempty, *drained, *mma_done;
     uint32_t *tmem_slot;
 };
 
@@ -90,7 +90,8 @@ __device__ __forceinline__ RSmem rcarve(uint8_t *raw) {
     s.empty = s.full + C::kStages;
     s.tfull = s.empty + C::kStages;
     s.tempty = s.tfull + 2;
-    s.mma_done = s.tempty + 2;
+    s.drained = s.tempty + 2;
+    s.mma_done = s.drained + 2;
     s.tmem_slot = reinterpret_cast<uint32_t *>(s.mma_done + 1);
     return s;
 }
@@ -245,7 +246,8 @@ __global__ void __launch_bounds__(RCfg<BN>::kThreads, 1)
         }
         for (int i = 0; i < 2; ++i) {
             mbar_init(&s.tfull[i], 1);
-            mbar_init(&s.tempty[i], 2 * kEpiWarps);  // the epilogue warps of both CTAs
+            mbar_init(&s.tempty[i], 2);          // one forwarded arrival from each CTA
+            mbar_init(&s.drained[i], kEpiWarps);  // this CTA's epilogue warps
         }
         mbar_init(s.mma_done, 1);
         fence_barrier_init();
@@ -370,9 +372,20 @@ __global__ void __launch_bounds__(RCfg<BN>::kThreads, 1)
                         sum[c0 + j] =
                             g0 == un.kb0 ? __uint_as_float(r[j]) : __fadd_rn(sum[c0 + j], __uint_as_float(r[j]));
                 }
+                // The buffer is free once every epilogue warp of both CTAs has
+                // read it: the warps arrive on this CTA's drained barrier and
+                // one thread forwards a single arrival to the leader's tempty.
                 tc_fence_before_sync();
                 __syncwarp();
-                if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(&s.tempty[buf]), 0));
+                if (lane == 0) mbar_arrive(&s.drained[buf]);
+                if (ew == 0 && lane == 0) {
+                    if (mbar_wait(&s.drained[buf], use & 1u, a.status))
+                        mbar_arrive_cluster(mapa_shared(smem_u32(&s.tempty[buf]), 0));
+                    else
+                        ok = false;
+                }
+                ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+                if (!ok) break;
             }
             if (!ok) break;
             // The finished unit: the logits (bias added) when a token tile is
