@@ -114,77 +114,104 @@ __device__ __forceinline__ Unit unit_of(const RouterFusedArgs &a, int u) {
     return r;
 }
 
-// Phase B for tokens [t_begin, t_end): a warp per token. The token's logits
-// are read (one unit per tile) or formed from the partials of its K splits,
-// added in split order two splits' loads at a time, plus the bias, and
-// written; then route_warp. A selection bias, the same for every token, is
-// loaded once. Leaves this warp's per-expert P sums in red[warp][.].
+// Phase B for tokens [t_begin, t_end): a warp routes two tokens at a time
+// (t and t + nwarps, interleaved by route_warp_n). A token's logits are read
+// (one unit per tile) or formed from the partials of its K splits, added in
+// split order two splits' loads at a time, plus the bias, and written. A
+// selection bias, the same for every token, is loaded once. Leaves this
+// warp's per-expert P sums in red[warp][.].
 template <int BN, int RE>
 __device__ __forceinline__ void route_tokens(const RouterFusedArgs &a, float *red, int warp, int nwarps, int lane,
                                              int t_begin, int t_end) {
+    constexpr int NT = 2;  // tokens a warp routes at once
     float pacc[RE];
 #pragma unroll
     for (int q = 0; q < RE; ++q) pacc[q] = 0.f;
     const int ks = a.ksplit;
     const bool merged = a.n_tiles * ks == 1;
     const bool has_add = a.noise != nullptr || a.sel_bias != nullptr;
-    float kadd[RE];
-    if (!a.noise) key_addend<RE>(0, lane, a, kadd);  // the selection bias (or nothing)
+    float kadd[NT][RE];
+    if (!a.noise) {  // the selection bias (or nothing), the same for every token
+        key_addend<RE>(0, lane, a, kadd[0]);
+#pragma unroll
+        for (int i = 1; i < NT; ++i)
+#pragma unroll
+            for (int q = 0; q < RE; ++q) kadd[i][q] = kadd[0][q];
+    }
     const int64_t split_stride = (int64_t)kTokTileR * BN;
-    for (int t = t_begin + warp; t < t_end; t += nwarps) {
-        float h[RE];
+    for (int t0 = t_begin + warp; t0 < t_end; t0 += NT * nwarps) {
+        int t[NT];
+        bool valid[NT];
+#pragma unroll
+        for (int i = 0; i < NT; ++i) {
+            t[i] = t0 + i * nwarps;
+            valid[i] = t[i] < t_end;
+        }
+        float h[NT][RE];
         if (merged) {
 #pragma unroll
-            for (int q = 0; q < RE; ++q) {
-                const int e = lane + 32 * q;
-                h[q] = e < a.E ? __ldcg(a.logits + (int64_t)t * a.E + e) : -INFINITY;
-            }
-        } else {
-            const int m = t / kTokTileR, tl = t - m * kTokTileR;
-            int64_t off[RE];
+            for (int i = 0; i < NT; ++i)
 #pragma unroll
-            for (int q = 0; q < RE; ++q) {
-                const int e = lane + 32 * q;
-                const int n = e / BN, c = e - n * BN;
-                off[q] = ((int64_t)((m * a.n_tiles + n) * ks) * kTokTileR + tl) * BN + c;
+                for (int q = 0; q < RE; ++q) {
+                    const int e = lane + 32 * q;
+                    h[i][q] = valid[i] ? (e < a.E ? __ldcg(a.logits + (int64_t)t[i] * a.E + e) : -INFINITY) : 0.f;
+                }
+        } else {
+            // Every split's partial of both tokens is loaded before any is
+            // summed (in split order), so the loads are in flight together.
+            int64_t off[NT][RE];
+#pragma unroll
+            for (int i = 0; i < NT; ++i) {
+                const int m = t[i] / kTokTileR, tl = t[i] - m * kTokTileR;
+#pragma unroll
+                for (int q = 0; q < RE; ++q) {
+                    const int e = lane + 32 * q;
+                    const int n = e / BN, c = e - n * BN;
+                    off[i][q] = ((int64_t)((m * a.n_tiles + n) * ks) * kTokTileR + tl) * BN + c;
+                }
             }
             for (int sp = 0; sp < ks; sp += 2) {
-                float v0[RE], v1[RE];
+                float v0[NT][RE], v1[NT][RE];
 #pragma unroll
-                for (int q = 0; q < RE; ++q) {
-                    const bool in = lane + 32 * q < a.E;
-                    v0[q] = in ? __ldcg(a.part + off[q] + sp * split_stride) : 0.f;
-                    v1[q] = in && sp + 1 < ks ? __ldcg(a.part + off[q] + (sp + 1) * split_stride) : 0.f;
-                }
+                for (int i = 0; i < NT; ++i)
 #pragma unroll
-                for (int q = 0; q < RE; ++q) {
-                    h[q] = sp == 0 ? v0[q] : __fadd_rn(h[q], v0[q]);
-                    if (sp + 1 < ks) h[q] = __fadd_rn(h[q], v1[q]);
-                }
+                    for (int q = 0; q < RE; ++q) {
+                        const bool in = valid[i] && lane + 32 * q < a.E;
+                        v0[i][q] = in ? __ldcg(a.part + off[i][q] + sp * split_stride) : 0.f;
+                        v1[i][q] = in && sp + 1 < ks ? __ldcg(a.part + off[i][q] + (sp + 1) * split_stride) : 0.f;
+                    }
+#pragma unroll
+                for (int i = 0; i < NT; ++i)
+#pragma unroll
+                    for (int q = 0; q < RE; ++q) {
+                        h[i][q] = sp == 0 ? v0[i][q] : __fadd_rn(h[i][q], v0[i][q]);
+                        if (sp + 1 < ks) h[i][q] = __fadd_rn(h[i][q], v1[i][q]);
+                    }
             }
 #pragma unroll
-            for (int q = 0; q < RE; ++q) {
-                const int e = lane + 32 * q;
-                if (e < a.E) {
-                    if (a.b_gate) h[q] = __fadd_rn(h[q], __ldg(a.b_gate + e));
-                    a.logits[(int64_t)t * a.E + e] = h[q];
-                } else {
-                    h[q] = -INFINITY;
+            for (int i = 0; i < NT; ++i)
+#pragma unroll
+                for (int q = 0; q < RE; ++q) {
+                    const int e = lane + 32 * q;
+                    if (e < a.E) {
+                        if (a.b_gate) h[i][q] = __fadd_rn(h[i][q], __ldg(a.b_gate + e));
+                        if (valid[i]) a.logits[(int64_t)t[i] * a.E + e] = h[i][q];
+                    } else {
+                        h[i][q] = -INFINITY;
+                    }
                 }
-            }
         }
         if (!a.route) continue;
         if (a.noise) {
-            float nz[RE];
 #pragma unroll
-            for (int q = 0; q < RE; ++q) {
-                const int e = lane + 32 * q;
-                nz[q] = e < a.E ? __ldg(a.noise + (int64_t)t * a.E + e) : 0.f;
-            }
-            route_warp<RE>(h, has_add, nz, t, lane, a, pacc);
-        } else {
-            route_warp<RE>(h, has_add, kadd, t, lane, a, pacc);
+            for (int i = 0; i < NT; ++i)
+#pragma unroll
+                for (int q = 0; q < RE; ++q) {
+                    const int e = lane + 32 * q;
+                    kadd[i][q] = valid[i] && e < a.E ? __ldg(a.noise + (int64_t)t[i] * a.E + e) : 0.f;
+                }
         }
+        route_warp_n<RE, NT>(h, has_add, kadd, t, valid, lane, a, pacc);
     }
 #pragma unroll
     for (int q = 0; q < RE; ++q) red[warp * 256 + lane + 32 * q] = pacc[q];
