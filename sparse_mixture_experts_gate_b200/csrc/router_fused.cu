@@ -35,9 +35,11 @@
 // all SMs; each CTA writes one row of per-expert P sums (its warps' sums added
 // in warp order).
 //
-// Roles (320 threads per CTA): warp 0 loads (TMA), warp 1 owns TMEM and, in
+// Roles (384 threads per CTA): warp 0 loads (TMA), warp 1 owns TMEM and, in
 // the leader, issues the MMAs; warps 2..9 drain the accumulators (two warps per
-// TMEM lane quarter, BN/2 columns each). In phase B all ten warps route. Every
+// TMEM lane quarter, BN/2 columns each); warps 10 and 11 have no phase-A role
+// (the registers the others need leave room for them). In phase B all twelve
+// warps route. Every
 // wait is bounded; on a timeout the roles stop, in-flight copies and MMAs are
 // drained, phase B is skipped, both CTAs meet at the cluster barrier and TMEM is
 // freed.
@@ -60,7 +62,8 @@ constexpr int kDrain = 4;
 template <int BN>
 struct RCfg {
     static constexpr int kEpiWarps = 8;
-    static constexpr int kThreads = 64 + 32 * kEpiWarps;
+    static constexpr int kRouteWarps = 2;  // warps with no phase-A role that route in phase B
+    static constexpr int kThreads = 64 + 32 * (kEpiWarps + kRouteWarps);
     static constexpr int kA = kTokCta * kBK * 2;          // x rows of this CTA, one K block
     static constexpr int kBHalf = (BN / 2) * kBK * 2;     // one plane, this CTA's BN/2 expert rows
     static constexpr int kStage = kA + 3 * kBHalf;
@@ -366,7 +369,7 @@ __global__ void __launch_bounds__(RCfg<BN>::kThreads, 1)
             tc_commit_pair(s.mma_done);
             mbar_wait_drain(s.mma_done, 0u);
         }
-    } else {
+    } else if (warp < 2 + kEpiWarps) {
         // ------------------------------------------------------------ epilogue (phase A)
         const int ew = warp - 2;
         const int q = warp & 3;                  // TMEM lane quarter this warp may access
