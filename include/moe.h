@@ -392,6 +392,22 @@ MOE_API int moe_selftest_bounded_wait(void *stream);
 MOE_API int moe_selftest_gemm_timeout(moe_layer_t *layer, const void *x, int32_t T, void *workspace, size_t ws_bytes,
                                       void *y, void *stream);
 
+/* Self-check of the bounded waits inside the fused router (no counterpart on
+ * the pages; failure detection): runs the router of a forward alone (no
+ * dispatch, expert GEMMs or combine), with a test-only launch argument that
+ * makes every CTA pair's leader skip its loads of the third pipeline stage and
+ * every wait of the launch give up after 20 ms. The MMA role's wait runs out,
+ * every role stops, copies in flight land, the CTAs pass the grid barrier
+ * without routing, both CTAs of each pair meet at the cluster barrier and TMEM
+ * is freed. Synchronises `stream`; returns MOE_OK if the status word reports
+ * the timeout, MOE_ERR_INTERNAL if it does not, the argument errors of
+ * moe_forward otherwise (GREEDY bf16 layers with a linear router and
+ * input_dim >= 192 only). The routing outputs are left incomplete, so the
+ * layer then has no forward for moe_aux_stats; the next moe_forward runs
+ * normally on the same layer and context. */
+MOE_API int moe_selftest_router_timeout(moe_layer_t *layer, const void *x, int32_t T, void *workspace,
+                                        size_t ws_bytes, void *stream);
+
 /* Device status word of the most recent forward: synchronises `stream`, then
  * returns MOE_OK, or MOE_ERR_TIMEOUT if a bounded device-side wait gave up. */
 MOE_API int moe_device_status(moe_layer_t *layer, void *stream);

@@ -24,7 +24,8 @@ MOE_PRIORITY = {"token": 0, "rank": 1}
 # Every symbol include/moe.h declares.
 EXPORTS = ("moe_config_default", "moe_layer_create", "moe_workspace_bytes", "moe_capacity", "moe_forward",
            "moe_forward_noalloc", "moe_aux_stats", "moe_stat_partials", "moe_stats_from_partials",
-           "moe_update_selection_bias", "moe_dro_update", "moe_selftest_bounded_wait", "moe_selftest_gemm_timeout", "moe_router_planes_bytes", "moe_prepare_router",
+           "moe_update_selection_bias", "moe_dro_update", "moe_selftest_bounded_wait", "moe_selftest_gemm_timeout",
+           "moe_selftest_router_timeout", "moe_router_planes_bytes", "moe_prepare_router",
            "moe_ep_dispatch", "moe_ep_layout", "moe_ep_experts_workspace_bytes", "moe_ep_experts", "moe_ep_combine", "moe_device_status", "moe_set_timing_events", "moe_launch_count", "moe_destroy", "moe_status_string",
            "moe_last_error")
 
@@ -115,6 +116,8 @@ def lib() -> ctypes.CDLL:
         L.moe_prepare_router.argtypes = [vp, vp, sz, vp]
         L.moe_selftest_gemm_timeout.restype = ctypes.c_int
         L.moe_selftest_gemm_timeout.argtypes = [vp, vp, i32, vp, sz, vp, vp]
+        L.moe_selftest_router_timeout.restype = ctypes.c_int
+        L.moe_selftest_router_timeout.argtypes = [vp, vp, i32, vp, sz, vp]
         L.moe_device_status.restype = ctypes.c_int
         L.moe_device_status.argtypes = [vp, vp]
         L.moe_set_timing_events.restype = ctypes.c_int
@@ -233,6 +236,11 @@ def moe_prepare_router(layer: int, planes: Optional[int], nbytes: int, stream: i
 def moe_selftest_gemm_timeout(layer: int, x: int, T: int, workspace: int, ws_bytes: int, y: int, stream: int) -> int:
     return _check(lib().moe_selftest_gemm_timeout(layer, x, T, workspace, ws_bytes, y, stream),
                   "moe_selftest_gemm_timeout")
+
+
+def moe_selftest_router_timeout(layer: int, x: int, T: int, workspace: int, ws_bytes: int, stream: int) -> int:
+    return _check(lib().moe_selftest_router_timeout(layer, x, T, workspace, ws_bytes, stream),
+                  "moe_selftest_router_timeout")
 
 
 def moe_device_status(layer: int, stream: int) -> int:

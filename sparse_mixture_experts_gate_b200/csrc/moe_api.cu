@@ -111,6 +111,7 @@ struct moe_layer {
     int num_pairs = 0;  // co-resident 2-CTA clusters of the expert GEMM
     int router_pairs = 0;  // and of the fused router
     int selftest_skip_stage = -1;  // moe_selftest_gemm_timeout only: GEMM 1's skipped stage
+    int selftest_router_skip = -1;  // moe_selftest_router_timeout only: the fused router's skipped stage
     void *planes = nullptr;        // moe_prepare_router's persistent bf16 planes of the router matrix, or null
     CUtensorMap map_w1, map_w2;
     // State of the most recent forward, read by moe_aux_stats.
@@ -374,7 +375,8 @@ namespace {
 // Router, dispatch and row scatter of one forward (everything before the
 // expert GEMMs); records what the later phases need in the layer.
 int fwd_route(moe_layer_t *L, const void *x, int32_t T, const float *logit_noise, void *workspace, size_t ws_bytes,
-              const moe_routing_t *routing, cudaStream_t s) {
+              const moe_routing_t *routing, cudaStream_t s,
+              bool router_only = false) {
     const moe_config_t &c = L->cfg;
     if (T < 0) return fail(MOE_ERR_INVALID_ARG, "T must be >= 0 (got %d)", T);
     if (c.max_tokens > 0 && T > c.max_tokens)
@@ -465,6 +467,10 @@ int fwd_route(moe_layer_t *L, const void *x, int32_t T, const float *logit_noise
         fa.counters = reinterpret_cast<int32_t *>(ws + p.o_rcnt);
         fa.status = status;
         fa.num_pairs = L->router_pairs;
+        if (L->selftest_router_skip >= 0) {  // the timeout self-test
+            fa.skip_stage = L->selftest_router_skip;
+            fa.wait_limit_ns = kSelftestWaitNs;
+        }
         MOE_LAUNCH(launch_router_fused(m_xr, m_ws, fa, s, nl));
         return MOE_OK;
     };
@@ -499,6 +505,7 @@ int fwd_route(moe_layer_t *L, const void *x, int32_t T, const float *logit_noise
         MOE_LAUNCH(launch_router(ra, s, nl));
     }
     MOE_MARK(L, 1, s);
+    if (router_only) return MOE_OK;
 
     DispatchArgs da;
     da.idx = idx;
@@ -1051,6 +1058,31 @@ int moe_selftest_gemm_timeout(moe_layer_t *L, const void *x, int32_t T, void *wo
     uint32_t st = 0;
     MOE_LAUNCH(cudaMemcpy(&st, L->ws + L->plan.o_ctrl + kCtrlStatus * 4, 4, cudaMemcpyDeviceToHost));
     if (!(st & kDevTimeout)) return fail(MOE_ERR_INTERNAL, "expert GEMM 1 missed a stage but reported no timeout");
+    return MOE_OK;
+}
+
+int moe_selftest_router_timeout(moe_layer_t *L, const void *x, int32_t T, void *workspace, size_t ws_bytes,
+                                void *stream_v) {
+    g_last_error.clear();
+    if (!L) return fail(MOE_ERR_INVALID_ARG, "layer is NULL");
+    if (!L->tc || L->cfg.use_mlp_gater)
+        return fail(MOE_ERR_UNSUPPORTED, "the self-test runs the fused router of a bf16 layer with a linear router");
+    if (L->cfg.top_k_method != MOE_TOPK_GREEDY) return fail(MOE_ERR_UNSUPPORTED, "the self-test needs GREEDY top-k");
+    if (T <= 0) return fail(MOE_ERR_INVALID_ARG, "the self-test needs T > 0");
+    if (L->cfg.input_dim < 3 * kBK)
+        return fail(MOE_ERR_UNSUPPORTED, "the self-test needs input_dim >= %d (three K stages)", 3 * kBK);
+    // The router alone: its outputs are incomplete after the timeout, so no
+    // later kernel of the forward may read them.
+    L->selftest_router_skip = 2;
+    int rc = fwd_route(L, x, T, nullptr, workspace, ws_bytes, nullptr, as_stream(stream_v), true);
+    L->selftest_router_skip = -1;
+    if (rc != MOE_OK) return rc;
+    L->has_forward = false;  // nothing for moe_aux_stats to read
+    cudaStream_t s = as_stream(stream_v);
+    MOE_LAUNCH(cudaStreamSynchronize(s));
+    uint32_t st = 0;
+    MOE_LAUNCH(cudaMemcpy(&st, L->ws + L->plan.o_ctrl + kCtrlStatus * 4, 4, cudaMemcpyDeviceToHost));
+    if (!(st & kDevTimeout)) return fail(MOE_ERR_INTERNAL, "the router missed a stage but reported no timeout");
     return MOE_OK;
 }
 

@@ -51,6 +51,11 @@ struct RouterFusedArgs {
     int32_t *counters;      // [1] grid-barrier counter, zero before the launch
     uint32_t *status;
     int num_pairs;          // CTA pairs to launch at most
+    // Self-test of the bounded waits only (moe_selftest_router_timeout): every
+    // leader's producer skips its loads of this pipeline stage (-1: none), and
+    // every wait of the launch gives up after wait_limit_ns.
+    int skip_stage = -1;
+    uint64_t wait_limit_ns = kWaitLimitNs;
 };
 int router_fused_epad(int E);    // padded expert count (rows of the split planes): 32, 64, 128 or 256
 int router_fused_bn(int E);      // expert tile: E_pad up to 128

@@ -309,13 +309,16 @@ __global__ void __launch_bounds__(RCfg<BN>::kThreads, 1)
                 const int st = it % kStages;
                 const uint32_t ph = (it / kStages) & 1u;
                 int got = 1;
-                if (lane == 0) got = mbar_wait(&s.empty[st], ph ^ 1u, a.status) ? 1 : 0;
+                if (lane == 0) got = mbar_wait(&s.empty[st], ph ^ 1u, a.status, a.wait_limit_ns) ? 1 : 0;
                 got = __shfl_sync(0xffffffffu, got, 0);
                 if (!got) {
                     ok = false;
                     break;
                 }
-                if (lane == 0) {
+                // Self-test of the timeout path: the leader neither announces
+                // nor loads this stage, so it never completes and the MMA
+                // role's bounded wait runs out.
+                if (lane == 0 && !(leader && static_cast<int>(it) == a.skip_stage)) {
                     if (leader) mbar_arrive_expect_tx(&s.full[st], 2u * C::kStage);
                     const uint32_t bar = mapa_shared(smem_u32(&s.full[st]), 0);
                     uint8_t *sA = s.stages + st * C::kStage;
@@ -336,7 +339,7 @@ __global__ void __launch_bounds__(RCfg<BN>::kThreads, 1)
                 const Unit un = unit_of(a, u);
                 for (int g0 = un.kb0; g0 < un.kb1 && ok; g0 += kDrain, ++gcount) {
                     const uint32_t buf = gcount & 1u, use = gcount >> 1;
-                    if (!mbar_wait(&s.tempty[buf], (use & 1u) ^ 1u, a.status)) {
+                    if (!mbar_wait(&s.tempty[buf], (use & 1u) ^ 1u, a.status, a.wait_limit_ns)) {
                         ok = false;
                         break;
                     }
@@ -346,7 +349,7 @@ __global__ void __launch_bounds__(RCfg<BN>::kThreads, 1)
                     for (int kb = g0; kb < g1; ++kb, ++it) {
                         const int st = it % kStages;
                         const uint32_t ph = (it / kStages) & 1u;
-                        if (!mbar_wait(&s.full[st], ph, a.status)) {
+                        if (!mbar_wait(&s.full[st], ph, a.status, a.wait_limit_ns)) {
                             ok = false;
                             break;
                         }
@@ -383,7 +386,7 @@ __global__ void __launch_bounds__(RCfg<BN>::kThreads, 1)
             for (int g0 = un.kb0; g0 < un.kb1; g0 += kDrain, ++gcount) {
                 const uint32_t buf = gcount & 1u, use = gcount >> 1;
                 int got = 1;
-                if (lane == 0) got = mbar_wait(&s.tfull[buf], use & 1u, a.status) ? 1 : 0;
+                if (lane == 0) got = mbar_wait(&s.tfull[buf], use & 1u, a.status, a.wait_limit_ns) ? 1 : 0;
                 if (!__shfl_sync(0xffffffffu, got, 0)) {
                     ok = false;
                     break;
@@ -412,7 +415,7 @@ __global__ void __launch_bounds__(RCfg<BN>::kThreads, 1)
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&s.drained[buf]);
                 if (ew == 0 && lane == 0) {
-                    if (mbar_wait(&s.drained[buf], use & 1u, a.status))
+                    if (mbar_wait(&s.drained[buf], use & 1u, a.status, a.wait_limit_ns))
                         mbar_arrive_cluster(mapa_shared(smem_u32(&s.tempty[buf]), 0));
                     else
                         ok = false;

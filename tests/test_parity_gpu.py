@@ -423,6 +423,26 @@ def test_expert_gemm_timeout_drains_and_context_survives():
     check_end_to_end(w, inp, g)
 
 
+def test_router_timeout_drains_and_context_survives():
+    """Failure detection inside the fused router: every CTA pair's leader skips
+    one stage's loads (a test-only launch argument) and the launch's waits give
+    up after 20 ms. The MMA role's wait runs out, every role stops, the CTAs
+    pass the grid barrier without routing and the kernel returns; the status
+    word reports the timeout; the same layer and context then run a forward that
+    matches the oracle."""
+    from sparse_mixture_experts_gate_b200 import binding
+    w = WORKLOADS["default"].with_(T=600)
+    inp = make_inputs(w, "cpu", seed=3)
+    layer = MoELayer(w, inp)
+    x = inp["x"].cuda()
+    ws, need = layer.workspace(w.T)
+    s = torch.cuda.current_stream().cuda_stream
+    assert binding.moe_selftest_router_timeout(layer.handle, x.data_ptr(), w.T, ws.data_ptr(), ws.numel(), s) == 0
+    g, _ = run_gpu(w, inp, layer=layer)  # asserts a clean status itself
+    check_same_logits_routing(w, inp, g)
+    check_end_to_end(w, inp, g)
+
+
 def _emulated_all_to_all(inputs, splits):
     """What all_to_all_single delivers to each rank q: from every rank r, in
     rank order, the rows r sends to q (splits[r][q] rows after the earlier ones)."""
