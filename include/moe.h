@@ -50,7 +50,7 @@ extern "C" {
 enum {
     MOE_OK = 0,
     MOE_ERR_INVALID_ARG = -1,  /* a NULL or inconsistent argument             */
-    MOE_ERR_UNSUPPORTED = -2,  /* a valid configuration this build cannot run */
+    MOE_ERR_UNSUPPORTED = -2,  /* a valid configuration this library does not support */
     MOE_ERR_CUDA = -3,         /* a CUDA runtime or driver call failed         */
     MOE_ERR_WORKSPACE = -4,    /* workspace NULL, misaligned or too small      */
     MOE_ERR_TIMEOUT = -5,      /* a bounded device-side wait gave up           */

@@ -101,7 +101,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, uint32
 // mbar_wait in every lane of the warp. Each lane acquires the completed phase
 // itself, so that every lane's later reads see what the arriving threads wrote
 // before they arrived (a wait in one lane followed by a shuffle orders nothing
-// for the other lanes' memory accesses). Returns the same verdict in all lanes.
+// for the other lanes' memory accesses). Returns the same result in all lanes.
 __device__ __forceinline__ bool mbar_wait_all_lanes(uint64_t *bar, uint32_t parity, uint32_t *status) {
     const bool ok = mbar_wait(bar, parity, status);
     return __all_sync(0xffffffffu, ok);

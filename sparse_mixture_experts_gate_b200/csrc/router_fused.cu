@@ -225,7 +225,7 @@ __device__ __forceinline__ void route_tokens(const RouterFusedArgs &a, float *re
 
 // Grid-wide barrier of the cooperative launch: every CTA counts itself once
 // its phase A writes are done and waits (bounded) until all have. Returns the
-// same verdict in every thread: true if all CTAs arrived and no bounded wait
+// same result in every thread: true if all CTAs arrived and no bounded wait
 // anywhere gave up (phase B may run), false otherwise.
 __device__ __forceinline__ bool grid_barrier(int32_t *counter, uint32_t *status) {
     __shared__ int go_s;
