@@ -175,14 +175,106 @@ __global__ void __launch_bounds__(kWarps * 32, 2) combine_kernel(CombineArgs a) 
     if (lane < k) a.credit[(int64_t)t * k + lane] = credit;
 }
 
+// The common case of bf16 layers (at most one shared expert, k <= 8) with one
+// warp per token, software-pipelined over the 256-column stretches: the loads
+// of stretch c + 256 are issued before stretch c is summed, so a lane keeps two
+// stretches of every term in flight (the general kernel keeps one and waits
+// out the memory latency once per stretch). Same arithmetic in the same order
+// as combine_kernel, so the results are bit-identical.
+template <bool SHARED>
+__global__ void __launch_bounds__(kWarps * 32, 2) combine_pipe_kernel(CombineArgs a) {
+    constexpr int V = 8;            // bf16 per 16-byte vector
+    constexpr int kStep = 32 * V;   // columns per stretch
+    constexpr int kTerms = kBatch + 1;  // routed terms, then the shared one
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int t = blockIdx.x * kWarps + warp;
+    if (t >= a.T) return;
+    const int k = a.k;
+    int my_row = -1;
+    float my_g = 0.f;
+    if (lane < k) {
+        my_row = a.row_of[(int64_t)t * k + lane];
+        my_g = a.gates[(int64_t)t * k + lane];
+    }
+    int rrow[kBatch];
+    float rg[kBatch];
+#pragma unroll
+    for (int r = 0; r < kBatch; ++r) {  // lanes >= k hold row -1
+        rrow[r] = __shfl_sync(0xffffffffu, my_row, r);
+        rg[r] = __shfl_sync(0xffffffffu, my_g, r);
+    }
+    const int srow = SHARED ? a.group_start[a.E] + t : -1;
+    const __nv_bfloat16 *o = static_cast<const __nv_bfloat16 *>(a.o);
+    __nv_bfloat16 *y = static_cast<__nv_bfloat16 *>(a.y) + (int64_t)t * a.O;
+    float ss[kBatch];
+#pragma unroll
+    for (int r = 0; r < kBatch; ++r) ss[r] = 0.f;
+    auto load = [&](uint4 (&u)[kTerms], int c) {
+#pragma unroll
+        for (int i = 0; i < kBatch; ++i)
+            if (rrow[i] >= 0) u[i] = load_raw(o + (int64_t)rrow[i] * a.O + c);
+        if (SHARED) u[kBatch] = load_raw(o + (int64_t)srow * a.O + c);
+    };
+    auto consume = [&](const uint4 (&u)[kTerms], int c) {
+        float acc[V];
+#pragma unroll
+        for (int j = 0; j < V; ++j) acc[j] = 0.f;
+        if (SHARED) {
+            float v[V];
+            Vec<__nv_bfloat16>::unpack(u[kBatch], v);
+#pragma unroll
+            for (int j = 0; j < V; ++j) acc[j] += v[j];
+        }
+#pragma unroll
+        for (int r = 0; r < kBatch; ++r) {
+            if (rrow[r] < 0) continue;
+            float v[V];
+            Vec<__nv_bfloat16>::unpack(u[r], v);
+#pragma unroll
+            for (int j = 0; j < V; ++j) {
+                acc[j] = fmaf(rg[r], v[j], acc[j]);
+                ss[r] = fmaf(v[j], v[j], ss[r]);
+            }
+        }
+        Vec<__nv_bfloat16>::store(y + c, acc);
+    };
+    uint4 u0[kTerms], u1[kTerms];
+    int c = lane * V;
+    if (c < a.O) load(u0, c);
+    for (; c < a.O; c += 2 * kStep) {
+        const int c1 = c + kStep;
+        if (c1 < a.O) load(u1, c1);
+        consume(u0, c);
+        if (c1 >= a.O) break;
+        if (c1 + kStep < a.O) load(u0, c1 + kStep);
+        consume(u1, c1);
+    }
+    // Credit of each routed assignment (fixed shuffle tree).
+    float credit = 0.f;
+#pragma unroll
+    for (int r = 0; r < kBatch; ++r) {
+        if (r >= k) break;
+        float v = ss[r];
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
+        if (lane == r && rrow[r] >= 0) credit = rg[r] * sqrtf(a.row_norm2 ? a.row_norm2[rrow[r]] : v);
+    }
+    if (lane < k) a.credit[(int64_t)t * k + lane] = credit;
+}
+
 template <typename T, int NB>
 void launch_t(const CombineArgs &a, int num_sms, cudaStream_t s) {
     // A block per token while one warp per token would leave fewer than eight
     // warps per SM.
+    const int blocks = (a.T + kWarps - 1) / kWarps;
     if (a.T < kWarps * num_sms)
         combine_kernel<T, NB, kWarps><<<a.T, kWarps * 32, 0, s>>>(a);
+    else if (a.bf16 && NB == 1 && a.S == 1)
+        combine_pipe_kernel<true><<<blocks, kWarps * 32, 0, s>>>(a);
+    else if (a.bf16 && NB == 1 && a.S == 0)
+        combine_pipe_kernel<false><<<blocks, kWarps * 32, 0, s>>>(a);
     else
-        combine_kernel<T, NB, 1><<<(a.T + kWarps - 1) / kWarps, kWarps * 32, 0, s>>>(a);
+        combine_kernel<T, NB, 1><<<blocks, kWarps * 32, 0, s>>>(a);
 }
 
 }  // namespace
