@@ -81,3 +81,49 @@ def test_gpus_flag_starts_that_many_ranks():
     assert len(lines) == 1, r.stdout
     d = json.loads(lines[0])
     assert d["impl"] == "reference" and d["n_gpus"] == 2
+
+
+def test_layer_roofline_counts_the_algorithmic_work():
+    """FLOPs of the kept and shared rows through both MLP layers; minimum bytes
+    of x, W_g, the touched experts' weights, y and routing metadata; the slower
+    of the two against each peak set."""
+    from sparse_mixture_experts_gate_b200.workloads import WORKLOADS
+    w = WORKLOADS["e64"]
+    kept, touched, ms = 40000, 65, 0.8
+    peaks = {"bf16": 1000.0, "bf16_sustained": 800.0, "hbm_gbs": 5000.0, "source": "test"}
+    r = bench.layer_roofline(w, kept, touched, ms, peaks)
+    rows = kept + w.S * w.T
+    flops = 2.0 * rows * w.F * (w.d + w.O)
+    bytes_min = (w.T * w.d * 2 + w.E * w.d * 4 + touched * (w.F * w.d + w.O * w.F) * 2 + w.T * w.O * 2
+                 + w.T * w.k * 12)
+    assert r["flops"] == flops and r["bytes_min"] == bytes_min
+    t = ms / 1e3
+    t_flop, t_bytes = flops / 1e15, bytes_min / 5e12
+    assert r["bound"] == ("tensor" if t_flop >= t_bytes else "hbm")
+    assert abs(r["layer_roofline_frac"] - max(t_flop, t_bytes) / t) < 1e-12
+    assert abs(r["layer_roofline_frac_sustained"] - max(flops / 8e14, t_bytes) / t) < 1e-12
+    t_spec = max(flops / (bench.SPEC_BF16_TFLOPS * 1e12), bytes_min / (bench.SPEC_HBM_GBS * 1e9))
+    assert abs(r["layer_roofline_frac_spec_sheet"] - t_spec / t) < 1e-12
+    assert abs(r["expert_gemm_tflops"] - flops / t / 1e12) < 1e-9
+
+
+def test_committed_traffic_scales_the_capture_and_checks_the_source(tmp_path, monkeypatch):
+    """The DRAM traffic of a scaled capture is scaled by the rows processed, and
+    is withheld when the expert-GEMM source differs from the captured one or the
+    workload was resized."""
+    import hashlib
+    from sparse_mixture_experts_gate_b200.workloads import WORKLOADS
+    src = tmp_path / "sparse_mixture_experts_gate_b200" / "csrc"
+    src.mkdir(parents=True)
+    (src / "gemm_pair.cu").write_text("// kernel source\n")
+    sha = hashlib.sha256(b"// kernel source\n").hexdigest()
+    prof = tmp_path / "profiles"
+    prof.mkdir()
+    (prof / "grouped_gemm_pair_e256_traffic.txt").write_text(
+        f"# a capture\nkernel_source_sha256: {sha}\ncapture_rows: 1000\ndram_bytes_per_launch_pair: 2.5e9\n")
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    w = WORKLOADS["e256"]
+    assert bench.committed_traffic(w, 4000) == 2.5e9 * 4
+    assert bench.committed_traffic(w.with_(T=1024), 4000) is None  # resized workload
+    (src / "gemm_pair.cu").write_text("// edited kernel source\n")
+    assert bench.committed_traffic(w, 4000) is None  # source changed since the capture
