@@ -24,14 +24,26 @@
 // E = 256 layer and the L2 reuse of the weight tiles collapses (GEMM 1 read
 // 41.6 GB from DRAM instead of ~15 GB).
 //
-// Per CTA (192 threads): warp 0 loads (TMA, signalling the leader's stage
+// Per CTA (192 threads with four epilogue warps): warp 0 loads (TMA, signalling the leader's stage
 // barrier, which expects both CTAs' bytes), warp 1 owns TMEM (2 accumulators x
 // 256 columns) and, in the leader, issues the pair MMAs and commits stages and
 // accumulators to both CTAs at once; warps 2..5 drain this CTA's 128 features:
 // each warp reads 32 features x 32 tokens from TMEM, adds the bias, applies the
-// activation, writes them transposed (token-major, bf16) to a shared staging box
-// and stores the box with a TMA tensor store. The epilogue releases an
-// accumulator by arriving on the leader's barrier (8 warps per tile).
+// activation, pairs neighbouring lanes' values so that each lane holds two
+// adjacent features of one token, and stores them to global memory (a warp
+// store covers 64 contiguous bytes of each of two token rows). No shared
+// memory is spent on staging the outputs, so it holds seven 32 KB pipeline
+// stages. The epilogue releases an accumulator by arriving on the leader's
+// barrier (one arrival per epilogue warp of both CTAs).
+//
+// Ragged last feature tile. When N leaves a last feature tile of at most 128
+// features (d_ff = 1408 = 5.5 x 256, say), a unit of that tile would leave
+// half of the pair's M side idle. Such units run transposed instead: the token
+// tile is the MMA's M side (each CTA's half of the tokens on its 128 TMEM
+// lanes) and the 128 features are its N side (64 weight rows staged per CTA),
+// so the pair stages a quarter fewer bytes and issues half the MMA work for
+// the same outputs. Their epilogue holds a token's 32 consecutive features per
+// lane and writes them to global memory directly (64 bytes per token row).
 //
 // Every wait is bounded (mbar_wait); on a timeout the roles stop, the leader
 // drains its MMAs, copies in flight are given time to land, both CTAs meet at
@@ -42,36 +54,36 @@
 namespace moe {
 namespace {
 
-constexpr int kThreads = 192;
+constexpr int kEpiWarps = 4;                        // epilogue warps per CTA (a multiple of 4)
+constexpr int kThreads = 64 + 32 * kEpiWarps;
 constexpr int kFeatPair = 256;                     // MMA M: features per pair tile
 constexpr int kFeatCta = 128;                      // features per CTA
 constexpr int kABytes = kFeatCta * kBK * 2;        // 16 KB: 128 weight rows x 64 K
 constexpr int kAccCols = 256;
-constexpr int kBoxTok = 32, kBoxFeat = 32;          // store box: 32 tokens x 32 features
-constexpr int kBoxBytes = kBoxTok * kBoxFeat * 2;
-constexpr int kStaging = 4 * 2 * kBoxBytes;         // 4 epilogue warps x 2 boxes
+constexpr int kBoxTok = 32;                         // tokens per TMEM load of the epilogue
 constexpr int kRowsPerLoad16 = 16;                  // rows of the narrow token box
 constexpr int kRing = 8;            // unit-index ring between the leader's producer and the consumers
-constexpr int kRingConsumers = 10;  // leader: MMA thread + 4 epilogue warps; peer: producer + 4 epilogue warps
+// leader: MMA thread + the epilogue warps; peer: producer + the epilogue warps
+constexpr int kRingConsumers = 2 * (1 + kEpiWarps);
 static_assert(kTokTile == 256 && kTokTile % (2 * kRowsPerLoad16) == 0, "token tile layout");
 static_assert(kNarrowTile % (2 * kRowsPerLoad16) == 0, "narrow token tile layout");
 
 // Stage layout for token tiles of up to TILE rows (each CTA stages TILE / 2):
-// 256-row tiles with 6 stages of 32 KB, or narrow 64-row tiles with 10 stages
-// of 20 KB, which keeps 160 KB of weight tiles in flight per SM when the
+// 256-row tiles with 7 stages of 32 KB, or narrow 64-row tiles with 11 stages
+// of 20 KB, which keeps 176 KB of weight tiles in flight per SM when the
 // token tiles are short and the GEMM streams weights.
 template <int TILE>
 struct PairCfg {
     static constexpr int kB = (TILE / 2) * kBK * 2;
     static constexpr int kStage = kABytes + kB;
-    static constexpr int kStages = TILE == kTokTile ? 6 : 10;
-    static constexpr int kSmem = 1024 + kStages * kStage + kStaging + 512;
+    static constexpr int kStages = TILE == kTokTile ? 7 : 11;
+    static constexpr int kSmem = 1024 + kStages * kStage + 512;
     static_assert(kSmem <= 232448, "exceeds the 227 KB of shared memory a CTA may use");
     static_assert(kB % 1024 == 0, "B stages keep the 1024-byte swizzle alignment");
 };
 
 struct Smem {
-    uint8_t *sA, *sB, *staging;
+    uint8_t *sA, *sB;
     uint64_t *full, *empty, *tfull, *tempty, *mma_done, *ring_full, *ring_empty;
     uint32_t *tmem_slot;
     int32_t *ring;
@@ -84,8 +96,7 @@ __device__ __forceinline__ Smem carve(uint8_t *raw) {
     Smem s;
     s.sA = base;
     s.sB = base + C::kStages * kABytes;
-    s.staging = base + C::kStages * C::kStage;
-    s.full = reinterpret_cast<uint64_t *>(s.staging + kStaging);
+    s.full = reinterpret_cast<uint64_t *>(base + C::kStages * C::kStage);
     s.empty = s.full + C::kStages;
     s.tfull = s.empty + C::kStages;
     s.tempty = s.tfull + 2;
@@ -99,9 +110,10 @@ __device__ __forceinline__ Smem carve(uint8_t *raw) {
 
 template <int ACT, int TILE>
 __global__ void __launch_bounds__(kThreads, 1)
-    grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap map_w, const __grid_constant__ CUtensorMap map_t,
+    grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap map_w, const __grid_constant__ CUtensorMap map_wh,
+                             const __grid_constant__ CUtensorMap map_t,
                              const __grid_constant__ CUtensorMap map_t16, const __grid_constant__ CUtensorMap map_s,
-                             const __grid_constant__ CUtensorMap map_s16, const __grid_constant__ CUtensorMap map_out,
+                             const __grid_constant__ CUtensorMap map_s16,
                              const PairGemmArgs a) {
     using C = PairCfg<TILE>;
     constexpr int kStages = C::kStages;
@@ -113,18 +125,18 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     if (threadIdx.x == 0) {
         tma_prefetch_desc(&map_w);
+        if (a.half_last) tma_prefetch_desc(&map_wh);
         tma_prefetch_desc(&map_t);
         tma_prefetch_desc(&map_t16);
         tma_prefetch_desc(&map_s);
         tma_prefetch_desc(&map_s16);
-        tma_prefetch_desc(&map_out);
         for (int i = 0; i < kStages; ++i) {
             mbar_init(&s.full[i], 1);
             mbar_init(&s.empty[i], 1);
         }
         for (int i = 0; i < 2; ++i) {
             mbar_init(&s.tfull[i], 1);
-            mbar_init(&s.tempty[i], 8);  // 4 epilogue warps in each CTA
+            mbar_init(&s.tempty[i], 2 * kEpiWarps);  // the epilogue warps of both CTAs
         }
         mbar_init(s.mma_done, 1);
         for (int i = 0; i < kRing; ++i) {
@@ -148,6 +160,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     // Weight-stack index of group g (shared groups may sit at another base).
     auto wgroup = [&](int g) { return g < a.E ? g : a.w_shared_base + (g - a.E); };
     const int kblocks = a.K / kBK;
+    // Units of the last feature tile run transposed (wide token tiles only).
+    const int tr_tile = (TILE == kTokTile && a.half_last) ? a.n_ftiles - 1 : -1;
     bool ok = true;
 
     // Units (token tile, feature tile) are handed out in index order from a
@@ -196,8 +210,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                 mt16 = &map_s16;
                 trow -= a.group_start[g];
             }
-            const int wrow = wgroup(g) * a.N + j * kFeatPair + static_cast<int>(rank) * kFeatCta;
-            const uint32_t tx_bytes = 2u * kABytes + static_cast<uint32_t>(ntok) * kBK * 2u;
+            const bool tr = j == tr_tile;  // 64 weight rows per CTA (the MMA's N side)
+            const int wrow = wgroup(g) * a.N + j * kFeatPair + static_cast<int>(rank) * (tr ? kFeatCta / 2 : kFeatCta);
+            const CUtensorMap *mw = tr ? &map_wh : &map_w;
+            const uint32_t tx_bytes = (tr ? 1u : 2u) * kABytes + static_cast<uint32_t>(ntok) * kBK * 2u;
             const int n16 = ntok / (2 * kRowsPerLoad16);
             for (int kb = 0; kb < kblocks; ++kb, ++it) {
                 const int st = it % kStages;
@@ -217,7 +233,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (leader && static_cast<int>(it) == a.skip_stage) continue;
                 const uint32_t bar = mapa_shared(smem_u32(&s.full[st]), 0);
                 uint8_t *sA = s.sA + st * kABytes, *sB = s.sB + st * C::kB;
-                if (lane == 0) tma_load_2d_pair(&map_w, bar, sA, kb * kBK, wrow);
+                if (lane == 0) tma_load_2d_pair(mw, bar, sA, kb * kBK, wrow);
                 if (ntok == kTokTile) {
                     if (lane == 1) tma_load_2d_pair(mt, bar, sB, kb * kBK, trow);
                 } else if (lane < n16) {
@@ -237,7 +253,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                     break;
                 }
                 const int ntok = tok_tiles[u / a.n_ftiles].z;
-                const uint32_t idesc = idesc_bf16_f32(kFeatPair, ntok);
+                // Transposed unit: A = the token tile (M = 256, each CTA's
+                // ntok / 2 rows first), B = the 128 features (64 rows per CTA).
+                const bool tr = u % a.n_ftiles == tr_tile;
+                const uint32_t idesc = tr ? idesc_bf16_f32(kTokTile, kFeatCta) : idesc_bf16_f32(kFeatPair, ntok);
                 const uint32_t acc = tcount & 1u, use = tcount >> 1;
                 if (!mbar_wait(&s.tempty[acc], (use & 1u) ^ 1u, a.status, a.wait_limit_ns)) break;
                 tc_fence_after_sync();
@@ -252,9 +271,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                     tc_fence_after_sync();
                     const uint64_t ad = sw128_kmajor_desc(smem_u32(s.sA + st * kABytes));
                     const uint64_t bd = sw128_kmajor_desc(smem_u32(s.sB + st * C::kB));
+                    const uint64_t da = tr ? bd : ad, db = tr ? ad : bd;
 #pragma unroll
                     for (int kk = 0; kk < kBK / 16; ++kk)
-                        tc_mma_bf16_pair(d_tmem, ad + 2u * kk, bd + 2u * kk, idesc, (kb | kk) != 0 ? 1u : 0u);
+                        tc_mma_bf16_pair(d_tmem, da + 2u * kk, db + 2u * kk, idesc, (kb | kk) != 0 ? 1u : 0u);
                     tc_commit_pair_mc(&s.empty[st], 0x3);
                 }
                 if (ok) tc_commit_pair_mc(&s.tfull[acc], 0x3);
@@ -265,8 +285,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     } else {
         // ------------------------------------------------------------ epilogue
         const int q = warp & 3;  // TMEM lane quarter this warp may access
-        uint8_t *my_stage = s.staging + (warp - 2) * 2 * kBoxBytes;
-        uint32_t sub = 0;
+        // The warps sharing a lane quarter take alternate 32-column chunks.
+        const int part = (warp - 2) >> 2, nparts = kEpiWarps / 4;
         for (uint32_t tcount = 0;; ++tcount) {
             int u = 0;
             if (lane == 0) u = take_unit(tcount);
@@ -281,47 +301,68 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (lane == 0) got = mbar_wait_idle(&s.tfull[acc], use & 1u, a.status, a.wait_limit_ns) ? 1 : 0;
             if (!__shfl_sync(0xffffffffu, got, 0)) break;
             tc_fence_after_sync();
-            if (fcol < a.N) {  // the last feature tile of a ragged N has an idle half
-                const float b = a.bias ? __ldg(a.bias + (int64_t)wgroup(g) * a.N + fcol + lane) : 0.f;
+            if (j == tr_tile) {
+                // Transposed unit: TMEM lane = token (this CTA's ntok / 2
+                // tokens first), column = feature. Each lane activates 32
+                // consecutive features of its token and stores them as 64
+                // bytes; chunks past N (N % 256 == 64) are not stored.
+                const int half = ntok / 2, tok = q * 32 + lane;
+                const int f0 = j * kFeatPair;
+                __nv_bfloat16 *orow = a.out + (static_cast<int64_t>(row0) + static_cast<int64_t>(rank) * half + tok) * a.N;
                 const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * kAccCols;
 #pragma unroll 1
-                for (int c = 0; c < ntok; c += kBoxTok) {
-                    uint8_t *buf = my_stage + (sub & 1u) * kBoxBytes;
-                    if (lane == 0) bulk_wait_group_read<1>();  // the store that last used `buf` has read it
-                    __syncwarp();
+                for (int c = 32 * part; c < kFeatCta && f0 + c < a.N; c += 32 * nparts) {
+                    const float bl = a.bias ? __ldg(a.bias + (int64_t)wgroup(g) * a.N + f0 + c + lane) : 0.f;
                     uint32_t r[32];
                     tmem_ld_32x32b_x32(taddr + c, r);
                     tmem_ld_wait();
-                    // Lane = feature, register = token; the box is token-major
-                    // (64 bytes per token). Neighbouring lanes trade one value per
-                    // token pair, so the even lane holds features (f, f+1) of
-                    // token t and the odd lane those of token t+1: one bf16x2
-                    // conversion and one 32-bit store each, the two rows in
-                    // opposite bank halves.
+                    uint32_t pk[16];
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) {
+                        const float z0 = activate_t<ACT>(__uint_as_float(r[2 * i]) + __shfl_sync(0xffffffffu, bl, 2 * i));
+                        const float z1 =
+                            activate_t<ACT>(__uint_as_float(r[2 * i + 1]) + __shfl_sync(0xffffffffu, bl, 2 * i + 1));
+                        __nv_bfloat162 p2 = __floats2bfloat162_rn(z0, z1);
+                        pk[i] = *reinterpret_cast<uint32_t *>(&p2);
+                    }
+                    if (tok < half) {
+                        uint4 *dst = reinterpret_cast<uint4 *>(orow + f0 + c);
+#pragma unroll
+                        for (int v = 0; v < 4; ++v)
+                            dst[v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
+                    }
+                }
+            } else if (fcol < a.N) {  // the last feature tile of a ragged N has an idle half
+                const float b = a.bias ? __ldg(a.bias + (int64_t)wgroup(g) * a.N + fcol + lane) : 0.f;
+                const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * kAccCols;
+#pragma unroll 1
+                for (int c = kBoxTok * part; c < ntok; c += kBoxTok * nparts) {
+                    uint32_t r[32];
+                    tmem_ld_32x32b_x32(taddr + c, r);
+                    tmem_ld_wait();
+                    // Lane = feature, register = token. Neighbouring lanes
+                    // trade one value per token pair, so the even lane holds
+                    // features (f, f+1) of token t and the odd lane those of
+                    // token t+1: one bf16x2 conversion and one 32-bit store
+                    // each, 16 lanes writing 64 contiguous bytes of a row.
                     const uint32_t odd = lane & 1u;
-                    uint32_t *words = reinterpret_cast<uint32_t *>(buf) + (lane >> 1);
+                    uint32_t *dst = reinterpret_cast<uint32_t *>(
+                        a.out + static_cast<int64_t>(row0 + c + static_cast<int>(odd)) * a.N + fcol + (lane & ~1u));
+                    const int64_t two_rows = static_cast<int64_t>(a.N);  // 2 rows in 32-bit words
 #pragma unroll
                     for (int t = 0; t < 32; t += 2) {
                         const float z0 = activate_t<ACT>(__uint_as_float(r[t]) + b);
                         const float z1 = activate_t<ACT>(__uint_as_float(r[t + 1]) + b);
                         const float other = __shfl_xor_sync(0xffffffffu, odd ? z0 : z1, 1);
                         __nv_bfloat162 p = odd ? __floats2bfloat162_rn(other, z1) : __floats2bfloat162_rn(z0, other);
-                        words[(t + odd) * (kBoxFeat / 2)] = *reinterpret_cast<uint32_t *>(&p);
+                        dst[(t / 2) * two_rows] = *reinterpret_cast<uint32_t *>(&p);
                     }
-                    fence_proxy_async_smem();
-                    __syncwarp();
-                    if (lane == 0) {
-                        tma_store_2d(&map_out, buf, fcol, row0 + c);
-                        bulk_commit_group();
-                    }
-                    ++sub;
                 }
             }
             tc_fence_before_sync();
             __syncwarp();
             if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(&s.tempty[acc]), 0));
         }
-        if (lane == 0) bulk_wait_group<0>();  // all stores complete before exit
     }
 
     // A role that gave up may leave its own TMA loads in flight; they land
@@ -337,8 +378,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 template <int ACT, int TILE>
-cudaError_t launch_act(const CUtensorMap &mw, const CUtensorMap &mt, const CUtensorMap &mt16, const CUtensorMap &ms,
-                       const CUtensorMap &ms16, const CUtensorMap &mo, const PairGemmArgs &a, cudaStream_t st) {
+cudaError_t launch_act(const CUtensorMap &mw, const CUtensorMap &mwh, const CUtensorMap &mt, const CUtensorMap &mt16, const CUtensorMap &ms,
+                       const CUtensorMap &ms16, const PairGemmArgs &a, cudaStream_t st) {
     constexpr int kSmem = PairCfg<TILE>::kSmem;
     auto kern = grouped_gemm_pair_kernel<ACT, TILE>;
     cudaError_t e = set_smem_limit_once<grouped_gemm_pair_kernel<ACT, TILE>>(kSmem);
@@ -355,7 +396,7 @@ cudaError_t launch_act(const CUtensorMap &mw, const CUtensorMap &mt, const CUten
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, kern, mw, mt, mt16, ms, ms16, mo, a);
+    return cudaLaunchKernelEx(&cfg, kern, mw, mwh, mt, mt16, ms, ms16, a);
 }
 
 }  // namespace
@@ -384,24 +425,26 @@ int gemm_pair_max_pairs(int num_sms) {
 
 int gemm_pair_ftiles(int N) { return (N + kFeatPair - 1) / kFeatPair; }
 
-cudaError_t launch_gemm_pair(const CUtensorMap &map_w, const CUtensorMap &map_t, const CUtensorMap &map_t16,
-                             const CUtensorMap &map_s, const CUtensorMap &map_s16, const CUtensorMap &map_out,
+int gemm_pair_half_last(int N) { return N % kFeatPair != 0 && N % kFeatPair <= kFeatCta ? 1 : 0; }
+
+cudaError_t launch_gemm_pair(const CUtensorMap &map_w, const CUtensorMap &map_wh, const CUtensorMap &map_t, const CUtensorMap &map_t16,
+                             const CUtensorMap &map_s, const CUtensorMap &map_s16,
                              const PairGemmArgs &a, cudaStream_t s, int *launches) {
     if (a.num_pairs <= 0) return cudaErrorInvalidConfiguration;
     ++*launches;
     if (a.narrow) {
         switch (a.act) {
-            case 0: return launch_act<0, kNarrowTile>(map_w, map_t, map_t16, map_s, map_s16, map_out, a, s);
-            case 1: return launch_act<1, kNarrowTile>(map_w, map_t, map_t16, map_s, map_s16, map_out, a, s);
-            case 2: return launch_act<2, kNarrowTile>(map_w, map_t, map_t16, map_s, map_s16, map_out, a, s);
-            default: return launch_act<-1, kNarrowTile>(map_w, map_t, map_t16, map_s, map_s16, map_out, a, s);
+            case 0: return launch_act<0, kNarrowTile>(map_w, map_wh, map_t, map_t16, map_s, map_s16, a, s);
+            case 1: return launch_act<1, kNarrowTile>(map_w, map_wh, map_t, map_t16, map_s, map_s16, a, s);
+            case 2: return launch_act<2, kNarrowTile>(map_w, map_wh, map_t, map_t16, map_s, map_s16, a, s);
+            default: return launch_act<-1, kNarrowTile>(map_w, map_wh, map_t, map_t16, map_s, map_s16, a, s);
         }
     }
     switch (a.act) {
-        case 0: return launch_act<0, kTokTile>(map_w, map_t, map_t16, map_s, map_s16, map_out, a, s);
-        case 1: return launch_act<1, kTokTile>(map_w, map_t, map_t16, map_s, map_s16, map_out, a, s);
-        case 2: return launch_act<2, kTokTile>(map_w, map_t, map_t16, map_s, map_s16, map_out, a, s);
-        default: return launch_act<-1, kTokTile>(map_w, map_t, map_t16, map_s, map_s16, map_out, a, s);
+        case 0: return launch_act<0, kTokTile>(map_w, map_wh, map_t, map_t16, map_s, map_s16, a, s);
+        case 1: return launch_act<1, kTokTile>(map_w, map_wh, map_t, map_t16, map_s, map_s16, a, s);
+        case 2: return launch_act<2, kTokTile>(map_w, map_wh, map_t, map_t16, map_s, map_s16, a, s);
+        default: return launch_act<-1, kTokTile>(map_w, map_wh, map_t, map_t16, map_s, map_s16, a, s);
     }
 }
 

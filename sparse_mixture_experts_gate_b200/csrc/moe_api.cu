@@ -66,20 +66,6 @@ bool encode_bf16_2d(CUtensorMap *m, const void *base, uint64_t inner, uint64_t r
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// Row-major bf16 [rows][inner] output map for the expert GEMM's stores: box of
-// 32 x 32 elements, no swizzle.
-bool encode_bf16_store(CUtensorMap *m, const void *base, uint64_t inner, uint64_t rows) {
-    EncodeTiledFn fn = encode_fn();
-    if (!fn || rows == 0) return false;
-    cuuint64_t dims[2] = {inner, rows};
-    cuuint64_t strides[1] = {inner * 2};
-    cuuint32_t box[2] = {32, 32};
-    cuuint32_t es[2] = {1, 1};
-    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box, es,
-              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE,
-              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
 struct Plan {
     int T = 0;
     int64_t C = 0;
@@ -114,6 +100,7 @@ struct moe_layer {
     int selftest_router_skip = -1;  // moe_selftest_router_timeout only: the fused router's skipped stage
     void *planes = nullptr;        // moe_prepare_router's persistent bf16 planes of the router matrix, or null
     CUtensorMap map_w1, map_w2;
+    CUtensorMap map_w1h, map_w2h;  // the same with boxes of 64 rows (transposed last feature tiles)
     // State of the most recent forward, read by moe_aux_stats.
     bool has_forward = false;
     Plan plan;
@@ -343,7 +330,9 @@ int moe_layer_create(const moe_config_t *cfg, const moe_weights_t *w, moe_layer_
     L->tc = cfg->dtype == MOE_DTYPE_BF16;
     if (L->tc) {
         if (!encode_bf16_2d(&L->map_w1, w->w1, cfg->input_dim, (uint64_t)L->G * cfg->expert_dim, 128) ||
-            !encode_bf16_2d(&L->map_w2, w->w2, cfg->expert_dim, (uint64_t)L->G * cfg->output_dim, 128)) {
+            !encode_bf16_2d(&L->map_w2, w->w2, cfg->expert_dim, (uint64_t)L->G * cfg->output_dim, 128) ||
+            !encode_bf16_2d(&L->map_w1h, w->w1, cfg->input_dim, (uint64_t)L->G * cfg->expert_dim, 64) ||
+            !encode_bf16_2d(&L->map_w2h, w->w2, cfg->expert_dim, (uint64_t)L->G * cfg->output_dim, 64)) {
             delete L;
             return fail(MOE_ERR_CUDA, "cuTensorMapEncodeTiled failed for the expert weights (16-byte alignment?)");
         }
@@ -594,6 +583,8 @@ int fwd_expert_gemms(moe_layer_t *L, cudaStream_t s, bool shared_only) {
             g1.narrow = 1;
         }
         g1.use_s = 1;
+        g1.half_last = !g1.narrow && gemm_pair_half_last(c.expert_dim);
+        g1.out = reinterpret_cast<__nv_bfloat16 *>(ws + p.o_h);
         g1.bias = L->w.b1;
         g1.act = c.activation;
         g1.status = status;
@@ -608,21 +599,21 @@ int fwd_expert_gemms(moe_layer_t *L, cudaStream_t s, bool shared_only) {
         g2.K = c.expert_dim;
         g2.n_ftiles = gemm_pair_ftiles(c.output_dim);
         g2.use_s = 0;
+        g2.half_last = !g2.narrow && gemm_pair_half_last(c.output_dim);
+        g2.out = reinterpret_cast<__nv_bfloat16 *>(ws + p.o_o);
         g2.bias = L->w.b2;
         g2.act = -1;
         g2.work_counter = ctrl + kCtrlWork2;
-        CUtensorMap m_xp, m_xp16, m_x, m_x16, m_h, m_h16, m_hs, m_os;
+        CUtensorMap m_xp, m_xp16, m_x, m_x16, m_h, m_h16;
         if (!encode_bf16_2d(&m_xp, ws + p.o_xp, c.input_dim, p.R_routed_max, 128) ||
             !encode_bf16_2d(&m_xp16, ws + p.o_xp, c.input_dim, p.R_routed_max, 16) ||
             !encode_bf16_2d(&m_x, x, c.input_dim, T, 128) || !encode_bf16_2d(&m_x16, x, c.input_dim, T, 16) ||
             !encode_bf16_2d(&m_h, ws + p.o_h, c.expert_dim, p.R_max, 128) ||
-            !encode_bf16_2d(&m_h16, ws + p.o_h, c.expert_dim, p.R_max, 16) ||
-            !encode_bf16_store(&m_hs, ws + p.o_h, c.expert_dim, p.R_max) ||
-            !encode_bf16_store(&m_os, ws + p.o_o, c.output_dim, p.R_max))
+            !encode_bf16_2d(&m_h16, ws + p.o_h, c.expert_dim, p.R_max, 16))
             return fail(MOE_ERR_CUDA, "cuTensorMapEncodeTiled failed for the activations");
-        MOE_LAUNCH(launch_gemm_pair(L->map_w1, m_xp, m_xp16, m_x, m_x16, m_hs, g1, s, nl));
+        MOE_LAUNCH(launch_gemm_pair(L->map_w1, L->map_w1h, m_xp, m_xp16, m_x, m_x16, g1, s, nl));
         MOE_MARK(L, 4, s);
-        MOE_LAUNCH(launch_gemm_pair(L->map_w2, m_h, m_h16, m_h, m_h16, m_os, g2, s, nl));
+        MOE_LAUNCH(launch_gemm_pair(L->map_w2, L->map_w2h, m_h, m_h16, m_h, m_h16, g2, s, nl));
         MOE_MARK(L, 5, s);
     } else {
         GemmSimtArgs s1;
@@ -826,6 +817,8 @@ int moe_ep_experts(moe_layer_t *L, const void *recv_x, const int32_t *recv_rows,
     g1.E = L->E_weights;  // every received group is a routed expert held here
     g1.w_shared_base = L->E_weights;
     g1.use_s = 0;
+    g1.half_last = gemm_pair_half_last(c.expert_dim);
+    g1.out = reinterpret_cast<__nv_bfloat16 *>(ws + q.o_h);
     g1.bias = L->w.b1;
     g1.act = c.activation;
     g1.status = reinterpret_cast<uint32_t *>(ctrl + kCtrlStatus);
@@ -835,17 +828,18 @@ int moe_ep_experts(moe_layer_t *L, const void *recv_x, const int32_t *recv_rows,
     g2.N = c.output_dim;
     g2.K = c.expert_dim;
     g2.n_ftiles = gemm_pair_ftiles(c.output_dim);
+    g2.half_last = gemm_pair_half_last(c.output_dim);
+    g2.out = reinterpret_cast<__nv_bfloat16 *>(recv_out);
     g2.bias = L->w.b2;
     g2.act = -1;
     g2.work_counter = ctrl + kCtrlWork2;
-    CUtensorMap m_x, m_x16, m_h, m_h16, m_hs, m_os;
+    CUtensorMap m_x, m_x16, m_h, m_h16;
     if (!encode_bf16_2d(&m_x, recv_x, c.input_dim, R, 128) || !encode_bf16_2d(&m_x16, recv_x, c.input_dim, R, 16) ||
         !encode_bf16_2d(&m_h, ws + q.o_h, c.expert_dim, R, 128) ||
-        !encode_bf16_2d(&m_h16, ws + q.o_h, c.expert_dim, R, 16) ||
-        !encode_bf16_store(&m_hs, ws + q.o_h, c.expert_dim, R) || !encode_bf16_store(&m_os, recv_out, c.output_dim, R))
+        !encode_bf16_2d(&m_h16, ws + q.o_h, c.expert_dim, R, 16))
         return fail(MOE_ERR_CUDA, "cuTensorMapEncodeTiled failed for the received rows");
-    MOE_LAUNCH(launch_gemm_pair(L->map_w1, m_x, m_x16, m_x, m_x16, m_hs, g1, s, &launches));
-    MOE_LAUNCH(launch_gemm_pair(L->map_w2, m_h, m_h16, m_h, m_h16, m_os, g2, s, &launches));
+    MOE_LAUNCH(launch_gemm_pair(L->map_w1, L->map_w1h, m_x, m_x16, m_x, m_x16, g1, s, &launches));
+    MOE_LAUNCH(launch_gemm_pair(L->map_w2, L->map_w2h, m_h, m_h16, m_h, m_h16, g2, s, &launches));
     return MOE_OK;
 }
 

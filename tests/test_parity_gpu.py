@@ -251,11 +251,14 @@ def test_dp_stats_two_shards_through_kernels():
     assert np.array_equal(out1["expert_loss"].cpu().numpy(), g_last["expert_loss"].astype(np.float32))
 
 
-def test_ragged_n_tiles_both_layers():
-    """Expert widths that are not multiples of the 256-column N tile: layer 1
-    ends with a 64-column tile (F = 1088), layer 2 with a 64-column tile that
-    also carries the credit's norm partials (O = 320)."""
-    w = WORKLOADS["default"].with_(T=777, F=1088, O=320, S=1, activation="swish")
+@pytest.mark.parametrize("F,O", [(1088, 320), (704, 384)])
+def test_ragged_n_tiles_both_layers(F, O):
+    """Expert widths that are not multiples of the 256-feature tile. A last
+    tile of at most 128 features runs as a transposed unit (tokens on the
+    MMA's M side): 64 features (F = 1088, O = 320) or 128 (O = 384); a last
+    tile of 192 features (F = 704) runs as an ordinary unit with a partly idle
+    M side."""
+    w = WORKLOADS["default"].with_(T=777, F=F, O=O, S=1, activation="swish")
     full_check(w, make_inputs(w, "cpu", seed=13, random_biases=True))
 
 
