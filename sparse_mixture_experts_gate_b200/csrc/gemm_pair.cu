@@ -54,17 +54,23 @@
 namespace moe {
 namespace {
 
-constexpr int kEpiWarps = 4;                        // epilogue warps per CTA (a multiple of 4)
+constexpr int kEpiWarps = 4;                        // epilogue warps per CTA, one per TMEM lane quarter
 constexpr int kThreads = 64 + 32 * kEpiWarps;
+// Output stores: true, the four epilogue warps fill a shared box of 32 tokens
+// x 128 features (256-byte rows) that one thread stores with a TMA tensor
+// store; false, every lane stores its own 32-bit pairs (64-byte pieces of rows).
+constexpr bool kWideStores = true;
 constexpr int kFeatPair = 256;                     // MMA M: features per pair tile
 constexpr int kFeatCta = 128;                      // features per CTA
+constexpr int kOutBoxBytes = 32 * kFeatCta * 2;    // one staged output box: 32 tokens x 128 features
 constexpr int kABytes = kFeatCta * kBK * 2;        // 16 KB: 128 weight rows x 64 K
 constexpr int kAccCols = 256;
 constexpr int kBoxTok = 32;                         // tokens per TMEM load of the epilogue
 constexpr int kRowsPerLoad16 = 16;                  // rows of the narrow token box
 constexpr int kRing = 8;            // unit-index ring between the leader's producer and the consumers
-// leader: MMA thread + the epilogue warps; peer: producer + the epilogue warps
-constexpr int kRingConsumers = 2 * (1 + kEpiWarps);
+// leader: MMA thread + the epilogue (its one unit-taking thread with wide
+// stores, else every epilogue warp); peer: producer + the epilogue
+constexpr int kRingConsumers = kWideStores ? 4 : 2 * (1 + kEpiWarps);
 static_assert(kTokTile == 256 && kTokTile % (2 * kRowsPerLoad16) == 0, "token tile layout");
 static_assert(kNarrowTile % (2 * kRowsPerLoad16) == 0, "narrow token tile layout");
 
@@ -76,17 +82,19 @@ template <int TILE>
 struct PairCfg {
     static constexpr int kB = (TILE / 2) * kBK * 2;
     static constexpr int kStage = kABytes + kB;
-    static constexpr int kStages = TILE == kTokTile ? 7 : 11;
-    static constexpr int kSmem = 1024 + kStages * kStage + 512;
+    static constexpr int kStaging = kWideStores ? 2 * kOutBoxBytes : 0;
+    static constexpr int kStages = (TILE == kTokTile ? 7 : 11) - (kWideStores ? 1 : 0);
+    static constexpr int kSmem = 1024 + kStages * kStage + kStaging + 512;
     static_assert(kSmem <= 232448, "exceeds the 227 KB of shared memory a CTA may use");
     static_assert(kB % 1024 == 0, "B stages keep the 1024-byte swizzle alignment");
 };
 
 struct Smem {
-    uint8_t *sA, *sB;
+    uint8_t *sA, *sB, *staging;
     uint64_t *full, *empty, *tfull, *tempty, *mma_done, *ring_full, *ring_empty;
     uint32_t *tmem_slot;
     int32_t *ring;
+    int32_t *epi_unit;  // [2] the unit the epilogue drains, by parity (wide stores)
 };
 
 template <int TILE>
@@ -96,7 +104,8 @@ __device__ __forceinline__ Smem carve(uint8_t *raw) {
     Smem s;
     s.sA = base;
     s.sB = base + C::kStages * kABytes;
-    s.full = reinterpret_cast<uint64_t *>(base + C::kStages * C::kStage);
+    s.staging = base + C::kStages * C::kStage;
+    s.full = reinterpret_cast<uint64_t *>(s.staging + C::kStaging);
     s.empty = s.full + C::kStages;
     s.tfull = s.empty + C::kStages;
     s.tempty = s.tfull + 2;
@@ -105,15 +114,19 @@ __device__ __forceinline__ Smem carve(uint8_t *raw) {
     s.ring_empty = s.ring_full + kRing;
     s.tmem_slot = reinterpret_cast<uint32_t *>(s.ring_empty + kRing);
     s.ring = reinterpret_cast<int32_t *>(s.tmem_slot + 4);
+    s.epi_unit = s.ring + kRing;
     return s;
 }
+
+// Named barrier 1 over the four epilogue warps (threads 64..191).
+__device__ __forceinline__ void epi_bar_sync() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
 
 template <int ACT, int TILE>
 __global__ void __launch_bounds__(kThreads, 1)
     grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap map_w, const __grid_constant__ CUtensorMap map_wh,
                              const __grid_constant__ CUtensorMap map_t,
                              const __grid_constant__ CUtensorMap map_t16, const __grid_constant__ CUtensorMap map_s,
-                             const __grid_constant__ CUtensorMap map_s16,
+                             const __grid_constant__ CUtensorMap map_s16, const __grid_constant__ CUtensorMap map_out,
                              const PairGemmArgs a) {
     using C = PairCfg<TILE>;
     constexpr int kStages = C::kStages;
@@ -130,6 +143,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         tma_prefetch_desc(&map_t16);
         tma_prefetch_desc(&map_s);
         tma_prefetch_desc(&map_s16);
+        if (kWideStores) tma_prefetch_desc(&map_out);
         for (int i = 0; i < kStages; ++i) {
             mbar_init(&s.full[i], 1);
             mbar_init(&s.empty[i], 1);
@@ -284,23 +298,40 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
     } else {
         // ------------------------------------------------------------ epilogue
-        const int q = warp & 3;  // TMEM lane quarter this warp may access
-        // The warps sharing a lane quarter take alternate 32-column chunks.
-        const int part = (warp - 2) >> 2, nparts = kEpiWarps / 4;
+        const int q = warp & 3;        // TMEM lane quarter this warp may access
+        const int ep = threadIdx.x - 64;  // 0..127 over the four epilogue warps
+        uint32_t sub = 0;              // output boxes staged so far (buffer parity)
         for (uint32_t tcount = 0;; ++tcount) {
-            int u = 0;
-            if (lane == 0) u = take_unit(tcount);
-            u = __shfl_sync(0xffffffffu, u, 0);
-            if (u < 0) break;
+            const uint32_t acc = tcount & 1u, use = tcount >> 1;
+            int u;
+            if constexpr (kWideStores) {
+                // One thread takes the unit and waits for its accumulator; the
+                // four warps agree on the outcome at a named barrier, so they
+                // all pass the same barriers below and leave together.
+                if (ep == 0) {
+                    int v = take_unit(tcount);
+                    if (v >= 0 && !mbar_wait_idle(&s.tfull[acc], use & 1u, a.status, a.wait_limit_ns)) v = -2;
+                    s.epi_unit[tcount & 1u] = v;
+                }
+                epi_bar_sync();
+                u = *reinterpret_cast<volatile int32_t *>(&s.epi_unit[tcount & 1u]);
+                if (u < 0) break;
+            } else {
+                u = 0;
+                if (lane == 0) u = take_unit(tcount);
+                u = __shfl_sync(0xffffffffu, u, 0);
+                if (u < 0) break;
+                int got = 1;  // one lane waits; tcgen05.ld below is warp-collective
+                if (lane == 0) got = mbar_wait_idle(&s.tfull[acc], use & 1u, a.status, a.wait_limit_ns) ? 1 : 0;
+                if (!__shfl_sync(0xffffffffu, got, 0)) break;
+            }
+            tc_fence_after_sync();
             const int tt = u / a.n_ftiles, j = u - tt * a.n_ftiles;
             const int4 tile = tok_tiles[tt];
             const int g = tile.x, row0 = tile.y, ntok = tile.z;
-            const int fcol = j * kFeatPair + static_cast<int>(rank) * kFeatCta + q * 32;
-            const uint32_t acc = tcount & 1u, use = tcount >> 1;
-            int got = 1;  // one lane waits; tcgen05.ld below is warp-collective
-            if (lane == 0) got = mbar_wait_idle(&s.tfull[acc], use & 1u, a.status, a.wait_limit_ns) ? 1 : 0;
-            if (!__shfl_sync(0xffffffffu, got, 0)) break;
-            tc_fence_after_sync();
+            const int fbase = j * kFeatPair + static_cast<int>(rank) * kFeatCta;
+            const int fcol = fbase + q * 32;
+            const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * kAccCols;
             if (j == tr_tile) {
                 // Transposed unit: TMEM lane = token (this CTA's ntok / 2
                 // tokens first), column = feature. Each lane activates 32
@@ -309,9 +340,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const int half = ntok / 2, tok = q * 32 + lane;
                 const int f0 = j * kFeatPair;
                 __nv_bfloat16 *orow = a.out + (static_cast<int64_t>(row0) + static_cast<int64_t>(rank) * half + tok) * a.N;
-                const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * kAccCols;
 #pragma unroll 1
-                for (int c = 32 * part; c < kFeatCta && f0 + c < a.N; c += 32 * nparts) {
+                for (int c = 0; c < kFeatCta && f0 + c < a.N; c += 32) {
                     const float bl = a.bias ? __ldg(a.bias + (int64_t)wgroup(g) * a.N + f0 + c + lane) : 0.f;
                     uint32_t r[32];
                     tmem_ld_32x32b_x32(taddr + c, r);
@@ -332,30 +362,53 @@ __global__ void __launch_bounds__(kThreads, 1)
                             dst[v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
                     }
                 }
-            } else if (fcol < a.N) {  // the last feature tile of a ragged N has an idle half
-                const float b = a.bias ? __ldg(a.bias + (int64_t)wgroup(g) * a.N + fcol + lane) : 0.f;
-                const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * kAccCols;
+            } else {
+                // Lane = feature, register = token. Neighbouring lanes trade
+                // one value per token pair, so the even lane holds features
+                // (f, f+1) of token t and the odd lane those of token t+1: one
+                // bf16x2 conversion and one 32-bit store each. The last
+                // feature tile of a ragged N leaves the warps past N idle.
+                const bool valid = fcol < a.N;
+                const float b = valid && a.bias ? __ldg(a.bias + (int64_t)wgroup(g) * a.N + fcol + lane) : 0.f;
+                const uint32_t odd = lane & 1u;
 #pragma unroll 1
-                for (int c = kBoxTok * part; c < ntok; c += kBoxTok * nparts) {
-                    uint32_t r[32];
-                    tmem_ld_32x32b_x32(taddr + c, r);
-                    tmem_ld_wait();
-                    // Lane = feature, register = token. Neighbouring lanes
-                    // trade one value per token pair, so the even lane holds
-                    // features (f, f+1) of token t and the odd lane those of
-                    // token t+1: one bf16x2 conversion and one 32-bit store
-                    // each, 16 lanes writing 64 contiguous bytes of a row.
-                    const uint32_t odd = lane & 1u;
-                    uint32_t *dst = reinterpret_cast<uint32_t *>(
-                        a.out + static_cast<int64_t>(row0 + c + static_cast<int>(odd)) * a.N + fcol + (lane & ~1u));
-                    const int64_t two_rows = static_cast<int64_t>(a.N);  // 2 rows in 32-bit words
+                for (int c = 0; c < ntok; c += kBoxTok) {
+                    uint32_t *dst;
+                    int64_t two_rows;  // the word stride of two token rows
+                    uint8_t *buf = nullptr;
+                    if constexpr (kWideStores) {
+                        // The box staged two boxes ago has been read by its store.
+                        buf = s.staging + (sub & 1u) * kOutBoxBytes;
+                        if (ep == 0) bulk_wait_group_read<1>();
+                        epi_bar_sync();
+                        dst = reinterpret_cast<uint32_t *>(buf) + odd * (kFeatCta / 2) + q * 16 + (lane >> 1);
+                        two_rows = kFeatCta;
+                    } else {
+                        dst = reinterpret_cast<uint32_t *>(a.out + static_cast<int64_t>(row0 + c + static_cast<int>(odd)) * a.N +
+                                                           fcol + (lane & ~1u));
+                        two_rows = a.N;
+                    }
+                    if (valid) {
+                        uint32_t r[32];
+                        tmem_ld_32x32b_x32(taddr + c, r);
+                        tmem_ld_wait();
 #pragma unroll
-                    for (int t = 0; t < 32; t += 2) {
-                        const float z0 = activate_t<ACT>(__uint_as_float(r[t]) + b);
-                        const float z1 = activate_t<ACT>(__uint_as_float(r[t + 1]) + b);
-                        const float other = __shfl_xor_sync(0xffffffffu, odd ? z0 : z1, 1);
-                        __nv_bfloat162 p = odd ? __floats2bfloat162_rn(other, z1) : __floats2bfloat162_rn(z0, other);
-                        dst[(t / 2) * two_rows] = *reinterpret_cast<uint32_t *>(&p);
+                        for (int t = 0; t < 32; t += 2) {
+                            const float z0 = activate_t<ACT>(__uint_as_float(r[t]) + b);
+                            const float z1 = activate_t<ACT>(__uint_as_float(r[t + 1]) + b);
+                            const float other = __shfl_xor_sync(0xffffffffu, odd ? z0 : z1, 1);
+                            __nv_bfloat162 p = odd ? __floats2bfloat162_rn(other, z1) : __floats2bfloat162_rn(z0, other);
+                            dst[(t / 2) * two_rows] = *reinterpret_cast<uint32_t *>(&p);
+                        }
+                    }
+                    if constexpr (kWideStores) {
+                        fence_proxy_async_smem();
+                        epi_bar_sync();
+                        if (ep == 0 && fbase < a.N) {  // columns past N are clipped by the store
+                            tma_store_2d(&map_out, buf, fbase, row0 + c);
+                            bulk_commit_group();
+                        }
+                        ++sub;
                     }
                 }
             }
@@ -363,6 +416,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             __syncwarp();
             if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(&s.tempty[acc]), 0));
         }
+        if (kWideStores && ep == 0) bulk_wait_group<0>();  // all stores complete before exit
     }
 
     // A role that gave up may leave its own TMA loads in flight; they land
@@ -379,7 +433,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 template <int ACT, int TILE>
 cudaError_t launch_act(const CUtensorMap &mw, const CUtensorMap &mwh, const CUtensorMap &mt, const CUtensorMap &mt16, const CUtensorMap &ms,
-                       const CUtensorMap &ms16, const PairGemmArgs &a, cudaStream_t st) {
+                       const CUtensorMap &ms16, const CUtensorMap &mo, const PairGemmArgs &a, cudaStream_t st) {
     constexpr int kSmem = PairCfg<TILE>::kSmem;
     auto kern = grouped_gemm_pair_kernel<ACT, TILE>;
     cudaError_t e = set_smem_limit_once<grouped_gemm_pair_kernel<ACT, TILE>>(kSmem);
@@ -396,7 +450,7 @@ cudaError_t launch_act(const CUtensorMap &mw, const CUtensorMap &mwh, const CUte
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, kern, mw, mwh, mt, mt16, ms, ms16, a);
+    return cudaLaunchKernelEx(&cfg, kern, mw, mwh, mt, mt16, ms, ms16, mo, a);
 }
 
 }  // namespace
@@ -428,23 +482,23 @@ int gemm_pair_ftiles(int N) { return (N + kFeatPair - 1) / kFeatPair; }
 int gemm_pair_half_last(int N) { return N % kFeatPair != 0 && N % kFeatPair <= kFeatCta ? 1 : 0; }
 
 cudaError_t launch_gemm_pair(const CUtensorMap &map_w, const CUtensorMap &map_wh, const CUtensorMap &map_t, const CUtensorMap &map_t16,
-                             const CUtensorMap &map_s, const CUtensorMap &map_s16,
+                             const CUtensorMap &map_s, const CUtensorMap &map_s16, const CUtensorMap &map_out,
                              const PairGemmArgs &a, cudaStream_t s, int *launches) {
     if (a.num_pairs <= 0) return cudaErrorInvalidConfiguration;
     ++*launches;
     if (a.narrow) {
         switch (a.act) {
-            case 0: return launch_act<0, kNarrowTile>(map_w, map_wh, map_t, map_t16, map_s, map_s16, a, s);
-            case 1: return launch_act<1, kNarrowTile>(map_w, map_wh, map_t, map_t16, map_s, map_s16, a, s);
-            case 2: return launch_act<2, kNarrowTile>(map_w, map_wh, map_t, map_t16, map_s, map_s16, a, s);
-            default: return launch_act<-1, kNarrowTile>(map_w, map_wh, map_t, map_t16, map_s, map_s16, a, s);
+            case 0: return launch_act<0, kNarrowTile>(map_w, map_wh, map_t, map_t16, map_s, map_s16, map_out, a, s);
+            case 1: return launch_act<1, kNarrowTile>(map_w, map_wh, map_t, map_t16, map_s, map_s16, map_out, a, s);
+            case 2: return launch_act<2, kNarrowTile>(map_w, map_wh, map_t, map_t16, map_s, map_s16, map_out, a, s);
+            default: return launch_act<-1, kNarrowTile>(map_w, map_wh, map_t, map_t16, map_s, map_s16, map_out, a, s);
         }
     }
     switch (a.act) {
-        case 0: return launch_act<0, kTokTile>(map_w, map_wh, map_t, map_t16, map_s, map_s16, a, s);
-        case 1: return launch_act<1, kTokTile>(map_w, map_wh, map_t, map_t16, map_s, map_s16, a, s);
-        case 2: return launch_act<2, kTokTile>(map_w, map_wh, map_t, map_t16, map_s, map_s16, a, s);
-        default: return launch_act<-1, kTokTile>(map_w, map_wh, map_t, map_t16, map_s, map_s16, a, s);
+        case 0: return launch_act<0, kTokTile>(map_w, map_wh, map_t, map_t16, map_s, map_s16, map_out, a, s);
+        case 1: return launch_act<1, kTokTile>(map_w, map_wh, map_t, map_t16, map_s, map_s16, map_out, a, s);
+        case 2: return launch_act<2, kTokTile>(map_w, map_wh, map_t, map_t16, map_s, map_s16, map_out, a, s);
+        default: return launch_act<-1, kTokTile>(map_w, map_wh, map_t, map_t16, map_s, map_s16, map_out, a, s);
     }
 }
 

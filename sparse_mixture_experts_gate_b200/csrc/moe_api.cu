@@ -66,6 +66,20 @@ bool encode_bf16_2d(CUtensorMap *m, const void *base, uint64_t inner, uint64_t r
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Row-major bf16 [rows][inner] output map for the expert GEMM's stores: box of
+// 128 x 32 elements (32 rows of 256 bytes), no swizzle.
+bool encode_bf16_store(CUtensorMap *m, const void *base, uint64_t inner, uint64_t rows) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn || rows == 0) return false;
+    cuuint64_t dims[2] = {inner, rows};
+    cuuint64_t strides[1] = {inner * 2};
+    cuuint32_t box[2] = {128, 32};
+    cuuint32_t es[2] = {1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box, es,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 struct Plan {
     int T = 0;
     int64_t C = 0;
@@ -604,16 +618,18 @@ int fwd_expert_gemms(moe_layer_t *L, cudaStream_t s, bool shared_only) {
         g2.bias = L->w.b2;
         g2.act = -1;
         g2.work_counter = ctrl + kCtrlWork2;
-        CUtensorMap m_xp, m_xp16, m_x, m_x16, m_h, m_h16;
+        CUtensorMap m_xp, m_xp16, m_x, m_x16, m_h, m_h16, m_hs, m_os;
         if (!encode_bf16_2d(&m_xp, ws + p.o_xp, c.input_dim, p.R_routed_max, 128) ||
             !encode_bf16_2d(&m_xp16, ws + p.o_xp, c.input_dim, p.R_routed_max, 16) ||
             !encode_bf16_2d(&m_x, x, c.input_dim, T, 128) || !encode_bf16_2d(&m_x16, x, c.input_dim, T, 16) ||
             !encode_bf16_2d(&m_h, ws + p.o_h, c.expert_dim, p.R_max, 128) ||
-            !encode_bf16_2d(&m_h16, ws + p.o_h, c.expert_dim, p.R_max, 16))
+            !encode_bf16_2d(&m_h16, ws + p.o_h, c.expert_dim, p.R_max, 16) ||
+            !encode_bf16_store(&m_hs, ws + p.o_h, c.expert_dim, p.R_max) ||
+            !encode_bf16_store(&m_os, ws + p.o_o, c.output_dim, p.R_max))
             return fail(MOE_ERR_CUDA, "cuTensorMapEncodeTiled failed for the activations");
-        MOE_LAUNCH(launch_gemm_pair(L->map_w1, L->map_w1h, m_xp, m_xp16, m_x, m_x16, g1, s, nl));
+        MOE_LAUNCH(launch_gemm_pair(L->map_w1, L->map_w1h, m_xp, m_xp16, m_x, m_x16, m_hs, g1, s, nl));
         MOE_MARK(L, 4, s);
-        MOE_LAUNCH(launch_gemm_pair(L->map_w2, L->map_w2h, m_h, m_h16, m_h, m_h16, g2, s, nl));
+        MOE_LAUNCH(launch_gemm_pair(L->map_w2, L->map_w2h, m_h, m_h16, m_h, m_h16, m_os, g2, s, nl));
         MOE_MARK(L, 5, s);
     } else {
         GemmSimtArgs s1;
@@ -833,13 +849,14 @@ int moe_ep_experts(moe_layer_t *L, const void *recv_x, const int32_t *recv_rows,
     g2.bias = L->w.b2;
     g2.act = -1;
     g2.work_counter = ctrl + kCtrlWork2;
-    CUtensorMap m_x, m_x16, m_h, m_h16;
+    CUtensorMap m_x, m_x16, m_h, m_h16, m_hs, m_os;
     if (!encode_bf16_2d(&m_x, recv_x, c.input_dim, R, 128) || !encode_bf16_2d(&m_x16, recv_x, c.input_dim, R, 16) ||
         !encode_bf16_2d(&m_h, ws + q.o_h, c.expert_dim, R, 128) ||
-        !encode_bf16_2d(&m_h16, ws + q.o_h, c.expert_dim, R, 16))
+        !encode_bf16_2d(&m_h16, ws + q.o_h, c.expert_dim, R, 16) ||
+        !encode_bf16_store(&m_hs, ws + q.o_h, c.expert_dim, R) || !encode_bf16_store(&m_os, recv_out, c.output_dim, R))
         return fail(MOE_ERR_CUDA, "cuTensorMapEncodeTiled failed for the received rows");
-    MOE_LAUNCH(launch_gemm_pair(L->map_w1, L->map_w1h, m_x, m_x16, m_x, m_x16, g1, s, &launches));
-    MOE_LAUNCH(launch_gemm_pair(L->map_w2, L->map_w2h, m_h, m_h16, m_h, m_h16, g2, s, &launches));
+    MOE_LAUNCH(launch_gemm_pair(L->map_w1, L->map_w1h, m_x, m_x16, m_x, m_x16, m_hs, g1, s, &launches));
+    MOE_LAUNCH(launch_gemm_pair(L->map_w2, L->map_w2h, m_h, m_h16, m_h, m_h16, m_os, g2, s, &launches));
     return MOE_OK;
 }
 

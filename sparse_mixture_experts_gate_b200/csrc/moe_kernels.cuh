@@ -139,8 +139,9 @@ cudaError_t launch_scatter(const ScatterArgs &a, int num_sms, cudaStream_t s, in
 // 256-feature tile). map_w: the weight stack [G*N][K] (box 64 x 128; map_wh
 // the same with box 64 x 64); map_t / map_t16: the token rows in row order
 // (box 64 x 128 and 64 x 16); map_s / map_s16: with use_s, the token rows of
-// shared-expert groups (x itself, in token order). The outputs are stored to
-// `out` ([rows][N] bf16). N and K must be multiples of 64.
+// shared-expert groups (x itself, in token order); map_out: the output
+// [rows][N] bf16 (box 128 x 32, no swizzle), also addressed directly through
+// `out`. N and K must be multiples of 64.
 struct PairGemmArgs {
     const int4 *tok_tiles;       // [max_tok_tiles] {group, first row, rows, 0}
     const int32_t *group_start;  // [G+1]
@@ -158,7 +159,7 @@ struct PairGemmArgs {
     // 1: the last feature tile holds at most 128 features (N % 256 in {64, 128})
     // and its units run transposed (wide token tiles only), storing through `out`.
     int half_last = 0;
-    __nv_bfloat16 *out = nullptr;  // [rows][N] bf16 output (row space), written directly
+    __nv_bfloat16 *out = nullptr;  // [rows][N] bf16 output (row space), the array map_out covers
     const float *bias;           // [G][N] or null
     int act;                     // activation code, -1 none
     uint32_t *status;            // device status word
@@ -175,7 +176,7 @@ int gemm_pair_ftiles(int N);
 int gemm_pair_half_last(int N);  // 1 when the last feature tile of N holds at most 128 features
 // map_wh: the weights with boxes of 64 rows (transposed last-tile units).
 cudaError_t launch_gemm_pair(const CUtensorMap &map_w, const CUtensorMap &map_wh, const CUtensorMap &map_t, const CUtensorMap &map_t16,
-                             const CUtensorMap &map_s, const CUtensorMap &map_s16,
+                             const CUtensorMap &map_s, const CUtensorMap &map_s16, const CUtensorMap &map_out,
                              const PairGemmArgs &a, cudaStream_t s, int *launches);
 
 // fp32 CUDA-core path: 32 x 32 output tiles over the 32-row blocks.
