@@ -24,17 +24,19 @@
 // E = 256 layer and the L2 reuse of the weight tiles collapses (GEMM 1 read
 // 41.6 GB from DRAM instead of ~15 GB).
 //
-// Per CTA (192 threads with four epilogue warps): warp 0 loads (TMA, signalling the leader's stage
+// Per CTA (192 threads): warp 0 loads (TMA, signalling the leader's stage
 // barrier, which expects both CTAs' bytes), warp 1 owns TMEM (2 accumulators x
 // 256 columns) and, in the leader, issues the pair MMAs and commits stages and
 // accumulators to both CTAs at once; warps 2..5 drain this CTA's 128 features:
 // each warp reads 32 features x 32 tokens from TMEM, adds the bias, applies the
 // activation, pairs neighbouring lanes' values so that each lane holds two
-// adjacent features of one token, and stores them to global memory (a warp
-// store covers 64 contiguous bytes of each of two token rows). No shared
-// memory is spent on staging the outputs, so it holds seven 32 KB pipeline
-// stages. The epilogue releases an accumulator by arriving on the leader's
-// barrier (one arrival per epilogue warp of both CTAs).
+// adjacent features of one token, and writes them into a shared box of 32
+// tokens x 128 features (token-major, 256-byte rows) that the four warps fill
+// together; one thread stores each box with a TMA tensor store. One epilogue
+// thread takes each unit and waits for its accumulator, and the four warps
+// agree on it at a named barrier, so all of them pass the same barriers and
+// leave together. The epilogue releases an accumulator by arriving on the
+// leader's barrier (one arrival per epilogue warp of both CTAs).
 //
 // Ragged last feature tile. When N leaves a last feature tile of at most 128
 // features (d_ff = 1408 = 5.5 x 256, say), a unit of that tile would leave
@@ -75,9 +77,10 @@ static_assert(kTokTile == 256 && kTokTile % (2 * kRowsPerLoad16) == 0, "token ti
 static_assert(kNarrowTile % (2 * kRowsPerLoad16) == 0, "narrow token tile layout");
 
 // Stage layout for token tiles of up to TILE rows (each CTA stages TILE / 2):
-// 256-row tiles with 7 stages of 32 KB, or narrow 64-row tiles with 11 stages
-// of 20 KB, which keeps 176 KB of weight tiles in flight per SM when the
-// token tiles are short and the GEMM streams weights.
+// 256-row tiles with 6 stages of 32 KB, or narrow 64-row tiles with 10 stages
+// of 20 KB, which keeps 160 KB of weight tiles in flight per SM when the
+// token tiles are short and the GEMM streams weights (one stage more of each
+// when the outputs are stored from registers, without staging boxes).
 template <int TILE>
 struct PairCfg {
     static constexpr int kB = (TILE / 2) * kBK * 2;
