@@ -150,6 +150,8 @@ __device__ __forceinline__ void dispatch_scan(const DispatchArgs &a) {
         a.group_start[a.E + e] = routed_rows + e * a.T_pad;
         a.group_rows[a.E + e] = a.T;
     }
+    if (a.tile_done)
+        for (int i = e; i < a.n_tile_done; i += kMaxE) a.tile_done[i] = 0;
     __syncthreads();
     if (e == 0) {
         int d = 0;

@@ -50,6 +50,8 @@
 // Every wait is bounded (mbar_wait); on a timeout the roles stop, the leader
 // drains its MMAs, copies in flight are given time to land, both CTAs meet at
 // the cluster barrier, and TMEM is freed.
+#include <type_traits>
+
 #include "moe_common.cuh"
 #include "moe_kernels.cuh"
 
@@ -126,11 +128,8 @@ __device__ __forceinline__ void epi_bar_sync() { asm volatile("bar.sync 1, 128;"
 
 template <int ACT, int TILE>
 __global__ void __launch_bounds__(kThreads, 1)
-    grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap map_w, const __grid_constant__ CUtensorMap map_wh,
-                             const __grid_constant__ CUtensorMap map_t,
-                             const __grid_constant__ CUtensorMap map_t16, const __grid_constant__ CUtensorMap map_s,
-                             const __grid_constant__ CUtensorMap map_s16, const __grid_constant__ CUtensorMap map_out,
-                             const PairGemmArgs a) {
+    grouped_gemm_pair_kernel(const __grid_constant__ PairMaps m1, const __grid_constant__ PairMaps m2,
+                             const PairGemmArgs a, const PairGemmArgs b) {
     using C = PairCfg<TILE>;
     constexpr int kStages = C::kStages;
     extern __shared__ uint8_t smem_raw[];
@@ -138,15 +137,21 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const uint32_t rank = cluster_ctarank();
     const bool leader = rank == 0;
+    const bool two = a.fuse2 != 0;  // layer 2 (b, m2) follows layer 1 (a, m1) in this launch
 
     if (threadIdx.x == 0) {
-        tma_prefetch_desc(&map_w);
-        if (a.half_last) tma_prefetch_desc(&map_wh);
-        tma_prefetch_desc(&map_t);
-        tma_prefetch_desc(&map_t16);
-        tma_prefetch_desc(&map_s);
-        tma_prefetch_desc(&map_s16);
-        if (kWideStores) tma_prefetch_desc(&map_out);
+        for (int l = 0; l < (two ? 2 : 1); ++l) {
+            const PairMaps &m = l ? m2 : m1;
+            tma_prefetch_desc(&m.w);
+            if ((l ? b : a).half_last) tma_prefetch_desc(&m.wh);
+            tma_prefetch_desc(&m.t);
+            tma_prefetch_desc(&m.t16);
+            if ((l ? b : a).use_s) {
+                tma_prefetch_desc(&m.s);
+                tma_prefetch_desc(&m.s16);
+            }
+            if (kWideStores) tma_prefetch_desc(&m.out);
+        }
         for (int i = 0; i < kStages; ++i) {
             mbar_init(&s.full[i], 1);
             mbar_init(&s.empty[i], 1);
@@ -173,20 +178,33 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     const int4 *tok_tiles = a.tok_tiles + (a.tile_base_word >= 0 ? a.ctrl[a.tile_base_word] : 0);
     const int n_tt = a.fixed_tiles > 0 ? a.fixed_tiles : min(a.ctrl[a.tiles_count_word], a.max_tok_tiles);
-    const int total = n_tt * a.n_ftiles;
+    // Units are numbered layer by layer: (token tile, feature tile) of layer
+    // 1, then of layer 2, which reads layer 1's output rows.
+    const int total1 = n_tt * a.n_ftiles;
+    const int total = total1 + (two ? n_tt * b.n_ftiles : 0);
+    // Layer of unit u, with its token tile and feature tile.
+    auto decode = [&](int u, int &tt, int &j) -> int {
+        const int l = u >= total1 ? 1 : 0;
+        const int v = u - (l ? total1 : 0), nf = l ? b.n_ftiles : a.n_ftiles;
+        tt = v / nf;
+        j = v - tt * nf;
+        return l;
+    };
     // Weight-stack index of group g (shared groups may sit at another base).
     auto wgroup = [&](int g) { return g < a.E ? g : a.w_shared_base + (g - a.E); };
-    const int kblocks = a.K / kBK;
-    // Units of the last feature tile run transposed (wide token tiles only).
-    const int tr_tile = (TILE == kTokTile && a.half_last) ? a.n_ftiles - 1 : -1;
+    // The last feature tile of a layer runs transposed (wide token tiles only).
+    auto tr_tile = [&](int l) {
+        const PairGemmArgs &P = l ? b : a;
+        return (TILE == kTokTile && P.half_last) ? P.n_ftiles - 1 : -1;
+    };
     bool ok = true;
 
-    // Units (token tile, feature tile) are handed out in index order from a
-    // global counter, so the pairs working at any moment hold a contiguous run
-    // of units and share their weight and token tiles through L2, however
-    // unequal the units' lengths. The leader's producer takes each unit and
-    // posts it to a ring in both CTAs; every consumer reads entry i for its
-    // i-th unit and releases it on the leader's ring_empty. -1 ends the work.
+    // Units are handed out in index order from a global counter, so the pairs
+    // working at any moment hold a contiguous run of units and share their
+    // weight and token tiles through L2, however unequal the units' lengths.
+    // The leader's producer takes each unit and posts it to a ring in both
+    // CTAs; every consumer reads entry i for its i-th unit and releases it on
+    // the leader's ring_empty. -1 ends the work.
     auto post_unit = [&](uint32_t i) -> int {  // leader's producer, lane 0
         const uint32_t slot = i % kRing, ph = (i / kRing) & 1u;
         if (!mbar_wait_cluster(&s.ring_empty[slot], ph ^ 1u, a.status, a.wait_limit_ns)) return -2;
@@ -217,21 +235,39 @@ __global__ void __launch_bounds__(kThreads, 1)
                 ok = u == -1;
                 break;
             }
-            const int tt = u / a.n_ftiles, j = u - tt * a.n_ftiles;
+            int tt, j;
+            const int l = decode(u, tt, j);
+            const PairGemmArgs &P = l ? b : a;
+            const PairMaps &m = l ? m2 : m1;
             const int4 tile = tok_tiles[tt];  // {group, first row, rows, -}
             const int g = tile.x, ntok = tile.z;
-            const CUtensorMap *mt = &map_t, *mt16 = &map_t16;
+            const CUtensorMap *mt = &m.t, *mt16 = &m.t16;
             int trow = tile.y + static_cast<int>(rank) * (ntok / 2);
-            if (a.use_s && g >= a.E) {  // shared expert: rows of x in token order
-                mt = &map_s;
-                mt16 = &map_s16;
+            if (P.use_s && g >= a.E) {  // shared expert: rows of x in token order
+                mt = &m.s;
+                mt16 = &m.s16;
                 trow -= a.group_start[g];
             }
-            const bool tr = j == tr_tile;  // 64 weight rows per CTA (the MMA's N side)
-            const int wrow = wgroup(g) * a.N + j * kFeatPair + static_cast<int>(rank) * (tr ? kFeatCta / 2 : kFeatCta);
-            const CUtensorMap *mw = tr ? &map_wh : &map_w;
+            if (l == 1) {
+                // Layer 2 reads the token tile's layer-1 outputs: wait until
+                // every layer-1 unit of the tile has stored them (both CTAs
+                // count), then order the tensor loads after that acquire.
+                int got = 1;
+                if (lane == 0)
+                    got = wait_counter_geq(a.tile_done + tt, 2 * a.n_ftiles, a.status, a.wait_limit_ns) ? 1 : 0;
+                got = __shfl_sync(0xffffffffu, got, 0);
+                if (!got) {
+                    ok = false;
+                    break;
+                }
+                fence_proxy_async_global();
+            }
+            const bool tr = j == tr_tile(l);  // 64 weight rows per CTA (the MMA's N side)
+            const int wrow = wgroup(g) * P.N + j * kFeatPair + static_cast<int>(rank) * (tr ? kFeatCta / 2 : kFeatCta);
+            const CUtensorMap *mw = tr ? &m.wh : &m.w;
             const uint32_t tx_bytes = (tr ? 1u : 2u) * kABytes + static_cast<uint32_t>(ntok) * kBK * 2u;
             const int n16 = ntok / (2 * kRowsPerLoad16);
+            const int kblocks = P.K / kBK;
             for (int kb = 0; kb < kblocks; ++kb, ++it) {
                 const int st = it % kStages;
                 const uint32_t ph = (it / kStages) & 1u;
@@ -269,10 +305,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                     ok = u == -1;
                     break;
                 }
-                const int ntok = tok_tiles[u / a.n_ftiles].z;
+                int tt, j;
+                const int l = decode(u, tt, j);
+                const int ntok = tok_tiles[tt].z;
+                const int kblocks = (l ? b : a).K / kBK;
                 // Transposed unit: A = the token tile (M = 256, each CTA's
                 // ntok / 2 rows first), B = the 128 features (64 rows per CTA).
-                const bool tr = u % a.n_ftiles == tr_tile;
+                const bool tr = j == tr_tile(l);
                 const uint32_t idesc = tr ? idesc_bf16_f32(kTokTile, kFeatCta) : idesc_bf16_f32(kFeatPair, ntok);
                 const uint32_t acc = tcount & 1u, use = tcount >> 1;
                 if (!mbar_wait(&s.tempty[acc], (use & 1u) ^ 1u, a.status, a.wait_limit_ns)) break;
@@ -304,6 +343,97 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int q = warp & 3;        // TMEM lane quarter this warp may access
         const int ep = threadIdx.x - 64;  // 0..127 over the four epilogue warps
         uint32_t sub = 0;              // output boxes staged so far (buffer parity)
+        // Drains one unit's accumulator with the activation ACT_C of its layer.
+        auto drain = [&](auto act_c, const PairGemmArgs &P, const PairMaps &m, int tr, int u_tt, int j,
+                         uint32_t acc) {
+            constexpr int A = decltype(act_c)::value;
+            const int4 tile = tok_tiles[u_tt];
+            const int g = tile.x, row0 = tile.y, ntok = tile.z;
+            const int fbase = j * kFeatPair + static_cast<int>(rank) * kFeatCta;
+            const int fcol = fbase + q * 32;
+            const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * kAccCols;
+            if (j == tr) {
+                // Transposed unit: TMEM lane = token (this CTA's ntok / 2
+                // tokens first), column = feature. Each lane activates 32
+                // consecutive features of its token and stores them as 64
+                // bytes; chunks past N (N % 256 == 64) are not stored.
+                const int half = ntok / 2, tok = q * 32 + lane;
+                const int f0 = j * kFeatPair;
+                __nv_bfloat16 *orow =
+                    P.out + (static_cast<int64_t>(row0) + static_cast<int64_t>(rank) * half + tok) * P.N;
+#pragma unroll 1
+                for (int c = 0; c < kFeatCta && f0 + c < P.N; c += 32) {
+                    const float bl = P.bias ? __ldg(P.bias + (int64_t)wgroup(g) * P.N + f0 + c + lane) : 0.f;
+                    uint32_t r[32];
+                    tmem_ld_32x32b_x32(taddr + c, r);
+                    tmem_ld_wait();
+                    uint32_t pk[16];
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) {
+                        const float z0 = activate_t<A>(__uint_as_float(r[2 * i]) + __shfl_sync(0xffffffffu, bl, 2 * i));
+                        const float z1 =
+                            activate_t<A>(__uint_as_float(r[2 * i + 1]) + __shfl_sync(0xffffffffu, bl, 2 * i + 1));
+                        __nv_bfloat162 p2 = __floats2bfloat162_rn(z0, z1);
+                        pk[i] = *reinterpret_cast<uint32_t *>(&p2);
+                    }
+                    if (tok < half) {
+                        uint4 *dst = reinterpret_cast<uint4 *>(orow + f0 + c);
+#pragma unroll
+                        for (int v = 0; v < 4; ++v)
+                            dst[v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
+                    }
+                }
+                return;
+            }
+            // Lane = feature, register = token. Neighbouring lanes trade one
+            // value per token pair, so the even lane holds features (f, f+1)
+            // of token t and the odd lane those of token t+1: one bf16x2
+            // conversion and one 32-bit store each. The last feature tile of
+            // a ragged N leaves the warps past N idle.
+            const bool valid = fcol < P.N;
+            const float bv = valid && P.bias ? __ldg(P.bias + (int64_t)wgroup(g) * P.N + fcol + lane) : 0.f;
+            const uint32_t odd = lane & 1u;
+#pragma unroll 1
+            for (int c = 0; c < ntok; c += kBoxTok) {
+                uint32_t *dst;
+                int64_t two_rows;  // the word stride of two token rows
+                uint8_t *buf = nullptr;
+                if constexpr (kWideStores) {
+                    // The box staged two boxes ago has been read by its store.
+                    buf = s.staging + (sub & 1u) * kOutBoxBytes;
+                    if (ep == 0) bulk_wait_group_read<1>();
+                    epi_bar_sync();
+                    dst = reinterpret_cast<uint32_t *>(buf) + odd * (kFeatCta / 2) + q * 16 + (lane >> 1);
+                    two_rows = kFeatCta;
+                } else {
+                    dst = reinterpret_cast<uint32_t *>(P.out + static_cast<int64_t>(row0 + c + static_cast<int>(odd)) * P.N +
+                                                       fcol + (lane & ~1u));
+                    two_rows = P.N;
+                }
+                if (valid) {
+                    uint32_t r[32];
+                    tmem_ld_32x32b_x32(taddr + c, r);
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int t = 0; t < 32; t += 2) {
+                        const float z0 = activate_t<A>(__uint_as_float(r[t]) + bv);
+                        const float z1 = activate_t<A>(__uint_as_float(r[t + 1]) + bv);
+                        const float other = __shfl_xor_sync(0xffffffffu, odd ? z0 : z1, 1);
+                        __nv_bfloat162 p = odd ? __floats2bfloat162_rn(other, z1) : __floats2bfloat162_rn(z0, other);
+                        dst[(t / 2) * two_rows] = *reinterpret_cast<uint32_t *>(&p);
+                    }
+                }
+                if constexpr (kWideStores) {
+                    fence_proxy_async_smem();
+                    epi_bar_sync();
+                    if (ep == 0 && fbase < P.N) {  // columns past N are clipped by the store
+                        tma_store_2d(&m.out, buf, fbase, row0 + c);
+                        bulk_commit_group();
+                    }
+                    ++sub;
+                }
+            }
+        };
         for (uint32_t tcount = 0;; ++tcount) {
             const uint32_t acc = tcount & 1u, use = tcount >> 1;
             int u;
@@ -329,95 +459,29 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (!__shfl_sync(0xffffffffu, got, 0)) break;
             }
             tc_fence_after_sync();
-            const int tt = u / a.n_ftiles, j = u - tt * a.n_ftiles;
-            const int4 tile = tok_tiles[tt];
-            const int g = tile.x, row0 = tile.y, ntok = tile.z;
-            const int fbase = j * kFeatPair + static_cast<int>(rank) * kFeatCta;
-            const int fcol = fbase + q * 32;
-            const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * kAccCols;
-            if (j == tr_tile) {
-                // Transposed unit: TMEM lane = token (this CTA's ntok / 2
-                // tokens first), column = feature. Each lane activates 32
-                // consecutive features of its token and stores them as 64
-                // bytes; chunks past N (N % 256 == 64) are not stored.
-                const int half = ntok / 2, tok = q * 32 + lane;
-                const int f0 = j * kFeatPair;
-                __nv_bfloat16 *orow = a.out + (static_cast<int64_t>(row0) + static_cast<int64_t>(rank) * half + tok) * a.N;
-#pragma unroll 1
-                for (int c = 0; c < kFeatCta && f0 + c < a.N; c += 32) {
-                    const float bl = a.bias ? __ldg(a.bias + (int64_t)wgroup(g) * a.N + f0 + c + lane) : 0.f;
-                    uint32_t r[32];
-                    tmem_ld_32x32b_x32(taddr + c, r);
-                    tmem_ld_wait();
-                    uint32_t pk[16];
-#pragma unroll
-                    for (int i = 0; i < 16; ++i) {
-                        const float z0 = activate_t<ACT>(__uint_as_float(r[2 * i]) + __shfl_sync(0xffffffffu, bl, 2 * i));
-                        const float z1 =
-                            activate_t<ACT>(__uint_as_float(r[2 * i + 1]) + __shfl_sync(0xffffffffu, bl, 2 * i + 1));
-                        __nv_bfloat162 p2 = __floats2bfloat162_rn(z0, z1);
-                        pk[i] = *reinterpret_cast<uint32_t *>(&p2);
-                    }
-                    if (tok < half) {
-                        uint4 *dst = reinterpret_cast<uint4 *>(orow + f0 + c);
-#pragma unroll
-                        for (int v = 0; v < 4; ++v)
-                            dst[v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
-                    }
-                }
-            } else {
-                // Lane = feature, register = token. Neighbouring lanes trade
-                // one value per token pair, so the even lane holds features
-                // (f, f+1) of token t and the odd lane those of token t+1: one
-                // bf16x2 conversion and one 32-bit store each. The last
-                // feature tile of a ragged N leaves the warps past N idle.
-                const bool valid = fcol < a.N;
-                const float b = valid && a.bias ? __ldg(a.bias + (int64_t)wgroup(g) * a.N + fcol + lane) : 0.f;
-                const uint32_t odd = lane & 1u;
-#pragma unroll 1
-                for (int c = 0; c < ntok; c += kBoxTok) {
-                    uint32_t *dst;
-                    int64_t two_rows;  // the word stride of two token rows
-                    uint8_t *buf = nullptr;
-                    if constexpr (kWideStores) {
-                        // The box staged two boxes ago has been read by its store.
-                        buf = s.staging + (sub & 1u) * kOutBoxBytes;
-                        if (ep == 0) bulk_wait_group_read<1>();
-                        epi_bar_sync();
-                        dst = reinterpret_cast<uint32_t *>(buf) + odd * (kFeatCta / 2) + q * 16 + (lane >> 1);
-                        two_rows = kFeatCta;
-                    } else {
-                        dst = reinterpret_cast<uint32_t *>(a.out + static_cast<int64_t>(row0 + c + static_cast<int>(odd)) * a.N +
-                                                           fcol + (lane & ~1u));
-                        two_rows = a.N;
-                    }
-                    if (valid) {
-                        uint32_t r[32];
-                        tmem_ld_32x32b_x32(taddr + c, r);
-                        tmem_ld_wait();
-#pragma unroll
-                        for (int t = 0; t < 32; t += 2) {
-                            const float z0 = activate_t<ACT>(__uint_as_float(r[t]) + b);
-                            const float z1 = activate_t<ACT>(__uint_as_float(r[t + 1]) + b);
-                            const float other = __shfl_xor_sync(0xffffffffu, odd ? z0 : z1, 1);
-                            __nv_bfloat162 p = odd ? __floats2bfloat162_rn(other, z1) : __floats2bfloat162_rn(z0, other);
-                            dst[(t / 2) * two_rows] = *reinterpret_cast<uint32_t *>(&p);
-                        }
-                    }
-                    if constexpr (kWideStores) {
-                        fence_proxy_async_smem();
-                        epi_bar_sync();
-                        if (ep == 0 && fbase < a.N) {  // columns past N are clipped by the store
-                            tma_store_2d(&map_out, buf, fbase, row0 + c);
-                            bulk_commit_group();
-                        }
-                        ++sub;
-                    }
-                }
-            }
+            int tt, j;
+            const int l = decode(u, tt, j);
+            if (l == 0)
+                drain(std::integral_constant<int, ACT>{}, a, m1, tr_tile(0), tt, j, acc);
+            else
+                drain(std::integral_constant<int, -1>{}, b, m2, tr_tile(1), tt, j, acc);
             tc_fence_before_sync();
             __syncwarp();
             if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(&s.tempty[acc]), 0));
+            if constexpr (kWideStores) {
+                if (two && l == 0) {
+                    // Publish this CTA's half of the unit's layer-1 outputs
+                    // for layer 2: the four warps' stores (the transposed
+                    // unit's direct ones included), the TMA stores'
+                    // completion, a proxy fence and a release increment.
+                    epi_bar_sync();
+                    if (ep == 0) {
+                        bulk_wait_group<0>();
+                        fence_proxy_async_global();
+                        red_release_add(a.tile_done + tt, 1);
+                    }
+                }
+            }
         }
         if (kWideStores && ep == 0) bulk_wait_group<0>();  // all stores complete before exit
     }
@@ -435,8 +499,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 template <int ACT, int TILE>
-cudaError_t launch_act(const CUtensorMap &mw, const CUtensorMap &mwh, const CUtensorMap &mt, const CUtensorMap &mt16, const CUtensorMap &ms,
-                       const CUtensorMap &ms16, const CUtensorMap &mo, const PairGemmArgs &a, cudaStream_t st) {
+cudaError_t launch_act(const PairMaps &m1, const PairMaps &m2, const PairGemmArgs &a, const PairGemmArgs &b,
+                       cudaStream_t st) {
     constexpr int kSmem = PairCfg<TILE>::kSmem;
     auto kern = grouped_gemm_pair_kernel<ACT, TILE>;
     cudaError_t e = set_smem_limit_once<grouped_gemm_pair_kernel<ACT, TILE>>(kSmem);
@@ -453,7 +517,7 @@ cudaError_t launch_act(const CUtensorMap &mw, const CUtensorMap &mwh, const CUte
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, kern, mw, mwh, mt, mt16, ms, ms16, mo, a);
+    return cudaLaunchKernelEx(&cfg, kern, m1, m2, a, b);
 }
 
 }  // namespace
@@ -484,24 +548,31 @@ int gemm_pair_ftiles(int N) { return (N + kFeatPair - 1) / kFeatPair; }
 
 int gemm_pair_half_last(int N) { return N % kFeatPair != 0 && N % kFeatPair <= kFeatCta ? 1 : 0; }
 
-cudaError_t launch_gemm_pair(const CUtensorMap &map_w, const CUtensorMap &map_wh, const CUtensorMap &map_t, const CUtensorMap &map_t16,
-                             const CUtensorMap &map_s, const CUtensorMap &map_s16, const CUtensorMap &map_out,
-                             const PairGemmArgs &a, cudaStream_t s, int *launches) {
+cudaError_t launch_gemm_pair(const PairMaps &m1, const PairGemmArgs &a, const PairMaps *m2, const PairGemmArgs *b,
+                             cudaStream_t s, int *launches) {
     if (a.num_pairs <= 0) return cudaErrorInvalidConfiguration;
+    // Two layers in one launch need the epilogue whose warps move together
+    // (kWideStores), a counter per token tile and the same tile table.
+    if ((m2 != nullptr) != (b != nullptr) || (b && (!kWideStores || !a.tile_done || b->narrow != a.narrow)))
+        return cudaErrorInvalidValue;
+    PairGemmArgs a1 = a;
+    a1.fuse2 = b ? 1 : 0;
+    const PairMaps &mm2 = m2 ? *m2 : m1;
+    const PairGemmArgs &bb = b ? *b : a;
     ++*launches;
     if (a.narrow) {
         switch (a.act) {
-            case 0: return launch_act<0, kNarrowTile>(map_w, map_wh, map_t, map_t16, map_s, map_s16, map_out, a, s);
-            case 1: return launch_act<1, kNarrowTile>(map_w, map_wh, map_t, map_t16, map_s, map_s16, map_out, a, s);
-            case 2: return launch_act<2, kNarrowTile>(map_w, map_wh, map_t, map_t16, map_s, map_s16, map_out, a, s);
-            default: return launch_act<-1, kNarrowTile>(map_w, map_wh, map_t, map_t16, map_s, map_s16, map_out, a, s);
+            case 0: return launch_act<0, kNarrowTile>(m1, mm2, a1, bb, s);
+            case 1: return launch_act<1, kNarrowTile>(m1, mm2, a1, bb, s);
+            case 2: return launch_act<2, kNarrowTile>(m1, mm2, a1, bb, s);
+            default: return launch_act<-1, kNarrowTile>(m1, mm2, a1, bb, s);
         }
     }
     switch (a.act) {
-        case 0: return launch_act<0, kTokTile>(map_w, map_wh, map_t, map_t16, map_s, map_s16, map_out, a, s);
-        case 1: return launch_act<1, kTokTile>(map_w, map_wh, map_t, map_t16, map_s, map_s16, map_out, a, s);
-        case 2: return launch_act<2, kTokTile>(map_w, map_wh, map_t, map_t16, map_s, map_s16, map_out, a, s);
-        default: return launch_act<-1, kTokTile>(map_w, map_wh, map_t, map_t16, map_s, map_s16, map_out, a, s);
+        case 0: return launch_act<0, kTokTile>(m1, mm2, a1, bb, s);
+        case 1: return launch_act<1, kTokTile>(m1, mm2, a1, bb, s);
+        case 2: return launch_act<2, kTokTile>(m1, mm2, a1, bb, s);
+        default: return launch_act<-1, kTokTile>(m1, mm2, a1, bb, s);
     }
 }
 

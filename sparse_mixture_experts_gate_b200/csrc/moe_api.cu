@@ -85,10 +85,11 @@ struct Plan {
     int64_t C = 0;
     int T_pad = 0, n_stat_chunks = 0, n_chunks = 0, R_routed_max = 0, R_max = 0, max_row_blocks = 0;
     int max_tok_tiles = 0, max_narrow_tiles = 0;
+    int n_tile_done = 0;  // per-token-tile counters of the two-layer expert GEMM launch
     int ksplit = 1, n_mtiles = 0;  // the fused router's K splits and token tiles
     size_t o_lpart = 0, ctrl_bytes = 0;
     size_t o_ctrl, o_rcnt, o_logits, o_idx, o_gates, o_slot, o_rowof, o_lse, o_psum, o_ccount, o_cbase, o_cpre, o_ckept,
-        o_gstart, o_grows, o_bgroup, o_toktiles, o_narrowtiles, o_rowassign, o_wsplit, o_xp, o_h, o_o, o_credit, o_partials,
+        o_gstart, o_grows, o_bgroup, o_toktiles, o_narrowtiles, o_tiledone, o_rowassign, o_wsplit, o_xp, o_h, o_o, o_credit, o_partials,
         o_prestart, o_gsorted, o_rownorm, o_gz;
     size_t total = 0;
 };
@@ -198,6 +199,8 @@ Plan make_plan(const moe_layer &L, int T) {
     p.o_bgroup = take((size_t)p.max_row_blocks * 4);
     p.o_toktiles = take((size_t)std::max(p.max_tok_tiles, 1) * 16);
     p.o_narrowtiles = take((size_t)std::max(p.max_narrow_tiles, 1) * 16);
+    p.n_tile_done = std::max(std::max(p.max_tok_tiles, p.max_narrow_tiles), 1);
+    p.o_tiledone = take((size_t)p.n_tile_done * 4);
     p.o_rowassign = take((size_t)p.R_max * 4);
     p.o_partials = take((size_t)(4 * E + 3) * 4);
     p.o_prestart = take((size_t)E * 4);
@@ -532,6 +535,8 @@ int fwd_route(moe_layer_t *L, const void *x, int32_t T, const float *logit_noise
     da.block_group = reinterpret_cast<int32_t *>(ws + p.o_bgroup);
     da.tok_tiles = reinterpret_cast<int4 *>(ws + p.o_toktiles);
     da.narrow_tiles = narrow_gemm(L, T) ? reinterpret_cast<int4 *>(ws + p.o_narrowtiles) : nullptr;
+    da.tile_done = reinterpret_cast<int32_t *>(ws + p.o_tiledone);
+    da.n_tile_done = p.n_tile_done;
     da.ctrl = ctrl;
     da.slot = slot;
     da.row_of = reinterpret_cast<int32_t *>(ws + p.o_rowof);
@@ -618,18 +623,36 @@ int fwd_expert_gemms(moe_layer_t *L, cudaStream_t s, bool shared_only) {
         g2.bias = L->w.b2;
         g2.act = -1;
         g2.work_counter = ctrl + kCtrlWork2;
-        CUtensorMap m_xp, m_xp16, m_x, m_x16, m_h, m_h16, m_hs, m_os;
-        if (!encode_bf16_2d(&m_xp, ws + p.o_xp, c.input_dim, p.R_routed_max, 128) ||
-            !encode_bf16_2d(&m_xp16, ws + p.o_xp, c.input_dim, p.R_routed_max, 16) ||
-            !encode_bf16_2d(&m_x, x, c.input_dim, T, 128) || !encode_bf16_2d(&m_x16, x, c.input_dim, T, 16) ||
-            !encode_bf16_2d(&m_h, ws + p.o_h, c.expert_dim, p.R_max, 128) ||
-            !encode_bf16_2d(&m_h16, ws + p.o_h, c.expert_dim, p.R_max, 16) ||
-            !encode_bf16_store(&m_hs, ws + p.o_h, c.expert_dim, p.R_max) ||
-            !encode_bf16_store(&m_os, ws + p.o_o, c.output_dim, p.R_max))
+        PairMaps m1, m2;
+        m1.w = L->map_w1;
+        m1.wh = L->map_w1h;
+        m2.w = L->map_w2;
+        m2.wh = L->map_w2h;
+        if (!encode_bf16_2d(&m1.t, ws + p.o_xp, c.input_dim, p.R_routed_max, 128) ||
+            !encode_bf16_2d(&m1.t16, ws + p.o_xp, c.input_dim, p.R_routed_max, 16) ||
+            !encode_bf16_2d(&m1.s, x, c.input_dim, T, 128) || !encode_bf16_2d(&m1.s16, x, c.input_dim, T, 16) ||
+            !encode_bf16_2d(&m2.t, ws + p.o_h, c.expert_dim, p.R_max, 128) ||
+            !encode_bf16_2d(&m2.t16, ws + p.o_h, c.expert_dim, p.R_max, 16) ||
+            !encode_bf16_store(&m1.out, ws + p.o_h, c.expert_dim, p.R_max) ||
+            !encode_bf16_store(&m2.out, ws + p.o_o, c.output_dim, p.R_max))
             return fail(MOE_ERR_CUDA, "cuTensorMapEncodeTiled failed for the activations");
-        MOE_LAUNCH(launch_gemm_pair(L->map_w1, L->map_w1h, m_xp, m_xp16, m_x, m_x16, m_hs, g1, s, nl));
-        MOE_MARK(L, 4, s);
-        MOE_LAUNCH(launch_gemm_pair(L->map_w2, L->map_w2h, m_h, m_h16, m_h, m_h16, m_os, g2, s, nl));
+        m2.s = m2.t;
+        m2.s16 = m2.t16;
+        if (!shared_only && g1.narrow) {
+            // Decode-sized batches run both layers in one launch: layer 2's
+            // units of a token tile start as soon as its layer-1 units have
+            // stored H, so layer 2's weight streaming fills layer 1's last
+            // wave (3% off the decode step; with wide tiles, the per-unit
+            // store completion wait cost more than the tail it saved). The
+            // stage events of the two GEMMs then both follow this launch.
+            g1.tile_done = reinterpret_cast<int32_t *>(ws + p.o_tiledone);
+            MOE_LAUNCH(launch_gemm_pair(m1, g1, &m2, &g2, s, nl));
+            MOE_MARK(L, 4, s);
+        } else {
+            MOE_LAUNCH(launch_gemm_pair(m1, g1, nullptr, nullptr, s, nl));
+            MOE_MARK(L, 4, s);
+            MOE_LAUNCH(launch_gemm_pair(m2, g2, nullptr, nullptr, s, nl));
+        }
         MOE_MARK(L, 5, s);
     } else {
         GemmSimtArgs s1;
@@ -849,14 +872,22 @@ int moe_ep_experts(moe_layer_t *L, const void *recv_x, const int32_t *recv_rows,
     g2.bias = L->w.b2;
     g2.act = -1;
     g2.work_counter = ctrl + kCtrlWork2;
-    CUtensorMap m_x, m_x16, m_h, m_h16, m_hs, m_os;
-    if (!encode_bf16_2d(&m_x, recv_x, c.input_dim, R, 128) || !encode_bf16_2d(&m_x16, recv_x, c.input_dim, R, 16) ||
-        !encode_bf16_2d(&m_h, ws + q.o_h, c.expert_dim, R, 128) ||
-        !encode_bf16_2d(&m_h16, ws + q.o_h, c.expert_dim, R, 16) ||
-        !encode_bf16_store(&m_hs, ws + q.o_h, c.expert_dim, R) || !encode_bf16_store(&m_os, recv_out, c.output_dim, R))
+    PairMaps m1, m2;
+    m1.w = L->map_w1;
+    m1.wh = L->map_w1h;
+    m2.w = L->map_w2;
+    m2.wh = L->map_w2h;
+    if (!encode_bf16_2d(&m1.t, recv_x, c.input_dim, R, 128) || !encode_bf16_2d(&m1.t16, recv_x, c.input_dim, R, 16) ||
+        !encode_bf16_2d(&m2.t, ws + q.o_h, c.expert_dim, R, 128) ||
+        !encode_bf16_2d(&m2.t16, ws + q.o_h, c.expert_dim, R, 16) ||
+        !encode_bf16_store(&m1.out, ws + q.o_h, c.expert_dim, R) || !encode_bf16_store(&m2.out, recv_out, c.output_dim, R))
         return fail(MOE_ERR_CUDA, "cuTensorMapEncodeTiled failed for the received rows");
-    MOE_LAUNCH(launch_gemm_pair(L->map_w1, L->map_w1h, m_x, m_x16, m_x, m_x16, m_hs, g1, s, &launches));
-    MOE_LAUNCH(launch_gemm_pair(L->map_w2, L->map_w2h, m_h, m_h16, m_h, m_h16, m_os, g2, s, &launches));
+    m1.s = m1.t;
+    m1.s16 = m1.t16;
+    m2.s = m2.t;
+    m2.s16 = m2.t16;
+    MOE_LAUNCH(launch_gemm_pair(m1, g1, nullptr, nullptr, s, &launches));
+    MOE_LAUNCH(launch_gemm_pair(m2, g2, nullptr, nullptr, s, &launches));
     return MOE_OK;
 }
 

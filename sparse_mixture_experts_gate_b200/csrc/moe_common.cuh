@@ -127,6 +127,40 @@ __device__ __forceinline__ bool mbar_wait_idle(uint64_t *bar, uint32_t parity, u
     }
 }
 
+// Waits until the global counter *p reaches `target` (gpu-scope acquire
+// loads, a short sleep between polls), bounded like mbar_wait.
+__device__ __forceinline__ bool wait_counter_geq(const int32_t *p, int target, uint32_t *status,
+                                                 uint64_t limit_ns = kWaitLimitNs) {
+    auto load = [p]() {
+        int v;
+        asm volatile("ld.acquire.gpu.global.s32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+        return v;
+    };
+    if (load() >= target) return true;
+    const uint64_t t0 = global_timer_ns();
+    for (;;) {
+        __nanosleep(64);
+        if (load() >= target) return true;
+        const uint64_t dt = global_timer_ns() - t0;
+        if (dt > kStatusPollNs && *reinterpret_cast<volatile uint32_t *>(status) != kDevOk) return false;
+        if (dt > limit_ns) {
+            atomicOr(status, kDevTimeout);
+            return false;
+        }
+    }
+}
+
+// Adds v to the global counter *p with gpu-scope release semantics.
+__device__ __forceinline__ void red_release_add(int32_t *p, int v) {
+    asm volatile("red.release.gpu.global.add.s32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+// Orders this thread's generic-proxy accesses of global memory with its
+// async-proxy ones (TMA loads and stores) in both directions.
+__device__ __forceinline__ void fence_proxy_async_global() {
+    asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+
 // Drain wait used on the way out (own copies / MMAs still in flight): bounded
 // by time only, so it still waits when the status word is already set.
 constexpr uint64_t kDrainLimitNs = 200000000ull;

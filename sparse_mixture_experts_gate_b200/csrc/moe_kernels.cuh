@@ -98,6 +98,8 @@ struct DispatchArgs {
     const float *gates;     // [T][k]
     int32_t *pre_start;     // [E]: exclusive scan of count_pre
     float *gate_sorted;     // [T*k]: every selection's gate, grouped by expert, token order
+    int32_t *tile_done = nullptr;  // [n_tile_done] zeroed by the scan (the expert GEMM's per-tile counters)
+    int n_tile_done = 0;
 };
 cudaError_t launch_dispatch(const DispatchArgs &a, cudaStream_t s, int *launches);
 
@@ -142,6 +144,13 @@ cudaError_t launch_scatter(const ScatterArgs &a, int num_sms, cudaStream_t s, in
 // shared-expert groups (x itself, in token order); map_out: the output
 // [rows][N] bf16 (box 128 x 32, no swizzle), also addressed directly through
 // `out`. N and K must be multiples of 64.
+// The tensor maps of one GEMM layer: weights (boxes of 128 and of 64 rows),
+// token rows in row order (boxes of 128 and 16 rows), shared-expert token rows
+// (x itself, with use_s) and the output (box 128 x 32).
+struct PairMaps {
+    CUtensorMap w, wh, t, t16, s, s16, out;
+};
+
 struct PairGemmArgs {
     const int4 *tok_tiles;       // [max_tok_tiles] {group, first row, rows, 0}
     const int32_t *group_start;  // [G+1]
@@ -159,6 +168,12 @@ struct PairGemmArgs {
     // 1: the last feature tile holds at most 128 features (N % 256 in {64, 128})
     // and its units run transposed (wide token tiles only), storing through `out`.
     int half_last = 0;
+    // Two layers in one launch (set by launch_gemm_pair): layer 2's units of a
+    // token tile wait until tile_done[tile] counts every layer-1 unit of it
+    // (each CTA of a pair adds 1 once its outputs are stored). tile_done has
+    // one zeroed int per token tile.
+    int fuse2 = 0;
+    int32_t *tile_done = nullptr;
     __nv_bfloat16 *out = nullptr;  // [rows][N] bf16 output (row space), the array map_out covers
     const float *bias;           // [G][N] or null
     int act;                     // activation code, -1 none
@@ -174,10 +189,10 @@ struct PairGemmArgs {
 int gemm_pair_max_pairs(int num_sms);
 int gemm_pair_ftiles(int N);
 int gemm_pair_half_last(int N);  // 1 when the last feature tile of N holds at most 128 features
-// map_wh: the weights with boxes of 64 rows (transposed last-tile units).
-cudaError_t launch_gemm_pair(const CUtensorMap &map_w, const CUtensorMap &map_wh, const CUtensorMap &map_t, const CUtensorMap &map_t16,
-                             const CUtensorMap &map_s, const CUtensorMap &map_s16, const CUtensorMap &map_out,
-                             const PairGemmArgs &a, cudaStream_t s, int *launches);
+// One launch of layer 1 (m1, a), or of layer 1 followed by layer 2 (m2, b:
+// same token tiles, its token rows layer 1's outputs) when m2 and b are given.
+cudaError_t launch_gemm_pair(const PairMaps &m1, const PairGemmArgs &a, const PairMaps *m2, const PairGemmArgs *b,
+                             cudaStream_t s, int *launches);
 
 // fp32 CUDA-core path: 32 x 32 output tiles over the 32-row blocks.
 struct GemmSimtArgs {

@@ -404,14 +404,17 @@ def test_bounded_wait_times_out_and_context_survives():
     full_check(w, make_inputs(w, "cpu", seed=2))
 
 
-def test_expert_gemm_timeout_drains_and_context_survives():
+@pytest.mark.parametrize("T", [600, 100])
+def test_expert_gemm_timeout_drains_and_context_survives(T):
     """Failure detection inside the real expert GEMM: GEMM 1's leader CTAs skip
     one stage's loads (a test-only launch argument) and the launch's waits give
     up after 20 ms. The MMA role's wait runs out, every role drains and the
     kernel returns; the device status reports the timeout; the same layer and
-    context then run a forward that matches the oracle."""
+    context then run a forward that matches the oracle. T = 100 is a
+    decode-sized batch (narrow token tiles), whose two GEMMs share one launch:
+    there the GEMM 2 units waiting for GEMM 1's rows give up as well."""
     from sparse_mixture_experts_gate_b200 import binding
-    w = WORKLOADS["default"].with_(T=600)
+    w = WORKLOADS["default"].with_(T=T)
     inp = make_inputs(w, "cpu", seed=2)
     layer = MoELayer(w, inp)
     x = inp["x"].cuda()
