@@ -126,10 +126,26 @@ __device__ __forceinline__ Smem carve(uint8_t *raw) {
 // Named barrier 1 over the four epilogue warps (threads 64..191).
 __device__ __forceinline__ void epi_bar_sync() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
 
-template <int ACT, int TILE>
+// Layer 2 of a two-layer launch: its maps and arguments. The one-layer kernel
+// takes an empty struct instead, so its launches carry half the parameters.
+template <bool TWO>
+struct Layer2 {
+    PairMaps m;
+    PairGemmArgs a;
+};
+template <>
+struct Layer2<false> {};
+__device__ __forceinline__ const PairMaps &maps2(const PairMaps &, const Layer2<true> &l) { return l.m; }
+__device__ __forceinline__ const PairMaps &maps2(const PairMaps &m1, const Layer2<false> &) { return m1; }
+__device__ __forceinline__ const PairGemmArgs &args2(const PairGemmArgs &, const Layer2<true> &l) { return l.a; }
+__device__ __forceinline__ const PairGemmArgs &args2(const PairGemmArgs &a, const Layer2<false> &) { return a; }
+
+template <int ACT, int TILE, bool TWO>
 __global__ void __launch_bounds__(kThreads, 1)
-    grouped_gemm_pair_kernel(const __grid_constant__ PairMaps m1, const __grid_constant__ PairMaps m2,
-                             const PairGemmArgs a, const PairGemmArgs b) {
+    grouped_gemm_pair_kernel(const __grid_constant__ PairMaps m1, const PairGemmArgs a,
+                             const __grid_constant__ Layer2<TWO> l2) {
+    const PairMaps &m2 = maps2(m1, l2);
+    const PairGemmArgs &b = args2(a, l2);
     using C = PairCfg<TILE>;
     constexpr int kStages = C::kStages;
     extern __shared__ uint8_t smem_raw[];
@@ -137,7 +153,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const uint32_t rank = cluster_ctarank();
     const bool leader = rank == 0;
-    const bool two = a.fuse2 != 0;  // layer 2 (b, m2) follows layer 1 (a, m1) in this launch
+    const bool two = TWO && a.fuse2 != 0;  // layer 2 (b, m2) follows layer 1 (a, m1) in this launch
 
     if (threadIdx.x == 0) {
         for (int l = 0; l < (two ? 2 : 1); ++l) {
@@ -498,12 +514,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
 }
 
+// Narrow-tile launches take the two-layer kernel (decode-sized batches run
+// both layers in one launch), wide-tile ones the one-layer kernel.
 template <int ACT, int TILE>
 cudaError_t launch_act(const PairMaps &m1, const PairMaps &m2, const PairGemmArgs &a, const PairGemmArgs &b,
                        cudaStream_t st) {
+    constexpr bool kTwo = TILE == kNarrowTile;
     constexpr int kSmem = PairCfg<TILE>::kSmem;
-    auto kern = grouped_gemm_pair_kernel<ACT, TILE>;
-    cudaError_t e = set_smem_limit_once<grouped_gemm_pair_kernel<ACT, TILE>>(kSmem);
+    auto kern = grouped_gemm_pair_kernel<ACT, TILE, kTwo>;
+    cudaError_t e = set_smem_limit_once<grouped_gemm_pair_kernel<ACT, TILE, kTwo>>(kSmem);
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(2 * a.num_pairs, 1, 1);
@@ -517,7 +536,16 @@ cudaError_t launch_act(const PairMaps &m1, const PairMaps &m2, const PairGemmArg
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, kern, m1, m2, a, b);
+    Layer2<kTwo> l2;
+    if constexpr (kTwo) {
+        l2.m = m2;
+        l2.a = b;
+    } else {
+        if (a.fuse2) return cudaErrorInvalidValue;  // two layers run only with narrow tiles
+        (void)m2;
+        (void)b;
+    }
+    return cudaLaunchKernelEx(&cfg, kern, m1, a, l2);
 }
 
 }  // namespace
@@ -537,7 +565,7 @@ int gemm_pair_max_pairs(int num_sms) {
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    auto kern = grouped_gemm_pair_kernel<-1, kTokTile>;
+    auto kern = grouped_gemm_pair_kernel<-1, kTokTile, false>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem) != cudaSuccess) return 0;
     int clusters = 0;
     if (cudaOccupancyMaxActiveClusters(&clusters, kern, &cfg) != cudaSuccess) return 0;
