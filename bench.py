@@ -316,8 +316,7 @@ def measure(w, args, dev, rank, world, headline):
     ms_max = float(ms_t.item())
     stage_ms = {n: statistics.mean(v) for n, v in stage.items()}
     if w.dtype == "bf16":
-        # The expert GEMMs are reported together: decode-sized batches run them
-        # in one launch, whose events bracket both.
+        # Both expert GEMMs run in one launch: their events bracket it together.
         stage_ms = {("gemms" if n == "gemm1" else n): (v + stage_ms["gemm2"] if n == "gemm1" else v)
                     for n, v in stage_ms.items() if n != "gemm2"}
     res = dict(w=w, inp=inp, T=T, K=K, ms_max=ms_max, ms_step=ms_max / K, ms_eager=statistics.mean(eager_steps),

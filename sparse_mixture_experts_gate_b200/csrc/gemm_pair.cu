@@ -126,26 +126,19 @@ __device__ __forceinline__ Smem carve(uint8_t *raw) {
 // Named barrier 1 over the four epilogue warps (threads 64..191).
 __device__ __forceinline__ void epi_bar_sync() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
 
-// Layer 2 of a two-layer launch: its maps and arguments. The one-layer kernel
-// takes an empty struct instead, so its launches carry half the parameters.
-template <bool TWO>
+// Layer 2 of a two-layer launch: its maps and arguments (a copy of layer 1's
+// in a one-layer launch, unused there).
 struct Layer2 {
     PairMaps m;
     PairGemmArgs a;
 };
-template <>
-struct Layer2<false> {};
-__device__ __forceinline__ const PairMaps &maps2(const PairMaps &, const Layer2<true> &l) { return l.m; }
-__device__ __forceinline__ const PairMaps &maps2(const PairMaps &m1, const Layer2<false> &) { return m1; }
-__device__ __forceinline__ const PairGemmArgs &args2(const PairGemmArgs &, const Layer2<true> &l) { return l.a; }
-__device__ __forceinline__ const PairGemmArgs &args2(const PairGemmArgs &a, const Layer2<false> &) { return a; }
 
-template <int ACT, int TILE, bool TWO>
+template <int ACT, int TILE>
 __global__ void __launch_bounds__(kThreads, 1)
     grouped_gemm_pair_kernel(const __grid_constant__ PairMaps m1, const PairGemmArgs a,
-                             const __grid_constant__ Layer2<TWO> l2) {
-    const PairMaps &m2 = maps2(m1, l2);
-    const PairGemmArgs &b = args2(a, l2);
+                             const __grid_constant__ Layer2 l2) {
+    const PairMaps &m2 = l2.m;
+    const PairGemmArgs &b = l2.a;
     using C = PairCfg<TILE>;
     constexpr int kStages = C::kStages;
     extern __shared__ uint8_t smem_raw[];
@@ -153,7 +146,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const uint32_t rank = cluster_ctarank();
     const bool leader = rank == 0;
-    const bool two = TWO && a.fuse2 != 0;  // layer 2 (b, m2) follows layer 1 (a, m1) in this launch
+    const bool two = a.fuse2 != 0;  // layer 2 (b, m2) follows layer 1 (a, m1) in this launch
 
     if (threadIdx.x == 0) {
         for (int l = 0; l < (two ? 2 : 1); ++l) {
@@ -359,6 +352,17 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int q = warp & 3;        // TMEM lane quarter this warp may access
         const int ep = threadIdx.x - 64;  // 0..127 over the four epilogue warps
         uint32_t sub = 0;              // output boxes staged so far (buffer parity)
+        // Two-layer launches: thread ep 0 publishes each layer-1 unit's outputs
+        // one unit late, once the next unit's stores are under way (its own
+        // bulk groups complete in order), so it rarely waits; the pending unit
+        // is published at once when the next unit is a layer-2 one or the work
+        // ends, before that unit's accumulator is awaited, so that no layer-2
+        // producer of this pair can wait on it.
+        int pend_tt = -1;
+        auto publish = [&](int tile) {
+            fence_proxy_async_global();
+            red_release_add(a.tile_done + tile, 1);
+        };
         // Drains one unit's accumulator with the activation ACT_C of its layer.
         auto drain = [&](auto act_c, const PairGemmArgs &P, const PairMaps &m, int tr, int u_tt, int j,
                          uint32_t acc) {
@@ -459,6 +463,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                 // all pass the same barriers below and leave together.
                 if (ep == 0) {
                     int v = take_unit(tcount);
+                    if (two && pend_tt >= 0 && (v < 0 || v >= total1)) {
+                        bulk_wait_group<0>();
+                        publish(pend_tt);
+                        pend_tt = -1;
+                    }
                     if (v >= 0 && !mbar_wait_idle(&s.tfull[acc], use & 1u, a.status, a.wait_limit_ns)) v = -2;
                     s.epi_unit[tcount & 1u] = v;
                 }
@@ -486,20 +495,31 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(&s.tempty[acc]), 0));
             if constexpr (kWideStores) {
                 if (two && l == 0) {
-                    // Publish this CTA's half of the unit's layer-1 outputs
-                    // for layer 2: the four warps' stores (the transposed
-                    // unit's direct ones included), the TMA stores'
-                    // completion, a proxy fence and a release increment.
+                    // This CTA's half of the unit's layer-1 outputs becomes
+                    // the pending one: every warp's stores of it (the
+                    // transposed unit's direct ones included) come before
+                    // thread ep 0's later release. The previous pending unit
+                    // is complete once at most this unit's own bulk groups
+                    // are outstanding, and is published: a proxy fence and a
+                    // release increment of its tile's counter.
                     epi_bar_sync();
                     if (ep == 0) {
-                        bulk_wait_group<0>();
-                        fence_proxy_async_global();
-                        red_release_add(a.tile_done + tt, 1);
+                        if (pend_tt >= 0) {
+                            const int4 tile = tok_tiles[tt];
+                            const int fb = j * kFeatPair + static_cast<int>(rank) * kFeatCta;
+                            const int nb = (j == tr_tile(0) || fb >= a.N) ? 0 : tile.z / kBoxTok;
+                            bulk_wait_group_dyn(nb);
+                            publish(pend_tt);
+                        }
+                        pend_tt = tt;
                     }
                 }
             }
         }
-        if (kWideStores && ep == 0) bulk_wait_group<0>();  // all stores complete before exit
+        if (kWideStores && ep == 0) {
+            bulk_wait_group<0>();  // all stores complete before exit
+            if (two && pend_tt >= 0) publish(pend_tt);  // the loop ended on an error
+        }
     }
 
     // A role that gave up may leave its own TMA loads in flight; they land
@@ -514,15 +534,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
 }
 
-// Narrow-tile launches take the two-layer kernel (decode-sized batches run
-// both layers in one launch), wide-tile ones the one-layer kernel.
 template <int ACT, int TILE>
 cudaError_t launch_act(const PairMaps &m1, const PairMaps &m2, const PairGemmArgs &a, const PairGemmArgs &b,
                        cudaStream_t st) {
-    constexpr bool kTwo = TILE == kNarrowTile;
     constexpr int kSmem = PairCfg<TILE>::kSmem;
-    auto kern = grouped_gemm_pair_kernel<ACT, TILE, kTwo>;
-    cudaError_t e = set_smem_limit_once<grouped_gemm_pair_kernel<ACT, TILE, kTwo>>(kSmem);
+    auto kern = grouped_gemm_pair_kernel<ACT, TILE>;
+    cudaError_t e = set_smem_limit_once<grouped_gemm_pair_kernel<ACT, TILE>>(kSmem);
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(2 * a.num_pairs, 1, 1);
@@ -536,15 +553,9 @@ cudaError_t launch_act(const PairMaps &m1, const PairMaps &m2, const PairGemmArg
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    Layer2<kTwo> l2;
-    if constexpr (kTwo) {
-        l2.m = m2;
-        l2.a = b;
-    } else {
-        if (a.fuse2) return cudaErrorInvalidValue;  // two layers run only with narrow tiles
-        (void)m2;
-        (void)b;
-    }
+    Layer2 l2;
+    l2.m = m2;
+    l2.a = b;
     return cudaLaunchKernelEx(&cfg, kern, m1, a, l2);
 }
 
@@ -565,7 +576,7 @@ int gemm_pair_max_pairs(int num_sms) {
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    auto kern = grouped_gemm_pair_kernel<-1, kTokTile, false>;
+    auto kern = grouped_gemm_pair_kernel<-1, kTokTile>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem) != cudaSuccess) return 0;
     int clusters = 0;
     if (cudaOccupancyMaxActiveClusters(&clusters, kern, &cfg) != cudaSuccess) return 0;

@@ -638,13 +638,13 @@ int fwd_expert_gemms(moe_layer_t *L, cudaStream_t s, bool shared_only) {
             return fail(MOE_ERR_CUDA, "cuTensorMapEncodeTiled failed for the activations");
         m2.s = m2.t;
         m2.s16 = m2.t16;
-        if (!shared_only && g1.narrow) {
-            // Decode-sized batches run both layers in one launch: layer 2's
-            // units of a token tile start as soon as its layer-1 units have
-            // stored H, so layer 2's weight streaming fills layer 1's last
-            // wave (3% off the decode step; with wide tiles, the per-unit
-            // store completion wait cost more than the tail it saved). The
-            // stage events of the two GEMMs then both follow this launch.
+        if (!shared_only) {
+            // Both layers in one launch: layer 2's units of a token tile start
+            // as soon as its layer-1 units have stored H, so layer 2 fills
+            // layer 1's last wave (3% off the decode step, where the two
+            // layers stream weights from HBM; a few tenths of a percent at
+            // e64). The stage events of the two GEMMs then both follow this
+            // launch.
             g1.tile_done = reinterpret_cast<int32_t *>(ws + p.o_tiledone);
             MOE_LAUNCH(launch_gemm_pair(m1, g1, &m2, &g2, s, nl));
             MOE_MARK(L, 4, s);

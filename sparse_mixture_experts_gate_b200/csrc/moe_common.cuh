@@ -218,6 +218,21 @@ __device__ __forceinline__ void bulk_wait_group() {
     asm volatile("cp.async.bulk.wait_group %0;" ::"n"(N) : "memory");
 }
 
+// bulk_wait_group with a run-time count (0..8; larger counts wait for 8).
+__device__ __forceinline__ void bulk_wait_group_dyn(int n) {
+    switch (n) {
+        case 0: bulk_wait_group<0>(); break;
+        case 1: bulk_wait_group<1>(); break;
+        case 2: bulk_wait_group<2>(); break;
+        case 3: bulk_wait_group<3>(); break;
+        case 4: bulk_wait_group<4>(); break;
+        case 5: bulk_wait_group<5>(); break;
+        case 6: bulk_wait_group<6>(); break;
+        case 7: bulk_wait_group<7>(); break;
+        default: bulk_wait_group<8>(); break;
+    }
+}
+
 // Orders this thread's generic-proxy shared-memory writes before later
 // async-proxy accesses (TMA, tcgen05) of the same memory.
 __device__ __forceinline__ void fence_proxy_async_smem() {
