@@ -4,12 +4,15 @@
 // two-layer MLP, w1/b1 -> activation -> w2/b2, on the rows dispatched to it;
 // shared experts ("Appendix C - Acronyms & Symbols", "Parameter accounting")
 // run the same MLP on every token. Both layers of every expert are dense
-// contractions, computed here as one grouped GEMM per layer over the permuted
-// row space:
+// contractions, computed here as grouped GEMMs over the permuted row space:
 //   out[row][f] = act( sum_k A[row][k] W[g][f][k] + b[g][f] ),  g = group of row.
 // Layer 1: A = the routed token rows scattered into row order (dispatch.cu), or
 // x itself for the shared experts, which read every token in order.
 // Layer 2: A = the hidden activations H (already in row order).
+// A forward runs both layers in one launch: layer 2's units of a token tile
+// start as soon as every layer-1 unit of that tile has stored its rows of H
+// (a per-tile counter, see the producer and the epilogue), so layer 2 fills
+// layer 1's last wave. Expert parallelism runs one layer per launch.
 //
 // Operand roles. The tensor cores compute out^T: the MMA's M side is 256 output
 // features (weights W[g], 128 per CTA of the pair) and its N side is a token
@@ -21,8 +24,8 @@
 // Units are handed out in index order from a global counter (see post_unit),
 // so the pairs at work hold a contiguous run of units whatever their lengths:
 // with a static round-robin the pairs drift apart over the ~140 waves of the
-// E = 256 layer and the L2 reuse of the weight tiles collapses (GEMM 1 read
-// 41.6 GB from DRAM instead of ~15 GB).
+// E = 256 layer's first GEMM and the L2 reuse of the weight tiles collapses (it
+// read 41.6 GB from DRAM instead of ~15 GB).
 //
 // Per CTA (192 threads): warp 0 loads (TMA, signalling the leader's stage
 // barrier, which expects both CTAs' bytes), warp 1 owns TMEM (2 accumulators x
