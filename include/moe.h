@@ -380,11 +380,12 @@ MOE_API int moe_selftest_bounded_wait(void *stream);
 
 /* Self-check of the bounded waits inside the real expert GEMM (no counterpart on
  * the pages): one moe_forward of this layer over x [T][d] (GREEDY top-k, bf16,
- * ep_size 1, d >= 192) with workspace and y as for moe_forward, in which expert
- * GEMM 1's leader CTAs announce the bytes of their third pipeline stage but load
- * none of them, and every wait of that launch gives up after 20 ms. The MMA
- * role's wait runs out, the kernel's roles stop, drain their copies and MMAs and
- * free TMEM, the rest of the forward runs on the unfinished outputs (y is
+ * ep_size 1, d >= 192) with workspace and y as for moe_forward, in which the
+ * expert-GEMM launch's leader CTAs announce the bytes of their third pipeline
+ * stage but load none of them, and every wait of that launch gives up after
+ * 20 ms. The MMA role's wait runs out, the kernel's roles stop (those waiting
+ * for a token tile's GEMM 1 rows too), drain their copies and MMAs and free
+ * TMEM, the rest of the forward runs on the unfinished outputs (y is
  * unspecified), and moe_device_status then reports MOE_ERR_TIMEOUT. Synchronises
  * `stream`. Returns MOE_OK when the timeout was detected and reported, MOE_ERR_
  * INTERNAL if it was not, the errors of moe_forward otherwise. The layer and
