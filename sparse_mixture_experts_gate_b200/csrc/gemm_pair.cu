@@ -277,13 +277,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const bool tr = j == tr_tile(l);  // 64 weight rows per CTA (the MMA's N side)
             const int wrow = wgroup(g) * P.N + j * kFeatPair + static_cast<int>(rank) * (tr ? kFeatCta / 2 : kFeatCta);
             const CUtensorMap *mw = tr ? &m.wh : &m.w;
-            // Wide tiles load each CTA's token rows as one 128-row box, a
-            // partial tile too (the rows past it are loaded but not used: the
-            // MMA's N is the tile's rows): a TMA request costs more than the
-            // bytes. Narrow tiles load 16-row boxes of their rows only.
-            const bool one_box = TILE == kTokTile;
-            const uint32_t tok_rows = one_box ? 2u * (kTokTile / 2) : static_cast<uint32_t>(ntok);
-            const uint32_t tx_bytes = (tr ? 1u : 2u) * kABytes + tok_rows * kBK * 2u;
+            const uint32_t tx_bytes = (tr ? 1u : 2u) * kABytes + static_cast<uint32_t>(ntok) * kBK * 2u;
             const int n16 = ntok / (2 * kRowsPerLoad16);
             const int kblocks = P.K / kBK;
             for (int kb = 0; kb < kblocks; ++kb, ++it) {
@@ -305,7 +299,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const uint32_t bar = mapa_shared(smem_u32(&s.full[st]), 0);
                 uint8_t *sA = s.sA + st * kABytes, *sB = s.sB + st * C::kB;
                 if (lane == 0) tma_load_2d_pair(mw, bar, sA, kb * kBK, wrow);
-                if (one_box) {
+                if (ntok == kTokTile) {
                     if (lane == 1) tma_load_2d_pair(mt, bar, sB, kb * kBK, trow);
                 } else if (lane < n16) {
                     tma_load_2d_pair(mt16, bar, sB + lane * kRowsPerLoad16 * 128, kb * kBK,
