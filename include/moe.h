@@ -421,10 +421,10 @@ MOE_API int moe_device_status(moe_layer_t *layer, void *stream);
  *                                       none: events[3] follows events[2]),
  *   events[4] after expert GEMM 1,      events[5] after expert GEMM 2,
  *   events[6] after the combine,
- * (bf16 layers run both expert GEMMs in one launch, so that GEMM 2 starts on a
- * token tile as soon as GEMM 1 has stored its hidden rows: events[4] and
- * events[5] then both follow that launch, and events[3]..events[5] time the
- * two GEMMs together)
+ * (moe_forward of a bf16 layer runs both expert GEMMs in one launch, so that
+ * GEMM 2 starts on a token tile as soon as GEMM 1 has stored its hidden rows:
+ * events[4] and events[5] then both follow that launch, and events[3]..
+ * events[5] time the two GEMMs together)
  * and every moe_aux_stats records events[7] after its kernels, all on the
  * call's stream. The array is copied; events == NULL turns timing off. Nothing
  * is allocated and nothing synchronises. */
