@@ -124,6 +124,29 @@ def test_determinism_bit_identical():
         assert np.array_equal(g1[k], g2[k], equal_nan=True), k
 
 
+@pytest.mark.parametrize("name,T", [("e64", 8192), ("default", 100), ("decode", 128)])
+def test_repeated_forwards_bit_identical(name, T):
+    """Both expert GEMM layers share one launch, GEMM 2's units of a token
+    tile waiting on a per-tile counter that GEMM 1's epilogues release once
+    their stores are complete. A missed or early release would let a unit
+    read hidden rows that are not written yet, so repeated forwards of the
+    same batch (full-size e64 with wide tiles, narrow-tile batches) must give
+    the same bits every time."""
+    w = WORKLOADS[name].with_(T=T)
+    inp = make_inputs(w, "cuda", seed=19)
+    layer = MoELayer(w, inp)
+    ref = None
+    for _ in range(12):
+        out = layer.forward(inp["x"], noise=inp.get("noise"))
+        torch.cuda.synchronize()
+        y = out["y"].view(torch.int16).cpu().numpy()
+        if ref is None:
+            ref = y.copy()
+        else:
+            assert np.array_equal(ref, y)
+    assert layer.device_status() == 0
+
+
 def test_forward_argument_errors_on_host():
     w = WORKLOADS["default"]
     inp = make_inputs(w.with_(T=8), "cpu")
